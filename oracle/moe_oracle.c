@@ -1,0 +1,372 @@
+/*
+ * moe_oracle.c -- plain, slow FP64 CPU oracle of the routed Mixture-of-Experts
+ * feed-forward layer (Gemma 4 26B-A4B shapes, Q4_0 experts).
+ *
+ * TEST INFRASTRUCTURE ONLY. Nothing on the product path may link, load or call
+ * this file: only the test suite, the smoke check and the benchmark's CPU
+ * baseline use it. It shares no code, header or table with the CUDA library.
+ *
+ * What it follows (page "Gemma 4 26B-A4B it QAT Q4_0 ... NInfer v3 artifact"):
+ *   - intro: every matrix keeps the release's ggml blocks byte for byte and the
+ *     engine multiplies the blocks in place (no requantisation);
+ *   - "What is inside": 128 routed experts per block, Q4_0, expert-major,
+ *     [gate; up] 2 x 704 rows and down 2,816 rows; router, router scale and
+ *     expert scales FP32;
+ *   - "Quality": kernels are checked against FP64 oracles.
+ * Steps the pages leave open take the plainest reading (all listed with the
+ * design notes): ggml block_q4_0 layout (fp16 d, element i = low nibble of
+ * code byte i, element i+16 = high nibble, value (q-8)*d); top-k on the router
+ * logits, ties to the lower expert index; softmax over the k selected logits;
+ * router scale multiplies the combine weights; GELU-tanh GeGLU with gate in the
+ * first f rows; expert scale multiplies the expert's output in the combine.
+ *
+ * Arithmetic: every sum is an FP64 sum taken in index order, one output element
+ * per loop, so results do not depend on the number of OpenMP threads.
+ */
+#include <math.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+#ifdef _OPENMP
+#include <omp.h>
+#endif
+
+#define Q4_0_QK 32
+#define Q4_0_BYTES 18
+
+/* ---------------------------------------------------------------- scalars */
+
+/* IEEE 754 binary16 -> double, from the field definition. */
+double oracle_fp16_to_double(uint16_t h)
+{
+    int sign = (h >> 15) & 1;
+    int ex = (h >> 10) & 0x1f;
+    int man = h & 0x3ff;
+    double v;
+    if (ex == 0)
+        v = ldexp((double)man, -24);               /* subnormal: man * 2^-24 */
+    else if (ex == 31)
+        v = man ? NAN : INFINITY;
+    else
+        v = ldexp((double)(1024 + man), ex - 25);  /* 1.man * 2^(ex-15) */
+    return sign ? -v : v;
+}
+
+/* bf16 -> double: a bf16 value is the upper half of a binary32. */
+double oracle_bf16_to_double(uint16_t b)
+{
+    uint32_t u = (uint32_t)b << 16;
+    float f;
+    memcpy(&f, &u, sizeof f);
+    return (double)f;
+}
+
+/* double -> bf16, round to nearest, ties to even, directly from the double
+ * (no intermediate binary32, so no double rounding). */
+uint16_t oracle_double_to_bf16_rne(double v)
+{
+    if (isnan(v))
+        return 0x7fc0;
+    uint16_t sign = signbit(v) ? 0x8000 : 0;
+    double a = fabs(v);
+    if (a == 0.0)
+        return sign;
+    if (isinf(a))
+        return sign | 0x7f80;
+    int e;
+    frexp(a, &e);                 /* a = m * 2^e, 0.5 <= m < 1 */
+    /* unbiased exponent of the leading bit is e-1; bf16 keeps 8 significant
+     * bits for normals (exponent >= -126), fixed quantum 2^-133 below that. */
+    int lead = e - 1;
+    int q_exp = (lead >= -126 ? lead : -126) - 7;   /* quantum = 2^q_exp */
+    double scaled = ldexp(a, -q_exp);                /* exact */
+    double r = floor(scaled);
+    double frac = scaled - r;
+    if (frac > 0.5 || (frac == 0.5 && fmod(r, 2.0) != 0.0))
+        r += 1.0;
+    double rv = ldexp(r, q_exp);                     /* rounded magnitude */
+    if (rv == 0.0)                                   /* rounded down to zero */
+        return sign;
+    if (rv >= 0x1p128)                               /* rounds beyond max finite */
+        return sign | 0x7f80;
+    /* encode */
+    int re;
+    frexp(rv, &re);
+    int rlead = re - 1;
+    if (rlead < -126) {           /* subnormal: mantissa = rv / 2^-133 */
+        uint16_t m = (uint16_t)ldexp(rv, 133);
+        return sign | m;
+    }
+    uint16_t bexp = (uint16_t)(rlead + 127);
+    uint16_t m = (uint16_t)(ldexp(rv, -rlead + 7) - 128.0);
+    return sign | (uint16_t)(bexp << 7) | m;
+}
+
+/* One ggml Q4_0 block (18 bytes) -> 32 values (q - 8) * d. */
+void oracle_q4_0_decode_block(const uint8_t *blk, double *out)
+{
+    double dd = oracle_fp16_to_double((uint16_t)(blk[0] | ((uint16_t)blk[1] << 8)));
+    for (int i = 0; i < 16; ++i) {
+        int lo = blk[2 + i] & 0x0f;
+        int hi = blk[2 + i] >> 4;
+        out[i] = (double)(lo - 8) * dd;
+        out[i + 16] = (double)(hi - 8) * dd;
+    }
+}
+
+/* GELU, tanh form (Hendrycks & Gimpel 2016):
+ * 0.5 z (1 + tanh(sqrt(2/pi) (z + 0.044715 z^3))). */
+double oracle_gelu_tanh(double z)
+{
+    const double c = sqrt(2.0 / 3.14159265358979323846);
+    return 0.5 * z * (1.0 + tanh(c * (z + 0.044715 * z * z * z)));
+}
+
+/* Dot product of one Q4_0 row (n values, n % 32 == 0) with a double vector. */
+static double q4_0_row_dot(const uint8_t *row, const double *v, int n)
+{
+    double blk[Q4_0_QK];
+    double s = 0.0;
+    for (int b = 0; b < n / Q4_0_QK; ++b) {
+        oracle_q4_0_decode_block(row + (size_t)b * Q4_0_BYTES, blk);
+        for (int i = 0; i < Q4_0_QK; ++i)
+            s += blk[i] * v[b * Q4_0_QK + i];
+    }
+    return s;
+}
+
+/* ----------------------------------------------------------------- router */
+
+/* logits[t*E + e] = sum_i W_r[e, i] * x[t, i]  (FP64, i ascending). */
+void oracle_router_logits(const uint16_t *x, const float *router_w, int T, int d, int E,
+                          double *logits)
+{
+#pragma omp parallel for schedule(static)
+    for (long te = 0; te < (long)T * E; ++te) {
+        int t = (int)(te / E), e = (int)(te % E);
+        double s = 0.0;
+        for (int i = 0; i < d; ++i)
+            s += (double)router_w[(size_t)e * d + i] * oracle_bf16_to_double(x[(size_t)t * d + i]);
+        logits[te] = s;
+    }
+}
+
+/*
+ * Top-k selection and softmax over the selected logits, per token.
+ *   - the selection compares the logits rounded to FP32 (the router's
+ *     precision); among equal values the lower expert index wins; ids come out
+ *     ordered by that comparison (largest first);
+ *   - p_j = exp(l_j - l_1) / sum_m exp(l_m - l_1) over the k selected FP64
+ *     logits; w_j = router_scale * p_j;
+ *   - flags[t] bit 0: the FP64 gap between the k-th and (k+1)-th largest logit
+ *     is <= tie_eps (selection not decided by the inputs at that precision);
+ *     bit 1: two selected logits are within tie_eps (their order is not).
+ */
+void oracle_topk_softmax(const double *logits, int T, int E, int k, double router_scale,
+                         double tie_eps, int32_t *ids, double *w, uint8_t *flags)
+{
+#pragma omp parallel for schedule(static)
+    for (int t = 0; t < T; ++t) {
+        const double *l = logits + (size_t)t * E;
+        char *taken = (char *)calloc((size_t)E, 1);
+        int32_t *id = ids + (size_t)t * k;
+        for (int j = 0; j < k; ++j) {
+            int best = -1;
+            float bv = 0.0f;
+            for (int e = 0; e < E; ++e) {
+                if (taken[e])
+                    continue;
+                float v = (float)l[e];
+                if (best < 0 || v > bv) {   /* strict: equal keeps the lower e */
+                    best = e;
+                    bv = v;
+                }
+            }
+            taken[best] = 1;
+            id[j] = best;
+        }
+        /* flags from the FP64 values */
+        uint8_t fl = 0;
+        if (k < E) {
+            double kth = INFINITY, next = -INFINITY;
+            for (int j = 0; j < k; ++j)
+                if (l[id[j]] < kth)
+                    kth = l[id[j]];
+            for (int e = 0; e < E; ++e)
+                if (!taken[e] && l[e] > next)
+                    next = l[e];
+            if (kth - next <= tie_eps)
+                fl |= 1;
+        }
+        for (int a = 0; a < k; ++a)
+            for (int b = a + 1; b < k; ++b)
+                if (fabs(l[id[a]] - l[id[b]]) <= tie_eps)
+                    fl |= 2;
+        flags[t] = fl;
+        free(taken);
+        double l1 = l[id[0]];
+        double z = 0.0;
+        for (int j = 0; j < k; ++j)
+            z += exp(l[id[j]] - l1);
+        for (int j = 0; j < k; ++j)
+            w[(size_t)t * k + j] = router_scale * exp(l[id[j]] - l1) / z;
+    }
+}
+
+/*
+ * Stable counting sort of the T*k slots s = t*k + j by expert id:
+ * counts[e], offsets[e] = sum_{e' < e} counts[e'] (offsets[E] = T*k),
+ * perm[offsets[e] + r] = r-th slot (ascending s) routed to e, inv[perm[p]] = p.
+ */
+void oracle_permutation(const int32_t *ids, int T, int k, int E,
+                        int32_t *counts, int32_t *offsets, int32_t *perm, int32_t *inv)
+{
+    long S = (long)T * k;
+    for (int e = 0; e < E; ++e)
+        counts[e] = 0;
+    for (long s = 0; s < S; ++s)
+        counts[ids[s]] += 1;
+    offsets[0] = 0;
+    for (int e = 0; e < E; ++e)
+        offsets[e + 1] = offsets[e] + counts[e];
+    int32_t *fill = (int32_t *)malloc(sizeof(int32_t) * (size_t)E);
+    for (int e = 0; e < E; ++e)
+        fill[e] = offsets[e];
+    for (long s = 0; s < S; ++s) {
+        int e = ids[s];
+        perm[fill[e]] = (int32_t)s;
+        if (inv)
+            inv[s] = fill[e];
+        fill[e] += 1;
+    }
+    free(fill);
+}
+
+/* ---------------------------------------------------------------- experts */
+
+/*
+ * One expert applied to one token:
+ *   g[c] = Wgu[c, :] . x,  u[c] = Wgu[f + c, :] . x   (c < f)
+ *   h[c] = gelu_tanh(g[c]) * u[c]
+ *   y[r] = Wd[r, :] . h                                (r < d)
+ * gate_up_e: [2f][d/32] Q4_0 blocks, down_e: [d][f/32] Q4_0 blocks.
+ * h may be NULL.
+ */
+void oracle_expert_ffn(const uint16_t *x_row, const uint8_t *gate_up_e, const uint8_t *down_e,
+                       int d, int f, double *h_out, double *y)
+{
+    size_t gu_row = (size_t)(d / Q4_0_QK) * Q4_0_BYTES;
+    size_t dn_row = (size_t)(f / Q4_0_QK) * Q4_0_BYTES;
+    double *xv = (double *)malloc(sizeof(double) * (size_t)d);
+    double *h = (double *)malloc(sizeof(double) * (size_t)f);
+    for (int i = 0; i < d; ++i)
+        xv[i] = oracle_bf16_to_double(x_row[i]);
+    for (int c = 0; c < f; ++c) {
+        double g = q4_0_row_dot(gate_up_e + (size_t)c * gu_row, xv, d);
+        double u = q4_0_row_dot(gate_up_e + (size_t)(f + c) * gu_row, xv, d);
+        h[c] = oracle_gelu_tanh(g) * u;
+    }
+    for (int r = 0; r < d; ++r)
+        y[r] = q4_0_row_dot(down_e + (size_t)r * dn_row, h, f);
+    if (h_out)
+        memcpy(h_out, h, sizeof(double) * (size_t)f);
+    free(h);
+    free(xv);
+}
+
+/*
+ * Experts and combine for a list of tokens, given the routing:
+ *   out[n, r] = sum_{j = 0..k-1} w[t, j] * expert_scale[e_tj] * y_tj[r],
+ * summed in j order, t = tokens[n]. out is [n_tokens, d] (FP64).
+ * h_out (optional) receives h for each (n, j): [n_tokens, k, f].
+ */
+void oracle_experts_combine(const uint16_t *x, const uint8_t *gate_up, const uint8_t *down,
+                            const float *expert_scale, const int32_t *ids, const double *w,
+                            int d, int f, int k, const int32_t *tokens, int n_tokens,
+                            double *out, double *h_out)
+{
+    size_t gu_expert = (size_t)2 * f * (d / Q4_0_QK) * Q4_0_BYTES;
+    size_t dn_expert = (size_t)d * (f / Q4_0_QK) * Q4_0_BYTES;
+    double *y = (double *)malloc(sizeof(double) * (size_t)n_tokens * k * d);
+#pragma omp parallel for schedule(dynamic, 1)
+    for (long nj = 0; nj < (long)n_tokens * k; ++nj) {
+        int n = (int)(nj / k), j = (int)(nj % k);
+        int t = tokens[n];
+        int e = ids[(size_t)t * k + j];
+        oracle_expert_ffn(x + (size_t)t * d, gate_up + (size_t)e * gu_expert,
+                          down + (size_t)e * dn_expert, d, f,
+                          h_out ? h_out + ((size_t)n * k + j) * f : NULL,
+                          y + (size_t)nj * d);
+    }
+#pragma omp parallel for schedule(static)
+    for (int n = 0; n < n_tokens; ++n) {
+        int t = tokens[n];
+        for (int r = 0; r < d; ++r) {
+            double s = 0.0;
+            for (int j = 0; j < k; ++j) {
+                int e = ids[(size_t)t * k + j];
+                s += w[(size_t)t * k + j] * (double)expert_scale[e] * y[((size_t)n * k + j) * d + r];
+            }
+            out[(size_t)n * d + r] = s;
+        }
+    }
+    free(y);
+}
+
+/*
+ * The whole layer for all T tokens: router, top-k + softmax, experts, combine.
+ * out [T, d] FP64; ids [T, k]; w [T, k]; flags [T]. Returns 0.
+ */
+int oracle_moe_layer(const uint16_t *x, const float *router_w, double router_scale,
+                     const uint8_t *gate_up, const uint8_t *down, const float *expert_scale,
+                     int T, int d, int f, int E, int k, double tie_eps,
+                     double *out, int32_t *ids, double *w, uint8_t *flags)
+{
+    if (T <= 0)
+        return 0;
+    double *logits = (double *)malloc(sizeof(double) * (size_t)T * E);
+    int32_t *tok = (int32_t *)malloc(sizeof(int32_t) * (size_t)T);
+    oracle_router_logits(x, router_w, T, d, E, logits);
+    oracle_topk_softmax(logits, T, E, k, router_scale, tie_eps, ids, w, flags);
+    for (int t = 0; t < T; ++t)
+        tok[t] = t;
+    oracle_experts_combine(x, gate_up, down, expert_scale, ids, w, d, f, k, tok, T, out, NULL);
+    free(tok);
+    free(logits);
+    return 0;
+}
+
+/*
+ * RMS normalisation with unit gain followed by the bf16 cast, between
+ * stacked layers: x[t, i] = bf16_rne(y[t, i] / sqrt(mean_i y[t, i]^2 + eps)).
+ */
+void oracle_rmsnorm_bf16(const double *y, int T, int d, double eps, uint16_t *x_out)
+{
+    for (int t = 0; t < T; ++t) {
+        double ss = 0.0;
+        for (int i = 0; i < d; ++i)
+            ss += y[(size_t)t * d + i] * y[(size_t)t * d + i];
+        double inv = 1.0 / sqrt(ss / d + eps);
+        for (int i = 0; i < d; ++i)
+            x_out[(size_t)t * d + i] = oracle_double_to_bf16_rne(y[(size_t)t * d + i] * inv);
+    }
+}
+
+int oracle_num_threads(void)
+{
+#ifdef _OPENMP
+    return omp_get_max_threads();
+#else
+    return 1;
+#endif
+}
+
+void oracle_set_num_threads(int n)
+{
+#ifdef _OPENMP
+    if (n > 0)
+        omp_set_num_threads(n);
+#else
+    (void)n;
+#endif
+}
