@@ -1,0 +1,410 @@
+#!/usr/bin/env python
+"""Benchmark of the routed-MoE layer on B200: one JSON line on rank 0.
+
+A step is one pass of the whole layer (router, top-k + softmax, permutation, gate_up +
+GeGLU, down + combine) over one batch of synthetic inputs, through the C ABI. The default
+workload is the eight-request decode batch (decode_T8: T = 8 tokens, d = 2816, f = 704,
+E = 128, k = 8). Consecutive steps rotate over several independent layers so that the
+active experts' weights of one step are not L2-resident in the next (inputs larger than L2).
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl ours|reference]
+
+Multi-GPU (torchrun, one rank per GPU): every rank runs an independent replica of the
+workload (weak scaling); timing is the max over ranks of the device-timed region.
+`--impl reference` times the FP64 CPU oracle on the host cores instead (rank 0 only).
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+
+import moe_inputs as mi  # noqa: E402
+
+METRIC = "MoE-layer tokens/s; decode HBM GB/s & prefill TFLOP/s as % of B200 roofline"
+
+
+def parse():
+    p = argparse.ArgumentParser()
+    p.add_argument("--gpus", type=int, default=1)
+    p.add_argument("--steps", type=int, default=200)
+    p.add_argument("--warmup", type=int, default=10)
+    p.add_argument("--workload", default="decode_T8", choices=mi.WORKLOADS)
+    p.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    p.add_argument("--layers", type=int, default=0, help="layers rotated across steps (0: auto)")
+    p.add_argument("--no-cpu-baseline", action="store_true")
+    return p.parse_args()
+
+
+# ----------------------------------------------------------------------------- peaks
+
+def measured_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as fh:
+            pk = json.load(fh)
+        return {"hbm_gbs": float(pk["hbm_gbs"]), "bf16_tflops": float(pk["bf16_tflops"]),
+                "bf16_tflops_sustained": float(pk.get("bf16_tflops_sustained", pk["bf16_tflops"])),
+                "source": "measured"}
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "source": "fallback"}
+
+
+# ----------------------------------------------------------------------------- clocks
+
+class ClockSampler:
+    """nvidia-smi clocks and throttle reasons sampled every 200 ms while running."""
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_id: str):
+        self.gpu_id = gpu_id
+        self.proc = None
+        self.lines = []
+        self.thread = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", self.gpu_id, f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except (OSError, ValueError):
+            self.proc = None
+            return
+        self.thread = threading.Thread(target=self._read, daemon=True)
+        self.thread.start()
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        if self.thread:
+            self.thread.join(timeout=2)
+        sm, mx, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            parts = [x.strip() for x in ln.split(",")]
+            if len(parts) < 8:
+                continue
+            try:
+                sm.append(float(parts[0]))
+                mx.append(float(parts[1]))
+            except ValueError:
+                continue
+            for nm, v in zip(names, parts[4:8]):
+                if v.lower().startswith("active"):
+                    reasons.add(nm)
+        if not sm:
+            return None
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(mx), "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# ----------------------------------------------------------------------------- helpers
+
+def flops_bytes(lw: mi.LayerWeights, T: int, k: int, counts: np.ndarray):
+    """Algorithmic work of one layer call given the per-expert token counts."""
+    d, f = lw.d, lw.f
+    active = int((counts > 0).sum())
+    gu_bytes = active * 2 * f * (d // 32) * 18
+    dn_bytes = active * d * (f // 32) * 18
+    router_bytes = lw.E * d * 4
+    act_bytes = T * d * 2 + T * d * 4          # x in, out
+    h_bytes = T * k * f * 4                    # h written by gate_up, read by down
+    flops = 2 * T * k * (2 * f * d + d * f) + 2 * T * lw.E * d
+    return {"active": active, "gateup_weight_bytes": gu_bytes, "down_weight_bytes": dn_bytes,
+            "router_bytes": router_bytes, "act_bytes": act_bytes, "h_bytes": h_bytes,
+            "total_bytes": gu_bytes + dn_bytes + router_bytes + act_bytes + 2 * h_bytes,
+            "flops": flops}
+
+
+def dist_env():
+    ws = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return ws, rank, local
+
+
+# ----------------------------------------------------------------------------- reference arm
+
+def run_reference(args):
+    ws, rank, _ = dist_env()
+    if rank != 0:
+        return 0
+    import oracle
+    wl = mi.make_workload(args.workload, n_layers=1 if args.workload == "stack30_T1" else None)
+    lw = wl.layers[0]
+    k = wl.k
+    # size one step: time a single token, then take as many tokens as fit ~0.5 s per step
+    t0 = time.perf_counter()
+    oracle.moe_layer(wl.x[:1], lw.router_w, lw.router_scale, lw.gate_up, lw.down, lw.expert_scale, k)
+    one = time.perf_counter() - t0
+    budget = 120.0 / max(1, args.steps + args.warmup)
+    n_tok = int(max(1, min(wl.T, budget / max(one, 1e-6))))
+    xs = wl.x[:n_tok]
+    for _ in range(args.warmup):
+        oracle.moe_layer(xs, lw.router_w, lw.router_scale, lw.gate_up, lw.down, lw.expert_scale, k)
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        oracle.moe_layer(xs, lw.router_w, lw.router_scale, lw.gate_up, lw.down, lw.expert_scale, k)
+    el = time.perf_counter() - t0
+    val = n_tok * args.steps / el
+    sample = f"{n_tok} of the {wl.T} tokens of {args.workload} per step (one layer, FP64 oracle)"
+    line = {"metric": METRIC, "value": val, "unit": "tokens/s", "n_gpus": args.gpus, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": 1e3 * el / args.steps, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": args.workload, "T": wl.T, "d": lw.d, "f": lw.f, "E": lw.E, "k": k},
+            "impl": "reference",
+            "cpu_baseline": {"value": val, "unit": "tokens/s", "cores": oracle.num_threads(), "kind": "oracle",
+                             "sample": sample},
+            "e2e": {"value": val, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# ----------------------------------------------------------------------------- our arm
+
+def main():
+    args = parse()
+    if args.impl == "reference":
+        return run_reference(args)
+
+    import torch
+    import torch.distributed as dist
+
+    ws, rank, local = dist_env()
+    if ws > 1:
+        from datetime import timedelta
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+
+    from mixture_experts_gemv_b200 import build as moe_build
+    moe_build.build()
+    import mixture_experts_gemv_b200 as moe
+
+    wl_name = args.workload
+    stack = wl_name == "stack30_T1"
+    base = mi.make_workload(wl_name, n_layers=30 if stack else None)
+    k = base.k
+    T = base.T
+    lw0 = base.layers[0]
+    d, f, E = lw0.d, lw0.f, lw0.E
+    if stack:
+        layers = base.layers
+        n_rot = 1
+    else:
+        n_rot = args.layers or (6 if T <= 16 else 1)
+        layers = [lw0] + [mi.make_layer(0, i) for i in range(1, n_rot)]
+        if wl_name == "skewed_T512":
+            for lw in layers[1:]:
+                mi.apply_router_bias(lw, base.x.copy(), 2.0 * mi.zipf_mean_one(E, 1.1))
+
+    def up(a):
+        a = np.ascontiguousarray(a)
+        if a.dtype == np.uint16:
+            a = a.view(np.int16)
+        return torch.from_numpy(a).to(dev)
+
+    dl = [dict(router_w=up(lw.router_w), router_scale=up(lw.router_scale), gate_up=up(lw.gate_up),
+               down=up(lw.down), expert_scale=up(lw.expert_scale)) for lw in layers]
+    x = up(base.x)
+    out = torch.empty((T, d), dtype=torch.float32, device=dev)
+    moe.moe_init(local, T, d, f, E, k)
+    moe.moe_set_path(moe.MOE_PATH_AUTO, 16)
+    stream = torch.cuda.current_stream(dev)
+
+    def step(i, xin=None, o=None):
+        xin = x if xin is None else xin
+        o = out if o is None else o
+        if stack:
+            moe.moe_stack_forward(xin, [q["router_w"] for q in dl], [q["router_scale"] for q in dl],
+                                  [q["gate_up"] for q in dl], [q["down"] for q in dl],
+                                  [q["expert_scale"] for q in dl], T, d, f, E, k, 1e-6, o, None, stream)
+        else:
+            q = dl[i % len(dl)]
+            moe.moe_layer_forward(xin, q["router_w"], q["router_scale"], q["gate_up"], q["down"],
+                                  q["expert_scale"], T, d, f, E, k, o, stream)
+
+    # per-layer work (from the GPU's own routing)
+    work = []
+    for i in range(len(dl) if not stack else len(layers)):
+        if stack:
+            break
+        step(i)
+        cnt = torch.empty(E, dtype=torch.int32, device=dev)
+        moe.moe_debug_get_routing(counts=cnt, stream=stream)
+        torch.cuda.synchronize()
+        work.append(flops_bytes(layers[i], T, k, cnt.cpu().numpy()))
+    if stack:
+        # per layer, the routing is only visible for the last call; run layers one by one
+        for i, lw in enumerate(layers):
+            q = dl[i]
+            moe.moe_layer_forward(x, q["router_w"], q["router_scale"], q["gate_up"], q["down"],
+                                  q["expert_scale"], T, d, f, E, k, out, stream)
+            cnt = torch.empty(E, dtype=torch.int32, device=dev)
+            moe.moe_debug_get_routing(counts=cnt, stream=stream)
+            torch.cuda.synchronize()
+            work.append(flops_bytes(lw, T, k, cnt.cpu().numpy()))
+    moe.moe_debug_check(stream)
+
+    def barrier():
+        if ws > 1:
+            dist.barrier()
+
+    for i in range(args.warmup):
+        step(i)
+    torch.cuda.synchronize()
+
+    props = torch.cuda.get_device_properties(dev)
+    gpu_id = f"GPU-{props.uuid}" if getattr(props, "uuid", None) else str(local)
+    sampler = ClockSampler(gpu_id)
+    sampler.start()
+    time.sleep(0.3)
+
+    # ---- timed region: K steps
+    barrier()
+    torch.cuda.synchronize()
+    ev0 = torch.cuda.Event(enable_timing=True)
+    ev1 = torch.cuda.Event(enable_timing=True)
+    ev0.record(stream)
+    for i in range(args.steps):
+        step(i)
+    ev1.record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    ms = ev0.elapsed_time(ev1)
+    clocks = sampler.stop()
+    moe.moe_debug_check(stream)
+    if ws > 1:
+        t = torch.tensor([ms], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms = float(t.item())
+    ms_step = ms / args.steps
+
+    # ---- per-kernel timing over a second pass of K steps (CUDA events on the launch stream)
+    barrier()
+    moe.moe_profile_begin()
+    for i in range(args.steps):
+        step(i)
+    prof = moe.moe_profile_end()
+
+    # ---- end to end through the C ABI with host buffers (pinned), copies inside the region
+    xh = torch.from_numpy(np.ascontiguousarray(base.x).view(np.int16)).pin_memory()
+    oh = torch.empty((T, d), dtype=torch.float32).pin_memory()
+    xd = torch.empty_like(x)
+    for i in range(3):
+        xd.copy_(xh, non_blocking=True)
+        step(i, xd)
+        oh.copy_(out, non_blocking=True)
+    torch.cuda.synchronize()
+    barrier()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for i in range(args.steps):
+        xd.copy_(xh, non_blocking=True)
+        step(i, xd)
+        oh.copy_(out, non_blocking=True)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    ms_e2e = e0.elapsed_time(e1)
+    if ws > 1:
+        t = torch.tensor([ms_e2e], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms_e2e = float(t.item())
+
+    # ---- roofline of the dominant kernel
+    pk = measured_peaks()
+    tokens_per_step = T
+    value = ws * tokens_per_step * args.steps / (ms / 1e3)
+    e2e_value = ws * tokens_per_step * args.steps / (ms_e2e / 1e3)
+    avg = {kk: float(np.mean([w[kk] for w in work])) for kk in work[0]}
+    n_layers_per_step = len(layers) if stack else 1
+    if T <= 16:
+        name = "gateup_gemv"
+        kms, nl = prof.get(name, (float("nan"), 1))
+        per_launch_bytes = avg["gateup_weight_bytes"] + T * d * 4 + T * k * f * 8
+        achieved = per_launch_bytes / (kms / nl / 1e3) / 1e9
+        roof = {"kernel": "k_gateup_gemv", "bound": "hbm", "achieved": achieved, "peak": pk["hbm_gbs"],
+                "unit": "GB/s", "frac": achieved / pk["hbm_gbs"], "traffic": None,
+                "peak_source": pk["source"] + " (hbm_gbs, copy bandwidth)",
+                "bytes_per_launch": per_launch_bytes, "ms_per_launch": kms / nl}
+        dtype = "f32"
+    else:
+        name = "gateup_gemm" if "gateup_gemm" in prof else "gateup_gemv"
+        kms, nl = prof.get(name, (float("nan"), 1))
+        fl = 2 * T * k * 2 * f * d
+        achieved = fl / (kms / nl / 1e3) / 1e12
+        roof = {"kernel": name, "bound": "tensor", "achieved": achieved, "peak": pk["bf16_tflops"],
+                "unit": "TFLOP/s", "frac": achieved / pk["bf16_tflops"], "traffic": None,
+                "peak_source": pk["source"] + " (bf16_tflops, burst)", "flops_per_launch": fl,
+                "ms_per_launch": kms / nl}
+        dtype = "bf16" if name == "gateup_gemm" else "f32"
+    launches_per_step = sum(n for (_, n) in prof.values()) / args.steps
+    step_gbs = avg["total_bytes"] * n_layers_per_step / (ms_step / 1e3) / 1e9
+
+    line = {"metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": ws, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": dtype, "data": "synthetic",
+            "config": {"workload": wl_name, "T": T, "d": d, "f": f, "E": E, "k": k,
+                       "layers_per_step": n_layers_per_step, "layers_rotated": len(dl) if not stack else 30,
+                       "active_experts_mean": avg["active"],
+                       "l2": "inputs larger than L2: consecutive steps use different layers' weights"
+                       if not stack else "inputs larger than L2: 30 layers (12.8 GB) per step",
+                       "parallelism": f"replicas x{ws}"},
+            "roofline": roof,
+            "step_bytes": avg["total_bytes"] * n_layers_per_step, "step_gbs": step_gbs,
+            "step_hbm_frac": step_gbs / pk["hbm_gbs"],
+            "kernel_ms_per_step": {kk: v[0] / args.steps for kk, v in prof.items()},
+            "gpu_launches": int(round(launches_per_step * args.steps)),
+            "e2e": {"value": e2e_value, "unit": "tokens/s", "h2d_bytes_per_step": T * d * 2,
+                    "d2h_bytes_per_step": T * d * 4},
+            "clocks": clocks}
+
+    if rank == 0 and ws == 1 and not args.no_cpu_baseline:
+        import oracle
+        lw = layers[0]
+        n_tok = T if T <= 8 else 2
+        t0 = time.perf_counter()
+        reps = 0
+        while True:
+            oracle.moe_layer(base.x[:n_tok], lw.router_w, lw.router_scale, lw.gate_up, lw.down,
+                             lw.expert_scale, k)
+            reps += 1
+            if time.perf_counter() - t0 > 10.0:
+                break
+        el = time.perf_counter() - t0
+        line["cpu_baseline"] = {"value": n_tok * reps / el, "unit": "tokens/s", "cores": oracle.num_threads(),
+                                "kind": "oracle",
+                                "sample": f"{reps} FP64 oracle layer calls on {n_tok} tokens of {wl_name}"}
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    moe.moe_destroy()
+    if ws > 1:
+        dist.destroy_process_group()
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,428 @@
+// moe_api.cu -- the C ABI (include/moe.h): context, workspace, argument checks, path
+// selection and the launches on the caller's stream. Nothing here computes the layer;
+// every step runs in the kernels of moe_route.cu, moe_gemv.cu and moe_gemm_sm100.cu.
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+#include <vector>
+
+#include "../../include/moe.h"
+#include "moe_common.cuh"
+
+namespace {
+
+struct Ctx {
+  bool init = false;
+  int device = -1;
+  int num_sms = 0;
+  int max_tokens = 0, max_d = 0, max_f = 0, max_E = 0, max_k = 0;
+  void *ws = nullptr;
+  size_t ws_bytes = 0;
+  uint32_t *err_host = nullptr;   // mapped pinned word
+  MoeWork W{};
+  __nv_bfloat16 *xbuf[2] = {nullptr, nullptr};   // stack: inter-layer activations
+  float *ylayer = nullptr;                       // stack: intermediate layer output
+  int path = MOE_PATH_AUTO;
+  int gemv_max_tokens = 1 << 30;   // AUTO threshold; lowered once the grouped GEMM is built
+  int last_T = 0, last_k = 0, last_E = 0, last_f = 0;
+  bool last_gemm = false;
+};
+
+Ctx g;
+char g_err[512] = "";
+
+// Per-kernel event timing: pairs of events recorded around each launch of a kernel group.
+struct Prof {
+  bool active = false;
+  std::vector<cudaEvent_t> pool;
+  size_t used = 0;
+  struct Rec { int id; cudaEvent_t a, b; };
+  std::vector<Rec> recs;
+  int open_id[MOE_K_COUNT];
+  cudaEvent_t open_ev[MOE_K_COUNT];
+  bool overflow = false;
+};
+Prof g_prof;
+
+cudaEvent_t prof_event() {
+  if (g_prof.used == g_prof.pool.size()) {
+    if (g_prof.pool.size() >= 65536) { g_prof.overflow = true; return nullptr; }
+    cudaEvent_t e;
+    if (cudaEventCreate(&e) != cudaSuccess) { g_prof.overflow = true; return nullptr; }
+    g_prof.pool.push_back(e);
+  }
+  return g_prof.pool[g_prof.used++];
+}
+
+int fail(int code, const char *fmt, ...) __attribute__((format(printf, 2, 3)));
+int fail(int code, const char *fmt, ...) {
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(g_err, sizeof g_err, fmt, ap);
+  va_end(ap);
+  return code;
+}
+
+int cuda_fail(cudaError_t e, const char *what) {
+  return fail(MOE_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
+}
+
+constexpr int kTileM = 128;   // rows per grouped-GEMM tile
+
+struct Layout {
+  size_t off[24];
+  size_t total;
+};
+
+size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
+
+Layout make_layout(int maxT, int max_d, int max_f, int max_E, int max_k) {
+  const size_t S = (size_t)maxT * max_k;
+  const size_t sizes[] = {
+      (size_t)maxT * max_E * 4,          // 0 logits
+      S * 4,                             // 1 ids
+      S * 4,                             // 2 w
+      (size_t)max_E * 4,                 // 3 counts
+      (size_t)(max_E + 1) * 4,           // 4 offsets
+      S * 4,                             // 5 perm
+      S * 4,                             // 6 inv
+      (size_t)max_E * 4,                 // 7 act
+      16,                                // 8 n_act, n_tiles
+      (size_t)maxT * max_d * 4,          // 9 xprep
+      (size_t)maxT * (max_d / 32) * 4,   // 10 xsum
+      S * max_f * 4,                     // 11 h
+      S * max_f * 4,                     // 12 hprep
+      S * max_d * 4,                     // 13 ybuf / yslot
+      (size_t)(2 + max_d / 8 + 1024) * 4,   // 14 counters
+      S * max_f * 2,                     // 15 hb (bf16)
+      (S / kTileM + max_E + 1) * 8,      // 16 tiles
+      (size_t)maxT * max_d * 2,          // 17 xbuf0
+      (size_t)maxT * max_d * 2,          // 18 xbuf1
+      (size_t)maxT * max_d * 4,          // 19 ylayer
+  };
+  Layout L{};
+  size_t o = 0;
+  for (size_t i = 0; i < sizeof(sizes) / sizeof(sizes[0]); ++i) {
+    L.off[i] = o;
+    o = align_up(o + sizes[i], 256);
+  }
+  L.total = o;
+  return L;
+}
+
+void release() {
+  if (g.ws) cudaFree(g.ws);
+  if (g.err_host) cudaFreeHost(g.err_host);
+  g = Ctx{};
+}
+
+bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+int check_device_error() {
+  if (g.err_host && *reinterpret_cast<volatile uint32_t *>(g.err_host) != 0) {
+    const uint32_t v = *reinterpret_cast<volatile uint32_t *>(g.err_host);
+    *reinterpret_cast<volatile uint32_t *>(g.err_host) = 0;
+    return fail(MOE_ERR_DEVICE_TIMEOUT, "device wait timed out (code %u at site %u)", v & 0xffffu, v >> 16);
+  }
+  return MOE_OK;
+}
+
+int check_shapes(int T, int d, int f, int E, int k) {
+  if (T < 0) return fail(MOE_ERR_BAD_ARG, "T = %d < 0", T);
+  if (d <= 0 || d % 32) return fail(MOE_ERR_BAD_ARG, "d = %d must be a positive multiple of 32", d);
+  if (f <= 0 || f % 32) return fail(MOE_ERR_BAD_ARG, "f = %d must be a positive multiple of 32", f);
+  if (E < 1 || E > MOE_MAX_E) return fail(MOE_ERR_BAD_ARG, "E = %d outside [1, %d]", E, MOE_MAX_E);
+  if (k < 1 || k > E) return fail(MOE_ERR_BAD_ARG, "k = %d outside [1, E = %d]", k, E);
+  return MOE_OK;
+}
+
+int check_limits(int T, int d, int f, int E, int k) {
+  if (!g.init) return fail(MOE_ERR_NOT_INIT, "moe_init has not succeeded");
+  if (T > g.max_tokens) return fail(MOE_ERR_BAD_ARG, "T = %d exceeds max_tokens = %d", T, g.max_tokens);
+  if (d > g.max_d || f > g.max_f || E > g.max_E || k > g.max_k)
+    return fail(MOE_ERR_BAD_ARG, "shape (d=%d, f=%d, E=%d, k=%d) exceeds the moe_init limits (%d, %d, %d, %d)",
+                d, f, E, k, g.max_d, g.max_f, g.max_E, g.max_k);
+  return MOE_OK;
+}
+
+int forward_impl(const void *x, const float *router_w, const float *router_scale, const uint8_t *gate_up_q4,
+                 const uint8_t *down_q4, const float *expert_scale, int T, int d, int f, int E, int k, float *out,
+                 cudaStream_t stream) {
+  MoeLaunch L{stream, false};
+  const bool gemm = (g.path == MOE_PATH_GEMM) || (g.path == MOE_PATH_AUTO && T > g.gemv_max_tokens);
+  int rc;
+  if (gemm) {
+    rc = moe_launch_route_prefill(L, g.W, x, router_w, router_scale, T, d, E, k, g.num_sms, false, kTileM);
+    if (rc) return cuda_fail(cudaGetLastError(), "routing launch");
+    const int max_tiles = (int)((size_t)g.max_tokens * g.max_k / kTileM + g.max_E + 1);
+    rc = moe_launch_gemm_experts(L, g.W, x, gate_up_q4, down_q4, expert_scale, T, d, f, E, k, out, g.num_sms,
+                                 max_tiles);
+    if (rc == -2) return fail(MOE_ERR_BAD_ARG, "shape not supported by the grouped-GEMM path");
+    if (rc) return cuda_fail(cudaGetLastError(), "grouped-GEMM launch");
+  } else {
+    if (T <= 16)
+      rc = moe_launch_route_decode(L, g.W, x, router_w, router_scale, T, d, E, k, g.num_sms);
+    else
+      rc = moe_launch_route_prefill(L, g.W, x, router_w, router_scale, T, d, E, k, g.num_sms, true, 0);
+    if (rc) return cuda_fail(cudaGetLastError(), "routing launch");
+    rc = moe_launch_gemv_experts(L, g.W, gate_up_q4, down_q4, expert_scale, T, d, f, E, k, out, g.num_sms);
+    if (rc == -2) return fail(MOE_ERR_BAD_ARG, "shape not supported by the GEMV path (d, f too large)");
+    if (rc) return cuda_fail(cudaGetLastError(), "GEMV launch");
+  }
+  g.last_T = T;
+  g.last_k = k;
+  g.last_E = E;
+  g.last_f = f;
+  g.last_gemm = gemm;
+  return MOE_OK;
+}
+
+}  // namespace
+
+void moe_prof_mark(cudaStream_t s, int id, bool begin) {
+  if (!g_prof.active || id < 0 || id >= MOE_K_COUNT) return;
+  cudaEvent_t e = prof_event();
+  if (!e) return;
+  cudaEventRecord(e, s);
+  if (begin) {
+    g_prof.open_ev[id] = e;
+  } else if (g_prof.open_ev[id]) {
+    g_prof.recs.push_back({id, g_prof.open_ev[id], e});
+    g_prof.open_ev[id] = nullptr;
+  }
+}
+
+extern "C" {
+
+int moe_profile_begin(void) {
+  if (!g.init) return fail(MOE_ERR_NOT_INIT, "moe_init has not succeeded");
+  g_prof.active = true;
+  g_prof.used = 0;
+  g_prof.recs.clear();
+  g_prof.overflow = false;
+  for (int i = 0; i < MOE_K_COUNT; ++i) g_prof.open_ev[i] = nullptr;
+  return MOE_OK;
+}
+
+int moe_profile_end(float *ms_total, int *launches) {
+  if (!g.init) return fail(MOE_ERR_NOT_INIT, "moe_init has not succeeded");
+  g_prof.active = false;
+  for (int i = 0; i < MOE_K_COUNT; ++i) {
+    if (ms_total) ms_total[i] = 0.f;
+    if (launches) launches[i] = 0;
+  }
+  for (auto &r : g_prof.recs) {
+    cudaError_t e = cudaEventSynchronize(r.b);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaEventSynchronize");
+    float ms = 0.f;
+    e = cudaEventElapsedTime(&ms, r.a, r.b);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaEventElapsedTime");
+    if (ms_total) ms_total[r.id] += ms;
+    if (launches) launches[r.id] += 1;
+  }
+  g_prof.recs.clear();
+  if (g_prof.overflow) return fail(MOE_ERR_BAD_ARG, "too many launches timed (limit 32768)");
+  return MOE_OK;
+}
+
+
+size_t moe_workspace_bytes(int max_tokens, int max_d, int max_f, int max_E, int max_k) {
+  if (max_tokens < 1 || max_d < 32 || max_f < 32 || max_E < 1 || max_k < 1) return 0;
+  return make_layout(max_tokens, max_d, max_f, max_E, max_k).total;
+}
+
+int moe_init(int device, int max_tokens, int max_d, int max_f, int max_E, int max_k) {
+  if (max_tokens < 1) return fail(MOE_ERR_BAD_ARG, "max_tokens = %d < 1", max_tokens);
+  if (max_d < 32 || max_d % 32 || max_f < 32 || max_f % 32)
+    return fail(MOE_ERR_BAD_ARG, "max_d = %d and max_f = %d must be positive multiples of 32", max_d, max_f);
+  if (max_E < 1 || max_E > MOE_MAX_E) return fail(MOE_ERR_BAD_ARG, "max_E = %d outside [1, %d]", max_E, MOE_MAX_E);
+  if (max_k < 1 || max_k > max_E) return fail(MOE_ERR_BAD_ARG, "max_k = %d outside [1, max_E]", max_k);
+  if (g.init) {
+    cudaSetDevice(g.device);
+    cudaDeviceSynchronize();
+    release();
+  }
+  cudaError_t e = cudaSetDevice(device);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaSetDevice");
+  cudaDeviceProp prop;
+  e = cudaGetDeviceProperties(&prop, device);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaGetDeviceProperties");
+  if (prop.major != 10 || prop.minor != 0)
+    return fail(MOE_ERR_UNSUPPORTED_DEVICE, "device %d is sm_%d%d; this library is built for sm_100a", device,
+                prop.major, prop.minor);
+  const Layout Lt = make_layout(max_tokens, max_d, max_f, max_E, max_k);
+  void *ws = nullptr;
+  e = cudaMalloc(&ws, Lt.total);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaMalloc(workspace)");
+  e = cudaMemset(ws, 0, Lt.total);
+  if (e != cudaSuccess) { cudaFree(ws); return cuda_fail(e, "cudaMemset(workspace)"); }
+  uint32_t *eh = nullptr;
+  e = cudaHostAlloc(reinterpret_cast<void **>(&eh), 64, cudaHostAllocMapped);
+  if (e != cudaSuccess) { cudaFree(ws); return cuda_fail(e, "cudaHostAlloc(error word)"); }
+  *eh = 0;
+  uint32_t *ed = nullptr;
+  e = cudaHostGetDevicePointer(reinterpret_cast<void **>(&ed), eh, 0);
+  if (e != cudaSuccess) { cudaFree(ws); cudaFreeHost(eh); return cuda_fail(e, "cudaHostGetDevicePointer"); }
+
+  char *b = static_cast<char *>(ws);
+  MoeWork W{};
+  W.logits = reinterpret_cast<float *>(b + Lt.off[0]);
+  W.ids = reinterpret_cast<int32_t *>(b + Lt.off[1]);
+  W.w = reinterpret_cast<float *>(b + Lt.off[2]);
+  W.counts = reinterpret_cast<int32_t *>(b + Lt.off[3]);
+  W.offsets = reinterpret_cast<int32_t *>(b + Lt.off[4]);
+  W.perm = reinterpret_cast<int32_t *>(b + Lt.off[5]);
+  W.inv = reinterpret_cast<int32_t *>(b + Lt.off[6]);
+  W.act = reinterpret_cast<int32_t *>(b + Lt.off[7]);
+  W.n_act = reinterpret_cast<int32_t *>(b + Lt.off[8]);
+  W.n_tiles = reinterpret_cast<int32_t *>(b + Lt.off[8] + 4);
+  W.xprep = reinterpret_cast<float *>(b + Lt.off[9]);
+  W.xsum = reinterpret_cast<float *>(b + Lt.off[10]);
+  W.h = reinterpret_cast<float *>(b + Lt.off[11]);
+  W.hprep = reinterpret_cast<float *>(b + Lt.off[12]);
+  W.ybuf = reinterpret_cast<float *>(b + Lt.off[13]);
+  W.yslot = W.ybuf;
+  W.counters = reinterpret_cast<uint32_t *>(b + Lt.off[14]);
+  W.hb = reinterpret_cast<__nv_bfloat16 *>(b + Lt.off[15]);
+  W.tiles = reinterpret_cast<int32_t *>(b + Lt.off[16]);
+  W.err = ed;
+
+  g.init = true;
+  g.device = device;
+  g.num_sms = prop.multiProcessorCount;
+  g.max_tokens = max_tokens;
+  g.max_d = max_d;
+  g.max_f = max_f;
+  g.max_E = max_E;
+  g.max_k = max_k;
+  g.ws = ws;
+  g.ws_bytes = Lt.total;
+  g.err_host = eh;
+  g.W = W;
+  g.xbuf[0] = reinterpret_cast<__nv_bfloat16 *>(b + Lt.off[17]);
+  g.xbuf[1] = reinterpret_cast<__nv_bfloat16 *>(b + Lt.off[18]);
+  g.ylayer = reinterpret_cast<float *>(b + Lt.off[19]);
+  return MOE_OK;
+}
+
+int moe_layer_forward(const void *x, const float *router_w, const float *router_scale, const uint8_t *gate_up_q4,
+                      const uint8_t *down_q4, const float *expert_scale, int T, int d, int f, int E, int k, float *out,
+                      void *stream) {
+  int rc = check_shapes(T, d, f, E, k);
+  if (rc) return rc;
+  if (!x || !router_w || !router_scale || !gate_up_q4 || !down_q4 || !expert_scale || !out)
+    return fail(MOE_ERR_BAD_ARG, "null pointer argument");
+  if (!aligned16(gate_up_q4) || !aligned16(down_q4) || !aligned16(router_w) || !aligned16(x))
+    return fail(MOE_ERR_BAD_ALIGN, "x, router_w, gate_up_q4 and down_q4 must be 16-byte aligned");
+  rc = check_limits(T, d, f, E, k);
+  if (rc) return rc;
+  rc = check_device_error();
+  if (rc) return rc;
+  if (T == 0) return MOE_OK;
+  return forward_impl(x, router_w, router_scale, gate_up_q4, down_q4, expert_scale, T, d, f, E, k, out,
+                      static_cast<cudaStream_t>(stream));
+}
+
+int moe_rmsnorm_bf16(const float *y, void *x_out, int T, int d, float eps, void *stream) {
+  if (T < 0 || d < 1) return fail(MOE_ERR_BAD_ARG, "bad shape T = %d, d = %d", T, d);
+  if (!y || !x_out) return fail(MOE_ERR_BAD_ARG, "null pointer argument");
+  if (!g.init) return fail(MOE_ERR_NOT_INIT, "moe_init has not succeeded");
+  if (T == 0) return MOE_OK;
+  if (moe_launch_rmsnorm(static_cast<cudaStream_t>(stream), y, x_out, T, d, eps))
+    return cuda_fail(cudaGetLastError(), "rmsnorm launch");
+  return MOE_OK;
+}
+
+int moe_stack_forward(const void *x_in, int L, const float *const *router_w, const float *const *router_scale,
+                      const uint8_t *const *gate_up_q4, const uint8_t *const *down_q4,
+                      const float *const *expert_scale, int T, int d, int f, int E, int k, float eps, float *out,
+                      void *x_trace, void *stream) {
+  int rc = check_shapes(T, d, f, E, k);
+  if (rc) return rc;
+  if (L < 1) return fail(MOE_ERR_BAD_ARG, "L = %d < 1", L);
+  if (!x_in || !router_w || !router_scale || !gate_up_q4 || !down_q4 || !expert_scale || !out)
+    return fail(MOE_ERR_BAD_ARG, "null pointer argument");
+  for (int i = 0; i < L; ++i) {
+    if (!router_w[i] || !router_scale[i] || !gate_up_q4[i] || !down_q4[i] || !expert_scale[i])
+      return fail(MOE_ERR_BAD_ARG, "null weight pointer for layer %d", i);
+    if (!aligned16(gate_up_q4[i]) || !aligned16(down_q4[i]) || !aligned16(router_w[i]))
+      return fail(MOE_ERR_BAD_ALIGN, "layer %d weights must be 16-byte aligned", i);
+  }
+  if (!aligned16(x_in)) return fail(MOE_ERR_BAD_ALIGN, "x_in must be 16-byte aligned");
+  rc = check_limits(T, d, f, E, k);
+  if (rc) return rc;
+  rc = check_device_error();
+  if (rc) return rc;
+  if (T == 0) return MOE_OK;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const void *xc = x_in;
+  for (int i = 0; i < L; ++i) {
+    if (x_trace) {
+      cudaError_t e = cudaMemcpyAsync(static_cast<char *>(x_trace) + (size_t)i * T * d * 2, xc,
+                                      (size_t)T * d * 2, cudaMemcpyDeviceToDevice, s);
+      if (e != cudaSuccess) return cuda_fail(e, "x_trace copy");
+    }
+    float *yo = (i == L - 1) ? out : g.ylayer;
+    rc = forward_impl(xc, router_w[i], router_scale[i], gate_up_q4[i], down_q4[i], expert_scale[i], T, d, f, E, k,
+                      yo, s);
+    if (rc) return rc;
+    if (i < L - 1) {
+      __nv_bfloat16 *xn = g.xbuf[i & 1];
+      if (moe_launch_rmsnorm(s, yo, xn, T, d, eps)) return cuda_fail(cudaGetLastError(), "rmsnorm launch");
+      xc = xn;
+    }
+  }
+  return MOE_OK;
+}
+
+int moe_set_path(int path, int gemv_max_tokens) {
+  if (path != MOE_PATH_AUTO && path != MOE_PATH_GEMV && path != MOE_PATH_GEMM)
+    return fail(MOE_ERR_BAD_ARG, "unknown path %d", path);
+  if (gemv_max_tokens < 0) return fail(MOE_ERR_BAD_ARG, "gemv_max_tokens = %d < 0", gemv_max_tokens);
+  g.path = path;
+  g.gemv_max_tokens = gemv_max_tokens;
+  return MOE_OK;
+}
+
+void moe_destroy(void) {
+  if (!g.init) return;
+  cudaSetDevice(g.device);
+  cudaDeviceSynchronize();
+  release();
+}
+
+const char *moe_last_error(void) { return g_err; }
+
+int moe_debug_get_routing(int32_t *ids, float *w, int32_t *counts, int32_t *offsets, int32_t *perm, void *stream) {
+  if (!g.init) return fail(MOE_ERR_NOT_INIT, "moe_init has not succeeded");
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const size_t S = (size_t)g.last_T * g.last_k;
+  struct Cp { void *dst; const void *src; size_t n; } cps[] = {
+      {ids, g.W.ids, S * 4}, {w, g.W.w, S * 4}, {counts, g.W.counts, (size_t)g.last_E * 4},
+      {offsets, g.W.offsets, (size_t)(g.last_E + 1) * 4}, {perm, g.W.perm, S * 4}};
+  for (auto &c : cps) {
+    if (!c.dst || c.n == 0) continue;
+    cudaError_t e = cudaMemcpyAsync(c.dst, c.src, c.n, cudaMemcpyDeviceToDevice, s);
+    if (e != cudaSuccess) return cuda_fail(e, "routing copy");
+  }
+  return MOE_OK;
+}
+
+int moe_debug_get_hidden(float *h, void *stream) {
+  if (!g.init) return fail(MOE_ERR_NOT_INIT, "moe_init has not succeeded");
+  if (!h) return fail(MOE_ERR_BAD_ARG, "null pointer argument");
+  if (g.last_T == 0) return MOE_OK;
+  if (moe_launch_hidden_to_slots(static_cast<cudaStream_t>(stream), g.W, h, g.last_T, g.last_f, g.last_k,
+                                 g.last_gemm))
+    return cuda_fail(cudaGetLastError(), "hidden copy");
+  return MOE_OK;
+}
+
+int moe_debug_check(void *stream) {
+  if (!g.init) return fail(MOE_ERR_NOT_INIT, "moe_init has not succeeded");
+  cudaError_t e = cudaStreamSynchronize(static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "cudaStreamSynchronize");
+  return check_device_error();
+}
+
+}  // extern "C"

@@ -1,0 +1,169 @@
+// moe_common.cuh -- shared definitions of the sm_100a routed-MoE kernels: workspace
+// layout, device error word, bounded waits, and thin inline-PTX wrappers for mbarriers
+// and bulk asynchronous copies (cp.async.bulk, no cluster multicast anywhere).
+#pragma once
+
+#include <cuda_runtime.h>
+#include <cuda_fp16.h>
+#include <cuda_bf16.h>
+#include <stdint.h>
+
+#define MOE_QK 32          // weights per Q4_0 block
+#define MOE_QBYTES 18      // bytes per Q4_0 block
+#define MOE_MAX_E 512
+#define MOE_WAIT_NS 2000000000ull   // 2 s bound on any device-side wait
+
+// Device error word: code in the low 16 bits, location in the high 16.
+#define MOE_DEV_ERR_TIMEOUT 1u
+
+// Routing and scratch produced and consumed inside one forward. All device pointers.
+struct MoeWork {
+  float *logits;      // [T, E]
+  int32_t *ids;       // [T*k]
+  float *w;           // [T*k]
+  int32_t *counts;    // [E]
+  int32_t *offsets;   // [E+1]
+  int32_t *perm;      // [T*k]  sorted position -> slot
+  int32_t *inv;       // [T*k]  slot -> sorted position
+  int32_t *act;       // [E]    active experts, ascending; act[E-1..] unused
+  int32_t *n_act;     // [1]
+  float *xprep;       // [T, d] x reordered/scaled for the Q4_0 GEMV (see moe_gemv.cu)
+  float *xsum;        // [T, d/32] per-block sums of x
+  float *h;           // [T*k, f] fp32 hidden (GEMV path), slot order
+  float *hprep;       // [T*k, f] h reordered/scaled for the down GEMV
+  float *ybuf;        // [T*k, d] per-slot expert outputs (GEMV path)
+  uint32_t *counters; // [n] zero-initialised arrival counters (reset by their users)
+  volatile uint32_t *err;   // mapped host word: device error code
+  // grouped-GEMM path
+  __nv_bfloat16 *hb;  // [T*k, f] bf16 hidden in expert-sorted order
+  float *yslot;       // [T*k, d] fp32 per-slot down outputs, expert-sorted order
+  int32_t *tiles;     // [max tiles] (expert, m0) work list
+  int32_t *n_tiles;   // [1]
+};
+
+// ---------------------------------------------------------------- small helpers
+
+__device__ __forceinline__ uint32_t smem_u32(const void *p) {
+  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+__device__ __forceinline__ uint64_t globaltimer_ns() {
+  uint64_t t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  return t;
+}
+
+__device__ __forceinline__ void report_error(volatile uint32_t *err, uint32_t code, uint32_t where) {
+  if (err) {
+    uint32_t v = code | (where << 16);
+    atomicCAS(const_cast<uint32_t *>(err), 0u, v);
+    __threadfence_system();
+  }
+}
+
+// ---------------------------------------------------------------- mbarrier
+
+__device__ __forceinline__ void mbar_init(uint64_t *bar, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count) : "memory");
+}
+
+__device__ __forceinline__ void fence_mbar_init() {
+  asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t *bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)), "r"(bytes)
+               : "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive(uint64_t *bar) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
+}
+
+__device__ __forceinline__ bool mbar_test(uint64_t *bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
+// Wait for the phase with the given parity to complete, at most MOE_WAIT_NS. Returns
+// false (and records a timeout in *err) when the bound expires.
+__device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, volatile uint32_t *err,
+                                          uint32_t where) {
+  if (mbar_test(bar, parity)) return true;
+  uint64_t t0 = globaltimer_ns();
+  while (!mbar_test(bar, parity)) {
+    if (globaltimer_ns() - t0 > MOE_WAIT_NS) {
+      report_error(err, MOE_DEV_ERR_TIMEOUT, where);
+      return false;
+    }
+  }
+  return true;
+}
+
+// ---------------------------------------------------------------- bulk async copy
+
+// 1-D bulk copy global -> shared, completion counted in bytes on `bar`. Both addresses
+// 16-byte aligned, size a multiple of 16.
+__device__ __forceinline__ void bulk_g2s(void *dst, const void *src, uint32_t bytes, uint64_t *bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+          smem_u32(dst)),
+      "l"(src), "r"(bytes), "r"(smem_u32(bar))
+      : "memory");
+}
+
+__device__ __forceinline__ void fence_proxy_async_smem() {
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
+// ---------------------------------------------------------------- programmatic dependent launch
+
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_launch_dependents() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
+// ---------------------------------------------------------------- host-side launch helpers
+
+struct MoeLaunch {
+  cudaStream_t stream;
+  bool pdl;   // launch with programmatic stream serialization
+};
+
+// Kernel groups for the optional per-kernel event timing (moe_profile_begin / _end).
+enum MoeKernelId {
+  MOE_K_ROUTE = 0,        // router + top-k + permutation (one or more launches)
+  MOE_K_GATEUP = 1,       // decode gate_up GEMV + GeGLU
+  MOE_K_DOWN = 2,         // decode down GEMV + combine
+  MOE_K_GEMM_GATEUP = 3,  // prefill gate_up grouped GEMM + GeGLU
+  MOE_K_GEMM_DOWN = 4,    // prefill down grouped GEMM
+  MOE_K_COMBINE = 5,      // prefill ordered combine
+  MOE_K_NORM = 6,         // inter-layer RMSNorm
+  MOE_K_COUNT = 8
+};
+// Record a CUDA event on `s` before (begin) / after a launch of kernel group `id`; a no-op
+// unless timing is active. Defined in moe_api.cu.
+void moe_prof_mark(cudaStream_t s, int id, bool begin);
+
+// Host prototypes of the kernel launchers (defined in the .cu files).
+int moe_launch_route_decode(const MoeLaunch &L, const MoeWork &W, const void *x, const float *router_w,
+                            const float *router_scale, int T, int d, int E, int k, int num_sms);
+int moe_launch_route_prefill(const MoeLaunch &L, const MoeWork &W, const void *x, const float *router_w,
+                             const float *router_scale, int T, int d, int E, int k, int num_sms,
+                             bool want_xprep, int tile_m);
+int moe_launch_gemv_experts(const MoeLaunch &L, const MoeWork &W, const uint8_t *gate_up_q4,
+                            const uint8_t *down_q4, const float *expert_scale, int T, int d, int f,
+                            int E, int k, float *out, int num_sms);
+int moe_launch_gemm_experts(const MoeLaunch &L, const MoeWork &W, const void *x, const uint8_t *gate_up_q4,
+                            const uint8_t *down_q4, const float *expert_scale, int T, int d, int f,
+                            int E, int k, float *out, int num_sms, int max_tiles);
+int moe_launch_rmsnorm(cudaStream_t s, const float *y, void *x_out, int T, int d, float eps);
+int moe_launch_hidden_to_slots(cudaStream_t s, const MoeWork &W, float *h, int T, int f, int k,
+                               bool gemm_path);

@@ -1,0 +1,446 @@
+// moe_route.cu -- router logits, top-k + softmax over the selected logits, and the
+// per-expert histogram / prefix sum / stable token permutation.
+//
+// Definition (page "Gemma 4 26B-A4B it QAT Q4_0 ... NInfer v3 artifact", "What is inside":
+// FP32 router and router scale, 128 routed experts): l[t,e] = sum_i W_r[e,i] x[t,i] in FP32;
+// the k largest logits are selected, equal logits going to the lower expert index;
+// w[t,j] = router_scale * exp(l_j - l_1) / sum_m exp(l_m - l_1) over the selected ones.
+// The permutation is the stable counting sort of slots s = t*k + j by expert id.
+#include "moe_common.cuh"
+
+namespace {
+
+constexpr int kRouteThreads = 512;             // 16 warps
+constexpr int kRouteWarps = kRouteThreads / 32;
+constexpr int kRouteParts = 4;                 // d split in 4 parts per expert (decode)
+constexpr int kDecodeMaxT = 16;
+
+// ---------------------------------------------------------------- x preparation
+//
+// The Q4_0 GEMV turns a 4-bit code q sitting at bit 4j of a 32-bit code word into the
+// exact float q * 2^(s_j) by OR-ing it into the mantissa of 2^23 and subtracting 2^23
+// (s_j = 4j for j <= 4; codes 5..7 are first shifted right by 12, s_j = 4(j-3)). The
+// matching activation is pre-multiplied by 2^(-s_j), which is exact, so the product is
+// q * x. Inside a block, code word i (bytes 4i..4i+3 of the codes) holds at nibble
+// position j = 2m the low nibble of byte 4i+m (element 4i+m) and at j = 2m+1 the high
+// nibble (element 16+4i+m). xprep stores, for each block, the 32 activations in that
+// (word, nibble) order, scaled; xsum stores the plain block sums (for the -8 offset).
+__device__ __forceinline__ float nib_scale(int j) {
+  // 2^-(4j) for j <= 4, 2^-(4(j-3)) for j = 5..7
+  const int s = (j <= 4) ? 4 * j : 4 * (j - 3);
+  return __int_as_float((127 - s) << 23);
+}
+
+__device__ __forceinline__ int nib_elem(int p) {   // position p = 8*i + j -> element
+  const int i = p >> 3, j = p & 7, m = j >> 1;
+  return (j & 1) ? (16 + 4 * i + m) : (4 * i + m);
+}
+
+// one (token, block) per thread, grid-stride
+__device__ void prep_x_range(const __nv_bfloat16 *x, float *xprep, float *xsum, int T, int d,
+                             int tid, int nthreads) {
+  const int nb = d / MOE_QK;
+  for (int it = tid; it < T * nb; it += nthreads) {
+    const int t = it / nb, b = it % nb;
+    const __nv_bfloat16 *xb = x + (size_t)t * d + (size_t)b * MOE_QK;
+    float v[MOE_QK];
+#pragma unroll
+    for (int i = 0; i < MOE_QK; ++i) v[i] = __bfloat162float(xb[i]);
+    float s = 0.f;
+#pragma unroll
+    for (int i = 0; i < MOE_QK; ++i) s += v[i];
+    float *dst = xprep + (size_t)t * d + (size_t)b * MOE_QK;
+#pragma unroll
+    for (int p = 0; p < MOE_QK; ++p) dst[p] = v[nib_elem(p)] * nib_scale(p & 7);
+    xsum[(size_t)t * nb + b] = s;
+  }
+}
+
+// ---------------------------------------------------------------- top-k + softmax
+
+// Warp-level selection for one token. Keys compare by logit (NaN treated as -inf),
+// then by lower index. Writes ids[k], w[k].
+// The selected logits are parked in w[] until the softmax overwrites them.
+__device__ void warp_topk_softmax(const float *lg, int E, int k, float rscale, int32_t *ids, float *w) {
+  const int lane = threadIdx.x & 31;
+  constexpr int kMaxPer = MOE_MAX_E / 32;
+  float v[kMaxPer];
+  uint32_t taken = 0;
+#pragma unroll
+  for (int i = 0; i < kMaxPer; ++i) {
+    const int e = lane + 32 * i;
+    float a = (e < E) ? __ldcg(lg + e) : -INFINITY;
+    if (a != a) a = -INFINITY;
+    v[i] = a;
+    if (e >= E) taken |= 1u << i;
+  }
+  for (int j = 0; j < k; ++j) {
+    // local best among untaken
+    float bv = -INFINITY;
+    int be = 0x7fffffff;
+#pragma unroll
+    for (int i = 0; i < kMaxPer; ++i) {
+      const int e = lane + 32 * i;
+      if (!((taken >> i) & 1u)) {
+        if (v[i] > bv || (v[i] == bv && e < be)) { bv = v[i]; be = e; }
+      }
+    }
+    // warp argmax: larger value, then lower index
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+      const float ov = __shfl_xor_sync(0xffffffffu, bv, o);
+      const int oe = __shfl_xor_sync(0xffffffffu, be, o);
+      if (ov > bv || (ov == bv && oe < be)) { bv = ov; be = oe; }
+    }
+    if ((be & 31) == lane) taken |= 1u << (be >> 5);
+    if (lane == 0) { ids[j] = be; w[j] = __ldcg(lg + be); }
+  }
+  __syncwarp();
+  __threadfence_block();
+  // softmax over the selected logits (original values, so NaN propagates)
+  const float l1 = w[0];
+  float part = 0.f;
+  float ev[MOE_MAX_E / 32];
+#pragma unroll
+  for (int i = 0; i < MOE_MAX_E / 32; ++i) {
+    const int j = lane + 32 * i;
+    ev[i] = (j < k) ? expf(w[j] - l1) : 0.f;
+    part += ev[i];
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) part += __shfl_xor_sync(0xffffffffu, part, o);
+  const float inv = rscale / part;
+  __syncwarp();
+#pragma unroll
+  for (int i = 0; i < MOE_MAX_E / 32; ++i) {
+    const int j = lane + 32 * i;
+    if (j < k) w[j] = ev[i] * inv;
+  }
+  __syncwarp();
+}
+
+// ---------------------------------------------------------------- permutation (one CTA)
+//
+// Stable counting sort of S slots by expert id, all in one CTA of kRouteThreads threads.
+// Warp w owns the contiguous slot range [w*S/NW, (w+1)*S/NW). Pass 1 counts, per warp and
+// expert, using __match_any_sync to rank equal ids inside each 32-slot round; the counts
+// are turned into per-(warp, expert) output bases; pass 2 repeats the ranking and places
+// each slot. Also writes the active-expert list and, if tiles != nullptr, the list of
+// (expert, first row) tiles of tile_m rows for the grouped GEMM.
+struct PermSmem {
+  int32_t cnt[kRouteWarps][MOE_MAX_E];
+  int32_t tot[MOE_MAX_E];
+  int32_t scan_tmp[kRouteWarps * 3];
+};
+
+__device__ void block_exclusive_scan3(int32_t a, int32_t b, int32_t c, int32_t &ea, int32_t &eb,
+                                      int32_t &ec, int32_t *tmp, int32_t &ta, int32_t &tb, int32_t &tc) {
+  // exclusive scan of three values over the CTA (thread order), plus totals
+  const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
+  int32_t ia = a, ib = b, ic = c;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int32_t na = __shfl_up_sync(0xffffffffu, ia, o);
+    const int32_t nb = __shfl_up_sync(0xffffffffu, ib, o);
+    const int32_t nc = __shfl_up_sync(0xffffffffu, ic, o);
+    if (lane >= o) { ia += na; ib += nb; ic += nc; }
+  }
+  if (lane == 31) { tmp[wid] = ia; tmp[kRouteWarps + wid] = ib; tmp[2 * kRouteWarps + wid] = ic; }
+  __syncthreads();
+  int32_t pa = 0, pb = 0, pc = 0;
+  ta = tb = tc = 0;
+  for (int i = 0; i < kRouteWarps; ++i) {
+    const int32_t xa = tmp[i], xb = tmp[kRouteWarps + i], xc = tmp[2 * kRouteWarps + i];
+    if (i < wid) { pa += xa; pb += xb; pc += xc; }
+    ta += xa; tb += xb; tc += xc;
+  }
+  ea = pa + ia - a;
+  eb = pb + ib - b;
+  ec = pc + ic - c;
+  __syncthreads();
+}
+
+__device__ void block_permutation(const int32_t *ids, int S, int E, int32_t *counts, int32_t *offsets,
+                                  int32_t *perm, int32_t *inv, int32_t *act, int32_t *n_act,
+                                  int32_t *tiles, int32_t *n_tiles, int tile_m, PermSmem &sm) {
+  const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
+  for (int i = threadIdx.x; i < kRouteWarps * MOE_MAX_E; i += blockDim.x) (&sm.cnt[0][0])[i] = 0;
+  __syncthreads();
+  const int s0 = (int)((long long)S * wid / kRouteWarps);
+  const int s1 = (int)((long long)S * (wid + 1) / kRouteWarps);
+  const uint32_t lt = (1u << lane) - 1u;
+  // pass 1: per-warp counts
+  for (int base = s0; base < s1; base += 32) {
+    const int s = base + lane;
+    const int id = (s < s1) ? ids[s] : -1 - lane;   // unique negative keys for the tail
+    const uint32_t peers = __match_any_sync(0xffffffffu, id);
+    const int leader = 31 - __clz(peers);
+    if (s < s1 && lane == leader) sm.cnt[wid][id] += __popc(peers);
+    __syncwarp();
+  }
+  __syncthreads();
+  // per-expert totals, then offsets, active list and tile counts by a CTA scan
+  int32_t cnt = 0, a = 0, nt = 0;
+  const int e = threadIdx.x;   // requires E <= blockDim.x
+  if (e < E) {
+    for (int w = 0; w < kRouteWarps; ++w) cnt += sm.cnt[w][e];
+    a = cnt > 0;
+    nt = tiles ? (cnt + tile_m - 1) / tile_m : 0;
+  }
+  int32_t off, aoff, toff, tot, atot, ttot;
+  block_exclusive_scan3(cnt, a, nt, off, aoff, toff, sm.scan_tmp, tot, atot, ttot);
+  if (e < E) {
+    counts[e] = cnt;
+    offsets[e] = off;
+    if (a) act[aoff] = e;
+    int32_t run = off;   // per-warp output bases for this expert
+    for (int w = 0; w < kRouteWarps; ++w) {
+      const int32_t c = sm.cnt[w][e];
+      sm.cnt[w][e] = run;
+      run += c;
+    }
+    if (tiles) {
+      for (int i = 0; i < nt; ++i) {
+        tiles[2 * (toff + i)] = e;
+        tiles[2 * (toff + i) + 1] = i * tile_m;
+      }
+    }
+  }
+  if (threadIdx.x == 0) {
+    offsets[E] = tot;
+    *n_act = atot;
+    if (n_tiles) *n_tiles = ttot;
+  }
+  __syncthreads();
+  // pass 2: placement
+  for (int base = s0; base < s1; base += 32) {
+    const int s = base + lane;
+    const int id = (s < s1) ? ids[s] : -1 - lane;
+    const uint32_t peers = __match_any_sync(0xffffffffu, id);
+    const int leader = 31 - __clz(peers);
+    if (s < s1) {
+      const int pos = sm.cnt[wid][id] + __popc(peers & lt);
+      perm[pos] = s;
+      inv[s] = pos;
+    }
+    __syncwarp();
+    if (s < s1 && lane == leader) sm.cnt[wid][id] += __popc(peers);
+    __syncwarp();
+  }
+  __syncthreads();
+}
+
+// ---------------------------------------------------------------- decode routing kernel
+//
+// T <= 16. CTA b handles experts 4b..4b+3, each split in kRouteParts parts of d; warp
+// (expert, part) accumulates lane-strided float4 chunks of W_r against every token, reduces
+// across the warp by a fixed xor tree, and the parts are summed in order. The last CTA to
+// finish (arrival counter) runs top-k + softmax for all tokens and the permutation.
+struct RouteDecodeSmem {
+  float part[4][kRouteParts][kDecodeMaxT];
+  PermSmem perm;
+  int last;
+};
+
+__global__ void __launch_bounds__(kRouteThreads)
+k_route_decode(const __nv_bfloat16 *__restrict__ x, const float *__restrict__ router_w,
+               const float *__restrict__ router_scale, int T, int d, int E, int k, MoeWork W) {
+  __shared__ RouteDecodeSmem sm;
+  const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
+  const int el = wid / kRouteParts, part = wid % kRouteParts;
+  const int e = blockIdx.x * 4 + el;
+  const int plen = d / kRouteParts;   // multiple of 8
+  if (e < E) {
+    float acc[kDecodeMaxT];
+#pragma unroll
+    for (int t = 0; t < kDecodeMaxT; ++t) acc[t] = 0.f;
+    const float *wr = router_w + (size_t)e * d + (size_t)part * plen;
+    const __nv_bfloat16 *xp = x + (size_t)part * plen;
+    for (int i = lane * 4; i < plen; i += 128) {
+      const float4 wv = __ldg(reinterpret_cast<const float4 *>(wr + i));
+#pragma unroll
+      for (int t = 0; t < kDecodeMaxT; ++t) {
+        if (t < T) {
+          const uint2 xv = __ldg(reinterpret_cast<const uint2 *>(xp + (size_t)t * d + i));
+          const float x0 = __uint_as_float(xv.x << 16), x1 = __uint_as_float(xv.x & 0xffff0000u);
+          const float x2 = __uint_as_float(xv.y << 16), x3 = __uint_as_float(xv.y & 0xffff0000u);
+          float a = acc[t];
+          a = fmaf(wv.x, x0, a);
+          a = fmaf(wv.y, x1, a);
+          a = fmaf(wv.z, x2, a);
+          a = fmaf(wv.w, x3, a);
+          acc[t] = a;
+        }
+      }
+    }
+#pragma unroll
+    for (int t = 0; t < kDecodeMaxT; ++t) {
+      float a = acc[t];
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) a += __shfl_xor_sync(0xffffffffu, a, o);
+      if (lane == 0) sm.part[el][part][t] = a;
+    }
+  }
+  prep_x_range(x, W.xprep, W.xsum, T, d, blockIdx.x * blockDim.x + threadIdx.x,
+               gridDim.x * blockDim.x);
+  __syncthreads();
+  if (threadIdx.x < 4 * kDecodeMaxT) {
+    const int le = threadIdx.x / kDecodeMaxT, t = threadIdx.x % kDecodeMaxT;
+    const int ee = blockIdx.x * 4 + le;
+    if (ee < E && t < T) {
+      float s = sm.part[le][0][t];
+#pragma unroll
+      for (int p = 1; p < kRouteParts; ++p) s += sm.part[le][p][t];
+      W.logits[(size_t)t * E + ee] = s;
+    }
+  }
+  // arrival: the last CTA selects experts for every token and builds the permutation
+  __threadfence();
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    const uint32_t prev = atomicAdd(&W.counters[0], 1u);
+    sm.last = (prev == gridDim.x - 1);
+  }
+  __syncthreads();
+  if (!sm.last) return;
+  __threadfence();
+  const float rs = *router_scale;
+  for (int t = wid; t < T; t += kRouteWarps)
+    warp_topk_softmax(W.logits + (size_t)t * E, E, k, rs, W.ids + (size_t)t * k, W.w + (size_t)t * k);
+  __threadfence_block();
+  __syncthreads();
+  block_permutation(W.ids, T * k, E, W.counts, W.offsets, W.perm, W.inv, W.act, W.n_act, nullptr,
+                    nullptr, 1, sm.perm);
+  if (threadIdx.x == 0) W.counters[0] = 0;
+}
+
+// ---------------------------------------------------------------- prefill routing
+//
+// Router logits as a tiled FP32 product: 64 tokens x 64 experts per CTA, K steps of 32,
+// 256 threads each owning a 4 x 4 patch. Each K step's 32-term partial is formed in its
+// own register before being added to the running sum (two-level accumulation).
+constexpr int kRgBM = 64, kRgBN = 64, kRgBK = 32;
+
+__global__ void __launch_bounds__(256)
+k_router_gemm(const __nv_bfloat16 *__restrict__ x, const float *__restrict__ router_w, int T, int d, int E,
+              float *__restrict__ logits) {
+  __shared__ float xs[kRgBK][kRgBM + 4];
+  __shared__ float ws[kRgBK][kRgBN + 4];
+  const int t0 = blockIdx.x * kRgBM, e0 = blockIdx.y * kRgBN;
+  const int tx = threadIdx.x % 16, ty = threadIdx.x / 16;
+  float acc[4][4] = {};
+  for (int k0 = 0; k0 < d; k0 += kRgBK) {
+    // load x tile: 64 rows x 32 bf16 -> transposed fp32
+    for (int i = threadIdx.x; i < kRgBM * kRgBK / 4; i += 256) {
+      const int r = i / (kRgBK / 4), c4 = (i % (kRgBK / 4)) * 4;
+      const int t = t0 + r;
+      float v0 = 0.f, v1 = 0.f, v2 = 0.f, v3 = 0.f;
+      if (t < T) {
+        const uint2 xv = __ldg(reinterpret_cast<const uint2 *>(x + (size_t)t * d + k0 + c4));
+        v0 = __uint_as_float(xv.x << 16); v1 = __uint_as_float(xv.x & 0xffff0000u);
+        v2 = __uint_as_float(xv.y << 16); v3 = __uint_as_float(xv.y & 0xffff0000u);
+      }
+      xs[c4][r] = v0; xs[c4 + 1][r] = v1; xs[c4 + 2][r] = v2; xs[c4 + 3][r] = v3;
+    }
+    for (int i = threadIdx.x; i < kRgBN * kRgBK / 4; i += 256) {
+      const int r = i / (kRgBK / 4), c4 = (i % (kRgBK / 4)) * 4;
+      const int e = e0 + r;
+      float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
+      if (e < E) v = __ldg(reinterpret_cast<const float4 *>(router_w + (size_t)e * d + k0 + c4));
+      ws[c4][r] = v.x; ws[c4 + 1][r] = v.y; ws[c4 + 2][r] = v.z; ws[c4 + 3][r] = v.w;
+    }
+    __syncthreads();
+    float p[4][4] = {};
+#pragma unroll 8
+    for (int kk = 0; kk < kRgBK; ++kk) {
+      float a[4], b[4];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) a[i] = xs[kk][ty * 4 + i];
+#pragma unroll
+      for (int j = 0; j < 4; ++j) b[j] = ws[kk][tx * 4 + j];
+#pragma unroll
+      for (int i = 0; i < 4; ++i)
+#pragma unroll
+        for (int j = 0; j < 4; ++j) p[i][j] = fmaf(a[i], b[j], p[i][j]);
+    }
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+#pragma unroll
+      for (int j = 0; j < 4; ++j) acc[i][j] += p[i][j];
+    __syncthreads();
+  }
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const int t = t0 + ty * 4 + i;
+    if (t >= T) continue;
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const int e = e0 + tx * 4 + j;
+      if (e < E) logits[(size_t)t * E + e] = acc[i][j];
+    }
+  }
+}
+
+__global__ void __launch_bounds__(256)
+k_topk(const float *__restrict__ logits, const float *__restrict__ router_scale, int T, int E, int k,
+       int32_t *ids, float *w) {
+  const int wid = threadIdx.x >> 5;
+  const int t = blockIdx.x * 8 + wid;
+  if (t >= T) return;
+  warp_topk_softmax(logits + (size_t)t * E, E, k, *router_scale, ids + (size_t)t * k, w + (size_t)t * k);
+}
+
+__global__ void __launch_bounds__(kRouteThreads)
+k_permute(int T, int E, int k, int tile_m, bool want_tiles, MoeWork W) {
+  __shared__ PermSmem sm;
+  block_permutation(W.ids, T * k, E, W.counts, W.offsets, W.perm, W.inv, W.act, W.n_act,
+                    want_tiles ? W.tiles : nullptr, want_tiles ? W.n_tiles : nullptr, tile_m, sm);
+}
+
+__global__ void __launch_bounds__(256)
+k_prep_x(const __nv_bfloat16 *__restrict__ x, int T, int d, MoeWork W) {
+  prep_x_range(x, W.xprep, W.xsum, T, d, blockIdx.x * blockDim.x + threadIdx.x, gridDim.x * blockDim.x);
+}
+
+}  // namespace
+
+// ---------------------------------------------------------------- launchers
+
+static int launch_err() { return cudaGetLastError() == cudaSuccess ? 0 : -1; }
+
+int moe_launch_route_decode(const MoeLaunch &L, const MoeWork &W, const void *x, const float *router_w,
+                            const float *router_scale, int T, int d, int E, int k, int num_sms) {
+  (void)num_sms;
+  if (T > kDecodeMaxT) return -2;
+  const int grid = (E + 3) / 4;
+  moe_prof_mark(L.stream, MOE_K_ROUTE, true);
+  k_route_decode<<<grid, kRouteThreads, 0, L.stream>>>(static_cast<const __nv_bfloat16 *>(x), router_w,
+                                                        router_scale, T, d, E, k, W);
+  if (launch_err()) return -1;
+  moe_prof_mark(L.stream, MOE_K_ROUTE, false);
+  return 0;
+}
+
+int moe_launch_route_prefill(const MoeLaunch &L, const MoeWork &W, const void *x, const float *router_w,
+                             const float *router_scale, int T, int d, int E, int k, int num_sms,
+                             bool want_xprep, int tile_m) {
+  const __nv_bfloat16 *xb = static_cast<const __nv_bfloat16 *>(x);
+  dim3 g1((T + kRgBM - 1) / kRgBM, (E + kRgBN - 1) / kRgBN);
+  moe_prof_mark(L.stream, MOE_K_ROUTE, true);
+  k_router_gemm<<<g1, 256, 0, L.stream>>>(xb, router_w, T, d, E, W.logits);
+  if (launch_err()) return -1;
+  k_topk<<<(T + 7) / 8, 256, 0, L.stream>>>(W.logits, router_scale, T, E, k, W.ids, W.w);
+  if (launch_err()) return -1;
+  k_permute<<<1, kRouteThreads, 0, L.stream>>>(T, E, k, tile_m, tile_m > 0, W);
+  if (launch_err()) return -1;
+  if (want_xprep) {
+    const int nb = d / MOE_QK;
+    const int items = T * nb;
+    int grid = (items + 255) / 256;
+    if (grid > 4 * num_sms) grid = 4 * num_sms;
+    k_prep_x<<<grid, 256, 0, L.stream>>>(xb, T, d, W);
+    if (launch_err()) return -1;
+  }
+  moe_prof_mark(L.stream, MOE_K_ROUTE, false);
+  return 0;
+}

@@ -1,0 +1,209 @@
+"""GPU parity: the CUDA path through the C ABI against the FP64 oracle on seeded inputs.
+
+Small shapes spanning several tiles and ragged tails, every edge case of the routing,
+and the five full-size workloads (sampled where the oracle would take minutes).
+"""
+import numpy as np
+import pytest
+import torch
+
+import moe_inputs as mi
+import oracle
+import mixture_experts_gemv_b200 as moe
+from gpu_util import (DevLayer, TOL_GEMM, TOL_GEMV, check_routing, dev, ensure_init, rel_err,
+                      run_layer)
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _built():
+    from mixture_experts_gemv_b200 import build
+    build.build()
+    yield
+    moe.moe_set_path(moe.MOE_PATH_AUTO, 16)
+
+
+def _tol(path, T):
+    if path == moe.MOE_PATH_GEMV:
+        return TOL_GEMV
+    if path == moe.MOE_PATH_GEMM:
+        return TOL_GEMM
+    return TOL_GEMV if T <= 16 else TOL_GEMM
+
+
+def _check_full(x, lw, k, path, tokens=None):
+    dl = DevLayer(lw)
+    res = run_layer(x, dl, k, path)
+    logits = oracle.router_logits(x, lw.router_w)
+    ids, w, flags = oracle.topk_softmax(logits, k, float(lw.router_scale[0]))
+    check_routing(res, ids, w, flags, k, lw.E)
+    T = x.shape[0]
+    tok = np.arange(T) if tokens is None else np.asarray(tokens)
+    tok = tok[(flags[tok] & 1) == 0]
+    ref = oracle.experts_combine(x, lw.gate_up, lw.down, lw.expert_scale, ids, w, lw.d, lw.f, tokens=tok)
+    err = rel_err(res["out"][tok], ref)
+    assert err <= _tol(path, T), f"relative error {err:.3e}"
+    return res, err
+
+
+# ------------------------------------------------------------------ small shapes
+
+SMALL = [  # (E, k, T, d, f)
+    (4, 1, 1, 64, 32), (4, 4, 7, 64, 32), (8, 2, 33, 256, 64), (8, 8, 2, 96, 64),
+    (128, 8, 1, 256, 96), (128, 8, 33, 512, 128), (128, 2, 300, 256, 64), (128, 128, 3, 64, 32),
+    (16, 3, 17, 2816, 64), (6, 2, 16, 320, 704),
+]
+
+
+@pytest.mark.parametrize("E,k,T,d,f", SMALL)
+def test_small_shapes_gemv(E, k, T, d, f):
+    lw = mi.make_layer(seed=E * 1000 + T, layer=0, d=d, f=f, E=E)
+    x = mi.make_tokens(E + T, T, d)
+    _check_full(x, lw, k, moe.MOE_PATH_GEMV)
+
+
+def test_zero_tokens_is_a_noop():
+    lw = mi.make_layer(seed=1, d=64, f=32, E=4)
+    dl = DevLayer(lw)
+    ensure_init(1, 64, 32, 4, 2)
+    out = torch.full((1, 64), 7.0, device="cuda:0")
+    x = torch.zeros((1, 64), dtype=torch.int16, device="cuda:0")
+    moe.moe_layer_forward(x, dl.router_w, dl.router_scale, dl.gate_up, dl.down, dl.expert_scale,
+                          0, 64, 32, 4, 2, out)
+    moe.moe_debug_check()
+    assert (out.cpu() == 7.0).all()
+
+
+def test_tied_logits_pick_lower_index():
+    E, d, f, k = 8, 64, 32, 2
+    lw = mi.make_layer(seed=3, d=d, f=f, E=E)
+    lw.router_w[:] = 0.0
+    lw.router_w[[1, 3, 5], 0] = 1.0          # experts 1, 3, 5 tie for the top logit
+    x = mi.make_tokens(5, 4, d)
+    x[:, 0] = mi.f32_to_bf16_bits(np.array([2.0], np.float32))[0]
+    res = run_layer(x, DevLayer(lw), k, moe.MOE_PATH_GEMV)
+    assert (res["ids"].reshape(4, k) == np.array([1, 3])).all()
+
+
+def test_router_scale_and_expert_scale_enter_the_output():
+    E, d, f, k, T = 8, 128, 64, 2, 3
+    lw = mi.make_layer(seed=4, d=d, f=f, E=E)
+    x = mi.make_tokens(6, T, d)
+    base = run_layer(x, DevLayer(lw), k, moe.MOE_PATH_GEMV)["out"]
+    lw.router_scale[0] = 0.5
+    half = run_layer(x, DevLayer(lw), k, moe.MOE_PATH_GEMV)["out"]
+    assert np.allclose(half, 0.5 * base, rtol=1e-6, atol=1e-12)
+    _check_full(x, lw, k, moe.MOE_PATH_GEMV)
+
+
+def test_nan_input_propagates():
+    E, d, f, k, T = 8, 64, 32, 2, 3
+    lw = mi.make_layer(seed=5, d=d, f=f, E=E)
+    x = mi.make_tokens(7, T, d)
+    x[1, 5] = 0x7FC0    # bf16 NaN in token 1
+    out = run_layer(x, DevLayer(lw), k, moe.MOE_PATH_GEMV, want_routing=False)["out"]
+    assert np.isnan(out[1]).all()
+    assert np.isfinite(out[0]).all() and np.isfinite(out[2]).all()
+
+
+def test_deterministic_bitwise():
+    lw = mi.make_layer(seed=8, d=512, f=128, E=32)
+    x = mi.make_tokens(9, 8, 512)
+    dl = DevLayer(lw)
+    a = run_layer(x, dl, 4, moe.MOE_PATH_GEMV)["out"]
+    b = run_layer(x, dl, 4, moe.MOE_PATH_GEMV)["out"]
+    assert np.array_equal(a.view(np.uint32), b.view(np.uint32))
+
+
+def test_hidden_matches_oracle():
+    E, d, f, k, T = 16, 256, 96, 3, 5
+    lw = mi.make_layer(seed=12, d=d, f=f, E=E)
+    x = mi.make_tokens(13, T, d)
+    run_layer(x, DevLayer(lw), k, moe.MOE_PATH_GEMV)
+    h = torch.empty((T * k, f), dtype=torch.float32, device="cuda:0")
+    moe.moe_debug_get_hidden(h)
+    torch.cuda.synchronize()
+    logits = oracle.router_logits(x, lw.router_w)
+    ids, w, flags = oracle.topk_softmax(logits, k, 1.0)
+    _, href = oracle.experts_combine(x, lw.gate_up, lw.down, lw.expert_scale, ids, w, d, f, want_h=True)
+    assert rel_err(h.cpu().numpy().reshape(T, k, f), href) <= TOL_GEMV
+
+
+def test_rmsnorm_matches_oracle_up_to_rounding_ties():
+    rng = np.random.default_rng(3)
+    y = (rng.standard_normal((4, 2816)) * 0.01).astype(np.float32)
+    ensure_init(4, 2816, 704, 128, 8)
+    xo = torch.empty((4, 2816), dtype=torch.int16, device="cuda:0")
+    moe.moe_rmsnorm_bf16(dev(y), xo, 4, 2816, 1e-6)
+    torch.cuda.synchronize()
+    got = xo.cpu().numpy().view(np.uint16)
+    ref = oracle.rmsnorm_bf16(y.astype(np.float64), 1e-6)
+    diff = got != ref
+    # a differing element must sit within FP32 error of a bf16 rounding midpoint
+    yd = y.astype(np.float64)
+    val = yd / np.sqrt((yd ** 2).mean(1, keepdims=True) + 1e-6)
+    for t, i in zip(*np.nonzero(diff)):
+        a, b = int(got[t, i]), int(ref[t, i])
+        assert abs(a - b) == 1
+        lo, hi = sorted([a, b])
+        mid = (mi.bf16_bits_to_f32(np.array([lo], np.uint16))[0].astype(np.float64) +
+               mi.bf16_bits_to_f32(np.array([hi], np.uint16))[0].astype(np.float64)) / 2
+        assert abs(val[t, i] - mid) <= 1e-6 * abs(mid)
+    assert diff.mean() < 1e-3
+
+
+# ------------------------------------------------------------------ full-size workloads
+
+def test_layer_T1():
+    wl = mi.make_workload("layer_T1")
+    _check_full(wl.x, wl.layers[0], wl.k, moe.MOE_PATH_AUTO)
+
+
+def test_decode_T8():
+    wl = mi.make_workload("decode_T8")
+    _check_full(wl.x, wl.layers[0], wl.k, moe.MOE_PATH_AUTO)
+
+
+def test_skewed_T512_sampled():
+    wl = mi.make_workload("skewed_T512")
+    lw = wl.layers[0]
+    rng = np.random.default_rng(0)
+    tok = np.sort(rng.choice(wl.T, 48, replace=False))
+    res, err = _check_full(wl.x, lw, wl.k, moe.MOE_PATH_AUTO, tokens=tok)
+    counts = res["counts"]
+    assert (counts > 100).sum() >= 3 and (counts <= 2).sum() >= 64
+
+
+def test_prefill_T4096_sampled():
+    wl = mi.make_workload("prefill_T4096")
+    rng = np.random.default_rng(1)
+    tok = np.sort(rng.choice(wl.T, 32, replace=False))
+    _check_full(wl.x, wl.layers[0], wl.k, moe.MOE_PATH_AUTO, tokens=tok)
+
+
+def test_stack_teacher_forced():
+    """Layer i's oracle consumes the GPU's own bf16 input x_i (recorded by x_trace)."""
+    L = 3
+    wl = mi.make_workload("stack30_T1", n_layers=L)
+    d, f, E, k = mi.D_MODEL, mi.D_FF, mi.N_EXPERTS, wl.k
+    dls = [DevLayer(lw) for lw in wl.layers]
+    ensure_init(1, d, f, E, k)
+    moe.moe_set_path(moe.MOE_PATH_AUTO, 16)
+    out = torch.empty((1, d), dtype=torch.float32, device="cuda:0")
+    trace = torch.empty((L, 1, d), dtype=torch.int16, device="cuda:0")
+    moe.moe_stack_forward(dev(wl.x), [q.router_w for q in dls], [q.router_scale for q in dls],
+                          [q.gate_up for q in dls], [q.down for q in dls], [q.expert_scale for q in dls],
+                          1, d, f, E, k, 1e-6, out, trace)
+    moe.moe_debug_check()
+    xs = trace.cpu().numpy().view(np.uint16)
+    assert np.array_equal(xs[0], wl.x)
+    for i, lw in enumerate(wl.layers):
+        ref, ids, w, flags = oracle.moe_layer(xs[i], lw.router_w, lw.router_scale, lw.gate_up, lw.down,
+                                              lw.expert_scale, k)
+        if i + 1 < L:
+            nxt = oracle.rmsnorm_bf16(ref)
+            close = np.abs(nxt.astype(np.int32) - xs[i + 1].astype(np.int32)) <= 1
+            assert close.all() and (nxt != xs[i + 1]).mean() < 0.02
+        else:
+            assert rel_err(out.cpu().numpy(), ref) <= TOL_GEMV
