@@ -23,7 +23,7 @@ struct Ctx {
   __nv_bfloat16 *xbuf[2] = {nullptr, nullptr};   // stack: inter-layer activations
   float *ylayer = nullptr;                       // stack: intermediate layer output
   int path = MOE_PATH_AUTO;
-  int gemv_max_tokens = 1 << 30;   // AUTO threshold; lowered once the grouped GEMM is built
+  int gemv_max_tokens = 16;   // AUTO: GEMV for T <= 16, grouped GEMM above
   int last_T = 0, last_k = 0, last_E = 0, last_f = 0;
   bool last_gemm = false;
 };
@@ -78,6 +78,7 @@ size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
 
 Layout make_layout(int maxT, int max_d, int max_f, int max_E, int max_k) {
   const size_t S = (size_t)maxT * max_k;
+  const size_t prow = (S / kTileM + max_E + 1) * kTileM;   // padded tile rows
   const size_t sizes[] = {
       (size_t)maxT * max_E * 4,          // 0 logits
       S * 4,                             // 1 ids
@@ -94,11 +95,13 @@ Layout make_layout(int maxT, int max_d, int max_f, int max_E, int max_k) {
       S * max_f * 4,                     // 12 hprep
       S * max_d * 4,                     // 13 ybuf / yslot
       (size_t)(2 + max_d / 8 + 1024) * 4,   // 14 counters
-      S * max_f * 2,                     // 15 hb (bf16)
+      prow * max_f * 2,                  // 15 hb (bf16, padded tiles)
       (S / kTileM + max_E + 1) * 8,      // 16 tiles
       (size_t)maxT * max_d * 2,          // 17 xbuf0
       (size_t)maxT * max_d * 2,          // 18 xbuf1
       (size_t)maxT * max_d * 4,          // 19 ylayer
+      prow * max_d * 2,                  // 20 xg (bf16, padded tiles)
+      (size_t)max_E * 4,                 // 21 toff
   };
   Layout L{};
   size_t o = 0;
@@ -285,6 +288,8 @@ int moe_init(int device, int max_tokens, int max_d, int max_f, int max_E, int ma
   W.counters = reinterpret_cast<uint32_t *>(b + Lt.off[14]);
   W.hb = reinterpret_cast<__nv_bfloat16 *>(b + Lt.off[15]);
   W.tiles = reinterpret_cast<int32_t *>(b + Lt.off[16]);
+  W.xg = reinterpret_cast<__nv_bfloat16 *>(b + Lt.off[20]);
+  W.toff = reinterpret_cast<int32_t *>(b + Lt.off[21]);
   W.err = ed;
 
   g.init = true;

@@ -1,11 +1,486 @@
 // moe_gemm_sm100.cu -- prefill path: grouped GEMMs of the routed experts on the sm_100
-// tensor cores (tcgen05 / TMEM). Placeholder until the kernels land.
+// tensor cores (tcgen05.mma, accumulators in TMEM), with the Q4_0 weights dequantised to
+// bf16 in shared memory and GELU-tanh gating fused into the gate_up epilogue.
+//
+// Page "Gemma 4 26B-A4B it QAT Q4_0 ... NInfer v3 artifact", "What is inside": expert-major
+// Q4_0 [gate; up] (2 x 704 rows) and down (2,816 rows) multiplied in place. With the slots
+// of expert e sorted together (stable permutation) the layer is, per expert, two GEMMs:
+//   H_e = gelu_tanh(X_e Wg_e^T) * (X_e Wu_e^T)      [M_e x f]
+//   Y_e = H_e Wd_e^T                                [M_e x d]
+// followed by out[t] = sum_j w_tj * s_e * Y[slot(t, j)] in j order.
+//
+// Layout: the routed rows of each expert are padded to whole 128-row tiles; tile i of the
+// tile list covers padded rows [128 i, 128 i + 128). X is gathered into that padded order
+// (k_gather_x) so both GEMMs read their A operand with plain 2-D TMA tiles (128 rows x 64
+// bf16, 128-byte swizzle, no multicast). The B operand (weights) never exists in bf16 in
+// global memory: producer warps read Q4_0 blocks, decode (q - 8) * d to bf16 and write the
+// swizzled K-major tile that tcgen05.mma reads.
+//
+// One CTA per SM, persistent over (tile, n-tile) work items, warp-specialised:
+//   warps 0-3  epilogue: tcgen05.ld of the 128 x 128 FP32 accumulator (lane = row)
+//   warp  4    TMEM allocation; lane 0 issues tcgen05.mma (M = 128, N = 128, K = 16)
+//   warps 5-12 producers: TMA for A, Q4_0 -> bf16 dequantisation for B
+// Shared-memory stages are handed over with mbarriers (every wait is time-bounded); the
+// accumulator is double-buffered in TMEM so the epilogue of one item overlaps the next.
+#include <cuda.h>
+#include <cudaTypedefs.h>
+
 #include "moe_common.cuh"
+
+namespace {
+
+constexpr int BM = 128, BN = 128, BK = 64;
+constexpr int kStages = 5;
+constexpr int kEpiWarps = 4;
+constexpr int kMmaWarp = 4;
+constexpr int kProdWarps = 8;
+constexpr int kProdThreads = kProdWarps * 32;
+constexpr int kThreads = (kEpiWarps + 1 + kProdWarps) * 32;   // 416
+constexpr uint32_t kTileBytes = BM * BK * 2;                  // 16 KB (A); B is BN x BK, same
+constexpr uint32_t kStageBytes = 2 * kTileBytes;
+constexpr uint32_t kTmemCols = 2 * BN;                        // two accumulator buffers
+constexpr int kSmemBytes = kStages * kStageBytes + 1024;
+
+// UMMA instruction descriptor, kind::f16: D FP32 (bits 4-5 = 1), A and B bf16 (bits 7-9,
+// 10-12 = 1), both K-major (bits 15, 16 = 0), N >> 3 in bits 17-22, M >> 4 in bits 24-28.
+constexpr uint32_t kIdesc = (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(BN >> 3) << 17) |
+                            ((uint32_t)(BM >> 4) << 24);
+
+// Shared-memory matrix descriptor: K-major operand, 128-byte swizzle (layout type 2),
+// rows of 128 bytes in 8-row atoms of 1024 bytes (stride byte offset 1024), version 1.
+__device__ __forceinline__ uint64_t sw128_desc(uint32_t saddr) {
+  return (uint64_t)((saddr & 0x3FFFFu) >> 4) | (1ull << 16) | (64ull << 32) | (1ull << 46) | (2ull << 61);
+}
+
+struct GemmBars {
+  uint64_t full[kStages];
+  uint64_t empty[kStages];
+  uint64_t acc_full[2];
+  uint64_t acc_empty[2];
+  uint32_t tmem_base;
+  int abort_flag;
+};
+
+// ---------------------------------------------------------------- PTX wrappers
+
+__device__ __forceinline__ void mbar_expect_tx(uint64_t *bar, uint32_t bytes) {
+  asm volatile("mbarrier.expect_tx.relaxed.cta.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(bytes)
+               : "memory");
+}
+
+__device__ __forceinline__ void tma_load_2d(void *dst, const CUtensorMap *map, int c0, int c1, uint64_t *bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], "
+      "[%4];" ::"r"(smem_u32(dst)),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(c0), "r"(c1), "r"(smem_u32(bar))
+      : "memory");
+}
+
+__device__ __forceinline__ void tmem_alloc(uint32_t *dst, uint32_t ncols) {
+  asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(dst)), "r"(ncols)
+               : "memory");
+}
+__device__ __forceinline__ void tmem_relinquish() {
+  asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void tmem_dealloc(uint32_t taddr, uint32_t ncols) {
+  asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols) : "memory");
+}
+__device__ __forceinline__ void umma_bf16(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "l"(adesc), "l"(bdesc), "r"(kIdesc), "r"(accumulate)
+      : "memory");
+}
+__device__ __forceinline__ void umma_commit(uint64_t *bar) {
+  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(smem_u32(bar))
+               : "memory");
+}
+__device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
+__device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
+
+__device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t (&r)[16]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, "
+      "%15}, [%16];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+        "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
+      : "r"(taddr));
+}
+__device__ __forceinline__ void tmem_ld_wait() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
+
+__device__ __forceinline__ void st_shared_v4(uint32_t addr, uint32_t a, uint32_t b, uint32_t c, uint32_t d) {
+  asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(a), "r"(b), "r"(c), "r"(d) : "memory");
+}
+
+__device__ __forceinline__ float gelu_tanh_f(float z) {
+  const float c = 0.7978845608028654f;   // sqrt(2/pi)
+  return 0.5f * z * (1.0f + tanhf(c * (z + 0.044715f * z * z * z)));
+}
+
+__device__ __forceinline__ uint32_t pack_bf16(float a, float b) {
+  const __nv_bfloat162 h = __floats2bfloat162_rn(a, b);
+  return *reinterpret_cast<const uint32_t *>(&h);
+}
+
+// ---------------------------------------------------------------- Q4_0 -> bf16
+
+// Four consecutive code bytes (one word) -> the bf16 pairs (q - 8) * d of their low nibbles
+// (lo01: bytes 0,1; lo23: bytes 2,3) and high nibbles (hi01, hi23). A code q is first made
+// the bf16 value 128 + q by OR-ing it into the mantissa of 128 (exact), then 136 is
+// subtracted (exact) and the result is multiplied by d (one rounding).
+__device__ __forceinline__ void dq_word(uint32_t w, __nv_bfloat162 d2, uint32_t &lo01, uint32_t &lo23,
+                                        uint32_t &hi01, uint32_t &hi23) {
+  const uint32_t v01 = __byte_perm(w, 0u, 0x4140u);   // [b0, 0, b1, 0]
+  const uint32_t v23 = __byte_perm(w, 0u, 0x4342u);   // [b2, 0, b3, 0]
+  const uint32_t kMag = 0x43004300u;                  // bf16 (128, 128)
+  const uint32_t l01 = (v01 & 0x000F000Fu) | kMag;
+  const uint32_t l23 = (v23 & 0x000F000Fu) | kMag;
+  const uint32_t h01 = ((v01 >> 4) & 0x000F000Fu) | kMag;
+  const uint32_t h23 = ((v23 >> 4) & 0x000F000Fu) | kMag;
+  const __nv_bfloat162 c136 = __halves2bfloat162(__ushort_as_bfloat16((unsigned short)0x4308),
+                                                 __ushort_as_bfloat16((unsigned short)0x4308));
+  auto cv = [&](uint32_t x) -> uint32_t {
+    __nv_bfloat162 v = *reinterpret_cast<const __nv_bfloat162 *>(&x);
+    v = __hmul2(__hsub2(v, c136), d2);
+    return *reinterpret_cast<const uint32_t *>(&v);
+  };
+  lo01 = cv(l01);
+  lo23 = cv(l23);
+  hi01 = cv(h01);
+  hi23 = cv(h23);
+}
+
+// Raw words of one 18-byte block at global byte address p (2-byte aligned): the 20-byte
+// window starting at p rounded down to 4 bytes. Never reads past the end of a Q4_0 matrix
+// whose rows are whole blocks (the last block of a matrix always starts at 2 mod 4).
+struct RawBlk {
+  uint32_t w[5];
+  uint32_t sh;
+};
+__device__ __forceinline__ RawBlk ld_raw_blk(const uint8_t *p) {
+  RawBlk r;
+  const uintptr_t a = reinterpret_cast<uintptr_t>(p);
+  const uint32_t *wp = reinterpret_cast<const uint32_t *>(a & ~(uintptr_t)3);
+#pragma unroll
+  for (int i = 0; i < 5; ++i) r.w[i] = __ldg(wp + i);
+  r.sh = (uint32_t)(a & 3u) * 8u;
+  return r;
+}
+
+// Decode one block into its 4 swizzled 16-byte chunks of row `row` (chunks cbase..cbase+3).
+__device__ __forceinline__ void store_blk_bf16(const RawBlk &r, uint32_t tile_saddr, int row, int cbase) {
+  const float d = __half2float(__ushort_as_half((unsigned short)((r.w[0] >> r.sh) & 0xffffu)));
+  const __nv_bfloat162 d2 = __float2bfloat162_rn(d);
+  const uint32_t s2 = r.sh + 16u;
+  uint32_t q[4];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) q[i] = __funnelshift_rc(r.w[i], r.w[i + 1], s2);
+  uint32_t lo[8], hi[8];   // element pairs (0,1),(2,3),...,(14,15) and (16,17),...,(30,31)
+#pragma unroll
+  for (int i = 0; i < 4; ++i) dq_word(q[i], d2, lo[2 * i], lo[2 * i + 1], hi[2 * i], hi[2 * i + 1]);
+  const uint32_t rowbase = tile_saddr + (uint32_t)row * 128u;
+  const uint32_t x = (uint32_t)(row & 7);
+  st_shared_v4(rowbase + (((uint32_t)(cbase + 0) ^ x) << 4), lo[0], lo[1], lo[2], lo[3]);   // elements 0-7
+  st_shared_v4(rowbase + (((uint32_t)(cbase + 1) ^ x) << 4), lo[4], lo[5], lo[6], lo[7]);   // 8-15
+  st_shared_v4(rowbase + (((uint32_t)(cbase + 2) ^ x) << 4), hi[0], hi[1], hi[2], hi[3]);   // 16-23
+  st_shared_v4(rowbase + (((uint32_t)(cbase + 3) ^ x) << 4), hi[4], hi[5], hi[6], hi[7]);   // 24-31
+}
+
+// ---------------------------------------------------------------- the grouped GEMM
+
+// GATEUP: A = gathered x [rows, d], B = gate rows n0..n0+63 and up rows f+n0..f+n0+63,
+//         K = d; epilogue h = gelu(gate) * up -> hb (bf16, padded row order).
+// DOWN:   A = hb [rows, f], B = down rows n0..n0+127, K = f; epilogue y * w * s -> yslot
+//         (bf16, slot order).
+template <bool GATEUP>
+__global__ void __launch_bounds__(kThreads, 1)
+k_moe_gemm(const __grid_constant__ CUtensorMap tmap_a, const uint8_t *__restrict__ wq,
+           const float *__restrict__ expert_scale, int d, int f, int k, MoeWork W) {
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  __shared__ GemmBars bars;
+  const uint32_t sbase = (smem_u32(smem_raw) + 1023u) & ~1023u;
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int K = GATEUP ? d : f;
+  const int ksteps = K / BK;
+  const int n_ntiles = GATEUP ? f / (BN / 2) : d / BN;
+  const int nb_row = K / MOE_QK;                       // Q4_0 blocks per weight row
+  const size_t rb = (size_t)nb_row * MOE_QBYTES;       // bytes per weight row
+  const size_t expert_bytes = (size_t)(GATEUP ? 2 * f : d) * rb;
+  const int n_tiles = *W.n_tiles;
+  const int n_items = n_tiles * n_ntiles;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kStages; ++s) {
+      mbar_init(&bars.full[s], kProdThreads);
+      mbar_init(&bars.empty[s], 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&bars.acc_full[b], 1);
+      mbar_init(&bars.acc_empty[b], kEpiWarps * 32);
+    }
+    bars.abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == kMmaWarp) {
+    tmem_alloc(&bars.tmem_base, kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = bars.tmem_base;
+
+  if (warp >= kMmaWarp + 1) {
+    // ------------------------------------------------------------ producers
+    const int pt = threadIdx.x - (kMmaWarp + 1) * 32;   // 0..255
+    const int row = pt >> 1, blk = pt & 1;              // one (row, block) of the B tile per step
+    int it = 0;
+    bool ok = true;
+    for (int item = blockIdx.x; item < n_items && ok; item += gridDim.x) {
+      const int tile = item / n_ntiles, nt = item % n_ntiles;
+      const int e = W.tiles[2 * tile];
+      const uint8_t *wrow;
+      if (GATEUP) {
+        const int half = BN / 2;
+        const int grow = (row < half) ? (nt * half + row) : (f + nt * half + row - half);
+        wrow = wq + (size_t)e * expert_bytes + (size_t)grow * rb;
+      } else {
+        wrow = wq + (size_t)e * expert_bytes + (size_t)(nt * BN + row) * rb;
+      }
+      RawBlk nxt = ld_raw_blk(wrow + (size_t)blk * MOE_QBYTES);
+      for (int ks = 0; ks < ksteps; ++ks, ++it) {
+        const int s = it % kStages;
+        const uint32_t par = ((uint32_t)(it / kStages) & 1u) ^ 1u;
+        if (!mbar_wait(&bars.empty[s], par, W.err, 10)) { ok = false; break; }
+        const uint32_t a_saddr = sbase + (uint32_t)s * kStageBytes;
+        const uint32_t b_saddr = a_saddr + kTileBytes;
+        if (pt == 0) {
+          mbar_expect_tx(&bars.full[s], kTileBytes);
+          tma_load_2d(reinterpret_cast<void *>(smem_raw + (a_saddr - smem_u32(smem_raw))), &tmap_a, ks * BK,
+                      tile * BM, &bars.full[s]);
+        }
+        const RawBlk cur = nxt;
+        if (ks + 1 < ksteps) nxt = ld_raw_blk(wrow + (size_t)((ks + 1) * 2 + blk) * MOE_QBYTES);
+        store_blk_bf16(cur, b_saddr, row, blk * 4);
+        fence_proxy_async_smem();
+        mbar_arrive(&bars.full[s]);
+      }
+    }
+    if (!ok) atomicExch(&bars.abort_flag, 1);
+  } else if (warp == kMmaWarp) {
+    // ------------------------------------------------------------ MMA issue (one thread)
+    if (lane == 0) {
+      int it = 0, j = 0;
+      bool ok = true;
+      for (int item = blockIdx.x; item < n_items && ok; item += gridDim.x, ++j) {
+        const int b = j & 1;
+        const uint32_t upar = ((uint32_t)(j >> 1) & 1u) ^ 1u;
+        if (!mbar_wait(&bars.acc_empty[b], upar, W.err, 11)) { ok = false; break; }
+        tc_fence_after();
+        const uint32_t dtm = tmem + (uint32_t)(b * BN);
+        for (int ks = 0; ks < ksteps; ++ks, ++it) {
+          const int s = it % kStages;
+          const uint32_t par = (uint32_t)(it / kStages) & 1u;
+          if (!mbar_wait(&bars.full[s], par, W.err, 12)) { ok = false; break; }
+          tc_fence_after();
+          const uint32_t a_saddr = sbase + (uint32_t)s * kStageBytes;
+          const uint32_t b_saddr = a_saddr + kTileBytes;
+#pragma unroll
+          for (int kk = 0; kk < BK / 16; ++kk)
+            umma_bf16(dtm, sw128_desc(a_saddr + kk * 32), sw128_desc(b_saddr + kk * 32),
+                      (ks > 0 || kk > 0) ? 1u : 0u);
+          umma_commit(&bars.empty[s]);
+        }
+        if (!ok) break;
+        umma_commit(&bars.acc_full[b]);
+      }
+      if (!ok) atomicExch(&bars.abort_flag, 1);
+    }
+    __syncwarp();
+  } else {
+    // ------------------------------------------------------------ epilogue (lane = row)
+    const int r = warp * 32 + lane;   // row inside the 128-row tile == TMEM lane
+    int j = 0;
+    for (int item = blockIdx.x; item < n_items; item += gridDim.x, ++j) {
+      const int b = j & 1;
+      const uint32_t par = (uint32_t)(j >> 1) & 1u;
+      const bool ok = mbar_wait(&bars.acc_full[b], par, W.err, 13);
+      if (__any_sync(0xffffffffu, !ok)) { atomicExch(&bars.abort_flag, 1); break; }
+      tc_fence_after();
+      const int tile = item / n_ntiles, nt = item % n_ntiles;
+      const int e = W.tiles[2 * tile], m0 = W.tiles[2 * tile + 1];
+      const int cnt = W.counts[e];
+      const bool valid = (m0 + r) < cnt;
+      const uint32_t taddr = tmem + ((uint32_t)(warp * 32) << 16) + (uint32_t)(b * BN);
+      if (GATEUP) {
+        __nv_bfloat16 *dst = W.hb + (size_t)(tile * BM + r) * f + (size_t)nt * (BN / 2);
+#pragma unroll
+        for (int c = 0; c < BN / 2; c += 16) {
+          uint32_t g[16], u[16];
+          tmem_ld16(taddr + (uint32_t)c, g);
+          tmem_ld16(taddr + (uint32_t)(BN / 2 + c), u);
+          tmem_ld_wait();
+          uint32_t o[8];
+#pragma unroll
+          for (int i = 0; i < 8; ++i) {
+            const float h0 = gelu_tanh_f(__uint_as_float(g[2 * i])) * __uint_as_float(u[2 * i]);
+            const float h1 = gelu_tanh_f(__uint_as_float(g[2 * i + 1])) * __uint_as_float(u[2 * i + 1]);
+            o[i] = pack_bf16(h0, h1);
+          }
+          if (valid) {
+            uint4 *dp = reinterpret_cast<uint4 *>(dst + c);
+            dp[0] = make_uint4(o[0], o[1], o[2], o[3]);
+            dp[1] = make_uint4(o[4], o[5], o[6], o[7]);
+          }
+        }
+      } else {
+        int slot = 0;
+        float scale = 0.f;
+        if (valid) {
+          slot = W.perm[W.offsets[e] + m0 + r];
+          scale = W.w[slot] * expert_scale[e];
+        }
+        __nv_bfloat16 *dst = reinterpret_cast<__nv_bfloat16 *>(W.yslot) + (size_t)slot * d + (size_t)nt * BN;
+#pragma unroll
+        for (int c = 0; c < BN; c += 16) {
+          uint32_t y[16];
+          tmem_ld16(taddr + (uint32_t)c, y);
+          tmem_ld_wait();
+          uint32_t o[8];
+#pragma unroll
+          for (int i = 0; i < 8; ++i)
+            o[i] = pack_bf16(__uint_as_float(y[2 * i]) * scale, __uint_as_float(y[2 * i + 1]) * scale);
+          if (valid) {
+            uint4 *dp = reinterpret_cast<uint4 *>(dst + c);
+            dp[0] = make_uint4(o[0], o[1], o[2], o[3]);
+            dp[1] = make_uint4(o[4], o[5], o[6], o[7]);
+          }
+        }
+      }
+      tc_fence_before();
+      mbar_arrive(&bars.acc_empty[b]);
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == kMmaWarp) {
+    tc_fence_after();
+    tmem_dealloc(tmem, kTmemCols);
+  }
+}
+
+// Gather the routed rows of x into the padded tile order: padded row 128 i + r of tile
+// i = (e, m0) holds x[token of slot perm[offsets[e] + m0 + r]] (zeros past the expert's rows).
+__global__ void __launch_bounds__(256) k_gather_x(const __nv_bfloat16 *__restrict__ x, int d, int k, MoeWork W,
+                                                  __nv_bfloat16 *__restrict__ xg) {
+  const int n_tiles = *W.n_tiles;
+  const int vpr = d / 8;   // 16-byte vectors per row
+  const long long total = (long long)n_tiles * BM * vpr;
+  for (long long i = blockIdx.x * (long long)blockDim.x + threadIdx.x; i < total;
+       i += (long long)gridDim.x * blockDim.x) {
+    const int prow = (int)(i / vpr), v = (int)(i % vpr);
+    const int tile = prow / BM, r = prow % BM;
+    const int e = W.tiles[2 * tile], m0 = W.tiles[2 * tile + 1];
+    uint4 val = make_uint4(0u, 0u, 0u, 0u);
+    if (m0 + r < W.counts[e]) {
+      const int slot = W.perm[W.offsets[e] + m0 + r];
+      val = __ldg(reinterpret_cast<const uint4 *>(x + (size_t)(slot / k) * d) + v);
+    }
+    reinterpret_cast<uint4 *>(xg + (size_t)prow * d)[v] = val;
+  }
+}
+
+// out[t, c] = sum_{j < k} yslot[t k + j, c] (already weighted), j ascending.
+__global__ void __launch_bounds__(256) k_combine(const __nv_bfloat16 *__restrict__ yslot, int T, int d, int k,
+                                                 float *__restrict__ out) {
+  const int vpr = d / 8;
+  const long long total = (long long)T * vpr;
+  for (long long i = blockIdx.x * (long long)blockDim.x + threadIdx.x; i < total;
+       i += (long long)gridDim.x * blockDim.x) {
+    const int t = (int)(i / vpr), v = (int)(i % vpr);
+    float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+    for (int j = 0; j < k; ++j) {
+      const uint4 q = __ldg(reinterpret_cast<const uint4 *>(yslot + (size_t)(t * k + j) * d) + v);
+      const uint32_t qq[4] = {q.x, q.y, q.z, q.w};
+#pragma unroll
+      for (int h = 0; h < 4; ++h) {
+        acc[2 * h] += __uint_as_float(qq[h] << 16);
+        acc[2 * h + 1] += __uint_as_float(qq[h] & 0xffff0000u);
+      }
+    }
+    float4 *op = reinterpret_cast<float4 *>(out + (size_t)t * d) + 2 * v;
+    op[0] = make_float4(acc[0], acc[1], acc[2], acc[3]);
+    op[1] = make_float4(acc[4], acc[5], acc[6], acc[7]);
+  }
+}
+
+}  // namespace
+
+static int launch_err() { return cudaGetLastError() == cudaSuccess ? 0 : -1; }
+
+// Tensor maps over the workspace's padded activation buffers, encoded once per (buffer,
+// shape) through the driver entry point.
+static PFN_cuTensorMapEncodeTiled_v12000 get_encode() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  if (!fn) {
+    cudaDriverEntryPointQueryResult q;
+    void *p = nullptr;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) != cudaSuccess ||
+        q != cudaDriverEntryPointSuccess)
+      return nullptr;
+    fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  }
+  return fn;
+}
+
+static bool make_tmap(CUtensorMap *m, const void *base, int cols, long long rows) {
+  auto enc = get_encode();
+  if (!enc) return false;
+  cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
+  cuuint64_t strides[1] = {(cuuint64_t)cols * 2};
+  cuuint32_t box[2] = {(cuuint32_t)BK, (cuuint32_t)BM};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(base), dims, strides, box, estr,
+                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
 
 int moe_launch_gemm_experts(const MoeLaunch &L, const MoeWork &W, const void *x, const uint8_t *gate_up_q4,
                             const uint8_t *down_q4, const float *expert_scale, int T, int d, int f, int E, int k,
                             float *out, int num_sms, int max_tiles) {
-  (void)L; (void)W; (void)x; (void)gate_up_q4; (void)down_q4; (void)expert_scale; (void)T; (void)d; (void)f;
-  (void)E; (void)k; (void)out; (void)num_sms; (void)max_tiles;
-  return -2;
+  (void)E;
+  if (d % BK || d % BN || f % BK || f % (BN / 2)) return -2;
+  const long long rows = (long long)max_tiles * BM;
+  CUtensorMap ta, th;
+  if (!make_tmap(&ta, W.xg, d, rows) || !make_tmap(&th, W.hb, f, rows)) return -1;
+  static bool attr = false;
+  if (!attr) {
+    if (cudaFuncSetAttribute(k_moe_gemm<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes) !=
+            cudaSuccess ||
+        cudaFuncSetAttribute(k_moe_gemm<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes) !=
+            cudaSuccess)
+      return -1;
+    attr = true;
+  }
+  moe_prof_mark(L.stream, MOE_K_GEMM_GATEUP, true);
+  k_gather_x<<<4 * num_sms, 256, 0, L.stream>>>(static_cast<const __nv_bfloat16 *>(x), d, k, W, W.xg);
+  if (launch_err()) return -1;
+  k_moe_gemm<true><<<num_sms, kThreads, kSmemBytes, L.stream>>>(ta, gate_up_q4, expert_scale, d, f, k, W);
+  if (launch_err()) return -1;
+  moe_prof_mark(L.stream, MOE_K_GEMM_GATEUP, false);
+  moe_prof_mark(L.stream, MOE_K_GEMM_DOWN, true);
+  k_moe_gemm<false><<<num_sms, kThreads, kSmemBytes, L.stream>>>(th, down_q4, expert_scale, d, f, k, W);
+  if (launch_err()) return -1;
+  moe_prof_mark(L.stream, MOE_K_GEMM_DOWN, false);
+  moe_prof_mark(L.stream, MOE_K_COMBINE, true);
+  k_combine<<<4 * num_sms, 256, 0, L.stream>>>(reinterpret_cast<const __nv_bfloat16 *>(W.yslot), T, d, k, out);
+  if (launch_err()) return -1;
+  moe_prof_mark(L.stream, MOE_K_COMBINE, false);
+  return 0;
 }

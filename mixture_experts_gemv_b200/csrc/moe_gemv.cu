@@ -416,11 +416,15 @@ k_down_gemv_combine(const uint8_t *__restrict__ down_q4, const float *__restrict
   }
 }
 
-__global__ void k_hidden_slots_from_bf16(const __nv_bfloat16 *hb, const int32_t *inv, int S, int f, float *h) {
+// h of the grouped-GEMM path (bf16, padded tile rows) -> fp32 slot order.
+__global__ void k_hidden_slots_from_bf16(const __nv_bfloat16 *hb, const int32_t *ids, const int32_t *inv,
+                                         const int32_t *offsets, const int32_t *toff, int S, int f, float *h) {
   const long long n = (long long)S * f;
   for (long long i = blockIdx.x * (long long)blockDim.x + threadIdx.x; i < n; i += (long long)gridDim.x * blockDim.x) {
     const int s = (int)(i / f), c = (int)(i % f);
-    h[i] = __bfloat162float(hb[(size_t)inv[s] * f + c]);
+    const int e = ids[s];
+    const long long prow = (long long)toff[e] * 128 + (inv[s] - offsets[e]);
+    h[i] = __bfloat162float(hb[prow * f + c]);
   }
 }
 
@@ -466,6 +470,6 @@ int moe_launch_hidden_to_slots(cudaStream_t s, const MoeWork &W, float *h, int T
     if (cudaMemcpyAsync(h, W.h, sizeof(float) * (size_t)S * f, cudaMemcpyDeviceToDevice, s) != cudaSuccess) return -1;
     return 0;
   }
-  k_hidden_slots_from_bf16<<<256, 256, 0, s>>>(W.hb, W.inv, S, f, h);
+  k_hidden_slots_from_bf16<<<256, 256, 0, s>>>(W.hb, W.ids, W.inv, W.offsets, W.toff, S, f, h);
   return launch_err();
 }

@@ -162,7 +162,7 @@ __device__ void block_exclusive_scan3(int32_t a, int32_t b, int32_t c, int32_t &
 
 __device__ void block_permutation(const int32_t *ids, int S, int E, int32_t *counts, int32_t *offsets,
                                   int32_t *perm, int32_t *inv, int32_t *act, int32_t *n_act,
-                                  int32_t *tiles, int32_t *n_tiles, int tile_m, PermSmem &sm) {
+                                  int32_t *tiles, int32_t *n_tiles, int32_t *toffs, int tile_m, PermSmem &sm) {
   const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
   for (int i = threadIdx.x; i < kRouteWarps * MOE_MAX_E; i += blockDim.x) (&sm.cnt[0][0])[i] = 0;
   __syncthreads();
@@ -200,6 +200,7 @@ __device__ void block_permutation(const int32_t *ids, int S, int E, int32_t *cou
       run += c;
     }
     if (tiles) {
+      toffs[e] = toff;
       for (int i = 0; i < nt; ++i) {
         tiles[2 * (toff + i)] = e;
         tiles[2 * (toff + i) + 1] = i * tile_m;
@@ -310,7 +311,7 @@ k_route_decode(const __nv_bfloat16 *__restrict__ x, const float *__restrict__ ro
   __threadfence_block();
   __syncthreads();
   block_permutation(W.ids, T * k, E, W.counts, W.offsets, W.perm, W.inv, W.act, W.n_act, nullptr,
-                    nullptr, 1, sm.perm);
+                    nullptr, nullptr, 1, sm.perm);
   if (threadIdx.x == 0) W.counters[0] = 0;
 }
 
@@ -394,7 +395,7 @@ __global__ void __launch_bounds__(kRouteThreads)
 k_permute(int T, int E, int k, int tile_m, bool want_tiles, MoeWork W) {
   __shared__ PermSmem sm;
   block_permutation(W.ids, T * k, E, W.counts, W.offsets, W.perm, W.inv, W.act, W.n_act,
-                    want_tiles ? W.tiles : nullptr, want_tiles ? W.n_tiles : nullptr, tile_m, sm);
+                    want_tiles ? W.tiles : nullptr, want_tiles ? W.n_tiles : nullptr, W.toff, tile_m, sm);
 }
 
 __global__ void __launch_bounds__(256)

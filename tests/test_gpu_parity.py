@@ -63,6 +63,45 @@ def test_small_shapes_gemv(E, k, T, d, f):
     _check_full(x, lw, k, moe.MOE_PATH_GEMV)
 
 
+SMALL_GEMM = [  # (E, k, T, d, f): d % 128 == 0, f % 64 == 0
+    (8, 2, 33, 256, 64), (4, 4, 130, 128, 128), (128, 8, 300, 512, 128), (16, 4, 257, 2816, 704),
+    (128, 2, 17, 256, 64), (3, 3, 40, 384, 192),
+]
+
+
+@pytest.mark.parametrize("E,k,T,d,f", SMALL_GEMM)
+def test_small_shapes_gemm(E, k, T, d, f):
+    lw = mi.make_layer(seed=E * 1000 + T + 7, layer=0, d=d, f=f, E=E)
+    x = mi.make_tokens(E + T + 7, T, d)
+    _check_full(x, lw, k, moe.MOE_PATH_GEMM)
+
+
+def test_gemm_hidden_matches_oracle():
+    E, d, f, k, T = 16, 256, 128, 3, 70
+    lw = mi.make_layer(seed=14, d=d, f=f, E=E)
+    x = mi.make_tokens(15, T, d)
+    run_layer(x, DevLayer(lw), k, moe.MOE_PATH_GEMM)
+    h = torch.empty((T * k, f), dtype=torch.float32, device="cuda:0")
+    moe.moe_debug_get_hidden(h)
+    torch.cuda.synchronize()
+    logits = oracle.router_logits(x, lw.router_w)
+    ids, w, flags = oracle.topk_softmax(logits, k, 1.0)
+    _, href = oracle.experts_combine(x, lw.gate_up, lw.down, lw.expert_scale, ids, w, d, f, want_h=True)
+    assert rel_err(h.cpu().numpy().reshape(T, k, f), href) <= TOL_GEMM
+
+
+def test_gemm_and_gemv_paths_agree():
+    E, d, f, k, T = 32, 512, 192, 4, 40
+    lw = mi.make_layer(seed=16, d=d, f=f, E=E)
+    x = mi.make_tokens(17, T, d)
+    dl = DevLayer(lw)
+    a = run_layer(x, dl, k, moe.MOE_PATH_GEMV)["out"]
+    b = run_layer(x, dl, k, moe.MOE_PATH_GEMM)
+    assert rel_err(b["out"], a.astype(np.float64)) <= TOL_GEMM
+    c = run_layer(x, dl, k, moe.MOE_PATH_GEMM)["out"]
+    assert np.array_equal(b["out"].view(np.uint32), c.view(np.uint32))
+
+
 def test_zero_tokens_is_a_noop():
     lw = mi.make_layer(seed=1, d=64, f=32, E=4)
     dl = DevLayer(lw)
