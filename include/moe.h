@@ -149,6 +149,36 @@ int moe_debug_check(void *stream);
 int moe_profile_begin(void);
 int moe_profile_end(float *ms_total, int *launches);
 
+/*
+ * moe_layer_forward_static: the decode (FP32-accumulate GEMV) path of moe_layer_forward, for
+ * callers that cannot let a library allocate device memory -- serving engines that reserve
+ * all device memory in their own pool, plugins inside a host that owns every allocation,
+ * loops that cannot afford an allocation's implicit synchronisation. It needs no moe_init
+ * and calls no cudaMalloc / cudaFree: its scratch is a fixed static device array of
+ * MOE_STATIC_SCRATCH_BYTES that every GPU loading this library holds until the process
+ * exits. The pages have no counterpart of this entry point; it exists for library users.
+ *   Arguments, layouts and results as moe_layer_forward (same kernels, same bits), on the
+ *   current device. Limits: T <= MOE_STATIC_MAX_TOKENS, T * k <= MOE_STATIC_MAX_SLOTS,
+ *   d <= MOE_STATIC_MAX_D, f <= MOE_STATIC_MAX_F, E <= MOE_STATIC_MAX_E; larger shapes
+ *   return MOE_ERR_BAD_ARG with the limits in moe_last_error().
+ *   The first call on each device (with that device current) looks up the array's device
+ *   address; make that first call before any stream capture.
+ *   All calls share the array and leave their contents in it; the counters that must start
+ *   at zero are cleared at the start of each call on `stream`. Calls whose work overlaps on
+ *   the GPU (other streams, other host threads) race on the array.
+ *   There is no device error word: a device-side wait that expires ends the kernels early.
+ */
+#define MOE_STATIC_SCRATCH_BYTES (4u << 20)
+#define MOE_STATIC_MAX_TOKENS 16
+#define MOE_STATIC_MAX_SLOTS 128
+#define MOE_STATIC_MAX_D 4096
+#define MOE_STATIC_MAX_F 1024
+#define MOE_STATIC_MAX_E 256
+int moe_layer_forward_static(const void *x, const float *router_w, const float *router_scale,
+                             const uint8_t *gate_up_q4, const uint8_t *down_q4,
+                             const float *expert_scale, int T, int d, int f, int E, int k,
+                             float *out, void *stream);
+
 /* moe_workspace_bytes: device bytes moe_init would allocate for the given limits. */
 size_t moe_workspace_bytes(int max_tokens, int max_d, int max_f, int max_E, int max_k);
 

@@ -29,6 +29,7 @@ EXPORTED = (
     "moe_init", "moe_layer_forward", "moe_rmsnorm_bf16", "moe_stack_forward", "moe_set_path",
     "moe_destroy", "moe_last_error", "moe_debug_get_routing", "moe_debug_get_hidden",
     "moe_debug_check", "moe_workspace_bytes", "moe_profile_begin", "moe_profile_end",
+    "moe_layer_forward_static",
 )
 PROF_GROUPS = ("route", "gateup_gemv", "down_gemv", "gateup_gemm", "down_gemm", "combine", "rmsnorm", "")
 
@@ -77,6 +78,8 @@ def lib():
         L.moe_profile_begin.restype = _i
         L.moe_profile_end.argtypes = [_p, _p]
         L.moe_profile_end.restype = _i
+        L.moe_layer_forward_static.argtypes = [_p, _p, _p, _p, _p, _p, _i, _i, _i, _i, _i, _p, _p]
+        L.moe_layer_forward_static.restype = _i
         L.moe_workspace_bytes.argtypes = [_i, _i, _i, _i, _i]
         L.moe_workspace_bytes.restype = ctypes.c_size_t
         _lib = L
@@ -175,3 +178,11 @@ def moe_profile_end() -> dict:
     n = (ctypes.c_int * 8)()
     _check(lib().moe_profile_end(ms, n))
     return {PROF_GROUPS[i]: (float(ms[i]), int(n[i])) for i in range(8) if n[i] > 0}
+
+
+def moe_layer_forward_static(x, router_w, router_scale, gate_up_q4, down_q4, expert_scale,
+                             T: int, d: int, f: int, E: int, k: int, out, stream=None) -> None:
+    """Decode path with a fixed static device scratch: no workspace, no allocation."""
+    _check(lib().moe_layer_forward_static(_ptr(x), _ptr(router_w), _ptr(router_scale),
+                                          _ptr(gate_up_q4), _ptr(down_q4), _ptr(expert_scale),
+                                          T, d, f, E, k, _ptr(out), _stream(stream)))

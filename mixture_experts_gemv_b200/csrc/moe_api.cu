@@ -182,6 +182,12 @@ int forward_impl(const void *x, const float *router_w, const float *router_scale
 
 }  // namespace
 
+// Lets other translation units of the library set the moe_last_error() text.
+int moe_report_error(int code, const char *msg) {
+  snprintf(g_err, sizeof g_err, "%s", msg);
+  return code;
+}
+
 void moe_prof_mark(cudaStream_t s, int id, bool begin) {
   if (!g_prof.active || id < 0 || id >= MOE_K_COUNT) return;
   cudaEvent_t e = prof_event();
