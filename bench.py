@@ -236,6 +236,7 @@ def main():
     def step(i, xin=None, o=None):
         xin = x if xin is None else xin
         o = out if o is None else o
+        stream = torch.cuda.current_stream(dev)   # the capture stream while recording a graph
         if stack:
             moe.moe_stack_forward(xin, [q["router_w"] for q in dl], [q["router_scale"] for q in dl],
                                   [q["gate_up"] for q in dl], [q["down"] for q in dl],
@@ -278,6 +279,23 @@ def main():
     props = torch.cuda.get_device_properties(dev)
     gpu_id = f"GPU-{props.uuid}" if getattr(props, "uuid", None) else str(local)
     sampler = ClockSampler(gpu_id)
+
+    # The K steps are captured once into a CUDA graph and replayed: the library only
+    # enqueues work, so a replay runs exactly the kernels of K eager steps without host
+    # launch gaps between them.
+    def capture(fn):
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            fn()
+        return g
+
+    def run_steps():
+        for i in range(args.steps):
+            step(i)
+
+    graph = capture(run_steps)
+    graph.replay()
+    torch.cuda.synchronize()
     sampler.start()
     time.sleep(0.3)
 
@@ -287,8 +305,7 @@ def main():
     ev0 = torch.cuda.Event(enable_timing=True)
     ev1 = torch.cuda.Event(enable_timing=True)
     ev0.record(stream)
-    for i in range(args.steps):
-        step(i)
+    graph.replay()
     ev1.record(stream)
     torch.cuda.synchronize()
     barrier()
@@ -301,38 +318,54 @@ def main():
         ms = float(t.item())
     ms_step = ms / args.steps
 
-    # ---- per-kernel timing over a second pass of K steps (CUDA events on the launch stream)
+    # ---- per-kernel timing: the same K steps with CUDA events recorded around every kernel
+    # group on the launch stream (captured as event nodes), replayed once
     barrier()
     moe.moe_profile_begin()
-    for i in range(args.steps):
-        step(i)
+    pgraph = capture(run_steps)
+    pgraph.replay()
+    torch.cuda.synchronize()
     prof = moe.moe_profile_end()
+    del pgraph
 
-    # ---- end to end through the C ABI with host buffers (pinned), copies inside the region
+    # ---- end to end through the C ABI with host buffers: every step copies x from pinned
+    # host memory and reads out back to pinned host memory
     xh = torch.from_numpy(np.ascontiguousarray(base.x).view(np.int16)).pin_memory()
     oh = torch.empty((T, d), dtype=torch.float32).pin_memory()
     xd = torch.empty_like(x)
-    for i in range(3):
-        xd.copy_(xh, non_blocking=True)
-        step(i, xd)
-        oh.copy_(out, non_blocking=True)
+
+    def e2e_steps():
+        for i in range(args.steps):
+            xd.copy_(xh, non_blocking=True)
+            step(i, xd)
+            oh.copy_(out, non_blocking=True)
+
+    e2e_steps()
+    torch.cuda.synchronize()
+    egraph = capture(e2e_steps)
+    egraph.replay()
     torch.cuda.synchronize()
     barrier()
     e0 = torch.cuda.Event(enable_timing=True)
     e1 = torch.cuda.Event(enable_timing=True)
     e0.record(stream)
-    for i in range(args.steps):
-        xd.copy_(xh, non_blocking=True)
-        step(i, xd)
-        oh.copy_(out, non_blocking=True)
+    egraph.replay()
     e1.record(stream)
     torch.cuda.synchronize()
     barrier()
     ms_e2e = e0.elapsed_time(e1)
+    # the same without a graph: one eager C-ABI call per step from Python
+    e0.record(stream)
+    e2e_steps()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    ms_e2e_eager = e0.elapsed_time(e1)
+    del egraph
     if ws > 1:
-        t = torch.tensor([ms_e2e], device=dev)
+        t = torch.tensor([ms_e2e, ms_e2e_eager], device=dev)
         dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms_e2e = float(t.item())
+        ms_e2e, ms_e2e_eager = float(t[0].item()), float(t[1].item())
 
     # ---- roofline of the dominant kernel
     pk = measured_peaks()
@@ -379,7 +412,8 @@ def main():
             "kernel_ms_per_step": {kk: v[0] / args.steps for kk, v in prof.items()},
             "gpu_launches": int(round(launches_per_step * args.steps)),
             "e2e": {"value": e2e_value, "unit": "tokens/s", "h2d_bytes_per_step": T * d * 2,
-                    "d2h_bytes_per_step": T * d * 4},
+                    "d2h_bytes_per_step": T * d * 4, "launch": "CUDA graph of K steps",
+                    "eager_value": ws * T * args.steps / (ms_e2e_eager / 1e3)},
             "clocks": clocks}
 
     if rank == 0 and ws == 1 and not args.no_cpu_baseline:

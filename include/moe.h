@@ -51,6 +51,8 @@ extern "C" {
 #define MOE_PATH_AUTO 0   /* GEMV when T <= the GEMV token limit, else grouped GEMM */
 #define MOE_PATH_GEMV 1   /* FP32-accumulate Q4_0 GEMV path (decode) */
 #define MOE_PATH_GEMM 2   /* bf16 tcgen05 grouped-GEMM path (prefill) */
+#define MOE_PATH_GEMV_SPLIT 3   /* GEMV path as separate routing / gate_up / down kernels
+                                   (MOE_PATH_GEMV uses one fused kernel when T <= 8) */
 
 /*
  * moe_init: select `device`, check it is sm_100, and allocate the workspace for
@@ -142,7 +144,7 @@ int moe_debug_check(void *stream);
  * milliseconds and the number of launches (arrays of MOE_PROF_GROUPS entries, may be NULL).
  * Groups: 0 routing (router, top-k, permutation), 1 decode gate_up GEMV + GeGLU, 2 decode
  * down GEMV + combine, 3 prefill gate_up grouped GEMM + GeGLU, 4 prefill down grouped GEMM,
- * 5 prefill combine, 6 RMSNorm. Recording events serialises nothing but does separate the
+ * 5 prefill combine, 6 RMSNorm, 7 fused decode kernel (routing to combine in one launch). Recording events serialises nothing but does separate the
  * launches, so a timed forward can run slightly slower than an untimed one.
  */
 #define MOE_PROF_GROUPS 8

@@ -23,6 +23,7 @@ MOE_ERR_UNSUPPORTED_DEVICE = -6
 MOE_PATH_AUTO = 0
 MOE_PATH_GEMV = 1
 MOE_PATH_GEMM = 2
+MOE_PATH_GEMV_SPLIT = 3
 
 # Every symbol include/moe.h declares.
 EXPORTED = (
@@ -31,7 +32,8 @@ EXPORTED = (
     "moe_debug_check", "moe_workspace_bytes", "moe_profile_begin", "moe_profile_end",
     "moe_layer_forward_static",
 )
-PROF_GROUPS = ("route", "gateup_gemv", "down_gemv", "gateup_gemm", "down_gemm", "combine", "rmsnorm", "")
+PROF_GROUPS = ("route", "gateup_gemv", "down_gemv", "gateup_gemm", "down_gemm", "combine", "rmsnorm",
+               "fused_decode")
 
 
 class MoeError(RuntimeError):

@@ -89,10 +89,10 @@ Layout make_layout(int maxT, int max_d, int max_f, int max_E, int max_k) {
       S * 4,                             // 6 inv
       (size_t)max_E * 4,                 // 7 act
       16,                                // 8 n_act, n_tiles
-      (size_t)maxT * max_d * 4,          // 9 xprep
-      (size_t)maxT * (max_d / 32) * 4,   // 10 xsum
+      (size_t)maxT * max_d * 2,          // 9 x16
+      (size_t)maxT * (max_d / 32) * 8,   // 10 xblk
       S * max_f * 4,                     // 11 h
-      S * max_f * 4,                     // 12 hprep
+      16,                                // 12 (unused)
       S * max_d * 4,                     // 13 ybuf / yslot
       (size_t)(2 + max_d / 8 + 1024) * 4,   // 14 counters
       prow * max_f * 2,                  // 15 hb (bf16, padded tiles)
@@ -102,6 +102,7 @@ Layout make_layout(int maxT, int max_d, int max_f, int max_E, int max_k) {
       (size_t)maxT * max_d * 4,          // 19 ylayer
       prow * max_d * 2,                  // 20 xg (bf16, padded tiles)
       (size_t)max_E * 4,                 // 21 toff
+      64,                                // 22 grid-barrier counter
   };
   Layout L{};
   size_t o = 0;
@@ -153,6 +154,8 @@ int forward_impl(const void *x, const float *router_w, const float *router_scale
                  cudaStream_t stream) {
   MoeLaunch L{stream, false};
   const bool gemm = (g.path == MOE_PATH_GEMM) || (g.path == MOE_PATH_AUTO && T > g.gemv_max_tokens);
+  // MOE_PATH_GEMV and AUTO below the threshold take the fused decode kernel when the shape
+  // fits it (T <= 8), else the separate routing / gate_up / down kernels (MOE_PATH_GEMV_SPLIT).
   int rc;
   if (gemm) {
     rc = moe_launch_route_prefill(L, g.W, x, router_w, router_scale, T, d, E, k, g.num_sms, false, kTileM);
@@ -162,6 +165,10 @@ int forward_impl(const void *x, const float *router_w, const float *router_scale
                                  max_tiles);
     if (rc == -2) return fail(MOE_ERR_BAD_ARG, "shape not supported by the grouped-GEMM path");
     if (rc) return cuda_fail(cudaGetLastError(), "grouped-GEMM launch");
+  } else if (g.path != MOE_PATH_GEMV_SPLIT && moe_fused_decode_supported(T, d, f, E, k)) {
+    rc = moe_launch_fused_decode(L, g.W, x, router_w, router_scale, gate_up_q4, down_q4, expert_scale, T, d, f, E,
+                                 k, out, g.num_sms);
+    if (rc) return cuda_fail(cudaGetLastError(), "fused decode launch");
   } else {
     if (T <= 16)
       rc = moe_launch_route_decode(L, g.W, x, router_w, router_scale, T, d, E, k, g.num_sms);
@@ -192,7 +199,13 @@ void moe_prof_mark(cudaStream_t s, int id, bool begin) {
   if (!g_prof.active || id < 0 || id >= MOE_K_COUNT) return;
   cudaEvent_t e = prof_event();
   if (!e) return;
-  cudaEventRecord(e, s);
+  // inside a stream capture the record must become an event-record node of the graph
+  cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
+  cudaStreamIsCapturing(s, &cs);
+  if (cs == cudaStreamCaptureStatusActive)
+    cudaEventRecordWithFlags(e, s, cudaEventRecordExternal);
+  else
+    cudaEventRecord(e, s);
   if (begin) {
     g_prof.open_ev[id] = e;
   } else if (g_prof.open_ev[id]) {
@@ -285,10 +298,9 @@ int moe_init(int device, int max_tokens, int max_d, int max_f, int max_E, int ma
   W.act = reinterpret_cast<int32_t *>(b + Lt.off[7]);
   W.n_act = reinterpret_cast<int32_t *>(b + Lt.off[8]);
   W.n_tiles = reinterpret_cast<int32_t *>(b + Lt.off[8] + 4);
-  W.xprep = reinterpret_cast<float *>(b + Lt.off[9]);
-  W.xsum = reinterpret_cast<float *>(b + Lt.off[10]);
+  W.x16 = reinterpret_cast<__half *>(b + Lt.off[9]);
+  W.xblk = reinterpret_cast<float2 *>(b + Lt.off[10]);
   W.h = reinterpret_cast<float *>(b + Lt.off[11]);
-  W.hprep = reinterpret_cast<float *>(b + Lt.off[12]);
   W.ybuf = reinterpret_cast<float *>(b + Lt.off[13]);
   W.yslot = W.ybuf;
   W.counters = reinterpret_cast<uint32_t *>(b + Lt.off[14]);
@@ -296,6 +308,7 @@ int moe_init(int device, int max_tokens, int max_d, int max_f, int max_E, int ma
   W.tiles = reinterpret_cast<int32_t *>(b + Lt.off[16]);
   W.xg = reinterpret_cast<__nv_bfloat16 *>(b + Lt.off[20]);
   W.toff = reinterpret_cast<int32_t *>(b + Lt.off[21]);
+  W.gbar = reinterpret_cast<unsigned long long *>(b + Lt.off[22]);
   W.err = ed;
 
   g.init = true;
@@ -387,7 +400,7 @@ int moe_stack_forward(const void *x_in, int L, const float *const *router_w, con
 }
 
 int moe_set_path(int path, int gemv_max_tokens) {
-  if (path != MOE_PATH_AUTO && path != MOE_PATH_GEMV && path != MOE_PATH_GEMM)
+  if (path != MOE_PATH_AUTO && path != MOE_PATH_GEMV && path != MOE_PATH_GEMM && path != MOE_PATH_GEMV_SPLIT)
     return fail(MOE_ERR_BAD_ARG, "unknown path %d", path);
   if (gemv_max_tokens < 0) return fail(MOE_ERR_BAD_ARG, "gemv_max_tokens = %d < 0", gemv_max_tokens);
   g.path = path;

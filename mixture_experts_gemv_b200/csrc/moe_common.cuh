@@ -27,10 +27,9 @@ struct MoeWork {
   int32_t *inv;       // [T*k]  slot -> sorted position
   int32_t *act;       // [E]    active experts, ascending; act[E-1..] unused
   int32_t *n_act;     // [1]
-  float *xprep;       // [T, d] x reordered/scaled for the Q4_0 GEMV (see moe_gemv.cu)
-  float *xsum;        // [T, d/32] per-block sums of x
+  __half *x16;        // [T, d] x as scaled f16 in the GEMV's word order (see moe_gemv.cu)
+  float2 *xblk;       // [T, d/32] per block: (-8 * sum of the scaled values, 2^sigma)
   float *h;           // [T*k, f] fp32 hidden (GEMV path), slot order
-  float *hprep;       // [T*k, f] h reordered/scaled for the down GEMV
   float *ybuf;        // [T*k, d] per-slot expert outputs (GEMV path)
   uint32_t *counters; // [n] zero-initialised arrival counters (reset by their users)
   volatile uint32_t *err;   // mapped host word: device error code
@@ -40,6 +39,7 @@ struct MoeWork {
   float *yslot;       // [T*k, d] per-slot weighted down outputs (bf16 in the GEMM path)
   int32_t *tiles;     // [max tiles] (expert, m0) work list
   int32_t *toff;      // [E] index of each expert's first tile
+  unsigned long long *gbar;   // grid-barrier counter of the fused decode kernel (monotonic)
   int32_t *n_tiles;   // [1]
 };
 
@@ -62,6 +62,28 @@ __device__ __forceinline__ void report_error(volatile uint32_t *err, uint32_t co
     __threadfence_system();
   }
 }
+
+// ---------------------------------------------------------------- f16 activations
+//
+// The GEMV path multiplies Q4_0 codes by f16 activations. Each 32-wide block of an
+// activation vector is scaled by a power of two 2^-sigma that puts its largest magnitude in
+// [2^14, 2^15), so converting a bf16 activation to f16 is exact (and an fp32 one keeps 11
+// significant bits); the block's results are multiplied back by 2^sigma.
+struct BlockScale {
+  float scale;   // 2^-sigma
+  float inv;     // 2^sigma
+};
+__device__ __forceinline__ BlockScale block_scale_for_max(float m) {
+  int eb = (int)((__float_as_uint(m) >> 23) & 0xffu);   // biased exponent of max |v|
+  eb = eb < 15 ? 15 : eb;                                  // tiny / zero blocks: scale 2^126
+  BlockScale r;
+  r.scale = __uint_as_float((uint32_t)(268 - eb) << 23);   // 2^(141 - e): max in [2^14, 2^15)
+  r.inv = __uint_as_float((uint32_t)(eb - 14) << 23);
+  return r;
+}
+// Position of element e (0..31) of a block in the GEMV's word order: code word i (bytes
+// 4i..4i+3) pairs with activations 4i..4i+3 (low nibbles) then 16+4i..16+4i+3 (high).
+__device__ __forceinline__ int gemv_pos(int e) { return (e < 16) ? ((e >> 2) * 8 + (e & 3)) : (((e - 16) >> 2) * 8 + 4 + (e & 3)); }
 
 // ---------------------------------------------------------------- mbarrier
 
@@ -148,6 +170,7 @@ enum MoeKernelId {
   MOE_K_GEMM_DOWN = 4,    // prefill down grouped GEMM
   MOE_K_COMBINE = 5,      // prefill ordered combine
   MOE_K_NORM = 6,         // inter-layer RMSNorm
+  MOE_K_FUSED = 7,        // fused decode kernel (router .. combine in one launch)
   MOE_K_COUNT = 8
 };
 // Record a CUDA event on `s` before (begin) / after a launch of kernel group `id`; a no-op
@@ -166,6 +189,11 @@ int moe_launch_gemv_experts(const MoeLaunch &L, const MoeWork &W, const uint8_t 
 int moe_launch_gemm_experts(const MoeLaunch &L, const MoeWork &W, const void *x, const uint8_t *gate_up_q4,
                             const uint8_t *down_q4, const float *expert_scale, int T, int d, int f,
                             int E, int k, float *out, int num_sms, int max_tiles);
+bool moe_fused_decode_supported(int T, int d, int f, int E, int k);
+int moe_launch_fused_decode(const MoeLaunch &L, const MoeWork &W, const void *x, const float *router_w,
+                            const float *router_scale, const uint8_t *gate_up_q4, const uint8_t *down_q4,
+                            const float *expert_scale, int T, int d, int f, int E, int k, float *out,
+                            int num_sms);
 int moe_launch_rmsnorm(cudaStream_t s, const float *y, void *x_out, int T, int d, float eps);
 int moe_launch_hidden_to_slots(cudaStream_t s, const MoeWork &W, float *h, int T, int f, int k,
                                bool gemm_path);

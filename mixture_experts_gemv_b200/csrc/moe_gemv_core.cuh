@@ -1,0 +1,303 @@
+// moe_gemv_core.cuh -- device building blocks of the Q4_0 decode GEMVs, shared by the
+// separate-kernel path (moe_gemv.cu) and the fused decode kernel (moe_decode.cu).
+//
+// Arithmetic: a Q4_0 weight is (q - 8) * d. The codes of one 4-byte code word are spread
+// into one byte each (low nibbles, then high nibbles); a byte holding q in 0..15 read as an
+// FP8 e4m3 value is exactly q * 2^-9 (subnormal for q < 8, normal above), so the hardware
+// e4m3 -> f16x2 conversion decodes two codes per instruction, exactly. Activations are f16
+// scaled per 32-wide block by a power of two (exact for bf16 x). Products q * 2^-9 * a are
+// formed exactly by the mixed-precision FMA (f16 x f16 + f32) and summed in FP32; per block
+// and token the row accumulator gets d * 2^sigma * (512 * sum - 8 * sum(a)).
+#pragma once
+
+#include "moe_common.cuh"
+
+namespace {
+
+
+constexpr int kGran = 8;        // blocks per granule: 144 bytes, 16-byte aligned in aligned rows
+constexpr int kMaxGran = 16;    // gate_up: one warp per granule, d <= 4096
+constexpr int kPairs = 16;      // row pairs (gate c, up f + c) per gate_up chunk
+constexpr int kUnit = 8;        // rows (or row pairs) per scheduling unit
+constexpr int kTX = 4;          // tokens per pass over a staged chunk
+constexpr int kGuStagesMax = 3;
+constexpr int kDnRows = 128;    // rows per down chunk
+constexpr int kDnThreads = 256; // 4 warps x 32 rows, 2 parts of the row's blocks
+constexpr int kDnStagesMax = 4;
+constexpr uint32_t kMagic = 0x4B000000u;   // 2^23
+constexpr int kSmemBudget = 222 * 1024;
+
+__device__ __forceinline__ float gelu_tanh_f(float z) {
+  const float c = 0.7978845608028654f;   // sqrt(2/pi)
+  return 0.5f * z * (1.0f + tanhf(c * (z + 0.044715f * z * z * z)));
+}
+
+// Two e4m3 bytes (the low or high 16 bits of v) -> f16x2.
+__device__ __forceinline__ uint32_t e4m3x2_lo(uint32_t v) {
+  uint32_t r;
+  asm("{.reg .b16 l, h;\n\tmov.b32 {l, h}, %1;\n\tcvt.rn.f16x2.e4m3x2 %0, l;}" : "=r"(r) : "r"(v));
+  return r;
+}
+__device__ __forceinline__ uint32_t e4m3x2_hi(uint32_t v) {
+  uint32_t r;
+  asm("{.reg .b16 l, h;\n\tmov.b32 {l, h}, %1;\n\tcvt.rn.f16x2.e4m3x2 %0, h;}" : "=r"(r) : "r"(v));
+  return r;
+}
+// c + a.lo * b.lo and c + a.hi * b.hi with f16 inputs, exact product, FP32 sum.
+__device__ __forceinline__ float fma_h_lo(uint32_t a, uint32_t b, float c) {
+  float r;
+  asm("{.reg .b16 al, ah, bl, bh;\n\tmov.b32 {al, ah}, %1;\n\tmov.b32 {bl, bh}, %2;\n\tfma.rn.f32.f16 %0, al, bl, %3;}"
+      : "=f"(r) : "r"(a), "r"(b), "f"(c));
+  return r;
+}
+__device__ __forceinline__ float fma_h_hi(uint32_t a, uint32_t b, float c) {
+  float r;
+  asm("{.reg .b16 al, ah, bl, bh;\n\tmov.b32 {al, ah}, %1;\n\tmov.b32 {bl, bh}, %2;\n\tfma.rn.f32.f16 %0, ah, bh, %3;}"
+      : "=f"(r) : "r"(a), "r"(b), "f"(c));
+  return r;
+}
+
+// The eight codes of one code word as f16 q * 2^-9, in the activation word order:
+// c0 = (e0, e1), c1 = (e2, e3) of the low nibbles, c2, c3 the same of the high nibbles.
+struct Codes8 {
+  uint32_t c[4];
+};
+__device__ __forceinline__ Codes8 decode8(uint32_t w) {
+  const uint32_t lo = w & 0x0F0F0F0Fu, hi = (w >> 4) & 0x0F0F0F0Fu;
+  Codes8 r;
+  r.c[0] = e4m3x2_lo(lo);
+  r.c[1] = e4m3x2_hi(lo);
+  r.c[2] = e4m3x2_lo(hi);
+  r.c[3] = e4m3x2_hi(hi);
+  return r;
+}
+// (a0, a1) += codes . activations (8 f16 in a uint4)
+__device__ __forceinline__ void dot8h(const Codes8 &k, const uint4 &xv, float &a0, float &a1) {
+  a0 = fma_h_lo(k.c[0], xv.x, a0);
+  a1 = fma_h_hi(k.c[0], xv.x, a1);
+  a0 = fma_h_lo(k.c[1], xv.y, a0);
+  a1 = fma_h_hi(k.c[1], xv.y, a1);
+  a0 = fma_h_lo(k.c[2], xv.z, a0);
+  a1 = fma_h_hi(k.c[2], xv.z, a1);
+  a0 = fma_h_lo(k.c[3], xv.w, a0);
+  a1 = fma_h_hi(k.c[3], xv.w, a1);
+}
+
+struct Blk {
+  float d;
+  uint32_t q[4];
+};
+
+// One 18-byte block at a 2-byte aligned shared-memory byte offset (five 32-bit loads).
+__device__ __forceinline__ Blk load_blk(const uint8_t *smem, uint32_t o) {
+  const uint32_t a = o & ~3u;
+  const uint32_t sh = (o & 3u) * 8u;   // 0 or 16
+  const uint32_t *wp = reinterpret_cast<const uint32_t *>(smem + a);
+  const uint32_t w0 = wp[0], w1 = wp[1], w2 = wp[2], w3 = wp[3], w4 = wp[4];
+  Blk b;
+  b.d = __half2float(__ushort_as_half((unsigned short)((w0 >> sh) & 0xffffu)));
+  const uint32_t s2 = sh + 16u;
+  b.q[0] = __funnelshift_rc(w0, w1, s2);
+  b.q[1] = __funnelshift_rc(w1, w2, s2);
+  b.q[2] = __funnelshift_rc(w2, w3, s2);
+  b.q[3] = __funnelshift_rc(w3, w4, s2);
+  return b;
+}
+
+// Two consecutive blocks from nine words w[0..8]: the first starts on word 0 (scale in its
+// low half, codes shifted by 16 bits), the second at byte 18 (scale in the high half of
+// word 4, codes in words 5..8).
+__device__ __forceinline__ void split_blk2(const uint32_t (&w)[10], Blk &b0, Blk &b1) {
+  b0.d = __half2float(__ushort_as_half((unsigned short)(w[0] & 0xffffu)));
+#pragma unroll
+  for (int i = 0; i < 4; ++i) b0.q[i] = __funnelshift_r(w[i], w[i + 1], 16);
+  b1.d = __half2float(__ushort_as_half((unsigned short)(w[4] >> 16)));
+#pragma unroll
+  for (int i = 0; i < 4; ++i) b1.q[i] = w[5 + i];
+}
+
+// Blocks 0, 1 of a 72-byte, 8-byte aligned four-block span: five 64-bit loads at o.
+__device__ __forceinline__ void load_blk2_lo(const uint8_t *smem, uint32_t o, Blk &b0, Blk &b1) {
+  const uint2 *wp = reinterpret_cast<const uint2 *>(smem + o);
+  uint32_t w[10];
+#pragma unroll
+  for (int i = 0; i < 5; ++i) {
+    const uint2 v = wp[i];
+    w[2 * i] = v.x;
+    w[2 * i + 1] = v.y;
+  }
+  split_blk2(w, b0, b1);
+}
+
+// Blocks 2, 3 of the same span: they start at byte 36 (4-byte aligned): one 32-bit load at
+// o + 36 and four 64-bit loads from the 8-byte aligned o + 40.
+__device__ __forceinline__ void load_blk2_hi(const uint8_t *smem, uint32_t o, Blk &b0, Blk &b1) {
+  uint32_t w[10];
+  w[0] = *reinterpret_cast<const uint32_t *>(smem + o + 36);
+  const uint2 *wp = reinterpret_cast<const uint2 *>(smem + o + 40);
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const uint2 v = wp[i];
+    w[1 + 2 * i] = v.x;
+    w[2 + 2 * i] = v.y;
+  }
+  w[9] = 0u;
+  split_blk2(w, b0, b1);
+}
+
+struct RingCtl {
+  uint64_t full[kDnStagesMax];
+};
+
+// Flat split of n units over the grid.
+__device__ __forceinline__ void my_units(int n, int &u0, int &u1) {
+  u0 = (int)((long long)n * blockIdx.x / gridDim.x);
+  u1 = (int)((long long)n * (blockIdx.x + 1) / gridDim.x);
+}
+
+__device__ __forceinline__ uint8_t *align128(uint8_t *p) {
+  return p + ((128u - (smem_u32(p) & 127u)) & 127u);
+}
+
+// ---------------------------------------------------------------- gate_up + GeGLU
+//
+// CTA = one warp per 144-byte granule of a row (11 warps for d = 2816). Lane = (row pair p,
+// half h): rows c0 + p (gate) and f + c0 + p (up), blocks 8 w + 4 h .. + 3. All lanes of a
+// warp read the same activations (shared-memory broadcast); the 2 G partials of each row
+// are summed in a fixed order at the end of the chunk, where the GeGLU is applied.
+
+struct GuChunk {
+  int a, c0, np;   // active-expert index, first row pair, row pairs (8 or 16)
+};
+
+__device__ __forceinline__ GuChunk gu_chunk(int u, int u1, int upe) {
+  GuChunk c;
+  c.a = u / upe;
+  c.c0 = (u % upe) * kUnit;
+  const int n = (u + 1 < u1 && (u + 1) / upe == c.a) ? 2 : 1;
+  c.np = n * kUnit;
+  return c;
+}
+
+template <int NT>
+__device__ __forceinline__ void gu_block(const Blk &bg, const Blk &bu, int b, int nb, const uint16_t *xs,
+                                         const float2 *ss, int d, float (&yg)[NT], float (&yu)[NT]) {
+  float ag0[NT], ag1[NT], au0[NT], au1[NT];
+#pragma unroll
+  for (int i = 0; i < NT; ++i) { ag0[i] = 0.f; ag1[i] = 0.f; au0[i] = 0.f; au1[i] = 0.f; }
+#pragma unroll
+  for (int wi = 0; wi < 4; ++wi) {
+    const Codes8 kg = decode8(bg.q[wi]);
+    const Codes8 ku = decode8(bu.q[wi]);
+#pragma unroll
+    for (int i = 0; i < NT; ++i) {
+      const uint4 xv = *reinterpret_cast<const uint4 *>(xs + (size_t)i * d + b * MOE_QK + 8 * wi);
+      dot8h(kg, xv, ag0[i], ag1[i]);
+      dot8h(ku, xv, au0[i], au1[i]);
+    }
+  }
+#pragma unroll
+  for (int i = 0; i < NT; ++i) {
+    const float2 sb = ss[i * nb + b];   // (-8 * sum a, 2^sigma)
+    yg[i] = fmaf(bg.d * sb.y, fmaf(512.f, ag0[i] + ag1[i], sb.x), yg[i]);
+    yu[i] = fmaf(bu.d * sb.y, fmaf(512.f, au0[i] + au1[i], sb.x), yu[i]);
+  }
+}
+
+template <int NT, bool ALIGNED>
+__device__ __forceinline__ void gu_compute(const uint8_t *st, uint32_t rb, int nb, const uint16_t *xs,
+                                           const float2 *ss, int d, float *red_out /* [NT][2] */) {
+  // called by every lane of the warp (rows past the chunk read stale shared memory and are
+  // not stored by the caller)
+  const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
+  const int p = lane >> 1, h = lane & 1;
+  float yg[NT], yu[NT];
+#pragma unroll
+  for (int i = 0; i < NT; ++i) { yg[i] = 0.f; yu[i] = 0.f; }
+  const int b0 = w * kGran + h * 4;
+  const uint32_t og = (uint32_t)p * rb + (uint32_t)b0 * MOE_QBYTES;
+  const uint32_t ou = (uint32_t)(kPairs + p) * rb + (uint32_t)b0 * MOE_QBYTES;
+  int nbl = nb - b0;
+  nbl = nbl < 0 ? 0 : (nbl > 4 ? 4 : nbl);
+  if (ALIGNED) {
+    {
+      Blk g0, g1, v0, v1;
+      load_blk2_lo(st, og, g0, g1);
+      load_blk2_lo(st, ou, v0, v1);
+      gu_block<NT>(g0, v0, b0, nb, xs, ss, d, yg, yu);
+      gu_block<NT>(g1, v1, b0 + 1, nb, xs, ss, d, yg, yu);
+    }
+    {
+      Blk g2, g3, v2, v3;
+      load_blk2_hi(st, og, g2, g3);
+      load_blk2_hi(st, ou, v2, v3);
+      gu_block<NT>(g2, v2, b0 + 2, nb, xs, ss, d, yg, yu);
+      gu_block<NT>(g3, v3, b0 + 3, nb, xs, ss, d, yg, yu);
+    }
+  } else {
+    for (int j = 0; j < nbl; ++j) {
+      const Blk g = load_blk(st, og + j * MOE_QBYTES);
+      const Blk v = load_blk(st, ou + j * MOE_QBYTES);
+      gu_block<NT>(g, v, b0 + j, nb, xs, ss, d, yg, yu);
+    }
+  }
+  // the two halves of a granule sit in adjacent lanes: combine them, even lanes store
+#pragma unroll
+  for (int i = 0; i < NT; ++i) {
+    const float g = yg[i] + __shfl_xor_sync(0xffffffffu, yg[i], 1);
+    const float u = yu[i] + __shfl_xor_sync(0xffffffffu, yu[i], 1);
+    if (h == 0) {
+      red_out[2 * i] = g;
+      red_out[2 * i + 1] = u;
+    }
+  }
+}
+
+struct DnChunk {
+  int a, r0, nr;
+};
+
+__device__ __forceinline__ DnChunk dn_chunk(int u, int u1, int upe) {
+  DnChunk c;
+  c.a = u / upe;
+  c.r0 = (u % upe) * kUnit;
+  int n = 1;
+  while (n < kDnRows / kUnit && u + n < u1 && (u + n) / upe == c.a) ++n;
+  c.nr = n * kUnit;
+  return c;
+}
+
+template <int NT>
+__device__ __forceinline__ void dn_compute(const uint8_t *st, uint32_t rb, int nbf, const uint16_t *hs,
+                                           const float2 *hb, int f, float *red_out /* [NT] */) {
+  const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
+  const int row = (w & 3) * 32 + lane, part = w >> 2;
+  const int bpp = (nbf + 1) / 2;
+  const int b0 = part * bpp, b1 = min(nbf, b0 + bpp);
+  float y[NT];
+#pragma unroll
+  for (int i = 0; i < NT; ++i) y[i] = 0.f;
+  const uint32_t orow = (uint32_t)row * rb;
+  for (int b = b0; b < b1; ++b) {
+    const Blk bk = load_blk(st, orow + (uint32_t)b * MOE_QBYTES);
+    float a0[NT], a1[NT];
+#pragma unroll
+    for (int i = 0; i < NT; ++i) { a0[i] = 0.f; a1[i] = 0.f; }
+#pragma unroll
+    for (int wi = 0; wi < 4; ++wi) {
+      const Codes8 kc = decode8(bk.q[wi]);
+#pragma unroll
+      for (int i = 0; i < NT; ++i)
+        dot8h(kc, *reinterpret_cast<const uint4 *>(hs + (size_t)i * f + b * MOE_QK + 8 * wi), a0[i], a1[i]);
+    }
+#pragma unroll
+    for (int i = 0; i < NT; ++i) {
+      const float2 sb = hb[i * nbf + b];
+      y[i] = fmaf(bk.d * sb.y, fmaf(512.f, a0[i] + a1[i], sb.x), y[i]);
+    }
+  }
+#pragma unroll
+  for (int i = 0; i < NT; ++i) red_out[i * kDnRows] = y[i];
+}
+
+}  // namespace

@@ -43,10 +43,9 @@ constexpr size_t kOffInv = align_up(kOffPerm + kS * 4);
 constexpr size_t kOffAct = align_up(kOffInv + kS * 4);
 constexpr size_t kOffNAct = align_up(kOffAct + kE * 4);
 constexpr size_t kOffXprep = align_up(kOffNAct + 16);
-constexpr size_t kOffXsum = align_up(kOffXprep + kT * kD * 4);
-constexpr size_t kOffH = align_up(kOffXsum + kT * (kD / 32) * 4);
-constexpr size_t kOffHprep = align_up(kOffH + kS * kF * 4);
-constexpr size_t kOffYbuf = align_up(kOffHprep + kS * kF * 4);
+constexpr size_t kOffXblk = align_up(kOffXprep + kT * kD * 2);
+constexpr size_t kOffH = align_up(kOffXblk + kT * (kD / 32) * 8);
+constexpr size_t kOffYbuf = align_up(kOffH + kS * kF * 4);
 constexpr size_t kCounterWords = 2 + kD / 8;
 constexpr size_t kOffCounters = align_up(kOffYbuf + kS * kD * 4);
 constexpr size_t kEnd = align_up(kOffCounters + kCounterWords * 4);
@@ -131,10 +130,9 @@ extern "C" int moe_layer_forward_static(const void *x, const float *router_w, co
   W.act = reinterpret_cast<int32_t *>(b + kOffAct);
   W.n_act = reinterpret_cast<int32_t *>(b + kOffNAct);
   W.n_tiles = reinterpret_cast<int32_t *>(b + kOffNAct + 4);
-  W.xprep = reinterpret_cast<float *>(b + kOffXprep);
-  W.xsum = reinterpret_cast<float *>(b + kOffXsum);
+  W.x16 = reinterpret_cast<__half *>(b + kOffXprep);
+  W.xblk = reinterpret_cast<float2 *>(b + kOffXblk);
   W.h = reinterpret_cast<float *>(b + kOffH);
-  W.hprep = reinterpret_cast<float *>(b + kOffHprep);
   W.ybuf = reinterpret_cast<float *>(b + kOffYbuf);
   W.yslot = W.ybuf;
   W.counters = reinterpret_cast<uint32_t *>(b + kOffCounters);

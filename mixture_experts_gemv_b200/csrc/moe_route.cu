@@ -6,118 +6,15 @@
 // the k largest logits are selected, equal logits going to the lower expert index;
 // w[t,j] = router_scale * exp(l_j - l_1) / sum_m exp(l_m - l_1) over the selected ones.
 // The permutation is the stable counting sort of slots s = t*k + j by expert id.
-#include "moe_common.cuh"
+#include "moe_route_core.cuh"
 
 namespace {
 
 constexpr int kRouteThreads = 512;             // 16 warps
 constexpr int kRouteWarps = kRouteThreads / 32;
-constexpr int kRouteParts = 4;                 // d split in 4 parts per expert (decode)
+constexpr int kRouteParts = 8;                 // d split in 8 parts per expert (decode)
+constexpr int kRouteEPC = kRouteWarps / kRouteParts;   // experts per CTA
 constexpr int kDecodeMaxT = 16;
-
-// ---------------------------------------------------------------- x preparation
-//
-// The Q4_0 GEMV turns a 4-bit code q sitting at bit 4j of a 32-bit code word into the
-// exact float q * 2^(s_j) by OR-ing it into the mantissa of 2^23 and subtracting 2^23
-// (s_j = 4j for j <= 4; codes 5..7 are first shifted right by 12, s_j = 4(j-3)). The
-// matching activation is pre-multiplied by 2^(-s_j), which is exact, so the product is
-// q * x. Inside a block, code word i (bytes 4i..4i+3 of the codes) holds at nibble
-// position j = 2m the low nibble of byte 4i+m (element 4i+m) and at j = 2m+1 the high
-// nibble (element 16+4i+m). xprep stores, for each block, the 32 activations in that
-// (word, nibble) order, scaled; xsum stores the plain block sums (for the -8 offset).
-__device__ __forceinline__ float nib_scale(int j) {
-  // 2^-(4j) for j <= 4, 2^-(4(j-3)) for j = 5..7
-  const int s = (j <= 4) ? 4 * j : 4 * (j - 3);
-  return __int_as_float((127 - s) << 23);
-}
-
-__device__ __forceinline__ int nib_elem(int p) {   // position p = 8*i + j -> element
-  const int i = p >> 3, j = p & 7, m = j >> 1;
-  return (j & 1) ? (16 + 4 * i + m) : (4 * i + m);
-}
-
-// one (token, block) per thread, grid-stride
-__device__ void prep_x_range(const __nv_bfloat16 *x, float *xprep, float *xsum, int T, int d,
-                             int tid, int nthreads) {
-  const int nb = d / MOE_QK;
-  for (int it = tid; it < T * nb; it += nthreads) {
-    const int t = it / nb, b = it % nb;
-    const __nv_bfloat16 *xb = x + (size_t)t * d + (size_t)b * MOE_QK;
-    float v[MOE_QK];
-#pragma unroll
-    for (int i = 0; i < MOE_QK; ++i) v[i] = __bfloat162float(xb[i]);
-    float s = 0.f;
-#pragma unroll
-    for (int i = 0; i < MOE_QK; ++i) s += v[i];
-    float *dst = xprep + (size_t)t * d + (size_t)b * MOE_QK;
-#pragma unroll
-    for (int p = 0; p < MOE_QK; ++p) dst[p] = v[nib_elem(p)] * nib_scale(p & 7);
-    xsum[(size_t)t * nb + b] = s;
-  }
-}
-
-// ---------------------------------------------------------------- top-k + softmax
-
-// Warp-level selection for one token. Keys compare by logit (NaN treated as -inf),
-// then by lower index. Writes ids[k], w[k].
-// The selected logits are parked in w[] until the softmax overwrites them.
-__device__ void warp_topk_softmax(const float *lg, int E, int k, float rscale, int32_t *ids, float *w) {
-  const int lane = threadIdx.x & 31;
-  constexpr int kMaxPer = MOE_MAX_E / 32;
-  float v[kMaxPer];
-  uint32_t taken = 0;
-#pragma unroll
-  for (int i = 0; i < kMaxPer; ++i) {
-    const int e = lane + 32 * i;
-    float a = (e < E) ? __ldcg(lg + e) : -INFINITY;
-    if (a != a) a = -INFINITY;
-    v[i] = a;
-    if (e >= E) taken |= 1u << i;
-  }
-  for (int j = 0; j < k; ++j) {
-    // local best among untaken
-    float bv = -INFINITY;
-    int be = 0x7fffffff;
-#pragma unroll
-    for (int i = 0; i < kMaxPer; ++i) {
-      const int e = lane + 32 * i;
-      if (!((taken >> i) & 1u)) {
-        if (v[i] > bv || (v[i] == bv && e < be)) { bv = v[i]; be = e; }
-      }
-    }
-    // warp argmax: larger value, then lower index
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) {
-      const float ov = __shfl_xor_sync(0xffffffffu, bv, o);
-      const int oe = __shfl_xor_sync(0xffffffffu, be, o);
-      if (ov > bv || (ov == bv && oe < be)) { bv = ov; be = oe; }
-    }
-    if ((be & 31) == lane) taken |= 1u << (be >> 5);
-    if (lane == 0) { ids[j] = be; w[j] = __ldcg(lg + be); }
-  }
-  __syncwarp();
-  __threadfence_block();
-  // softmax over the selected logits (original values, so NaN propagates)
-  const float l1 = w[0];
-  float part = 0.f;
-  float ev[MOE_MAX_E / 32];
-#pragma unroll
-  for (int i = 0; i < MOE_MAX_E / 32; ++i) {
-    const int j = lane + 32 * i;
-    ev[i] = (j < k) ? expf(w[j] - l1) : 0.f;
-    part += ev[i];
-  }
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) part += __shfl_xor_sync(0xffffffffu, part, o);
-  const float inv = rscale / part;
-  __syncwarp();
-#pragma unroll
-  for (int i = 0; i < MOE_MAX_E / 32; ++i) {
-    const int j = lane + 32 * i;
-    if (j < k) w[j] = ev[i] * inv;
-  }
-  __syncwarp();
-}
 
 // ---------------------------------------------------------------- permutation (one CTA)
 //
@@ -233,13 +130,16 @@ __device__ void block_permutation(const int32_t *ids, int S, int E, int32_t *cou
 
 // ---------------------------------------------------------------- decode routing kernel
 //
-// T <= 16. CTA b handles experts 4b..4b+3, each split in kRouteParts parts of d; warp
+// T <= 16. CTA b handles kRouteEPC experts, each split in kRouteParts parts of d; warp
 // (expert, part) accumulates lane-strided float4 chunks of W_r against every token, reduces
 // across the warp by a fixed xor tree, and the parts are summed in order. The last CTA to
 // finish (arrival counter) runs top-k + softmax for all tokens and the permutation.
 struct RouteDecodeSmem {
-  float part[4][kRouteParts][kDecodeMaxT];
-  PermSmem perm;
+  float part[kRouteEPC][kRouteParts][kDecodeMaxT];
+  union {
+    PermSmem perm;
+    int32_t cnt[MOE_MAX_E];
+  } u;
   int last;
 };
 
@@ -249,8 +149,8 @@ k_route_decode(const __nv_bfloat16 *__restrict__ x, const float *__restrict__ ro
   __shared__ RouteDecodeSmem sm;
   const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
   const int el = wid / kRouteParts, part = wid % kRouteParts;
-  const int e = blockIdx.x * 4 + el;
-  const int plen = d / kRouteParts;   // multiple of 8
+  const int e = blockIdx.x * kRouteEPC + el;
+  const int plen = d / kRouteParts;   // multiple of 4
   if (e < E) {
     float acc[kDecodeMaxT];
 #pragma unroll
@@ -282,12 +182,12 @@ k_route_decode(const __nv_bfloat16 *__restrict__ x, const float *__restrict__ ro
       if (lane == 0) sm.part[el][part][t] = a;
     }
   }
-  prep_x_range(x, W.xprep, W.xsum, T, d, blockIdx.x * blockDim.x + threadIdx.x,
+  prep_x_range(x, W.x16, W.xblk, T, d, blockIdx.x * blockDim.x + threadIdx.x,
                gridDim.x * blockDim.x);
   __syncthreads();
-  if (threadIdx.x < 4 * kDecodeMaxT) {
+  if (threadIdx.x < kRouteEPC * kDecodeMaxT) {
     const int le = threadIdx.x / kDecodeMaxT, t = threadIdx.x % kDecodeMaxT;
-    const int ee = blockIdx.x * 4 + le;
+    const int ee = blockIdx.x * kRouteEPC + le;
     if (ee < E && t < T) {
       float s = sm.part[le][0][t];
 #pragma unroll
@@ -310,8 +210,13 @@ k_route_decode(const __nv_bfloat16 *__restrict__ x, const float *__restrict__ ro
     warp_topk_softmax(W.logits + (size_t)t * E, E, k, rs, W.ids + (size_t)t * k, W.w + (size_t)t * k);
   __threadfence_block();
   __syncthreads();
-  block_permutation(W.ids, T * k, E, W.counts, W.offsets, W.perm, W.inv, W.act, W.n_act, nullptr,
-                    nullptr, nullptr, 1, sm.perm);
+  if (T * k <= kSmallPermMax) {
+    if (wid == 0)
+      warp_permutation_small(W.ids, T * k, E, W.counts, W.offsets, W.perm, W.inv, W.act, W.n_act, sm.u.cnt);
+  } else {
+    block_permutation(W.ids, T * k, E, W.counts, W.offsets, W.perm, W.inv, W.act, W.n_act, nullptr, nullptr,
+                      nullptr, 1, sm.u.perm);
+  }
   if (threadIdx.x == 0) W.counters[0] = 0;
 }
 
@@ -400,7 +305,7 @@ k_permute(int T, int E, int k, int tile_m, bool want_tiles, MoeWork W) {
 
 __global__ void __launch_bounds__(256)
 k_prep_x(const __nv_bfloat16 *__restrict__ x, int T, int d, MoeWork W) {
-  prep_x_range(x, W.xprep, W.xsum, T, d, blockIdx.x * blockDim.x + threadIdx.x, gridDim.x * blockDim.x);
+  prep_x_range(x, W.x16, W.xblk, T, d, blockIdx.x * blockDim.x + threadIdx.x, gridDim.x * blockDim.x);
 }
 
 }  // namespace
@@ -413,7 +318,8 @@ int moe_launch_route_decode(const MoeLaunch &L, const MoeWork &W, const void *x,
                             const float *router_scale, int T, int d, int E, int k, int num_sms) {
   (void)num_sms;
   if (T > kDecodeMaxT) return -2;
-  const int grid = (E + 3) / 4;
+  if ((d / kRouteParts) % 4) return -2;
+  const int grid = (E + kRouteEPC - 1) / kRouteEPC;
   moe_prof_mark(L.stream, MOE_K_ROUTE, true);
   k_route_decode<<<grid, kRouteThreads, 0, L.stream>>>(static_cast<const __nv_bfloat16 *>(x), router_w,
                                                         router_scale, T, d, E, k, W);

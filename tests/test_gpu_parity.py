@@ -25,7 +25,7 @@ def _built():
 
 
 def _tol(path, T):
-    if path == moe.MOE_PATH_GEMV:
+    if path in (moe.MOE_PATH_GEMV, moe.MOE_PATH_GEMV_SPLIT):
         return TOL_GEMV
     if path == moe.MOE_PATH_GEMM:
         return TOL_GEMM
@@ -61,6 +61,27 @@ def test_small_shapes_gemv(E, k, T, d, f):
     lw = mi.make_layer(seed=E * 1000 + T, layer=0, d=d, f=f, E=E)
     x = mi.make_tokens(E + T, T, d)
     _check_full(x, lw, k, moe.MOE_PATH_GEMV)
+
+
+@pytest.mark.parametrize("E,k,T,d,f", SMALL)
+def test_small_shapes_gemv_split(E, k, T, d, f):
+    """The same shapes through the separate routing / gate_up / down kernels."""
+    lw = mi.make_layer(seed=E * 1000 + T, layer=0, d=d, f=f, E=E)
+    x = mi.make_tokens(E + T, T, d)
+    _check_full(x, lw, k, moe.MOE_PATH_GEMV_SPLIT)
+
+
+@pytest.mark.parametrize("T", [1, 3, 8])
+def test_fused_and_split_decode_agree(T):
+    lw = mi.make_layer(seed=40 + T, d=2816, f=704, E=128)
+    x = mi.make_tokens(41 + T, T, 2816)
+    dl = DevLayer(lw)
+    a = run_layer(x, dl, 8, moe.MOE_PATH_GEMV)
+    b = run_layer(x, dl, 8, moe.MOE_PATH_GEMV_SPLIT)
+    assert np.array_equal(a["ids"], b["ids"]) and np.array_equal(a["perm"], b["perm"])
+    assert rel_err(a["out"], b["out"].astype(np.float64)) <= 1e-5
+    c = run_layer(x, dl, 8, moe.MOE_PATH_GEMV)
+    assert np.array_equal(a["out"].view(np.uint32), c["out"].view(np.uint32))
 
 
 SMALL_GEMM = [  # (E, k, T, d, f): d % 128 == 0, f % 64 == 0
@@ -241,8 +262,10 @@ def test_stack_teacher_forced():
         ref, ids, w, flags = oracle.moe_layer(xs[i], lw.router_w, lw.router_scale, lw.gate_up, lw.down,
                                               lw.expert_scale, k)
         if i + 1 < L:
-            nxt = oracle.rmsnorm_bf16(ref)
-            close = np.abs(nxt.astype(np.int32) - xs[i + 1].astype(np.int32)) <= 1
-            assert close.all() and (nxt != xs[i + 1]).mean() < 0.02
+            # x_{i+1} = bf16(rmsnorm(out_i)): the 1e-3 output bound plus one bf16 rounding on
+            # each side gives max |dx| <= (1e-3 + 2^-8) max |x|
+            nxt = mi.bf16_bits_to_f32(oracle.rmsnorm_bf16(ref)).astype(np.float64)
+            got = mi.bf16_bits_to_f32(xs[i + 1]).astype(np.float64)
+            assert rel_err(got, nxt) <= 1e-3 + 2.0 ** -8
         else:
             assert rel_err(out.cpu().numpy(), ref) <= TOL_GEMV
