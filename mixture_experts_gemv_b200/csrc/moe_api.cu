@@ -89,7 +89,7 @@ Layout make_layout(int maxT, int max_d, int max_f, int max_E, int max_k) {
       S * 4,                             // 6 inv
       (size_t)max_E * 4,                 // 7 act
       16,                                // 8 n_act, n_tiles
-      (size_t)maxT * max_d * 2,          // 9 x16
+      (size_t)maxT * max_d * 2,          // 9 xq
       (size_t)maxT * (max_d / 32) * 8,   // 10 xblk
       S * max_f * 4,                     // 11 h
       16,                                // 12 (unused)
@@ -298,8 +298,8 @@ int moe_init(int device, int max_tokens, int max_d, int max_f, int max_E, int ma
   W.act = reinterpret_cast<int32_t *>(b + Lt.off[7]);
   W.n_act = reinterpret_cast<int32_t *>(b + Lt.off[8]);
   W.n_tiles = reinterpret_cast<int32_t *>(b + Lt.off[8] + 4);
-  W.x16 = reinterpret_cast<__half *>(b + Lt.off[9]);
-  W.xblk = reinterpret_cast<float2 *>(b + Lt.off[10]);
+  W.xq = reinterpret_cast<int16_t *>(b + Lt.off[9]);
+  W.xblk = reinterpret_cast<ActBlk *>(b + Lt.off[10]);
   W.h = reinterpret_cast<float *>(b + Lt.off[11]);
   W.ybuf = reinterpret_cast<float *>(b + Lt.off[13]);
   W.yslot = W.ybuf;

@@ -27,8 +27,8 @@ struct MoeWork {
   int32_t *inv;       // [T*k]  slot -> sorted position
   int32_t *act;       // [E]    active experts, ascending; act[E-1..] unused
   int32_t *n_act;     // [1]
-  __half *x16;        // [T, d] x as scaled f16 in the GEMV's word order (see moe_gemv.cu)
-  float2 *xblk;       // [T, d/32] per block: (-8 * sum of the scaled values, 2^sigma)
+  int16_t *xq;        // [T, d] x as block-scaled int16 in the GEMV's word order
+  struct ActBlk *xblk;   // [T, d/32] per block of xq: -8 * sum of the values, 2^sigma
   float *h;           // [T*k, f] fp32 hidden (GEMV path), slot order
   float *ybuf;        // [T*k, d] per-slot expert outputs (GEMV path)
   uint32_t *counters; // [n] zero-initialised arrival counters (reset by their users)
@@ -63,12 +63,14 @@ __device__ __forceinline__ void report_error(volatile uint32_t *err, uint32_t co
   }
 }
 
-// ---------------------------------------------------------------- f16 activations
+// ---------------------------------------------------------------- int16 activations
 //
-// The GEMV path multiplies Q4_0 codes by f16 activations. Each 32-wide block of an
+// The GEMV path multiplies Q4_0 codes by int16 activations. Each 32-wide block of an
 // activation vector is scaled by a power of two 2^-sigma that puts its largest magnitude in
-// [2^14, 2^15), so converting a bf16 activation to f16 is exact (and an fp32 one keeps 11
-// significant bits); the block's results are multiplied back by 2^sigma.
+// [2^14, 2^15) and rounded to the nearest integer: exact for bf16 values within 2^7 of the
+// block's largest, an error of at most 2^-15 of the largest otherwise. The block's results
+// are multiplied back by 2^sigma. A block holding a NaN or an infinity gets sigma = NaN, so
+// the non-finite value reaches the output.
 struct BlockScale {
   float scale;   // 2^-sigma
   float inv;     // 2^sigma
@@ -81,6 +83,14 @@ __device__ __forceinline__ BlockScale block_scale_for_max(float m) {
   r.inv = __uint_as_float((uint32_t)(eb - 14) << 23);
   return r;
 }
+__device__ __forceinline__ int act_to_i16(float v, float scale) {
+  return __float2int_rn(fminf(fmaxf(v * scale, -32768.f), 32767.f));
+}
+// Per block of an int16 activation vector: -8 * (sum of its 32 values) and 2^sigma.
+struct ActBlk {
+  int neg8sum;
+  float scale;
+};
 // Position of element e (0..31) of a block in the GEMV's word order: code word i (bytes
 // 4i..4i+3) pairs with activations 4i..4i+3 (low nibbles) then 16+4i..16+4i+3 (high).
 __device__ __forceinline__ int gemv_pos(int e) { return (e < 16) ? ((e >> 2) * 8 + (e & 3)) : (((e - 16) >> 2) * 8 + 4 + (e & 3)); }

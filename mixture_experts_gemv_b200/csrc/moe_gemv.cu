@@ -12,13 +12,8 @@
 // units through a ring of shared-memory stages filled by 1-D bulk asynchronous copies
 // (cp.async.bulk, mbarrier completion), so HBM reads stay in flight while the SM decodes.
 //
-// Arithmetic: a Q4_0 weight is (q - 8) * d. The codes of one 4-byte code word are spread
-// into one byte each (low nibbles, then high nibbles); a byte holding q in 0..15 read as an
-// FP8 e4m3 value is exactly q * 2^-9 (subnormal for q < 8, normal above), so the hardware
-// e4m3 -> f16x2 conversion decodes two codes per instruction, exactly. Activations are f16
-// scaled per 32-wide block by a power of two (exact for bf16 x). Products q * 2^-9 * a are
-// formed exactly by the mixed-precision FMA (f16 x f16 + f32) and summed in FP32; per block
-// and token the row accumulator gets d * 2^sigma * (512 * sum - 8 * sum(a)).
+// Arithmetic (moe_gemv_core.cuh): int16 block-scaled activations, dp2a integer dot
+// products of codes and activations, exact per block; one FP32 rounding per block and row.
 
 #include "moe_gemv_core.cuh"
 
@@ -36,8 +31,8 @@ k_gateup_gemv(const uint8_t *__restrict__ gate_up_q4, int d, int f, int k, int n
   const uint32_t rb = (uint32_t)nb * MOE_QBYTES;
   const uint32_t stage_bytes = (2u * kPairs * rb + 16u + 15u) & ~15u;
   uint8_t *smem = align128(smem_raw);
-  uint16_t *xs = reinterpret_cast<uint16_t *>(smem + (size_t)nstages * stage_bytes);   // [kTX][d] f16
-  float2 *ss = reinterpret_cast<float2 *>(xs + (size_t)kTX * d);                         // [kTX][nb]
+  uint16_t *xs = reinterpret_cast<uint16_t *>(smem + (size_t)nstages * stage_bytes);   // [kTX][d] int16
+  ActBlk *ss = reinterpret_cast<ActBlk *>(xs + (size_t)kTX * d);                         // [kTX][nb]
   float *red = reinterpret_cast<float *>(ss + (size_t)kTX * nb);                         // [G*2][kPairs][kTX][2]
   const int upe = f / kUnit;
   const int n_act = *W.n_act;
@@ -92,11 +87,12 @@ k_gateup_gemv(const uint8_t *__restrict__ gate_up_q4, int d, int f, int k, int n
           const int i = i2 / (d / 8), v = i2 % (d / 8);
           const int tok = W.perm[off + g0 + i] / k;
           reinterpret_cast<uint4 *>(xs + (size_t)i * d)[v] =
-              __ldcg(reinterpret_cast<const uint4 *>(W.x16 + (size_t)tok * d) + v);
+              __ldcg(reinterpret_cast<const uint4 *>(W.xq + (size_t)tok * d) + v);
         }
         for (int i2 = threadIdx.x; i2 < ng * nb; i2 += blockDim.x) {
           const int i = i2 / nb, b = i2 % nb;
-          ss[i * nb + b] = __ldcg(W.xblk + (size_t)(W.perm[off + g0 + i] / k) * nb + b);
+          const int2 v = __ldcg(reinterpret_cast<const int2 *>(W.xblk) + (size_t)(W.perm[off + g0 + i] / k) * nb + b);
+          ss[i * nb + b] = ActBlk{v.x, __int_as_float(v.y)};
         }
         __syncthreads();
         if (threadIdx.x == 0) { st_key[0] = e; st_key[1] = g0; }
@@ -151,8 +147,8 @@ k_down_gemv_combine(const uint8_t *__restrict__ down_q4, const float *__restrict
   const uint32_t rb = (uint32_t)nbf * MOE_QBYTES;
   const uint32_t stage_bytes = ((uint32_t)kDnRows * rb + 16u + 15u) & ~15u;
   uint8_t *smem = align128(smem_raw);
-  uint16_t *hs = reinterpret_cast<uint16_t *>(smem + (size_t)nstages * stage_bytes);   // [kTX][f] f16 h
-  float2 *hblk = reinterpret_cast<float2 *>(hs + (size_t)kTX * f);                      // [kTX][nbf]
+  uint16_t *hs = reinterpret_cast<uint16_t *>(smem + (size_t)nstages * stage_bytes);   // [kTX][f] int16 h
+  ActBlk *hblk = reinterpret_cast<ActBlk *>(hs + (size_t)kTX * f);                      // [kTX][nbf]
   float *red = reinterpret_cast<float *>(hblk + (size_t)kTX * nbf);                     // [2][kTX][kDnRows]
   const int upe = d / kUnit;
   const int n_act = *W.n_act;
@@ -201,21 +197,22 @@ k_down_gemv_combine(const uint8_t *__restrict__ down_q4, const float *__restrict
     for (int g0 = 0; g0 < cnt; g0 += kTX) {
       const int ng = min(kTX, cnt - g0);
       if (st_key[0] != e || st_key[1] != g0) {
-        // h of these slots -> f16 scaled per 32-wide block, in the word order; one warp
-        // per (slot, block): lane = element
+        // h of these slots -> block-scaled int16 in the word order; one warp per (slot,
+        // block): lane = element
         for (int it2 = wq; it2 < ng * nbf; it2 += kDnThreads / 32) {
           const int i = it2 / nbf, cb = it2 % nbf;
           const float v = __ldcg(W.h + (size_t)W.perm[off + g0 + i] * f + (size_t)cb * MOE_QK + lane);
           float m = fabsf(v);
 #pragma unroll
           for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+          const bool finite = __all_sync(0xffffffffu, isfinite(v));
           const BlockScale bs = block_scale_for_max(m);
-          const __half hv = __float2half_rn(v * bs.scale);
-          hs[(size_t)i * f + (size_t)cb * MOE_QK + gemv_pos(lane)] = __half_as_ushort(hv);
-          float sm = __half2float(hv);
+          const int a = act_to_i16(v, bs.scale);
+          hs[(size_t)i * f + (size_t)cb * MOE_QK + gemv_pos(lane)] = (uint16_t)(a & 0xffff);
+          int sm = a;
 #pragma unroll
           for (int o = 16; o > 0; o >>= 1) sm += __shfl_xor_sync(0xffffffffu, sm, o);
-          if (lane == 0) hblk[i * nbf + cb] = make_float2(-8.f * sm, bs.inv);
+          if (lane == 0) hblk[i * nbf + cb] = ActBlk{-8 * sm, finite ? bs.inv : __int_as_float(0x7fffffff)};
         }
         __syncthreads();
         if (threadIdx.x == 0) { st_key[0] = e; st_key[1] = g0; }

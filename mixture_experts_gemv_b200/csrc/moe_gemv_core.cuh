@@ -1,19 +1,17 @@
 // moe_gemv_core.cuh -- device building blocks of the Q4_0 decode GEMVs, shared by the
 // separate-kernel path (moe_gemv.cu) and the fused decode kernel (moe_decode.cu).
 //
-// Arithmetic: a Q4_0 weight is (q - 8) * d. The codes of one 4-byte code word are spread
-// into one byte each (low nibbles, then high nibbles); a byte holding q in 0..15 read as an
-// FP8 e4m3 value is exactly q * 2^-9 (subnormal for q < 8, normal above), so the hardware
-// e4m3 -> f16x2 conversion decodes two codes per instruction, exactly. Activations are f16
-// scaled per 32-wide block by a power of two (exact for bf16 x). Products q * 2^-9 * a are
-// formed exactly by the mixed-precision FMA (f16 x f16 + f32) and summed in FP32; per block
-// and token the row accumulator gets d * 2^sigma * (512 * sum - 8 * sum(a)).
+// Arithmetic: a Q4_0 weight is (q - 8) * d. Activations are int16, block-scaled by a power
+// of two (moe_common.cuh). The low nibbles of a 4-byte code word, masked in place, are four
+// bytes q; the high nibbles, masked in place, are four bytes 16 q. The integer dot-product
+// instruction dp2a multiplies two int16 activations by two code bytes and adds both to an
+// int32 accumulator, exactly. Per block and token: r = sum(q a) - 8 sum(a), an exact
+// integer with |r| < 2^23, and the row accumulator gets d * 2^sigma * r (one FP32 rounding).
 #pragma once
 
 #include "moe_common.cuh"
 
 namespace {
-
 
 constexpr int kGran = 8;        // blocks per granule: 144 bytes, 16-byte aligned in aligned rows
 constexpr int kMaxGran = 16;    // gate_up: one warp per granule, d <= 4096
@@ -24,7 +22,6 @@ constexpr int kGuStagesMax = 3;
 constexpr int kDnRows = 128;    // rows per down chunk
 constexpr int kDnThreads = 256; // 4 warps x 32 rows, 2 parts of the row's blocks
 constexpr int kDnStagesMax = 4;
-constexpr uint32_t kMagic = 0x4B000000u;   // 2^23
 constexpr int kSmemBudget = 222 * 1024;
 
 __device__ __forceinline__ float gelu_tanh_f(float z) {
@@ -32,55 +29,29 @@ __device__ __forceinline__ float gelu_tanh_f(float z) {
   return 0.5f * z * (1.0f + tanhf(c * (z + 0.044715f * z * z * z)));
 }
 
-// Two e4m3 bytes (the low or high 16 bits of v) -> f16x2.
-__device__ __forceinline__ uint32_t e4m3x2_lo(uint32_t v) {
-  uint32_t r;
-  asm("{.reg .b16 l, h;\n\tmov.b32 {l, h}, %1;\n\tcvt.rn.f16x2.e4m3x2 %0, l;}" : "=r"(r) : "r"(v));
+// c + a.h0 * b.byte0 + a.h1 * b.byte1 (lo) or bytes 2, 3 (hi): a two signed 16-bit values,
+// b four unsigned bytes.
+__device__ __forceinline__ int dp2a_lo(uint32_t a, uint32_t b, int c) {
+  int r;
+  asm("dp2a.lo.s32.u32 %0, %1, %2, %3;" : "=r"(r) : "r"(a), "r"(b), "r"(c));
   return r;
 }
-__device__ __forceinline__ uint32_t e4m3x2_hi(uint32_t v) {
-  uint32_t r;
-  asm("{.reg .b16 l, h;\n\tmov.b32 {l, h}, %1;\n\tcvt.rn.f16x2.e4m3x2 %0, h;}" : "=r"(r) : "r"(v));
+__device__ __forceinline__ int dp2a_hi(uint32_t a, uint32_t b, int c) {
+  int r;
+  asm("dp2a.hi.s32.u32 %0, %1, %2, %3;" : "=r"(r) : "r"(a), "r"(b), "r"(c));
   return r;
 }
-// c + a.lo * b.lo and c + a.hi * b.hi with f16 inputs, exact product, FP32 sum.
-__device__ __forceinline__ float fma_h_lo(uint32_t a, uint32_t b, float c) {
-  float r;
-  asm("{.reg .b16 al, ah, bl, bh;\n\tmov.b32 {al, ah}, %1;\n\tmov.b32 {bl, bh}, %2;\n\tfma.rn.f32.f16 %0, al, bl, %3;}"
-      : "=f"(r) : "r"(a), "r"(b), "f"(c));
-  return r;
+// One code word against 8 activations in the word order: lo = w & 0x0F0F0F0F (codes of
+// elements 4i..4i+3), hi = w & 0xF0F0F0F0 (16 x codes of 16+4i..16+4i+3).
+__device__ __forceinline__ void dot8i(uint32_t lo, uint32_t hi, const uint4 &xv, int &al, int &ah) {
+  al = dp2a_lo(xv.x, lo, al);
+  al = dp2a_hi(xv.y, lo, al);
+  ah = dp2a_lo(xv.z, hi, ah);
+  ah = dp2a_hi(xv.w, hi, ah);
 }
-__device__ __forceinline__ float fma_h_hi(uint32_t a, uint32_t b, float c) {
-  float r;
-  asm("{.reg .b16 al, ah, bl, bh;\n\tmov.b32 {al, ah}, %1;\n\tmov.b32 {bl, bh}, %2;\n\tfma.rn.f32.f16 %0, ah, bh, %3;}"
-      : "=f"(r) : "r"(a), "r"(b), "f"(c));
-  return r;
-}
-
-// The eight codes of one code word as f16 q * 2^-9, in the activation word order:
-// c0 = (e0, e1), c1 = (e2, e3) of the low nibbles, c2, c3 the same of the high nibbles.
-struct Codes8 {
-  uint32_t c[4];
-};
-__device__ __forceinline__ Codes8 decode8(uint32_t w) {
-  const uint32_t lo = w & 0x0F0F0F0Fu, hi = (w >> 4) & 0x0F0F0F0Fu;
-  Codes8 r;
-  r.c[0] = e4m3x2_lo(lo);
-  r.c[1] = e4m3x2_hi(lo);
-  r.c[2] = e4m3x2_lo(hi);
-  r.c[3] = e4m3x2_hi(hi);
-  return r;
-}
-// (a0, a1) += codes . activations (8 f16 in a uint4)
-__device__ __forceinline__ void dot8h(const Codes8 &k, const uint4 &xv, float &a0, float &a1) {
-  a0 = fma_h_lo(k.c[0], xv.x, a0);
-  a1 = fma_h_hi(k.c[0], xv.x, a1);
-  a0 = fma_h_lo(k.c[1], xv.y, a0);
-  a1 = fma_h_hi(k.c[1], xv.y, a1);
-  a0 = fma_h_lo(k.c[2], xv.z, a0);
-  a1 = fma_h_hi(k.c[2], xv.z, a1);
-  a0 = fma_h_lo(k.c[3], xv.w, a0);
-  a1 = fma_h_hi(k.c[3], xv.w, a1);
+// y += d * 2^sigma * (al + ah / 16) where al started at -8 sum(a): exact integer, one rounding
+__device__ __forceinline__ float block_finish(float y, float d, float scale, int al, int ah) {
+  return fmaf(d * scale, (float)(al + (ah >> 4)), y);
 }
 
 struct Blk {
@@ -181,32 +152,35 @@ __device__ __forceinline__ GuChunk gu_chunk(int u, int u1, int upe) {
 
 template <int NT>
 __device__ __forceinline__ void gu_block(const Blk &bg, const Blk &bu, int b, int nb, const uint16_t *xs,
-                                         const float2 *ss, int d, float (&yg)[NT], float (&yu)[NT]) {
-  float ag0[NT], ag1[NT], au0[NT], au1[NT];
+                                         const ActBlk *ss, int d, float (&yg)[NT], float (&yu)[NT]) {
+  int gl[NT], gh[NT], ul[NT], uh[NT];
+  float sc[NT];
 #pragma unroll
-  for (int i = 0; i < NT; ++i) { ag0[i] = 0.f; ag1[i] = 0.f; au0[i] = 0.f; au1[i] = 0.f; }
+  for (int i = 0; i < NT; ++i) {
+    const ActBlk ab = ss[i * nb + b];
+    gl[i] = ab.neg8sum; ul[i] = ab.neg8sum; gh[i] = 0; uh[i] = 0; sc[i] = ab.scale;
+  }
 #pragma unroll
   for (int wi = 0; wi < 4; ++wi) {
-    const Codes8 kg = decode8(bg.q[wi]);
-    const Codes8 ku = decode8(bu.q[wi]);
+    const uint32_t glo = bg.q[wi] & 0x0F0F0F0Fu, ghi = bg.q[wi] & 0xF0F0F0F0u;
+    const uint32_t ulo = bu.q[wi] & 0x0F0F0F0Fu, uhi = bu.q[wi] & 0xF0F0F0F0u;
 #pragma unroll
     for (int i = 0; i < NT; ++i) {
       const uint4 xv = *reinterpret_cast<const uint4 *>(xs + (size_t)i * d + b * MOE_QK + 8 * wi);
-      dot8h(kg, xv, ag0[i], ag1[i]);
-      dot8h(ku, xv, au0[i], au1[i]);
+      dot8i(glo, ghi, xv, gl[i], gh[i]);
+      dot8i(ulo, uhi, xv, ul[i], uh[i]);
     }
   }
 #pragma unroll
   for (int i = 0; i < NT; ++i) {
-    const float2 sb = ss[i * nb + b];   // (-8 * sum a, 2^sigma)
-    yg[i] = fmaf(bg.d * sb.y, fmaf(512.f, ag0[i] + ag1[i], sb.x), yg[i]);
-    yu[i] = fmaf(bu.d * sb.y, fmaf(512.f, au0[i] + au1[i], sb.x), yu[i]);
+    yg[i] = block_finish(yg[i], bg.d, sc[i], gl[i], gh[i]);
+    yu[i] = block_finish(yu[i], bu.d, sc[i], ul[i], uh[i]);
   }
 }
 
 template <int NT, bool ALIGNED>
 __device__ __forceinline__ void gu_compute(const uint8_t *st, uint32_t rb, int nb, const uint16_t *xs,
-                                           const float2 *ss, int d, float *red_out /* [NT][2] */) {
+                                           const ActBlk *ss, int d, float *red_out /* [NT][2] */) {
   // called by every lane of the warp (rows past the chunk read stale shared memory and are
   // not stored by the caller)
   const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
@@ -269,7 +243,7 @@ __device__ __forceinline__ DnChunk dn_chunk(int u, int u1, int upe) {
 
 template <int NT>
 __device__ __forceinline__ void dn_compute(const uint8_t *st, uint32_t rb, int nbf, const uint16_t *hs,
-                                           const float2 *hb, int f, float *red_out /* [NT] */) {
+                                           const ActBlk *hb, int f, float *red_out /* [NT] */) {
   const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
   const int row = (w & 3) * 32 + lane, part = w >> 2;
   const int bpp = (nbf + 1) / 2;
@@ -280,21 +254,22 @@ __device__ __forceinline__ void dn_compute(const uint8_t *st, uint32_t rb, int n
   const uint32_t orow = (uint32_t)row * rb;
   for (int b = b0; b < b1; ++b) {
     const Blk bk = load_blk(st, orow + (uint32_t)b * MOE_QBYTES);
-    float a0[NT], a1[NT];
-#pragma unroll
-    for (int i = 0; i < NT; ++i) { a0[i] = 0.f; a1[i] = 0.f; }
-#pragma unroll
-    for (int wi = 0; wi < 4; ++wi) {
-      const Codes8 kc = decode8(bk.q[wi]);
-#pragma unroll
-      for (int i = 0; i < NT; ++i)
-        dot8h(kc, *reinterpret_cast<const uint4 *>(hs + (size_t)i * f + b * MOE_QK + 8 * wi), a0[i], a1[i]);
-    }
+    int al[NT], ah[NT];
+    float sc[NT];
 #pragma unroll
     for (int i = 0; i < NT; ++i) {
-      const float2 sb = hb[i * nbf + b];
-      y[i] = fmaf(bk.d * sb.y, fmaf(512.f, a0[i] + a1[i], sb.x), y[i]);
+      const ActBlk ab = hb[i * nbf + b];
+      al[i] = ab.neg8sum; ah[i] = 0; sc[i] = ab.scale;
     }
+#pragma unroll
+    for (int wi = 0; wi < 4; ++wi) {
+      const uint32_t lo = bk.q[wi] & 0x0F0F0F0Fu, hi = bk.q[wi] & 0xF0F0F0F0u;
+#pragma unroll
+      for (int i = 0; i < NT; ++i)
+        dot8i(lo, hi, *reinterpret_cast<const uint4 *>(hs + (size_t)i * f + b * MOE_QK + 8 * wi), al[i], ah[i]);
+    }
+#pragma unroll
+    for (int i = 0; i < NT; ++i) y[i] = block_finish(y[i], bk.d, sc[i], al[i], ah[i]);
   }
 #pragma unroll
   for (int i = 0; i < NT; ++i) red_out[i * kDnRows] = y[i];

@@ -130,8 +130,8 @@ extern "C" int moe_layer_forward_static(const void *x, const float *router_w, co
   W.act = reinterpret_cast<int32_t *>(b + kOffAct);
   W.n_act = reinterpret_cast<int32_t *>(b + kOffNAct);
   W.n_tiles = reinterpret_cast<int32_t *>(b + kOffNAct + 4);
-  W.x16 = reinterpret_cast<__half *>(b + kOffXprep);
-  W.xblk = reinterpret_cast<float2 *>(b + kOffXblk);
+  W.xq = reinterpret_cast<int16_t *>(b + kOffXprep);
+  W.xblk = reinterpret_cast<ActBlk *>(b + kOffXblk);
   W.h = reinterpret_cast<float *>(b + kOffH);
   W.ybuf = reinterpret_cast<float *>(b + kOffYbuf);
   W.yslot = W.ybuf;

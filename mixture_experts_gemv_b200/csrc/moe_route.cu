@@ -182,7 +182,7 @@ k_route_decode(const __nv_bfloat16 *__restrict__ x, const float *__restrict__ ro
       if (lane == 0) sm.part[el][part][t] = a;
     }
   }
-  prep_x_range(x, W.x16, W.xblk, T, d, blockIdx.x * blockDim.x + threadIdx.x,
+  prep_x_range(x, W.xq, W.xblk, T, d, blockIdx.x * blockDim.x + threadIdx.x,
                gridDim.x * blockDim.x);
   __syncthreads();
   if (threadIdx.x < kRouteEPC * kDecodeMaxT) {
@@ -305,7 +305,7 @@ k_permute(int T, int E, int k, int tile_m, bool want_tiles, MoeWork W) {
 
 __global__ void __launch_bounds__(256)
 k_prep_x(const __nv_bfloat16 *__restrict__ x, int T, int d, MoeWork W) {
-  prep_x_range(x, W.x16, W.xblk, T, d, blockIdx.x * blockDim.x + threadIdx.x, gridDim.x * blockDim.x);
+  prep_x_range(x, W.xq, W.xblk, T, d, blockIdx.x * blockDim.x + threadIdx.x, gridDim.x * blockDim.x);
 }
 
 }  // namespace

@@ -15,10 +15,10 @@ namespace {
 
 // ---------------------------------------------------------------- x preparation
 //
-// For the Q4_0 GEMV: each 32-wide block of x becomes f16 scaled by 2^-sigma (exact for
-// bf16 values, see block_scale_for_max), stored in the GEMV's word order, with the block's
-// (-8 * sum of the scaled values, 2^sigma). One (token, block) per thread, grid-stride.
-__device__ void prep_x_range(const __nv_bfloat16 *x, __half *x16, float2 *xblk, int T, int d, int tid,
+// For the Q4_0 GEMV: each 32-wide block of x becomes block-scaled int16 (moe_common.cuh),
+// stored in the GEMV's word order, with the block's ActBlk. One (token, block) per thread,
+// grid-stride.
+__device__ void prep_x_range(const __nv_bfloat16 *x, int16_t *xq, ActBlk *xblk, int T, int d, int tid,
                              int nthreads) {
   const int nb = d / MOE_QK;
   for (int it = tid; it < T * nb; it += nthreads) {
@@ -36,25 +36,29 @@ __device__ void prep_x_range(const __nv_bfloat16 *x, __half *x16, float2 *xblk, 
       }
     }
     float m = 0.f;
+    bool finite = true;
 #pragma unroll
-    for (int i = 0; i < MOE_QK; ++i) m = fmaxf(m, fabsf(v[i]));
+    for (int i = 0; i < MOE_QK; ++i) {
+      m = fmaxf(m, fabsf(v[i]));
+      finite = finite && isfinite(v[i]);
+    }
     const BlockScale bs = block_scale_for_max(m);
     // output position p = 8 i + r holds element 4 i + r (r < 4) or 16 + 4 i + r - 4
     uint32_t pk[MOE_QK / 2];
-    float s = 0.f;
+    int s = 0;
 #pragma unroll
     for (int p = 0; p < MOE_QK; ++p) {
       const int i = p >> 3, r = p & 7;
       const int e = (r < 4) ? (4 * i + r) : (16 + 4 * i + r - 4);
-      const __half hv = __float2half_rn(v[e] * bs.scale);
-      s += __half2float(hv);
-      const uint32_t bits = (uint32_t)__half_as_ushort(hv);
+      const int a = act_to_i16(v[e], bs.scale);
+      s += a;
+      const uint32_t bits = (uint32_t)a & 0xffffu;
       if (p & 1) pk[p >> 1] |= bits << 16; else pk[p >> 1] = bits;
     }
-    uint4 *dst = reinterpret_cast<uint4 *>(x16 + (size_t)t * d + (size_t)b * MOE_QK);
+    uint4 *dst = reinterpret_cast<uint4 *>(xq + (size_t)t * d + (size_t)b * MOE_QK);
 #pragma unroll
     for (int i = 0; i < 4; ++i) dst[i] = make_uint4(pk[4 * i], pk[4 * i + 1], pk[4 * i + 2], pk[4 * i + 3]);
-    xblk[(size_t)t * nb + b] = make_float2(-8.f * s, bs.inv);
+    xblk[(size_t)t * nb + b] = ActBlk{-8 * s, finite ? bs.inv : __int_as_float(0x7fffffff)};
   }
 }
 
@@ -119,15 +123,94 @@ __device__ void warp_topk_softmax_t(const float *lg, int E, int k, float rscale,
   __syncwarp();
 }
 
+// k <= 8: every lane sorts its keys, then five butterfly steps merge sorted top-8 lists
+// (exchange with the partner lane, keep the 8 largest of the 16 by a bitonic merge), so
+// every lane ends with the token's sorted top 8 after 5 shuffle rounds instead of k
+// dependent warp maxima.
+template <int kMaxPer>
+__device__ void warp_top8_softmax_t(const float *lg, int E, int k, float rscale, int32_t *ids, float *w) {
+  const int lane = threadIdx.x & 31;
+  uint64_t t[8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) t[i] = 0ull;
+  // insert this lane's keys into a sorted (descending) list of 8
+#pragma unroll
+  for (int i = 0; i < kMaxPer; ++i) {
+    const int e = lane + 32 * i;
+    uint64_t v = (e < E) ? topk_key(__ldcg(lg + e), e) : 0ull;
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      const uint64_t hi = t[j] > v ? t[j] : v, lo = t[j] > v ? v : t[j];
+      t[j] = hi;
+      v = lo;
+    }
+  }
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    uint64_t u[8];
+#pragma unroll
+    for (int j = 0; j < 8; ++j) u[j] = __shfl_xor_sync(0xffffffffu, t[j], o);
+    // top 8 of two descending lists: pairwise max against the reversed partner list is a
+    // bitonic sequence holding the 8 largest; sort it descending
+#pragma unroll
+    for (int j = 0; j < 8; ++j) t[j] = t[j] > u[7 - j] ? t[j] : u[7 - j];
+#pragma unroll
+    for (int s2 = 4; s2 > 0; s2 >>= 1) {
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        if ((j & s2) == 0) {
+          const uint64_t a2 = t[j], b2 = t[j + s2];
+          t[j] = a2 > b2 ? a2 : b2;
+          t[j + s2] = a2 > b2 ? b2 : a2;
+        }
+      }
+    }
+  }
+  // every lane holds the sorted top 8; lanes j < k publish pick j
+  const float l1 = topk_key_value(t[0]);
+  float part = 0.f;
+  float mine_v = 0.f;
+  int mine_e = 0;
+#pragma unroll
+  for (int j = 0; j < 8; ++j) {
+    if (j < k) {
+      const float v = topk_key_value(t[j]);
+      const float ev = expf(v - l1);
+      part += ev;
+      if (j == lane) { mine_v = ev; mine_e = (int)(0xffffffffu - (uint32_t)t[j]); }
+    }
+  }
+  if (lane < k) {
+    ids[lane] = mine_e;
+    w[lane] = mine_v * (rscale / part);
+  }
+  __syncwarp();
+}
+
 // E <= 32 * kMaxPer logits per lane-strided register file.
+// kMaxE: the largest E the caller supports (the register file of the selection grows with it).
+template <int kMaxE = MOE_MAX_E>
 __device__ __forceinline__ void warp_topk_softmax(const float *lg, int E, int k, float rscale, int32_t *ids,
                                                   float *w) {
-  if (E <= 128)
+  if (k <= 8 && E <= 128) {
+    warp_top8_softmax_t<4>(lg, E, k, rscale, ids, w);
+    return;
+  }
+  if (k <= 8 && E <= 256) {
+    warp_top8_softmax_t<8>(lg, E, k, rscale, ids, w);
+    return;
+  }
+  if (E <= 128) {
     warp_topk_softmax_t<4>(lg, E, k, rscale, ids, w);
-  else if (E <= 256)
-    warp_topk_softmax_t<8>(lg, E, k, rscale, ids, w);
-  else
-    warp_topk_softmax_t<MOE_MAX_E / 32>(lg, E, k, rscale, ids, w);
+    return;
+  }
+  if constexpr (kMaxE > 128) {
+    if (E <= 256) {
+      warp_topk_softmax_t<8>(lg, E, k, rscale, ids, w);
+      return;
+    }
+  }
+  if constexpr (kMaxE > 256) warp_topk_softmax_t<MOE_MAX_E / 32>(lg, E, k, rscale, ids, w);
 }
 
 // Exclusive prefix sums of two int sequences a[0..n), b[0..n) in shared memory, in place,
@@ -164,6 +247,67 @@ __device__ void block_exclusive_scan2_smem(int32_t *a, int32_t *b, int n, int32_
     rb += vb;
   }
   __syncthreads();
+}
+
+// Stable counting sort of S slot ids (shared memory) by one warp, no CTA barrier. Slots
+// are taken 32 at a time: __match_any groups the lanes of one expert, a slot's rank is the
+// number of its expert's slots in earlier rounds plus its lanes below it in this round.
+// Offsets, the active list and n_act come from a lane-chunked scan of the counts. inv[]
+// holds the rank until the last step, which turns it into the sorted position.
+__device__ void warp_permutation(const int32_t *ids, int S, int E, int32_t *counts, int32_t *offsets,
+                                 int32_t *perm, int32_t *inv, int32_t *act, int32_t *n_act) {
+  const int lane = threadIdx.x & 31;
+  for (int e = lane; e < E; e += 32) counts[e] = 0;
+  __syncwarp();
+  const uint32_t below = (1u << lane) - 1u;
+  for (int s0 = 0; s0 < S; s0 += 32) {
+    const int s = s0 + lane;
+    const bool valid = s < S;
+    const int id = valid ? ids[s] : -1 - lane;   // padding lanes get ids of their own
+    const uint32_t m = __match_any_sync(0xffffffffu, id);
+    const int base = valid ? counts[id] : 0;
+    __syncwarp();
+    if (valid) {
+      if ((m & below) == 0) counts[id] = base + __popc(m);
+      inv[s] = base + __popc(m & below);
+    }
+    __syncwarp();
+  }
+  const int per = (E + 31) / 32;
+  const int e0 = min(E, lane * per), e1 = min(E, e0 + per);
+  int c_sum = 0, a_sum = 0;
+  for (int e = e0; e < e1; ++e) {
+    const int c = counts[e];
+    c_sum += c;
+    a_sum += c > 0;
+  }
+  int c_inc = c_sum, a_inc = a_sum;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int nc = __shfl_up_sync(0xffffffffu, c_inc, o), na = __shfl_up_sync(0xffffffffu, a_inc, o);
+    if (lane >= o) {
+      c_inc += nc;
+      a_inc += na;
+    }
+  }
+  int c_run = c_inc - c_sum, a_run = a_inc - a_sum;
+  for (int e = e0; e < e1; ++e) {
+    const int c = counts[e];
+    offsets[e] = c_run;
+    if (c > 0) act[a_run++] = e;
+    c_run += c;
+  }
+  if (lane == 31) {
+    offsets[E] = c_inc;
+    *n_act = a_inc;
+  }
+  __syncwarp();
+  for (int s = lane; s < S; s += 32) {
+    const int pos = offsets[ids[s]] + inv[s];
+    perm[pos] = s;
+    inv[s] = pos;
+  }
+  __syncwarp();
 }
 
 // Stable counting sort of S small slot ids (shared memory) by the whole CTA: per-expert counts
