@@ -31,13 +31,19 @@ constexpr int kFStages = 3;
 constexpr int kFMaxCompute = 22;   // compute warps (one more warp produces)
 constexpr int kFMinCompute = 8;
 constexpr int kDnGroups = kDnRows / 32;   // 32-row groups of a down chunk
-constexpr int kBarCompute = 1;            // named barrier of the compute warps
+// Named barriers (0 is __syncthreads): compute warps only; FULL / EMPTY of the two reduction
+// buffers between the compute warps and the epilogue warp; compute + epilogue warps.
+constexpr int kBarCompute = 1;
+constexpr int kBarFull0 = 2;
+constexpr int kBarEmpty0 = 4;
+constexpr int kBarTeam = 6;
+constexpr int kTXg = 3;                   // tokens per gate_up pass (register budget)
 // Cost of a scheduling unit of an expert with T_e tokens: reading the codes is shared by
 // the tokens, the multiply-adds are per token.
 constexpr int kUnitDecode = 5, kUnitToken = 4;
 
-// Compute warps per CTA: two gate_up work items (gate rows, up rows) per granule, at least
-// enough for the down row groups.
+// Compute warps per CTA: one per gate_up work item (2 per granule), at least enough for the
+// down row groups. Two more warps: the producer and the epilogue warp.
 __host__ __device__ inline int fused_compute_warps(int G) {
   const int w = 2 * G;
   return w < kFMinCompute ? kFMinCompute : (w > kFMaxCompute ? kFMaxCompute : w);
@@ -54,13 +60,16 @@ struct FusedShared {
   int32_t counts[kFMaxE];
   int32_t offsets[kFMaxE + 1];
   int32_t act[kFMaxE];
-  int32_t pc[kFMaxE + 1];     // exclusive prefix of the per-unit costs over the active experts
+  union {
+    float part[kFMaxCompute + 2][kFMaxT];   // router partial sums (phase 0)
+    int32_t pc[kFMaxE + 1];   // exclusive prefix of the per-unit costs over the active experts
+  };
   int32_t wcnt[kFMaxE / 32];  // active experts per 32-expert group
   uint32_t xb[4];             // cost positions of this CTA's unit boundaries
-  float part[kFMaxCompute + 1][kFMaxT];
   int n_act;
   int seq[4];                 // this CTA's unit ranges: gate_up [0, 1), down [2, 3)
   int ok;
+  int abort;                  // set by any expired wait: the warps keep their barrier sequence, skip work
 };
 
 __device__ __forceinline__ unsigned long long ld_acquire_u64(const unsigned long long *p) {
@@ -72,18 +81,6 @@ __device__ __forceinline__ unsigned long long ld_acquire_u64(const unsigned long
 __device__ __forceinline__ void named_sync(int id, int n) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(n) : "memory");
 }
-// Named barrier that also returns whether any participating thread passed pred != 0.
-__device__ __forceinline__ int named_sync_or(int id, int n, int pred) {
-  int r;
-  asm volatile(
-      "{\n\t.reg .pred p, q;\n\tsetp.ne.s32 p, %1, 0;\n\t"
-      "bar.red.or.pred q, %2, %3, p;\n\tselp.s32 %0, 1, 0, q;\n\t}"
-      : "=r"(r)
-      : "r"(pred), "r"(id), "r"(n)
-      : "memory");
-  return r;
-}
-
 // Grid-wide barrier on a monotonically increasing 64-bit counter, split in two: arrival k of
 // a phase returns the end of its window of gridDim.x arrivals; the wait spins (bounded) until
 // the counter reaches it. One thread per CTA, after the CTA's writes are ordered before it.
@@ -109,12 +106,32 @@ __device__ bool grid_wait(const unsigned long long *ctr, unsigned long long targ
   __threadfence();
   return ok;
 }
-// The compute warps' grid barrier (named barrier inside the CTA).
-__device__ bool grid_barrier_c(unsigned long long *ctr, volatile uint32_t *err, uint32_t where, int nct, int &ok_s) {
-  named_sync(kBarCompute, nct);
-  if (threadIdx.x == 0) ok_s = grid_wait(ctr, grid_arrive(ctr), err, where) ? 1 : 0;
-  named_sync(kBarCompute, nct);
-  return ok_s != 0;
+__device__ __forceinline__ void named_arrive(int id, int n) {
+  asm volatile("bar.arrive %0, %1;" ::"r"(id), "r"(n) : "memory");
+}
+// Grid barrier of the compute and epilogue warps (the named barrier kBarTeam inside the CTA).
+// An expired wait sets *abort; the caller keeps going.
+__device__ void grid_barrier_team(unsigned long long *ctr, volatile uint32_t *err, uint32_t where, int nteam,
+                                  volatile int *abort) {
+  named_sync(kBarTeam, nteam);
+  if (threadIdx.x == 0 && !grid_wait(ctr, grid_arrive(ctr), err, where)) *abort = 1;
+  named_sync(kBarTeam, nteam);
+}
+// Wait for an mbarrier phase, at most MOE_WAIT_NS; gives up at once when *abort is set and
+// sets it when the bound expires.
+__device__ bool wait_phase(uint64_t *bar, uint32_t parity, volatile int *abort, volatile uint32_t *err,
+                           uint32_t where) {
+  if (mbar_test(bar, parity)) return true;
+  const uint64_t t0 = globaltimer_ns();
+  while (!mbar_test(bar, parity)) {
+    if (*abort) return false;
+    if (globaltimer_ns() - t0 > MOE_WAIT_NS) {
+      report_error(err, MOE_DEV_ERR_TIMEOUT, where);
+      *abort = 1;
+      return false;
+    }
+  }
+  return true;
 }
 
 struct FChunk {
@@ -150,9 +167,11 @@ struct FSeq {
 
 // Four consecutive lanes turn one 32-wide block into block-scaled int16 in the GEMV word
 // order (moe_common.cuh): lane q = lane & 3 holds elements 8q .. 8q+7 in v[], which go to
-// positions p1 .. p1+3 and p1+8 .. p1+11, p1 = 16 (q & 1) + 4 (q >> 1). The block's ActBlk
+// positions p1 .. p1+3 and p1+8 .. p1+11, p1 = 16 (q & 1) + 4 (q >> 1). With sw = 1 the
+// block's 16-byte words are stored swapped in pairs (word w at w ^ 1). The block's ActBlk
 // goes to *blk_s. Every lane of the warp calls.
-__device__ __forceinline__ void stage_block_q(const float (&v)[8], bool valid, uint16_t *blk16, ActBlk *blk_s) {
+__device__ __forceinline__ void stage_block_q(const float (&v)[8], bool valid, int sw, uint16_t *blk16,
+                                              ActBlk *blk_s) {
   const int q = threadIdx.x & 3;
   float m = 0.f;
   bool finite = true;
@@ -179,45 +198,88 @@ __device__ __forceinline__ void stage_block_q(const float (&v)[8], bool valid, u
   s += __shfl_xor_sync(0xffffffffu, s, 2);
   if (valid) {
     const int p1 = 16 * (q & 1) + 4 * (q >> 1);
-    *reinterpret_cast<uint2 *>(blk16 + p1) = make_uint2(pk[0], pk[1]);
-    *reinterpret_cast<uint2 *>(blk16 + p1 + 8) = make_uint2(pk[2], pk[3]);
+    const int wa = (p1 >> 3) ^ sw, wb = ((p1 >> 3) + 1) ^ sw;
+    *reinterpret_cast<uint2 *>(blk16 + 8 * wa + (p1 & 7)) = make_uint2(pk[0], pk[1]);
+    *reinterpret_cast<uint2 *>(blk16 + 8 * wb + (p1 & 7)) = make_uint2(pk[2], pk[3]);
     if (q == 0) *blk_s = ActBlk{-8 * s, fin ? bs.inv : __int_as_float(0x7fffffff)};
   }
 }
 
-// One gate or up row block against NT tokens' staged activations.
+// Two consecutive Q4_0 blocks (36 bytes) of a row at a shared-memory byte offset o that is
+// 8-byte aligned (ODD = false) or 4 bytes past it (ODD = true).
+template <bool ODD>
+__device__ __forceinline__ void load_span2(const uint8_t *smem, uint32_t o, Blk &b0, Blk &b1) {
+  uint32_t w[10];
+  if (!ODD) {
+    const uint2 *wp = reinterpret_cast<const uint2 *>(smem + o);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const uint2 v = wp[i];
+      w[2 * i] = v.x;
+      w[2 * i + 1] = v.y;
+    }
+    w[8] = *reinterpret_cast<const uint32_t *>(smem + o + 32);
+  } else {
+    w[0] = *reinterpret_cast<const uint32_t *>(smem + o);
+    const uint2 *wp = reinterpret_cast<const uint2 *>(smem + o + 4);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const uint2 v = wp[i];
+      w[1 + 2 * i] = v.x;
+      w[2 + 2 * i] = v.y;
+    }
+  }
+  w[9] = 0u;
+  split_blk2(w, b0, b1);
+}
+
+// One block of a gate row and its up row against NT tokens' staged activations (the
+// activation words of block b are swizzled by sw).
 template <int NT>
-__device__ __forceinline__ void gu_row_block(const Blk &bk, int b, const uint16_t *xs, const ActBlk *ss,
-                                             const uint32_t (&xo)[NT], const uint32_t (&so)[NT], float (&y)[NT]) {
-  int al[NT], ah[NT];
+__device__ __forceinline__ void gu_pair_block(const Blk &bg, const Blk &bu, int b, int sw, const uint16_t *xs,
+                                              const ActBlk *ss, const uint32_t (&xo)[NT], const uint32_t (&so)[NT],
+                                              float (&yg)[NT], float (&yu)[NT]) {
+  int gl[NT], gh[NT], ul[NT], uh[NT];
   float sc[NT];
 #pragma unroll
   for (int i = 0; i < NT; ++i) {
     const ActBlk ab = ss[so[i] + b];
-    al[i] = ab.neg8sum;
-    ah[i] = 0;
+    gl[i] = ab.neg8sum;
+    ul[i] = ab.neg8sum;
+    gh[i] = 0;
+    uh[i] = 0;
     sc[i] = ab.scale;
   }
 #pragma unroll
   for (int wi = 0; wi < 4; ++wi) {
-    const uint32_t lo = bk.q[wi] & 0x0F0F0F0Fu, hi = bk.q[wi] & 0xF0F0F0F0u;
+    const uint32_t glo = bg.q[wi] & 0x0F0F0F0Fu, ghi = bg.q[wi] & 0xF0F0F0F0u;
+    const uint32_t ulo = bu.q[wi] & 0x0F0F0F0Fu, uhi = bu.q[wi] & 0xF0F0F0F0u;
 #pragma unroll
-    for (int i = 0; i < NT; ++i)
-      dot8i(lo, hi, *reinterpret_cast<const uint4 *>(xs + xo[i] + b * MOE_QK + 8 * wi), al[i], ah[i]);
+    for (int i = 0; i < NT; ++i) {
+      const uint4 xv = *reinterpret_cast<const uint4 *>(xs + xo[i] + b * MOE_QK + 8 * (wi ^ sw));
+      dot8i(glo, ghi, xv, gl[i], gh[i]);
+      dot8i(ulo, uhi, xv, ul[i], uh[i]);
+    }
   }
 #pragma unroll
-  for (int i = 0; i < NT; ++i) y[i] = block_finish(y[i], bk.d, sc[i], al[i], ah[i]);
+  for (int i = 0; i < NT; ++i) {
+    yg[i] = block_finish(yg[i], bg.d, sc[i], gl[i], gh[i]);
+    yu[i] = block_finish(yu[i], bu.d, sc[i], ul[i], uh[i]);
+  }
 }
 
 // gate_up pass over one staged chunk (kPairs row pairs) for NT tokens, by the compute warps.
-// Work item = (granule, gate or up); lane = (row pair p, half h) covering blocks
-// 8 granule + 4 h .. + 3. The halves are combined by a shuffle;
-// red_b[(item * kPairs + p) * kTX + i] gets the partial.
+// Work item = (granule g, piece parity hp), 2 G items; lane = (row pair p, s): the lane
+// multiplies the gate and the up row of pair p over blocks 8 g + 4 s + 2 hp and the next
+// (a 2-block piece; pieces of one item share their offset mod 8 bytes). The two lanes of a
+// pair are combined by a shuffle; red_b[((item * kPairs + p) * kTX + i) * 2 + {0, 1}] gets the
+// gate and up partials. Activation words of blocks with (b >> 2) & 1 = 1 are stored swapped
+// in pairs, so the two halves of the warp read different banks.
 template <int NT, bool ALIGNED>
 __device__ __forceinline__ void gu_pass(const uint8_t *st, uint32_t rb, int nb, int n_items, int nwc, int d,
                                         const uint16_t *xs, const ActBlk *ss, const int32_t *ptok, float *red_b) {
   const int lane = threadIdx.x & 31;
-  const int p = lane >> 1, h = lane & 1;
+  const int p = lane >> 1, sl = lane & 1;
   uint32_t xo[NT], so[NT];
 #pragma unroll
   for (int i = 0; i < NT; ++i) {
@@ -226,37 +288,36 @@ __device__ __forceinline__ void gu_pass(const uint8_t *st, uint32_t rb, int nb, 
     so[i] = (uint32_t)(t * nb);
   }
   for (int item = threadIdx.x >> 5; item < n_items; item += nwc) {
-    const int gran = item >> 1, type = item & 1;
-    const int b0 = gran * kGran + h * 4;
-    const uint32_t o = (uint32_t)(type * kPairs + p) * rb + (uint32_t)b0 * MOE_QBYTES;
-    float y[NT];
+    const int gran = item >> 1, hp = item & 1;
+    const int b0 = gran * kGran + sl * 4 + hp * 2;
+    const uint32_t og = (uint32_t)p * rb + (uint32_t)b0 * MOE_QBYTES;
+    const uint32_t ou = og + (uint32_t)kPairs * rb;
+    float yg[NT], yu[NT];
 #pragma unroll
-    for (int i = 0; i < NT; ++i) y[i] = 0.f;
+    for (int i = 0; i < NT; ++i) { yg[i] = 0.f; yu[i] = 0.f; }
     if (ALIGNED) {
-      {
-        Blk k0, k1;
-        load_blk2_lo(st, o, k0, k1);
-        gu_row_block<NT>(k0, b0, xs, ss, xo, so, y);
-        gu_row_block<NT>(k1, b0 + 1, xs, ss, xo, so, y);
+      Blk g0, g1, u0, u1;
+      if (hp == 0) {
+        load_span2<false>(st, og, g0, g1);
+        load_span2<false>(st, ou, u0, u1);
+      } else {
+        load_span2<true>(st, og, g0, g1);
+        load_span2<true>(st, ou, u0, u1);
       }
-      {
-        Blk k2, k3;
-        load_blk2_hi(st, o, k2, k3);
-        gu_row_block<NT>(k2, b0 + 2, xs, ss, xo, so, y);
-        gu_row_block<NT>(k3, b0 + 3, xs, ss, xo, so, y);
-      }
+      gu_pair_block<NT>(g0, u0, b0, sl, xs, ss, xo, so, yg, yu);
+      gu_pair_block<NT>(g1, u1, b0 + 1, sl, xs, ss, xo, so, yg, yu);
     } else {
-      int nbl = nb - b0;
-      nbl = nbl < 0 ? 0 : (nbl > 4 ? 4 : nbl);
-      for (int j = 0; j < nbl; ++j) {
-        const Blk kb = load_blk(st, o + (uint32_t)j * MOE_QBYTES);
-        gu_row_block<NT>(kb, b0 + j, xs, ss, xo, so, y);
+      for (int j = 0; j < 2 && b0 + j < nb; ++j) {
+        const Blk bg = load_blk(st, og + (uint32_t)j * MOE_QBYTES);
+        const Blk bu = load_blk(st, ou + (uint32_t)j * MOE_QBYTES);
+        gu_pair_block<NT>(bg, bu, b0 + j, sl, xs, ss, xo, so, yg, yu);
       }
     }
 #pragma unroll
     for (int i = 0; i < NT; ++i) {
-      const float yy = y[i] + __shfl_xor_sync(0xffffffffu, y[i], 1);
-      if (h == 0) red_b[((size_t)item * kPairs + p) * kTX + i] = yy;
+      const float g = yg[i] + __shfl_xor_sync(0xffffffffu, yg[i], 1);
+      const float u = yu[i] + __shfl_xor_sync(0xffffffffu, yu[i], 1);
+      if (sl == 0) *reinterpret_cast<float2 *>(red_b + (((size_t)item * kPairs + p) * kTX + i) * 2) = make_float2(g, u);
     }
   }
 }
@@ -307,7 +368,7 @@ __device__ __forceinline__ void dn_pass(const uint8_t *st, uint32_t rb, int nbf,
   for (int i = 0; i < NT; ++i) red_b[((size_t)part * kTX + i) * kDnRows + row] = y[i];
 }
 
-__global__ void __launch_bounds__((kFMaxCompute + 1) * 32, 1)
+__global__ void __launch_bounds__((kFMaxCompute + 2) * 32, 1)
 k_moe_decode(const __nv_bfloat16 *__restrict__ x, const float *__restrict__ router_w,
              const float *__restrict__ router_scale, const uint8_t *__restrict__ gate_up_q4,
              const uint8_t *__restrict__ down_q4, const float *__restrict__ expert_scale, int T, int d, int f,
@@ -316,7 +377,8 @@ k_moe_decode(const __nv_bfloat16 *__restrict__ x, const float *__restrict__ rout
   extern __shared__ __align__(128) uint8_t smem_raw[];
   __shared__ FusedShared sh;
   const int tid = threadIdx.x, lane = tid & 31, wq = tid >> 5, nw = blockDim.x >> 5;
-  const int nwc = nw - 1, nct = nwc * 32;   // compute warps 0 .. nwc-1; warp nwc produces
+  const int nwc = nw - 2, nct = nwc * 32;   // compute warps 0 .. nwc-1; warp nwc produces, nwc+1 epilogues
+  const int nteam = nct + 32;
   const int nb = d / MOE_QK, nbf = f / MOE_QK;
   const int G = (nb + kGran - 1) / kGran;
   const int P = nwc / kDnGroups;
@@ -334,9 +396,10 @@ k_moe_decode(const __nv_bfloat16 *__restrict__ x, const float *__restrict__ rout
   if (tid == 0) {
     for (int s = 0; s < kFStages; ++s) {
       mbar_init(&sh.full[s], 1);
-      mbar_init(&sh.empty[s], 1);
+      mbar_init(&sh.empty[s], nwc);
     }
     fence_mbar_init();
+    sh.abort = 0;
   }
   const float rs = __ldg(router_scale);
 
@@ -401,7 +464,7 @@ k_moe_decode(const __nv_bfloat16 *__restrict__ x, const float *__restrict__ rout
 #pragma unroll
         for (int r = 0; r < 8; ++r) v[r] = 0.f;
       }
-      stage_block_q(v, valid, xs + (size_t)t * d + (size_t)b * MOE_QK, ss + (size_t)t * nb + b);
+      stage_block_q(v, valid, (b >> 2) & 1, xs + (size_t)t * d + (size_t)b * MOE_QK, ss + (size_t)t * nb + b);
     }
   }
   if (tid == 0) sh.ok = grid_wait(W.gbar, target, W.err, 20) ? 1 : 0;
@@ -502,7 +565,7 @@ k_moe_decode(const __nv_bfloat16 *__restrict__ x, const float *__restrict__ rout
       for (int it = 0; u < n_units; ++it) {
         const int slot = it % kFStages;
         if (it >= kFStages &&
-            !mbar_wait(&sh.empty[slot], (uint32_t)(it / kFStages - 1) & 1u, W.err, 24))
+            !wait_phase(&sh.empty[slot], (uint32_t)(it / kFStages - 1) & 1u, &sh.abort, W.err, 24))
           break;
         const FChunk c = seq.at(u);
         const int e = sh.act[c.a];
@@ -524,7 +587,7 @@ k_moe_decode(const __nv_bfloat16 *__restrict__ x, const float *__restrict__ rout
     return;
   }
 
-  if (blockIdx.x == 0) {   // routing copies for the debug readers
+  if (blockIdx.x == 0 && wq < nwc) {   // routing copies for the debug readers
     for (int i = tid; i < S; i += nct) {
       W.ids[i] = sh.ids[i];
       W.w[i] = sh.w[i];
@@ -543,132 +606,158 @@ k_moe_decode(const __nv_bfloat16 *__restrict__ x, const float *__restrict__ rout
   }
 
   // ---------------------------------------------------------------- phases 2, 3: the GEMVs
+  // Compute warps multiply a staged chunk into one of two reduction buffers and move on; the
+  // epilogue warp turns a full buffer into h (GeGLU) or per-slot outputs and hands it back.
   const bool aligned = (nb % kGran) == 0;
   const int n_items = 2 * G;
-  const int lg = G <= 1 ? 1 : (G <= 2 ? 2 : (G <= 4 ? 4 : (G <= 8 ? 8 : 16)));   // lanes per epilogue item
   bool down_phase = false;
-  int hw0 = 0, hw1 = 0;   // sorted positions whose hidden vectors are staged in hs
   int pass = 0;
-  for (int u = 0, it = 0; u < n_units; ++it) {
-    const FChunk c = seq.at(u);
-    if (c.down && !down_phase) {
-      // all h written before any CTA reads it
-      if (!grid_barrier_c(W.gbar, W.err, 21, nct, sh.ok)) return;
-      down_phase = true;
-    }
-    const int slot = it % kFStages;
-    const uint32_t par = (uint32_t)(it / kFStages) & 1u;
-    const bool okw = mbar_wait(&sh.full[slot], par, W.err, 22);
-    if (named_sync_or(kBarCompute, nct, !okw)) return;
-    const int e = sh.act[c.a];
-    const int cnt = sh.counts[e];
-    const int off = sh.offsets[e];
-    const uint8_t *st = smem + (size_t)slot * stage_bytes;
-    if (!c.down) {
-      const int np = c.n * kUnit;
-      for (int g0 = 0; g0 < cnt; g0 += kTX) {
-        const int ng = min(kTX, cnt - g0);
-        float *red_b = red + (size_t)(pass & 1) * red_half;
-        ++pass;
-        const int32_t *pt = sh.ptok + off + g0;
-        if (aligned) {
-          switch (ng) {
-            case 1: gu_pass<1, true>(st, rb_g, nb, n_items, nwc, d, xs, ss, pt, red_b); break;
-            case 2: gu_pass<2, true>(st, rb_g, nb, n_items, nwc, d, xs, ss, pt, red_b); break;
-            case 3: gu_pass<3, true>(st, rb_g, nb, n_items, nwc, d, xs, ss, pt, red_b); break;
-            default: gu_pass<4, true>(st, rb_g, nb, n_items, nwc, d, xs, ss, pt, red_b); break;
-          }
-        } else {
-          switch (ng) {
-            case 1: gu_pass<1, false>(st, rb_g, nb, n_items, nwc, d, xs, ss, pt, red_b); break;
-            case 2: gu_pass<2, false>(st, rb_g, nb, n_items, nwc, d, xs, ss, pt, red_b); break;
-            case 3: gu_pass<3, false>(st, rb_g, nb, n_items, nwc, d, xs, ss, pt, red_b); break;
-            default: gu_pass<4, false>(st, rb_g, nb, n_items, nwc, d, xs, ss, pt, red_b); break;
-          }
-        }
-        named_sync(kBarCompute, nct);
-        if (g0 + kTX >= cnt && tid == 0) mbar_arrive(&sh.empty[slot]);   // last read of the stage
-        // h = gelu(gate) * up: lg lanes per (row pair, token), partials summed by a shuffle tree
-        const int per_warp = 32 / lg, n_it = np * ng;
-        for (int base = wq * per_warp; base < n_it; base += nwc * per_warp) {
-          const int itm = base + lane / lg, q = lane % lg;
-          const int i = itm / np, pp = itm - i * np;
-          float g = 0.f, uu = 0.f;
-          if (itm < n_it && q < G) {
-            g = red_b[((size_t)(2 * q) * kPairs + pp) * kTX + i];
-            uu = red_b[((size_t)(2 * q + 1) * kPairs + pp) * kTX + i];
-          }
-          for (int o = lg >> 1; o > 0; o >>= 1) {
-            g += __shfl_xor_sync(0xffffffffu, g, o);
-            uu += __shfl_xor_sync(0xffffffffu, uu, o);
-          }
-          if (q == 0 && itm < n_it)
-            W.h[(size_t)sh.perm[off + g0 + i] * f + c.r0 + pp] = gelu_tanh_f(g) * uu;
-        }
-        // no barrier: the next pass writes the other half of red
+  if (wq < nwc) {
+    int hw0 = 0, hw1 = 0;   // sorted positions whose hidden vectors are staged in hs
+    for (int u = 0, it = 0; u < n_units; ++it) {
+      const FChunk c = seq.at(u);
+      if (c.down && !down_phase) {
+        // all h written (the epilogue warp included) before any CTA reads it
+        grid_barrier_team(W.gbar, W.err, 21, nteam, &sh.abort);
+        down_phase = true;
       }
-    } else {
-      if (off < hw0 || off + cnt > hw1) {
-        // stage the hidden vectors of the slots from this expert on, up to the end of this
-        // CTA's last expert or the window's capacity
-        const int a_last = (seq.d1 - 1) / seq.upe_d;
-        const int e_last = sh.act[a_last];
-        hw0 = off;
-        hw1 = min(sh.offsets[e_last] + sh.counts[e_last], off + hcap);
-        const int ntask = (hw1 - hw0) * nbf * 4;
-        for (int base = wq * 32; base < ntask; base += nwc * 32) {
-          const int task = base + lane;
-          const bool valid = task < ntask;
-          const int blk = valid ? task >> 2 : 0, q = task & 3;
-          const int i = blk / nbf, cb = blk - i * nbf;
-          float v[8];
-          if (valid) {
-            const float4 *src =
-                reinterpret_cast<const float4 *>(W.h + (size_t)sh.perm[hw0 + i] * f + (size_t)cb * MOE_QK + 8 * q);
-            const float4 v0 = __ldcg(src), v1 = __ldcg(src + 1);
-            v[0] = v0.x; v[1] = v0.y; v[2] = v0.z; v[3] = v0.w;
-            v[4] = v1.x; v[5] = v1.y; v[6] = v1.z; v[7] = v1.w;
-          } else {
+      const int slot = it % kFStages;
+      const bool okw = wait_phase(&sh.full[slot], (uint32_t)(it / kFStages) & 1u, &sh.abort, W.err, 22);
+      const int e = sh.act[c.a];
+      const int cnt = sh.counts[e];
+      const int off = sh.offsets[e];
+      const uint8_t *st = smem + (size_t)slot * stage_bytes;
+      if (!c.down) {
+        for (int g0 = 0; g0 < cnt; g0 += kTXg, ++pass) {
+          const int ng = min(kTXg, cnt - g0);
+          const int b = pass & 1;
+          if (pass >= 2) named_sync(kBarEmpty0 + b, nteam);
+          float *red_b = red + (size_t)b * red_half;
+          const int32_t *pt = sh.ptok + off + g0;
+          if (okw) {
+            if (aligned) {
+              switch (ng) {
+                case 1: gu_pass<1, true>(st, rb_g, nb, n_items, nwc, d, xs, ss, pt, red_b); break;
+                case 2: gu_pass<2, true>(st, rb_g, nb, n_items, nwc, d, xs, ss, pt, red_b); break;
+                default: gu_pass<3, true>(st, rb_g, nb, n_items, nwc, d, xs, ss, pt, red_b); break;
+              }
+            } else {
+              switch (ng) {
+                case 1: gu_pass<1, false>(st, rb_g, nb, n_items, nwc, d, xs, ss, pt, red_b); break;
+                case 2: gu_pass<2, false>(st, rb_g, nb, n_items, nwc, d, xs, ss, pt, red_b); break;
+                default: gu_pass<3, false>(st, rb_g, nb, n_items, nwc, d, xs, ss, pt, red_b); break;
+              }
+            }
+          }
+          named_arrive(kBarFull0 + b, nteam);
+        }
+      } else {
+        if (off < hw0 || off + cnt > hw1) {
+          // stage the hidden vectors of the slots from this expert on, up to the end of this
+          // CTA's last expert or the window's capacity
+          named_sync(kBarCompute, nct);   // every compute warp is done with the previous window
+          const int a_last = (seq.d1 - 1) / seq.upe_d;
+          const int e_last = sh.act[a_last];
+          hw0 = off;
+          hw1 = min(sh.offsets[e_last] + sh.counts[e_last], off + hcap);
+          const int ntask = okw ? (hw1 - hw0) * nbf * 4 : 0;
+          for (int base = wq * 32; base < ntask; base += nwc * 32) {
+            const int task = base + lane;
+            const bool valid = task < ntask;
+            const int blk = valid ? task >> 2 : 0, q = task & 3;
+            const int i = blk / nbf, cb = blk - i * nbf;
+            float v[8];
+            if (valid) {
+              const float4 *src = reinterpret_cast<const float4 *>(W.h + (size_t)sh.perm[hw0 + i] * f +
+                                                                   (size_t)cb * MOE_QK + 8 * q);
+              const float4 v0 = __ldcg(src), v1 = __ldcg(src + 1);
+              v[0] = v0.x; v[1] = v0.y; v[2] = v0.z; v[3] = v0.w;
+              v[4] = v1.x; v[5] = v1.y; v[6] = v1.z; v[7] = v1.w;
+            } else {
 #pragma unroll
-            for (int r = 0; r < 8; ++r) v[r] = 0.f;
+              for (int r = 0; r < 8; ++r) v[r] = 0.f;
+            }
+            stage_block_q(v, valid, 0, hs + (size_t)i * f + (size_t)cb * MOE_QK, hbk + (size_t)i * nbf + cb);
           }
-          stage_block_q(v, valid, hs + (size_t)i * f + (size_t)cb * MOE_QK, hbk + (size_t)i * nbf + cb);
+          named_sync(kBarCompute, nct);
         }
-        named_sync(kBarCompute, nct);
-      }
-      const int nr = c.n * kUnit;
-      for (int g0 = 0; g0 < cnt; g0 += kTX) {
-        const int ng = min(kTX, cnt - g0);
-        float *red_b = red + (size_t)(pass & 1) * red_half;
-        ++pass;
-        const int rel0 = off + g0 - hw0;
-        switch (ng) {
-          case 1: dn_pass<1>(st, rb_d, nbf, P, nr, f, hs, hbk, rel0, red_b); break;
-          case 2: dn_pass<2>(st, rb_d, nbf, P, nr, f, hs, hbk, rel0, red_b); break;
-          case 3: dn_pass<3>(st, rb_d, nbf, P, nr, f, hs, hbk, rel0, red_b); break;
-          default: dn_pass<4>(st, rb_d, nbf, P, nr, f, hs, hbk, rel0, red_b); break;
-        }
-        named_sync(kBarCompute, nct);
-        if (g0 + kTX >= cnt && tid == 0) mbar_arrive(&sh.empty[slot]);   // last read of the stage
-        for (int i2 = tid; i2 < nr * ng; i2 += nct) {
-          const int i = i2 / nr, row = i2 - i * nr;
-          float s = 0.f;
-          for (int pt = 0; pt < P; ++pt) s += red_b[((size_t)pt * kTX + i) * kDnRows + row];
-          W.ybuf[(size_t)sh.perm[off + g0 + i] * d + c.r0 + row] = s;
+        const int nr = c.n * kUnit;
+        for (int g0 = 0; g0 < cnt; g0 += kTX, ++pass) {
+          const int ng = min(kTX, cnt - g0);
+          const int b = pass & 1;
+          if (pass >= 2) named_sync(kBarEmpty0 + b, nteam);
+          float *red_b = red + (size_t)b * red_half;
+          const int rel0 = off + g0 - hw0;
+          if (okw) {
+            switch (ng) {
+              case 1: dn_pass<1>(st, rb_d, nbf, P, nr, f, hs, hbk, rel0, red_b); break;
+              case 2: dn_pass<2>(st, rb_d, nbf, P, nr, f, hs, hbk, rel0, red_b); break;
+              case 3: dn_pass<3>(st, rb_d, nbf, P, nr, f, hs, hbk, rel0, red_b); break;
+              default: dn_pass<4>(st, rb_d, nbf, P, nr, f, hs, hbk, rel0, red_b); break;
+            }
+          }
+          named_arrive(kBarFull0 + b, nteam);
         }
       }
+      if (lane == 0) mbar_arrive(&sh.empty[slot]);   // this warp's last read of the stage
+      u += c.n;
     }
-    u += c.n;
-  }
-  if (!down_phase) {
-    // this CTA had no down rows: it still takes part in the h barrier
-    if (!grid_barrier_c(W.gbar, W.err, 21, nct, sh.ok)) return;
+    if (!down_phase) grid_barrier_team(W.gbar, W.err, 21, nteam, &sh.abort);   // no down rows here
+    for (int q = pass < 2 ? 0 : pass - 2; q < pass; ++q) named_sync(kBarEmpty0 + (q & 1), nteam);
+  } else {
+    // the epilogue warp: the same sequence of chunks and passes
+    for (int u = 0; u < n_units;) {
+      const FChunk c = seq.at(u);
+      if (c.down && !down_phase) {
+        grid_barrier_team(W.gbar, W.err, 21, nteam, &sh.abort);
+        down_phase = true;
+      }
+      const int e = sh.act[c.a];
+      const int cnt = sh.counts[e];
+      const int off = sh.offsets[e];
+      const int step = c.down ? kTX : kTXg;
+      for (int g0 = 0; g0 < cnt; g0 += step, ++pass) {
+        const int ng = min(step, cnt - g0);
+        const int b = pass & 1;
+        named_sync(kBarFull0 + b, nteam);
+        const float *red_b = red + (size_t)b * red_half;
+        if (!sh.abort) {
+          if (!c.down) {
+            // h = gelu(gate) * up; the partials of the 2 G work items summed in order
+            const int np = c.n * kUnit, sh_np = np == 16 ? 4 : 3;
+            for (int itm = lane; itm < np * ng; itm += 32) {
+              const int i = itm >> sh_np, pp = itm & (np - 1);
+              float g = 0.f, uu = 0.f;
+              for (int q = 0; q < n_items; ++q) {
+                const float2 v = *reinterpret_cast<const float2 *>(red_b + (((size_t)q * kPairs + pp) * kTX + i) * 2);
+                g += v.x;
+                uu += v.y;
+              }
+              W.h[(size_t)sh.perm[off + g0 + i] * f + c.r0 + pp] = gelu_tanh_f(g) * uu;
+            }
+          } else {
+            const int nr = c.n * kUnit;
+            for (int i2 = lane; i2 < nr * ng; i2 += 32) {
+              const int i = i2 / nr, row = i2 - i * nr;
+              float s = 0.f;
+              for (int pt = 0; pt < P; ++pt) s += red_b[((size_t)pt * kTX + i) * kDnRows + row];
+              W.ybuf[(size_t)sh.perm[off + g0 + i] * d + c.r0 + row] = s;
+            }
+          }
+        }
+        named_arrive(kBarEmpty0 + b, nteam);
+      }
+      u += c.n;
+    }
+    if (!down_phase) grid_barrier_team(W.gbar, W.err, 21, nteam, &sh.abort);
   }
   // ---------------------------------------------------------------- phase 4: combine
-  if (!grid_barrier_c(W.gbar, W.err, 23, nct, sh.ok)) return;
+  grid_barrier_team(W.gbar, W.err, 23, nteam, &sh.abort);
+  if (sh.abort) return;
+  const int ti = wq < nwc ? tid : nct + lane;
   const int r0 = (int)((long long)d * blockIdx.x / gridDim.x), r1 = (int)((long long)d * (blockIdx.x + 1) / gridDim.x);
   const int nr = r1 - r0;
-  for (int i2 = tid; i2 < nr * T; i2 += nct) {
+  for (int i2 = ti; i2 < nr * T; i2 += nteam) {
     const int t = i2 / nr, r = r0 + i2 % nr;
     float s = 0.f;
     for (int j = 0; j < k; ++j) {
@@ -696,7 +785,7 @@ static FusedSmem fused_smem(int T, int d, int f) {
   r.stage_bytes = (uint32_t)(((sg > sd ? sg : sd) + 15u) & ~(size_t)15u);
   const size_t xg = (size_t)T * (2 * d + 8 * nb), xh = (size_t)T * (2 * f + 8 * nbf);
   r.x_bytes = (uint32_t)(((xg > xh ? xg : xh) + 15u) & ~(size_t)15u);
-  const size_t rg = (size_t)2 * G * kPairs * kTX, rd = (size_t)P * kTX * kDnRows;
+  const size_t rg = (size_t)2 * G * kPairs * kTX * 2, rd = (size_t)P * kTX * kDnRows;
   r.red_half = (uint32_t)(rg > rd ? rg : rd);
   r.total = (size_t)kFStages * r.stage_bytes + r.x_bytes + (size_t)2 * r.red_half * 4 + 128;
   return r;
@@ -724,7 +813,7 @@ int moe_launch_fused_decode(const MoeLaunch &L, const MoeWork &W, const void *x,
   const int G = (d / MOE_QK + kGran - 1) / kGran;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(num_sms);
-  cfg.blockDim = dim3(32 * (fused_compute_warps(G) + 1));
+  cfg.blockDim = dim3(32 * (fused_compute_warps(G) + 2));
   cfg.dynamicSmemBytes = fs.total;
   cfg.stream = L.stream;
   cudaLaunchAttribute attr[1];
