@@ -137,6 +137,40 @@ def flops_bytes(lw: mi.LayerWeights, T: int, k: int, counts: np.ndarray):
             "flops": flops}
 
 
+def sources_sha256() -> str:
+    """Hash of the CUDA sources; a recorded ncu traffic figure is valid only for this hash."""
+    import glob
+    import hashlib
+    h = hashlib.sha256()
+    for p in sorted(glob.glob(os.path.join(ROOT, "mixture_experts_gemv_b200", "csrc", "*"))):
+        with open(p, "rb") as fh:
+            h.update(os.path.basename(p).encode() + b"\0" + fh.read())
+    return h.hexdigest()
+
+
+def recorded_traffic(kernel: str, workload: str, units_per_launch: float):
+    """DRAM bytes (read + write) per launch of `kernel` from the ncu summary in profiles/,
+    scaled to this launch's units when the capture ran a smaller case; None when no summary
+    exists or the sources changed since it was captured."""
+    path = os.path.join(ROOT, "profiles", f"{kernel}_{workload}.md")
+    if not os.path.exists(path):
+        return None
+    fields = {}
+    with open(path) as fh:
+        for ln in fh:
+            if ln.startswith("- ") and ":" in ln:
+                key, _, val = ln[2:].partition(":")
+                fields[key.strip()] = val.strip().strip("`")
+    try:
+        if fields.get("sources_sha256") != sources_sha256():
+            return None
+        traffic = float(fields["dram_bytes_per_launch"])
+        units = float(fields.get("units_per_launch", units_per_launch))
+        return traffic * units_per_launch / units
+    except (KeyError, ValueError):
+        return None
+
+
 def dist_env():
     ws = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
@@ -374,26 +408,41 @@ def main():
     e2e_value = ws * tokens_per_step * args.steps / (ms_e2e / 1e3)
     avg = {kk: float(np.mean([w[kk] for w in work])) for kk in work[0]}
     n_layers_per_step = len(layers) if stack else 1
-    if T <= 16:
+    if T <= 16 and "fused_decode" in prof:
+        # the whole layer is one kernel: its algorithmic bytes are the active experts' Q4_0
+        # weights, the router weights, x, out and the scales
+        kms, nl = prof["fused_decode"]
+        per_launch_bytes = (avg["gateup_weight_bytes"] + avg["down_weight_bytes"] + avg["router_bytes"] +
+                            avg["act_bytes"] + 4 * (E + 1))
+        achieved = per_launch_bytes / (kms / nl / 1e3) / 1e9
+        roof = {"kernel": "k_moe_decode", "bound": "hbm", "achieved": achieved, "peak": pk["hbm_gbs"],
+                "unit": "GB/s", "frac": achieved / pk["hbm_gbs"],
+                "traffic": recorded_traffic("k_moe_decode", wl_name, per_launch_bytes),
+                "peak_source": pk["source"] + " (hbm_gbs, copy bandwidth)",
+                "bytes_per_launch": per_launch_bytes, "ms_per_launch": kms / nl}
+        dtype = "int16xq4->int32, f32"
+    elif T <= 16:
         name = "gateup_gemv"
         kms, nl = prof.get(name, (float("nan"), 1))
         per_launch_bytes = avg["gateup_weight_bytes"] + T * d * 4 + T * k * f * 8
         achieved = per_launch_bytes / (kms / nl / 1e3) / 1e9
         roof = {"kernel": "k_gateup_gemv", "bound": "hbm", "achieved": achieved, "peak": pk["hbm_gbs"],
-                "unit": "GB/s", "frac": achieved / pk["hbm_gbs"], "traffic": None,
+                "unit": "GB/s", "frac": achieved / pk["hbm_gbs"],
+                "traffic": recorded_traffic("k_gateup_gemv", wl_name, per_launch_bytes),
                 "peak_source": pk["source"] + " (hbm_gbs, copy bandwidth)",
                 "bytes_per_launch": per_launch_bytes, "ms_per_launch": kms / nl}
-        dtype = "f32"
+        dtype = "int16xq4->int32, f32"
     else:
         name = "gateup_gemm" if "gateup_gemm" in prof else "gateup_gemv"
         kms, nl = prof.get(name, (float("nan"), 1))
         fl = 2 * T * k * 2 * f * d
         achieved = fl / (kms / nl / 1e3) / 1e12
         roof = {"kernel": name, "bound": "tensor", "achieved": achieved, "peak": pk["bf16_tflops"],
-                "unit": "TFLOP/s", "frac": achieved / pk["bf16_tflops"], "traffic": None,
+                "unit": "TFLOP/s", "frac": achieved / pk["bf16_tflops"],
+                "traffic": recorded_traffic("k_moe_gemm" if name == "gateup_gemm" else "k_gateup_gemv", wl_name, fl),
                 "peak_source": pk["source"] + " (bf16_tflops, burst)", "flops_per_launch": fl,
                 "ms_per_launch": kms / nl}
-        dtype = "bf16" if name == "gateup_gemm" else "f32"
+        dtype = "bf16" if name == "gateup_gemm" else "int16xq4->int32, f32"
     launches_per_step = sum(n for (_, n) in prof.values()) / args.steps
     step_gbs = avg["total_bytes"] * n_layers_per_step / (ms_step / 1e3) / 1e9
 

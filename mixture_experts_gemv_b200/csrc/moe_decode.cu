@@ -442,29 +442,41 @@ k_moe_decode(const __nv_bfloat16 *__restrict__ x, const float *__restrict__ rout
     __syncthreads();
   }
   // arrive; stage every token's activations while the other CTAs finish their logits
+  __syncthreads();
   unsigned long long target = 0;
   if (tid == 0) target = grid_arrive(W.gbar);
   {
-    const int ntask = T * nb * 4;
-    for (int base = wq * 32; base < ntask; base += nw * 32) {
-      const int task = base + lane;
-      const bool valid = task < ntask;
-      const int blk = valid ? task >> 2 : 0, q = task & 3;
-      const int t = blk / nb, b = blk - t * nb;
-      float v[8];
-      if (valid) {
-        const uint4 u = __ldg(reinterpret_cast<const uint4 *>(x + (size_t)t * d + (size_t)b * MOE_QK + 8 * q));
-        const uint32_t uu[4] = {u.x, u.y, u.z, u.w};
+    // four (token, block, quarter) tasks per thread: all loads first, then the conversions
+    const int ntask = T * nb * 4, stride = nw * 32;
+    for (int base = wq * 32; base < ntask; base += 4 * stride) {
+      uint4 raw[4];
 #pragma unroll
-        for (int r = 0; r < 4; ++r) {
-          v[2 * r] = __uint_as_float(uu[r] << 16);
-          v[2 * r + 1] = __uint_as_float(uu[r] & 0xffff0000u);
+      for (int r = 0; r < 4; ++r) {
+        const int task = base + r * stride + lane;
+        if (task < ntask) {
+          const int blk = task >> 2, q = task & 3;
+          const int t = blk / nb, b = blk - t * nb;
+          raw[r] = __ldg(reinterpret_cast<const uint4 *>(x + (size_t)t * d + (size_t)b * MOE_QK + 8 * q));
+        } else {
+          raw[r] = make_uint4(0u, 0u, 0u, 0u);
         }
-      } else {
-#pragma unroll
-        for (int r = 0; r < 8; ++r) v[r] = 0.f;
       }
-      stage_block_q(v, valid, (b >> 2) & 1, xs + (size_t)t * d + (size_t)b * MOE_QK, ss + (size_t)t * nb + b);
+#pragma unroll
+      for (int r = 0; r < 4; ++r) {
+        if (base + r * stride >= ntask) break;   // warp-uniform
+        const int task = base + r * stride + lane;
+        const bool valid = task < ntask;
+        const int blk = valid ? task >> 2 : 0;
+        const int t = blk / nb, b = blk - t * nb;
+        const uint32_t uu[4] = {raw[r].x, raw[r].y, raw[r].z, raw[r].w};
+        float v[8];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          v[2 * i] = __uint_as_float(uu[i] << 16);
+          v[2 * i + 1] = __uint_as_float(uu[i] & 0xffff0000u);
+        }
+        stage_block_q(v, valid, (b >> 2) & 1, xs + (size_t)t * d + (size_t)b * MOE_QK, ss + (size_t)t * nb + b);
+      }
     }
   }
   if (tid == 0) sh.ok = grid_wait(W.gbar, target, W.err, 20) ? 1 : 0;
@@ -660,24 +672,35 @@ k_moe_decode(const __nv_bfloat16 *__restrict__ x, const float *__restrict__ rout
           const int e_last = sh.act[a_last];
           hw0 = off;
           hw1 = min(sh.offsets[e_last] + sh.counts[e_last], off + hcap);
-          const int ntask = okw ? (hw1 - hw0) * nbf * 4 : 0;
-          for (int base = wq * 32; base < ntask; base += nwc * 32) {
-            const int task = base + lane;
-            const bool valid = task < ntask;
-            const int blk = valid ? task >> 2 : 0, q = task & 3;
-            const int i = blk / nbf, cb = blk - i * nbf;
-            float v[8];
-            if (valid) {
-              const float4 *src = reinterpret_cast<const float4 *>(W.h + (size_t)sh.perm[hw0 + i] * f +
-                                                                   (size_t)cb * MOE_QK + 8 * q);
-              const float4 v0 = __ldcg(src), v1 = __ldcg(src + 1);
-              v[0] = v0.x; v[1] = v0.y; v[2] = v0.z; v[3] = v0.w;
-              v[4] = v1.x; v[5] = v1.y; v[6] = v1.z; v[7] = v1.w;
-            } else {
+          const int ntask = okw ? (hw1 - hw0) * nbf * 4 : 0, stride = nwc * 32;
+          for (int base = wq * 32; base < ntask; base += 2 * stride) {
+            float4 raw[2][2];
 #pragma unroll
-              for (int r = 0; r < 8; ++r) v[r] = 0.f;
+            for (int r = 0; r < 2; ++r) {
+              const int task = base + r * stride + lane;
+              if (task < ntask) {
+                const int blk = task >> 2, q = task & 3;
+                const int i = blk / nbf, cb = blk - i * nbf;
+                const float4 *src = reinterpret_cast<const float4 *>(W.h + (size_t)sh.perm[hw0 + i] * f +
+                                                                     (size_t)cb * MOE_QK + 8 * q);
+                raw[r][0] = __ldcg(src);
+                raw[r][1] = __ldcg(src + 1);
+              } else {
+                raw[r][0] = make_float4(0.f, 0.f, 0.f, 0.f);
+                raw[r][1] = raw[r][0];
+              }
             }
-            stage_block_q(v, valid, 0, hs + (size_t)i * f + (size_t)cb * MOE_QK, hbk + (size_t)i * nbf + cb);
+#pragma unroll
+            for (int r = 0; r < 2; ++r) {
+              if (base + r * stride >= ntask) break;   // warp-uniform
+              const int task = base + r * stride + lane;
+              const bool valid = task < ntask;
+              const int blk = valid ? task >> 2 : 0;
+              const int i = blk / nbf, cb = blk - i * nbf;
+              const float v[8] = {raw[r][0].x, raw[r][0].y, raw[r][0].z, raw[r][0].w,
+                                  raw[r][1].x, raw[r][1].y, raw[r][1].z, raw[r][1].w};
+              stage_block_q(v, valid, 0, hs + (size_t)i * f + (size_t)cb * MOE_QK, hbk + (size_t)i * nbf + cb);
+            }
           }
           named_sync(kBarCompute, nct);
         }
