@@ -28,9 +28,10 @@ constexpr int kFMaxT = 8;          // tokens per call on the fused path
 constexpr int kFMaxSlots = 128;    // T * k
 constexpr int kFMaxE = 256;
 constexpr int kFStages = 3;
-constexpr int kFMaxCompute = 22;   // compute warps (one more warp produces)
+constexpr int kFMaxCompute = 12;   // compute warps (128 registers a thread)
 constexpr int kFMinCompute = 8;
 constexpr int kDnGroups = kDnRows / 32;   // 32-row groups of a down chunk
+constexpr int kDnParts = 5;               // parts of a down row's blocks (work items: groups x parts)
 // Named barriers (0 is __syncthreads): compute warps only; FULL / EMPTY of the two reduction
 // buffers between the compute warps and the epilogue warp; compute + epilogue warps.
 constexpr int kBarCompute = 1;
@@ -42,10 +43,10 @@ constexpr int kTXg = 3;                   // tokens per gate_up pass (register b
 // the tokens, the multiply-adds are per token.
 constexpr int kUnitDecode = 5, kUnitToken = 4;
 
-// Compute warps per CTA: one per gate_up work item (2 per granule), at least enough for the
-// down row groups. Two more warps: the producer and the epilogue warp.
+// Compute warps per CTA: one per gate_up work item (a granule), at least kFMinCompute. Two
+// more warps: the producer and the epilogue warp.
 __host__ __device__ inline int fused_compute_warps(int G) {
-  const int w = 2 * G;
+  const int w = G;
   return w < kFMinCompute ? kFMinCompute : (w > kFMaxCompute ? kFMaxCompute : w);
 }
 
@@ -139,70 +140,68 @@ struct FChunk {
   int a, r0, n;
 };
 
-// The CTA's chunk sequence: its gate_up units (chunks of up to 2 units of 8 row pairs inside
-// one expert), then its down units (chunks of up to 16 units of 8 rows inside one expert).
-struct FSeq {
-  int g0, g1, d0, d1, upe_g, upe_d;
-  __device__ FChunk at(int u) const {   // u: position in the concatenated unit sequence
+// The CTA's chunk sequence: its gate_up units [seq[0], seq[1]) (chunks of up to 2 units of 8
+// row pairs inside one expert), then its down units [seq[2], seq[3]) (chunks of up to 16 units
+// of 8 rows inside one expert), walked without a division per chunk.
+struct FWalk {
+  int down, a, r, left;    // phase, active-expert index, unit within the expert, units left in the phase
+  __device__ void start(int u0, int u1, int upe, int dn) {
+    down = dn;
+    a = u0 / upe;
+    r = u0 - a * upe;
+    left = u1 - u0;
+  }
+  __device__ void init(const int *seq, int upe_g, int upe_d) {
+    start(seq[0], seq[1], upe_g, 0);
+    if (left == 0) start(seq[2], seq[3], upe_d, 1);
+  }
+  __device__ bool done() const { return down && left == 0; }
+  __device__ FChunk cur(int upe_g, int upe_d) const {
     FChunk c;
-    if (u < g1 - g0) {
-      const int v = g0 + u;
-      c.down = 0;
-      c.a = v / upe_g;
-      const int r = v - c.a * upe_g;
-      c.r0 = r * kUnit;
-      c.n = (v + 1 < g1 && r + 1 < upe_g) ? 2 : 1;
-    } else {
-      const int v = d0 + (u - (g1 - g0));
-      c.down = 1;
-      c.a = v / upe_d;
-      const int r = v - c.a * upe_d;
-      c.r0 = r * kUnit;
-      c.n = min(kDnRows / kUnit, min(d1 - v, upe_d - r));
-    }
+    c.down = down;
+    c.a = a;
+    c.r0 = r * kUnit;
+    c.n = down ? min(kDnRows / kUnit, min(left, upe_d - r)) : ((left >= 2 && r + 1 < upe_g) ? 2 : 1);
     return c;
   }
-  __device__ int total() const { return (g1 - g0) + (d1 - d0); }
+  __device__ void advance(int n, const int *seq, int upe_g, int upe_d) {
+    left -= n;
+    r += n;
+    if (r == (down ? upe_d : upe_g)) {
+      ++a;
+      r = 0;
+    }
+    if (!down && left == 0) start(seq[2], seq[3], upe_d, 1);
+  }
 };
 
-// Four consecutive lanes turn one 32-wide block into block-scaled int16 in the GEMV word
-// order (moe_common.cuh): lane q = lane & 3 holds elements 8q .. 8q+7 in v[], which go to
-// positions p1 .. p1+3 and p1+8 .. p1+11, p1 = 16 (q & 1) + 4 (q >> 1). With sw = 1 the
-// block's 16-byte words are stored swapped in pairs (word w at w ^ 1). The block's ActBlk
-// goes to *blk_s. Every lane of the warp calls.
-__device__ __forceinline__ void stage_block_q(const float (&v)[8], bool valid, int sw, uint16_t *blk16,
-                                              ActBlk *blk_s) {
-  const int q = threadIdx.x & 3;
+// One thread turns one 32-wide block v[] into block-scaled int16 in the GEMV word order
+// (moe_common.cuh); with sw = 1 the block's 16-byte words are stored swapped in pairs (word w
+// at w ^ 1). The block's ActBlk goes to *blk_s.
+__device__ __forceinline__ void stage_block_t(const float (&v)[MOE_QK], int sw, uint16_t *blk16, ActBlk *blk_s) {
   float m = 0.f;
   bool finite = true;
 #pragma unroll
-  for (int r = 0; r < 8; ++r) {
-    m = fmaxf(m, fabsf(v[r]));
-    finite = finite && isfinite(v[r]);
+  for (int i = 0; i < MOE_QK; ++i) {
+    m = fmaxf(m, fabsf(v[i]));
+    finite = finite && isfinite(v[i]);
   }
-  m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 1));
-  m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 2));
-  int fin = finite ? 1 : 0;
-  fin &= __shfl_xor_sync(0xffffffffu, fin, 1);
-  fin &= __shfl_xor_sync(0xffffffffu, fin, 2);
   const BlockScale bs = block_scale_for_max(m);
-  uint32_t pk[4];
   int s = 0;
 #pragma unroll
-  for (int r = 0; r < 8; r += 2) {
-    const int a0 = act_to_i16(v[r], bs.scale), a1 = act_to_i16(v[r + 1], bs.scale);
-    s += a0 + a1;
-    pk[r >> 1] = ((uint32_t)a0 & 0xffffu) | ((uint32_t)a1 << 16);
+  for (int wi = 0; wi < 4; ++wi) {
+    // word wi: elements 4wi..4wi+3 (low nibbles), then 16+4wi..16+4wi+3 (high nibbles)
+    uint32_t pk[4];
+#pragma unroll
+    for (int h = 0; h < 4; ++h) {
+      const int e0 = h < 2 ? 4 * wi + 2 * h : 16 + 4 * wi + 2 * (h - 2);
+      const int a0 = act_to_i16(v[e0], bs.scale), a1 = act_to_i16(v[e0 + 1], bs.scale);
+      s += a0 + a1;
+      pk[h] = ((uint32_t)a0 & 0xffffu) | ((uint32_t)a1 << 16);
+    }
+    *reinterpret_cast<uint4 *>(blk16 + 8 * (wi ^ sw)) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
   }
-  s += __shfl_xor_sync(0xffffffffu, s, 1);
-  s += __shfl_xor_sync(0xffffffffu, s, 2);
-  if (valid) {
-    const int p1 = 16 * (q & 1) + 4 * (q >> 1);
-    const int wa = (p1 >> 3) ^ sw, wb = ((p1 >> 3) + 1) ^ sw;
-    *reinterpret_cast<uint2 *>(blk16 + 8 * wa + (p1 & 7)) = make_uint2(pk[0], pk[1]);
-    *reinterpret_cast<uint2 *>(blk16 + 8 * wb + (p1 & 7)) = make_uint2(pk[2], pk[3]);
-    if (q == 0) *blk_s = ActBlk{-8 * s, fin ? bs.inv : __int_as_float(0x7fffffff)};
-  }
+  *blk_s = ActBlk{-8 * s, finite ? bs.inv : __int_as_float(0x7fffffff)};
 }
 
 // Two consecutive Q4_0 blocks (36 bytes) of a row at a shared-memory byte offset o that is
@@ -268,16 +267,17 @@ __device__ __forceinline__ void gu_pair_block(const Blk &bg, const Blk &bu, int 
   }
 }
 
-// gate_up pass over one staged chunk (kPairs row pairs) for NT tokens, by the compute warps.
-// Work item = (granule g, piece parity hp), 2 G items; lane = (row pair p, s): the lane
-// multiplies the gate and the up row of pair p over blocks 8 g + 4 s + 2 hp and the next
-// (a 2-block piece; pieces of one item share their offset mod 8 bytes). The two lanes of a
-// pair are combined by a shuffle; red_b[((item * kPairs + p) * kTX + i) * 2 + {0, 1}] gets the
-// gate and up partials. Activation words of blocks with (b >> 2) & 1 = 1 are stored swapped
-// in pairs, so the two halves of the warp read different banks.
+// gate_up pass over one staged chunk (kPairs row pairs) for NT tokens, by the compute warps:
+// items first, first + nwc, ... Work item = granule g (G items); lane = (row pair p, s): the
+// lane multiplies the gate and the up row of pair p over blocks 8 g + 4 s .. + 3, read as two
+// 2-block spans (the first 8-byte aligned, the second 4 bytes past). The two lanes of a pair
+// are combined by a shuffle; red_b[((g * kTX + i) * kPairs + p) * 2 + {0, 1}] gets the gate
+// and up partials. Activation words of blocks with (b >> 2) & 1 = 1 are stored swapped in
+// pairs, so the two halves of the warp read different banks.
 template <int NT, bool ALIGNED>
-__device__ __forceinline__ void gu_pass(const uint8_t *st, uint32_t rb, int nb, int n_items, int nwc, int d,
-                                        const uint16_t *xs, const ActBlk *ss, const int32_t *ptok, float *red_b) {
+__device__ __forceinline__ void gu_pass(const uint8_t *st, uint32_t rb, int nb, int n_items, int nwc, int first,
+                                        int d, const uint16_t *xs, const ActBlk *ss, const int32_t *ptok,
+                                        float *red_b) {
   const int lane = threadIdx.x & 31;
   const int p = lane >> 1, sl = lane & 1;
   uint32_t xo[NT], so[NT];
@@ -287,27 +287,25 @@ __device__ __forceinline__ void gu_pass(const uint8_t *st, uint32_t rb, int nb, 
     xo[i] = (uint32_t)(t * d);
     so[i] = (uint32_t)(t * nb);
   }
-  for (int item = threadIdx.x >> 5; item < n_items; item += nwc) {
-    const int gran = item >> 1, hp = item & 1;
-    const int b0 = gran * kGran + sl * 4 + hp * 2;
+  for (int item = first; item < n_items; item += nwc) {
+    const int b0 = item * kGran + sl * 4;
     const uint32_t og = (uint32_t)p * rb + (uint32_t)b0 * MOE_QBYTES;
     const uint32_t ou = og + (uint32_t)kPairs * rb;
     float yg[NT], yu[NT];
 #pragma unroll
     for (int i = 0; i < NT; ++i) { yg[i] = 0.f; yu[i] = 0.f; }
     if (ALIGNED) {
-      Blk g0, g1, u0, u1;
-      if (hp == 0) {
-        load_span2<false>(st, og, g0, g1);
-        load_span2<false>(st, ou, u0, u1);
-      } else {
-        load_span2<true>(st, og, g0, g1);
-        load_span2<true>(st, ou, u0, u1);
-      }
+      Blk g0, g1, u0, u1, g2, g3, u2, u3;
+      load_span2<false>(st, og, g0, g1);
+      load_span2<false>(st, ou, u0, u1);
+      load_span2<true>(st, og + 2 * MOE_QBYTES, g2, g3);
+      load_span2<true>(st, ou + 2 * MOE_QBYTES, u2, u3);
       gu_pair_block<NT>(g0, u0, b0, sl, xs, ss, xo, so, yg, yu);
       gu_pair_block<NT>(g1, u1, b0 + 1, sl, xs, ss, xo, so, yg, yu);
+      gu_pair_block<NT>(g2, u2, b0 + 2, sl, xs, ss, xo, so, yg, yu);
+      gu_pair_block<NT>(g3, u3, b0 + 3, sl, xs, ss, xo, so, yg, yu);
     } else {
-      for (int j = 0; j < 2 && b0 + j < nb; ++j) {
+      for (int j = 0; j < 4 && b0 + j < nb; ++j) {
         const Blk bg = load_blk(st, og + (uint32_t)j * MOE_QBYTES);
         const Blk bu = load_blk(st, ou + (uint32_t)j * MOE_QBYTES);
         gu_pair_block<NT>(bg, bu, b0 + j, sl, xs, ss, xo, so, yg, yu);
@@ -317,55 +315,92 @@ __device__ __forceinline__ void gu_pass(const uint8_t *st, uint32_t rb, int nb, 
     for (int i = 0; i < NT; ++i) {
       const float g = yg[i] + __shfl_xor_sync(0xffffffffu, yg[i], 1);
       const float u = yu[i] + __shfl_xor_sync(0xffffffffu, yu[i], 1);
-      if (sl == 0) *reinterpret_cast<float2 *>(red_b + (((size_t)item * kPairs + p) * kTX + i) * 2) = make_float2(g, u);
+      if (sl == 0) *reinterpret_cast<float2 *>(red_b + (((size_t)item * kTX + i) * kPairs + p) * 2) = make_float2(g, u);
     }
   }
 }
 
-// down pass over one staged chunk (up to kDnRows rows) for NT slots: warp = (32-row group,
-// part of the row's blocks), lane = row; red_b[(part * kTX + i) * kDnRows + row].
+// Blocks b, b + 1 (b even) of a row whose byte offset o is 4-byte aligned: nine 32-bit loads.
+__device__ __forceinline__ void load_pair_w(const uint8_t *smem, uint32_t o, Blk &b0, Blk &b1) {
+  const uint32_t *wp = reinterpret_cast<const uint32_t *>(smem + o);
+  uint32_t w[10];
+#pragma unroll
+  for (int i = 0; i < 9; ++i) w[i] = wp[i];
+  w[9] = 0u;
+  split_blk2(w, b0, b1);
+}
+
+// One down-row block against NT slots' staged hidden vectors.
 template <int NT>
-__device__ __forceinline__ void dn_pass(const uint8_t *st, uint32_t rb, int nbf, int P, int nr, int f,
-                                        const uint16_t *hs, const ActBlk *hbk, int rel0, float *red_b) {
-  const int lane = threadIdx.x & 31, wq = threadIdx.x >> 5;
-  if (wq >= kDnGroups * P) return;
-  const int grp = wq % kDnGroups, part = wq / kDnGroups;
-  const int row = grp * 32 + lane;
-  if (row >= nr) return;
+__device__ __forceinline__ void dn_block(const Blk &bk, int b, const uint16_t *hs, const ActBlk *hbk,
+                                         const uint32_t (&ho)[NT], const uint32_t (&bo)[NT], float (&y)[NT]) {
+  int al[NT], ah[NT];
+  float sc[NT];
+#pragma unroll
+  for (int i = 0; i < NT; ++i) {
+    const ActBlk ab = hbk[bo[i] + b];
+    al[i] = ab.neg8sum;
+    ah[i] = 0;
+    sc[i] = ab.scale;
+  }
+#pragma unroll
+  for (int wi = 0; wi < 4; ++wi) {
+    const uint32_t lo = bk.q[wi] & 0x0F0F0F0Fu, hi = bk.q[wi] & 0xF0F0F0F0u;
+#pragma unroll
+    for (int i = 0; i < NT; ++i)
+      dot8i(lo, hi, *reinterpret_cast<const uint4 *>(hs + ho[i] + b * MOE_QK + 8 * wi), al[i], ah[i]);
+  }
+#pragma unroll
+  for (int i = 0; i < NT; ++i) y[i] = block_finish(y[i], bk.d, sc[i], al[i], ah[i]);
+}
+
+// down pass over one staged chunk (up to kDnRows rows) for NT slots, by the compute warps:
+// items first, first + nwc, ... Work item = (32-row group, part of the row's
+// blocks), lane = row; red_b[(part * kTX + i) * kDnRows + row]. With PAIRED
+// (an even number of blocks per row, so every row starts 4-byte aligned) a part takes whole
+// block pairs and the blocks left over go one each to the first parts; otherwise parts are
+// contiguous block ranges read block by block.
+template <int NT, bool PAIRED>
+__device__ __forceinline__ void dn_pass(const uint8_t *st, uint32_t rb, int nbf, int P, int nwc, int first, int nr,
+                                        int f, const uint16_t *hs, const ActBlk *hbk, int rel0, float *red_b) {
+  const int lane = threadIdx.x & 31;
   uint32_t ho[NT], bo[NT];
 #pragma unroll
   for (int i = 0; i < NT; ++i) {
     ho[i] = (uint32_t)((rel0 + i) * f);
     bo[i] = (uint32_t)((rel0 + i) * nbf);
   }
-  const int b0 = part * nbf / P, b1 = (part + 1) * nbf / P;
-  float y[NT];
+  for (int item = first; item < kDnGroups * P; item += nwc) {
+    const int grp = item % kDnGroups, part = item / kDnGroups;
+    const int row = grp * 32 + lane;
+    if (grp * 32 >= nr) continue;   // warp-uniform: this row group is past the chunk
+    float y[NT];
 #pragma unroll
-  for (int i = 0; i < NT; ++i) y[i] = 0.f;
-  const uint32_t orow = (uint32_t)row * rb;
-  for (int b = b0; b < b1; ++b) {
-    const Blk bk = load_blk(st, orow + (uint32_t)b * MOE_QBYTES);
-    int al[NT], ah[NT];
-    float sc[NT];
+    for (int i = 0; i < NT; ++i) y[i] = 0.f;
+    if (row < nr) {
+      const uint32_t orow = (uint32_t)row * rb;
+      if (PAIRED) {
+        const int per = nbf / (2 * P);   // pairs per part
+        for (int pr = part * per; pr < (part + 1) * per; ++pr) {
+          Blk k0, k1;
+          load_pair_w(st, orow + (uint32_t)(2 * pr) * MOE_QBYTES, k0, k1);
+          dn_block<NT>(k0, 2 * pr, hs, hbk, ho, bo, y);
+          dn_block<NT>(k1, 2 * pr + 1, hs, hbk, ho, bo, y);
+        }
+        for (int b = 2 * P * per + part; b < nbf; b += P) {
+          const Blk kb = load_blk(st, orow + (uint32_t)b * MOE_QBYTES);
+          dn_block<NT>(kb, b, hs, hbk, ho, bo, y);
+        }
+      } else {
+        for (int b = part * nbf / P; b < (part + 1) * nbf / P; ++b) {
+          const Blk kb = load_blk(st, orow + (uint32_t)b * MOE_QBYTES);
+          dn_block<NT>(kb, b, hs, hbk, ho, bo, y);
+        }
+      }
 #pragma unroll
-    for (int i = 0; i < NT; ++i) {
-      const ActBlk ab = hbk[bo[i] + b];
-      al[i] = ab.neg8sum;
-      ah[i] = 0;
-      sc[i] = ab.scale;
+      for (int i = 0; i < NT; ++i) red_b[((size_t)part * kTX + i) * kDnRows + row] = y[i];
     }
-#pragma unroll
-    for (int wi = 0; wi < 4; ++wi) {
-      const uint32_t lo = bk.q[wi] & 0x0F0F0F0Fu, hi = bk.q[wi] & 0xF0F0F0F0u;
-#pragma unroll
-      for (int i = 0; i < NT; ++i)
-        dot8i(lo, hi, *reinterpret_cast<const uint4 *>(hs + ho[i] + b * MOE_QK + 8 * wi), al[i], ah[i]);
-    }
-#pragma unroll
-    for (int i = 0; i < NT; ++i) y[i] = block_finish(y[i], bk.d, sc[i], al[i], ah[i]);
   }
-#pragma unroll
-  for (int i = 0; i < NT; ++i) red_b[((size_t)part * kTX + i) * kDnRows + row] = y[i];
 }
 
 __global__ void __launch_bounds__((kFMaxCompute + 2) * 32, 1)
@@ -381,7 +416,7 @@ k_moe_decode(const __nv_bfloat16 *__restrict__ x, const float *__restrict__ rout
   const int nteam = nct + 32;
   const int nb = d / MOE_QK, nbf = f / MOE_QK;
   const int G = (nb + kGran - 1) / kGran;
-  const int P = nwc / kDnGroups;
+  const int P = kDnParts;
   const uint32_t rb_g = (uint32_t)nb * MOE_QBYTES, rb_d = (uint32_t)nbf * MOE_QBYTES;
   uint8_t *smem = align128(smem_raw);
   uint8_t *xreg = smem + (size_t)kFStages * stage_bytes;
@@ -441,43 +476,29 @@ k_moe_decode(const __nv_bfloat16 *__restrict__ x, const float *__restrict__ rout
     }
     __syncthreads();
   }
-  // arrive; stage every token's activations while the other CTAs finish their logits
+  // arrive at the grid barrier; the thread that arrives waits
   __syncthreads();
   unsigned long long target = 0;
   if (tid == 0) target = grid_arrive(W.gbar);
-  {
-    // four (token, block, quarter) tasks per thread: all loads first, then the conversions
-    const int ntask = T * nb * 4, stride = nw * 32;
-    for (int base = wq * 32; base < ntask; base += 4 * stride) {
-      uint4 raw[4];
+  // every token's activations, staged while the other CTAs finish their logits: one
+  // (token, block) per thread
+  for (int blk = tid; blk < T * nb; blk += blockDim.x) {
+    const int t = blk / nb, b = blk - t * nb;
+    const uint4 *src = reinterpret_cast<const uint4 *>(x + (size_t)t * d + (size_t)b * MOE_QK);
+    uint4 raw[4];
 #pragma unroll
-      for (int r = 0; r < 4; ++r) {
-        const int task = base + r * stride + lane;
-        if (task < ntask) {
-          const int blk = task >> 2, q = task & 3;
-          const int t = blk / nb, b = blk - t * nb;
-          raw[r] = __ldg(reinterpret_cast<const uint4 *>(x + (size_t)t * d + (size_t)b * MOE_QK + 8 * q));
-        } else {
-          raw[r] = make_uint4(0u, 0u, 0u, 0u);
-        }
-      }
+    for (int i = 0; i < 4; ++i) raw[i] = __ldg(src + i);
+    float v[MOE_QK];
 #pragma unroll
-      for (int r = 0; r < 4; ++r) {
-        if (base + r * stride >= ntask) break;   // warp-uniform
-        const int task = base + r * stride + lane;
-        const bool valid = task < ntask;
-        const int blk = valid ? task >> 2 : 0;
-        const int t = blk / nb, b = blk - t * nb;
-        const uint32_t uu[4] = {raw[r].x, raw[r].y, raw[r].z, raw[r].w};
-        float v[8];
+    for (int i = 0; i < 4; ++i) {
+      const uint32_t uu[4] = {raw[i].x, raw[i].y, raw[i].z, raw[i].w};
 #pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          v[2 * i] = __uint_as_float(uu[i] << 16);
-          v[2 * i + 1] = __uint_as_float(uu[i] & 0xffff0000u);
-        }
-        stage_block_q(v, valid, (b >> 2) & 1, xs + (size_t)t * d + (size_t)b * MOE_QK, ss + (size_t)t * nb + b);
+      for (int h = 0; h < 4; ++h) {
+        v[8 * i + 2 * h] = __uint_as_float(uu[h] << 16);
+        v[8 * i + 2 * h + 1] = __uint_as_float(uu[h] & 0xffff0000u);
       }
     }
+    stage_block_t(v, (b >> 2) & 1, xs + (size_t)t * d + (size_t)b * MOE_QK, ss + (size_t)t * nb + b);
   }
   if (tid == 0) sh.ok = grid_wait(W.gbar, target, W.err, 20) ? 1 : 0;
   __syncthreads();
@@ -561,25 +582,18 @@ k_moe_decode(const __nv_bfloat16 *__restrict__ x, const float *__restrict__ rout
     }
   }
   __syncthreads();
-  FSeq seq;
-  seq.upe_g = upe_g;
-  seq.upe_d = upe_d;
-  seq.g0 = sh.seq[0];
-  seq.g1 = sh.seq[1];
-  seq.d0 = sh.seq[2];
-  seq.d1 = sh.seq[3];
-  const int n_units = seq.total();
 
   // ---------------------------------------------------------------- producer warp
   if (wq == nwc) {
     if (lane == 0) {
-      int u = 0;
-      for (int it = 0; u < n_units; ++it) {
+      FWalk wk;
+      wk.init(sh.seq, upe_g, upe_d);
+      for (int it = 0; !wk.done(); ++it) {
         const int slot = it % kFStages;
         if (it >= kFStages &&
             !wait_phase(&sh.empty[slot], (uint32_t)(it / kFStages - 1) & 1u, &sh.abort, W.err, 24))
           break;
-        const FChunk c = seq.at(u);
+        const FChunk c = wk.cur(upe_g, upe_d);
         const int e = sh.act[c.a];
         uint8_t *dst = smem + (size_t)slot * stage_bytes;
         if (!c.down) {
@@ -593,7 +607,7 @@ k_moe_decode(const __nv_bfloat16 *__restrict__ x, const float *__restrict__ rout
           mbar_arrive_expect_tx(&sh.full[slot], bytes);
           bulk_g2s(dst, down_q4 + (size_t)e * d * rb_d + (size_t)c.r0 * rb_d, bytes, &sh.full[slot]);
         }
-        u += c.n;
+        wk.advance(c.n, sh.seq, upe_g, upe_d);
       }
     }
     return;
@@ -621,13 +635,15 @@ k_moe_decode(const __nv_bfloat16 *__restrict__ x, const float *__restrict__ rout
   // Compute warps multiply a staged chunk into one of two reduction buffers and move on; the
   // epilogue warp turns a full buffer into h (GeGLU) or per-slot outputs and hands it back.
   const bool aligned = (nb % kGran) == 0;
-  const int n_items = 2 * G;
+  const int n_items = G;
   bool down_phase = false;
   int pass = 0;
   if (wq < nwc) {
     int hw0 = 0, hw1 = 0;   // sorted positions whose hidden vectors are staged in hs
-    for (int u = 0, it = 0; u < n_units; ++it) {
-      const FChunk c = seq.at(u);
+    FWalk wk;
+    wk.init(sh.seq, upe_g, upe_d);
+    for (int it = 0; !wk.done(); ++it) {
+      const FChunk c = wk.cur(upe_g, upe_d);
       if (c.down && !down_phase) {
         // all h written (the epilogue warp included) before any CTA reads it
         grid_barrier_team(W.gbar, W.err, 21, nteam, &sh.abort);
@@ -646,18 +662,21 @@ k_moe_decode(const __nv_bfloat16 *__restrict__ x, const float *__restrict__ rout
           if (pass >= 2) named_sync(kBarEmpty0 + b, nteam);
           float *red_b = red + (size_t)b * red_half;
           const int32_t *pt = sh.ptok + off + g0;
+          const int first = wq;
           if (okw) {
             if (aligned) {
               switch (ng) {
-                case 1: gu_pass<1, true>(st, rb_g, nb, n_items, nwc, d, xs, ss, pt, red_b); break;
-                case 2: gu_pass<2, true>(st, rb_g, nb, n_items, nwc, d, xs, ss, pt, red_b); break;
-                default: gu_pass<3, true>(st, rb_g, nb, n_items, nwc, d, xs, ss, pt, red_b); break;
+                case 1: gu_pass<1, true>(st, rb_g, nb, n_items, nwc, first, d, xs, ss, pt, red_b); break;
+                case 2: gu_pass<2, true>(st, rb_g, nb, n_items, nwc, first, d, xs, ss, pt, red_b); break;
+                case 3: gu_pass<3, true>(st, rb_g, nb, n_items, nwc, first, d, xs, ss, pt, red_b); break;
+                default: gu_pass<4, true>(st, rb_g, nb, n_items, nwc, first, d, xs, ss, pt, red_b); break;
               }
             } else {
               switch (ng) {
-                case 1: gu_pass<1, false>(st, rb_g, nb, n_items, nwc, d, xs, ss, pt, red_b); break;
-                case 2: gu_pass<2, false>(st, rb_g, nb, n_items, nwc, d, xs, ss, pt, red_b); break;
-                default: gu_pass<3, false>(st, rb_g, nb, n_items, nwc, d, xs, ss, pt, red_b); break;
+                case 1: gu_pass<1, false>(st, rb_g, nb, n_items, nwc, first, d, xs, ss, pt, red_b); break;
+                case 2: gu_pass<2, false>(st, rb_g, nb, n_items, nwc, first, d, xs, ss, pt, red_b); break;
+                case 3: gu_pass<3, false>(st, rb_g, nb, n_items, nwc, first, d, xs, ss, pt, red_b); break;
+                default: gu_pass<4, false>(st, rb_g, nb, n_items, nwc, first, d, xs, ss, pt, red_b); break;
               }
             }
           }
@@ -668,39 +687,21 @@ k_moe_decode(const __nv_bfloat16 *__restrict__ x, const float *__restrict__ rout
           // stage the hidden vectors of the slots from this expert on, up to the end of this
           // CTA's last expert or the window's capacity
           named_sync(kBarCompute, nct);   // every compute warp is done with the previous window
-          const int a_last = (seq.d1 - 1) / seq.upe_d;
+          const int a_last = (sh.seq[3] - 1) / upe_d;
           const int e_last = sh.act[a_last];
           hw0 = off;
           hw1 = min(sh.offsets[e_last] + sh.counts[e_last], off + hcap);
-          const int ntask = okw ? (hw1 - hw0) * nbf * 4 : 0, stride = nwc * 32;
-          for (int base = wq * 32; base < ntask; base += 2 * stride) {
-            float4 raw[2][2];
+          const int nblk = okw ? (hw1 - hw0) * nbf : 0;
+          for (int blk = tid; blk < nblk; blk += nct) {
+            const int i = blk / nbf, cb = blk - i * nbf;
+            const float4 *src = reinterpret_cast<const float4 *>(W.h + (size_t)sh.perm[hw0 + i] * f + (size_t)cb * MOE_QK);
+            float v[MOE_QK];
 #pragma unroll
-            for (int r = 0; r < 2; ++r) {
-              const int task = base + r * stride + lane;
-              if (task < ntask) {
-                const int blk = task >> 2, q = task & 3;
-                const int i = blk / nbf, cb = blk - i * nbf;
-                const float4 *src = reinterpret_cast<const float4 *>(W.h + (size_t)sh.perm[hw0 + i] * f +
-                                                                     (size_t)cb * MOE_QK + 8 * q);
-                raw[r][0] = __ldcg(src);
-                raw[r][1] = __ldcg(src + 1);
-              } else {
-                raw[r][0] = make_float4(0.f, 0.f, 0.f, 0.f);
-                raw[r][1] = raw[r][0];
-              }
+            for (int q = 0; q < 8; ++q) {
+              const float4 a4 = __ldcg(src + q);
+              v[4 * q] = a4.x; v[4 * q + 1] = a4.y; v[4 * q + 2] = a4.z; v[4 * q + 3] = a4.w;
             }
-#pragma unroll
-            for (int r = 0; r < 2; ++r) {
-              if (base + r * stride >= ntask) break;   // warp-uniform
-              const int task = base + r * stride + lane;
-              const bool valid = task < ntask;
-              const int blk = valid ? task >> 2 : 0;
-              const int i = blk / nbf, cb = blk - i * nbf;
-              const float v[8] = {raw[r][0].x, raw[r][0].y, raw[r][0].z, raw[r][0].w,
-                                  raw[r][1].x, raw[r][1].y, raw[r][1].z, raw[r][1].w};
-              stage_block_q(v, valid, 0, hs + (size_t)i * f + (size_t)cb * MOE_QK, hbk + (size_t)i * nbf + cb);
-            }
+            stage_block_t(v, 0, hs + (size_t)i * f + (size_t)cb * MOE_QK, hbk + (size_t)i * nbf + cb);
           }
           named_sync(kBarCompute, nct);
         }
@@ -711,26 +712,38 @@ k_moe_decode(const __nv_bfloat16 *__restrict__ x, const float *__restrict__ rout
           if (pass >= 2) named_sync(kBarEmpty0 + b, nteam);
           float *red_b = red + (size_t)b * red_half;
           const int rel0 = off + g0 - hw0;
+          const int first = wq;
           if (okw) {
-            switch (ng) {
-              case 1: dn_pass<1>(st, rb_d, nbf, P, nr, f, hs, hbk, rel0, red_b); break;
-              case 2: dn_pass<2>(st, rb_d, nbf, P, nr, f, hs, hbk, rel0, red_b); break;
-              case 3: dn_pass<3>(st, rb_d, nbf, P, nr, f, hs, hbk, rel0, red_b); break;
-              default: dn_pass<4>(st, rb_d, nbf, P, nr, f, hs, hbk, rel0, red_b); break;
+            if ((nbf & 1) == 0) {
+              switch (ng) {
+                case 1: dn_pass<1, true>(st, rb_d, nbf, P, nwc, first, nr, f, hs, hbk, rel0, red_b); break;
+                case 2: dn_pass<2, true>(st, rb_d, nbf, P, nwc, first, nr, f, hs, hbk, rel0, red_b); break;
+                case 3: dn_pass<3, true>(st, rb_d, nbf, P, nwc, first, nr, f, hs, hbk, rel0, red_b); break;
+                default: dn_pass<4, true>(st, rb_d, nbf, P, nwc, first, nr, f, hs, hbk, rel0, red_b); break;
+              }
+            } else {
+              switch (ng) {
+                case 1: dn_pass<1, false>(st, rb_d, nbf, P, nwc, first, nr, f, hs, hbk, rel0, red_b); break;
+                case 2: dn_pass<2, false>(st, rb_d, nbf, P, nwc, first, nr, f, hs, hbk, rel0, red_b); break;
+                case 3: dn_pass<3, false>(st, rb_d, nbf, P, nwc, first, nr, f, hs, hbk, rel0, red_b); break;
+                default: dn_pass<4, false>(st, rb_d, nbf, P, nwc, first, nr, f, hs, hbk, rel0, red_b); break;
+              }
             }
           }
           named_arrive(kBarFull0 + b, nteam);
         }
       }
       if (lane == 0) mbar_arrive(&sh.empty[slot]);   // this warp's last read of the stage
-      u += c.n;
+      wk.advance(c.n, sh.seq, upe_g, upe_d);
     }
     if (!down_phase) grid_barrier_team(W.gbar, W.err, 21, nteam, &sh.abort);   // no down rows here
     for (int q = pass < 2 ? 0 : pass - 2; q < pass; ++q) named_sync(kBarEmpty0 + (q & 1), nteam);
   } else {
     // the epilogue warp: the same sequence of chunks and passes
-    for (int u = 0; u < n_units;) {
-      const FChunk c = seq.at(u);
+    FWalk wk;
+    wk.init(sh.seq, upe_g, upe_d);
+    while (!wk.done()) {
+      const FChunk c = wk.cur(upe_g, upe_d);
       if (c.down && !down_phase) {
         grid_barrier_team(W.gbar, W.err, 21, nteam, &sh.abort);
         down_phase = true;
@@ -746,13 +759,13 @@ k_moe_decode(const __nv_bfloat16 *__restrict__ x, const float *__restrict__ rout
         const float *red_b = red + (size_t)b * red_half;
         if (!sh.abort) {
           if (!c.down) {
-            // h = gelu(gate) * up; the partials of the 2 G work items summed in order
+            // h = gelu(gate) * up; the partials of the G work items summed in order
             const int np = c.n * kUnit, sh_np = np == 16 ? 4 : 3;
             for (int itm = lane; itm < np * ng; itm += 32) {
               const int i = itm >> sh_np, pp = itm & (np - 1);
               float g = 0.f, uu = 0.f;
               for (int q = 0; q < n_items; ++q) {
-                const float2 v = *reinterpret_cast<const float2 *>(red_b + (((size_t)q * kPairs + pp) * kTX + i) * 2);
+                const float2 v = *reinterpret_cast<const float2 *>(red_b + (((size_t)q * kTX + i) * kPairs + pp) * 2);
                 g += v.x;
                 uu += v.y;
               }
@@ -770,7 +783,7 @@ k_moe_decode(const __nv_bfloat16 *__restrict__ x, const float *__restrict__ rout
         }
         named_arrive(kBarEmpty0 + b, nteam);
       }
-      u += c.n;
+      wk.advance(c.n, sh.seq, upe_g, upe_d);
     }
     if (!down_phase) grid_barrier_team(W.gbar, W.err, 21, nteam, &sh.abort);
   }
@@ -801,14 +814,14 @@ struct FusedSmem {
 static FusedSmem fused_smem(int T, int d, int f) {
   const int nb = d / MOE_QK, nbf = f / MOE_QK;
   const int G = (nb + kGran - 1) / kGran;
-  const int P = fused_compute_warps(G) / kDnGroups;
+  const int P = kDnParts;
   FusedSmem r;
   const size_t sg = 2u * kPairs * (size_t)nb * MOE_QBYTES + 16u;
   const size_t sd = (size_t)kDnRows * nbf * MOE_QBYTES + 16u;
   r.stage_bytes = (uint32_t)(((sg > sd ? sg : sd) + 15u) & ~(size_t)15u);
   const size_t xg = (size_t)T * (2 * d + 8 * nb), xh = (size_t)T * (2 * f + 8 * nbf);
   r.x_bytes = (uint32_t)(((xg > xh ? xg : xh) + 15u) & ~(size_t)15u);
-  const size_t rg = (size_t)2 * G * kPairs * kTX * 2, rd = (size_t)P * kTX * kDnRows;
+  const size_t rg = (size_t)G * kPairs * kTX * 2, rd = (size_t)P * kTX * kDnRows;
   r.red_half = (uint32_t)(rg > rd ? rg : rd);
   r.total = (size_t)kFStages * r.stage_bytes + r.x_bytes + (size_t)2 * r.red_half * 4 + 128;
   return r;
