@@ -586,6 +586,7 @@ k_moe_decode(const __nv_bfloat16 *__restrict__ x, const float *__restrict__ rout
   // ---------------------------------------------------------------- producer warp
   if (wq == nwc) {
     if (lane == 0) {
+      const uint64_t pol = l2_evict_first_policy();   // expert weights are read once per call
       FWalk wk;
       wk.init(sh.seq, upe_g, upe_d);
       for (int it = 0; !wk.done(); ++it) {
@@ -600,12 +601,12 @@ k_moe_decode(const __nv_bfloat16 *__restrict__ x, const float *__restrict__ rout
           const uint8_t *base = gate_up_q4 + (size_t)e * 2 * f * rb_g;
           const uint32_t bytes = (uint32_t)(c.n * kUnit) * rb_g;
           mbar_arrive_expect_tx(&sh.full[slot], 2u * bytes);
-          bulk_g2s(dst, base + (size_t)c.r0 * rb_g, bytes, &sh.full[slot]);
-          bulk_g2s(dst + kPairs * rb_g, base + (size_t)(f + c.r0) * rb_g, bytes, &sh.full[slot]);
+          bulk_g2s_hint(dst, base + (size_t)c.r0 * rb_g, bytes, &sh.full[slot], pol);
+          bulk_g2s_hint(dst + kPairs * rb_g, base + (size_t)(f + c.r0) * rb_g, bytes, &sh.full[slot], pol);
         } else {
           const uint32_t bytes = (uint32_t)(c.n * kUnit) * rb_d;
           mbar_arrive_expect_tx(&sh.full[slot], bytes);
-          bulk_g2s(dst, down_q4 + (size_t)e * d * rb_d + (size_t)c.r0 * rb_d, bytes, &sh.full[slot]);
+          bulk_g2s_hint(dst, down_q4 + (size_t)e * d * rb_d + (size_t)c.r0 * rb_d, bytes, &sh.full[slot], pol);
         }
         wk.advance(c.n, sh.seq, upe_g, upe_d);
       }

@@ -47,6 +47,7 @@ k_gateup_gemv(const uint8_t *__restrict__ gate_up_q4, int d, int f, int k, int n
   }
   __syncthreads();
 
+  const uint64_t pol = l2_evict_first_policy();   // expert weights are read once per call
   auto issue = [&](int u, int slot) {
     const GuChunk c = gu_chunk(u, u1, upe);
     const int e = W.act[c.a];
@@ -54,8 +55,8 @@ k_gateup_gemv(const uint8_t *__restrict__ gate_up_q4, int d, int f, int k, int n
     uint8_t *dst = smem + (size_t)slot * stage_bytes;
     const uint32_t bytes = (uint32_t)c.np * rb;
     mbar_arrive_expect_tx(&ring.full[slot], 2u * bytes);
-    bulk_g2s(dst, base + (size_t)c.c0 * rb, bytes, &ring.full[slot]);
-    bulk_g2s(dst + kPairs * rb, base + (size_t)(f + c.c0) * rb, bytes, &ring.full[slot]);
+    bulk_g2s_hint(dst, base + (size_t)c.c0 * rb, bytes, &ring.full[slot], pol);
+    bulk_g2s_hint(dst + kPairs * rb, base + (size_t)(f + c.c0) * rb, bytes, &ring.full[slot], pol);
   };
   int u_issue = u0;
   if (threadIdx.x == 0) {
@@ -163,13 +164,14 @@ k_down_gemv_combine(const uint8_t *__restrict__ down_q4, const float *__restrict
   }
   __syncthreads();
 
+  const uint64_t pol = l2_evict_first_policy();
   auto issue = [&](int u, int slot) {
     const DnChunk c = dn_chunk(u, u1, upe);
     const int e = W.act[c.a];
     const uint8_t *src = down_q4 + (size_t)e * d * rb + (size_t)c.r0 * rb;
     const uint32_t bytes = (uint32_t)c.nr * rb;
     mbar_arrive_expect_tx(&ring.full[slot], bytes);
-    bulk_g2s(smem + (size_t)slot * stage_bytes, src, bytes, &ring.full[slot]);
+    bulk_g2s_hint(smem + (size_t)slot * stage_bytes, src, bytes, &ring.full[slot], pol);
   };
   int u_issue = u0;
   if (threadIdx.x == 0) {
