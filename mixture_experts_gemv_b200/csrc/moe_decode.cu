@@ -53,6 +53,7 @@ __host__ __device__ inline int fused_compute_warps(int G) {
 struct FusedShared {
   uint64_t full[kFStages];
   uint64_t empty[kFStages];
+  uint64_t xbar;              // x copied into shared memory
   int32_t ids[kFMaxSlots];
   float w[kFMaxSlots];
   int32_t perm[kFMaxSlots];
@@ -416,7 +417,6 @@ k_moe_decode(const __nv_bfloat16 *__restrict__ x, const float *__restrict__ rout
   const int nteam = nct + 32;
   const int nb = d / MOE_QK, nbf = f / MOE_QK;
   const int G = (nb + kGran - 1) / kGran;
-  const int P = kDnParts;
   const uint32_t rb_g = (uint32_t)nb * MOE_QBYTES, rb_d = (uint32_t)nbf * MOE_QBYTES;
   uint8_t *smem = align128(smem_raw);
   uint8_t *xreg = smem + (size_t)kFStages * stage_bytes;
@@ -433,8 +433,12 @@ k_moe_decode(const __nv_bfloat16 *__restrict__ x, const float *__restrict__ rout
       mbar_init(&sh.full[s], 1);
       mbar_init(&sh.empty[s], nwc);
     }
+    mbar_init(&sh.xbar, 1);
     fence_mbar_init();
     sh.abort = 0;
+    // x (bf16) into the activation region now; it is converted in place before the first barrier
+    mbar_arrive_expect_tx(&sh.xbar, (uint32_t)(T * d * 2));
+    bulk_g2s(xreg, x, (uint32_t)(T * d * 2), &sh.xbar);
   }
   const float rs = __ldg(router_scale);
 
@@ -480,29 +484,34 @@ k_moe_decode(const __nv_bfloat16 *__restrict__ x, const float *__restrict__ rout
   __syncthreads();
   unsigned long long target = 0;
   if (tid == 0) target = grid_arrive(W.gbar);
-  // every token's activations, staged while the other CTAs finish their logits: one
-  // (token, block) per thread
-  for (int blk = tid; blk < T * nb; blk += blockDim.x) {
-    const int t = blk / nb, b = blk - t * nb;
-    const uint4 *src = reinterpret_cast<const uint4 *>(x + (size_t)t * d + (size_t)b * MOE_QK);
-    uint4 raw[4];
+  // every token's activations, converted in place (x was copied into the activation region at
+  // the start) while the other CTAs finish their logits: one (token, block) per thread
+  if (wait_phase(&sh.xbar, 0u, &sh.abort, W.err, 26)) {
+    for (int blk = tid; blk < T * nb; blk += blockDim.x) {
+      const int t = blk / nb, b = blk - t * nb;
+      const uint4 *src = reinterpret_cast<const uint4 *>(xs + (size_t)t * d + (size_t)b * MOE_QK);
+      uint4 raw[4];
 #pragma unroll
-    for (int i = 0; i < 4; ++i) raw[i] = __ldg(src + i);
-    float v[MOE_QK];
+      for (int i = 0; i < 4; ++i) raw[i] = src[i];
+      float v[MOE_QK];
 #pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      const uint32_t uu[4] = {raw[i].x, raw[i].y, raw[i].z, raw[i].w};
+      for (int i = 0; i < 4; ++i) {
+        const uint32_t uu[4] = {raw[i].x, raw[i].y, raw[i].z, raw[i].w};
 #pragma unroll
-      for (int h = 0; h < 4; ++h) {
-        v[8 * i + 2 * h] = __uint_as_float(uu[h] << 16);
-        v[8 * i + 2 * h + 1] = __uint_as_float(uu[h] & 0xffff0000u);
+        for (int h = 0; h < 4; ++h) {
+          v[8 * i + 2 * h] = __uint_as_float(uu[h] << 16);
+          v[8 * i + 2 * h + 1] = __uint_as_float(uu[h] & 0xffff0000u);
+        }
       }
+      stage_block_t(v, (b >> 2) & 1, xs + (size_t)t * d + (size_t)b * MOE_QK, ss + (size_t)t * nb + b);
     }
-    stage_block_t(v, (b >> 2) & 1, xs + (size_t)t * d + (size_t)b * MOE_QK, ss + (size_t)t * nb + b);
   }
   if (tid == 0) sh.ok = grid_wait(W.gbar, target, W.err, 20) ? 1 : 0;
   __syncthreads();
-  if (!sh.ok) return;
+  if (!sh.ok) {
+    if (tid == 0) mbar_wait(&sh.xbar, 0u, W.err, 27);   // no copy may land after the CTA exits
+    return;
+  }
 
   // ---------------------------------------------------------------- phase 1: selection
   for (int t = wq; t < T; t += nw)
@@ -589,7 +598,8 @@ k_moe_decode(const __nv_bfloat16 *__restrict__ x, const float *__restrict__ rout
       const uint64_t pol = l2_evict_first_policy();   // expert weights are read once per call
       FWalk wk;
       wk.init(sh.seq, upe_g, upe_d);
-      for (int it = 0; !wk.done(); ++it) {
+      int it = 0;
+      for (; !wk.done(); ++it) {
         const int slot = it % kFStages;
         if (it >= kFStages &&
             !wait_phase(&sh.empty[slot], (uint32_t)(it / kFStages - 1) & 1u, &sh.abort, W.err, 24))
@@ -610,6 +620,9 @@ k_moe_decode(const __nv_bfloat16 *__restrict__ x, const float *__restrict__ rout
         }
         wk.advance(c.n, sh.seq, upe_g, upe_d);
       }
+      // every copy issued has landed before this warp leaves (at once unless the call aborted)
+      for (int q = it - 1; q >= 0 && q >= it - kFStages; --q)
+        mbar_wait(&sh.full[q % kFStages], (uint32_t)(q / kFStages) & 1u, W.err, 28);
     }
     return;
   }
@@ -637,6 +650,7 @@ k_moe_decode(const __nv_bfloat16 *__restrict__ x, const float *__restrict__ rout
   // epilogue warp turns a full buffer into h (GeGLU) or per-slot outputs and hands it back.
   const bool aligned = (nb % kGran) == 0;
   const int n_items = G;
+  const int P = kDnParts;
   bool down_phase = false;
   int pass = 0;
   if (wq < nwc) {
@@ -815,14 +829,13 @@ struct FusedSmem {
 static FusedSmem fused_smem(int T, int d, int f) {
   const int nb = d / MOE_QK, nbf = f / MOE_QK;
   const int G = (nb + kGran - 1) / kGran;
-  const int P = kDnParts;
   FusedSmem r;
   const size_t sg = 2u * kPairs * (size_t)nb * MOE_QBYTES + 16u;
   const size_t sd = (size_t)kDnRows * nbf * MOE_QBYTES + 16u;
   r.stage_bytes = (uint32_t)(((sg > sd ? sg : sd) + 15u) & ~(size_t)15u);
   const size_t xg = (size_t)T * (2 * d + 8 * nb), xh = (size_t)T * (2 * f + 8 * nbf);
   r.x_bytes = (uint32_t)(((xg > xh ? xg : xh) + 15u) & ~(size_t)15u);
-  const size_t rg = (size_t)G * kPairs * kTX * 2, rd = (size_t)P * kTX * kDnRows;
+  const size_t rg = (size_t)G * kPairs * kTX * 2, rd = (size_t)kDnParts * kTX * kDnRows;
   r.red_half = (uint32_t)(rg > rd ? rg : rd);
   r.total = (size_t)kFStages * r.stage_bytes + r.x_bytes + (size_t)2 * r.red_half * 4 + 128;
   return r;
