@@ -10,21 +10,20 @@
 // followed by out[t] = sum_j w_tj * s_e * Y[slot(t, j)] in j order.
 //
 // Layout: the routed rows of each expert are padded to whole 128-row tiles; tile i of the
-// tile list covers padded rows [128 i, 128 i + 128). X is gathered into that padded order
-// (k_gather_x) so both GEMMs read their A operand with plain 2-D TMA tiles (128 rows x 64
-// bf16, 128-byte swizzle, no multicast). The B operand (weights) never exists in bf16 in
-// global memory: producer warps read Q4_0 blocks, decode (q - 8) * d to bf16 and write the
-// swizzled K-major tile that tcgen05.mma reads.
+// tile list covers padded rows [128 i, 128 i + 128). The producers gather the A rows
+// (gate_up: the tokens' rows of x; down: the padded rows of h) straight into the 128-byte
+// swizzled K-major tile with 16-byte asynchronous copies (zero-filled past the expert's
+// rows), and copy the raw Q4_0 bytes of the B rows into a staging ring with 4-byte
+// asynchronous copies, several K steps ahead of the MMA. The weights never exist in bf16 in
+// global memory: the producers decode (q - 8) * d from the staged bytes and write the
+// swizzled K-major B tile that tcgen05.mma reads.
 //
 // One CTA per SM, persistent over (tile, n-tile) work items, warp-specialised:
 //   warps 0-3  epilogue: tcgen05.ld of the 128 x 128 FP32 accumulator (lane = row)
 //   warp  4    TMEM allocation; lane 0 issues tcgen05.mma (M = 128, N = 128, K = 16)
-//   warps 5-12 producers: TMA for A, Q4_0 -> bf16 dequantisation for B
+//   warps 5-12 producers: gathered A rows, staged Q4_0 -> bf16 dequantisation for B
 // Shared-memory stages are handed over with mbarriers (every wait is time-bounded); the
 // accumulator is double-buffered in TMEM so the epilogue of one item overlaps the next.
-#include <cuda.h>
-#include <cudaTypedefs.h>
-
 #include "moe_common.cuh"
 
 namespace {
@@ -33,13 +32,18 @@ constexpr int BM = 128, BN = 128, BK = 64;
 constexpr int kStages = 5;
 constexpr int kEpiWarps = 4;
 constexpr int kMmaWarp = 4;
-constexpr int kProdWarps = 8;
+constexpr int kProdGroups = 2;                                // producer groups take alternate K steps
+constexpr int kProdWarps = 8 * kProdGroups;
 constexpr int kProdThreads = kProdWarps * 32;
-constexpr int kThreads = (kEpiWarps + 1 + kProdWarps) * 32;   // 416
+constexpr int kGroupThreads = kProdThreads / kProdGroups;     // one (row, block) of the B tile each
+constexpr int kThreads = (kEpiWarps + 1 + kProdWarps) * 32;
 constexpr uint32_t kTileBytes = BM * BK * 2;                  // 16 KB (A); B is BN x BK, same
 constexpr uint32_t kStageBytes = 2 * kTileBytes;
 constexpr uint32_t kTmemCols = 2 * BN;                        // two accumulator buffers
-constexpr int kSmemBytes = kStages * kStageBytes + 1024;
+constexpr int kPrefetch = kStages - 1;                        // K steps the copies run ahead
+constexpr uint32_t kRawRowBytes = 64;                          // 16-byte-aligned window over a row's 36 bytes
+constexpr uint32_t kRawStageBytes = BN * kRawRowBytes;
+constexpr int kSmemBytes = kStages * (kStageBytes + kRawStageBytes) + 1024;
 
 // UMMA instruction descriptor, kind::f16: D FP32 (bits 4-5 = 1), A and B bf16 (bits 7-9,
 // 10-12 = 1), both K-major (bits 15, 16 = 0), N >> 3 in bits 17-22, M >> 4 in bits 24-28.
@@ -63,17 +67,14 @@ struct GemmBars {
 
 // ---------------------------------------------------------------- PTX wrappers
 
-__device__ __forceinline__ void mbar_expect_tx(uint64_t *bar, uint32_t bytes) {
-  asm volatile("mbarrier.expect_tx.relaxed.cta.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(bytes)
-               : "memory");
+// 16-byte asynchronous copy global -> shared; bytes past src_bytes (0 or 16) are zero-filled.
+__device__ __forceinline__ void cp_async16(uint32_t dst, const void *src, uint32_t src_bytes) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src), "r"(src_bytes) : "memory");
 }
-
-__device__ __forceinline__ void tma_load_2d(void *dst, const CUtensorMap *map, int c0, int c1, uint64_t *bar) {
-  asm volatile(
-      "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], "
-      "[%4];" ::"r"(smem_u32(dst)),
-      "l"(reinterpret_cast<uint64_t>(map)), "r"(c0), "r"(c1), "r"(smem_u32(bar))
-      : "memory");
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait() {
+  asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
 }
 
 __device__ __forceinline__ void tmem_alloc(uint32_t *dst, uint32_t ncols) {
@@ -153,22 +154,13 @@ __device__ __forceinline__ void dq_word(uint32_t w, __nv_bfloat162 d2, uint32_t 
   hi23 = cv(h23);
 }
 
-// Raw words of one 18-byte block at global byte address p (2-byte aligned): the 20-byte
-// window starting at p rounded down to 4 bytes. Never reads past the end of a Q4_0 matrix
-// whose rows are whole blocks (the last block of a matrix always starts at 2 mod 4).
+// The 20-byte window holding one 18-byte Q4_0 block (starting at the block's address rounded
+// down to 4 bytes; never past the end of a Q4_0 matrix whose rows are whole blocks, since
+// the last block of a matrix starts at 2 mod 4) and the block's offset in it, in bits.
 struct RawBlk {
   uint32_t w[5];
   uint32_t sh;
 };
-__device__ __forceinline__ RawBlk ld_raw_blk(const uint8_t *p) {
-  RawBlk r;
-  const uintptr_t a = reinterpret_cast<uintptr_t>(p);
-  const uint32_t *wp = reinterpret_cast<const uint32_t *>(a & ~(uintptr_t)3);
-#pragma unroll
-  for (int i = 0; i < 5; ++i) r.w[i] = __ldg(wp + i);
-  r.sh = (uint32_t)(a & 3u) * 8u;
-  return r;
-}
 
 // Decode one block into its 4 swizzled 16-byte chunks of row `row` (chunks cbase..cbase+3).
 __device__ __forceinline__ void store_blk_bf16(const RawBlk &r, uint32_t tile_saddr, int row, int cbase) {
@@ -191,13 +183,13 @@ __device__ __forceinline__ void store_blk_bf16(const RawBlk &r, uint32_t tile_sa
 
 // ---------------------------------------------------------------- the grouped GEMM
 
-// GATEUP: A = gathered x [rows, d], B = gate rows n0..n0+63 and up rows f+n0..f+n0+63,
-//         K = d; epilogue h = gelu(gate) * up -> hb (bf16, padded row order).
-// DOWN:   A = hb [rows, f], B = down rows n0..n0+127, K = f; epilogue y * w * s -> yslot
-//         (bf16, slot order).
+// GATEUP: A = the tokens' rows of x [T, d] (a_src = x), B = gate rows n0..n0+63 and up
+//         rows f+n0..f+n0+63, K = d; epilogue h = gelu(gate) * up -> hb (bf16, padded order).
+// DOWN:   A = hb [padded rows, f] (a_src = hb), B = down rows n0..n0+127, K = f; epilogue
+//         y * w * s -> yslot (bf16, slot order).
 template <bool GATEUP>
 __global__ void __launch_bounds__(kThreads, 1)
-k_moe_gemm(const __grid_constant__ CUtensorMap tmap_a, const uint8_t *__restrict__ wq,
+k_moe_gemm(const __nv_bfloat16 *__restrict__ a_src, const uint8_t *__restrict__ wq, const uint8_t *wq_end,
            const float *__restrict__ expert_scale, int d, int f, int k, MoeWork W) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   __shared__ GemmBars bars;
@@ -215,7 +207,7 @@ k_moe_gemm(const __grid_constant__ CUtensorMap tmap_a, const uint8_t *__restrict
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < kStages; ++s) {
-      mbar_init(&bars.full[s], kProdThreads);
+      mbar_init(&bars.full[s], kGroupThreads);   // the step's producer group arrives
       mbar_init(&bars.empty[s], 1);
     }
     for (int b = 0; b < 2; ++b) {
@@ -236,40 +228,117 @@ k_moe_gemm(const __grid_constant__ CUtensorMap tmap_a, const uint8_t *__restrict
 
   if (warp >= kMmaWarp + 1) {
     // ------------------------------------------------------------ producers
-    const int pt = threadIdx.x - (kMmaWarp + 1) * 32;   // 0..255
-    const int row = pt >> 1, blk = pt & 1;              // one (row, block) of the B tile per step
-    int it = 0;
-    bool ok = true;
-    for (int item = blockIdx.x; item < n_items && ok; item += gridDim.x) {
-      const int tile = item / n_ntiles, nt = item % n_ntiles;
-      const int e = W.tiles[2 * tile];
+    // Producer group pg takes the K steps g with g % kProdGroups == pg. Thread pt of a group
+    // owns row r = pt / 2 of both tiles: A chunks 4 h .. 4 h + 3 (h = pt & 1) of the row's
+    // 128-byte K-step segment, and Q4_0 block h of the row's two blocks per K step.
+    const int pq = threadIdx.x - (kMmaWarp + 1) * 32;
+    const int pg = pq / kGroupThreads, pt = pq - pg * kGroupThreads;   // pt 0..255
+    const int row = pt >> 1, hsel = pt & 1;
+    // the raw Q4_0 bytes of row `row` for a K step (two blocks, 36 bytes) arrive in a 64-byte
+    // window starting at their address rounded down to 16; hsel copies its half of it
+    const uint32_t raw_row = sbase + (uint32_t)kStages * kStageBytes + (uint32_t)row * kRawRowBytes;
+    const int my_items = blockIdx.x < n_items ? (n_items - 1 - (int)blockIdx.x) / (int)gridDim.x + 1 : 0;
+    const int total = my_items * ksteps;
+    // sources of this thread's row for the CTA's jj-th work item: the A row (null past the
+    // expert's rows) and the B row
+    struct RowSrc {
+      const __nv_bfloat16 *arow;
       const uint8_t *wrow;
+    };
+    auto item_src = [&](int jj) -> RowSrc {
+      const int item = (int)blockIdx.x + jj * (int)gridDim.x;
+      const int tile = item / n_ntiles, nt = item - tile * n_ntiles;
+      const int e = W.tiles[2 * tile], m0 = W.tiles[2 * tile + 1];
+      const bool valid = m0 + row < W.counts[e];
+      RowSrc rs;
       if (GATEUP) {
+        rs.arow = valid ? a_src + (size_t)(W.perm[W.offsets[e] + m0 + row] / k) * d : nullptr;
         const int half = BN / 2;
         const int grow = (row < half) ? (nt * half + row) : (f + nt * half + row - half);
-        wrow = wq + (size_t)e * expert_bytes + (size_t)grow * rb;
+        rs.wrow = wq + (size_t)e * expert_bytes + (size_t)grow * rb;
       } else {
-        wrow = wq + (size_t)e * expert_bytes + (size_t)(nt * BN + row) * rb;
+        rs.arow = valid ? a_src + (size_t)(tile * BM + row) * f : nullptr;
+        rs.wrow = wq + (size_t)e * expert_bytes + (size_t)(nt * BN + row) * rb;
       }
-      RawBlk nxt = ld_raw_blk(wrow + (size_t)blk * MOE_QBYTES);
-      for (int ks = 0; ks < ksteps; ++ks, ++it) {
-        const int s = it % kStages;
-        const uint32_t par = ((uint32_t)(it / kStages) & 1u) ^ 1u;
-        if (!mbar_wait(&bars.empty[s], par, W.err, 10)) { ok = false; break; }
-        const uint32_t a_saddr = sbase + (uint32_t)s * kStageBytes;
-        const uint32_t b_saddr = a_saddr + kTileBytes;
-        if (pt == 0) {
-          mbar_expect_tx(&bars.full[s], kTileBytes);
-          tma_load_2d(reinterpret_cast<void *>(smem_raw + (a_saddr - smem_u32(smem_raw))), &tmap_a, ks * BK,
-                      tile * BM, &bars.full[s]);
-        }
-        const RawBlk cur = nxt;
-        if (ks + 1 < ksteps) nxt = ld_raw_blk(wrow + (size_t)((ks + 1) * 2 + blk) * MOE_QBYTES);
-        store_blk_bf16(cur, b_saddr, row, blk * 4);
-        fence_proxy_async_smem();
-        mbar_arrive(&bars.full[s]);
+      return rs;
+    };
+    auto issue = [&](const RowSrc &rs, int ks, int s) {
+      const uint32_t a_saddr = sbase + (uint32_t)s * kStageBytes;
+      const __nv_bfloat16 *ap = rs.arow ? rs.arow + (size_t)ks * BK + (size_t)hsel * (BK / 2) : a_src;
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        const uint32_t chunk = (uint32_t)(hsel * 4 + c);
+        cp_async16(a_saddr + (uint32_t)row * 128u + ((chunk ^ (uint32_t)(row & 7)) << 4), ap + (rs.arow ? 8 * c : 0),
+                   rs.arow ? 16u : 0u);
       }
+      const uintptr_t wa = (reinterpret_cast<uintptr_t>(rs.wrow) + (uintptr_t)ks * 2 * MOE_QBYTES) & ~(uintptr_t)15;
+      const uint32_t rdst = raw_row + (uint32_t)s * kRawStageBytes + (uint32_t)hsel * 32u;
+#pragma unroll
+      for (int c = 0; c < 2; ++c) {
+        const uintptr_t src = wa + (uintptr_t)(hsel * 32 + c * 16);
+        const uintptr_t end = reinterpret_cast<uintptr_t>(wq_end);
+        const uint32_t nbytes = src >= end ? 0u : (end - src >= 16 ? 16u : (uint32_t)(end - src));
+        cp_async16(rdst + 16u * c, reinterpret_cast<const void *>(nbytes ? src : reinterpret_cast<uintptr_t>(wq)),
+                   nbytes);
+      }
+    };
+    bool ok = true;
+    // issue side and consume side walk this group's steps g = pg, pg + G, ... (G groups);
+    // copies run kAhead group steps ahead of the decode
+    constexpr int kAhead = kPrefetch / kProdGroups > 0 ? kPrefetch / kProdGroups : 1;
+    RowSrc isrc{}, csrc{};
+    int ijj = 0, iks = pg, cjj = 0, cks = pg;
+    while (iks >= ksteps && ijj < my_items) { iks -= ksteps; ++ijj; }
+    cjj = ijj;
+    cks = iks;
+    if (ijj < my_items) { isrc = item_src(ijj); csrc = isrc; }
+    auto adv = [&](int &jj, int &ks, RowSrc &src) {
+      ks += kProdGroups;
+      bool moved = false;
+      while (ks >= ksteps) { ks -= ksteps; ++jj; moved = true; }
+      if (moved && jj < my_items) src = item_src(jj);
+    };
+    int gi = pg;
+    for (int a = 0; a < kAhead; ++a, gi += kProdGroups) {   // the first stages are free
+      if (gi < total) {
+        issue(isrc, iks, gi % kStages);
+        adv(ijj, iks, isrc);
+      }
+      cp_async_commit();
     }
+    for (int g = pg; g < total; g += kProdGroups, gi += kProdGroups) {
+      // step g: its copies have landed (issued kAhead group steps ago); decode B, hand over
+      cp_async_wait<kAhead - 1>();
+      __syncwarp();   // the row's window is copied by two lanes
+      const int s = g % kStages;
+      const uint32_t b_saddr = sbase + (uint32_t)s * kStageBytes + kTileBytes;
+      // this thread's block inside the row's window: 20 bytes from its offset rounded down to 4
+      RawBlk cur;
+      {
+        const uintptr_t babs = reinterpret_cast<uintptr_t>(csrc.wrow) + (uintptr_t)(cks * 2 + hsel) * MOE_QBYTES;
+        const uintptr_t wa = (reinterpret_cast<uintptr_t>(csrc.wrow) + (uintptr_t)cks * 2 * MOE_QBYTES) & ~(uintptr_t)15;
+        const uint32_t off = (uint32_t)(babs - wa);   // < 48
+        const uint32_t *rp = reinterpret_cast<const uint32_t *>(smem_raw + (raw_row - smem_u32(smem_raw)) +
+                                                                (size_t)s * kRawStageBytes + (off & ~3u));
+#pragma unroll
+        for (int i = 0; i < 5; ++i) cur.w[i] = rp[i];
+        cur.sh = (off & 3u) * 8u;
+      }
+      store_blk_bf16(cur, b_saddr, row, hsel * 4);
+      fence_proxy_async_smem();
+      mbar_arrive(&bars.full[s]);
+      adv(cjj, cks, csrc);
+      // then refill the stage that step gi uses, once the MMA has released it
+      if (gi < total) {
+        const int si = gi % kStages;
+        const uint32_t par = ((uint32_t)(gi / kStages) & 1u) ^ 1u;
+        if (!mbar_wait(&bars.empty[si], par, W.err, 10)) { ok = false; break; }
+        issue(isrc, iks, si);
+        adv(ijj, iks, isrc);
+      }
+      cp_async_commit();
+    }
+    cp_async_wait<0>();   // no copy lands after this thread leaves
     if (!ok) atomicExch(&bars.abort_flag, 1);
   } else if (warp == kMmaWarp) {
     // ------------------------------------------------------------ MMA issue (one thread)
@@ -374,27 +443,6 @@ k_moe_gemm(const __grid_constant__ CUtensorMap tmap_a, const uint8_t *__restrict
   }
 }
 
-// Gather the routed rows of x into the padded tile order: padded row 128 i + r of tile
-// i = (e, m0) holds x[token of slot perm[offsets[e] + m0 + r]] (zeros past the expert's rows).
-__global__ void __launch_bounds__(256) k_gather_x(const __nv_bfloat16 *__restrict__ x, int d, int k, MoeWork W,
-                                                  __nv_bfloat16 *__restrict__ xg) {
-  const int n_tiles = *W.n_tiles;
-  const int vpr = d / 8;   // 16-byte vectors per row
-  const long long total = (long long)n_tiles * BM * vpr;
-  for (long long i = blockIdx.x * (long long)blockDim.x + threadIdx.x; i < total;
-       i += (long long)gridDim.x * blockDim.x) {
-    const int prow = (int)(i / vpr), v = (int)(i % vpr);
-    const int tile = prow / BM, r = prow % BM;
-    const int e = W.tiles[2 * tile], m0 = W.tiles[2 * tile + 1];
-    uint4 val = make_uint4(0u, 0u, 0u, 0u);
-    if (m0 + r < W.counts[e]) {
-      const int slot = W.perm[W.offsets[e] + m0 + r];
-      val = __ldg(reinterpret_cast<const uint4 *>(x + (size_t)(slot / k) * d) + v);
-    }
-    reinterpret_cast<uint4 *>(xg + (size_t)prow * d)[v] = val;
-  }
-}
-
 // out[t, c] = sum_{j < k} yslot[t k + j, c] (already weighted), j ascending.
 __global__ void __launch_bounds__(256) k_combine(const __nv_bfloat16 *__restrict__ yslot, int T, int d, int k,
                                                  float *__restrict__ out) {
@@ -423,42 +471,11 @@ __global__ void __launch_bounds__(256) k_combine(const __nv_bfloat16 *__restrict
 
 static int launch_err() { return cudaGetLastError() == cudaSuccess ? 0 : -1; }
 
-// Tensor maps over the workspace's padded activation buffers, encoded once per (buffer,
-// shape) through the driver entry point.
-static PFN_cuTensorMapEncodeTiled_v12000 get_encode() {
-  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
-  if (!fn) {
-    cudaDriverEntryPointQueryResult q;
-    void *p = nullptr;
-    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) != cudaSuccess ||
-        q != cudaDriverEntryPointSuccess)
-      return nullptr;
-    fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
-  }
-  return fn;
-}
-
-static bool make_tmap(CUtensorMap *m, const void *base, int cols, long long rows) {
-  auto enc = get_encode();
-  if (!enc) return false;
-  cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
-  cuuint64_t strides[1] = {(cuuint64_t)cols * 2};
-  cuuint32_t box[2] = {(cuuint32_t)BK, (cuuint32_t)BM};
-  cuuint32_t estr[2] = {1, 1};
-  CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(base), dims, strides, box, estr,
-                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-  return r == CUDA_SUCCESS;
-}
-
 int moe_launch_gemm_experts(const MoeLaunch &L, const MoeWork &W, const void *x, const uint8_t *gate_up_q4,
                             const uint8_t *down_q4, const float *expert_scale, int T, int d, int f, int E, int k,
                             float *out, int num_sms, int max_tiles) {
-  (void)E;
+  (void)max_tiles;
   if (d % BK || d % BN || f % BK || f % (BN / 2)) return -2;
-  const long long rows = (long long)max_tiles * BM;
-  CUtensorMap ta, th;
-  if (!make_tmap(&ta, W.xg, d, rows) || !make_tmap(&th, W.hb, f, rows)) return -1;
   static bool attr = false;
   if (!attr) {
     if (cudaFuncSetAttribute(k_moe_gemm<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes) !=
@@ -469,13 +486,14 @@ int moe_launch_gemm_experts(const MoeLaunch &L, const MoeWork &W, const void *x,
     attr = true;
   }
   moe_prof_mark(L.stream, MOE_K_GEMM_GATEUP, true);
-  k_gather_x<<<4 * num_sms, 256, 0, L.stream>>>(static_cast<const __nv_bfloat16 *>(x), d, k, W, W.xg);
-  if (launch_err()) return -1;
-  k_moe_gemm<true><<<num_sms, kThreads, kSmemBytes, L.stream>>>(ta, gate_up_q4, expert_scale, d, f, k, W);
+  const uint8_t *gu_end = gate_up_q4 + (size_t)E * 2 * f * (d / MOE_QK) * MOE_QBYTES;
+  const uint8_t *dn_end = down_q4 + (size_t)E * d * (f / MOE_QK) * MOE_QBYTES;
+  k_moe_gemm<true><<<num_sms, kThreads, kSmemBytes, L.stream>>>(static_cast<const __nv_bfloat16 *>(x), gate_up_q4,
+                                                                 gu_end, expert_scale, d, f, k, W);
   if (launch_err()) return -1;
   moe_prof_mark(L.stream, MOE_K_GEMM_GATEUP, false);
   moe_prof_mark(L.stream, MOE_K_GEMM_DOWN, true);
-  k_moe_gemm<false><<<num_sms, kThreads, kSmemBytes, L.stream>>>(th, down_q4, expert_scale, d, f, k, W);
+  k_moe_gemm<false><<<num_sms, kThreads, kSmemBytes, L.stream>>>(W.hb, down_q4, dn_end, expert_scale, d, f, k, W);
   if (launch_err()) return -1;
   moe_prof_mark(L.stream, MOE_K_GEMM_DOWN, false);
   moe_prof_mark(L.stream, MOE_K_COMBINE, true);

@@ -222,85 +222,200 @@ k_route_decode(const __nv_bfloat16 *__restrict__ x, const float *__restrict__ ro
 
 // ---------------------------------------------------------------- prefill routing
 //
-// Router logits as a tiled FP32 product: 64 tokens x 64 experts per CTA, K steps of 32,
-// 256 threads each owning a 4 x 4 patch. Each K step's 32-term partial is formed in its
-// own register before being added to the running sum (two-level accumulation).
-constexpr int kRgBM = 64, kRgBN = 64, kRgBK = 32;
+// Router logits as a tiled FP32 product: 128 tokens x 128 experts per CTA, 256 threads each
+// owning an 8 x 8 patch, K steps of 16 staged in shared memory (double-buffered), the d axis
+// split in kRgSplit ranges for parallelism. Each output's terms are summed in K order inside
+// its range; k_topk adds the range partials in range order.
+constexpr int kRgM = 128, kRgN = 128, kRgK = 16, kRgSplit = 4;
 
 __global__ void __launch_bounds__(256)
 k_router_gemm(const __nv_bfloat16 *__restrict__ x, const float *__restrict__ router_w, int T, int d, int E,
-              float *__restrict__ logits) {
-  __shared__ float xs[kRgBK][kRgBM + 4];
-  __shared__ float ws[kRgBK][kRgBN + 4];
-  const int t0 = blockIdx.x * kRgBM, e0 = blockIdx.y * kRgBN;
-  const int tx = threadIdx.x % 16, ty = threadIdx.x / 16;
-  float acc[4][4] = {};
-  for (int k0 = 0; k0 < d; k0 += kRgBK) {
-    // load x tile: 64 rows x 32 bf16 -> transposed fp32
-    for (int i = threadIdx.x; i < kRgBM * kRgBK / 4; i += 256) {
-      const int r = i / (kRgBK / 4), c4 = (i % (kRgBK / 4)) * 4;
-      const int t = t0 + r;
-      float v0 = 0.f, v1 = 0.f, v2 = 0.f, v3 = 0.f;
-      if (t < T) {
-        const uint2 xv = __ldg(reinterpret_cast<const uint2 *>(x + (size_t)t * d + k0 + c4));
-        v0 = __uint_as_float(xv.x << 16); v1 = __uint_as_float(xv.x & 0xffff0000u);
-        v2 = __uint_as_float(xv.y << 16); v3 = __uint_as_float(xv.y & 0xffff0000u);
+              float *__restrict__ part /* [kRgSplit][T][E] */) {
+  __shared__ __align__(16) float xs[2][kRgK][kRgM];
+  __shared__ __align__(16) float ws[2][kRgK][kRgN];
+  const int tid = threadIdx.x;
+  const int t0 = blockIdx.x * kRgM, e0 = blockIdx.y * kRgN, split = blockIdx.z;
+  const int nk = d / kRgK;                       // K steps in total (d % 32 == 0)
+  const int k0 = (int)((long long)nk * split / kRgSplit), k1 = (int)((long long)nk * (split + 1) / kRgSplit);
+  const int ty = tid >> 4, tx = tid & 15;        // tokens ty*4 + {0..3}, 64 + ty*4 + {0..3}; experts alike
+  // loaders: x row (tid >> 1), 8 elements at (tid & 1) * 8; W row (tid >> 1), 8 floats
+  const int lr = tid >> 1, lc = (tid & 1) * 8;
+  const int lt = t0 + lr, le = e0 + lr;
+  float acc[8][8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i)
+#pragma unroll
+    for (int j = 0; j < 8; ++j) acc[i][j] = 0.f;
+  auto load = [&](int ks, int buf) {
+    const int kc = ks * kRgK + lc;
+    float xv[8], wv[8];
+    if (lt < T) {
+      const uint4 q = __ldg(reinterpret_cast<const uint4 *>(x + (size_t)lt * d + kc));
+      const uint32_t qq[4] = {q.x, q.y, q.z, q.w};
+#pragma unroll
+      for (int h = 0; h < 4; ++h) {
+        xv[2 * h] = __uint_as_float(qq[h] << 16);
+        xv[2 * h + 1] = __uint_as_float(qq[h] & 0xffff0000u);
       }
-      xs[c4][r] = v0; xs[c4 + 1][r] = v1; xs[c4 + 2][r] = v2; xs[c4 + 3][r] = v3;
+    } else {
+#pragma unroll
+      for (int h = 0; h < 8; ++h) xv[h] = 0.f;
     }
-    for (int i = threadIdx.x; i < kRgBN * kRgBK / 4; i += 256) {
-      const int r = i / (kRgBK / 4), c4 = (i % (kRgBK / 4)) * 4;
-      const int e = e0 + r;
-      float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
-      if (e < E) v = __ldg(reinterpret_cast<const float4 *>(router_w + (size_t)e * d + k0 + c4));
-      ws[c4][r] = v.x; ws[c4 + 1][r] = v.y; ws[c4 + 2][r] = v.z; ws[c4 + 3][r] = v.w;
-    }
-    __syncthreads();
-    float p[4][4] = {};
-#pragma unroll 8
-    for (int kk = 0; kk < kRgBK; ++kk) {
-      float a[4], b[4];
+    if (le < E) {
+      const float4 a = __ldg(reinterpret_cast<const float4 *>(router_w + (size_t)le * d + kc));
+      const float4 b = __ldg(reinterpret_cast<const float4 *>(router_w + (size_t)le * d + kc + 4));
+      wv[0] = a.x; wv[1] = a.y; wv[2] = a.z; wv[3] = a.w; wv[4] = b.x; wv[5] = b.y; wv[6] = b.z; wv[7] = b.w;
+    } else {
 #pragma unroll
-      for (int i = 0; i < 4; ++i) a[i] = xs[kk][ty * 4 + i];
-#pragma unroll
-      for (int j = 0; j < 4; ++j) b[j] = ws[kk][tx * 4 + j];
-#pragma unroll
-      for (int i = 0; i < 4; ++i)
-#pragma unroll
-        for (int j = 0; j < 4; ++j) p[i][j] = fmaf(a[i], b[j], p[i][j]);
+      for (int h = 0; h < 8; ++h) wv[h] = 0.f;
     }
 #pragma unroll
-    for (int i = 0; i < 4; ++i)
+    for (int h = 0; h < 8; ++h) {
+      xs[buf][lc + h][lr] = xv[h];
+      ws[buf][lc + h][lr] = wv[h];
+    }
+  };
+  if (k0 < k1) load(k0, 0);
+  __syncthreads();
+  for (int ks = k0; ks < k1; ++ks) {
+    const int buf = (ks - k0) & 1;
+    if (ks + 1 < k1) load(ks + 1, buf ^ 1);
 #pragma unroll
-      for (int j = 0; j < 4; ++j) acc[i][j] += p[i][j];
+    for (int kk = 0; kk < kRgK; ++kk) {
+      const float4 a0 = *reinterpret_cast<const float4 *>(&xs[buf][kk][ty * 4]);
+      const float4 a1 = *reinterpret_cast<const float4 *>(&xs[buf][kk][64 + ty * 4]);
+      const float4 b0 = *reinterpret_cast<const float4 *>(&ws[buf][kk][tx * 4]);
+      const float4 b1 = *reinterpret_cast<const float4 *>(&ws[buf][kk][64 + tx * 4]);
+      const float a[8] = {a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w};
+      const float bb[8] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
+#pragma unroll
+      for (int i = 0; i < 8; ++i)
+#pragma unroll
+        for (int j = 0; j < 8; ++j) acc[i][j] = fmaf(a[i], bb[j], acc[i][j]);
+    }
     __syncthreads();
   }
+  float *dst = part + (size_t)split * T * E;
 #pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    const int t = t0 + ty * 4 + i;
+  for (int i = 0; i < 8; ++i) {
+    const int t = t0 + (i < 4 ? ty * 4 + i : 64 + ty * 4 + i - 4);
     if (t >= T) continue;
 #pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      const int e = e0 + tx * 4 + j;
-      if (e < E) logits[(size_t)t * E + e] = acc[i][j];
+    for (int j = 0; j < 8; ++j) {
+      const int e = e0 + (j < 4 ? tx * 4 + j : 64 + tx * 4 + j - 4);
+      if (e < E) dst[(size_t)t * E + e] = acc[i][j];
     }
   }
 }
 
+// logits = the kRgSplit range partials added in range order; then top-k + softmax per token
+// (one warp per token).
 __global__ void __launch_bounds__(256)
-k_topk(const float *__restrict__ logits, const float *__restrict__ router_scale, int T, int E, int k,
-       int32_t *ids, float *w) {
-  const int wid = threadIdx.x >> 5;
+k_topk(const float *__restrict__ part, float *__restrict__ logits, const float *__restrict__ router_scale, int T,
+       int E, int k, int32_t *ids, float *w) {
+  const int wid = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int t = blockIdx.x * 8 + wid;
   if (t >= T) return;
+  for (int e = lane; e < E; e += 32) {
+    float v = part[(size_t)t * E + e];
+#pragma unroll
+    for (int sp = 1; sp < kRgSplit; ++sp) v += part[((size_t)sp * T + t) * E + e];
+    logits[(size_t)t * E + e] = v;
+  }
+  __syncwarp();
   warp_topk_softmax(logits + (size_t)t * E, E, k, *router_scale, ids + (size_t)t * k, w + (size_t)t * k);
 }
 
-__global__ void __launch_bounds__(kRouteThreads)
-k_permute(int T, int E, int k, int tile_m, bool want_tiles, MoeWork W) {
-  __shared__ PermSmem sm;
-  block_permutation(W.ids, T * k, E, W.counts, W.offsets, W.perm, W.inv, W.act, W.n_act,
-                    want_tiles ? W.tiles : nullptr, want_tiles ? W.n_tiles : nullptr, W.toff, tile_m, sm);
+// Stable permutation over many CTAs: CTA c owns slots [c * kPermSlots, (c + 1) * kPermSlots).
+// count: per-CTA per-expert counts; scan: expert offsets, active list, tiles and each CTA's
+// output base per expert; place: each slot's position = its CTA's base for its expert + the
+// slots of that expert before it inside the CTA (warps in order, lanes ranked by match_any).
+constexpr int kPermSlots = kRouteThreads;   // one slot per thread
+
+__device__ void cta_warp_counts(const int32_t *ids, int S, int s0, int32_t (*cnt)[MOE_MAX_E]) {
+  const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
+  const int s = s0 + wid * 32 + lane;
+  const int id = s < S ? ids[s] : -1 - lane;
+  const uint32_t peers = __match_any_sync(0xffffffffu, id);
+  if (s < S && lane == 31 - __clz(peers)) cnt[wid][id] = __popc(peers);
+}
+
+__global__ void __launch_bounds__(kRouteThreads) k_perm_count(const int32_t *__restrict__ ids, int S, int E,
+                                                              int32_t *__restrict__ ccnt /* [nc][E] */) {
+  __shared__ int32_t cnt[kRouteWarps][MOE_MAX_E];
+  for (int i = threadIdx.x; i < kRouteWarps * E; i += blockDim.x) cnt[i / E][i % E] = 0;
+  __syncthreads();
+  cta_warp_counts(ids, S, blockIdx.x * kPermSlots, cnt);
+  __syncthreads();
+  for (int e = threadIdx.x; e < E; e += blockDim.x) {
+    int c = 0;
+    for (int w = 0; w < kRouteWarps; ++w) c += cnt[w][e];
+    ccnt[(size_t)blockIdx.x * E + e] = c;
+  }
+}
+
+__global__ void __launch_bounds__(kRouteThreads) k_perm_scan(int nc, int E, int tile_m, bool want_tiles,
+                                                             int32_t *__restrict__ ccnt, MoeWork W) {
+  __shared__ int32_t scan_tmp[kRouteWarps * 3];
+  const int e = threadIdx.x;   // E <= blockDim.x
+  int32_t cnt = 0;
+  if (e < E)
+    for (int c = 0; c < nc; ++c) cnt += ccnt[(size_t)c * E + e];
+  const int32_t a = (e < E) && cnt > 0;
+  const int32_t nt = (e < E && want_tiles) ? (cnt + tile_m - 1) / tile_m : 0;
+  int32_t off, aoff, toff, tot, atot, ttot;
+  block_exclusive_scan3(e < E ? cnt : 0, a, nt, off, aoff, toff, scan_tmp, tot, atot, ttot);
+  if (e < E) {
+    W.counts[e] = cnt;
+    W.offsets[e] = off;
+    if (a) W.act[aoff] = e;
+    int32_t run = off;   // per-CTA output bases for this expert
+    for (int c = 0; c < nc; ++c) {
+      const int32_t v = ccnt[(size_t)c * E + e];
+      ccnt[(size_t)c * E + e] = run;
+      run += v;
+    }
+    if (want_tiles) {
+      W.toff[e] = toff;
+      for (int i = 0; i < nt; ++i) {
+        W.tiles[2 * (toff + i)] = e;
+        W.tiles[2 * (toff + i) + 1] = i * tile_m;
+      }
+    }
+  }
+  if (threadIdx.x == 0) {
+    W.offsets[E] = tot;
+    *W.n_act = atot;
+    if (want_tiles) *W.n_tiles = ttot;
+  }
+}
+
+__global__ void __launch_bounds__(kRouteThreads) k_perm_place(int S, int E, const int32_t *__restrict__ cbase,
+                                                              MoeWork W) {
+  __shared__ int32_t cnt[kRouteWarps][MOE_MAX_E];
+  const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
+  for (int i = threadIdx.x; i < kRouteWarps * E; i += blockDim.x) cnt[i / E][i % E] = 0;
+  __syncthreads();
+  const int s0 = blockIdx.x * kPermSlots;
+  cta_warp_counts(W.ids, S, s0, cnt);
+  __syncthreads();
+  for (int e = threadIdx.x; e < E; e += blockDim.x) {   // per-warp bases inside the CTA
+    int32_t run = cbase[(size_t)blockIdx.x * E + e];
+    for (int w = 0; w < kRouteWarps; ++w) {
+      const int32_t c = cnt[w][e];
+      cnt[w][e] = run;
+      run += c;
+    }
+  }
+  __syncthreads();
+  const int s = s0 + wid * 32 + lane;
+  const int id = s < S ? W.ids[s] : -1 - lane;
+  const uint32_t peers = __match_any_sync(0xffffffffu, id);
+  if (s < S) {
+    const int pos = cnt[wid][id] + __popc(peers & ((1u << lane) - 1u));
+    W.perm[pos] = s;
+    W.inv[s] = pos;
+  }
 }
 
 __global__ void __launch_bounds__(256)
@@ -332,13 +447,24 @@ int moe_launch_route_prefill(const MoeLaunch &L, const MoeWork &W, const void *x
                              const float *router_scale, int T, int d, int E, int k, int num_sms,
                              bool want_xprep, int tile_m) {
   const __nv_bfloat16 *xb = static_cast<const __nv_bfloat16 *>(x);
-  dim3 g1((T + kRgBM - 1) / kRgBM, (E + kRgBN - 1) / kRgBN);
+  if (E > kRouteThreads) return -2;
+  // scratch of the forward's per-slot outputs, free until the expert GEMMs run: the router's
+  // range partials, then the per-CTA expert counts of the permutation
+  float *part = W.ybuf;
+  const int S = T * k;
+  const int nc = (S + kPermSlots - 1) / kPermSlots;
+  int32_t *ccnt = reinterpret_cast<int32_t *>(W.ybuf + (size_t)kRgSplit * T * E);
+  dim3 g1((T + kRgM - 1) / kRgM, (E + kRgN - 1) / kRgN, kRgSplit);
   moe_prof_mark(L.stream, MOE_K_ROUTE, true);
-  k_router_gemm<<<g1, 256, 0, L.stream>>>(xb, router_w, T, d, E, W.logits);
+  k_router_gemm<<<g1, 256, 0, L.stream>>>(xb, router_w, T, d, E, part);
   if (launch_err()) return -1;
-  k_topk<<<(T + 7) / 8, 256, 0, L.stream>>>(W.logits, router_scale, T, E, k, W.ids, W.w);
+  k_topk<<<(T + 7) / 8, 256, 0, L.stream>>>(part, W.logits, router_scale, T, E, k, W.ids, W.w);
   if (launch_err()) return -1;
-  k_permute<<<1, kRouteThreads, 0, L.stream>>>(T, E, k, tile_m, tile_m > 0, W);
+  k_perm_count<<<nc, kRouteThreads, 0, L.stream>>>(W.ids, S, E, ccnt);
+  if (launch_err()) return -1;
+  k_perm_scan<<<1, kRouteThreads, 0, L.stream>>>(nc, E, tile_m, tile_m > 0, ccnt, W);
+  if (launch_err()) return -1;
+  k_perm_place<<<nc, kRouteThreads, 0, L.stream>>>(S, E, ccnt, W);
   if (launch_err()) return -1;
   if (want_xprep) {
     const int nb = d / MOE_QK;
