@@ -100,7 +100,7 @@ Layout make_layout(int maxT, int max_d, int max_f, int max_E, int max_k) {
       (size_t)maxT * max_d * 2,          // 17 xbuf0
       (size_t)maxT * max_d * 2,          // 18 xbuf1
       (size_t)maxT * max_d * 4,          // 19 ylayer
-      prow * max_d * 2,                  // 20 xg (bf16, padded tiles)
+      16,                                // 20 (unused)
       (size_t)max_E * 4,                 // 21 toff
       64,                                // 22 grid-barrier counter
   };
@@ -306,7 +306,6 @@ int moe_init(int device, int max_tokens, int max_d, int max_f, int max_E, int ma
   W.counters = reinterpret_cast<uint32_t *>(b + Lt.off[14]);
   W.hb = reinterpret_cast<__nv_bfloat16 *>(b + Lt.off[15]);
   W.tiles = reinterpret_cast<int32_t *>(b + Lt.off[16]);
-  W.xg = reinterpret_cast<__nv_bfloat16 *>(b + Lt.off[20]);
   W.toff = reinterpret_cast<int32_t *>(b + Lt.off[21]);
   W.gbar = reinterpret_cast<unsigned long long *>(b + Lt.off[22]);
   W.err = ed;

@@ -34,7 +34,6 @@ struct MoeWork {
   uint32_t *counters; // [n] zero-initialised arrival counters (reset by their users)
   volatile uint32_t *err;   // mapped host word: device error code
   // grouped-GEMM path
-  __nv_bfloat16 *xg;  // [tiles*128, d] x rows gathered into the padded tile order
   __nv_bfloat16 *hb;  // [tiles*128, f] bf16 hidden, padded tile order
   float *yslot;       // [T*k, d] per-slot weighted down outputs (bf16 in the GEMM path)
   int32_t *tiles;     // [max tiles] (expert, m0) work list

@@ -24,6 +24,9 @@
 //   warps 5-12 producers: gathered A rows, staged Q4_0 -> bf16 dequantisation for B
 // Shared-memory stages are handed over with mbarriers (every wait is time-bounded); the
 // accumulator is double-buffered in TMEM so the epilogue of one item overlaps the next.
+#include <cuda.h>
+#include <cudaTypedefs.h>
+
 #include "moe_common.cuh"
 
 namespace {
@@ -66,6 +69,19 @@ struct GemmBars {
 };
 
 // ---------------------------------------------------------------- PTX wrappers
+
+__device__ __forceinline__ void mbar_expect_tx(uint64_t *bar, uint32_t bytes) {
+  asm volatile("mbarrier.expect_tx.relaxed.cta.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(bytes)
+               : "memory");
+}
+// 2-D tiled TMA load (no multicast), completion on `bar` in bytes.
+__device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap *map, int c0, int c1, uint64_t *bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], "
+      "[%4];" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(c0), "r"(c1), "r"(smem_u32(bar))
+      : "memory");
+}
 
 // 16-byte asynchronous copy global -> shared; bytes past src_bytes (0 or 16) are zero-filled.
 __device__ __forceinline__ void cp_async16(uint32_t dst, const void *src, uint32_t src_bytes) {
@@ -185,11 +201,12 @@ __device__ __forceinline__ void store_blk_bf16(const RawBlk &r, uint32_t tile_sa
 
 // GATEUP: A = the tokens' rows of x [T, d] (a_src = x), B = gate rows n0..n0+63 and up
 //         rows f+n0..f+n0+63, K = d; epilogue h = gelu(gate) * up -> hb (bf16, padded order).
-// DOWN:   A = hb [padded rows, f] (a_src = hb), B = down rows n0..n0+127, K = f; epilogue
-//         y * w * s -> yslot (bf16, slot order).
+// DOWN:   A = hb [padded rows, f] (tmap_h: 2-D tiles of 128 rows x 64 columns by TMA), B =
+//         down rows n0..n0+127, K = f; epilogue y * w * s -> yslot (bf16, slot order).
 template <bool GATEUP>
 __global__ void __launch_bounds__(kThreads, 1)
-k_moe_gemm(const __nv_bfloat16 *__restrict__ a_src, const uint8_t *__restrict__ wq, const uint8_t *wq_end,
+k_moe_gemm(const __grid_constant__ CUtensorMap tmap_h, const __nv_bfloat16 *__restrict__ a_src,
+           const uint8_t *__restrict__ wq, const uint8_t *wq_end,
            const float *__restrict__ expert_scale, int d, int f, int k, MoeWork W) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   __shared__ GemmBars bars;
@@ -244,6 +261,7 @@ k_moe_gemm(const __nv_bfloat16 *__restrict__ a_src, const uint8_t *__restrict__ 
     struct RowSrc {
       const __nv_bfloat16 *arow;
       const uint8_t *wrow;
+      int tile;
     };
     auto item_src = [&](int jj) -> RowSrc {
       const int item = (int)blockIdx.x + jj * (int)gridDim.x;
@@ -251,25 +269,33 @@ k_moe_gemm(const __nv_bfloat16 *__restrict__ a_src, const uint8_t *__restrict__ 
       const int e = W.tiles[2 * tile], m0 = W.tiles[2 * tile + 1];
       const bool valid = m0 + row < W.counts[e];
       RowSrc rs;
+      rs.tile = tile;
       if (GATEUP) {
         rs.arow = valid ? a_src + (size_t)(W.perm[W.offsets[e] + m0 + row] / k) * d : nullptr;
         const int half = BN / 2;
         const int grow = (row < half) ? (nt * half + row) : (f + nt * half + row - half);
         rs.wrow = wq + (size_t)e * expert_bytes + (size_t)grow * rb;
       } else {
-        rs.arow = valid ? a_src + (size_t)(tile * BM + row) * f : nullptr;
+        rs.arow = nullptr;   // the A tile comes by TMA
         rs.wrow = wq + (size_t)e * expert_bytes + (size_t)(nt * BN + row) * rb;
       }
       return rs;
     };
     auto issue = [&](const RowSrc &rs, int ks, int s) {
       const uint32_t a_saddr = sbase + (uint32_t)s * kStageBytes;
-      const __nv_bfloat16 *ap = rs.arow ? rs.arow + (size_t)ks * BK + (size_t)hsel * (BK / 2) : a_src;
+      if (GATEUP) {
+        const __nv_bfloat16 *ap = rs.arow ? rs.arow + (size_t)ks * BK + (size_t)hsel * (BK / 2) : a_src;
 #pragma unroll
-      for (int c = 0; c < 4; ++c) {
-        const uint32_t chunk = (uint32_t)(hsel * 4 + c);
-        cp_async16(a_saddr + (uint32_t)row * 128u + ((chunk ^ (uint32_t)(row & 7)) << 4), ap + (rs.arow ? 8 * c : 0),
-                   rs.arow ? 16u : 0u);
+        for (int c = 0; c < 4; ++c) {
+          const uint32_t chunk = (uint32_t)(hsel * 4 + c);
+          cp_async16(a_saddr + (uint32_t)row * 128u + ((chunk ^ (uint32_t)(row & 7)) << 4),
+                     ap + (rs.arow ? 8 * c : 0), rs.arow ? 16u : 0u);
+        }
+      } else if (pt == 0) {
+        // the 128 x 64 tile of h by TMA: its bytes join the stage's full barrier, whose phase
+        // cannot complete before this thread's own arrival for the step (after this call)
+        mbar_expect_tx(&bars.full[s], kTileBytes);
+        tma_load_2d(a_saddr, &tmap_h, ks * BK, rs.tile * BM, &bars.full[s]);
       }
       const uintptr_t wa = (reinterpret_cast<uintptr_t>(rs.wrow) + (uintptr_t)ks * 2 * MOE_QBYTES) & ~(uintptr_t)15;
       const uint32_t rdst = raw_row + (uint32_t)s * kRawStageBytes + (uint32_t)hsel * 32u;
@@ -471,10 +497,37 @@ __global__ void __launch_bounds__(256) k_combine(const __nv_bfloat16 *__restrict
 
 static int launch_err() { return cudaGetLastError() == cudaSuccess ? 0 : -1; }
 
+// Tensor map (driver entry point) of the padded h [rows, f] bf16 for the down GEMM's A tiles:
+// box 64 columns x 128 rows, 128-byte swizzle (the layout the MMA descriptors expect).
+static PFN_cuTensorMapEncodeTiled_v12000 get_encode() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  if (!fn) {
+    cudaDriverEntryPointQueryResult q;
+    void *p = nullptr;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) != cudaSuccess ||
+        q != cudaDriverEntryPointSuccess)
+      return nullptr;
+    fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  }
+  return fn;
+}
+
+static bool make_tmap_h(CUtensorMap *m, const void *base, int cols, long long rows) {
+  auto enc = get_encode();
+  if (!enc) return false;
+  cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
+  cuuint64_t strides[1] = {(cuuint64_t)cols * 2};
+  cuuint32_t box[2] = {(cuuint32_t)BK, (cuuint32_t)BM};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(base), dims, strides, box, estr,
+                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
 int moe_launch_gemm_experts(const MoeLaunch &L, const MoeWork &W, const void *x, const uint8_t *gate_up_q4,
                             const uint8_t *down_q4, const float *expert_scale, int T, int d, int f, int E, int k,
                             float *out, int num_sms, int max_tiles) {
-  (void)max_tiles;
   if (d % BK || d % BN || f % BK || f % (BN / 2)) return -2;
   static bool attr = false;
   if (!attr) {
@@ -488,12 +541,15 @@ int moe_launch_gemm_experts(const MoeLaunch &L, const MoeWork &W, const void *x,
   moe_prof_mark(L.stream, MOE_K_GEMM_GATEUP, true);
   const uint8_t *gu_end = gate_up_q4 + (size_t)E * 2 * f * (d / MOE_QK) * MOE_QBYTES;
   const uint8_t *dn_end = down_q4 + (size_t)E * d * (f / MOE_QK) * MOE_QBYTES;
-  k_moe_gemm<true><<<num_sms, kThreads, kSmemBytes, L.stream>>>(static_cast<const __nv_bfloat16 *>(x), gate_up_q4,
-                                                                 gu_end, expert_scale, d, f, k, W);
+  CUtensorMap th;
+  if (!make_tmap_h(&th, W.hb, f, (long long)max_tiles * BM)) return -1;
+  k_moe_gemm<true><<<num_sms, kThreads, kSmemBytes, L.stream>>>(th, static_cast<const __nv_bfloat16 *>(x),
+                                                                 gate_up_q4, gu_end, expert_scale, d, f, k, W);
   if (launch_err()) return -1;
   moe_prof_mark(L.stream, MOE_K_GEMM_GATEUP, false);
   moe_prof_mark(L.stream, MOE_K_GEMM_DOWN, true);
-  k_moe_gemm<false><<<num_sms, kThreads, kSmemBytes, L.stream>>>(W.hb, down_q4, dn_end, expert_scale, d, f, k, W);
+  k_moe_gemm<false><<<num_sms, kThreads, kSmemBytes, L.stream>>>(th, W.hb, down_q4, dn_end, expert_scale, d, f, k,
+                                                                  W);
   if (launch_err()) return -1;
   moe_prof_mark(L.stream, MOE_K_GEMM_DOWN, false);
   moe_prof_mark(L.stream, MOE_K_COMBINE, true);
