@@ -79,6 +79,9 @@ size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
 Layout make_layout(int maxT, int max_d, int max_f, int max_E, int max_k) {
   const size_t S = (size_t)maxT * max_k;
   const size_t prow = (S / kTileM + max_E + 1) * kTileM;   // padded tile rows
+  const size_t ybuf_bytes = S * max_d * 4 > moe_route_scratch_bytes(maxT, max_E, max_k)
+                                ? S * max_d * 4
+                                : moe_route_scratch_bytes(maxT, max_E, max_k);
   const size_t sizes[] = {
       (size_t)maxT * max_E * 4,          // 0 logits
       S * 4,                             // 1 ids
@@ -93,7 +96,7 @@ Layout make_layout(int maxT, int max_d, int max_f, int max_E, int max_k) {
       (size_t)maxT * (max_d / 32) * 8,   // 10 xblk
       S * max_f * 4,                     // 11 h
       16,                                // 12 (unused)
-      S * max_d * 4,                     // 13 ybuf / yslot
+      ybuf_bytes,                        // 13 ybuf / yslot (and routing scratch)
       (size_t)(2 + max_d / 8 + 1024) * 4,   // 14 counters
       prow * max_f * 2,                  // 15 hb (bf16, padded tiles)
       (S / kTileM + max_E + 1) * 8,      // 16 tiles

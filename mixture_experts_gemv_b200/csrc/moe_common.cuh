@@ -207,6 +207,9 @@ void moe_prof_mark(cudaStream_t s, int id, bool begin);
 // Host prototypes of the kernel launchers (defined in the .cu files).
 int moe_launch_route_decode(const MoeLaunch &L, const MoeWork &W, const void *x, const float *router_w,
                             const float *router_scale, int T, int d, int E, int k, int num_sms);
+// Bytes of the ybuf slot the prefill routing uses as scratch (range partials of the router
+// product, then per-CTA expert counts of the permutation).
+size_t moe_route_scratch_bytes(int max_tokens, int max_E, int max_k);
 int moe_launch_route_prefill(const MoeLaunch &L, const MoeWork &W, const void *x, const float *router_w,
                              const float *router_scale, int T, int d, int E, int k, int num_sms,
                              bool want_xprep, int tile_m);

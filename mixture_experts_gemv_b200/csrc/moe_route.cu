@@ -223,10 +223,11 @@ k_route_decode(const __nv_bfloat16 *__restrict__ x, const float *__restrict__ ro
 // ---------------------------------------------------------------- prefill routing
 //
 // Router logits as a tiled FP32 product: 128 tokens x 128 experts per CTA, 256 threads each
-// owning an 8 x 8 patch, K steps of 16 staged in shared memory (double-buffered), the d axis
-// split in kRgSplit ranges for parallelism. Each output's terms are summed in K order inside
-// its range; k_topk adds the range partials in range order.
-constexpr int kRgM = 128, kRgN = 128, kRgK = 16, kRgSplit = 4;
+// owning an 8 x 8 patch, K steps of 16 staged in shared memory (double-buffered: the next
+// step's global loads are in flight during this step's FMAs), the d axis split in kRgSplit
+// ranges for parallelism (32 token tiles x 9 ranges = 288 CTAs, two per SM). Each output's
+// terms are summed in K order inside its range; k_topk adds the range partials in range order.
+constexpr int kRgM = 128, kRgN = 128, kRgK = 16, kRgSplit = 9;
 
 __global__ void __launch_bounds__(256)
 k_router_gemm(const __nv_bfloat16 *__restrict__ x, const float *__restrict__ router_w, int T, int d, int E,
@@ -246,9 +247,9 @@ k_router_gemm(const __nv_bfloat16 *__restrict__ x, const float *__restrict__ rou
   for (int i = 0; i < 8; ++i)
 #pragma unroll
     for (int j = 0; j < 8; ++j) acc[i][j] = 0.f;
-  auto load = [&](int ks, int buf) {
+  float xv[8], wv[8];
+  auto gload = [&](int ks) {   // this thread's share of K step ks, into registers
     const int kc = ks * kRgK + lc;
-    float xv[8], wv[8];
     if (lt < T) {
       const uint4 q = __ldg(reinterpret_cast<const uint4 *>(x + (size_t)lt * d + kc));
       const uint32_t qq[4] = {q.x, q.y, q.z, q.w};
@@ -269,17 +270,22 @@ k_router_gemm(const __nv_bfloat16 *__restrict__ x, const float *__restrict__ rou
 #pragma unroll
       for (int h = 0; h < 8; ++h) wv[h] = 0.f;
     }
+  };
+  auto sstore = [&](int buf) {
 #pragma unroll
     for (int h = 0; h < 8; ++h) {
       xs[buf][lc + h][lr] = xv[h];
       ws[buf][lc + h][lr] = wv[h];
     }
   };
-  if (k0 < k1) load(k0, 0);
+  if (k0 < k1) {
+    gload(k0);
+    sstore(0);
+  }
   __syncthreads();
   for (int ks = k0; ks < k1; ++ks) {
     const int buf = (ks - k0) & 1;
-    if (ks + 1 < k1) load(ks + 1, buf ^ 1);
+    if (ks + 1 < k1) gload(ks + 1);   // lands while this step computes
 #pragma unroll
     for (int kk = 0; kk < kRgK; ++kk) {
       const float4 a0 = *reinterpret_cast<const float4 *>(&xs[buf][kk][ty * 4]);
@@ -293,6 +299,8 @@ k_router_gemm(const __nv_bfloat16 *__restrict__ x, const float *__restrict__ rou
 #pragma unroll
         for (int j = 0; j < 8; ++j) acc[i][j] = fmaf(a[i], bb[j], acc[i][j]);
     }
+    // buffer buf ^ 1 was last read in the previous step, which every thread has left
+    if (ks + 1 < k1) sstore(buf ^ 1);
     __syncthreads();
   }
   float *dst = part + (size_t)split * T * E;
@@ -441,6 +449,12 @@ int moe_launch_route_decode(const MoeLaunch &L, const MoeWork &W, const void *x,
   if (launch_err()) return -1;
   moe_prof_mark(L.stream, MOE_K_ROUTE, false);
   return 0;
+}
+
+size_t moe_route_scratch_bytes(int max_tokens, int max_E, int max_k) {
+  const size_t S = (size_t)max_tokens * max_k;
+  const size_t nc = (S + kPermSlots - 1) / kPermSlots;
+  return ((size_t)kRgSplit * max_tokens * max_E + nc * max_E) * 4;
 }
 
 int moe_launch_route_prefill(const MoeLaunch &L, const MoeWork &W, const void *x, const float *router_w,
