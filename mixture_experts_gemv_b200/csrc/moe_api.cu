@@ -67,7 +67,7 @@ int cuda_fail(cudaError_t e, const char *what) {
   return fail(MOE_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
 }
 
-constexpr int kTileM = 128;   // rows per grouped-GEMM tile
+constexpr int kTileM = MOE_GEMM_TILE_ROWS;   // rows per grouped-GEMM tile
 
 struct Layout {
   size_t off[24];
@@ -91,7 +91,7 @@ Layout make_layout(int maxT, int max_d, int max_f, int max_E, int max_k) {
       S * 4,                             // 5 perm
       S * 4,                             // 6 inv
       (size_t)max_E * 4,                 // 7 act
-      16,                                // 8 n_act, n_tiles
+      16,                                // 8 n_act, n_tiles, n_pairs
       (size_t)maxT * max_d * 2,          // 9 xq
       (size_t)maxT * (max_d / 32) * 8,   // 10 xblk
       S * max_f * 4,                     // 11 h
@@ -103,7 +103,7 @@ Layout make_layout(int maxT, int max_d, int max_f, int max_E, int max_k) {
       (size_t)maxT * max_d * 2,          // 17 xbuf0
       (size_t)maxT * max_d * 2,          // 18 xbuf1
       (size_t)maxT * max_d * 4,          // 19 ylayer
-      16,                                // 20 (unused)
+      (S / kTileM + max_E + 1) * 8,      // 20 tile pairs
       (size_t)max_E * 4,                 // 21 toff
       64,                                // 22 grid-barrier counter
   };
@@ -301,6 +301,8 @@ int moe_init(int device, int max_tokens, int max_d, int max_f, int max_E, int ma
   W.act = reinterpret_cast<int32_t *>(b + Lt.off[7]);
   W.n_act = reinterpret_cast<int32_t *>(b + Lt.off[8]);
   W.n_tiles = reinterpret_cast<int32_t *>(b + Lt.off[8] + 4);
+  W.n_pairs = reinterpret_cast<int32_t *>(b + Lt.off[8] + 8);
+  W.pairs = reinterpret_cast<int32_t *>(b + Lt.off[20]);
   W.xq = reinterpret_cast<int16_t *>(b + Lt.off[9]);
   W.xblk = reinterpret_cast<ActBlk *>(b + Lt.off[10]);
   W.h = reinterpret_cast<float *>(b + Lt.off[11]);

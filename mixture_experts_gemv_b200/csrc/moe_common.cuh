@@ -17,6 +17,10 @@
 #define MOE_DEV_ERR_TIMEOUT 1u
 
 // Routing and scratch produced and consumed inside one forward. All device pointers.
+// Rows per tile of the grouped-GEMM tile list (the routed rows of each expert are padded to
+// whole tiles; tile i covers padded rows [128 i, 128 i + 128)).
+constexpr int MOE_GEMM_TILE_ROWS = 128;
+
 struct MoeWork {
   float *logits;      // [T, E]
   int32_t *ids;       // [T*k]
@@ -40,6 +44,8 @@ struct MoeWork {
   int32_t *toff;      // [E] index of each expert's first tile
   unsigned long long *gbar;   // grid-barrier counter of the fused decode kernel (monotonic)
   int32_t *n_tiles;   // [1]
+  int32_t *pairs;     // [n_pairs][2]: first tile of up to two consecutive tiles of one expert, second present
+  int32_t *n_pairs;   // [1]
 };
 
 // ---------------------------------------------------------------- small helpers

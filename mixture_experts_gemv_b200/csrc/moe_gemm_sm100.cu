@@ -10,20 +10,25 @@
 // followed by out[t] = sum_j w_tj * s_e * Y[slot(t, j)] in j order.
 //
 // Layout: the routed rows of each expert are padded to whole 128-row tiles; tile i of the
-// tile list covers padded rows [128 i, 128 i + 128). The producers gather the A rows
-// (gate_up: the tokens' rows of x; down: the padded rows of h) straight into the 128-byte
-// swizzled K-major tile with 16-byte asynchronous copies (zero-filled past the expert's
-// rows), and copy the raw Q4_0 bytes of the B rows into a staging ring with 4-byte
-// asynchronous copies, several K steps ahead of the MMA. The weights never exist in bf16 in
-// global memory: the producers decode (q - 8) * d from the staged bytes and write the
-// swizzled K-major B tile that tcgen05.mma reads.
+// tile list covers padded rows [128 i, 128 i + 128). A gate_up work item is one tile and one
+// n-tile; a down work item is up to two consecutive tiles of one expert (M = 256 as two
+// 128-row MMA halves sharing the B tile, so the decode work per MMA halves) and one n-tile.
+// The A tile of a K step lands in the 128-byte swizzled K-major layout: gate_up's producers
+// gather the tokens' rows of x with 16-byte asynchronous copies (zero-filled past the
+// expert's rows); down's 128 x 64 tiles of the padded h come by 2-D TMA copies. The raw
+// Q4_0 bytes of the B rows are copied (16-byte asynchronous copies of a 64-byte window per
+// row) into a staging buffer of the stage. The weights never exist in bf16 in global memory:
+// the producers decode (q - 8) * d from the staged bytes and write the swizzled K-major B
+// tile that tcgen05.mma reads.
 //
-// One CTA per SM, persistent over (tile, n-tile) work items, warp-specialised:
-//   warps 0-3  epilogue: tcgen05.ld of the 128 x 128 FP32 accumulator (lane = row)
-//   warp  4    TMEM allocation; lane 0 issues tcgen05.mma (M = 128, N = 128, K = 16)
-//   warps 5-12 producers: gathered A rows, staged Q4_0 -> bf16 dequantisation for B
+// One CTA per SM, persistent over work items, warp-specialised:
+//   warps 0-3  epilogue: tcgen05.ld of the 128 x 128 FP32 accumulators (lane = row)
+//   warp  4    TMEM allocation; lane 0 issues tcgen05.mma (M = 128, N = 128, K = 16, one
+//              per 16-wide K slice and item half)
+//   warps 5-20 producers in two groups taking alternate K steps: A copies (gate_up) or the
+//              TMA issue (down), raw-window copies, Q4_0 -> bf16 dequantisation for B
 // Shared-memory stages are handed over with mbarriers (every wait is time-bounded); the
-// accumulator is double-buffered in TMEM so the epilogue of one item overlaps the next.
+// accumulators are double-buffered in TMEM so the epilogue of one item overlaps the next.
 #include <cuda.h>
 #include <cudaTypedefs.h>
 
@@ -32,7 +37,8 @@
 namespace {
 
 constexpr int BM = 128, BN = 128, BK = 64;
-constexpr int kStages = 5;
+static_assert(BM == MOE_GEMM_TILE_ROWS, "the tile list is built with this tile height");
+constexpr int kMaxStages = 5;
 constexpr int kEpiWarps = 4;
 constexpr int kMmaWarp = 4;
 constexpr int kProdGroups = 2;                                // producer groups take alternate K steps
@@ -40,13 +46,25 @@ constexpr int kProdWarps = 8 * kProdGroups;
 constexpr int kProdThreads = kProdWarps * 32;
 constexpr int kGroupThreads = kProdThreads / kProdGroups;     // one (row, block) of the B tile each
 constexpr int kThreads = (kEpiWarps + 1 + kProdWarps) * 32;
-constexpr uint32_t kTileBytes = BM * BK * 2;                  // 16 KB (A); B is BN x BK, same
-constexpr uint32_t kStageBytes = 2 * kTileBytes;
-constexpr uint32_t kTmemCols = 2 * BN;                        // two accumulator buffers
-constexpr int kPrefetch = kStages - 1;                        // K steps the copies run ahead
+constexpr uint32_t kTileBytes = BM * BK * 2;                  // 16 KB: one A half; B is BN x BK, same
+constexpr int kAhead = 2;                                     // group steps the copies run ahead
 constexpr uint32_t kRawRowBytes = 64;                          // 16-byte-aligned window over a row's 36 bytes
 constexpr uint32_t kRawStageBytes = BN * kRawRowBytes;
-constexpr int kSmemBytes = kStages * (kStageBytes + kRawStageBytes) + 1024;
+
+// Per GEMM: gate_up items are one 128-row tile (its A rows are gathered by the producers);
+// down items are up to two consecutive tiles of one expert, M = 256 as two 128-row halves
+// that share the dequantised B tile (A comes by TMA), so the decode work per MMA halves.
+template <bool GATEUP>
+struct GemmCfg {
+  static constexpr int kHalves = GATEUP ? 1 : 2;
+  static constexpr int kStages = GATEUP ? 5 : 4;
+  static constexpr uint32_t kBOff = kHalves * kTileBytes;        // B tile after the A halves
+  static constexpr uint32_t kStageBytes = kBOff + kTileBytes;
+  static constexpr uint32_t kTmemCols = 2 * kHalves * BN;        // two accumulator buffers
+  static constexpr int kSmemBytes = kStages * (kStageBytes + kRawStageBytes) + 1024;
+  static_assert(kAhead * kProdGroups <= kStages, "the prologue's stages must be free");
+  static_assert(kStages <= kMaxStages && kTmemCols <= 512, "limits");
+};
 
 // UMMA instruction descriptor, kind::f16: D FP32 (bits 4-5 = 1), A and B bf16 (bits 7-9,
 // 10-12 = 1), both K-major (bits 15, 16 = 0), N >> 3 in bits 17-22, M >> 4 in bits 24-28.
@@ -60,8 +78,8 @@ __device__ __forceinline__ uint64_t sw128_desc(uint32_t saddr) {
 }
 
 struct GemmBars {
-  uint64_t full[kStages];
-  uint64_t empty[kStages];
+  uint64_t full[kMaxStages];
+  uint64_t empty[kMaxStages];
   uint64_t acc_full[2];
   uint64_t acc_empty[2];
   uint32_t tmem_base;
@@ -219,8 +237,22 @@ k_moe_gemm(const __grid_constant__ CUtensorMap tmap_h, const __nv_bfloat16 *__re
   const int nb_row = K / MOE_QK;                       // Q4_0 blocks per weight row
   const size_t rb = (size_t)nb_row * MOE_QBYTES;       // bytes per weight row
   const size_t expert_bytes = (size_t)(GATEUP ? 2 * f : d) * rb;
-  const int n_tiles = *W.n_tiles;
-  const int n_items = n_tiles * n_ntiles;
+  using C = GemmCfg<GATEUP>;
+  constexpr int kHalves = C::kHalves, kStages = C::kStages;
+  constexpr uint32_t kBOff = C::kBOff, kStageBytes = C::kStageBytes, kTmemCols = C::kTmemCols;
+  const int n_items = (GATEUP ? *W.n_tiles : *W.n_pairs) * n_ntiles;
+  // work item -> its first tile, and whether a second tile (rows 128 .. 255 past the first
+  // tile's start) belongs to it (down only)
+  auto item_tile = [&](int item, int &tile, bool &h1) {
+    const int q = item / n_ntiles;
+    if (GATEUP) {
+      tile = q;
+      h1 = false;
+    } else {
+      tile = W.pairs[2 * q];
+      h1 = W.pairs[2 * q + 1] != 0;
+    }
+  };
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < kStages; ++s) {
@@ -256,27 +288,35 @@ k_moe_gemm(const __grid_constant__ CUtensorMap tmap_h, const __nv_bfloat16 *__re
     const uint32_t raw_row = sbase + (uint32_t)kStages * kStageBytes + (uint32_t)row * kRawRowBytes;
     const int my_items = blockIdx.x < n_items ? (n_items - 1 - (int)blockIdx.x) / (int)gridDim.x + 1 : 0;
     const int total = my_items * ksteps;
-    // sources of this thread's row for the CTA's jj-th work item: the A row (null past the
-    // expert's rows) and the B row
+    // sources of this thread's rows for the CTA's jj-th work item: the A rows of both halves
+    // (null past the expert's rows; gate_up only), the B row, the tile, and whether the
+    // second half holds any of the expert's rows
     struct RowSrc {
-      const __nv_bfloat16 *arow;
+      const __nv_bfloat16 *arow[kHalves];
       const uint8_t *wrow;
-      int tile;
+      int tile, h1;
     };
     auto item_src = [&](int jj) -> RowSrc {
       const int item = (int)blockIdx.x + jj * (int)gridDim.x;
-      const int tile = item / n_ntiles, nt = item - tile * n_ntiles;
+      const int nt = item % n_ntiles;
+      int tile;
+      bool h1;
+      item_tile(item, tile, h1);
       const int e = W.tiles[2 * tile], m0 = W.tiles[2 * tile + 1];
-      const bool valid = m0 + row < W.counts[e];
+      const int cnt = W.counts[e];
       RowSrc rs;
       rs.tile = tile;
+      rs.h1 = h1;
+#pragma unroll
+      for (int h = 0; h < kHalves; ++h) {
+        const int r = m0 + h * BM + row;
+        rs.arow[h] = (GATEUP && r < cnt) ? a_src + (size_t)(W.perm[W.offsets[e] + r] / k) * d : nullptr;
+      }
       if (GATEUP) {
-        rs.arow = valid ? a_src + (size_t)(W.perm[W.offsets[e] + m0 + row] / k) * d : nullptr;
         const int half = BN / 2;
         const int grow = (row < half) ? (nt * half + row) : (f + nt * half + row - half);
         rs.wrow = wq + (size_t)e * expert_bytes + (size_t)grow * rb;
       } else {
-        rs.arow = nullptr;   // the A tile comes by TMA
         rs.wrow = wq + (size_t)e * expert_bytes + (size_t)(nt * BN + row) * rb;
       }
       return rs;
@@ -284,18 +324,24 @@ k_moe_gemm(const __grid_constant__ CUtensorMap tmap_h, const __nv_bfloat16 *__re
     auto issue = [&](const RowSrc &rs, int ks, int s) {
       const uint32_t a_saddr = sbase + (uint32_t)s * kStageBytes;
       if (GATEUP) {
-        const __nv_bfloat16 *ap = rs.arow ? rs.arow + (size_t)ks * BK + (size_t)hsel * (BK / 2) : a_src;
 #pragma unroll
-        for (int c = 0; c < 4; ++c) {
-          const uint32_t chunk = (uint32_t)(hsel * 4 + c);
-          cp_async16(a_saddr + (uint32_t)row * 128u + ((chunk ^ (uint32_t)(row & 7)) << 4),
-                     ap + (rs.arow ? 8 * c : 0), rs.arow ? 16u : 0u);
+        for (int h = 0; h < kHalves; ++h) {
+          if (h > 0 && !rs.h1) break;   // the MMA skips an empty second half
+          const __nv_bfloat16 *ap = rs.arow[h] ? rs.arow[h] + (size_t)ks * BK + (size_t)hsel * (BK / 2) : a_src;
+          const uint32_t tile_a = a_saddr + (uint32_t)h * kTileBytes;
+#pragma unroll
+          for (int c = 0; c < 4; ++c) {
+            const uint32_t chunk = (uint32_t)(hsel * 4 + c);
+            cp_async16(tile_a + (uint32_t)row * 128u + ((chunk ^ (uint32_t)(row & 7)) << 4),
+                       ap + (rs.arow[h] ? 8 * c : 0), rs.arow[h] ? 16u : 0u);
+          }
         }
       } else if (pt == 0) {
-        // the 128 x 64 tile of h by TMA: its bytes join the stage's full barrier, whose phase
-        // cannot complete before this thread's own arrival for the step (after this call)
-        mbar_expect_tx(&bars.full[s], kTileBytes);
+        // the 128 x 64 tiles of h by TMA: their bytes join the stage's full barrier, whose
+        // phase cannot complete before this thread's own arrival for the step (after this call)
+        mbar_expect_tx(&bars.full[s], kTileBytes * (rs.h1 ? 2u : 1u));
         tma_load_2d(a_saddr, &tmap_h, ks * BK, rs.tile * BM, &bars.full[s]);
+        if (rs.h1) tma_load_2d(a_saddr + kTileBytes, &tmap_h, ks * BK, rs.tile * BM + BM, &bars.full[s]);
       }
       const uintptr_t wa = (reinterpret_cast<uintptr_t>(rs.wrow) + (uintptr_t)ks * 2 * MOE_QBYTES) & ~(uintptr_t)15;
       const uint32_t rdst = raw_row + (uint32_t)s * kRawStageBytes + (uint32_t)hsel * 32u;
@@ -311,7 +357,6 @@ k_moe_gemm(const __grid_constant__ CUtensorMap tmap_h, const __nv_bfloat16 *__re
     bool ok = true;
     // issue side and consume side walk this group's steps g = pg, pg + G, ... (G groups);
     // copies run kAhead group steps ahead of the decode
-    constexpr int kAhead = kPrefetch / kProdGroups > 0 ? kPrefetch / kProdGroups : 1;
     RowSrc isrc{}, csrc{};
     int ijj = 0, iks = pg, cjj = 0, cks = pg;
     while (iks >= ksteps && ijj < my_items) { iks -= ksteps; ++ijj; }
@@ -337,7 +382,7 @@ k_moe_gemm(const __grid_constant__ CUtensorMap tmap_h, const __nv_bfloat16 *__re
       cp_async_wait<kAhead - 1>();
       __syncwarp();   // the row's window is copied by two lanes
       const int s = g % kStages;
-      const uint32_t b_saddr = sbase + (uint32_t)s * kStageBytes + kTileBytes;
+      const uint32_t b_saddr = sbase + (uint32_t)s * kStageBytes + kBOff;
       // this thread's block inside the row's window: 20 bytes from its offset rounded down to 4
       RawBlk cur;
       {
@@ -376,18 +421,25 @@ k_moe_gemm(const __grid_constant__ CUtensorMap tmap_h, const __nv_bfloat16 *__re
         const uint32_t upar = ((uint32_t)(j >> 1) & 1u) ^ 1u;
         if (!mbar_wait(&bars.acc_empty[b], upar, W.err, 11)) { ok = false; break; }
         tc_fence_after();
-        const uint32_t dtm = tmem + (uint32_t)(b * BN);
+        // the second half only where the item holds a second tile
+        int tile;
+        bool h1;
+        item_tile(item, tile, h1);
+        const uint32_t dtm = tmem + (uint32_t)(b * kHalves * BN);
         for (int ks = 0; ks < ksteps; ++ks, ++it) {
           const int s = it % kStages;
           const uint32_t par = (uint32_t)(it / kStages) & 1u;
           if (!mbar_wait(&bars.full[s], par, W.err, 12)) { ok = false; break; }
           tc_fence_after();
           const uint32_t a_saddr = sbase + (uint32_t)s * kStageBytes;
-          const uint32_t b_saddr = a_saddr + kTileBytes;
+          const uint32_t b_saddr = a_saddr + kBOff;
 #pragma unroll
-          for (int kk = 0; kk < BK / 16; ++kk)
-            umma_bf16(dtm, sw128_desc(a_saddr + kk * 32), sw128_desc(b_saddr + kk * 32),
-                      (ks > 0 || kk > 0) ? 1u : 0u);
+          for (int kk = 0; kk < BK / 16; ++kk) {
+            const uint64_t bdesc = sw128_desc(b_saddr + kk * 32);
+            const uint32_t acc = (ks > 0 || kk > 0) ? 1u : 0u;
+            umma_bf16(dtm, sw128_desc(a_saddr + kk * 32), bdesc, acc);
+            if (h1) umma_bf16(dtm + BN, sw128_desc(a_saddr + kTileBytes + kk * 32), bdesc, acc);
+          }
           umma_commit(&bars.empty[s]);
         }
         if (!ok) break;
@@ -398,7 +450,7 @@ k_moe_gemm(const __grid_constant__ CUtensorMap tmap_h, const __nv_bfloat16 *__re
     __syncwarp();
   } else {
     // ------------------------------------------------------------ epilogue (lane = row)
-    const int r = warp * 32 + lane;   // row inside the 128-row tile == TMEM lane
+    const int r = warp * 32 + lane;   // row inside a 128-row half == TMEM lane
     int j = 0;
     for (int item = blockIdx.x; item < n_items; item += gridDim.x, ++j) {
       const int b = j & 1;
@@ -406,53 +458,60 @@ k_moe_gemm(const __grid_constant__ CUtensorMap tmap_h, const __nv_bfloat16 *__re
       const bool ok = mbar_wait(&bars.acc_full[b], par, W.err, 13);
       if (__any_sync(0xffffffffu, !ok)) { atomicExch(&bars.abort_flag, 1); break; }
       tc_fence_after();
-      const int tile = item / n_ntiles, nt = item % n_ntiles;
+      const int nt = item % n_ntiles;
+      int tile;
+      bool h1;
+      item_tile(item, tile, h1);
       const int e = W.tiles[2 * tile], m0 = W.tiles[2 * tile + 1];
       const int cnt = W.counts[e];
-      const bool valid = (m0 + r) < cnt;
-      const uint32_t taddr = tmem + ((uint32_t)(warp * 32) << 16) + (uint32_t)(b * BN);
-      if (GATEUP) {
-        __nv_bfloat16 *dst = W.hb + (size_t)(tile * BM + r) * f + (size_t)nt * (BN / 2);
+      const int nh = h1 ? 2 : 1;   // halves of this item (warp-uniform)
+      for (int h = 0; h < nh; ++h) {
+        const int mr = m0 + h * BM + r;        // row of the expert
+        const bool valid = mr < cnt;
+        const uint32_t taddr = tmem + ((uint32_t)(warp * 32) << 16) + (uint32_t)((b * kHalves + h) * BN);
+        if (GATEUP) {
+          __nv_bfloat16 *dst = W.hb + (size_t)((tile + h) * BM + r) * f + (size_t)nt * (BN / 2);
 #pragma unroll
-        for (int c = 0; c < BN / 2; c += 16) {
-          uint32_t g[16], u[16];
-          tmem_ld16(taddr + (uint32_t)c, g);
-          tmem_ld16(taddr + (uint32_t)(BN / 2 + c), u);
-          tmem_ld_wait();
-          uint32_t o[8];
+          for (int c = 0; c < BN / 2; c += 16) {
+            uint32_t g[16], u[16];
+            tmem_ld16(taddr + (uint32_t)c, g);
+            tmem_ld16(taddr + (uint32_t)(BN / 2 + c), u);
+            tmem_ld_wait();
+            uint32_t o[8];
 #pragma unroll
-          for (int i = 0; i < 8; ++i) {
-            const float h0 = gelu_tanh_f(__uint_as_float(g[2 * i])) * __uint_as_float(u[2 * i]);
-            const float h1 = gelu_tanh_f(__uint_as_float(g[2 * i + 1])) * __uint_as_float(u[2 * i + 1]);
-            o[i] = pack_bf16(h0, h1);
+            for (int i = 0; i < 8; ++i) {
+              const float h0 = gelu_tanh_f(__uint_as_float(g[2 * i])) * __uint_as_float(u[2 * i]);
+              const float hv1 = gelu_tanh_f(__uint_as_float(g[2 * i + 1])) * __uint_as_float(u[2 * i + 1]);
+              o[i] = pack_bf16(h0, hv1);
+            }
+            if (valid) {
+              uint4 *dp = reinterpret_cast<uint4 *>(dst + c);
+              dp[0] = make_uint4(o[0], o[1], o[2], o[3]);
+              dp[1] = make_uint4(o[4], o[5], o[6], o[7]);
+            }
           }
+        } else {
+          int slot = 0;
+          float scale = 0.f;
           if (valid) {
-            uint4 *dp = reinterpret_cast<uint4 *>(dst + c);
-            dp[0] = make_uint4(o[0], o[1], o[2], o[3]);
-            dp[1] = make_uint4(o[4], o[5], o[6], o[7]);
+            slot = W.perm[W.offsets[e] + mr];
+            scale = W.w[slot] * expert_scale[e];
           }
-        }
-      } else {
-        int slot = 0;
-        float scale = 0.f;
-        if (valid) {
-          slot = W.perm[W.offsets[e] + m0 + r];
-          scale = W.w[slot] * expert_scale[e];
-        }
-        __nv_bfloat16 *dst = reinterpret_cast<__nv_bfloat16 *>(W.yslot) + (size_t)slot * d + (size_t)nt * BN;
+          __nv_bfloat16 *dst = reinterpret_cast<__nv_bfloat16 *>(W.yslot) + (size_t)slot * d + (size_t)nt * BN;
 #pragma unroll
-        for (int c = 0; c < BN; c += 16) {
-          uint32_t y[16];
-          tmem_ld16(taddr + (uint32_t)c, y);
-          tmem_ld_wait();
-          uint32_t o[8];
+          for (int c = 0; c < BN; c += 16) {
+            uint32_t y[16];
+            tmem_ld16(taddr + (uint32_t)c, y);
+            tmem_ld_wait();
+            uint32_t o[8];
 #pragma unroll
-          for (int i = 0; i < 8; ++i)
-            o[i] = pack_bf16(__uint_as_float(y[2 * i]) * scale, __uint_as_float(y[2 * i + 1]) * scale);
-          if (valid) {
-            uint4 *dp = reinterpret_cast<uint4 *>(dst + c);
-            dp[0] = make_uint4(o[0], o[1], o[2], o[3]);
-            dp[1] = make_uint4(o[4], o[5], o[6], o[7]);
+            for (int i = 0; i < 8; ++i)
+              o[i] = pack_bf16(__uint_as_float(y[2 * i]) * scale, __uint_as_float(y[2 * i + 1]) * scale);
+            if (valid) {
+              uint4 *dp = reinterpret_cast<uint4 *>(dst + c);
+              dp[0] = make_uint4(o[0], o[1], o[2], o[3]);
+              dp[1] = make_uint4(o[4], o[5], o[6], o[7]);
+            }
           }
         }
       }
@@ -531,10 +590,10 @@ int moe_launch_gemm_experts(const MoeLaunch &L, const MoeWork &W, const void *x,
   if (d % BK || d % BN || f % BK || f % (BN / 2)) return -2;
   static bool attr = false;
   if (!attr) {
-    if (cudaFuncSetAttribute(k_moe_gemm<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes) !=
-            cudaSuccess ||
-        cudaFuncSetAttribute(k_moe_gemm<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes) !=
-            cudaSuccess)
+    if (cudaFuncSetAttribute(k_moe_gemm<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             GemmCfg<true>::kSmemBytes) != cudaSuccess ||
+        cudaFuncSetAttribute(k_moe_gemm<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             GemmCfg<false>::kSmemBytes) != cudaSuccess)
       return -1;
     attr = true;
   }
@@ -543,13 +602,13 @@ int moe_launch_gemm_experts(const MoeLaunch &L, const MoeWork &W, const void *x,
   const uint8_t *dn_end = down_q4 + (size_t)E * d * (f / MOE_QK) * MOE_QBYTES;
   CUtensorMap th;
   if (!make_tmap_h(&th, W.hb, f, (long long)max_tiles * BM)) return -1;
-  k_moe_gemm<true><<<num_sms, kThreads, kSmemBytes, L.stream>>>(th, static_cast<const __nv_bfloat16 *>(x),
-                                                                 gate_up_q4, gu_end, expert_scale, d, f, k, W);
+  constexpr int kSmemG = GemmCfg<true>::kSmemBytes, kSmemD = GemmCfg<false>::kSmemBytes;
+  k_moe_gemm<true><<<num_sms, kThreads, kSmemG, L.stream>>>(th, static_cast<const __nv_bfloat16 *>(x), gate_up_q4,
+                                                            gu_end, expert_scale, d, f, k, W);
   if (launch_err()) return -1;
   moe_prof_mark(L.stream, MOE_K_GEMM_GATEUP, false);
   moe_prof_mark(L.stream, MOE_K_GEMM_DOWN, true);
-  k_moe_gemm<false><<<num_sms, kThreads, kSmemBytes, L.stream>>>(th, W.hb, down_q4, dn_end, expert_scale, d, f, k,
-                                                                  W);
+  k_moe_gemm<false><<<num_sms, kThreads, kSmemD, L.stream>>>(th, W.hb, down_q4, dn_end, expert_scale, d, f, k, W);
   if (launch_err()) return -1;
   moe_prof_mark(L.stream, MOE_K_GEMM_DOWN, false);
   moe_prof_mark(L.stream, MOE_K_COMBINE, true);

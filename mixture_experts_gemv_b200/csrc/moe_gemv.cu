@@ -282,7 +282,7 @@ __global__ void k_hidden_slots_from_bf16(const __nv_bfloat16 *hb, const int32_t 
   for (long long i = blockIdx.x * (long long)blockDim.x + threadIdx.x; i < n; i += (long long)gridDim.x * blockDim.x) {
     const int s = (int)(i / f), c = (int)(i % f);
     const int e = ids[s];
-    const long long prow = (long long)toff[e] * 128 + (inv[s] - offsets[e]);
+    const long long prow = (long long)toff[e] * MOE_GEMM_TILE_ROWS + (inv[s] - offsets[e]);
     h[i] = __bfloat162float(hb[prow * f + c]);
   }
 }

@@ -391,10 +391,23 @@ __global__ void __launch_bounds__(kRouteThreads) k_perm_scan(int nc, int E, int 
       }
     }
   }
+  // the down GEMM's work list: consecutive tiles of one expert in pairs (the last may be alone)
+  const int32_t np = (nt + 1) / 2;
+  int32_t poff, u0, u1, ptot, v0, v1;
+  block_exclusive_scan3(np, 0, 0, poff, u0, u1, scan_tmp, ptot, v0, v1);
+  if (e < E && want_tiles) {
+    for (int i = 0; i < np; ++i) {
+      W.pairs[2 * (poff + i)] = toff + 2 * i;
+      W.pairs[2 * (poff + i) + 1] = 2 * i + 1 < nt ? 1 : 0;
+    }
+  }
   if (threadIdx.x == 0) {
     W.offsets[E] = tot;
     *W.n_act = atot;
-    if (want_tiles) *W.n_tiles = ttot;
+    if (want_tiles) {
+      *W.n_tiles = ttot;
+      *W.n_pairs = ptot;
+    }
   }
 }
 
