@@ -17,6 +17,21 @@
 #define MOE_DEV_ERR_TIMEOUT 1u
 
 // Routing and scratch produced and consumed inside one forward. All device pointers.
+// Decode layout shared by the fused decode kernel and the separate decode kernels, so that
+// both give the same bits and a token's output does not depend on the batch it is decoded in:
+// - router: the d axis of an expert is cut into P = moe_decode_router_parts(d) slices, slice q
+//   = [q s, q s + s) with s = (d / 4) / P * 4 and the last one running to d; lane l of a slice
+//   takes the float4 groups at 4 l + 128 j; lanes are summed by an xor butterfly, slices in
+//   order. P is the fused kernel's warp count (its compute warps, clamped to [8, 12], + 2).
+// - down: a row's blocks are split in MOE_DN_PARTS parts (block pairs first when the row has
+//   an even number of blocks), each summed in block order, the parts summed in order.
+constexpr int MOE_DECODE_MIN_COMPUTE = 8, MOE_DECODE_MAX_COMPUTE = 12;
+constexpr int MOE_DN_PARTS = 5;
+__host__ __device__ inline int moe_decode_router_parts(int d) {
+  const int g = (d / 32 + 7) / 8;   // 8-block granules of a gate_up row
+  return (g < MOE_DECODE_MIN_COMPUTE ? MOE_DECODE_MIN_COMPUTE : (g > MOE_DECODE_MAX_COMPUTE ? MOE_DECODE_MAX_COMPUTE : g)) + 2;
+}
+
 // Rows per tile of the grouped-GEMM tile list (the routed rows of each expert are padded to
 // whole tiles; tile i covers padded rows [128 i, 128 i + 128)).
 constexpr int MOE_GEMM_TILE_ROWS = 128;

@@ -32,6 +32,9 @@ constexpr int kFMaxCompute = 12;   // compute warps (128 registers a thread)
 constexpr int kFMinCompute = 8;
 constexpr int kDnGroups = kDnRows / 32;   // 32-row groups of a down chunk
 constexpr int kDnParts = 5;               // parts of a down row's blocks (work items: groups x parts)
+static_assert(kDnParts == MOE_DN_PARTS && kFMinCompute == MOE_DECODE_MIN_COMPUTE &&
+                  kFMaxCompute == MOE_DECODE_MAX_COMPUTE && kGran == 8,
+              "the separate decode kernels reproduce this kernel's router slices and down parts");
 // Named barriers (0 is __syncthreads): compute warps only; FULL / EMPTY of the two reduction
 // buffers between the compute warps and the epilogue warp; compute + epilogue warps.
 constexpr int kBarCompute = 1;

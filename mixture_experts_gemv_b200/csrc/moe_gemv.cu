@@ -132,8 +132,10 @@ k_gateup_gemv(const uint8_t *__restrict__ gate_up_q4, int d, int f, int k, int n
 
 // ---------------------------------------------------------------- down + combine
 //
-// CTA = 8 warps: warp w owns rows 32 (w & 3) .. + 31 of the chunk and half (w >> 2) of each
-// row's blocks; lane = row. All lanes of a warp read the same hidden values (broadcast).
+// CTA = 8 warps over the work items (32-row group, part of the row's blocks) of a chunk, the
+// parts as in the fused decode kernel (same block split, parts summed in order, so both paths
+// give the same bits); lane = row. All lanes of a warp read the same hidden values
+// (broadcast).
 
 __global__ void __launch_bounds__(kDnThreads, 1)
 k_down_gemv_combine(const uint8_t *__restrict__ down_q4, const float *__restrict__ expert_scale, int T,
@@ -150,7 +152,7 @@ k_down_gemv_combine(const uint8_t *__restrict__ down_q4, const float *__restrict
   uint8_t *smem = align128(smem_raw);
   uint16_t *hs = reinterpret_cast<uint16_t *>(smem + (size_t)nstages * stage_bytes);   // [kTX][f] int16 h
   ActBlk *hblk = reinterpret_cast<ActBlk *>(hs + (size_t)kTX * f);                      // [kTX][nbf]
-  float *red = reinterpret_cast<float *>(hblk + (size_t)kTX * nbf);                     // [2][kTX][kDnRows]
+  float *red = reinterpret_cast<float *>(hblk + (size_t)kTX * nbf);                     // [parts][kTX][kDnRows]
   const int upe = d / kUnit;
   const int n_act = *W.n_act;
   int u0, u1;
@@ -182,7 +184,6 @@ k_down_gemv_combine(const uint8_t *__restrict__ down_q4, const float *__restrict
   }
 
   const int lane = threadIdx.x & 31, wq = threadIdx.x >> 5;
-  float *my_red = red + (size_t)(wq >> 2) * kTX * kDnRows + (wq & 3) * 32 + lane;
   int it = 0;
   for (int u = u0; u < u1; ++it) {
     const DnChunk c = dn_chunk(u, u1, upe);
@@ -219,19 +220,18 @@ k_down_gemv_combine(const uint8_t *__restrict__ down_q4, const float *__restrict
         __syncthreads();
         if (threadIdx.x == 0) { st_key[0] = e; st_key[1] = g0; }
       }
-      if ((wq & 3) * 32 + lane < c.nr) {
-        switch (ng) {
-          case 1: dn_compute<1>(st, rb, nbf, hs, hblk, f, my_red); break;
-          case 2: dn_compute<2>(st, rb, nbf, hs, hblk, f, my_red); break;
-          case 3: dn_compute<3>(st, rb, nbf, hs, hblk, f, my_red); break;
-          default: dn_compute<4>(st, rb, nbf, hs, hblk, f, my_red); break;
-        }
+      switch (ng) {
+        case 1: dn_compute<1>(st, rb, nbf, c.nr, hs, hblk, f, red); break;
+        case 2: dn_compute<2>(st, rb, nbf, c.nr, hs, hblk, f, red); break;
+        case 3: dn_compute<3>(st, rb, nbf, c.nr, hs, hblk, f, red); break;
+        default: dn_compute<4>(st, rb, nbf, c.nr, hs, hblk, f, red); break;
       }
       __syncthreads();
       for (int i2 = threadIdx.x; i2 < kDnRows * ng; i2 += kDnThreads) {
         const int pp = i2 % kDnRows, i = i2 / kDnRows;
         if (pp < c.nr) {
-          const float s = red[(size_t)i * kDnRows + pp] + red[(size_t)(kTX + i) * kDnRows + pp];
+          float s = 0.f;   // the parts in order
+          for (int pt = 0; pt < MOE_DN_PARTS; ++pt) s += red[((size_t)pt * kTX + i) * kDnRows + pp];
           W.ybuf[(size_t)W.perm[off + g0 + i] * d + c.r0 + pp] = s;
         }
       }
@@ -301,7 +301,8 @@ int moe_launch_gemv_experts(const MoeLaunch &L, const MoeWork &W, const uint8_t 
   const size_t gu_stage = (2u * kPairs * (size_t)nb * MOE_QBYTES + 16u + 15u) & ~(size_t)15u;
   const size_t gu_extra = (size_t)kTX * d * 2 + (size_t)kTX * nb * 8 + (size_t)G * 2 * kPairs * kTX * 2 * 4 + 128;
   const size_t dn_stage = ((size_t)kDnRows * nbf * MOE_QBYTES + 16u + 15u) & ~(size_t)15u;
-  const size_t dn_extra = (size_t)kTX * f * 2 + (size_t)kTX * nbf * 8 + (size_t)2 * kTX * kDnRows * 4 + 128;
+  const size_t dn_extra =
+      (size_t)kTX * f * 2 + (size_t)kTX * nbf * 8 + (size_t)MOE_DN_PARTS * kTX * kDnRows * 4 + 128;
   int gu_st = (int)((kSmemBudget - (long long)gu_extra) / (long long)gu_stage);
   int dn_st = (int)((kSmemBudget - (long long)dn_extra) / (long long)dn_stage);
   if (gu_st > kGuStagesMax) gu_st = kGuStagesMax;

@@ -241,38 +241,59 @@ __device__ __forceinline__ DnChunk dn_chunk(int u, int u1, int upe) {
   return c;
 }
 
+// One down-row block against NT slots' staged hidden vectors, accumulated into y[].
 template <int NT>
-__device__ __forceinline__ void dn_compute(const uint8_t *st, uint32_t rb, int nbf, const uint16_t *hs,
-                                           const ActBlk *hb, int f, float *red_out /* [NT] */) {
-  const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
-  const int row = (w & 3) * 32 + lane, part = w >> 2;
-  const int bpp = (nbf + 1) / 2;
-  const int b0 = part * bpp, b1 = min(nbf, b0 + bpp);
-  float y[NT];
+__device__ __forceinline__ void dn_block_acc(const Blk &bk, int b, int nbf, const uint16_t *hs, const ActBlk *hb,
+                                             int f, float (&y)[NT]) {
+  int al[NT], ah[NT];
+  float sc[NT];
 #pragma unroll
-  for (int i = 0; i < NT; ++i) y[i] = 0.f;
-  const uint32_t orow = (uint32_t)row * rb;
-  for (int b = b0; b < b1; ++b) {
-    const Blk bk = load_blk(st, orow + (uint32_t)b * MOE_QBYTES);
-    int al[NT], ah[NT];
-    float sc[NT];
-#pragma unroll
-    for (int i = 0; i < NT; ++i) {
-      const ActBlk ab = hb[i * nbf + b];
-      al[i] = ab.neg8sum; ah[i] = 0; sc[i] = ab.scale;
-    }
-#pragma unroll
-    for (int wi = 0; wi < 4; ++wi) {
-      const uint32_t lo = bk.q[wi] & 0x0F0F0F0Fu, hi = bk.q[wi] & 0xF0F0F0F0u;
-#pragma unroll
-      for (int i = 0; i < NT; ++i)
-        dot8i(lo, hi, *reinterpret_cast<const uint4 *>(hs + (size_t)i * f + b * MOE_QK + 8 * wi), al[i], ah[i]);
-    }
-#pragma unroll
-    for (int i = 0; i < NT; ++i) y[i] = block_finish(y[i], bk.d, sc[i], al[i], ah[i]);
+  for (int i = 0; i < NT; ++i) {
+    const ActBlk ab = hb[i * nbf + b];
+    al[i] = ab.neg8sum; ah[i] = 0; sc[i] = ab.scale;
   }
 #pragma unroll
-  for (int i = 0; i < NT; ++i) red_out[i * kDnRows] = y[i];
+  for (int wi = 0; wi < 4; ++wi) {
+    const uint32_t lo = bk.q[wi] & 0x0F0F0F0Fu, hi = bk.q[wi] & 0xF0F0F0F0u;
+#pragma unroll
+    for (int i = 0; i < NT; ++i)
+      dot8i(lo, hi, *reinterpret_cast<const uint4 *>(hs + (size_t)i * f + b * MOE_QK + 8 * wi), al[i], ah[i]);
+  }
+#pragma unroll
+  for (int i = 0; i < NT; ++i) y[i] = block_finish(y[i], bk.d, sc[i], al[i], ah[i]);
+}
+
+// Down rows of a staged chunk (nr rows) for NT slots, by every warp of the CTA: work items
+// (32-row group, part) with the row's blocks split in MOE_DN_PARTS parts exactly as the fused
+// decode kernel splits them (block pairs first when the row has an even number of blocks,
+// leftovers one each to the first parts; otherwise contiguous ranges); lane = row.
+// red_out[(part * kTX + i) * kDnRows + row].
+template <int NT>
+__device__ __forceinline__ void dn_compute(const uint8_t *st, uint32_t rb, int nbf, int nr, const uint16_t *hs,
+                                           const ActBlk *hb, int f, float *red_out) {
+  constexpr int P = MOE_DN_PARTS;
+  const int lane = threadIdx.x & 31, w = threadIdx.x >> 5, nw = blockDim.x >> 5;
+  for (int item = w; item < (kDnRows / 32) * P; item += nw) {
+    const int grp = item % (kDnRows / 32), part = item / (kDnRows / 32);
+    const int row = grp * 32 + lane;
+    if (row >= nr) continue;
+    float y[NT];
+#pragma unroll
+    for (int i = 0; i < NT; ++i) y[i] = 0.f;
+    const uint32_t orow = (uint32_t)row * rb;
+    if ((nbf & 1) == 0) {
+      const int per = nbf / (2 * P);   // block pairs per part
+      for (int b = 2 * part * per; b < 2 * (part + 1) * per; ++b)
+        dn_block_acc<NT>(load_blk(st, orow + (uint32_t)b * MOE_QBYTES), b, nbf, hs, hb, f, y);
+      for (int b = 2 * P * per + part; b < nbf; b += P)
+        dn_block_acc<NT>(load_blk(st, orow + (uint32_t)b * MOE_QBYTES), b, nbf, hs, hb, f, y);
+    } else {
+      for (int b = part * nbf / P; b < (part + 1) * nbf / P; ++b)
+        dn_block_acc<NT>(load_blk(st, orow + (uint32_t)b * MOE_QBYTES), b, nbf, hs, hb, f, y);
+    }
+#pragma unroll
+    for (int i = 0; i < NT; ++i) red_out[((size_t)part * kTX + i) * kDnRows + row] = y[i];
+  }
 }
 
 }  // namespace

@@ -12,8 +12,6 @@ namespace {
 
 constexpr int kRouteThreads = 512;             // 16 warps
 constexpr int kRouteWarps = kRouteThreads / 32;
-constexpr int kRouteParts = 8;                 // d split in 8 parts per expert (decode)
-constexpr int kRouteEPC = kRouteWarps / kRouteParts;   // experts per CTA
 constexpr int kDecodeMaxT = 16;
 
 // ---------------------------------------------------------------- permutation (one CTA)
@@ -130,12 +128,13 @@ __device__ void block_permutation(const int32_t *ids, int S, int E, int32_t *cou
 
 // ---------------------------------------------------------------- decode routing kernel
 //
-// T <= 16. CTA b handles kRouteEPC experts, each split in kRouteParts parts of d; warp
-// (expert, part) accumulates lane-strided float4 chunks of W_r against every token, reduces
-// across the warp by a fixed xor tree, and the parts are summed in order. The last CTA to
-// finish (arrival counter) runs top-k + softmax for all tokens and the permutation.
+// T <= 16. CTA b handles epc = kRouteWarps / P experts, each cut in the P slices of d that the
+// fused decode kernel uses (moe_common.cuh): warp (expert, slice) accumulates lane-strided
+// float4 chunks of W_r against every token, reduces across the warp by a fixed xor tree, and
+// the slices are summed in order, so the logits are the fused kernel's bit for bit. The last
+// CTA to finish (arrival counter) runs top-k + softmax for all tokens and the permutation.
 struct RouteDecodeSmem {
-  float part[kRouteEPC][kRouteParts][kDecodeMaxT];
+  float part[kRouteWarps][kDecodeMaxT];
   union {
     PermSmem perm;
     int32_t cnt[MOE_MAX_E];
@@ -143,26 +142,27 @@ struct RouteDecodeSmem {
   int last;
 };
 
-__global__ void __launch_bounds__(kRouteThreads)
+__global__ void __launch_bounds__(kRouteThreads, 1)
 k_route_decode(const __nv_bfloat16 *__restrict__ x, const float *__restrict__ router_w,
                const float *__restrict__ router_scale, int T, int d, int E, int k, MoeWork W) {
   __shared__ RouteDecodeSmem sm;
   const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
-  const int el = wid / kRouteParts, part = wid % kRouteParts;
-  const int e = blockIdx.x * kRouteEPC + el;
-  const int plen = d / kRouteParts;   // multiple of 4
-  if (e < E) {
+  const int P = moe_decode_router_parts(d), epc = kRouteWarps / P;
+  const int el = wid / P, part = wid % P;
+  const int e = blockIdx.x * epc + el;
+  const int seg = (d / 4) / P * 4;   // float4-aligned slice; the last slice takes the tail
+  const int i0 = part * seg, i1 = (part == P - 1) ? d : i0 + seg;
+  if (el < epc && e < E) {
     float acc[kDecodeMaxT];
 #pragma unroll
     for (int t = 0; t < kDecodeMaxT; ++t) acc[t] = 0.f;
-    const float *wr = router_w + (size_t)e * d + (size_t)part * plen;
-    const __nv_bfloat16 *xp = x + (size_t)part * plen;
-    for (int i = lane * 4; i < plen; i += 128) {
+    const float *wr = router_w + (size_t)e * d;
+    for (int i = i0 + lane * 4; i + 3 < i1; i += 128) {
       const float4 wv = __ldg(reinterpret_cast<const float4 *>(wr + i));
 #pragma unroll
       for (int t = 0; t < kDecodeMaxT; ++t) {
         if (t < T) {
-          const uint2 xv = __ldg(reinterpret_cast<const uint2 *>(xp + (size_t)t * d + i));
+          const uint2 xv = __ldg(reinterpret_cast<const uint2 *>(x + (size_t)t * d + i));
           const float x0 = __uint_as_float(xv.x << 16), x1 = __uint_as_float(xv.x & 0xffff0000u);
           const float x2 = __uint_as_float(xv.y << 16), x3 = __uint_as_float(xv.y & 0xffff0000u);
           float a = acc[t];
@@ -179,19 +179,18 @@ k_route_decode(const __nv_bfloat16 *__restrict__ x, const float *__restrict__ ro
       float a = acc[t];
 #pragma unroll
       for (int o = 16; o > 0; o >>= 1) a += __shfl_xor_sync(0xffffffffu, a, o);
-      if (lane == 0) sm.part[el][part][t] = a;
+      if (lane == 0) sm.part[wid][t] = a;
     }
   }
   prep_x_range(x, W.xq, W.xblk, T, d, blockIdx.x * blockDim.x + threadIdx.x,
                gridDim.x * blockDim.x);
   __syncthreads();
-  if (threadIdx.x < kRouteEPC * kDecodeMaxT) {
+  if (threadIdx.x < epc * kDecodeMaxT) {
     const int le = threadIdx.x / kDecodeMaxT, t = threadIdx.x % kDecodeMaxT;
-    const int ee = blockIdx.x * kRouteEPC + le;
+    const int ee = blockIdx.x * epc + le;
     if (ee < E && t < T) {
-      float s = sm.part[le][0][t];
-#pragma unroll
-      for (int p = 1; p < kRouteParts; ++p) s += sm.part[le][p][t];
+      float s = 0.f;
+      for (int p = 0; p < P; ++p) s += sm.part[le * P + p][t];
       W.logits[(size_t)t * E + ee] = s;
     }
   }
@@ -454,8 +453,9 @@ int moe_launch_route_decode(const MoeLaunch &L, const MoeWork &W, const void *x,
                             const float *router_scale, int T, int d, int E, int k, int num_sms) {
   (void)num_sms;
   if (T > kDecodeMaxT) return -2;
-  if ((d / kRouteParts) % 4) return -2;
-  const int grid = (E + kRouteEPC - 1) / kRouteEPC;
+  const int P = moe_decode_router_parts(d), epc = kRouteWarps / P;
+  if (d % 32 || epc < 1) return -2;
+  const int grid = (E + epc - 1) / epc;
   moe_prof_mark(L.stream, MOE_K_ROUTE, true);
   k_route_decode<<<grid, kRouteThreads, 0, L.stream>>>(static_cast<const __nv_bfloat16 *>(x), router_w,
                                                         router_scale, T, d, E, k, W);

@@ -176,6 +176,25 @@ def test_deterministic_bitwise():
     assert np.array_equal(a.view(np.uint32), b.view(np.uint32))
 
 
+def test_batch_invariant_decode():
+    """A token's output does not depend on the other tokens of the call, for every T the
+    GEMV path takes (T <= 8: the fused decode kernel; 9 <= T <= 16: the separate decode
+    kernels, which cut the router and the down rows as the fused kernel does): the verification
+    pass of speculative decoding must give plain decoding's logits bit for bit (page "Gemma 4
+    26B-A4B it QAT Q4_0 ... NInfer v3 artifact", "Speculative decoding", "Quality"). Singles,
+    pairs, fours, eights, twelves and the reversed batch against the batch of sixteen."""
+    E, d, f, k = 64, 1024, 256, 8
+    lw = mi.make_layer(seed=21, d=d, f=f, E=E)
+    x = mi.make_tokens(22, 16, d)
+    dl = DevLayer(lw)
+    full = run_layer(x, dl, k, moe.MOE_PATH_AUTO, want_routing=False)["out"].view(np.uint32)
+    subsets = ([0], [5], [15], [0, 1], [14, 2], [2, 3, 4, 5], [9, 1, 12, 7], list(range(8)),
+               list(range(8, 16)), list(range(9)), list(range(3, 15)), list(range(15, -1, -1)))
+    for sel in subsets:
+        part = run_layer(x[sel], dl, k, moe.MOE_PATH_AUTO, want_routing=False)["out"].view(np.uint32)
+        assert np.array_equal(part, full[sel]), sel
+
+
 def test_hidden_matches_oracle():
     E, d, f, k, T = 16, 256, 96, 3, 5
     lw = mi.make_layer(seed=12, d=d, f=f, E=E)
