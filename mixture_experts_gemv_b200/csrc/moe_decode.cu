@@ -446,28 +446,46 @@ k_moe_decode(const __nv_bfloat16 *__restrict__ x, const float *__restrict__ rout
   const float rs = __ldg(router_scale);
 
   // ---------------------------------------------------------------- phase 0: router
+  // A lane loads its router weights first (up to kRtrW float4 groups at once: their HBM
+  // latency overlaps), then multiplies them with x from the shared-memory copy; the terms are
+  // summed in the same order as a one-group-at-a-time loop (the separate router's order).
+  constexpr int kRtrW = 4;
   for (int e = blockIdx.x; e < E; e += gridDim.x) {
-    float acc[kFMaxT];
-#pragma unroll
-    for (int t = 0; t < kFMaxT; ++t) acc[t] = 0.f;
     const int seg = (d / 4) / nw * 4;   // float4-aligned slice per warp; the last warp takes the tail
     const int i0 = wq * seg, i1 = (wq == nw - 1) ? d : i0 + seg;
     const float *wr = router_w + (size_t)e * d;
-    for (int i = i0 + lane * 4; i + 3 < i1; i += 128) {
-      const float4 wv = __ldg(reinterpret_cast<const float4 *>(wr + i));
+    float4 wv[kRtrW];
+#pragma unroll
+    for (int j = 0; j < kRtrW; ++j) {
+      const int i = i0 + lane * 4 + 128 * j;
+      wv[j] = (i + 3 < i1) ? __ldg(reinterpret_cast<const float4 *>(wr + i)) : make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+    __syncthreads();   // the x copy's mbarrier is initialised; sh.part is free
+    wait_phase(&sh.xbar, 0u, &sh.abort, W.err, 26);
+    float acc[kFMaxT];
+#pragma unroll
+    for (int t = 0; t < kFMaxT; ++t) acc[t] = 0.f;
+    auto mac = [&](const float4 &w4, int i) {
 #pragma unroll
       for (int t = 0; t < kFMaxT; ++t) {
         if (t < T) {
-          const uint2 xv = __ldg(reinterpret_cast<const uint2 *>(x + (size_t)t * d + i));
+          const uint2 xv = *reinterpret_cast<const uint2 *>(xs + (size_t)t * d + i);
           float a = acc[t];
-          a = fmaf(wv.x, __uint_as_float(xv.x << 16), a);
-          a = fmaf(wv.y, __uint_as_float(xv.x & 0xffff0000u), a);
-          a = fmaf(wv.z, __uint_as_float(xv.y << 16), a);
-          a = fmaf(wv.w, __uint_as_float(xv.y & 0xffff0000u), a);
+          a = fmaf(w4.x, __uint_as_float(xv.x << 16), a);
+          a = fmaf(w4.y, __uint_as_float(xv.x & 0xffff0000u), a);
+          a = fmaf(w4.z, __uint_as_float(xv.y << 16), a);
+          a = fmaf(w4.w, __uint_as_float(xv.y & 0xffff0000u), a);
           acc[t] = a;
         }
       }
+    };
+#pragma unroll
+    for (int j = 0; j < kRtrW; ++j) {
+      const int i = i0 + lane * 4 + 128 * j;
+      if (i + 3 < i1) mac(wv[j], i);
     }
+    for (int i = i0 + lane * 4 + 128 * kRtrW; i + 3 < i1; i += 128)
+      mac(__ldg(reinterpret_cast<const float4 *>(wr + i)), i);
 #pragma unroll
     for (int t = 0; t < kFMaxT; ++t) {
       float a = acc[t];
