@@ -358,9 +358,45 @@ __device__ __forceinline__ void dn_block(const Blk &bk, int b, const uint16_t *h
   for (int i = 0; i < NT; ++i) y[i] = block_finish(y[i], bk.d, sc[i], al[i], ah[i]);
 }
 
+// One block of two down rows (k0, k1) against NT slots' staged hidden vectors: dn_block for
+// each row, with one activation load serving both.
+template <int NT>
+__device__ __forceinline__ void dn_block2(const Blk &k0, const Blk &k1, int b, const uint16_t *hs, const ActBlk *hbk,
+                                          const uint32_t (&ho)[NT], const uint32_t (&bo)[NT], float (&y0)[NT],
+                                          float (&y1)[NT]) {
+  int al0[NT], ah0[NT], al1[NT], ah1[NT];
+  float sc[NT];
+#pragma unroll
+  for (int i = 0; i < NT; ++i) {
+    const ActBlk ab = hbk[bo[i] + b];
+    al0[i] = ab.neg8sum;
+    al1[i] = ab.neg8sum;
+    ah0[i] = 0;
+    ah1[i] = 0;
+    sc[i] = ab.scale;
+  }
+#pragma unroll
+  for (int wi = 0; wi < 4; ++wi) {
+    const uint32_t lo0 = k0.q[wi] & 0x0F0F0F0Fu, hi0 = k0.q[wi] & 0xF0F0F0F0u;
+    const uint32_t lo1 = k1.q[wi] & 0x0F0F0F0Fu, hi1 = k1.q[wi] & 0xF0F0F0F0u;
+#pragma unroll
+    for (int i = 0; i < NT; ++i) {
+      const uint4 xv = *reinterpret_cast<const uint4 *>(hs + ho[i] + b * MOE_QK + 8 * wi);
+      dot8i(lo0, hi0, xv, al0[i], ah0[i]);
+      dot8i(lo1, hi1, xv, al1[i], ah1[i]);
+    }
+  }
+#pragma unroll
+  for (int i = 0; i < NT; ++i) {
+    y0[i] = block_finish(y0[i], k0.d, sc[i], al0[i], ah0[i]);
+    y1[i] = block_finish(y1[i], k1.d, sc[i], al1[i], ah1[i]);
+  }
+}
+
 // down pass over one staged chunk (up to kDnRows rows) for NT slots, by the compute warps:
-// items first, first + nwc, ... Work item = (32-row group, part of the row's
-// blocks), lane = row; red_b[(part * kTX + i) * kDnRows + row]. With PAIRED
+// items first, first + nwc, ... Work item = (pair of 32-row groups g2 and g2 + 2, part of the
+// row's blocks); the lane takes one row of each group (an activation load serves both);
+// red_b[(part * kTX + i) * kDnRows + row]. With PAIRED
 // (an even number of blocks per row, so every row starts 4-byte aligned) a part takes whole
 // block pairs and the blocks left over go one each to the first parts; otherwise parts are
 // contiguous block ranges read block by block.
@@ -374,35 +410,39 @@ __device__ __forceinline__ void dn_pass(const uint8_t *st, uint32_t rb, int nbf,
     ho[i] = (uint32_t)((rel0 + i) * f);
     bo[i] = (uint32_t)((rel0 + i) * nbf);
   }
-  for (int item = first; item < kDnGroups * P; item += nwc) {
-    const int grp = item % kDnGroups, part = item / kDnGroups;
-    const int row = grp * 32 + lane;
-    if (grp * 32 >= nr) continue;   // warp-uniform: this row group is past the chunk
-    float y[NT];
+  // work item = (row-group pair g2, part): the lane takes rows g2 * 32 + lane and that + 64
+  for (int item = first; item < 2 * P; item += nwc) {
+    const int g2 = item & 1, part = item >> 1;
+    if (g2 * 32 >= nr) continue;   // warp-uniform: these rows are past the chunk
+    const int r0 = g2 * 32 + lane, r1 = r0 + 64;
+    const bool v0 = r0 < nr, v1 = r1 < nr;
+    float y0[NT], y1[NT];
 #pragma unroll
-    for (int i = 0; i < NT; ++i) y[i] = 0.f;
-    if (row < nr) {
-      const uint32_t orow = (uint32_t)row * rb;
-      if (PAIRED) {
-        const int per = nbf / (2 * P);   // pairs per part
-        for (int pr = part * per; pr < (part + 1) * per; ++pr) {
-          Blk k0, k1;
-          load_pair_w(st, orow + (uint32_t)(2 * pr) * MOE_QBYTES, k0, k1);
-          dn_block<NT>(k0, 2 * pr, hs, hbk, ho, bo, y);
-          dn_block<NT>(k1, 2 * pr + 1, hs, hbk, ho, bo, y);
-        }
-        for (int b = 2 * P * per + part; b < nbf; b += P) {
-          const Blk kb = load_blk(st, orow + (uint32_t)b * MOE_QBYTES);
-          dn_block<NT>(kb, b, hs, hbk, ho, bo, y);
-        }
-      } else {
-        for (int b = part * nbf / P; b < (part + 1) * nbf / P; ++b) {
-          const Blk kb = load_blk(st, orow + (uint32_t)b * MOE_QBYTES);
-          dn_block<NT>(kb, b, hs, hbk, ho, bo, y);
-        }
+    for (int i = 0; i < NT; ++i) { y0[i] = 0.f; y1[i] = 0.f; }
+    const uint32_t o0 = (uint32_t)(v0 ? r0 : 0) * rb, o1 = (uint32_t)(v1 ? r1 : 0) * rb;   // in the stage
+    if (PAIRED) {
+      const int per = nbf / (2 * P);   // pairs per part
+      for (int pr = part * per; pr < (part + 1) * per; ++pr) {
+        Blk a0, a1, c0, c1;
+        load_pair_w(st, o0 + (uint32_t)(2 * pr) * MOE_QBYTES, a0, a1);
+        load_pair_w(st, o1 + (uint32_t)(2 * pr) * MOE_QBYTES, c0, c1);
+        dn_block2<NT>(a0, c0, 2 * pr, hs, hbk, ho, bo, y0, y1);
+        dn_block2<NT>(a1, c1, 2 * pr + 1, hs, hbk, ho, bo, y0, y1);
       }
+      for (int b = 2 * P * per + part; b < nbf; b += P) {
+        const Blk a = load_blk(st, o0 + (uint32_t)b * MOE_QBYTES), c = load_blk(st, o1 + (uint32_t)b * MOE_QBYTES);
+        dn_block2<NT>(a, c, b, hs, hbk, ho, bo, y0, y1);
+      }
+    } else {
+      for (int b = part * nbf / P; b < (part + 1) * nbf / P; ++b) {
+        const Blk a = load_blk(st, o0 + (uint32_t)b * MOE_QBYTES), c = load_blk(st, o1 + (uint32_t)b * MOE_QBYTES);
+        dn_block2<NT>(a, c, b, hs, hbk, ho, bo, y0, y1);
+      }
+    }
 #pragma unroll
-      for (int i = 0; i < NT; ++i) red_b[((size_t)part * kTX + i) * kDnRows + row] = y[i];
+    for (int i = 0; i < NT; ++i) {
+      if (v0) red_b[((size_t)part * kTX + i) * kDnRows + r0] = y0[i];
+      if (v1) red_b[((size_t)part * kTX + i) * kDnRows + r1] = y1[i];
     }
   }
 }
