@@ -30,7 +30,6 @@ constexpr int kFMaxE = 256;
 constexpr int kFStages = 3;
 constexpr int kFMaxCompute = 12;   // compute warps (128 registers a thread)
 constexpr int kFMinCompute = 8;
-constexpr int kDnGroups = kDnRows / 32;   // 32-row groups of a down chunk
 constexpr int kDnParts = 5;               // parts of a down row's blocks (work items: groups x parts)
 static_assert(kDnParts == MOE_DN_PARTS && kFMinCompute == MOE_DECODE_MIN_COMPUTE &&
                   kFMaxCompute == MOE_DECODE_MAX_COMPUTE && kGran == 8,
@@ -334,32 +333,9 @@ __device__ __forceinline__ void load_pair_w(const uint8_t *smem, uint32_t o, Blk
   split_blk2(w, b0, b1);
 }
 
-// One down-row block against NT slots' staged hidden vectors.
-template <int NT>
-__device__ __forceinline__ void dn_block(const Blk &bk, int b, const uint16_t *hs, const ActBlk *hbk,
-                                         const uint32_t (&ho)[NT], const uint32_t (&bo)[NT], float (&y)[NT]) {
-  int al[NT], ah[NT];
-  float sc[NT];
-#pragma unroll
-  for (int i = 0; i < NT; ++i) {
-    const ActBlk ab = hbk[bo[i] + b];
-    al[i] = ab.neg8sum;
-    ah[i] = 0;
-    sc[i] = ab.scale;
-  }
-#pragma unroll
-  for (int wi = 0; wi < 4; ++wi) {
-    const uint32_t lo = bk.q[wi] & 0x0F0F0F0Fu, hi = bk.q[wi] & 0xF0F0F0F0u;
-#pragma unroll
-    for (int i = 0; i < NT; ++i)
-      dot8i(lo, hi, *reinterpret_cast<const uint4 *>(hs + ho[i] + b * MOE_QK + 8 * wi), al[i], ah[i]);
-  }
-#pragma unroll
-  for (int i = 0; i < NT; ++i) y[i] = block_finish(y[i], bk.d, sc[i], al[i], ah[i]);
-}
-
-// One block of two down rows (k0, k1) against NT slots' staged hidden vectors: dn_block for
-// each row, with one activation load serving both.
+// One block of two down rows (k0, k1) against NT slots' staged hidden vectors (the block's
+// integer dot products, then one rounding into y per row and slot), one activation load
+// serving both rows.
 template <int NT>
 __device__ __forceinline__ void dn_block2(const Blk &k0, const Blk &k1, int b, const uint16_t *hs, const ActBlk *hbk,
                                           const uint32_t (&ho)[NT], const uint32_t (&bo)[NT], float (&y0)[NT],

@@ -213,137 +213,6 @@ __device__ __forceinline__ void warp_topk_softmax(const float *lg, int E, int k,
   if constexpr (kMaxE > 256) warp_topk_softmax_t<MOE_MAX_E / 32>(lg, E, k, rscale, ids, w);
 }
 
-// Exclusive prefix sums of two int sequences a[0..n), b[0..n) in shared memory, in place,
-// by the whole CTA; totals returned through ta, tb. tmp: shared int[2 * 32].
-__device__ void block_exclusive_scan2_smem(int32_t *a, int32_t *b, int n, int32_t *tmp, int32_t &ta, int32_t &tb) {
-  const int nt = blockDim.x, tid = threadIdx.x, lane = tid & 31, wid = tid >> 5, nwarp = nt >> 5;
-  const int per = (n + nt - 1) / nt;
-  const int i0 = tid * per, i1 = min(n, i0 + per);
-  int32_t sa = 0, sb = 0;
-  for (int i = i0; i < i1; ++i) { sa += a[i]; sb += b[i]; }
-  int32_t xa = sa, xb = sb;
-#pragma unroll
-  for (int o = 1; o < 32; o <<= 1) {
-    const int32_t ya = __shfl_up_sync(0xffffffffu, xa, o), yb = __shfl_up_sync(0xffffffffu, xb, o);
-    if (lane >= o) { xa += ya; xb += yb; }
-  }
-  if (lane == 31) { tmp[wid] = xa; tmp[32 + wid] = xb; }
-  __syncthreads();
-  int32_t pa = 0, pb = 0;
-  ta = 0;
-  tb = 0;
-  for (int q = 0; q < nwarp; ++q) {
-    if (q < wid) { pa += tmp[q]; pb += tmp[32 + q]; }
-    ta += tmp[q];
-    tb += tmp[32 + q];
-  }
-  int32_t ra = pa + xa - sa, rb = pb + xb - sb;
-  __syncthreads();
-  for (int i = i0; i < i1; ++i) {
-    const int32_t va = a[i], vb = b[i];
-    a[i] = ra;
-    b[i] = rb;
-    ra += va;
-    rb += vb;
-  }
-  __syncthreads();
-}
-
-// Stable counting sort of S slot ids (shared memory) by one warp, no CTA barrier. Slots
-// are taken 32 at a time: __match_any groups the lanes of one expert, a slot's rank is the
-// number of its expert's slots in earlier rounds plus its lanes below it in this round.
-// Offsets, the active list and n_act come from a lane-chunked scan of the counts. inv[]
-// holds the rank until the last step, which turns it into the sorted position.
-__device__ void warp_permutation(const int32_t *ids, int S, int E, int32_t *counts, int32_t *offsets,
-                                 int32_t *perm, int32_t *inv, int32_t *act, int32_t *n_act) {
-  const int lane = threadIdx.x & 31;
-  for (int e = lane; e < E; e += 32) counts[e] = 0;
-  __syncwarp();
-  const uint32_t below = (1u << lane) - 1u;
-  for (int s0 = 0; s0 < S; s0 += 32) {
-    const int s = s0 + lane;
-    const bool valid = s < S;
-    const int id = valid ? ids[s] : -1 - lane;   // padding lanes get ids of their own
-    const uint32_t m = __match_any_sync(0xffffffffu, id);
-    const int base = valid ? counts[id] : 0;
-    __syncwarp();
-    if (valid) {
-      if ((m & below) == 0) counts[id] = base + __popc(m);
-      inv[s] = base + __popc(m & below);
-    }
-    __syncwarp();
-  }
-  const int per = (E + 31) / 32;
-  const int e0 = min(E, lane * per), e1 = min(E, e0 + per);
-  int c_sum = 0, a_sum = 0;
-  for (int e = e0; e < e1; ++e) {
-    const int c = counts[e];
-    c_sum += c;
-    a_sum += c > 0;
-  }
-  int c_inc = c_sum, a_inc = a_sum;
-#pragma unroll
-  for (int o = 1; o < 32; o <<= 1) {
-    const int nc = __shfl_up_sync(0xffffffffu, c_inc, o), na = __shfl_up_sync(0xffffffffu, a_inc, o);
-    if (lane >= o) {
-      c_inc += nc;
-      a_inc += na;
-    }
-  }
-  int c_run = c_inc - c_sum, a_run = a_inc - a_sum;
-  for (int e = e0; e < e1; ++e) {
-    const int c = counts[e];
-    offsets[e] = c_run;
-    if (c > 0) act[a_run++] = e;
-    c_run += c;
-  }
-  if (lane == 31) {
-    offsets[E] = c_inc;
-    *n_act = a_inc;
-  }
-  __syncwarp();
-  for (int s = lane; s < S; s += 32) {
-    const int pos = offsets[ids[s]] + inv[s];
-    perm[pos] = s;
-    inv[s] = pos;
-  }
-  __syncwarp();
-}
-
-// Stable counting sort of S small slot ids (shared memory) by the whole CTA: per-expert counts
-// by direct counting, CTA scans for the offsets and the active-expert list, and each slot's
-// rank among the earlier slots of its expert by direct comparison (S * S / 2 compares).
-// offsets/act/... are shared-memory arrays; flag[] is shared scratch of E ints.
-__device__ void block_permutation_direct(const int32_t *ids, int S, int E, int32_t *counts, int32_t *offsets,
-                                         int32_t *perm, int32_t *inv, int32_t *act, int32_t *n_act, int32_t *flag,
-                                         int32_t *tmp) {
-  for (int e = threadIdx.x; e < E; e += blockDim.x) {
-    int c = 0;
-    for (int s = 0; s < S; ++s) c += ids[s] == e;
-    counts[e] = c;
-    offsets[e] = c;
-    flag[e] = c > 0;
-  }
-  __syncthreads();
-  int32_t tot, atot;
-  block_exclusive_scan2_smem(offsets, flag, E, tmp, tot, atot);
-  for (int e = threadIdx.x; e < E; e += blockDim.x)
-    if (counts[e] > 0) act[flag[e]] = e;
-  if (threadIdx.x == 0) {
-    offsets[E] = tot;
-    *n_act = atot;
-  }
-  for (int s = threadIdx.x; s < S; s += blockDim.x) {
-    const int id = ids[s];
-    int r = 0;
-    for (int q = 0; q < s; ++q) r += ids[q] == id;
-    const int pos = offsets[id] + r;
-    perm[pos] = s;
-    inv[s] = pos;
-  }
-  __syncthreads();
-}
-
 // Stable counting sort of S <= 1024 slots by expert id in one warp: ranks from
 // __match_any_sync in slot order, a warp scan of the counts, then placement.
 constexpr int kSmallPermMax = 1024;
