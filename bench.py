@@ -160,7 +160,10 @@ def recorded_traffic(kernel: str, workload: str, units_per_launch: float):
         for ln in fh:
             if ln.startswith("- ") and ":" in ln:
                 key, _, val = ln[2:].partition(":")
-                fields[key.strip()] = val.strip().strip("`")
+                val = val.strip()
+                if val.startswith("`"):   # the value is the first back-quoted token
+                    val = val[1:].partition("`")[0]
+                fields[key.strip()] = val
     try:
         if fields.get("sources_sha256") != sources_sha256():
             return None
