@@ -169,8 +169,8 @@ int forward_impl(const void *x, const float *router_w, const float *router_scale
     if (rc == -2) return fail(MOE_ERR_BAD_ARG, "shape not supported by the grouped-GEMM path");
     if (rc) return cuda_fail(cudaGetLastError(), "grouped-GEMM launch");
   } else if (g.path != MOE_PATH_GEMV_SPLIT && moe_fused_decode_supported(T, d, f, E, k)) {
-    rc = moe_launch_fused_decode(L, g.W, x, router_w, router_scale, gate_up_q4, down_q4, expert_scale, T, d, f, E,
-                                 k, out, g.num_sms);
+    rc = moe_launch_fused_decode(L, g.W, x, nullptr, 0.f, nullptr, router_w, router_scale, gate_up_q4, down_q4,
+                                 expert_scale, T, d, f, E, k, out, g.num_sms);
     if (rc) return cuda_fail(cudaGetLastError(), "fused decode launch");
   } else {
     if (T <= 16)
@@ -383,18 +383,30 @@ int moe_stack_forward(const void *x_in, int L, const float *const *router_w, con
   if (rc) return rc;
   if (T == 0) return MOE_OK;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
+  // Layers that take the fused decode kernel normalise the previous layer's output inside
+  // it (no separate norm launch); the others get moe_rmsnorm_bf16's x. Both give the same x.
+  const bool fused = !(g.path == MOE_PATH_GEMM || (g.path == MOE_PATH_AUTO && T > g.gemv_max_tokens)) &&
+                     g.path != MOE_PATH_GEMV_SPLIT && moe_fused_decode_supported(T, d, f, E, k);
   const void *xc = x_in;
   for (int i = 0; i < L; ++i) {
+    char *trace_i = x_trace ? static_cast<char *>(x_trace) + (size_t)i * T * d * 2 : nullptr;
+    float *yo = (i == L - 1) ? out : g.ylayer;
+    if (i > 0 && fused) {
+      // y_prev = g.ylayer is read before the kernel's first grid barrier, yo written after its last
+      MoeLaunch Lf{s, false};
+      rc = moe_launch_fused_decode(Lf, g.W, nullptr, g.ylayer, eps, trace_i, router_w[i], router_scale[i],
+                                   gate_up_q4[i], down_q4[i], expert_scale[i], T, d, f, E, k, yo, g.num_sms);
+      if (rc) return cuda_fail(cudaGetLastError(), "fused decode launch");
+      continue;
+    }
     if (x_trace) {
-      cudaError_t e = cudaMemcpyAsync(static_cast<char *>(x_trace) + (size_t)i * T * d * 2, xc,
-                                      (size_t)T * d * 2, cudaMemcpyDeviceToDevice, s);
+      cudaError_t e = cudaMemcpyAsync(trace_i, xc, (size_t)T * d * 2, cudaMemcpyDeviceToDevice, s);
       if (e != cudaSuccess) return cuda_fail(e, "x_trace copy");
     }
-    float *yo = (i == L - 1) ? out : g.ylayer;
     rc = forward_impl(xc, router_w[i], router_scale[i], gate_up_q4[i], down_q4[i], expert_scale[i], T, d, f, E, k,
                       yo, s);
     if (rc) return rc;
-    if (i < L - 1) {
+    if (i < L - 1 && !fused) {
       __nv_bfloat16 *xn = g.xbuf[i & 1];
       if (moe_launch_rmsnorm(s, yo, xn, T, d, eps)) return cuda_fail(cudaGetLastError(), "rmsnorm launch");
       xc = xn;

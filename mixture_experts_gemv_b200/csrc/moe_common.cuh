@@ -241,10 +241,13 @@ int moe_launch_gemm_experts(const MoeLaunch &L, const MoeWork &W, const void *x,
                             const uint8_t *down_q4, const float *expert_scale, int T, int d, int f,
                             int E, int k, float *out, int num_sms, int max_tiles);
 bool moe_fused_decode_supported(int T, int d, int f, int E, int k);
-int moe_launch_fused_decode(const MoeLaunch &L, const MoeWork &W, const void *x, const float *router_w,
-                            const float *router_scale, const uint8_t *gate_up_q4, const uint8_t *down_q4,
-                            const float *expert_scale, int T, int d, int f, int E, int k, float *out,
-                            int num_sms);
+// The fused decode kernel: x (bf16 [T, d]) as the layer input, or, with y_prev not null, the
+// previous layer's FP32 output normalised in the kernel (x_out, when not null, receives that
+// bf16 x; y_prev may equal out).
+int moe_launch_fused_decode(const MoeLaunch &L, const MoeWork &W, const void *x, const float *y_prev, float eps,
+                            void *x_out, const float *router_w, const float *router_scale,
+                            const uint8_t *gate_up_q4, const uint8_t *down_q4, const float *expert_scale, int T,
+                            int d, int f, int E, int k, float *out, int num_sms);
 int moe_launch_rmsnorm(cudaStream_t s, const float *y, void *x_out, int T, int d, float eps);
 int moe_launch_hidden_to_slots(cudaStream_t s, const MoeWork &W, float *h, int T, int f, int k,
                                bool gemm_path);

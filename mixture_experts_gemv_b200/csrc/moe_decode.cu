@@ -423,12 +423,17 @@ __device__ __forceinline__ void dn_pass(const uint8_t *st, uint32_t rb, int nbf,
   }
 }
 
+// NORM_IN: the layer input is the previous layer's FP32 output y_prev, normalised here
+// (unit-gain RMSNorm + bf16 cast, as moe_norm.cu) instead of a bf16 x; CTA 0 also writes the
+// bf16 x to x_out when it is not null. y_prev may be the buffer `out` of this call: every CTA
+// reads it before its first grid-barrier arrival, `out` is written after the last barrier.
+template <bool NORM_IN>
 __global__ void __launch_bounds__((kFMaxCompute + 2) * 32, 1)
-k_moe_decode(const __nv_bfloat16 *__restrict__ x, const float *__restrict__ router_w,
-             const float *__restrict__ router_scale, const uint8_t *__restrict__ gate_up_q4,
-             const uint8_t *__restrict__ down_q4, const float *__restrict__ expert_scale, int T, int d, int f,
-             int E, int k, float *__restrict__ out, uint32_t stage_bytes, uint32_t x_bytes, uint32_t red_half,
-             MoeWork W) {
+k_moe_decode(const __nv_bfloat16 *__restrict__ x, const float *y_prev, float eps, __nv_bfloat16 *x_out,
+             const float *__restrict__ router_w, const float *__restrict__ router_scale,
+             const uint8_t *__restrict__ gate_up_q4, const uint8_t *__restrict__ down_q4,
+             const float *__restrict__ expert_scale, int T, int d, int f, int E, int k, float *out,
+             uint32_t stage_bytes, uint32_t x_bytes, uint32_t red_half, MoeWork W) {
   extern __shared__ __align__(128) uint8_t smem_raw[];
   __shared__ FusedShared sh;
   const int tid = threadIdx.x, lane = tid & 31, wq = tid >> 5, nw = blockDim.x >> 5;
@@ -455,9 +460,37 @@ k_moe_decode(const __nv_bfloat16 *__restrict__ x, const float *__restrict__ rout
     mbar_init(&sh.xbar, 1);
     fence_mbar_init();
     sh.abort = 0;
-    // x (bf16) into the activation region now; it is converted in place before the first barrier
-    mbar_arrive_expect_tx(&sh.xbar, (uint32_t)(T * d * 2));
-    bulk_g2s(xreg, x, (uint32_t)(T * d * 2), &sh.xbar);
+    if constexpr (!NORM_IN) {
+      // x (bf16) into the activation region now; it is converted in place before the first barrier
+      mbar_arrive_expect_tx(&sh.xbar, (uint32_t)(T * d * 2));
+      bulk_g2s(xreg, x, (uint32_t)(T * d * 2), &sh.xbar);
+    }
+  }
+  if constexpr (NORM_IN) {
+    // x = bf16(y / sqrt(mean(y^2) + eps)) per token with moe_norm.cu's arithmetic (256 lanes,
+    // the same summation order), written straight into the activation region
+    __syncthreads();   // the mbarriers are initialised
+    __nv_bfloat16 *xb = reinterpret_cast<__nv_bfloat16 *>(xreg);
+    for (int t = 0; t < T; ++t) {
+      const float *yr = y_prev + (size_t)t * d;
+      if (tid < 256) {
+        float s = 0.f;
+        for (int i = tid; i < d; i += 256) s = fmaf(yr[i], yr[i], s);
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
+        if (lane == 0) sh.part[wq][0] = s;
+      }
+      __syncthreads();
+      float tot = 0.f;
+#pragma unroll
+      for (int w = 0; w < 8; ++w) tot += sh.part[w][0];
+      const float inv = 1.0f / sqrtf(tot / (float)d + eps);
+      for (int i = tid; i < d; i += blockDim.x) xb[(size_t)t * d + i] = __float2bfloat16_rn(yr[i] * inv);
+      __syncthreads();   // sh.part is reused for the next token
+    }
+    if (blockIdx.x == 0 && x_out != nullptr)
+      for (int i = tid; i < T * d; i += blockDim.x) x_out[i] = xb[i];
+    if (tid == 0) mbar_arrive(&sh.xbar);   // the activation region holds x (no copy to wait for)
   }
   const float rs = __ldg(router_scale);
 
@@ -884,18 +917,19 @@ bool moe_fused_decode_supported(int T, int d, int f, int E, int k) {
          fused_smem(T, d, f).total + sizeof(FusedShared) <= 227 * 1024;
 }
 
-int moe_launch_fused_decode(const MoeLaunch &L, const MoeWork &W, const void *x, const float *router_w,
-                            const float *router_scale, const uint8_t *gate_up_q4, const uint8_t *down_q4,
-                            const float *expert_scale, int T, int d, int f, int E, int k, float *out,
-                            int num_sms) {
+int moe_launch_fused_decode(const MoeLaunch &L, const MoeWork &W, const void *x, const float *y_prev, float eps,
+                            void *x_out, const float *router_w, const float *router_scale,
+                            const uint8_t *gate_up_q4, const uint8_t *down_q4, const float *expert_scale, int T,
+                            int d, int f, int E, int k, float *out, int num_sms) {
   if (!moe_fused_decode_supported(T, d, f, E, k)) return -2;
   const FusedSmem fs = fused_smem(T, d, f);
-  static size_t set = 0;
-  if (fs.total > set) {
-    if (cudaFuncSetAttribute(k_moe_decode, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)fs.total) !=
-        cudaSuccess)
+  static size_t set[2] = {0, 0};
+  const bool norm_in = y_prev != nullptr;
+  if (fs.total > set[norm_in]) {
+    if (cudaFuncSetAttribute(norm_in ? k_moe_decode<true> : k_moe_decode<false>,
+                             cudaFuncAttributeMaxDynamicSharedMemorySize, (int)fs.total) != cudaSuccess)
       return -1;
-    set = fs.total;
+    set[norm_in] = fs.total;
   }
   const int G = (d / MOE_QK + kGran - 1) / kGran;
   cudaLaunchConfig_t cfg = {};
@@ -909,9 +943,11 @@ int moe_launch_fused_decode(const MoeLaunch &L, const MoeWork &W, const void *x,
   cfg.attrs = attr;
   cfg.numAttrs = 1;
   moe_prof_mark(L.stream, MOE_K_FUSED, true);
-  const cudaError_t e = cudaLaunchKernelEx(&cfg, k_moe_decode, static_cast<const __nv_bfloat16 *>(x), router_w,
-                                           router_scale, gate_up_q4, down_q4, expert_scale, T, d, f, E, k, out,
-                                           fs.stage_bytes, fs.x_bytes, fs.red_half, W);
+  const cudaError_t e =
+      cudaLaunchKernelEx(&cfg, norm_in ? k_moe_decode<true> : k_moe_decode<false>,
+                         static_cast<const __nv_bfloat16 *>(x), y_prev, eps, static_cast<__nv_bfloat16 *>(x_out),
+                         router_w, router_scale, gate_up_q4, down_q4, expert_scale, T, d, f, E, k, out,
+                         fs.stage_bytes, fs.x_bytes, fs.red_half, W);
   if (e != cudaSuccess) return -1;
   moe_prof_mark(L.stream, MOE_K_FUSED, false);
   return 0;

@@ -261,6 +261,30 @@ def test_prefill_T4096_sampled():
     _check_full(wl.x, wl.layers[0], wl.k, moe.MOE_PATH_AUTO, tokens=tok)
 
 
+def test_stack_in_kernel_norm_matches_separate_norm():
+    """In a stack, the fused decode kernel normalises the previous layer's output itself; the
+    separate path launches moe_rmsnorm_bf16 and the separate decode kernels. Same bits for
+    every layer's x and for the output."""
+    L = 3
+    wl = mi.make_workload("stack30_T1", n_layers=L)
+    d, f, E, k = mi.D_MODEL, mi.D_FF, mi.N_EXPERTS, wl.k
+    dls = [DevLayer(lw) for lw in wl.layers]
+    ensure_init(1, d, f, E, k)
+    res = []
+    for path in (moe.MOE_PATH_AUTO, moe.MOE_PATH_GEMV_SPLIT):
+        moe.moe_set_path(path, 16)
+        out = torch.empty((1, d), dtype=torch.float32, device="cuda:0")
+        trace = torch.empty((L, 1, d), dtype=torch.int16, device="cuda:0")
+        moe.moe_stack_forward(dev(wl.x), [q.router_w for q in dls], [q.router_scale for q in dls],
+                              [q.gate_up for q in dls], [q.down for q in dls], [q.expert_scale for q in dls],
+                              1, d, f, E, k, 1e-6, out, trace)
+        moe.moe_debug_check()
+        res.append((out.cpu().numpy().view(np.uint32), trace.cpu().numpy()))
+    moe.moe_set_path(moe.MOE_PATH_AUTO, 16)
+    assert np.array_equal(res[0][1], res[1][1])
+    assert np.array_equal(res[0][0], res[1][0])
+
+
 def test_stack_teacher_forced():
     """Layer i's oracle consumes the GPU's own bf16 input x_i (recorded by x_trace)."""
     L = 3
