@@ -174,6 +174,23 @@ def recorded_traffic(kernel: str, workload: str, units_per_launch: float):
         return None
 
 
+def max_over_ranks(vals, device):
+    """Element-wise maximum of this rank's timings over all ranks (the slowest rank decides a
+    multi-GPU time); the values themselves at one rank."""
+    import torch
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return [float(v) for v in vals]
+    t = torch.tensor([float(v) for v in vals], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return [float(v) for v in t.tolist()]
+
+
+def job_throughput(ws: int, units_per_rank_step: float, steps: int, ms_max: float) -> float:
+    """Whole-job units per second: every rank's units over the slowest rank's time."""
+    return ws * units_per_rank_step * steps / (ms_max / 1e3)
+
+
 def dist_env():
     ws = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
@@ -349,10 +366,7 @@ def main():
     ms = ev0.elapsed_time(ev1)
     clocks = sampler.stop()
     moe.moe_debug_check(stream)
-    if ws > 1:
-        t = torch.tensor([ms], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms = float(t.item())
+    ms = max_over_ranks([ms], dev)[0]
     ms_step = ms / args.steps
 
     # ---- per-kernel timing: the same K steps with CUDA events recorded around every kernel
@@ -427,16 +441,13 @@ def main():
     barrier()
     ms_e2e_eager = e0.elapsed_time(e1)
     del egraph
-    if ws > 1:
-        t = torch.tensor([ms_e2e, ms_e2e_eager], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms_e2e, ms_e2e_eager = float(t[0].item()), float(t[1].item())
+    ms_e2e, ms_e2e_eager = max_over_ranks([ms_e2e, ms_e2e_eager], dev)
 
     # ---- roofline of the dominant kernel
     pk = measured_peaks()
     tokens_per_step = T
-    value = ws * tokens_per_step * args.steps / (ms / 1e3)
-    e2e_value = ws * tokens_per_step * args.steps / (ms_e2e / 1e3)
+    value = job_throughput(ws, tokens_per_step, args.steps, ms)
+    e2e_value = job_throughput(ws, tokens_per_step, args.steps, ms_e2e)
     avg = {kk: float(np.mean([w[kk] for w in work])) for kk in work[0]}
     n_layers_per_step = len(layers) if stack else 1
     if T <= 16 and "fused_decode" in prof:
@@ -500,7 +511,7 @@ def main():
             "e2e": {"value": e2e_value, "unit": "tokens/s", "h2d_bytes_per_step": T * d * 2,
                     "d2h_bytes_per_step": T * d * 4,
                     "launch": "CUDA graph of K steps; copies pipelined on two copy streams, double-buffered",
-                    "eager_value": ws * T * args.steps / (ms_e2e_eager / 1e3)},
+                    "eager_value": job_throughput(ws, T, args.steps, ms_e2e_eager)},
             "clocks": clocks}
 
     if rank == 0 and ws == 1 and not args.no_cpu_baseline:

@@ -28,3 +28,42 @@ def test_recorded_traffic_stale_or_missing(tmp_path, monkeypatch):
     _write_summary(str(tmp_path), "k_x", "w", "old", 1000, 500)
     assert bench.recorded_traffic("k_x", "w", 500) is None      # sources changed since the capture
     assert bench.recorded_traffic("k_y", "w", 500) is None      # no summary at all
+
+
+def _rank_main(rank, ws, port, q):
+    import torch.distributed as dist
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("gloo", rank=rank, world_size=ws)
+    try:
+        # rank r timed (10 + r) ms for the steps and (20 - r) ms end to end
+        got = bench.max_over_ranks([10.0 + rank, 20.0 - rank], "cpu")
+        q.put((rank, got, bench.job_throughput(ws, 8, 100, got[0])))
+    finally:
+        dist.destroy_process_group()
+
+
+def test_max_over_ranks_gloo_two_ranks():
+    """The N > 1 reduction on two CPU ranks (gloo): every rank gets the element-wise maximum,
+    and the whole-job throughput counts every rank's tokens over the slowest rank's time."""
+    import socket
+    import torch.multiprocessing as tmp
+    with socket.socket() as sk:
+        sk.bind(("127.0.0.1", 0))
+        port = sk.getsockname()[1]
+    ctx = tmp.get_context("spawn")
+    q = ctx.Queue()
+    procs = [ctx.Process(target=_rank_main, args=(r, 2, port, q)) for r in range(2)]
+    for p in procs:
+        p.start()
+    res = sorted(q.get(timeout=120) for _ in procs)
+    for p in procs:
+        p.join(timeout=60)
+        assert p.exitcode == 0
+    for rank, got, thr in res:
+        assert got == [11.0, 20.0]
+        assert abs(thr - 2 * 8 * 100 / 0.011) < 1e-6 * thr
+
+
+def test_max_over_ranks_single_process():
+    assert bench.max_over_ranks([3.0, 4.5], "cpu") == [3.0, 4.5]
+    assert bench.job_throughput(1, 8, 200, 11.0) == 8 * 200 / 0.011
