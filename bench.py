@@ -137,14 +137,41 @@ def flops_bytes(lw: mi.LayerWeights, T: int, k: int, counts: np.ndarray):
             "flops": flops}
 
 
+def strip_c_comments(src: str) -> str:
+    """C/C++ source without its comments and blank lines (string and character literals kept
+    intact), so that editing a comment does not count as changing a kernel."""
+    out, i, n = [], 0, len(src)
+    while i < n:
+        c = src[i]
+        if c in "\"'":                                   # a literal: copy it to its closing quote
+            j = i + 1
+            while j < n and src[j] != c:
+                j += 2 if src[j] == "\\" else 1
+            out.append(src[i:j + 1])
+            i = j + 1
+        elif src.startswith("//", i):
+            j = src.find("\n", i)
+            i = n if j < 0 else j
+        elif src.startswith("/*", i):
+            j = src.find("*/", i + 2)
+            i = n if j < 0 else j + 2
+        else:
+            out.append(c)
+            i += 1
+    lines = (ln.rstrip() for ln in "".join(out).splitlines())
+    return "\n".join(ln for ln in lines if ln)
+
+
 def sources_sha256() -> str:
-    """Hash of the CUDA sources; a recorded ncu traffic figure is valid only for this hash."""
+    """Hash of the CUDA sources' code (comments and blank lines removed); a recorded ncu
+    traffic figure is valid only for this hash."""
     import glob
     import hashlib
     h = hashlib.sha256()
     for p in sorted(glob.glob(os.path.join(ROOT, "mixture_experts_gemv_b200", "csrc", "*"))):
-        with open(p, "rb") as fh:
-            h.update(os.path.basename(p).encode() + b"\0" + fh.read())
+        with open(p, encoding="utf-8") as fh:
+            code = strip_c_comments(fh.read())
+        h.update(os.path.basename(p).encode() + b"\0" + code.encode())
     return h.hexdigest()
 
 

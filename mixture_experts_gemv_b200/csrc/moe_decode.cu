@@ -1,8 +1,10 @@
 // moe_decode.cu -- the whole routed-MoE layer for small token counts (decode) in one
 // persistent kernel: one CTA per SM, launched cooperatively so all CTAs are resident.
 //
-//   phase 0  router logits (one expert per CTA, warps split d); arrive at the grid barrier,
-//            stage every token's GEMV activations in shared memory, then wait (bounded)
+//   phase 0  x into shared memory (a bulk copy of the bf16 input, or, in a layer stack, the
+//            previous layer's FP32 output normalised in place: NORM_IN); router logits (one
+//            expert per CTA, warps split d); arrive at the grid barrier, stage every token's
+//            GEMV activations in shared memory, then wait (bounded)
 //   phase 1  every CTA selects the top-k experts of every token, builds the stable
 //            permutation and its cost-weighted share of the work in its own shared memory
 //   phase 2  gate_up GEMV + GeGLU over this CTA's share of the active experts' rows
@@ -17,8 +19,9 @@
 // stage through an mbarrier and synchronise among themselves with a named barrier.
 //
 // Definitions as in moe_route.cu / moe_gemv.cu (page "Gemma 4 26B-A4B it QAT Q4_0 ... NInfer
-// v3 artifact", "What is inside"). Results equal the separate-kernel path's up to the order
-// of the router's FP32 partial sums.
+// v3 artifact", "What is inside"). Results equal the separate-kernel path's bit for bit: both
+// cut the router's d axis and the down rows the same way and sum in the same orders
+// (moe_common.cuh), so a token's output does not depend on the batch it is decoded in.
 #include "moe_gemv_core.cuh"
 #include "moe_route_core.cuh"
 

@@ -67,3 +67,13 @@ def test_max_over_ranks_gloo_two_ranks():
 def test_max_over_ranks_single_process():
     assert bench.max_over_ranks([3.0, 4.5], "cpu") == [3.0, 4.5]
     assert bench.job_throughput(1, 8, 200, 11.0) == 8 * 200 / 0.011
+
+
+def test_code_hash_ignores_comments_only():
+    """The profile summaries stay valid across comment edits, not across code edits."""
+    a = 'int f(int x) {  // twice\n  return 2 * x;  /* doubled */\n}\nconst char *s = "//not a comment";\n'
+    b = '/* a new header */\nint f(int x) {\n\n  return 2 * x;\n}\nconst char *s = "//not a comment";\n'
+    c = 'int f(int x) {\n  return 3 * x;\n}\nconst char *s = "//not a comment";\n'
+    assert bench.strip_c_comments(a) == bench.strip_c_comments(b)
+    assert bench.strip_c_comments(a) != bench.strip_c_comments(c)
+    assert '"//not a comment"' in bench.strip_c_comments(a)
