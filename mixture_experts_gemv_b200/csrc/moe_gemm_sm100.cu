@@ -537,13 +537,21 @@ __global__ void __launch_bounds__(256) k_combine(const __nv_bfloat16 *__restrict
        i += (long long)gridDim.x * blockDim.x) {
     const int t = (int)(i / vpr), v = (int)(i % vpr);
     float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-    for (int j = 0; j < k; ++j) {
-      const uint4 q = __ldg(reinterpret_cast<const uint4 *>(yslot + (size_t)(t * k + j) * d) + v);
-      const uint32_t qq[4] = {q.x, q.y, q.z, q.w};
+    for (int j0 = 0; j0 < k; j0 += 8) {   // eight slots' loads in flight, then the sums in j order
+      uint4 q[8];
 #pragma unroll
-      for (int h = 0; h < 4; ++h) {
-        acc[2 * h] += __uint_as_float(qq[h] << 16);
-        acc[2 * h + 1] += __uint_as_float(qq[h] & 0xffff0000u);
+      for (int u = 0; u < 8; ++u)
+        q[u] = j0 + u < k ? __ldg(reinterpret_cast<const uint4 *>(yslot + (size_t)(t * k + j0 + u) * d) + v)
+                          : make_uint4(0u, 0u, 0u, 0u);
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        if (j0 + u >= k) break;
+        const uint32_t qq[4] = {q[u].x, q[u].y, q[u].z, q[u].w};
+#pragma unroll
+        for (int h = 0; h < 4; ++h) {
+          acc[2 * h] += __uint_as_float(qq[h] << 16);
+          acc[2 * h + 1] += __uint_as_float(qq[h] & 0xffff0000u);
+        }
       }
     }
     float4 *op = reinterpret_cast<float4 *>(out + (size_t)t * d) + 2 * v;
