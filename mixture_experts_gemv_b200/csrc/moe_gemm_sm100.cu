@@ -47,7 +47,6 @@ constexpr int kProdThreads = kProdWarps * 32;
 constexpr int kGroupThreads = kProdThreads / kProdGroups;     // one (row, block) of the B tile each
 constexpr int kThreads = (kEpiWarps + 1 + kProdWarps) * 32;
 constexpr uint32_t kTileBytes = BM * BK * 2;                  // 16 KB: one A half; B is BN x BK, same
-constexpr int kAhead = 2;                                     // group steps the copies run ahead
 constexpr uint32_t kRawRowBytes = 64;                          // 16-byte-aligned window over a row's 36 bytes
 constexpr uint32_t kRawStageBytes = BN * kRawRowBytes;
 
@@ -58,6 +57,10 @@ template <bool GATEUP>
 struct GemmCfg {
   static constexpr int kHalves = GATEUP ? 1 : 2;
   static constexpr int kStages = GATEUP ? 5 : 4;
+  // group steps the copies run ahead of the decode (measured: gate_up, whose producers
+  // gather A, gains from the deeper lookahead; down, whose A comes by TMA, from refilling a
+  // stage that an older MMA released)
+  static constexpr int kAhead = GATEUP ? 2 : 1;
   static constexpr uint32_t kBOff = kHalves * kTileBytes;        // B tile after the A halves
   static constexpr uint32_t kStageBytes = kBOff + kTileBytes;
   static constexpr uint32_t kTmemCols = 2 * kHalves * BN;        // two accumulator buffers
@@ -238,7 +241,7 @@ k_moe_gemm(const __grid_constant__ CUtensorMap tmap_h, const __nv_bfloat16 *__re
   const size_t rb = (size_t)nb_row * MOE_QBYTES;       // bytes per weight row
   const size_t expert_bytes = (size_t)(GATEUP ? 2 * f : d) * rb;
   using C = GemmCfg<GATEUP>;
-  constexpr int kHalves = C::kHalves, kStages = C::kStages;
+  constexpr int kHalves = C::kHalves, kStages = C::kStages, kAhead = C::kAhead;
   constexpr uint32_t kBOff = C::kBOff, kStageBytes = C::kStageBytes, kTmemCols = C::kTmemCols;
   const int n_items = (GATEUP ? *W.n_tiles : *W.n_pairs) * n_ntiles;
   // work item -> its first tile, and whether a second tile (rows 128 .. 255 past the first
