@@ -99,8 +99,9 @@ int moe_rmsnorm_bf16(const float *y, void *x_out, int T, int d, float eps, void 
  *   x_in     device bf16 [T, d], input of layer 0
  *   out      device fp32 [T, d], output of layer L-1
  *   x_trace  optional device bf16 [L, T, d]: receives each layer's input (NULL to skip)
- * Same shape rules as moe_layer_forward. The inter-layer bf16 activations live in the
- * workspace.
+ * Same shape rules as moe_layer_forward. The inter-layer activations live in the workspace.
+ * Layers that take the fused decode kernel apply the normalisation inside that kernel (the
+ * same arithmetic and bits as moe_rmsnorm_bf16), so such a stack is one launch per layer.
  */
 int moe_stack_forward(const void *x_in, int L, const float *const *router_w,
                       const float *const *router_scale, const uint8_t *const *gate_up_q4,
