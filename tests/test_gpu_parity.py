@@ -87,6 +87,7 @@ def test_fused_and_split_decode_agree(T):
 SMALL_GEMM = [  # (E, k, T, d, f): d % 128 == 0, f % 64 == 0
     (8, 2, 33, 256, 64), (4, 4, 130, 128, 128), (128, 8, 300, 512, 128), (16, 4, 257, 2816, 704),
     (128, 2, 17, 256, 64), (3, 3, 40, 384, 192),
+    (2, 2, 600, 256, 64),   # 600 rows per expert: five tiles, two tile pairs and a ragged single
 ]
 
 
