@@ -135,8 +135,25 @@ int moe_debug_get_routing(int32_t *ids, float *w, int32_t *counts, int32_t *offs
  */
 int moe_debug_get_hidden(float *h, void *stream);
 
-/* moe_debug_check: synchronise `stream` and report the device error word (timeouts). */
+/* moe_debug_check: synchronise `stream` and report the device error word (timeouts). After a
+ * reported timeout the next forward first zeroes the workspace's arrival counters. */
 int moe_debug_check(void *stream);
+
+/*
+ * Failure detection, for tests. Every device-side wait (mbarrier phases, grid barriers) is
+ * bounded; a wait that runs out records MOE_ERR_DEVICE_TIMEOUT in the error word, the
+ * kernel ends on its own (it waits, again bounded, for its copies in flight first) and the
+ * context stays usable.
+ *   moe_debug_set_wait_ns: bound of every device-side wait of later forwards, in
+ *     nanoseconds (0 restores the default of 2 s).
+ *   moe_debug_inject: make the next forward simulate a fault by skipping one step --
+ *     MOE_INJECT_SKIP_ROUTER_ARRIVAL: in the fused decode kernel, CTA 0 never arrives at the
+ *     first grid barrier, so every other CTA's wait there runs out. Cleared by that forward.
+ */
+#define MOE_INJECT_NONE 0
+#define MOE_INJECT_SKIP_ROUTER_ARRIVAL 1
+int moe_debug_set_wait_ns(unsigned long long ns);
+int moe_debug_inject(int fault);
 
 /*
  * Per-kernel timing with CUDA events, for measurement. After moe_profile_begin, every
@@ -151,6 +168,9 @@ int moe_debug_check(void *stream);
 #define MOE_PROF_GROUPS 8
 int moe_profile_begin(void);
 int moe_profile_end(float *ms_total, int *launches);
+/* moe_profile_kernel_launches: kernels this library launched (or recorded into a stream
+ * capture) since the last moe_profile_begin; a group above can hold several kernels. */
+long long moe_profile_kernel_launches(void);
 
 /*
  * moe_layer_forward_static: the decode (FP32-accumulate GEMV) path of moe_layer_forward, for
@@ -168,8 +188,11 @@ int moe_profile_end(float *ms_total, int *launches);
  *   address; make that first call before any stream capture.
  *   All calls share the array and leave their contents in it; the counters that must start
  *   at zero are cleared at the start of each call on `stream`. Calls whose work overlaps on
- *   the GPU (other streams, other host threads) race on the array.
- *   There is no device error word: a device-side wait that expires ends the kernels early.
+ *   the GPU (other streams, other host threads) race on the array. First calls made from
+ *   several host threads at once are safe: the set-up runs once per device.
+ *   A device-side wait that runs out of time (2 s) ends the kernels early, leaving `out` not
+ *   fully written; it is recorded in a device error word inside the array, which stays set
+ *   until moe_layer_forward_static_check reads it.
  */
 #define MOE_STATIC_SCRATCH_BYTES (4u << 20)
 #define MOE_STATIC_MAX_TOKENS 16
@@ -181,6 +204,11 @@ int moe_layer_forward_static(const void *x, const float *router_w, const float *
                              const uint8_t *gate_up_q4, const uint8_t *down_q4,
                              const float *expert_scale, int T, int d, int f, int E, int k,
                              float *out, void *stream);
+/* moe_layer_forward_static_check: synchronise `stream`, then read and clear the static entry's
+ * device error word on the current device: MOE_ERR_DEVICE_TIMEOUT if a call since the last
+ * check had a device-side wait run out (its output is then not valid), else MOE_OK.
+ * Allocates nothing. */
+int moe_layer_forward_static_check(void *stream);
 
 /* moe_workspace_bytes: device bytes moe_init would allocate for the given limits. */
 size_t moe_workspace_bytes(int max_tokens, int max_d, int max_f, int max_E, int max_k);

@@ -9,5 +9,7 @@ from ._lib import (  # noqa: F401
     MOE_PATH_GEMM, MOE_PATH_GEMV_SPLIT, MoeError, lib, moe_init, moe_layer_forward, moe_rmsnorm_bf16,
     moe_stack_forward, moe_set_path, moe_destroy, moe_last_error, moe_debug_get_routing,
     moe_debug_get_hidden, moe_debug_check, moe_workspace_bytes, moe_profile_begin,
-    moe_profile_end, PROF_GROUPS, EXPORTED, moe_layer_forward_static,
+    moe_profile_end, PROF_GROUPS, EXPORTED, moe_layer_forward_static, moe_profile_kernel_launches,
+    moe_layer_forward_static_check, moe_debug_set_wait_ns, moe_debug_inject, MOE_INJECT_NONE,
+    MOE_INJECT_SKIP_ROUTER_ARRIVAL,
 )

@@ -30,8 +30,11 @@ EXPORTED = (
     "moe_init", "moe_layer_forward", "moe_rmsnorm_bf16", "moe_stack_forward", "moe_set_path",
     "moe_destroy", "moe_last_error", "moe_debug_get_routing", "moe_debug_get_hidden",
     "moe_debug_check", "moe_workspace_bytes", "moe_profile_begin", "moe_profile_end",
-    "moe_layer_forward_static",
+    "moe_layer_forward_static", "moe_profile_kernel_launches", "moe_layer_forward_static_check",
+    "moe_debug_set_wait_ns", "moe_debug_inject",
 )
+MOE_INJECT_NONE = 0
+MOE_INJECT_SKIP_ROUTER_ARRIVAL = 1
 PROF_GROUPS = ("route", "gateup_gemv", "down_gemv", "gateup_gemm", "down_gemm", "combine", "rmsnorm",
                "fused_decode")
 
@@ -82,6 +85,14 @@ def lib():
         L.moe_profile_end.restype = _i
         L.moe_layer_forward_static.argtypes = [_p, _p, _p, _p, _p, _p, _i, _i, _i, _i, _i, _p, _p]
         L.moe_layer_forward_static.restype = _i
+        L.moe_layer_forward_static_check.argtypes = [_p]
+        L.moe_layer_forward_static_check.restype = _i
+        L.moe_debug_set_wait_ns.argtypes = [ctypes.c_ulonglong]
+        L.moe_debug_set_wait_ns.restype = _i
+        L.moe_debug_inject.argtypes = [_i]
+        L.moe_debug_inject.restype = _i
+        L.moe_profile_kernel_launches.argtypes = []
+        L.moe_profile_kernel_launches.restype = ctypes.c_longlong
         L.moe_workspace_bytes.argtypes = [_i, _i, _i, _i, _i]
         L.moe_workspace_bytes.restype = ctypes.c_size_t
         _lib = L
@@ -182,9 +193,27 @@ def moe_profile_end() -> dict:
     return {PROF_GROUPS[i]: (float(ms[i]), int(n[i])) for i in range(8) if n[i] > 0}
 
 
+def moe_profile_kernel_launches() -> int:
+    """Kernels launched (or captured) since moe_profile_begin."""
+    return int(lib().moe_profile_kernel_launches())
+
+
 def moe_layer_forward_static(x, router_w, router_scale, gate_up_q4, down_q4, expert_scale,
                              T: int, d: int, f: int, E: int, k: int, out, stream=None) -> None:
     """Decode path with a fixed static device scratch: no workspace, no allocation."""
     _check(lib().moe_layer_forward_static(_ptr(x), _ptr(router_w), _ptr(router_scale),
                                           _ptr(gate_up_q4), _ptr(down_q4), _ptr(expert_scale),
                                           T, d, f, E, k, _ptr(out), _stream(stream)))
+
+
+def moe_layer_forward_static_check(stream=None) -> None:
+    """Raise MoeError(MOE_ERR_DEVICE_TIMEOUT) if a static-entry call timed out since the last check."""
+    _check(lib().moe_layer_forward_static_check(_stream(stream)))
+
+
+def moe_debug_set_wait_ns(ns: int) -> None:
+    _check(lib().moe_debug_set_wait_ns(int(ns)))
+
+
+def moe_debug_inject(fault: int) -> None:
+    _check(lib().moe_debug_inject(int(fault)))

@@ -1,15 +1,18 @@
-"""Build libmoe.so (the sm_100a kernels + C ABI) in-tree with nvcc."""
+"""Build libmoe.so (the sm_100a kernels + C ABI) in-tree with nvcc: each CUDA source is
+compiled to an object in parallel, then the objects are linked into the shared library."""
 from __future__ import annotations
 
 import glob
 import os
 import subprocess
+from concurrent.futures import ThreadPoolExecutor
 
 HERE = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(HERE)
 LIB_PATH = os.path.join(HERE, "libmoe.so")
-NVCC_FLAGS = ["-gencode", "arch=compute_100a,code=sm_100a", "-O3", "-std=c++17", "-lineinfo",
-              "-Xcompiler", "-fPIC", "-shared"]
+OBJ_DIR = os.path.join(HERE, "_build")
+ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
+NVCC_FLAGS = [*ARCH, "-O3", "-std=c++17", "-lineinfo", "-Xcompiler", "-fPIC"]
 
 
 def sources() -> list[str]:
@@ -27,12 +30,27 @@ def build(force: bool = False, verbose: bool = False) -> str:
         if all(os.path.getmtime(p) <= t for p in deps()):
             return LIB_PATH
     nvcc = os.environ.get("NVCC", "nvcc")
-    tmp = LIB_PATH + f".tmp{os.getpid()}"
-    cmd = [nvcc, *NVCC_FLAGS, "-I", os.path.join(ROOT, "include"), "-o", tmp, *sources()]
-    if verbose:
-        cmd.insert(1, "-Xptxas=-v")
-    subprocess.run(cmd, check=True)
-    os.replace(tmp, LIB_PATH)
+    os.makedirs(OBJ_DIR, exist_ok=True)
+    pid = os.getpid()
+
+    def compile_one(src):
+        obj = os.path.join(OBJ_DIR, os.path.basename(src)[:-3] + f".{pid}.o")
+        cmd = [nvcc, *NVCC_FLAGS, "-I", os.path.join(ROOT, "include"), "-c", "-o", obj, src]
+        if verbose:
+            cmd.insert(1, "-Xptxas=-v")
+        subprocess.run(cmd, check=True)
+        return obj
+
+    with ThreadPoolExecutor(max_workers=min(8, os.cpu_count() or 1)) as ex:
+        objs = list(ex.map(compile_one, sources()))
+    tmp = LIB_PATH + f".tmp{pid}"
+    try:
+        subprocess.run([nvcc, *ARCH, "-shared", "-o", tmp, *objs], check=True)
+        os.replace(tmp, LIB_PATH)
+    finally:
+        for o in objs:
+            if os.path.exists(o):
+                os.remove(o)
     return LIB_PATH
 
 

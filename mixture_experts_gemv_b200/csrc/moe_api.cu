@@ -26,6 +26,8 @@ struct Ctx {
   int gemv_max_tokens = 16;   // AUTO: GEMV for T <= 16, grouped GEMM above
   int last_T = 0, last_k = 0, last_E = 0, last_f = 0;
   bool last_gemm = false;
+  size_t counters_bytes = 0;
+  bool reset_pending = false;   // a device wait expired: zero the barrier words before the next launch
 };
 
 Ctx g;
@@ -41,6 +43,7 @@ struct Prof {
   int open_id[MOE_K_COUNT];
   cudaEvent_t open_ev[MOE_K_COUNT];
   bool overflow = false;
+  long long kernels = 0;   // kernel launches since moe_profile_begin
 };
 Prof g_prof;
 
@@ -129,8 +132,21 @@ int check_device_error() {
   if (g.err_host && *reinterpret_cast<volatile uint32_t *>(g.err_host) != 0) {
     const uint32_t v = *reinterpret_cast<volatile uint32_t *>(g.err_host);
     *reinterpret_cast<volatile uint32_t *>(g.err_host) = 0;
+    // the kernels that gave up left their arrival counters mid-count
+    g.reset_pending = true;
     return fail(MOE_ERR_DEVICE_TIMEOUT, "device wait timed out (code %u at site %u)", v & 0xffffu, v >> 16);
   }
+  return MOE_OK;
+}
+
+// After an expired wait: the grid-barrier counter and the arrival counters start again from
+// zero (enqueued on the stream of the next launch).
+int reset_counters_if_needed(cudaStream_t s) {
+  if (!g.reset_pending) return MOE_OK;
+  cudaError_t e = cudaMemsetAsync(g.W.gbar, 0, 64, s);
+  if (e == cudaSuccess) e = cudaMemsetAsync(g.W.counters, 0, g.counters_bytes, s);
+  if (e != cudaSuccess) return cuda_fail(e, "resetting the arrival counters");
+  g.reset_pending = false;
   return MOE_OK;
 }
 
@@ -156,10 +172,11 @@ int forward_impl(const void *x, const float *router_w, const float *router_scale
                  const uint8_t *down_q4, const float *expert_scale, int T, int d, int f, int E, int k, float *out,
                  cudaStream_t stream) {
   MoeLaunch L{stream, false};
+  int rc = reset_counters_if_needed(stream);
+  if (rc) return rc;
   const bool gemm = (g.path == MOE_PATH_GEMM) || (g.path == MOE_PATH_AUTO && T > g.gemv_max_tokens);
   // MOE_PATH_GEMV and AUTO below the threshold take the fused decode kernel when the shape
   // fits it (T <= 8), else the separate routing / gate_up / down kernels (MOE_PATH_GEMV_SPLIT).
-  int rc;
   if (gemm) {
     rc = moe_launch_route_prefill(L, g.W, x, router_w, router_scale, T, d, E, k, g.num_sms, false, kTileM);
     if (rc) return cuda_fail(cudaGetLastError(), "routing launch");
@@ -182,6 +199,7 @@ int forward_impl(const void *x, const float *router_w, const float *router_scale
     if (rc == -2) return fail(MOE_ERR_BAD_ARG, "shape not supported by the GEMV path (d, f too large)");
     if (rc) return cuda_fail(cudaGetLastError(), "GEMV launch");
   }
+  g.W.inject = MOE_INJECT_NONE;   // a test fault applies to one forward only
   g.last_T = T;
   g.last_k = k;
   g.last_E = E;
@@ -217,7 +235,29 @@ void moe_prof_mark(cudaStream_t s, int id, bool begin) {
   }
 }
 
+void moe_prof_count(int n) {
+  if (g_prof.active) g_prof.kernels += n;
+}
+
+bool moe_allow_dyn_smem(const void *fn, unsigned long long *done_mask) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return false;
+  const unsigned long long bit = 1ull << dev;
+  if (__atomic_load_n(done_mask, __ATOMIC_ACQUIRE) & bit) return true;
+  int optin = 0;
+  if (cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev) != cudaSuccess) return false;
+  cudaFuncAttributes fa;
+  if (cudaFuncGetAttributes(&fa, fn) != cudaSuccess) return false;
+  if (cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, optin - (int)fa.sharedSizeBytes) !=
+      cudaSuccess)
+    return false;
+  __atomic_fetch_or(done_mask, bit, __ATOMIC_RELEASE);
+  return true;
+}
+
 extern "C" {
+
+long long moe_profile_kernel_launches(void) { return g_prof.kernels; }
 
 int moe_profile_begin(void) {
   if (!g.init) return fail(MOE_ERR_NOT_INIT, "moe_init has not succeeded");
@@ -225,6 +265,7 @@ int moe_profile_begin(void) {
   g_prof.used = 0;
   g_prof.recs.clear();
   g_prof.overflow = false;
+  g_prof.kernels = 0;
   for (int i = 0; i < MOE_K_COUNT; ++i) g_prof.open_ev[i] = nullptr;
   return MOE_OK;
 }
@@ -314,6 +355,8 @@ int moe_init(int device, int max_tokens, int max_d, int max_f, int max_E, int ma
   W.toff = reinterpret_cast<int32_t *>(b + Lt.off[21]);
   W.gbar = reinterpret_cast<unsigned long long *>(b + Lt.off[22]);
   W.err = ed;
+  W.wait_ns = MOE_WAIT_NS;
+  W.inject = MOE_INJECT_NONE;
 
   g.init = true;
   g.device = device;
@@ -325,6 +368,7 @@ int moe_init(int device, int max_tokens, int max_d, int max_f, int max_E, int ma
   g.max_k = max_k;
   g.ws = ws;
   g.ws_bytes = Lt.total;
+  g.counters_bytes = (size_t)(2 + max_d / 8 + 1024) * 4;
   g.err_host = eh;
   g.W = W;
   g.xbuf[0] = reinterpret_cast<__nv_bfloat16 *>(b + Lt.off[17]);
@@ -383,6 +427,8 @@ int moe_stack_forward(const void *x_in, int L, const float *const *router_w, con
   if (rc) return rc;
   if (T == 0) return MOE_OK;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
+  rc = reset_counters_if_needed(s);
+  if (rc) return rc;
   // Layers that take the fused decode kernel normalise the previous layer's output inside
   // it (no separate norm launch); the others get moe_rmsnorm_bf16's x. Both give the same x.
   const bool fused = !(g.path == MOE_PATH_GEMM || (g.path == MOE_PATH_AUTO && T > g.gemv_max_tokens)) &&
@@ -463,6 +509,20 @@ int moe_debug_check(void *stream) {
   cudaError_t e = cudaStreamSynchronize(static_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) return cuda_fail(e, "cudaStreamSynchronize");
   return check_device_error();
+}
+
+int moe_debug_set_wait_ns(unsigned long long ns) {
+  if (!g.init) return fail(MOE_ERR_NOT_INIT, "moe_init has not succeeded");
+  g.W.wait_ns = ns ? ns : MOE_WAIT_NS;
+  return MOE_OK;
+}
+
+int moe_debug_inject(int fault) {
+  if (!g.init) return fail(MOE_ERR_NOT_INIT, "moe_init has not succeeded");
+  if (fault != MOE_INJECT_NONE && fault != MOE_INJECT_SKIP_ROUTER_ARRIVAL)
+    return fail(MOE_ERR_BAD_ARG, "unknown fault %d", fault);
+  g.W.inject = fault;
+  return MOE_OK;
 }
 
 }  // extern "C"

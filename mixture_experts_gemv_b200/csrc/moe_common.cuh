@@ -8,10 +8,12 @@
 #include <cuda_bf16.h>
 #include <stdint.h>
 
+#include "../../include/moe.h"
+
 #define MOE_QK 32          // weights per Q4_0 block
 #define MOE_QBYTES 18      // bytes per Q4_0 block
 #define MOE_MAX_E 512
-#define MOE_WAIT_NS 2000000000ull   // 2 s bound on any device-side wait
+#define MOE_WAIT_NS 2000000000ull   // default bound on any device-side wait: 2 s
 
 // Device error word: code in the low 16 bits, location in the high 16.
 #define MOE_DEV_ERR_TIMEOUT 1u
@@ -61,7 +63,13 @@ struct MoeWork {
   int32_t *n_tiles;   // [1]
   int32_t *pairs;     // [n_pairs][2]: first tile of up to two consecutive tiles of one expert, second present
   int32_t *n_pairs;   // [1]
+  unsigned long long wait_ns;   // bound on every device-side wait of this launch
+  int inject;         // test-only fault (MOE_INJECT_*), 0 in normal operation
 };
+
+// Test-only faults a launch can be asked to simulate (MOE_INJECT_* of moe.h, set with
+// moe_debug_inject): the failure is made by skipping a step, never by a bad address or an
+// unbounded wait, so the kernel still ends on its own when its bounded waits run out.
 
 // ---------------------------------------------------------------- small helpers
 
@@ -146,14 +154,14 @@ __device__ __forceinline__ bool mbar_test(uint64_t *bar, uint32_t parity) {
   return ok != 0;
 }
 
-// Wait for the phase with the given parity to complete, at most MOE_WAIT_NS. Returns
-// false (and records a timeout in *err) when the bound expires.
+// Wait for the phase with the given parity to complete, at most limit_ns. Returns false
+// (and records a timeout in *err) when the bound expires.
 __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, volatile uint32_t *err,
-                                          uint32_t where) {
+                                          uint32_t where, uint64_t limit_ns) {
   if (mbar_test(bar, parity)) return true;
   uint64_t t0 = globaltimer_ns();
   while (!mbar_test(bar, parity)) {
-    if (globaltimer_ns() - t0 > MOE_WAIT_NS) {
+    if (globaltimer_ns() - t0 > limit_ns) {
       report_error(err, MOE_DEV_ERR_TIMEOUT, where);
       return false;
     }
@@ -224,6 +232,12 @@ enum MoeKernelId {
 // Record a CUDA event on `s` before (begin) / after a launch of kernel group `id`; a no-op
 // unless timing is active. Defined in moe_api.cu.
 void moe_prof_mark(cudaStream_t s, int id, bool begin);
+// Count n kernel launches made by this library while timing is active (moe_api.cu).
+void moe_prof_count(int n);
+// Let kernel `fn` use the device's whole opt-in shared memory on the current device. The
+// attribute belongs to each device's context, so it is set once per device (bit `device` of
+// *done_mask records it; setting the same value twice is harmless). Returns false on error.
+bool moe_allow_dyn_smem(const void *fn, unsigned long long *done_mask);
 
 // Host prototypes of the kernel launchers (defined in the .cu files).
 int moe_launch_route_decode(const MoeLaunch &L, const MoeWork &W, const void *x, const float *router_w,

@@ -98,12 +98,12 @@ __device__ __forceinline__ unsigned long long grid_arrive(unsigned long long *ct
   return (old / n + 1ull) * n;
 }
 __device__ bool grid_wait(const unsigned long long *ctr, unsigned long long target, volatile uint32_t *err,
-                          uint32_t where) {
+                          uint32_t where, uint64_t limit_ns) {
   bool ok = true;
   if (ld_acquire_u64(ctr) < target) {
     const uint64_t t0 = globaltimer_ns();
     while (ld_acquire_u64(ctr) < target) {
-      if (globaltimer_ns() - t0 > MOE_WAIT_NS) {
+      if (globaltimer_ns() - t0 > limit_ns) {
         report_error(err, MOE_DEV_ERR_TIMEOUT, where);
         ok = false;
         break;
@@ -119,20 +119,20 @@ __device__ __forceinline__ void named_arrive(int id, int n) {
 // Grid barrier of the compute and epilogue warps (the named barrier kBarTeam inside the CTA).
 // An expired wait sets *abort; the caller keeps going.
 __device__ void grid_barrier_team(unsigned long long *ctr, volatile uint32_t *err, uint32_t where, int nteam,
-                                  volatile int *abort) {
+                                  volatile int *abort, uint64_t limit_ns) {
   named_sync(kBarTeam, nteam);
-  if (threadIdx.x == 0 && !grid_wait(ctr, grid_arrive(ctr), err, where)) *abort = 1;
+  if (threadIdx.x == 0 && !grid_wait(ctr, grid_arrive(ctr), err, where, limit_ns)) *abort = 1;
   named_sync(kBarTeam, nteam);
 }
-// Wait for an mbarrier phase, at most MOE_WAIT_NS; gives up at once when *abort is set and
-// sets it when the bound expires.
+// Wait for an mbarrier phase, at most limit_ns; gives up at once when *abort is set and sets
+// it when the bound expires.
 __device__ bool wait_phase(uint64_t *bar, uint32_t parity, volatile int *abort, volatile uint32_t *err,
-                           uint32_t where) {
+                           uint32_t where, uint64_t limit_ns) {
   if (mbar_test(bar, parity)) return true;
   const uint64_t t0 = globaltimer_ns();
   while (!mbar_test(bar, parity)) {
     if (*abort) return false;
-    if (globaltimer_ns() - t0 > MOE_WAIT_NS) {
+    if (globaltimer_ns() - t0 > limit_ns) {
       report_error(err, MOE_DEV_ERR_TIMEOUT, where);
       *abort = 1;
       return false;
@@ -513,7 +513,7 @@ k_moe_decode(const __nv_bfloat16 *__restrict__ x, const float *y_prev, float eps
       wv[j] = (i + 3 < i1) ? __ldg(reinterpret_cast<const float4 *>(wr + i)) : make_float4(0.f, 0.f, 0.f, 0.f);
     }
     __syncthreads();   // the x copy's mbarrier is initialised; sh.part is free
-    wait_phase(&sh.xbar, 0u, &sh.abort, W.err, 26);
+    wait_phase(&sh.xbar, 0u, &sh.abort, W.err, 26, W.wait_ns);
     float acc[kFMaxT];
 #pragma unroll
     for (int t = 0; t < kFMaxT; ++t) acc[t] = 0.f;
@@ -556,10 +556,13 @@ k_moe_decode(const __nv_bfloat16 *__restrict__ x, const float *y_prev, float eps
   // arrive at the grid barrier; the thread that arrives waits
   __syncthreads();
   unsigned long long target = 0;
-  if (tid == 0) target = grid_arrive(W.gbar);
+  // test-only fault: CTA 0 leaves without arriving, so every other CTA's bounded wait below
+  // runs out and reports a timeout
+  const bool skip_arrival = W.inject == MOE_INJECT_SKIP_ROUTER_ARRIVAL && blockIdx.x == 0;
+  if (tid == 0 && !skip_arrival) target = grid_arrive(W.gbar);
   // every token's activations, converted in place (x was copied into the activation region at
   // the start) while the other CTAs finish their logits: one (token, block) per thread
-  if (wait_phase(&sh.xbar, 0u, &sh.abort, W.err, 26)) {
+  if (wait_phase(&sh.xbar, 0u, &sh.abort, W.err, 26, W.wait_ns)) {
     for (int blk = tid; blk < T * nb; blk += blockDim.x) {
       const int t = blk / nb, b = blk - t * nb;
       const uint4 *src = reinterpret_cast<const uint4 *>(xs + (size_t)t * d + (size_t)b * MOE_QK);
@@ -579,10 +582,10 @@ k_moe_decode(const __nv_bfloat16 *__restrict__ x, const float *y_prev, float eps
       stage_block_t(v, (b >> 2) & 1, xs + (size_t)t * d + (size_t)b * MOE_QK, ss + (size_t)t * nb + b);
     }
   }
-  if (tid == 0) sh.ok = grid_wait(W.gbar, target, W.err, 20) ? 1 : 0;
+  if (tid == 0) sh.ok = (!skip_arrival && grid_wait(W.gbar, target, W.err, 20, W.wait_ns)) ? 1 : 0;
   __syncthreads();
   if (!sh.ok) {
-    if (tid == 0) mbar_wait(&sh.xbar, 0u, W.err, 27);   // no copy may land after the CTA exits
+    if (tid == 0) mbar_wait(&sh.xbar, 0u, W.err, 27, W.wait_ns);   // no copy may land after the CTA exits
     return;
   }
 
@@ -675,7 +678,7 @@ k_moe_decode(const __nv_bfloat16 *__restrict__ x, const float *y_prev, float eps
       for (; !wk.done(); ++it) {
         const int slot = it % kFStages;
         if (it >= kFStages &&
-            !wait_phase(&sh.empty[slot], (uint32_t)(it / kFStages - 1) & 1u, &sh.abort, W.err, 24))
+            !wait_phase(&sh.empty[slot], (uint32_t)(it / kFStages - 1) & 1u, &sh.abort, W.err, 24, W.wait_ns))
           break;
         const FChunk c = wk.cur(upe_g, upe_d);
         const int e = sh.act[c.a];
@@ -695,7 +698,7 @@ k_moe_decode(const __nv_bfloat16 *__restrict__ x, const float *y_prev, float eps
       }
       // every copy issued has landed before this warp leaves (at once unless the call aborted)
       for (int q = it - 1; q >= 0 && q >= it - kFStages; --q)
-        mbar_wait(&sh.full[q % kFStages], (uint32_t)(q / kFStages) & 1u, W.err, 28);
+        mbar_wait(&sh.full[q % kFStages], (uint32_t)(q / kFStages) & 1u, W.err, 28, W.wait_ns);
     }
     return;
   }
@@ -734,11 +737,11 @@ k_moe_decode(const __nv_bfloat16 *__restrict__ x, const float *y_prev, float eps
       const FChunk c = wk.cur(upe_g, upe_d);
       if (c.down && !down_phase) {
         // all h written (the epilogue warp included) before any CTA reads it
-        grid_barrier_team(W.gbar, W.err, 21, nteam, &sh.abort);
+        grid_barrier_team(W.gbar, W.err, 21, nteam, &sh.abort, W.wait_ns);
         down_phase = true;
       }
       const int slot = it % kFStages;
-      const bool okw = wait_phase(&sh.full[slot], (uint32_t)(it / kFStages) & 1u, &sh.abort, W.err, 22);
+      const bool okw = wait_phase(&sh.full[slot], (uint32_t)(it / kFStages) & 1u, &sh.abort, W.err, 22, W.wait_ns);
       const int e = sh.act[c.a];
       const int cnt = sh.counts[e];
       const int off = sh.offsets[e];
@@ -824,7 +827,7 @@ k_moe_decode(const __nv_bfloat16 *__restrict__ x, const float *y_prev, float eps
       if (lane == 0) mbar_arrive(&sh.empty[slot]);   // this warp's last read of the stage
       wk.advance(c.n, sh.seq, upe_g, upe_d);
     }
-    if (!down_phase) grid_barrier_team(W.gbar, W.err, 21, nteam, &sh.abort);   // no down rows here
+    if (!down_phase) grid_barrier_team(W.gbar, W.err, 21, nteam, &sh.abort, W.wait_ns);   // no down rows here
     for (int q = pass < 2 ? 0 : pass - 2; q < pass; ++q) named_sync(kBarEmpty0 + (q & 1), nteam);
   } else {
     // the epilogue warp: the same sequence of chunks and passes
@@ -833,7 +836,7 @@ k_moe_decode(const __nv_bfloat16 *__restrict__ x, const float *y_prev, float eps
     while (!wk.done()) {
       const FChunk c = wk.cur(upe_g, upe_d);
       if (c.down && !down_phase) {
-        grid_barrier_team(W.gbar, W.err, 21, nteam, &sh.abort);
+        grid_barrier_team(W.gbar, W.err, 21, nteam, &sh.abort, W.wait_ns);
         down_phase = true;
       }
       const int e = sh.act[c.a];
@@ -873,10 +876,10 @@ k_moe_decode(const __nv_bfloat16 *__restrict__ x, const float *y_prev, float eps
       }
       wk.advance(c.n, sh.seq, upe_g, upe_d);
     }
-    if (!down_phase) grid_barrier_team(W.gbar, W.err, 21, nteam, &sh.abort);
+    if (!down_phase) grid_barrier_team(W.gbar, W.err, 21, nteam, &sh.abort, W.wait_ns);
   }
   // ---------------------------------------------------------------- phase 4: combine
-  grid_barrier_team(W.gbar, W.err, 23, nteam, &sh.abort);
+  grid_barrier_team(W.gbar, W.err, 23, nteam, &sh.abort, W.wait_ns);
   if (sh.abort) return;
   const int ti = wq < nwc ? tid : nct + lane;
   const int r0 = (int)((long long)d * blockIdx.x / gridDim.x), r1 = (int)((long long)d * (blockIdx.x + 1) / gridDim.x);
@@ -926,14 +929,11 @@ int moe_launch_fused_decode(const MoeLaunch &L, const MoeWork &W, const void *x,
                             int d, int f, int E, int k, float *out, int num_sms) {
   if (!moe_fused_decode_supported(T, d, f, E, k)) return -2;
   const FusedSmem fs = fused_smem(T, d, f);
-  static size_t set[2] = {0, 0};
+  static unsigned long long smem_ok[2] = {0ull, 0ull};   // per device, per kernel
   const bool norm_in = y_prev != nullptr;
-  if (fs.total > set[norm_in]) {
-    if (cudaFuncSetAttribute(norm_in ? k_moe_decode<true> : k_moe_decode<false>,
-                             cudaFuncAttributeMaxDynamicSharedMemorySize, (int)fs.total) != cudaSuccess)
-      return -1;
-    set[norm_in] = fs.total;
-  }
+  if (!moe_allow_dyn_smem(reinterpret_cast<const void *>(norm_in ? k_moe_decode<true> : k_moe_decode<false>),
+                          &smem_ok[norm_in]))
+    return -1;
   const int G = (d / MOE_QK + kGran - 1) / kGran;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(num_sms);
@@ -952,6 +952,7 @@ int moe_launch_fused_decode(const MoeLaunch &L, const MoeWork &W, const void *x,
                          router_w, router_scale, gate_up_q4, down_q4, expert_scale, T, d, f, E, k, out,
                          fs.stage_bytes, fs.x_bytes, fs.red_half, W);
   if (e != cudaSuccess) return -1;
+  moe_prof_count(1);
   moe_prof_mark(L.stream, MOE_K_FUSED, false);
   return 0;
 }

@@ -406,7 +406,7 @@ k_moe_gemm(const __grid_constant__ CUtensorMap tmap_h, const __nv_bfloat16 *__re
       if (gi < total) {
         const int si = gi % kStages;
         const uint32_t par = ((uint32_t)(gi / kStages) & 1u) ^ 1u;
-        if (!mbar_wait(&bars.empty[si], par, W.err, 10)) { ok = false; break; }
+        if (!mbar_wait(&bars.empty[si], par, W.err, 10, W.wait_ns)) { ok = false; break; }
         issue(isrc, iks, si);
         adv(ijj, iks, isrc);
       }
@@ -422,7 +422,7 @@ k_moe_gemm(const __grid_constant__ CUtensorMap tmap_h, const __nv_bfloat16 *__re
       for (int item = blockIdx.x; item < n_items && ok; item += gridDim.x, ++j) {
         const int b = j & 1;
         const uint32_t upar = ((uint32_t)(j >> 1) & 1u) ^ 1u;
-        if (!mbar_wait(&bars.acc_empty[b], upar, W.err, 11)) { ok = false; break; }
+        if (!mbar_wait(&bars.acc_empty[b], upar, W.err, 11, W.wait_ns)) { ok = false; break; }
         tc_fence_after();
         // the second half only where the item holds a second tile
         int tile;
@@ -432,7 +432,7 @@ k_moe_gemm(const __grid_constant__ CUtensorMap tmap_h, const __nv_bfloat16 *__re
         for (int ks = 0; ks < ksteps; ++ks, ++it) {
           const int s = it % kStages;
           const uint32_t par = (uint32_t)(it / kStages) & 1u;
-          if (!mbar_wait(&bars.full[s], par, W.err, 12)) { ok = false; break; }
+          if (!mbar_wait(&bars.full[s], par, W.err, 12, W.wait_ns)) { ok = false; break; }
           tc_fence_after();
           const uint32_t a_saddr = sbase + (uint32_t)s * kStageBytes;
           const uint32_t b_saddr = a_saddr + kBOff;
@@ -458,7 +458,7 @@ k_moe_gemm(const __grid_constant__ CUtensorMap tmap_h, const __nv_bfloat16 *__re
     for (int item = blockIdx.x; item < n_items; item += gridDim.x, ++j) {
       const int b = j & 1;
       const uint32_t par = (uint32_t)(j >> 1) & 1u;
-      const bool ok = mbar_wait(&bars.acc_full[b], par, W.err, 13);
+      const bool ok = mbar_wait(&bars.acc_full[b], par, W.err, 13, W.wait_ns);
       if (__any_sync(0xffffffffu, !ok)) { atomicExch(&bars.abort_flag, 1); break; }
       tc_fence_after();
       const int nt = item % n_ntiles;
@@ -599,15 +599,10 @@ int moe_launch_gemm_experts(const MoeLaunch &L, const MoeWork &W, const void *x,
                             const uint8_t *down_q4, const float *expert_scale, int T, int d, int f, int E, int k,
                             float *out, int num_sms, int max_tiles) {
   if (d % BK || d % BN || f % BK || f % (BN / 2)) return -2;
-  static bool attr = false;
-  if (!attr) {
-    if (cudaFuncSetAttribute(k_moe_gemm<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             GemmCfg<true>::kSmemBytes) != cudaSuccess ||
-        cudaFuncSetAttribute(k_moe_gemm<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             GemmCfg<false>::kSmemBytes) != cudaSuccess)
-      return -1;
-    attr = true;
-  }
+  static unsigned long long smem_ok[2] = {0ull, 0ull};   // per device, per kernel
+  if (!moe_allow_dyn_smem(reinterpret_cast<const void *>(k_moe_gemm<true>), &smem_ok[0]) ||
+      !moe_allow_dyn_smem(reinterpret_cast<const void *>(k_moe_gemm<false>), &smem_ok[1]))
+    return -1;
   moe_prof_mark(L.stream, MOE_K_GEMM_GATEUP, true);
   const uint8_t *gu_end = gate_up_q4 + (size_t)E * 2 * f * (d / MOE_QK) * MOE_QBYTES;
   const uint8_t *dn_end = down_q4 + (size_t)E * d * (f / MOE_QK) * MOE_QBYTES;
@@ -617,14 +612,17 @@ int moe_launch_gemm_experts(const MoeLaunch &L, const MoeWork &W, const void *x,
   k_moe_gemm<true><<<num_sms, kThreads, kSmemG, L.stream>>>(th, static_cast<const __nv_bfloat16 *>(x), gate_up_q4,
                                                             gu_end, expert_scale, d, f, k, W);
   if (launch_err()) return -1;
+  moe_prof_count(1);
   moe_prof_mark(L.stream, MOE_K_GEMM_GATEUP, false);
   moe_prof_mark(L.stream, MOE_K_GEMM_DOWN, true);
   k_moe_gemm<false><<<num_sms, kThreads, kSmemD, L.stream>>>(th, W.hb, down_q4, dn_end, expert_scale, d, f, k, W);
   if (launch_err()) return -1;
+  moe_prof_count(1);
   moe_prof_mark(L.stream, MOE_K_GEMM_DOWN, false);
   moe_prof_mark(L.stream, MOE_K_COMBINE, true);
   k_combine<<<4 * num_sms, 256, 0, L.stream>>>(reinterpret_cast<const __nv_bfloat16 *>(W.yslot), T, d, k, out);
   if (launch_err()) return -1;
+  moe_prof_count(1);
   moe_prof_mark(L.stream, MOE_K_COMBINE, false);
   return 0;
 }

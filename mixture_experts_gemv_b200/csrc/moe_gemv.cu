@@ -73,7 +73,7 @@ k_gateup_gemv(const uint8_t *__restrict__ gate_up_q4, int d, int f, int k, int n
     const GuChunk c = gu_chunk(u, u1, upe);
     const int slot = it % nstages;
     const uint32_t par = (uint32_t)(it / nstages) & 1u;
-    const bool ok = mbar_wait(&ring.full[slot], par, W.err, 1);
+    const bool ok = mbar_wait(&ring.full[slot], par, W.err, 1, W.wait_ns);
     if (__syncthreads_or(!ok)) return;
 
     const int e = W.act[c.a];
@@ -189,7 +189,7 @@ k_down_gemv_combine(const uint8_t *__restrict__ down_q4, const float *__restrict
     const DnChunk c = dn_chunk(u, u1, upe);
     const int slot = it % nstages;
     const uint32_t par = (uint32_t)(it / nstages) & 1u;
-    const bool ok = mbar_wait(&ring.full[slot], par, W.err, 2);
+    const bool ok = mbar_wait(&ring.full[slot], par, W.err, 2, W.wait_ns);
     if (__syncthreads_or(!ok)) return;
 
     const int e = W.act[c.a];
@@ -310,25 +310,20 @@ int moe_launch_gemv_experts(const MoeLaunch &L, const MoeWork &W, const uint8_t 
   if (gu_st < 2 || dn_st < 2) return -2;
   const size_t gu_smem = (size_t)gu_st * gu_stage + gu_extra, dn_smem = (size_t)dn_st * dn_stage + dn_extra;
   const bool aligned = (nb % kGran) == 0;
-  static size_t gu_set[2] = {0, 0}, dn_set = 0;
+  static unsigned long long smem_ok[3] = {0ull, 0ull, 0ull};   // per device, per kernel
   auto gu_kernel = aligned ? k_gateup_gemv<true> : k_gateup_gemv<false>;
-  if (gu_smem > gu_set[aligned]) {
-    if (cudaFuncSetAttribute(gu_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)gu_smem) != cudaSuccess)
-      return -1;
-    gu_set[aligned] = gu_smem;
-  }
-  if (dn_smem > dn_set) {
-    if (cudaFuncSetAttribute(k_down_gemv_combine, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)dn_smem) != cudaSuccess)
-      return -1;
-    dn_set = dn_smem;
-  }
+  if (!moe_allow_dyn_smem(reinterpret_cast<const void *>(gu_kernel), &smem_ok[aligned]) ||
+      !moe_allow_dyn_smem(reinterpret_cast<const void *>(k_down_gemv_combine), &smem_ok[2]))
+    return -1;
   moe_prof_mark(L.stream, MOE_K_GATEUP, true);
   gu_kernel<<<num_sms, 32 * G, gu_smem, L.stream>>>(gate_up_q4, d, f, k, gu_st, W);
   if (launch_err()) return -1;
+  moe_prof_count(1);
   moe_prof_mark(L.stream, MOE_K_GATEUP, false);
   moe_prof_mark(L.stream, MOE_K_DOWN, true);
   k_down_gemv_combine<<<num_sms, kDnThreads, dn_smem, L.stream>>>(down_q4, expert_scale, T, d, f, k, dn_st, out, W);
   if (launch_err()) return -1;
+  moe_prof_count(1);
   moe_prof_mark(L.stream, MOE_K_DOWN, false);
   return 0;
 }

@@ -21,7 +21,13 @@
 // must start at zero are cleared at the start of every call (cudaMemsetAsync on the
 // caller's stream), and two calls whose work overlaps on the GPU (different streams, or
 // different host threads) race on the array.
+//
+// One word of the array is the device error word of these calls: a device-side wait that
+// runs out of time records itself there (the kernels then end early and `out` is not fully
+// written). It stays set until moe_layer_forward_static_check reads and clears it.
+#include <atomic>
 #include <cstdio>
+#include <mutex>
 
 #include "../../include/moe.h"
 #include "moe_common.cuh"
@@ -48,18 +54,29 @@ constexpr size_t kOffH = align_up(kOffXblk + kT * (kD / 32) * 8);
 constexpr size_t kOffYbuf = align_up(kOffH + kS * kF * 4);
 constexpr size_t kCounterWords = 2 + kD / 8;
 constexpr size_t kOffCounters = align_up(kOffYbuf + kS * kD * 4);
-constexpr size_t kEnd = align_up(kOffCounters + kCounterWords * 4);
+constexpr size_t kOffErr = align_up(kOffCounters + kCounterWords * 4);   // device error word
+constexpr size_t kEnd = align_up(kOffErr + 16);
 static_assert(kEnd <= MOE_STATIC_SCRATCH_BYTES, "static scratch layout exceeds MOE_STATIC_SCRATCH_BYTES");
 
 static __device__ __align__(256) unsigned char g_moe_static_scratch[MOE_STATIC_SCRATCH_BYTES];
 
 struct StaticDevice {
-  bool ready = false;
+  std::atomic<bool> ready{false};     // set (release) after scratch and num_sms are stored
   unsigned char *scratch = nullptr;   // device address of g_moe_static_scratch
   int num_sms = 0;
 };
 constexpr int kMaxDevices = 64;
 StaticDevice g_dev[kMaxDevices];
+std::mutex g_setup;   // the one-time set-up of a device runs under it (first calls may race)
+
+int current_device(int *dev, char *msg, size_t n) {
+  const cudaError_t e = cudaGetDevice(dev);
+  if (e != cudaSuccess || *dev < 0 || *dev >= kMaxDevices) {
+    snprintf(msg, n, "moe_layer_forward_static: cudaGetDevice: %s", cudaGetErrorString(e));
+    return MOE_ERR_CUDA;
+  }
+  return MOE_OK;
+}
 
 }  // namespace
 
@@ -91,31 +108,32 @@ extern "C" int moe_layer_forward_static(const void *x, const float *router_w, co
   if (T == 0) return MOE_OK;
 
   int dev = -1;
-  cudaError_t e = cudaGetDevice(&dev);
-  if (e != cudaSuccess || dev < 0 || dev >= kMaxDevices) {
-    snprintf(msg, sizeof msg, "moe_layer_forward_static: cudaGetDevice: %s", cudaGetErrorString(e));
-    return moe_report_error(MOE_ERR_CUDA, msg);
-  }
+  if (current_device(&dev, msg, sizeof msg) != MOE_OK) return moe_report_error(MOE_ERR_CUDA, msg);
+  cudaError_t e;
   StaticDevice &sd = g_dev[dev];
-  if (!sd.ready) {
-    // one-time set-up for this device, made while it is current
-    int major = 0, minor = 0, sms = 0;
-    cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev);
-    cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev);
-    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-    if (major != 10 || minor != 0) {
-      snprintf(msg, sizeof msg, "moe_layer_forward_static: device %d is sm_%d%d, not sm_100", dev, major, minor);
-      return moe_report_error(MOE_ERR_UNSUPPORTED_DEVICE, msg);
+  if (!sd.ready.load(std::memory_order_acquire)) {
+    // one-time set-up for this device, made while it is current; host threads making their
+    // first call at the same time wait here for the one that does it
+    std::lock_guard<std::mutex> lock(g_setup);
+    if (!sd.ready.load(std::memory_order_relaxed)) {
+      int major = 0, minor = 0, sms = 0;
+      cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev);
+      cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev);
+      cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+      if (major != 10 || minor != 0) {
+        snprintf(msg, sizeof msg, "moe_layer_forward_static: device %d is sm_%d%d, not sm_100", dev, major, minor);
+        return moe_report_error(MOE_ERR_UNSUPPORTED_DEVICE, msg);
+      }
+      void *p = nullptr;
+      e = cudaGetSymbolAddress(&p, g_moe_static_scratch);
+      if (e != cudaSuccess || p == nullptr) {
+        snprintf(msg, sizeof msg, "moe_layer_forward_static: cudaGetSymbolAddress: %s", cudaGetErrorString(e));
+        return moe_report_error(MOE_ERR_CUDA, msg);
+      }
+      sd.scratch = static_cast<unsigned char *>(p);
+      sd.num_sms = sms;
+      sd.ready.store(true, std::memory_order_release);
     }
-    void *p = nullptr;
-    e = cudaGetSymbolAddress(&p, g_moe_static_scratch);
-    if (e != cudaSuccess || p == nullptr) {
-      snprintf(msg, sizeof msg, "moe_layer_forward_static: cudaGetSymbolAddress: %s", cudaGetErrorString(e));
-      return moe_report_error(MOE_ERR_CUDA, msg);
-    }
-    sd.scratch = static_cast<unsigned char *>(p);
-    sd.num_sms = sms;
-    sd.ready = true;
   }
 
   unsigned char *b = sd.scratch;
@@ -136,7 +154,9 @@ extern "C" int moe_layer_forward_static(const void *x, const float *router_w, co
   W.ybuf = reinterpret_cast<float *>(b + kOffYbuf);
   W.yslot = W.ybuf;
   W.counters = reinterpret_cast<uint32_t *>(b + kOffCounters);
-  W.err = nullptr;   // no error word: an expired device wait ends the kernels early
+  W.err = reinterpret_cast<volatile uint32_t *>(b + kOffErr);   // sticky until the check call clears it
+  W.wait_ns = MOE_WAIT_NS;
+  W.inject = MOE_INJECT_NONE;
 
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   e = cudaMemsetAsync(W.counters, 0, kCounterWords * 4, s);
@@ -154,6 +174,32 @@ extern "C" int moe_layer_forward_static(const void *x, const float *router_w, co
   if (rc != 0) {
     snprintf(msg, sizeof msg, "moe_layer_forward_static: GEMV launch: %s", cudaGetErrorString(cudaGetLastError()));
     return moe_report_error(MOE_ERR_CUDA, msg);
+  }
+  return MOE_OK;
+}
+
+extern "C" int moe_layer_forward_static_check(void *stream) {
+  char msg[256];
+  int dev = -1;
+  if (current_device(&dev, msg, sizeof msg) != MOE_OK) return moe_report_error(MOE_ERR_CUDA, msg);
+  StaticDevice &sd = g_dev[dev];
+  if (!sd.ready.load(std::memory_order_acquire)) return MOE_OK;   // no call has run on this device
+  cudaError_t e = cudaStreamSynchronize(static_cast<cudaStream_t>(stream));
+  uint32_t v = 0;
+  if (e == cudaSuccess) e = cudaMemcpy(&v, sd.scratch + kOffErr, sizeof v, cudaMemcpyDeviceToHost);
+  if (e == cudaSuccess && v != 0) {
+    const uint32_t zero = 0;
+    e = cudaMemcpy(sd.scratch + kOffErr, &zero, sizeof zero, cudaMemcpyHostToDevice);
+  }
+  if (e != cudaSuccess) {
+    snprintf(msg, sizeof msg, "moe_layer_forward_static_check: %s", cudaGetErrorString(e));
+    return moe_report_error(MOE_ERR_CUDA, msg);
+  }
+  if (v != 0) {
+    snprintf(msg, sizeof msg,
+             "moe_layer_forward_static: a device wait timed out (code %u at site %u); the output of that call "
+             "is not valid", v & 0xffffu, v >> 16);
+    return moe_report_error(MOE_ERR_DEVICE_TIMEOUT, msg);
   }
   return MOE_OK;
 }

@@ -31,6 +31,7 @@ int moe_launch_rmsnorm(cudaStream_t s, const float *y, void *x_out, int T, int d
   moe_prof_mark(s, MOE_K_NORM, true);
   k_rmsnorm_bf16<<<T, 256, 0, s>>>(y, static_cast<__nv_bfloat16 *>(x_out), d, eps);
   if (cudaGetLastError() != cudaSuccess) return -1;
+  moe_prof_count(1);
   moe_prof_mark(s, MOE_K_NORM, false);
   return 0;
 }

@@ -460,6 +460,7 @@ int moe_launch_route_decode(const MoeLaunch &L, const MoeWork &W, const void *x,
   k_route_decode<<<grid, kRouteThreads, 0, L.stream>>>(static_cast<const __nv_bfloat16 *>(x), router_w,
                                                         router_scale, T, d, E, k, W);
   if (launch_err()) return -1;
+  moe_prof_count(1);
   moe_prof_mark(L.stream, MOE_K_ROUTE, false);
   return 0;
 }
@@ -493,6 +494,7 @@ int moe_launch_route_prefill(const MoeLaunch &L, const MoeWork &W, const void *x
   if (launch_err()) return -1;
   k_perm_place<<<nc, kRouteThreads, 0, L.stream>>>(S, E, ccnt, W);
   if (launch_err()) return -1;
+  moe_prof_count(5);   // router product, top-k, count, scan, place
   if (want_xprep) {
     const int nb = d / MOE_QK;
     const int items = T * nb;
@@ -500,6 +502,7 @@ int moe_launch_route_prefill(const MoeLaunch &L, const MoeWork &W, const void *x
     if (grid > 4 * num_sms) grid = 4 * num_sms;
     k_prep_x<<<grid, 256, 0, L.stream>>>(xb, T, d, W);
     if (launch_err()) return -1;
+    moe_prof_count(1);
   }
   moe_prof_mark(L.stream, MOE_K_ROUTE, false);
   return 0;

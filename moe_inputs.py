@@ -159,23 +159,40 @@ WORKLOADS = (
 )
 
 
-def make_workload(name: str, n_layers: int | None = None) -> Workload:
+def make_layers(indices, seed: int = 0, threads: int = 8) -> list:
+    """make_layer(seed, i) for every i of `indices`, drawn on a few threads at once (each
+    layer has its own generators, so the bytes do not depend on the threading)."""
+    idx = list(indices)
+    if len(idx) <= 1 or threads <= 1:
+        return [make_layer(seed, i) for i in idx]
+    from concurrent.futures import ThreadPoolExecutor
+    with ThreadPoolExecutor(max_workers=min(threads, len(idx))) as ex:
+        return list(ex.map(lambda i: make_layer(seed, i), idx))
+
+
+def make_workload(name: str, n_layers: int | None = None, layer_fn=None) -> Workload:
     """Build one named workload; weights always come from seed 0 (layer i: [0, id, i]).
 
     skewed_T512 biases the router logits by 2.0 * z_e, z the mean-one
-    Zipf(s = 1.1) pmf over expert ids.
+    Zipf(s = 1.1) pmf over expert ids (on a copy of the router weights).
+    `layer_fn(i)`, when given, returns layer i of seed 0 (e.g. from a cache); it must
+    return make_layer(0, i).
     """
+    get = layer_fn if layer_fn is not None else (lambda i: make_layer(0, i))
     if name == "layer_T1":
-        return Workload(name, make_tokens(0, 1), [make_layer(0, 0)])
+        return Workload(name, make_tokens(0, 1), [get(0)])
     if name == "decode_T8":
-        return Workload(name, make_tokens_per_seed(range(1, 9)), [make_layer(0, 0)])
+        return Workload(name, make_tokens_per_seed(range(1, 9)), [get(0)])
     if name == "stack30_T1":
         L = 30 if n_layers is None else n_layers
-        return Workload(name, make_tokens(0, 1), [make_layer(0, i) for i in range(L)])
+        layers = [get(i) for i in range(L)] if layer_fn is not None else make_layers(range(L))
+        return Workload(name, make_tokens(0, 1), layers)
     if name == "prefill_T4096":
-        return Workload(name, make_tokens(3, 4096), [make_layer(0, 0)])
+        return Workload(name, make_tokens(3, 4096), [get(0)])
     if name == "skewed_T512":
-        lw = make_layer(0, 0)
+        lw = get(0)
+        lw = LayerWeights(router_w=lw.router_w.copy(), router_scale=lw.router_scale, gate_up=lw.gate_up,
+                          down=lw.down, expert_scale=lw.expert_scale, d=lw.d, f=lw.f, E=lw.E)
         x = make_tokens(4, 512)
         apply_router_bias(lw, x, 2.0 * zipf_mean_one(lw.E, 1.1))
         return Workload(name, x, [lw])

@@ -77,3 +77,24 @@ def test_code_hash_ignores_comments_only():
     assert bench.strip_c_comments(a) == bench.strip_c_comments(b)
     assert bench.strip_c_comments(a) != bench.strip_c_comments(c)
     assert '"//not a comment"' in bench.strip_c_comments(a)
+
+
+def test_clock_summary_keeps_only_samples_under_load():
+    """Clock samples outside the loaded window (nvidia-smi start-up, idle tail) do not count."""
+    ln = "{sm}, 1965, 700.5, 0x0000000000000000, Not Active, Not Active, Not Active, {cap}"
+    lines = [(0.0, ln.format(sm=345, cap="Not Active")), (1.0, ln.format(sm=1965, cap="Not Active")),
+             (1.2, ln.format(sm=1800, cap="Active")), (1.4, ln.format(sm=1965, cap="Not Active")),
+             (9.0, ln.format(sm=400, cap="Not Active"))]
+    got = bench.summarize_clock_lines(lines, 0.5, 2.0)
+    assert got["samples"] == 3 and got["sm_mhz"] == 1965.0 and got["sm_max_mhz"] == 1965.0
+    assert got["reasons"] == ["sw_power_cap"]
+    assert bench.summarize_clock_lines(lines)["samples"] == 5
+    assert bench.summarize_clock_lines([(0.0, "garbage")]) is None
+
+
+def test_extra_workloads_default_and_none():
+    a = bench.parse([])
+    assert a.workload == "decode_T8"
+    assert bench.extra_workloads(a) == ["layer_T1", "prefill_T4096", "stack30_T1"]
+    assert bench.extra_workloads(bench.parse(["--extra", "none"])) == []
+    assert bench.extra_workloads(bench.parse(["--workload", "prefill_T4096"])) == ["layer_T1", "stack30_T1"]

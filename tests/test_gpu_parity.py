@@ -245,31 +245,56 @@ def test_decode_T8():
     _check_full(wl.x, wl.layers[0], wl.k, moe.MOE_PATH_AUTO)
 
 
-def test_skewed_T512_sampled():
+def _near_tie_band(x, lw, k, lo=1e-6, hi=1e-4):
+    """Unflagged tokens whose FP64 gap between the k-th and (k+1)-th logit lies in (lo, hi]:
+    at logits of magnitude ~58 one FP32 ulp is 3.8e-6, so a gap just above the 1e-6 flag
+    can be below the FP32 router's own rounding. Reported, and still compared exactly."""
+    lg = np.sort(oracle.router_logits(x, lw.router_w), axis=1)[:, ::-1]
+    gap = lg[:, k - 1] - lg[:, k]
+    return int(((gap > lo) & (gap <= hi)).sum()), float(np.abs(lg).max())
+
+
+def test_skewed_T512_every_token():
+    """Every one of the 512 tokens against the oracle (2e-2 on the tensor-core path), plus
+    the skew the workload is meant to have: a few experts above 100 rows, most near empty."""
     wl = mi.make_workload("skewed_T512")
     lw = wl.layers[0]
-    rng = np.random.default_rng(0)
-    tok = np.sort(rng.choice(wl.T, 48, replace=False))
-    res, err = _check_full(wl.x, lw, wl.k, moe.MOE_PATH_AUTO, tokens=tok)
+    band, lmax = _near_tie_band(wl.x, lw, wl.k)
+    print(f"skewed_T512: {band} unflagged tokens with a k-th / (k+1)-th FP64 logit gap in "
+          f"(1e-6, 1e-4]; max |logit| {lmax:.2f}")
+    res, err = _check_full(wl.x, lw, wl.k, moe.MOE_PATH_AUTO)
     counts = res["counts"]
     assert (counts > 100).sum() >= 3 and (counts <= 2).sum() >= 64
+    print(f"skewed_T512: max relative error {err:.3e} over all tokens")
 
 
-def test_prefill_T4096_sampled():
+def test_skewed_T512_every_token_on_the_gemv_path():
+    """The same 512 tokens forced onto the FP32-accumulate GEMV path, at 1e-3."""
+    wl = mi.make_workload("skewed_T512")
+    _check_full(wl.x, wl.layers[0], wl.k, moe.MOE_PATH_GEMV_SPLIT)
+
+
+def test_prefill_T4096_every_token():
+    """All 4,096 tokens (every row of every tile pair and every ragged tail) against the
+    oracle, element by element, at 2e-2."""
     wl = mi.make_workload("prefill_T4096")
-    rng = np.random.default_rng(1)
-    tok = np.sort(rng.choice(wl.T, 32, replace=False))
-    _check_full(wl.x, wl.layers[0], wl.k, moe.MOE_PATH_AUTO, tokens=tok)
+    res, err = _check_full(wl.x, wl.layers[0], wl.k, moe.MOE_PATH_AUTO)
+    print(f"prefill_T4096: max relative error {err:.3e} over all tokens")
 
 
-def test_stack_in_kernel_norm_matches_separate_norm():
+@pytest.fixture(scope="module")
+def stack30():
+    wl = mi.make_workload("stack30_T1")
+    return wl, [DevLayer(lw) for lw in wl.layers]
+
+
+def test_stack_in_kernel_norm_matches_separate_norm(stack30):
     """In a stack, the fused decode kernel normalises the previous layer's output itself; the
     separate path launches moe_rmsnorm_bf16 and the separate decode kernels. Same bits for
-    every layer's x and for the output."""
-    L = 3
-    wl = mi.make_workload("stack30_T1", n_layers=L)
+    every layer's x and for the output, over all 30 layers."""
+    wl, dls = stack30
+    L = len(wl.layers)
     d, f, E, k = mi.D_MODEL, mi.D_FF, mi.N_EXPERTS, wl.k
-    dls = [DevLayer(lw) for lw in wl.layers]
     ensure_init(1, d, f, E, k)
     res = []
     for path in (moe.MOE_PATH_AUTO, moe.MOE_PATH_GEMV_SPLIT):
@@ -286,12 +311,13 @@ def test_stack_in_kernel_norm_matches_separate_norm():
     assert np.array_equal(res[0][0], res[1][0])
 
 
-def test_stack_teacher_forced():
-    """Layer i's oracle consumes the GPU's own bf16 input x_i (recorded by x_trace)."""
-    L = 3
-    wl = mi.make_workload("stack30_T1", n_layers=L)
+def test_stack_teacher_forced(stack30):
+    """All 30 layers: layer i's oracle consumes the GPU's own bf16 input x_i (recorded by
+    x_trace); each layer's output is checked through the next layer's input, the last one
+    directly."""
+    wl, dls = stack30
+    L = len(wl.layers)
     d, f, E, k = mi.D_MODEL, mi.D_FF, mi.N_EXPERTS, wl.k
-    dls = [DevLayer(lw) for lw in wl.layers]
     ensure_init(1, d, f, E, k)
     moe.moe_set_path(moe.MOE_PATH_AUTO, 16)
     out = torch.empty((1, d), dtype=torch.float32, device="cuda:0")
@@ -306,10 +332,12 @@ def test_stack_teacher_forced():
         ref, ids, w, flags = oracle.moe_layer(xs[i], lw.router_w, lw.router_scale, lw.gate_up, lw.down,
                                               lw.expert_scale, k)
         if i + 1 < L:
-            # x_{i+1} = bf16(rmsnorm(out_i)): the 1e-3 output bound plus one bf16 rounding on
-            # each side gives max |dx| <= (1e-3 + 2^-8) max |x|
+            # x_{i+1} = bf16(rmsnorm(out_i)), element by element: the 1e-3 output bound (with
+            # the norm's own scale, 1.1e-3 of the largest element) plus at most one bf16 ulp
+            # of rounding difference, and one ulp of a bf16 value v is at most 2^-7 |v|
             nxt = mi.bf16_bits_to_f32(oracle.rmsnorm_bf16(ref)).astype(np.float64)
             got = mi.bf16_bits_to_f32(xs[i + 1]).astype(np.float64)
-            assert rel_err(got, nxt) <= 1e-3 + 2.0 ** -8
+            bound = 1.1e-3 * np.abs(nxt).max() + 2.0 ** -7 * np.abs(nxt)
+            assert (np.abs(got - nxt) <= bound).all(), f"layer {i}: x_{i + 1} outside the bound"
         else:
             assert rel_err(out.cpu().numpy(), ref) <= TOL_GEMV
