@@ -672,6 +672,19 @@ k_moe_decode(const __nv_bfloat16 *__restrict__ x, const float *y_prev, float eps
   if (wq == nwc) {
     if (lane == 0) {
       const uint64_t pol = l2_evict_first_policy();   // expert weights are read once per call
+      // the down rows this CTA multiplies after the h barrier start moving into L2 now, so
+      // they load while the gate_up rows are multiplied (and during the barrier) and the down
+      // phase reads them from L2
+      {
+        FWalk pf;
+        pf.start(sh.seq[2], sh.seq[3], upe_d, 1);
+        while (pf.left > 0) {
+          const FChunk c = pf.cur(upe_g, upe_d);
+          const int e = sh.act[c.a];
+          bulk_prefetch_l2(down_q4 + (size_t)e * d * rb_d + (size_t)c.r0 * rb_d, (uint32_t)(c.n * kUnit) * rb_d);
+          pf.advance(c.n, sh.seq, upe_g, upe_d);
+        }
+      }
       FWalk wk;
       wk.init(sh.seq, upe_g, upe_d);
       int it = 0;
