@@ -5,8 +5,9 @@ A step is one pass of the whole layer (router, top-k + softmax, permutation, gat
 GeGLU, down + combine) over one batch of synthetic inputs, through the C ABI. The headline
 workload is the eight-request decode batch (decode_T8: T = 8 tokens, d = 2816, f = 704,
 E = 128, k = 8); the same line carries, under "workloads", the single-token layer
-(layer_T1), the 4,096-token prefill (prefill_T4096, the tensor-core half of the metric) and
-the 30-layer single-token stack (stack30_T1), each with its own timing, roofline,
+(layer_T1), the 4,096-token prefill (prefill_T4096, the tensor-core half of the metric), the
+30-layer single-token stack (stack30_T1) and the long prompts of 10,000 and 40,000 tokens
+(prefill_T10000, prefill_T40000: chunks of 4,096 tokens), each with its own timing, roofline,
 end-to-end figure and clocks. Consecutive decode steps rotate over several independent
 layers so that the active experts' weights of one step are not L2-resident in the next
 (inputs larger than L2); a prefill step reads all 428 MB of a layer's experts, a stack step
@@ -38,7 +39,11 @@ import numpy as np  # noqa: E402
 import moe_inputs as mi  # noqa: E402
 
 METRIC = "MoE-layer tokens/s; decode HBM GB/s & prefill TFLOP/s as % of B200 roofline"
-EXTRA_DEFAULT = "layer_T1,prefill_T4096,stack30_T1"
+EXTRA_DEFAULT = "layer_T1,prefill_T4096,stack30_T1,prefill_T10000,prefill_T40000"
+# tokens of each workload, and the workspace's token capacity (longer calls run in chunks)
+WORKLOAD_T = {"layer_T1": 1, "decode_T8": 8, "stack30_T1": 1, "prefill_T4096": 4096, "skewed_T512": 512,
+              "prefill_T10000": 10000, "prefill_T40000": 40000}
+CHUNK_TOKENS = 4096
 
 
 def parse(argv=None):
@@ -376,8 +381,7 @@ class Bench:
     def measure(self, name):
         torch, moe, args, dev = self.torch, self.moe, self.args, self.dev
         stack = name == "stack30_T1"
-        T_of = {"layer_T1": 1, "decode_T8": 8, "stack30_T1": 1, "prefill_T4096": 4096, "skewed_T512": 512}
-        T = T_of[name]
+        T = WORKLOAD_T[name]
         if stack:
             idx = list(range(30))
         else:
@@ -585,11 +589,17 @@ class Bench:
                     "bytes_per_launch": per_launch_bytes, "ms_per_launch": kms / nl}
             dtype = "int16xq4->int32, f32"
         else:
+            # one GEMM launch per chunk of CHUNK_TOKENS tokens: a launch's flops are the step's
+            # over the launches per step
             kms, nl = prof.get("gateup_gemm", (float("nan"), 1))
-            roof = gemm_roofline(avg["gateup_flops"], kms, nl, pk, "k_moe_gemm<gate_up>", name)
+            per_step = max(1, round(nl / args.steps))
+            roof = gemm_roofline(avg["gateup_flops"] / per_step, kms, nl, pk, "k_moe_gemm<gate_up>", name)
             if "down_gemm" in prof:
                 dms, dnl = prof["down_gemm"]
-                extra["roofline_down"] = gemm_roofline(avg["down_flops"], dms, dnl, pk, "k_moe_gemm<down>", name)
+                extra["roofline_down"] = gemm_roofline(avg["down_flops"] / per_step, dms, dnl, pk, "k_moe_gemm<down>",
+                                                       name)
+            if per_step > 1:
+                extra["chunks_per_step"] = per_step
             extra["tflops_per_step"] = avg["flops"] / (ms_step / 1e3) / 1e12
             dtype = "bf16"
         step_gbs = avg["total_bytes"] * n_layers / (ms_step / 1e3) / 1e9
@@ -597,6 +607,7 @@ class Bench:
                "ms_per_step": ms_step, "steps": args.steps, "warmup": args.warmup, "dtype": dtype,
                "config": {"workload": name, "T": T, "d": d, "f": f, "E": E, "k": k, "layers_per_step": n_layers,
                           "layers_rotated": 30 if stack else len(dl), "active_experts_mean": avg["active"],
+                          "chunk_tokens": CHUNK_TOKENS,
                           "l2": ("inputs larger than L2: 30 layers (12.8 GB) per step" if stack else
                                  "inputs larger than L2: consecutive steps use different layers' weights"
                                  if len(dl) > 1 else
@@ -637,9 +648,8 @@ def main():
     import mixture_experts_gemv_b200 as moe
 
     names = [args.workload] + extra_workloads(args)
-    T_max = max({"layer_T1": 1, "decode_T8": 8, "stack30_T1": 1, "prefill_T4096": 4096,
-                 "skewed_T512": 512}[n] for n in names)
-    moe.moe_init(local, T_max, mi.D_MODEL, mi.D_FF, mi.N_EXPERTS, mi.TOP_K)
+    T_max = max(WORKLOAD_T[n] for n in names)
+    moe.moe_init(local, min(T_max, CHUNK_TOKENS), mi.D_MODEL, mi.D_FF, mi.N_EXPERTS, mi.TOP_K)
     moe.moe_set_path(moe.MOE_PATH_AUTO, 16)
     b = Bench(args, moe, dev, ws)
 
@@ -652,7 +662,7 @@ def main():
             "warmup": args.warmup, "ms_per_step": head["ms_per_step"], "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": head["dtype"], "data": "synthetic",
             "config": head["config"], "roofline": head["roofline"]}
-    for kk in ("roofline_down", "tflops_per_step", "step_bytes", "step_gbs", "step_hbm_frac",
+    for kk in ("roofline_down", "chunks_per_step", "tflops_per_step", "step_bytes", "step_gbs", "step_hbm_frac",
                "kernel_ms_per_step", "gpu_launches", "e2e", "clocks", "stack_steps_per_s"):
         if kk in head:
             line[kk] = head[kk]

@@ -55,9 +55,9 @@ extern "C" {
                                    (MOE_PATH_GEMV uses one fused kernel when T <= 8) */
 
 /*
- * moe_init: select `device`, check it is sm_100, and allocate the workspace for
- * forwards of up to max_tokens tokens with d <= max_d, f <= max_f, E <= max_E,
- * k <= max_k. Calling it again releases the previous context first.
+ * moe_init: select `device`, check it is sm_100, and allocate the workspace for passes of
+ * up to max_tokens tokens (longer calls run in chunks of max_tokens) with d <= max_d,
+ * f <= max_f, E <= max_E, k <= max_k. Calling it again releases the previous context first.
  * Limits: 1 <= max_E <= 512, 1 <= max_k <= max_E, max_d and max_f multiples of 32.
  */
 int moe_init(int device, int max_tokens, int max_d, int max_f, int max_E, int max_k);
@@ -71,7 +71,11 @@ int moe_init(int device, int max_tokens, int max_d, int max_f, int max_E, int ma
  *                gate and f..2f-1 up; 16-byte aligned
  *   down_q4      device, Q4_0 [E][d][f/32] blocks, expert-major; 16-byte aligned
  *   expert_scale device, fp32 [E]
- *   T            tokens, 0 <= T <= max_tokens (T = 0 is a no-op)
+ *   T            tokens, T >= 0 (T = 0 is a no-op). A call with T > max_tokens runs as
+ *                consecutive chunks of max_tokens tokens on the path the whole call selects,
+ *                so the workspace stays bounded by moe_init's limits whatever T is; the
+ *                output equals one pass's bit for bit (a token's output depends only on its
+ *                own x).
  *   d, f, E, k   hidden width, expert width, experts, experts per token; d % 32 == 0,
  *                f % 32 == 0, 1 <= k <= E, all within the moe_init limits
  *   out          device, fp32 [T, d] row-major; written, never read
@@ -99,7 +103,8 @@ int moe_rmsnorm_bf16(const float *y, void *x_out, int T, int d, float eps, void 
  *   x_in     device bf16 [T, d], input of layer 0
  *   out      device fp32 [T, d], output of layer L-1
  *   x_trace  optional device bf16 [L, T, d]: receives each layer's input (NULL to skip)
- * Same shape rules as moe_layer_forward. The inter-layer activations live in the workspace.
+ * Same shape rules as moe_layer_forward (a call above max_tokens runs the whole stack on one
+ * chunk of tokens after another). The inter-layer activations live in the workspace.
  * Layers that take the fused decode kernel apply the normalisation inside that kernel (the
  * same arithmetic and bits as moe_rmsnorm_bf16), so such a stack is one launch per layer.
  */
@@ -120,7 +125,8 @@ void moe_destroy(void);
 const char *moe_last_error(void);
 
 /*
- * moe_debug_get_routing: copy the routing of the last moe_layer_forward (device-to-device,
+ * moe_debug_get_routing: copy the routing of the last pass (the last chunk of a chunked call) of
+ * the last moe_layer_forward (device-to-device,
  * enqueued on `stream`): ids int32 [T, k] (per token, logit descending, ties by index),
  * w fp32 [T, k], counts int32 [E], offsets int32 [E + 1], perm int32 [T * k] (slot
  * s = t * k + j of the r-th row of expert e sits at perm[offsets[e] + r], in increasing s).

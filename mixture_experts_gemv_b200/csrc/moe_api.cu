@@ -161,20 +161,25 @@ int check_shapes(int T, int d, int f, int E, int k) {
 
 int check_limits(int T, int d, int f, int E, int k) {
   if (!g.init) return fail(MOE_ERR_NOT_INIT, "moe_init has not succeeded");
-  if (T > g.max_tokens) return fail(MOE_ERR_BAD_ARG, "T = %d exceeds max_tokens = %d", T, g.max_tokens);
+  (void)T;   // any T: calls above max_tokens run in chunks of max_tokens tokens
   if (d > g.max_d || f > g.max_f || E > g.max_E || k > g.max_k)
     return fail(MOE_ERR_BAD_ARG, "shape (d=%d, f=%d, E=%d, k=%d) exceeds the moe_init limits (%d, %d, %d, %d)",
                 d, f, E, k, g.max_d, g.max_f, g.max_E, g.max_k);
   return MOE_OK;
 }
 
+// The path a call of T_call tokens takes (every chunk of a chunked call takes the same one).
+bool gemm_path_for(int T_call) {
+  return (g.path == MOE_PATH_GEMM) || (g.path == MOE_PATH_AUTO && T_call > g.gemv_max_tokens);
+}
+
+// One pass of T <= max_tokens tokens; `gemm` chooses the path.
 int forward_impl(const void *x, const float *router_w, const float *router_scale, const uint8_t *gate_up_q4,
                  const uint8_t *down_q4, const float *expert_scale, int T, int d, int f, int E, int k, float *out,
-                 cudaStream_t stream) {
+                 cudaStream_t stream, bool gemm) {
   MoeLaunch L{stream, false};
   int rc = reset_counters_if_needed(stream);
   if (rc) return rc;
-  const bool gemm = (g.path == MOE_PATH_GEMM) || (g.path == MOE_PATH_AUTO && T > g.gemv_max_tokens);
   // MOE_PATH_GEMV and AUTO below the threshold take the fused decode kernel when the shape
   // fits it (T <= 8), else the separate routing / gate_up / down kernels (MOE_PATH_GEMV_SPLIT).
   if (gemm) {
@@ -391,8 +396,17 @@ int moe_layer_forward(const void *x, const float *router_w, const float *router_
   rc = check_device_error();
   if (rc) return rc;
   if (T == 0) return MOE_OK;
-  return forward_impl(x, router_w, router_scale, gate_up_q4, down_q4, expert_scale, T, d, f, E, k, out,
-                      static_cast<cudaStream_t>(stream));
+  // Calls above the workspace's token capacity run as consecutive chunks of max_tokens tokens
+  // on the path the whole call selects; a token's output depends only on its own x, so the
+  // result is the same as one pass.
+  const bool gemm = gemm_path_for(T);
+  for (int c0 = 0; c0 < T; c0 += g.max_tokens) {
+    const int Tc = T - c0 < g.max_tokens ? T - c0 : g.max_tokens;
+    rc = forward_impl(static_cast<const char *>(x) + (size_t)c0 * d * 2, router_w, router_scale, gate_up_q4, down_q4,
+                      expert_scale, Tc, d, f, E, k, out + (size_t)c0 * d, static_cast<cudaStream_t>(stream), gemm);
+    if (rc) return rc;
+  }
+  return MOE_OK;
 }
 
 int moe_rmsnorm_bf16(const float *y, void *x_out, int T, int d, float eps, void *stream) {
@@ -429,33 +443,39 @@ int moe_stack_forward(const void *x_in, int L, const float *const *router_w, con
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   rc = reset_counters_if_needed(s);
   if (rc) return rc;
+  // Tokens are independent through every layer, so a call above max_tokens runs the whole
+  // stack on one chunk of tokens after another.
+  const bool gemm = gemm_path_for(T);
   // Layers that take the fused decode kernel normalise the previous layer's output inside
   // it (no separate norm launch); the others get moe_rmsnorm_bf16's x. Both give the same x.
-  const bool fused = !(g.path == MOE_PATH_GEMM || (g.path == MOE_PATH_AUTO && T > g.gemv_max_tokens)) &&
-                     g.path != MOE_PATH_GEMV_SPLIT && moe_fused_decode_supported(T, d, f, E, k);
-  const void *xc = x_in;
-  for (int i = 0; i < L; ++i) {
-    char *trace_i = x_trace ? static_cast<char *>(x_trace) + (size_t)i * T * d * 2 : nullptr;
-    float *yo = (i == L - 1) ? out : g.ylayer;
-    if (i > 0 && fused) {
-      // y_prev = g.ylayer is read before the kernel's first grid barrier, yo written after its last
-      MoeLaunch Lf{s, false};
-      rc = moe_launch_fused_decode(Lf, g.W, nullptr, g.ylayer, eps, trace_i, router_w[i], router_scale[i],
-                                   gate_up_q4[i], down_q4[i], expert_scale[i], T, d, f, E, k, yo, g.num_sms);
-      if (rc) return cuda_fail(cudaGetLastError(), "fused decode launch");
-      continue;
-    }
-    if (x_trace) {
-      cudaError_t e = cudaMemcpyAsync(trace_i, xc, (size_t)T * d * 2, cudaMemcpyDeviceToDevice, s);
-      if (e != cudaSuccess) return cuda_fail(e, "x_trace copy");
-    }
-    rc = forward_impl(xc, router_w[i], router_scale[i], gate_up_q4[i], down_q4[i], expert_scale[i], T, d, f, E, k,
-                      yo, s);
-    if (rc) return rc;
-    if (i < L - 1 && !fused) {
-      __nv_bfloat16 *xn = g.xbuf[i & 1];
-      if (moe_launch_rmsnorm(s, yo, xn, T, d, eps)) return cuda_fail(cudaGetLastError(), "rmsnorm launch");
-      xc = xn;
+  for (int c0 = 0; c0 < T; c0 += g.max_tokens) {
+    const int Tc = T - c0 < g.max_tokens ? T - c0 : g.max_tokens;
+    const bool fused = !gemm && g.path != MOE_PATH_GEMV_SPLIT && moe_fused_decode_supported(Tc, d, f, E, k);
+    const void *xc = static_cast<const char *>(x_in) + (size_t)c0 * d * 2;
+    float *out_c = out + (size_t)c0 * d;
+    for (int i = 0; i < L; ++i) {
+      char *trace_i = x_trace ? static_cast<char *>(x_trace) + ((size_t)i * T + c0) * d * 2 : nullptr;
+      float *yo = (i == L - 1) ? out_c : g.ylayer;
+      if (i > 0 && fused) {
+        // y_prev = g.ylayer is read before the kernel's first grid barrier, yo written after its last
+        MoeLaunch Lf{s, false};
+        rc = moe_launch_fused_decode(Lf, g.W, nullptr, g.ylayer, eps, trace_i, router_w[i], router_scale[i],
+                                     gate_up_q4[i], down_q4[i], expert_scale[i], Tc, d, f, E, k, yo, g.num_sms);
+        if (rc) return cuda_fail(cudaGetLastError(), "fused decode launch");
+        continue;
+      }
+      if (x_trace) {
+        cudaError_t e = cudaMemcpyAsync(trace_i, xc, (size_t)Tc * d * 2, cudaMemcpyDeviceToDevice, s);
+        if (e != cudaSuccess) return cuda_fail(e, "x_trace copy");
+      }
+      rc = forward_impl(xc, router_w[i], router_scale[i], gate_up_q4[i], down_q4[i], expert_scale[i], Tc, d, f, E,
+                        k, yo, s, gemm);
+      if (rc) return rc;
+      if (i < L - 1 && !fused) {
+        __nv_bfloat16 *xn = g.xbuf[i & 1];
+        if (moe_launch_rmsnorm(s, yo, xn, Tc, d, eps)) return cuda_fail(cudaGetLastError(), "rmsnorm launch");
+        xc = xn;
+      }
     }
   }
   return MOE_OK;

@@ -199,12 +199,6 @@ __device__ __forceinline__ void bulk_g2s_hint(void *dst, const void *src, uint32
       : "memory");
 }
 
-// Bulk prefetch of [src, src + bytes) into L2 (no shared memory involved, no completion to
-// wait for). src 16-byte aligned, bytes a multiple of 16.
-__device__ __forceinline__ void bulk_prefetch_l2(const void *src, uint32_t bytes) {
-  asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(src), "r"(bytes) : "memory");
-}
-
 __device__ __forceinline__ void fence_proxy_async_smem() {
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }

@@ -34,6 +34,10 @@ constexpr int kFStages = 3;
 constexpr int kFMaxCompute = 12;   // compute warps (128 registers a thread)
 constexpr int kFMinCompute = 8;
 constexpr int kDnParts = 5;               // parts of a down row's blocks (work items: groups x parts)
+static_assert(kFMaxE / 32 <= kFMinCompute + 2 && kFMaxSlots / 32 <= kFMinCompute + 2,
+              "the permutation needs a warp per 32 experts and per 32 slots");
+static_assert(2 * kDnParts * kTX * kDnRows >= (kFMaxSlots / 32) * kFMaxE + 2 * (kFMaxE / 32),
+              "the reduction buffers hold the permutation scratch");
 static_assert(kDnParts == MOE_DN_PARTS && kFMinCompute == MOE_DECODE_MIN_COMPUTE &&
                   kFMaxCompute == MOE_DECODE_MAX_COMPUTE && kGran == 8,
               "the separate decode kernels reproduce this kernel's router slices and down parts");
@@ -71,8 +75,6 @@ struct FusedShared {
     float part[kFMaxCompute + 2][kFMaxT];   // router partial sums (phase 0)
     int32_t pc[kFMaxE + 1];   // exclusive prefix of the per-unit costs over the active experts
   };
-  int32_t wcnt[kFMaxE / 32];  // active experts per 32-expert group
-  uint32_t xb[4];             // cost positions of this CTA's unit boundaries
   int n_act;
   int seq[4];                 // this CTA's unit ranges: gate_up [0, 1), down [2, 3)
   int ok;
@@ -553,17 +555,18 @@ k_moe_decode(const __nv_bfloat16 *__restrict__ x, const float *y_prev, float eps
     }
     __syncthreads();
   }
-  // arrive at the grid barrier; the thread that arrives waits
+  // arrive at the grid barrier: lane 0 of the last warp arrives and waits, while the other
+  // warps convert every token's activations in place (x was copied into the activation region
+  // at the start), one (token, block) per thread
   __syncthreads();
-  unsigned long long target = 0;
   // test-only fault: CTA 0 leaves without arriving, so every other CTA's bounded wait below
   // runs out and reports a timeout
   const bool skip_arrival = W.inject == MOE_INJECT_SKIP_ROUTER_ARRIVAL && blockIdx.x == 0;
-  if (tid == 0 && !skip_arrival) target = grid_arrive(W.gbar);
-  // every token's activations, converted in place (x was copied into the activation region at
-  // the start) while the other CTAs finish their logits: one (token, block) per thread
-  if (wait_phase(&sh.xbar, 0u, &sh.abort, W.err, 26, W.wait_ns)) {
-    for (int blk = tid; blk < T * nb; blk += blockDim.x) {
+  const int bar_tid = (int)blockDim.x - 32, nconv = (int)blockDim.x - 32;
+  if (tid == bar_tid)
+    sh.ok = (!skip_arrival && grid_wait(W.gbar, grid_arrive(W.gbar), W.err, 20, W.wait_ns)) ? 1 : 0;
+  if (tid < nconv && wait_phase(&sh.xbar, 0u, &sh.abort, W.err, 26, W.wait_ns)) {
+    for (int blk = tid; blk < T * nb; blk += nconv) {
       const int t = blk / nb, b = blk - t * nb;
       const uint4 *src = reinterpret_cast<const uint4 *>(xs + (size_t)t * d + (size_t)b * MOE_QK);
       uint4 raw[4];
@@ -582,7 +585,6 @@ k_moe_decode(const __nv_bfloat16 *__restrict__ x, const float *y_prev, float eps
       stage_block_t(v, (b >> 2) & 1, xs + (size_t)t * d + (size_t)b * MOE_QK, ss + (size_t)t * nb + b);
     }
   }
-  if (tid == 0) sh.ok = (!skip_arrival && grid_wait(W.gbar, target, W.err, 20, W.wait_ns)) ? 1 : 0;
   __syncthreads();
   if (!sh.ok) {
     if (tid == 0) mbar_wait(&sh.xbar, 0u, W.err, 27, W.wait_ns);   // no copy may land after the CTA exits
@@ -594,74 +596,34 @@ k_moe_decode(const __nv_bfloat16 *__restrict__ x, const float *y_prev, float eps
     warp_topk_softmax<kFMaxE>(W.logits + (size_t)t * E, E, k, rs, sh.ids + t * k, sh.w + t * k);
   __syncthreads();
   const int S = T * k;
-  const int Ew = (E + 31) & ~31;
-  // per expert (threads e < E): slots routed to it and slots routed to lower experts; per
-  // slot (threads Ew + s): its sorted position = slots of lower experts + earlier slots of
-  // its own expert (the stable counting sort, written out)
-  int my_c = 0;
-  uint32_t my_bal = 0;
-  if (tid < Ew) {
-    int lt = 0;
-    if (tid < E) {
-      for (int s = 0; s < S; ++s) {
-        const int id = sh.ids[s];
-        my_c += id == tid;
-        lt += id < tid;
-      }
-      sh.counts[tid] = my_c;
-      sh.offsets[tid] = lt;
-    }
-    my_bal = __ballot_sync(0xffffffffu, my_c > 0);
-    if (lane == 0) sh.wcnt[wq] = __popc(my_bal);
-  }
-  for (int s = tid - Ew; s < S; s += (int)blockDim.x - Ew) {
-    if (s < 0) break;
-    const int id = sh.ids[s];
-    int p = 0;
-    for (int q = 0; q < S; ++q) {
-      const int iq = sh.ids[q];
-      p += (iq < id) | ((iq == id) & (q < s));
-    }
-    sh.inv[s] = p;
-    sh.perm[p] = s;
-    sh.ptok[p] = s / k;
-  }
   const int upe_g = f / kUnit, upe_d = d / kUnit;
-  __syncthreads();
-  // active experts in ascending order; unit-cost prefix in closed form:
-  // pc[a] = sum over earlier active experts of (kUnitDecode + kUnitToken * T_e)
-  if (tid < E && my_c > 0) {
-    int a = __popc(my_bal & ((1u << lane) - 1u));
-    for (int q = 0; q < wq; ++q) a += sh.wcnt[q];
-    sh.act[a] = tid;
-    sh.pc[a] = kUnitDecode * a + kUnitToken * sh.offsets[tid];
-  }
+  // the stable counting sort of the slots by expert, over the whole CTA (its scratch: the
+  // reduction buffers, unused until the GEMVs)
+  cta_permutation_small<kFMaxSlots / 32, kFMaxE / 32>(sh.ids, S, E, sh.counts, sh.offsets, sh.perm, sh.inv, sh.act, &sh.n_act,
+                                         reinterpret_cast<int32_t *>(red));
+  const int n_act = sh.n_act;
+  // each sorted position's token, and the unit-cost prefix over the active experts in closed
+  // form: pc[a] = sum over earlier active experts of (kUnitDecode + kUnitToken * T_e)
+  for (int p = tid; p < S; p += blockDim.x) sh.ptok[p] = sh.perm[p] / k;
+  for (int a = tid; a < n_act; a += blockDim.x) sh.pc[a] = kUnitDecode * a + kUnitToken * sh.offsets[sh.act[a]];
+  const uint32_t ptot = (uint32_t)(kUnitDecode * n_act + kUnitToken * S);
   if (tid < 4) {
-    int n_act = 0;
-    for (int q = 0; q < Ew / 32; ++q) n_act += sh.wcnt[q];
-    const uint32_t ptot = (uint32_t)(kUnitDecode * n_act + kUnitToken * S);
     const uint32_t upe = tid < 2 ? upe_g : upe_d;
     const uint32_t bb = blockIdx.x + (tid & 1);
-    sh.xb[tid] = (uint32_t)((unsigned long long)upe * ptot * bb / gridDim.x);
     if (bb >= gridDim.x) sh.seq[tid] = n_act * (int)upe;
-    if (tid == 0) {
-      sh.n_act = n_act;
-      sh.pc[n_act] = (int)ptot;
-      sh.offsets[E] = S;
-    }
+    if (tid == 0) sh.pc[n_act] = (int)ptot;
   }
   __syncthreads();
-  const int n_act = sh.n_act;
   // this CTA's unit ranges: boundary j lies in the cost interval of exactly one active expert
   for (int a = tid; a < n_act; a += blockDim.x) {
     const int c = kUnitDecode + kUnitToken * sh.counts[sh.act[a]];
 #pragma unroll
     for (int j = 0; j < 4; ++j) {
       const uint32_t upe = j < 2 ? upe_g : upe_d;
+      const uint32_t xb = (uint32_t)((unsigned long long)upe * ptot * (blockIdx.x + (j & 1)) / gridDim.x);
       const uint32_t lo = upe * (uint32_t)sh.pc[a], hi = upe * (uint32_t)sh.pc[a + 1];
-      const uint32_t xj = sh.xb[j];
-      if (xj >= lo && xj < hi) {
-        const uint32_t inexp = (xj - lo + (uint32_t)c - 1u) / (uint32_t)c;
+      if (xb >= lo && xb < hi) {
+        const uint32_t inexp = (xb - lo + (uint32_t)c - 1u) / (uint32_t)c;
         sh.seq[j] = a * (int)upe + (int)(inexp < upe ? inexp : upe);
       }
     }
@@ -672,19 +634,6 @@ k_moe_decode(const __nv_bfloat16 *__restrict__ x, const float *y_prev, float eps
   if (wq == nwc) {
     if (lane == 0) {
       const uint64_t pol = l2_evict_first_policy();   // expert weights are read once per call
-      // the down rows this CTA multiplies after the h barrier start moving into L2 now, so
-      // they load while the gate_up rows are multiplied (and during the barrier) and the down
-      // phase reads them from L2
-      {
-        FWalk pf;
-        pf.start(sh.seq[2], sh.seq[3], upe_d, 1);
-        while (pf.left > 0) {
-          const FChunk c = pf.cur(upe_g, upe_d);
-          const int e = sh.act[c.a];
-          bulk_prefetch_l2(down_q4 + (size_t)e * d * rb_d + (size_t)c.r0 * rb_d, (uint32_t)(c.n * kUnit) * rb_d);
-          pf.advance(c.n, sh.seq, upe_g, upe_d);
-        }
-      }
       FWalk wk;
       wk.init(sh.seq, upe_g, upe_d);
       int it = 0;
@@ -911,6 +860,7 @@ k_moe_decode(const __nv_bfloat16 *__restrict__ x, const float *y_prev, float eps
 }  // namespace
 
 // Dynamic shared memory of k_moe_decode for these shapes, with the sizes of its regions.
+// (the reduction buffers also hold the permutation's scratch in phase 1)
 struct FusedSmem {
   uint32_t stage_bytes, x_bytes, red_half;   // red_half in floats
   size_t total;

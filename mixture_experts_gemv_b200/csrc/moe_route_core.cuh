@@ -123,61 +123,63 @@ __device__ void warp_topk_softmax_t(const float *lg, int E, int k, float rscale,
   __syncwarp();
 }
 
-// k <= 8: every lane sorts its keys, then five butterfly steps merge sorted top-8 lists
-// (exchange with the partner lane, keep the 8 largest of the 16 by a bitonic merge), so
-// every lane ends with the token's sorted top 8 after 5 shuffle rounds instead of k
-// dependent warp maxima.
+// Order-preserving 32-bit image of a logit (larger float -> larger unsigned; NaN ranks as
+// -inf). Every value maps above 0, which marks a taken or absent entry.
+__device__ __forceinline__ uint32_t logit_ord(float v) {
+  uint32_t u = __float_as_uint(v);
+  if (v != v) u = 0xff800000u;
+  return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+}
+__device__ __forceinline__ float logit_from_ord(uint32_t o) {
+  return __uint_as_float((o & 0x80000000u) ? (o & 0x7fffffffu) : ~o);
+}
+
+// k <= 8: k rounds of a warp maximum, each as two 32-bit warp reductions (redux.sync): the
+// largest logit, then, among the lanes holding it, the lowest expert index. A lane keeps its
+// kMaxPer logits (experts lane + 32 i) and clears the one picked. Picks come out in the
+// order (logit descending, index ascending), the same picks as a sort of the 64-bit keys.
 template <int kMaxPer>
 __device__ void warp_top8_softmax_t(const float *lg, int E, int k, float rscale, int32_t *ids, float *w) {
   const int lane = threadIdx.x & 31;
-  uint64_t t[8];
-#pragma unroll
-  for (int i = 0; i < 8; ++i) t[i] = 0ull;
-  // insert this lane's keys into a sorted (descending) list of 8
+  uint32_t o[kMaxPer];
 #pragma unroll
   for (int i = 0; i < kMaxPer; ++i) {
     const int e = lane + 32 * i;
-    uint64_t v = (e < E) ? topk_key(__ldcg(lg + e), e) : 0ull;
+    o[i] = (e < E) ? logit_ord(__ldcg(lg + e)) : 0u;
+  }
+  uint32_t pick_o[8];
+  int pick_e[8];
 #pragma unroll
-    for (int j = 0; j < 8; ++j) {
-      const uint64_t hi = t[j] > v ? t[j] : v, lo = t[j] > v ? v : t[j];
-      t[j] = hi;
-      v = lo;
+  for (int j = 0; j < 8; ++j) {
+    pick_o[j] = 0u;
+    pick_e[j] = 0;
+    if (j < k) {
+      uint32_t bo = o[0];
+      int bi = 0;
+#pragma unroll
+      for (int i = 1; i < kMaxPer; ++i)
+        if (o[i] > bo) { bo = o[i]; bi = i; }   // strict: the lower index among equal logits
+      const uint32_t mo = __reduce_max_sync(0xffffffffu, bo);
+      const uint32_t cand = (bo == mo) ? (uint32_t)(lane + 32 * bi) : 0xffffffffu;
+      const uint32_t me = __reduce_min_sync(0xffffffffu, cand);
+#pragma unroll
+      for (int i = 0; i < kMaxPer; ++i)
+        if (cand == me && i == bi) o[i] = 0u;   // taken
+      pick_o[j] = mo;
+      pick_e[j] = (int)me;
     }
   }
-#pragma unroll
-  for (int o = 1; o < 32; o <<= 1) {
-    uint64_t u[8];
-#pragma unroll
-    for (int j = 0; j < 8; ++j) u[j] = __shfl_xor_sync(0xffffffffu, t[j], o);
-    // top 8 of two descending lists: pairwise max against the reversed partner list is a
-    // bitonic sequence holding the 8 largest; sort it descending
-#pragma unroll
-    for (int j = 0; j < 8; ++j) t[j] = t[j] > u[7 - j] ? t[j] : u[7 - j];
-#pragma unroll
-    for (int s2 = 4; s2 > 0; s2 >>= 1) {
-#pragma unroll
-      for (int j = 0; j < 8; ++j) {
-        if ((j & s2) == 0) {
-          const uint64_t a2 = t[j], b2 = t[j + s2];
-          t[j] = a2 > b2 ? a2 : b2;
-          t[j + s2] = a2 > b2 ? b2 : a2;
-        }
-      }
-    }
-  }
-  // every lane holds the sorted top 8; lanes j < k publish pick j
-  const float l1 = topk_key_value(t[0]);
+  // softmax over the selected logits, relative to the largest, summed in pick order
+  const float l1 = logit_from_ord(pick_o[0]);
   float part = 0.f;
   float mine_v = 0.f;
   int mine_e = 0;
 #pragma unroll
   for (int j = 0; j < 8; ++j) {
     if (j < k) {
-      const float v = topk_key_value(t[j]);
-      const float ev = expf(v - l1);
+      const float ev = expf(logit_from_ord(pick_o[j]) - l1);
       part += ev;
-      if (j == lane) { mine_v = ev; mine_e = (int)(0xffffffffu - (uint32_t)t[j]); }
+      if (j == lane) { mine_v = ev; mine_e = pick_e[j]; }
     }
   }
   if (lane < k) {
@@ -213,9 +215,10 @@ __device__ __forceinline__ void warp_topk_softmax(const float *lg, int E, int k,
   if constexpr (kMaxE > 256) warp_topk_softmax_t<MOE_MAX_E / 32>(lg, E, k, rscale, ids, w);
 }
 
-// Stable counting sort of S <= 1024 slots by expert id in one warp: ranks from
+// Stable counting sort of S <= kMaxS slots by expert id in one warp: ranks from
 // __match_any_sync in slot order, a warp scan of the counts, then placement.
 constexpr int kSmallPermMax = 1024;
+template <int kMaxS = kSmallPermMax>
 __device__ void warp_permutation_small(const int32_t *ids, int S, int E, int32_t *counts, int32_t *offsets,
                                        int32_t *perm, int32_t *inv, int32_t *act, int32_t *n_act,
                                        int32_t *cnt /* smem [E] */) {
@@ -223,9 +226,9 @@ __device__ void warp_permutation_small(const int32_t *ids, int S, int E, int32_t
   const uint32_t lt = (1u << lane) - 1u;
   for (int e = lane; e < E; e += 32) cnt[e] = 0;
   __syncwarp();
-  int rk[kSmallPermMax / 32], idr[kSmallPermMax / 32];
+  int rk[kMaxS / 32], idr[kMaxS / 32];
 #pragma unroll
-  for (int r = 0; r < kSmallPermMax / 32; ++r) {
+  for (int r = 0; r < kMaxS / 32; ++r) {
     const int s = r * 32 + lane;
     if (r * 32 < S) {
       const int id = (s < S) ? ids[s] : -1 - lane;   // written earlier by this CTA
@@ -262,7 +265,7 @@ __device__ void warp_permutation_small(const int32_t *ids, int S, int E, int32_t
   if (lane == 0) { offsets[E] = c_tot; *n_act = a_tot; }
   __syncwarp();
 #pragma unroll
-  for (int r = 0; r < kSmallPermMax / 32; ++r) {
+  for (int r = 0; r < kMaxS / 32; ++r) {
     const int s = r * 32 + lane;
     if (r * 32 < S && s < S) {
       const int pos = cnt[idr[r]] + rk[r];
@@ -270,6 +273,81 @@ __device__ void warp_permutation_small(const int32_t *ids, int S, int E, int32_t
       inv[s] = pos;
     }
   }
+}
+
+// Stable counting sort of S <= 32 * kSlotWarps slots by expert id (E <= 32 * kExpWarps) by
+// the calling CTA (every thread calls it; the block has at least max(kSlotWarps, kExpWarps)
+// warps): warp w < kSlotWarps ranks its slots s = 32 w + lane among equal ids with
+// __match_any_sync and records its per-expert counts; thread e < E sums the warps' counts
+// of expert e in warp order (giving each warp's base inside the expert), and an exclusive
+// scan over the experts gives the offsets and the active list; each slot's position is then
+// its expert's offset + its warp's base + its rank in the warp.
+// scratch: shared memory of kSlotWarps * E + 2 * kExpWarps ints.
+template <int kSlotWarps, int kExpWarps>
+__device__ void cta_permutation_small(const int32_t *ids, int S, int E, int32_t *counts, int32_t *offsets,
+                                      int32_t *perm, int32_t *inv, int32_t *act, int32_t *n_act,
+                                      int32_t *scratch) {
+  const int tid = threadIdx.x, lane = tid & 31, wq = tid >> 5;
+  int32_t *wc = scratch;                        // [kSlotWarps][E]: slots of expert e in warp w
+  int32_t *tot = scratch + kSlotWarps * E;      // [kExpWarps] count totals, [kExpWarps] active totals
+  for (int i = tid; i < kSlotWarps * E; i += blockDim.x) wc[i] = 0;
+  __syncthreads();
+  int id = -1, rank = 0;
+  if (wq < kSlotWarps) {
+    const int s = wq * 32 + lane;
+    id = s < S ? ids[s] : -1 - lane;            // unique negative keys past the end
+    const uint32_t peers = __match_any_sync(0xffffffffu, id);
+    rank = __popc(peers & ((1u << lane) - 1u));
+    if (s < S && lane == 31 - __clz(peers)) wc[wq * E + id] = __popc(peers);
+  }
+  __syncthreads();
+  // thread e: count of expert e, and the bases of the slot warps inside it
+  int c = 0, ic = 0, ia = 0;
+  if (wq < kExpWarps) {
+    if (tid < E) {
+      for (int w = 0; w < kSlotWarps; ++w) {
+        const int v = wc[w * E + tid];
+        wc[w * E + tid] = c;
+        c += v;
+      }
+    }
+    ic = c;
+    ia = c > 0;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {          // inclusive warp scans of count and active
+      const int nc = __shfl_up_sync(0xffffffffu, ic, o), na = __shfl_up_sync(0xffffffffu, ia, o);
+      if (lane >= o) { ic += nc; ia += na; }
+    }
+    if (lane == 31) { tot[wq] = ic; tot[kExpWarps + wq] = ia; }
+  }
+  __syncthreads();
+  if (wq < kExpWarps) {
+    int bc = 0, ba = 0, tc = 0, ta = 0;
+    for (int w = 0; w < kExpWarps; ++w) {
+      if (w < wq) { bc += tot[w]; ba += tot[kExpWarps + w]; }
+      tc += tot[w];
+      ta += tot[kExpWarps + w];
+    }
+    if (tid < E) {
+      counts[tid] = c;
+      offsets[tid] = bc + ic - c;
+      if (c > 0) act[ba + ia - 1] = tid;
+    }
+    if (tid == 0) {
+      offsets[E] = tc;
+      *n_act = ta;
+    }
+  }
+  __syncthreads();
+  if (wq < kSlotWarps) {
+    const int s = wq * 32 + lane;
+    if (s < S) {
+      const int pos = offsets[id] + wc[wq * E + id] + rank;
+      perm[pos] = s;
+      inv[s] = pos;
+    }
+  }
+  __syncthreads();
 }
 
 }  // namespace

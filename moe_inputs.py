@@ -156,6 +156,8 @@ WORKLOADS = (
     "stack30_T1",       # 30 independent layers of the same shapes, one token
     "prefill_T4096",    # 4,096-token prefill, x from seed 3, unskewed router
     "skewed_T512",      # 512 tokens, x from seed 4, Zipf-biased router
+    "prefill_T10000",   # 10,000-token prefill, x from seed 5 (a long prompt)
+    "prefill_T40000",   # 40,000-token prefill, x from seed 6 (the longest prompt)
 )
 
 
@@ -189,6 +191,10 @@ def make_workload(name: str, n_layers: int | None = None, layer_fn=None) -> Work
         return Workload(name, make_tokens(0, 1), layers)
     if name == "prefill_T4096":
         return Workload(name, make_tokens(3, 4096), [get(0)])
+    if name == "prefill_T10000":
+        return Workload(name, make_tokens(5, 10000), [get(0)])
+    if name == "prefill_T40000":
+        return Workload(name, make_tokens(6, 40000), [get(0)])
     if name == "skewed_T512":
         lw = get(0)
         lw = LayerWeights(router_w=lw.router_w.copy(), router_scale=lw.router_scale, gate_up=lw.gate_up,

@@ -341,3 +341,58 @@ def test_stack_teacher_forced(stack30):
             assert (np.abs(got - nxt) <= bound).all(), f"layer {i}: x_{i + 1} outside the bound"
         else:
             assert rel_err(out.cpu().numpy(), ref) <= TOL_GEMV
+
+
+# ------------------------------------------------------------------ long prompts (chunked)
+
+def _tile_boundary_tokens(T, chunk, k, rng, n_random):
+    """Tokens at the chunk boundaries (the first and last 128 of every chunk) plus n_random
+    others."""
+    edges = set()
+    for c0 in range(0, T, chunk):
+        c1 = min(T, c0 + chunk)
+        edges.update(range(c0, min(c1, c0 + 128)))
+        edges.update(range(max(c0, c1 - 128), c1))
+    rest = np.setdiff1d(np.arange(T), np.fromiter(edges, dtype=np.int64))
+    pick = rng.choice(rest, min(n_random, rest.size), replace=False)
+    return np.sort(np.concatenate([np.fromiter(edges, dtype=np.int64), pick]))
+
+
+def test_chunked_prefill_is_bitwise_one_pass():
+    """A 4,096-token prefill through a workspace of 1,024 tokens (four chunks) gives the bits
+    of one 4,096-token pass: chunking bounds the workspace without changing any output."""
+    import gpu_util
+    wl = mi.make_workload("prefill_T4096")
+    lw = wl.layers[0]
+    d, f, E, k = lw.d, lw.f, lw.E, wl.k
+    dl = DevLayer(lw)
+    x = dev(wl.x)
+    outs = []
+    for cap in (4096, 1024):
+        moe.moe_init(0, cap, d, f, E, k)
+        gpu_util._limits = (cap, d, f, E, k)
+        moe.moe_set_path(moe.MOE_PATH_AUTO, 16)
+        o = torch.full((wl.T, d), float("nan"), dtype=torch.float32, device="cuda:0")
+        moe.moe_layer_forward(x, dl.router_w, dl.router_scale, dl.gate_up, dl.down, dl.expert_scale,
+                              wl.T, d, f, E, k, o)
+        moe.moe_debug_check()
+        outs.append(o)
+    assert torch.equal(outs[0], outs[1])
+    assert moe.moe_workspace_bytes(1024, d, f, E, k) < moe.moe_workspace_bytes(4096, d, f, E, k)
+
+
+def test_prefill_T10000_every_token():
+    """The 10,000-token prompt (three 4,096-token chunks, the last one ragged): every token
+    against the oracle at 2e-2."""
+    wl = mi.make_workload("prefill_T10000")
+    _, err = _check_full(wl.x, wl.layers[0], wl.k, moe.MOE_PATH_AUTO)
+    print(f"prefill_T10000: max relative error {err:.3e} over all tokens")
+
+
+def test_prefill_T40000_boundaries_and_sample():
+    """The 40,000-token prompt (ten chunks): every token of the first and last 128-row tile of
+    each chunk, plus 1,000 random tokens, against the oracle at 2e-2."""
+    wl = mi.make_workload("prefill_T40000")
+    tok = _tile_boundary_tokens(wl.T, 4096, wl.k, np.random.default_rng(2), 1000)
+    _, err = _check_full(wl.x, wl.layers[0], wl.k, moe.MOE_PATH_AUTO, tokens=tok)
+    print(f"prefill_T40000: max relative error {err:.3e} over {tok.size} tokens")
