@@ -38,6 +38,12 @@ TENSOR_ROUTER_W = 1
 TENSOR_GATE_UP = 2
 TENSOR_DOWN = 3
 TENSOR_EXPERT_SCALE = 4
+TENSOR_DENSE_GATE_UP = 5
+TENSOR_DENSE_DOWN = 6
+# Width of the block's dense MLP in the benchmark and full-size tests: the page stores its gate
+# and up rows as one Q4_0 parent but gives no width; the one MLP width it gives for this
+# block is a routed expert's, 704.
+D_FF_DENSE = 704
 
 
 def _rng(config_seed: int, tensor_id: int, layer: int = 0) -> np.random.Generator:
@@ -106,6 +112,14 @@ def make_layer(seed: int = 0, layer: int = 0, d: int = D_MODEL, f: int = D_FF,
                         router_scale=np.array([router_scale], dtype=np.float32),
                         gate_up=gu, down=dn, expert_scale=es.astype(np.float32),
                         d=d, f=f, E=E)
+
+
+def make_dense(seed: int = 0, layer: int = 0, d: int = D_MODEL, f_dense: int = D_FF_DENSE):
+    """The block's dense MLP weights with the experts' recipe: (gate_up [2 f_dense, d/32*18],
+    down [d, f_dense/32*18]) Q4_0 bytes, gate rows first in the one [gate; up] parent."""
+    gu = random_q4_0(_rng(seed, TENSOR_DENSE_GATE_UP, layer), 2 * f_dense, d)
+    dn = random_q4_0(_rng(seed, TENSOR_DENSE_DOWN, layer), d, f_dense)
+    return gu, dn
 
 
 def make_tokens(seed: int, T: int, d: int = D_MODEL) -> np.ndarray:

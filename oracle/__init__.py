@@ -53,6 +53,11 @@ def lib():
         L.oracle_moe_layer.argtypes = [_p, _p, _d, _p, _p, _p, _i, _i, _i, _i, _i, _d,
                                        _p, _p, _p, _p]
         L.oracle_moe_layer.restype = _i
+        L.oracle_dense_mlp.argtypes = [_p, _p, _p, _i, _i, _p, _i, _p]
+        L.oracle_dense_mlp.restype = None
+        L.oracle_block_ffn.argtypes = [_p, _p, _d, _p, _p, _p, _p, _p, _i, _i, _i, _i, _i, _i, _d,
+                                       _p, _p, _p, _p]
+        L.oracle_block_ffn.restype = _i
         L.oracle_rmsnorm_bf16.argtypes = [_p, _i, _i, _d, _p]
         L.oracle_rmsnorm_bf16.restype = None
         L.oracle_num_threads.argtypes = []
@@ -173,6 +178,41 @@ def moe_layer(x_bits, router_w, router_scale, gate_up, down, expert_scale, k: in
     lib().oracle_moe_layer(_ptr(x), _ptr(W), float(np.asarray(router_scale).reshape(-1)[0]),
                            _ptr(gu), _ptr(_c(down, np.uint8)),
                            _ptr(_c(expert_scale, np.float32)), T, d, f, E, k, float(tie_eps),
+                           _ptr(out), _ptr(ids), _ptr(w), _ptr(flags))
+    return out, ids, w, flags
+
+
+def dense_mlp(x_bits, gate_up_dense, down_dense, tokens=None):
+    """The block's dense MLP (GELU-tanh GeGLU of width f_dense) on the given tokens: [n, d] f64."""
+    x = _c(x_bits, np.uint16)
+    T, d = x.shape
+    gu = _c(gate_up_dense, np.uint8)
+    f_dense = gu.shape[0] // 2
+    tok = _c(np.arange(T) if tokens is None else tokens, np.int32)
+    out = np.empty((tok.shape[0], d), dtype=np.float64)
+    lib().oracle_dense_mlp(_ptr(x), _ptr(gu), _ptr(_c(down_dense, np.uint8)), d, f_dense, _ptr(tok),
+                           tok.shape[0], _ptr(out))
+    return out
+
+
+def block_ffn(x_bits, router_w, router_scale, gate_up, down, expert_scale, gate_up_dense, down_dense, k: int,
+              tie_eps: float = TIE_EPS):
+    """Routed layer plus dense MLP for all tokens: (out [T,d] f64, ids, w, flags)."""
+    x = _c(x_bits, np.uint16)
+    T, d = x.shape
+    W = _c(router_w, np.float32)
+    E = W.shape[0]
+    gu = _c(gate_up, np.uint8)
+    f = gu.shape[1] // 2
+    gud = _c(gate_up_dense, np.uint8)
+    f_dense = gud.shape[0] // 2
+    out = np.empty((T, d), dtype=np.float64)
+    ids = np.empty((T, k), dtype=np.int32)
+    w = np.empty((T, k), dtype=np.float64)
+    flags = np.empty(T, dtype=np.uint8)
+    lib().oracle_block_ffn(_ptr(x), _ptr(W), float(np.asarray(router_scale).reshape(-1)[0]), _ptr(gu),
+                           _ptr(_c(down, np.uint8)), _ptr(_c(expert_scale, np.float32)), _ptr(gud),
+                           _ptr(_c(down_dense, np.uint8)), T, d, f, f_dense, E, k, float(tie_eps),
                            _ptr(out), _ptr(ids), _ptr(w), _ptr(flags))
     return out, ids, w, flags
 

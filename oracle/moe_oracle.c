@@ -337,6 +337,51 @@ int oracle_moe_layer(const uint16_t *x, const float *router_w, double router_sca
 }
 
 /*
+ * The block's dense MLP beside the routed experts (page "Gemma 4 26B-A4B it QAT Q4_0 ...
+ * NInfer v3 artifact", table "What is inside": the dense MLP's gate and up rows stored as one
+ * Q4_0 parent). The page gives no width and no formula; the reading taken: a GELU-tanh GeGLU
+ * of width f_dense on every token, like an expert,
+ *   out_dense[t, r] = Wd[r, :] . (gelu_tanh(Wg x_t) * (Wu x_t)),
+ * with [gate; up] = gate_up_dense [2 f_dense][d/32] and Wd = down_dense [d][f_dense/32] Q4_0
+ * blocks. out [n_tokens, d] FP64 for t = tokens[n].
+ */
+void oracle_dense_mlp(const uint16_t *x, const uint8_t *gate_up_dense, const uint8_t *down_dense, int d,
+                      int f_dense, const int32_t *tokens, int n_tokens, double *out)
+{
+#pragma omp parallel for schedule(dynamic, 1)
+    for (int n = 0; n < n_tokens; ++n)
+        oracle_expert_ffn(x + (size_t)tokens[n] * d, gate_up_dense, down_dense, d, f_dense, NULL,
+                          out + (size_t)n * d);
+}
+
+/*
+ * The block's feed-forward output: the routed layer plus the dense MLP, read as a plain sum
+ * (the dense output joins the combine with weight 1):
+ *   out[t, r] = sum_j w_tj s_e y_tj[r] + out_dense[t, r].
+ * out [T, d] FP64; ids, w, flags as oracle_moe_layer. Returns 0.
+ */
+int oracle_block_ffn(const uint16_t *x, const float *router_w, double router_scale, const uint8_t *gate_up,
+                     const uint8_t *down, const float *expert_scale, const uint8_t *gate_up_dense,
+                     const uint8_t *down_dense, int T, int d, int f, int f_dense, int E, int k, double tie_eps,
+                     double *out, int32_t *ids, double *w, uint8_t *flags)
+{
+    if (T <= 0)
+        return 0;
+    oracle_moe_layer(x, router_w, router_scale, gate_up, down, expert_scale, T, d, f, E, k, tie_eps, out, ids, w,
+                     flags);
+    double *dense = (double *)malloc(sizeof(double) * (size_t)T * d);
+    int32_t *tok = (int32_t *)malloc(sizeof(int32_t) * (size_t)T);
+    for (int t = 0; t < T; ++t)
+        tok[t] = t;
+    oracle_dense_mlp(x, gate_up_dense, down_dense, d, f_dense, tok, T, dense);
+    for (size_t i = 0; i < (size_t)T * d; ++i)
+        out[i] += dense[i];
+    free(tok);
+    free(dense);
+    return 0;
+}
+
+/*
  * RMS normalisation with unit gain followed by the bf16 cast, between
  * stacked layers: x[t, i] = bf16_rne(y[t, i] / sqrt(mean_i y[t, i]^2 + eps)).
  */

@@ -405,3 +405,43 @@ def test_oracle_regression_fixture(orc):
     assert ids.ravel().tolist() == [int(v) for v in rows["ids"]]
     assert w.ravel().tolist() == [float(v) for v in rows["w"]]
     assert out.ravel().tolist() == [float(v) for v in rows["out"]]
+
+
+# ------------------------------------------------------------------ the block's dense MLP
+
+def test_dense_mlp_matches_numpy_decode_and_matmul(orc):
+    """The dense MLP (gate rows first in the one [gate; up] parent, GELU-tanh GeGLU, down)
+    against NumPy's float16 decode and matmuls, on every token and on a token subset."""
+    d, fd, T = 96, 64, 5
+    gu, dn = mi.make_dense(11, 0, d, fd)
+    x = mi.make_tokens(12, T, d)
+    got = orc.dense_mlp(x, gu, dn)
+    xv = np_ref.bf16_field_decode(x)
+    Wg = np_ref.decode_q4_0(gu, d)
+    Wd = np_ref.decode_q4_0(dn, fd)
+    ref = (np_ref.gelu_tanh(xv @ Wg[:fd].T) * (xv @ Wg[fd:].T)) @ Wd.T
+    assert got.shape == (T, d)
+    assert np.max(np.abs(got - ref)) <= 1e-13 * np.max(np.abs(ref))
+    sub = orc.dense_mlp(x, gu, dn, tokens=np.array([4, 1]))
+    assert np.array_equal(sub, got[[4, 1]])
+
+
+def test_block_is_routed_layer_plus_dense_mlp(orc):
+    """The block's output is the routed layer's plus the dense MLP's: zero dense weights (code
+    8) leave the routed layer's bits, zero expert weights leave the dense MLP's, and in general
+    the two add up (to FP64 rounding)."""
+    E, d, f, fd, k, T = 6, 64, 32, 96, 2, 4
+    W, gu, dn, es = _tiny_layer(51, E, d, f, 0.05, 0.2)
+    gud, dnd = mi.make_dense(52, 0, d, fd)
+    x = mi.make_tokens(53, T, d)
+    routed, ids, w, fl = orc.moe_layer(x, W, 0.7, gu, dn, es, k)
+    out, ids2, w2, fl2 = orc.block_ffn(x, W, 0.7, gu, dn, es, gud, dnd, k)
+    assert np.array_equal(ids, ids2) and np.array_equal(w, w2)
+    dense = orc.dense_mlp(x, gud, dnd)
+    assert np.max(np.abs(out - (routed + dense))) <= 1e-14 * np.max(np.abs(out))
+    zero_gud = _const_q4(2 * fd, d, 8)
+    out0, *_ = orc.block_ffn(x, W, 0.7, gu, dn, es, zero_gud, dnd, k)
+    assert np.array_equal(out0, routed)
+    zero_gu = np.stack([_const_q4(2 * f, d, 8)] * E)
+    out1, *_ = orc.block_ffn(x, W, 0.7, zero_gu, dn, es, gud, dnd, k)
+    assert np.array_equal(out1, dense)

@@ -30,6 +30,7 @@ MUTANTS = {
     "unstable_perm": ("for (long s = 0; s < S; ++s) {\n        int e = ids[s];",
                       "for (long s = S - 1; s >= 0; --s) {\n        int e = ids[s];"),
     "router_transposed": ("(double)router_w[(size_t)e * d + i]", "(double)router_w[(size_t)i * E + e]"),
+    "dense_subtracted": ("out[i] += dense[i];", "out[i] -= dense[i];"),
 }
 
 
