@@ -91,6 +91,25 @@ int moe_layer_forward(const void *x, const float *router_w, const float *router_
                       float *out, void *stream);
 
 /*
+ * moe_block_forward: the block's feed-forward output, the routed layer plus the block's dense
+ * MLP (same page, table "What is inside": the dense MLP's gate and up rows are one Q4_0
+ * parent; the page gives no width, so it is an argument, and the MLP is read as a GELU-tanh
+ * GeGLU whose output is added to the routed combine):
+ *   out_t = [moe_layer_forward]_t + Wd_dense (gelu_tanh(Wg_dense x_t) * (Wu_dense x_t))
+ *   gate_up_dense_q4  device, Q4_0 [2 f_dense][d/32] blocks: gate rows 0..f_dense-1, then up
+ *                     rows; 16-byte aligned
+ *   down_dense_q4     device, Q4_0 [d][f_dense/32] blocks; 16-byte aligned
+ *   f_dense           positive multiple of 32, <= max_f of moe_init
+ * Other arguments as moe_layer_forward. The dense MLP runs through the layer's own kernels as
+ * one more expert that every token selects with weight 1, in a pass of its own (after the
+ * routed pass of each chunk) whose combine adds into out.
+ */
+int moe_block_forward(const void *x, const float *router_w, const float *router_scale,
+                      const uint8_t *gate_up_q4, const uint8_t *down_q4, const float *expert_scale,
+                      const uint8_t *gate_up_dense_q4, const uint8_t *down_dense_q4, int T, int d,
+                      int f, int f_dense, int E, int k, float *out, void *stream);
+
+/*
  * moe_rmsnorm_bf16: the fixed normalisation between stacked layers,
  *   x[t, i] = bf16_rne(y[t, i] / sqrt(mean_i y[t, i]^2 + eps))   (unit gain, FP32 math)
  *   y  device fp32 [T, d];  x_out device bf16 [T, d];  1 <= d, T >= 0.

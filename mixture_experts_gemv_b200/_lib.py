@@ -31,7 +31,7 @@ EXPORTED = (
     "moe_destroy", "moe_last_error", "moe_debug_get_routing", "moe_debug_get_hidden",
     "moe_debug_check", "moe_workspace_bytes", "moe_profile_begin", "moe_profile_end",
     "moe_layer_forward_static", "moe_profile_kernel_launches", "moe_layer_forward_static_check",
-    "moe_debug_set_wait_ns", "moe_debug_inject",
+    "moe_debug_set_wait_ns", "moe_debug_inject", "moe_block_forward",
 )
 MOE_INJECT_NONE = 0
 MOE_INJECT_SKIP_ROUTER_ARRIVAL = 1
@@ -62,6 +62,8 @@ def lib():
         L.moe_init.restype = _i
         L.moe_layer_forward.argtypes = [_p, _p, _p, _p, _p, _p, _i, _i, _i, _i, _i, _p, _p]
         L.moe_layer_forward.restype = _i
+        L.moe_block_forward.argtypes = [_p, _p, _p, _p, _p, _p, _p, _p, _i, _i, _i, _i, _i, _i, _p, _p]
+        L.moe_block_forward.restype = _i
         L.moe_rmsnorm_bf16.argtypes = [_p, _p, _i, _i, ctypes.c_float, _p]
         L.moe_rmsnorm_bf16.restype = _i
         L.moe_stack_forward.argtypes = [_p, _i, _p, _p, _p, _p, _p, _i, _i, _i, _i, _i,
@@ -131,6 +133,13 @@ def moe_layer_forward(x, router_w, router_scale, gate_up_q4, down_q4, expert_sca
     _check(lib().moe_layer_forward(_ptr(x), _ptr(router_w), _ptr(router_scale), _ptr(gate_up_q4),
                                    _ptr(down_q4), _ptr(expert_scale), T, d, f, E, k, _ptr(out),
                                    _stream(stream)))
+
+
+def moe_block_forward(x, router_w, router_scale, gate_up_q4, down_q4, expert_scale, gate_up_dense_q4,
+                      down_dense_q4, T: int, d: int, f: int, f_dense: int, E: int, k: int, out, stream=None) -> None:
+    _check(lib().moe_block_forward(_ptr(x), _ptr(router_w), _ptr(router_scale), _ptr(gate_up_q4),
+                                   _ptr(down_q4), _ptr(expert_scale), _ptr(gate_up_dense_q4),
+                                   _ptr(down_dense_q4), T, d, f, f_dense, E, k, _ptr(out), _stream(stream)))
 
 
 def moe_rmsnorm_bf16(y, x_out, T: int, d: int, eps: float, stream=None) -> None:

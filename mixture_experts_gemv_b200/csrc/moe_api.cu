@@ -27,7 +27,9 @@ struct Ctx {
   int last_T = 0, last_k = 0, last_E = 0, last_f = 0;
   bool last_gemm = false;
   size_t counters_bytes = 0;
-  bool reset_pending = false;   // a device wait expired: zero the barrier words before the next launch
+  bool reset_pending = false;
+  float *dense_router = nullptr;   // [max_d] zeros: the router of the dense MLP's one-expert pass
+  float *one = nullptr;            // 1.0f: its router scale and expert scale   // a device wait expired: zero the barrier words before the next launch
 };
 
 Ctx g;
@@ -109,6 +111,7 @@ Layout make_layout(int maxT, int max_d, int max_f, int max_E, int max_k) {
       (S / kTileM + max_E + 1) * 8,      // 20 tile pairs
       (size_t)max_E * 4,                 // 21 toff
       64,                                // 22 grid-barrier counter
+      (size_t)max_d * 4 + 16,            // 23 dense MLP pass: zero router row, then 1.0f
   };
   Layout L{};
   size_t o = 0;
@@ -176,8 +179,8 @@ bool gemm_path_for(int T_call) {
 // One pass of T <= max_tokens tokens; `gemm` chooses the path.
 int forward_impl(const void *x, const float *router_w, const float *router_scale, const uint8_t *gate_up_q4,
                  const uint8_t *down_q4, const float *expert_scale, int T, int d, int f, int E, int k, float *out,
-                 cudaStream_t stream, bool gemm) {
-  MoeLaunch L{stream, false};
+                 cudaStream_t stream, bool gemm, bool accumulate = false) {
+  MoeLaunch L{stream, false, accumulate};
   int rc = reset_counters_if_needed(stream);
   if (rc) return rc;
   // MOE_PATH_GEMV and AUTO below the threshold take the fused decode kernel when the shape
@@ -327,6 +330,11 @@ int moe_init(int device, int max_tokens, int max_d, int max_f, int max_E, int ma
   if (e != cudaSuccess) return cuda_fail(e, "cudaMalloc(workspace)");
   e = cudaMemset(ws, 0, Lt.total);
   if (e != cudaSuccess) { cudaFree(ws); return cuda_fail(e, "cudaMemset(workspace)"); }
+  {
+    const float one = 1.0f;
+    e = cudaMemcpy(static_cast<char *>(ws) + Lt.off[23] + (size_t)max_d * 4, &one, sizeof one, cudaMemcpyHostToDevice);
+    if (e != cudaSuccess) { cudaFree(ws); return cuda_fail(e, "workspace constants"); }
+  }
   uint32_t *eh = nullptr;
   e = cudaHostAlloc(reinterpret_cast<void **>(&eh), 64, cudaHostAllocMapped);
   if (e != cudaSuccess) { cudaFree(ws); return cuda_fail(e, "cudaHostAlloc(error word)"); }
@@ -374,6 +382,8 @@ int moe_init(int device, int max_tokens, int max_d, int max_f, int max_E, int ma
   g.ws = ws;
   g.ws_bytes = Lt.total;
   g.counters_bytes = (size_t)(2 + max_d / 8 + 1024) * 4;
+  g.dense_router = reinterpret_cast<float *>(b + Lt.off[23]);   // zeroed with the workspace
+  g.one = g.dense_router + max_d;
   g.err_host = eh;
   g.W = W;
   g.xbuf[0] = reinterpret_cast<__nv_bfloat16 *>(b + Lt.off[17]);
@@ -404,6 +414,43 @@ int moe_layer_forward(const void *x, const float *router_w, const float *router_
     const int Tc = T - c0 < g.max_tokens ? T - c0 : g.max_tokens;
     rc = forward_impl(static_cast<const char *>(x) + (size_t)c0 * d * 2, router_w, router_scale, gate_up_q4, down_q4,
                       expert_scale, Tc, d, f, E, k, out + (size_t)c0 * d, static_cast<cudaStream_t>(stream), gemm);
+    if (rc) return rc;
+  }
+  return MOE_OK;
+}
+
+int moe_block_forward(const void *x, const float *router_w, const float *router_scale, const uint8_t *gate_up_q4,
+                      const uint8_t *down_q4, const float *expert_scale, const uint8_t *gate_up_dense_q4,
+                      const uint8_t *down_dense_q4, int T, int d, int f, int f_dense, int E, int k, float *out,
+                      void *stream) {
+  int rc = check_shapes(T, d, f, E, k);
+  if (rc) return rc;
+  if (f_dense <= 0 || f_dense % 32)
+    return fail(MOE_ERR_BAD_ARG, "f_dense = %d must be a positive multiple of 32", f_dense);
+  if (!x || !router_w || !router_scale || !gate_up_q4 || !down_q4 || !expert_scale || !gate_up_dense_q4 ||
+      !down_dense_q4 || !out)
+    return fail(MOE_ERR_BAD_ARG, "null pointer argument");
+  if (!aligned16(gate_up_q4) || !aligned16(down_q4) || !aligned16(router_w) || !aligned16(x) ||
+      !aligned16(gate_up_dense_q4) || !aligned16(down_dense_q4))
+    return fail(MOE_ERR_BAD_ALIGN, "x, router_w and the Q4_0 matrices must be 16-byte aligned");
+  rc = check_limits(T, d, f, E, k);
+  if (rc) return rc;
+  if (f_dense > g.max_f) return fail(MOE_ERR_BAD_ARG, "f_dense = %d exceeds max_f = %d", f_dense, g.max_f);
+  rc = check_device_error();
+  if (rc) return rc;
+  if (T == 0) return MOE_OK;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const bool gemm = gemm_path_for(T);
+  for (int c0 = 0; c0 < T; c0 += g.max_tokens) {
+    const int Tc = T - c0 < g.max_tokens ? T - c0 : g.max_tokens;
+    const void *xc = static_cast<const char *>(x) + (size_t)c0 * d * 2;
+    float *oc = out + (size_t)c0 * d;
+    rc = forward_impl(xc, router_w, router_scale, gate_up_q4, down_q4, expert_scale, Tc, d, f, E, k, oc, s, gemm);
+    if (rc) return rc;
+    // the dense MLP: one expert every token selects with weight 1 (a zero router row, router
+    // and expert scale 1.0), its combine adding into out
+    rc = forward_impl(xc, g.dense_router, g.one, gate_up_dense_q4, down_dense_q4, g.one, Tc, d, f_dense, 1, 1, oc, s,
+                      gemm, true);
     if (rc) return rc;
   }
   return MOE_OK;

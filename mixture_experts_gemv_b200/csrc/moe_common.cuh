@@ -214,7 +214,8 @@ __device__ __forceinline__ void pdl_launch_dependents() {
 
 struct MoeLaunch {
   cudaStream_t stream;
-  bool pdl;   // launch with programmatic stream serialization
+  bool pdl;                 // launch with programmatic stream serialization
+  bool accumulate = false;  // the combine adds into out (out += ...) instead of writing it
 };
 
 // Kernel groups for the optional per-kernel event timing (moe_profile_begin / _end).

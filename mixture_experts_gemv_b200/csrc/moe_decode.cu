@@ -438,7 +438,7 @@ k_moe_decode(const __nv_bfloat16 *__restrict__ x, const float *y_prev, float eps
              const float *__restrict__ router_w, const float *__restrict__ router_scale,
              const uint8_t *__restrict__ gate_up_q4, const uint8_t *__restrict__ down_q4,
              const float *__restrict__ expert_scale, int T, int d, int f, int E, int k, float *out,
-             uint32_t stage_bytes, uint32_t x_bytes, uint32_t red_half, MoeWork W) {
+             uint32_t stage_bytes, uint32_t x_bytes, uint32_t red_half, MoeWork W, int accumulate) {
   extern __shared__ __align__(128) uint8_t smem_raw[];
   __shared__ FusedShared sh;
   const int tid = threadIdx.x, lane = tid & 31, wq = tid >> 5, nw = blockDim.x >> 5;
@@ -853,7 +853,7 @@ k_moe_decode(const __nv_bfloat16 *__restrict__ x, const float *y_prev, float eps
       const int slotid = t * k + j;
       s += sh.w[slotid] * __ldg(expert_scale + sh.ids[slotid]) * __ldcg(W.ybuf + (size_t)slotid * d + r);
     }
-    out[(size_t)t * d + r] = s;
+    out[(size_t)t * d + r] = accumulate ? out[(size_t)t * d + r] + s : s;
   }
 }
 
@@ -913,7 +913,7 @@ int moe_launch_fused_decode(const MoeLaunch &L, const MoeWork &W, const void *x,
       cudaLaunchKernelEx(&cfg, norm_in ? k_moe_decode<true> : k_moe_decode<false>,
                          static_cast<const __nv_bfloat16 *>(x), y_prev, eps, static_cast<__nv_bfloat16 *>(x_out),
                          router_w, router_scale, gate_up_q4, down_q4, expert_scale, T, d, f, E, k, out,
-                         fs.stage_bytes, fs.x_bytes, fs.red_half, W);
+                         fs.stage_bytes, fs.x_bytes, fs.red_half, W, L.accumulate ? 1 : 0);
   if (e != cudaSuccess) return -1;
   moe_prof_count(1);
   moe_prof_mark(L.stream, MOE_K_FUSED, false);

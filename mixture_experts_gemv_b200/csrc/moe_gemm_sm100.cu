@@ -36,7 +36,7 @@
 
 namespace {
 
-constexpr int BM = 128, BN = 128, BK = 64;
+constexpr int BM = 128, BK = 64;
 static_assert(BM == MOE_GEMM_TILE_ROWS, "the tile list is built with this tile height");
 constexpr int kMaxStages = 5;
 constexpr int kEpiWarps = 4;
@@ -46,33 +46,42 @@ constexpr int kProdWarps = 8 * kProdGroups;
 constexpr int kProdThreads = kProdWarps * 32;
 constexpr int kGroupThreads = kProdThreads / kProdGroups;     // one (row, block) of the B tile each
 constexpr int kThreads = (kEpiWarps + 1 + kProdWarps) * 32;
-constexpr uint32_t kTileBytes = BM * BK * 2;                  // 16 KB: one A half; B is BN x BK, same
+constexpr uint32_t kTileBytes = BM * BK * 2;                  // 16 KB: one 128-row A half
 constexpr uint32_t kRawRowBytes = 64;                          // 16-byte-aligned window over a row's 36 bytes
-constexpr uint32_t kRawStageBytes = BN * kRawRowBytes;
-
-// Per GEMM: gate_up items are one 128-row tile (its A rows are gathered by the producers);
-// down items are up to two consecutive tiles of one expert, M = 256 as two 128-row halves
-// that share the dequantised B tile (A comes by TMA), so the decode work per MMA halves.
-template <bool GATEUP>
-struct GemmCfg {
-  static constexpr int kHalves = GATEUP ? 1 : 2;
-  static constexpr int kStages = GATEUP ? 5 : 4;
-  // group steps the copies run ahead of the decode (measured: gate_up, whose producers
-  // gather A, gains from the deeper lookahead; down, whose A comes by TMA, from refilling a
-  // stage that an older MMA released)
-  static constexpr int kAhead = GATEUP ? 2 : 1;
-  static constexpr uint32_t kBOff = kHalves * kTileBytes;        // B tile after the A halves
-  static constexpr uint32_t kStageBytes = kBOff + kTileBytes;
-  static constexpr uint32_t kTmemCols = 2 * kHalves * BN;        // two accumulator buffers
-  static constexpr int kSmemBytes = kStages * (kStageBytes + kRawStageBytes) + 1024;
-  static_assert(kAhead * kProdGroups <= kStages, "the prologue's stages must be free");
-  static_assert(kStages <= kMaxStages && kTmemCols <= 512, "limits");
-};
 
 // UMMA instruction descriptor, kind::f16: D FP32 (bits 4-5 = 1), A and B bf16 (bits 7-9,
 // 10-12 = 1), both K-major (bits 15, 16 = 0), N >> 3 in bits 17-22, M >> 4 in bits 24-28.
-constexpr uint32_t kIdesc = (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(BN >> 3) << 17) |
-                            ((uint32_t)(BM >> 4) << 24);
+constexpr uint32_t umma_idesc(int n) {
+  return (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(n >> 3) << 17) | ((uint32_t)(BM >> 4) << 24);
+}
+
+// Per GEMM:
+//  gate_up: an item is one 128-row tile and N = 256 columns, the 128 gate rows c0 .. c0+127 and
+//    the matching 128 up rows (rows past f are zero); measured: one tcgen05.mma of N = 256 does
+//    twice the work of an N = 128 one in about the same pipeline time. A rows are gathered by
+//    the producers.
+//  down: an item is up to two consecutive tiles of one expert, M = 256 as two 128-row halves
+//    that share the dequantised N = 128 B tile (A comes by TMA), so the decode work per MMA
+//    halves.
+template <bool GATEUP>
+struct GemmCfg {
+  static constexpr int kBN = GATEUP ? 256 : 128;                 // MMA N
+  static constexpr int kHalves = GATEUP ? 1 : 2;
+  static constexpr int kStages = GATEUP ? 3 : 4;
+  // group steps the copies run ahead of the decode
+  static constexpr int kAhead = 1;
+  static constexpr uint32_t kBBytes = (uint32_t)kBN * BK * 2;
+  static constexpr uint32_t kBOff = kHalves * kTileBytes;        // B tile after the A halves
+  static constexpr uint32_t kStageBytes = kBOff + kBBytes;
+  static constexpr uint32_t kRawStageBytes = (uint32_t)kBN * kRawRowBytes;
+  static constexpr uint32_t kTmemCols = 2 * kHalves * kBN;       // two accumulator buffers
+  static constexpr int kSmemBytes = kStages * (kStageBytes + kRawStageBytes) + 1024;
+  static constexpr int kRowsPerThread = kBN / (kGroupThreads / 2);   // B rows a producer thread decodes
+  static constexpr uint32_t kIdesc = umma_idesc(kBN);
+  static_assert(kAhead * kProdGroups <= kStages, "the prologue's stages must be free");
+  static_assert(kStages <= kMaxStages && kTmemCols <= 512, "limits");
+  static_assert(kRowsPerThread * (kGroupThreads / 2) == kBN, "producer threads cover the B rows");
+};
 
 // Shared-memory matrix descriptor: K-major operand, 128-byte swizzle (layout type 2),
 // rows of 128 bytes in 8-row atoms of 1024 bytes (stride byte offset 1024), version 1.
@@ -124,12 +133,13 @@ __device__ __forceinline__ void tmem_relinquish() {
 __device__ __forceinline__ void tmem_dealloc(uint32_t taddr, uint32_t ncols) {
   asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols) : "memory");
 }
-__device__ __forceinline__ void umma_bf16(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t accumulate) {
+__device__ __forceinline__ void umma_bf16(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                                          uint32_t accumulate) {
   asm volatile(
       "{\n\t.reg .pred p;\n\t"
       "setp.ne.b32 p, %4, 0;\n\t"
       "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
-      "l"(adesc), "l"(bdesc), "r"(kIdesc), "r"(accumulate)
+      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
       : "memory");
 }
 __device__ __forceinline__ void umma_commit(uint64_t *bar) {
@@ -218,10 +228,19 @@ __device__ __forceinline__ void store_blk_bf16(const RawBlk &r, uint32_t tile_sa
   st_shared_v4(rowbase + (((uint32_t)(cbase + 3) ^ x) << 4), hi[4], hi[5], hi[6], hi[7]);   // 24-31
 }
 
+// Zeros into the 4 swizzled 16-byte chunks of row `row` (chunks cbase..cbase+3).
+__device__ __forceinline__ void store_blk_zero(uint32_t tile_saddr, int row, int cbase) {
+  const uint32_t rowbase = tile_saddr + (uint32_t)row * 128u;
+  const uint32_t x = (uint32_t)(row & 7);
+#pragma unroll
+  for (int c = 0; c < 4; ++c) st_shared_v4(rowbase + (((uint32_t)(cbase + c) ^ x) << 4), 0u, 0u, 0u, 0u);
+}
+
 // ---------------------------------------------------------------- the grouped GEMM
 
-// GATEUP: A = the tokens' rows of x [T, d] (a_src = x), B = gate rows n0..n0+63 and up
-//         rows f+n0..f+n0+63, K = d; epilogue h = gelu(gate) * up -> hb (bf16, padded order).
+// GATEUP: A = the tokens' rows of x [T, d] (a_src = x), B = gate rows c0..c0+127 and up
+//         rows f+c0..f+c0+127 (zero past f), K = d; epilogue h = gelu(gate) * up -> hb (bf16,
+//         padded order).
 // DOWN:   A = hb [padded rows, f] (tmap_h: 2-D tiles of 128 rows x 64 columns by TMA), B =
 //         down rows n0..n0+127, K = f; epilogue y * w * s -> yslot (bf16, slot order).
 template <bool GATEUP>
@@ -236,13 +255,15 @@ k_moe_gemm(const __grid_constant__ CUtensorMap tmap_h, const __nv_bfloat16 *__re
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int K = GATEUP ? d : f;
   const int ksteps = K / BK;
-  const int n_ntiles = GATEUP ? f / (BN / 2) : d / BN;
+  using C = GemmCfg<GATEUP>;
+  constexpr int kBN = C::kBN, kRows = C::kRowsPerThread;
+  const int n_ntiles = GATEUP ? (f + kBN / 2 - 1) / (kBN / 2) : d / kBN;
   const int nb_row = K / MOE_QK;                       // Q4_0 blocks per weight row
   const size_t rb = (size_t)nb_row * MOE_QBYTES;       // bytes per weight row
   const size_t expert_bytes = (size_t)(GATEUP ? 2 * f : d) * rb;
-  using C = GemmCfg<GATEUP>;
   constexpr int kHalves = C::kHalves, kStages = C::kStages, kAhead = C::kAhead;
   constexpr uint32_t kBOff = C::kBOff, kStageBytes = C::kStageBytes, kTmemCols = C::kTmemCols;
+  constexpr uint32_t kRawStageBytes = C::kRawStageBytes;
   const int n_items = (GATEUP ? *W.n_tiles : *W.n_pairs) * n_ntiles;
   // work item -> its first tile, and whether a second tile (rows 128 .. 255 past the first
   // tile's start) belongs to it (down only)
@@ -281,22 +302,24 @@ k_moe_gemm(const __grid_constant__ CUtensorMap tmap_h, const __nv_bfloat16 *__re
   if (warp >= kMmaWarp + 1) {
     // ------------------------------------------------------------ producers
     // Producer group pg takes the K steps g with g % kProdGroups == pg. Thread pt of a group
-    // owns row r = pt / 2 of both tiles: A chunks 4 h .. 4 h + 3 (h = pt & 1) of the row's
-    // 128-byte K-step segment, and Q4_0 block h of the row's two blocks per K step.
+    // owns A row r = pt / 2 (of each half): chunks 4 h .. 4 h + 3 (h = pt & 1) of the row's
+    // 128-byte K-step segment; and B rows r + 128 j (j < kRows): Q4_0 block h of each row's two
+    // blocks per K step.
     const int pq = threadIdx.x - (kMmaWarp + 1) * 32;
     const int pg = pq / kGroupThreads, pt = pq - pg * kGroupThreads;   // pt 0..255
     const int row = pt >> 1, hsel = pt & 1;
-    // the raw Q4_0 bytes of row `row` for a K step (two blocks, 36 bytes) arrive in a 64-byte
+    // the raw Q4_0 bytes of B row n for a K step (two blocks, 36 bytes) arrive in a 64-byte
     // window starting at their address rounded down to 16; hsel copies its half of it
-    const uint32_t raw_row = sbase + (uint32_t)kStages * kStageBytes + (uint32_t)row * kRawRowBytes;
+    const uint32_t raw_base = sbase + (uint32_t)kStages * kStageBytes;
     const int my_items = blockIdx.x < n_items ? (n_items - 1 - (int)blockIdx.x) / (int)gridDim.x + 1 : 0;
     const int total = my_items * ksteps;
     // sources of this thread's rows for the CTA's jj-th work item: the A rows of both halves
-    // (null past the expert's rows; gate_up only), the B row, the tile, and whether the
-    // second half holds any of the expert's rows
+    // (null past the expert's rows; gate_up only), the B rows (null past the expert's f gate
+    // or up rows: decoded as zeros), the tile, and whether the second half holds any of the
+    // expert's rows
     struct RowSrc {
       const __nv_bfloat16 *arow[kHalves];
-      const uint8_t *wrow;
+      const uint8_t *wrow[kRows];
       int tile, h1;
     };
     auto item_src = [&](int jj) -> RowSrc {
@@ -315,12 +338,16 @@ k_moe_gemm(const __grid_constant__ CUtensorMap tmap_h, const __nv_bfloat16 *__re
         const int r = m0 + h * BM + row;
         rs.arow[h] = (GATEUP && r < cnt) ? a_src + (size_t)(W.perm[W.offsets[e] + r] / k) * d : nullptr;
       }
-      if (GATEUP) {
-        const int half = BN / 2;
-        const int grow = (row < half) ? (nt * half + row) : (f + nt * half + row - half);
-        rs.wrow = wq + (size_t)e * expert_bytes + (size_t)grow * rb;
-      } else {
-        rs.wrow = wq + (size_t)e * expert_bytes + (size_t)(nt * BN + row) * rb;
+      const uint8_t *ebase = wq + (size_t)e * expert_bytes;
+#pragma unroll
+      for (int j = 0; j < kRows; ++j) {
+        if (GATEUP) {
+          // B row j * 128 + row: gate row c0 + row (j = 0) or up row f + c0 + row (j = 1)
+          const int c = nt * (kBN / 2) + row;
+          rs.wrow[j] = c < f ? ebase + (size_t)(j * f + c) * rb : nullptr;
+        } else {
+          rs.wrow[j] = ebase + (size_t)(nt * kBN + j * 128 + row) * rb;
+        }
       }
       return rs;
     };
@@ -346,15 +373,20 @@ k_moe_gemm(const __grid_constant__ CUtensorMap tmap_h, const __nv_bfloat16 *__re
         tma_load_2d(a_saddr, &tmap_h, ks * BK, rs.tile * BM, &bars.full[s]);
         if (rs.h1) tma_load_2d(a_saddr + kTileBytes, &tmap_h, ks * BK, rs.tile * BM + BM, &bars.full[s]);
       }
-      const uintptr_t wa = (reinterpret_cast<uintptr_t>(rs.wrow) + (uintptr_t)ks * 2 * MOE_QBYTES) & ~(uintptr_t)15;
-      const uint32_t rdst = raw_row + (uint32_t)s * kRawStageBytes + (uint32_t)hsel * 32u;
 #pragma unroll
-      for (int c = 0; c < 2; ++c) {
-        const uintptr_t src = wa + (uintptr_t)(hsel * 32 + c * 16);
-        const uintptr_t end = reinterpret_cast<uintptr_t>(wq_end);
-        const uint32_t nbytes = src >= end ? 0u : (end - src >= 16 ? 16u : (uint32_t)(end - src));
-        cp_async16(rdst + 16u * c, reinterpret_cast<const void *>(nbytes ? src : reinterpret_cast<uintptr_t>(wq)),
-                   nbytes);
+      for (int j = 0; j < kRows; ++j) {
+        if (!rs.wrow[j]) continue;   // a zero row: nothing to copy
+        const uintptr_t wa = (reinterpret_cast<uintptr_t>(rs.wrow[j]) + (uintptr_t)ks * 2 * MOE_QBYTES) & ~(uintptr_t)15;
+        const uint32_t rdst = raw_base + (uint32_t)s * kRawStageBytes + (uint32_t)(j * 128 + row) * kRawRowBytes +
+                              (uint32_t)hsel * 32u;
+#pragma unroll
+        for (int c = 0; c < 2; ++c) {
+          const uintptr_t src = wa + (uintptr_t)(hsel * 32 + c * 16);
+          const uintptr_t end = reinterpret_cast<uintptr_t>(wq_end);
+          const uint32_t nbytes = src >= end ? 0u : (end - src >= 16 ? 16u : (uint32_t)(end - src));
+          cp_async16(rdst + 16u * c, reinterpret_cast<const void *>(nbytes ? src : reinterpret_cast<uintptr_t>(wq)),
+                     nbytes);
+        }
       }
     };
     bool ok = true;
@@ -383,22 +415,29 @@ k_moe_gemm(const __grid_constant__ CUtensorMap tmap_h, const __nv_bfloat16 *__re
     for (int g = pg; g < total; g += kProdGroups, gi += kProdGroups) {
       // step g: its copies have landed (issued kAhead group steps ago); decode B, hand over
       cp_async_wait<kAhead - 1>();
-      __syncwarp();   // the row's window is copied by two lanes
+      __syncwarp();   // a row's window is copied by two lanes
       const int s = g % kStages;
       const uint32_t b_saddr = sbase + (uint32_t)s * kStageBytes + kBOff;
-      // this thread's block inside the row's window: 20 bytes from its offset rounded down to 4
-      RawBlk cur;
-      {
-        const uintptr_t babs = reinterpret_cast<uintptr_t>(csrc.wrow) + (uintptr_t)(cks * 2 + hsel) * MOE_QBYTES;
-        const uintptr_t wa = (reinterpret_cast<uintptr_t>(csrc.wrow) + (uintptr_t)cks * 2 * MOE_QBYTES) & ~(uintptr_t)15;
-        const uint32_t off = (uint32_t)(babs - wa);   // < 48
-        const uint32_t *rp = reinterpret_cast<const uint32_t *>(smem_raw + (raw_row - smem_u32(smem_raw)) +
-                                                                (size_t)s * kRawStageBytes + (off & ~3u));
 #pragma unroll
-        for (int i = 0; i < 5; ++i) cur.w[i] = rp[i];
-        cur.sh = (off & 3u) * 8u;
+      for (int j = 0; j < kRows; ++j) {
+        const int n = j * 128 + row;   // B row
+        if (csrc.wrow[j]) {
+          // this thread's block inside the row's window: 20 bytes from its offset rounded down to 4
+          RawBlk cur;
+          const uintptr_t babs = reinterpret_cast<uintptr_t>(csrc.wrow[j]) + (uintptr_t)(cks * 2 + hsel) * MOE_QBYTES;
+          const uintptr_t wa = (reinterpret_cast<uintptr_t>(csrc.wrow[j]) + (uintptr_t)cks * 2 * MOE_QBYTES) & ~(uintptr_t)15;
+          const uint32_t off = (uint32_t)(babs - wa);   // < 48
+          const uint32_t *rp = reinterpret_cast<const uint32_t *>(
+              smem_raw + (raw_base - smem_u32(smem_raw)) + (size_t)s * kRawStageBytes + (size_t)n * kRawRowBytes +
+              (off & ~3u));
+#pragma unroll
+          for (int i = 0; i < 5; ++i) cur.w[i] = rp[i];
+          cur.sh = (off & 3u) * 8u;
+          store_blk_bf16(cur, b_saddr, n, hsel * 4);
+        } else {
+          store_blk_zero(b_saddr, n, hsel * 4);
+        }
       }
-      store_blk_bf16(cur, b_saddr, row, hsel * 4);
       fence_proxy_async_smem();
       mbar_arrive(&bars.full[s]);
       adv(cjj, cks, csrc);
@@ -428,7 +467,7 @@ k_moe_gemm(const __grid_constant__ CUtensorMap tmap_h, const __nv_bfloat16 *__re
         int tile;
         bool h1;
         item_tile(item, tile, h1);
-        const uint32_t dtm = tmem + (uint32_t)(b * kHalves * BN);
+        const uint32_t dtm = tmem + (uint32_t)(b * kHalves * kBN);
         for (int ks = 0; ks < ksteps; ++ks, ++it) {
           const int s = it % kStages;
           const uint32_t par = (uint32_t)(it / kStages) & 1u;
@@ -440,8 +479,8 @@ k_moe_gemm(const __grid_constant__ CUtensorMap tmap_h, const __nv_bfloat16 *__re
           for (int kk = 0; kk < BK / 16; ++kk) {
             const uint64_t bdesc = sw128_desc(b_saddr + kk * 32);
             const uint32_t acc = (ks > 0 || kk > 0) ? 1u : 0u;
-            umma_bf16(dtm, sw128_desc(a_saddr + kk * 32), bdesc, acc);
-            if (h1) umma_bf16(dtm + BN, sw128_desc(a_saddr + kTileBytes + kk * 32), bdesc, acc);
+            umma_bf16(dtm, sw128_desc(a_saddr + kk * 32), bdesc, C::kIdesc, acc);
+            if (h1) umma_bf16(dtm + kBN, sw128_desc(a_saddr + kTileBytes + kk * 32), bdesc, C::kIdesc, acc);
           }
           umma_commit(&bars.empty[s]);
         }
@@ -471,14 +510,16 @@ k_moe_gemm(const __grid_constant__ CUtensorMap tmap_h, const __nv_bfloat16 *__re
       for (int h = 0; h < nh; ++h) {
         const int mr = m0 + h * BM + r;        // row of the expert
         const bool valid = mr < cnt;
-        const uint32_t taddr = tmem + ((uint32_t)(warp * 32) << 16) + (uint32_t)((b * kHalves + h) * BN);
+        const uint32_t taddr = tmem + ((uint32_t)(warp * 32) << 16) + (uint32_t)((b * kHalves + h) * kBN);
         if (GATEUP) {
-          __nv_bfloat16 *dst = W.hb + (size_t)((tile + h) * BM + r) * f + (size_t)nt * (BN / 2);
+          const int c0 = nt * (kBN / 2);   // first h column of this item
+          __nv_bfloat16 *dst = W.hb + (size_t)((tile + h) * BM + r) * f + (size_t)c0;
 #pragma unroll
-          for (int c = 0; c < BN / 2; c += 16) {
+          for (int c = 0; c < kBN / 2; c += 16) {
+            if (c0 + c >= f) break;   // warp-uniform: the item's columns past f are zero rows
             uint32_t g[16], u[16];
             tmem_ld16(taddr + (uint32_t)c, g);
-            tmem_ld16(taddr + (uint32_t)(BN / 2 + c), u);
+            tmem_ld16(taddr + (uint32_t)(kBN / 2 + c), u);
             tmem_ld_wait();
             uint32_t o[8];
 #pragma unroll
@@ -500,9 +541,9 @@ k_moe_gemm(const __grid_constant__ CUtensorMap tmap_h, const __nv_bfloat16 *__re
             slot = W.perm[W.offsets[e] + mr];
             scale = W.w[slot] * expert_scale[e];
           }
-          __nv_bfloat16 *dst = reinterpret_cast<__nv_bfloat16 *>(W.yslot) + (size_t)slot * d + (size_t)nt * BN;
+          __nv_bfloat16 *dst = reinterpret_cast<__nv_bfloat16 *>(W.yslot) + (size_t)slot * d + (size_t)nt * kBN;
 #pragma unroll
-          for (int c = 0; c < BN; c += 16) {
+          for (int c = 0; c < kBN; c += 16) {
             uint32_t y[16];
             tmem_ld16(taddr + (uint32_t)c, y);
             tmem_ld_wait();
@@ -533,7 +574,7 @@ k_moe_gemm(const __grid_constant__ CUtensorMap tmap_h, const __nv_bfloat16 *__re
 
 // out[t, c] = sum_{j < k} yslot[t k + j, c] (already weighted), j ascending.
 __global__ void __launch_bounds__(256) k_combine(const __nv_bfloat16 *__restrict__ yslot, int T, int d, int k,
-                                                 float *__restrict__ out) {
+                                                 float *__restrict__ out, int accumulate) {
   const int vpr = d / 8;
   const long long total = (long long)T * vpr;
   for (long long i = blockIdx.x * (long long)blockDim.x + threadIdx.x; i < total;
@@ -558,6 +599,11 @@ __global__ void __launch_bounds__(256) k_combine(const __nv_bfloat16 *__restrict
       }
     }
     float4 *op = reinterpret_cast<float4 *>(out + (size_t)t * d) + 2 * v;
+    if (accumulate) {   // out += the sum (one FP32 addition per element)
+      const float4 o0 = op[0], o1 = op[1];
+      acc[0] = o0.x + acc[0]; acc[1] = o0.y + acc[1]; acc[2] = o0.z + acc[2]; acc[3] = o0.w + acc[3];
+      acc[4] = o1.x + acc[4]; acc[5] = o1.y + acc[5]; acc[6] = o1.z + acc[6]; acc[7] = o1.w + acc[7];
+    }
     op[0] = make_float4(acc[0], acc[1], acc[2], acc[3]);
     op[1] = make_float4(acc[4], acc[5], acc[6], acc[7]);
   }
@@ -598,7 +644,8 @@ static bool make_tmap_h(CUtensorMap *m, const void *base, int cols, long long ro
 int moe_launch_gemm_experts(const MoeLaunch &L, const MoeWork &W, const void *x, const uint8_t *gate_up_q4,
                             const uint8_t *down_q4, const float *expert_scale, int T, int d, int f, int E, int k,
                             float *out, int num_sms, int max_tiles) {
-  if (d % BK || d % BN || f % BK || f % (BN / 2)) return -2;
+  // K of both GEMMs in whole 64-wide steps; down's output in whole 128-column tiles
+  if (d % BK || d % GemmCfg<false>::kBN || f % BK) return -2;
   static unsigned long long smem_ok[2] = {0ull, 0ull};   // per device, per kernel
   if (!moe_allow_dyn_smem(reinterpret_cast<const void *>(k_moe_gemm<true>), &smem_ok[0]) ||
       !moe_allow_dyn_smem(reinterpret_cast<const void *>(k_moe_gemm<false>), &smem_ok[1]))
@@ -620,7 +667,8 @@ int moe_launch_gemm_experts(const MoeLaunch &L, const MoeWork &W, const void *x,
   moe_prof_count(1);
   moe_prof_mark(L.stream, MOE_K_GEMM_DOWN, false);
   moe_prof_mark(L.stream, MOE_K_COMBINE, true);
-  k_combine<<<4 * num_sms, 256, 0, L.stream>>>(reinterpret_cast<const __nv_bfloat16 *>(W.yslot), T, d, k, out);
+  k_combine<<<4 * num_sms, 256, 0, L.stream>>>(reinterpret_cast<const __nv_bfloat16 *>(W.yslot), T, d, k, out,
+                                               L.accumulate ? 1 : 0);
   if (launch_err()) return -1;
   moe_prof_count(1);
   moe_prof_mark(L.stream, MOE_K_COMBINE, false);

@@ -139,7 +139,7 @@ k_gateup_gemv(const uint8_t *__restrict__ gate_up_q4, int d, int f, int k, int n
 
 __global__ void __launch_bounds__(kDnThreads, 1)
 k_down_gemv_combine(const uint8_t *__restrict__ down_q4, const float *__restrict__ expert_scale, int T,
-                    int d, int f, int k, int nstages, float *__restrict__ out, MoeWork W) {
+                    int d, int f, int k, int nstages, float *__restrict__ out, MoeWork W, int accumulate) {
   extern __shared__ __align__(128) uint8_t smem_raw[];
   __shared__ RingCtl ring;
   __shared__ int done_units[kDnRows / kUnit];
@@ -261,7 +261,7 @@ k_down_gemv_combine(const uint8_t *__restrict__ down_q4, const float *__restrict
           const int slotid = t * k + j;
           s += W.w[slotid] * expert_scale[W.ids[slotid]] * __ldcg(W.ybuf + (size_t)slotid * d + r);
         }
-        out[(size_t)t * d + r] = s;
+        out[(size_t)t * d + r] = accumulate ? out[(size_t)t * d + r] + s : s;
       }
       __syncthreads();
       if (threadIdx.x < n_done) W.counters[1 + done_units[threadIdx.x]] = 0;
@@ -321,7 +321,8 @@ int moe_launch_gemv_experts(const MoeLaunch &L, const MoeWork &W, const uint8_t 
   moe_prof_count(1);
   moe_prof_mark(L.stream, MOE_K_GATEUP, false);
   moe_prof_mark(L.stream, MOE_K_DOWN, true);
-  k_down_gemv_combine<<<num_sms, kDnThreads, dn_smem, L.stream>>>(down_q4, expert_scale, T, d, f, k, dn_st, out, W);
+  k_down_gemv_combine<<<num_sms, kDnThreads, dn_smem, L.stream>>>(down_q4, expert_scale, T, d, f, k, dn_st, out, W,
+                                                                      L.accumulate ? 1 : 0);
   if (launch_err()) return -1;
   moe_prof_count(1);
   moe_prof_mark(L.stream, MOE_K_DOWN, false);

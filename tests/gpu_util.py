@@ -62,7 +62,7 @@ def run_layer(x_bits, dl: DevLayer, k, path=moe.MOE_PATH_AUTO, want_routing=True
                           T, d, lw.f, lw.E, k, out)
     res = {"out": out[:T]}
     if want_routing and T > 0:
-        S = T * k
+        S = (T - ((T - 1) // CHUNK) * CHUNK) * k   # the routing readers hold the last chunk's
         ids = torch.empty(S, dtype=torch.int32, device="cuda:0")
         w = torch.empty(S, dtype=torch.float32, device="cuda:0")
         counts = torch.empty(lw.E, dtype=torch.int32, device="cuda:0")
