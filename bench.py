@@ -7,7 +7,8 @@ workload is the eight-request decode batch (decode_T8: T = 8 tokens, d = 2816, f
 E = 128, k = 8); the same line carries, under "workloads", the single-token layer
 (layer_T1), the 4,096-token prefill (prefill_T4096, the tensor-core half of the metric), the
 30-layer single-token stack (stack30_T1) and the long prompts of 10,000 and 40,000 tokens
-(prefill_T10000, prefill_T40000: chunks of 4,096 tokens), each with its own timing, roofline,
+(prefill_T10000, prefill_T40000: chunks of 4,096 tokens) and the decode batch through the
+routed experts plus the block's dense MLP (block_T8), each with its own timing, roofline,
 end-to-end figure and clocks. Consecutive decode steps rotate over several independent
 layers so that the active experts' weights of one step are not L2-resident in the next
 (inputs larger than L2); a prefill step reads all 428 MB of a layer's experts, a stack step
@@ -39,10 +40,10 @@ import numpy as np  # noqa: E402
 import moe_inputs as mi  # noqa: E402
 
 METRIC = "MoE-layer tokens/s; decode HBM GB/s & prefill TFLOP/s as % of B200 roofline"
-EXTRA_DEFAULT = "layer_T1,prefill_T4096,stack30_T1,prefill_T10000,prefill_T40000"
+EXTRA_DEFAULT = "layer_T1,prefill_T4096,stack30_T1,prefill_T10000,prefill_T40000,block_T8"
 # tokens of each workload, and the workspace's token capacity (longer calls run in chunks)
 WORKLOAD_T = {"layer_T1": 1, "decode_T8": 8, "stack30_T1": 1, "prefill_T4096": 4096, "skewed_T512": 512,
-              "prefill_T10000": 10000, "prefill_T40000": 40000}
+              "prefill_T10000": 10000, "prefill_T40000": 40000, "block_T8": 8}
 CHUNK_TOKENS = 4096
 
 
@@ -381,6 +382,7 @@ class Bench:
     def measure(self, name):
         torch, moe, args, dev = self.torch, self.moe, self.args, self.dev
         stack = name == "stack30_T1"
+        block = name == "block_T8"   # the routed experts plus the block's dense MLP (f_dense = 704)
         T = WORKLOAD_T[name]
         if stack:
             idx = list(range(30))
@@ -402,6 +404,12 @@ class Bench:
         else:
             layers = [(("plain", i), self.layer(i)) for i in idx]
         dl = [self.dev_layer(key, lw) for key, lw in layers]
+        fd = mi.D_FF_DENSE
+        dense = []
+        if block:
+            for key, _ in layers:
+                gud, dnd = mi.make_dense(0, key[1], d, fd)
+                dense.append((self.up(gud), self.up(dnd)))
         x = self.up(base.x)
         out = torch.empty((T, d), dtype=torch.float32, device=dev)
 
@@ -413,6 +421,10 @@ class Bench:
                 moe.moe_stack_forward(xin, [q["router_w"] for q in dl], [q["router_scale"] for q in dl],
                                       [q["gate_up"] for q in dl], [q["down"] for q in dl],
                                       [q["expert_scale"] for q in dl], T, d, f, E, k, 1e-6, o, None, stream)
+            elif block:
+                q, dq = dl[i % len(dl)], dense[i % len(dl)]
+                moe.moe_block_forward(xin, q["router_w"], q["router_scale"], q["gate_up"], q["down"],
+                                      q["expert_scale"], dq[0], dq[1], T, d, f, fd, E, k, o, stream)
             else:
                 q = dl[i % len(dl)]
                 moe.moe_layer_forward(xin, q["router_w"], q["router_scale"], q["gate_up"], q["down"],
@@ -429,7 +441,14 @@ class Bench:
             cnt = torch.empty(E, dtype=torch.int32, device=dev)
             moe.moe_debug_get_routing(counts=cnt, stream=stream)
             torch.cuda.synchronize()
-            work.append(flops_bytes(lw, T, k, cnt.cpu().numpy()))
+            wk = flops_bytes(lw, T, k, cnt.cpu().numpy())
+            if block:
+                # the dense MLP's pass: its Q4_0 weights, a one-row zero router, x and out again
+                dense_w = 2 * fd * (d // 32) * 18 + d * (fd // 32) * 18
+                wk["dense_bytes"] = dense_w + d * 4 + T * d * 6
+                wk["total_bytes"] += wk["dense_bytes"]
+                wk["flops"] += 2 * T * (2 * fd * d + d * fd)
+            work.append(wk)
         moe.moe_debug_check(stream)
         avg = {kk: float(np.mean([w[kk] for w in work])) for kk in work[0]}
 
@@ -570,12 +589,17 @@ class Bench:
         extra = {}
         if T <= 16 and "fused_decode" in prof:
             # the whole layer is one kernel: its algorithmic bytes are the active experts' Q4_0
-            # weights, the router weights, x, out and the scales
+            # weights, the router weights, x, out and the scales (with the dense MLP, a step is
+            # two launches: the bytes per launch are the step's over two)
             kms, nl = prof["fused_decode"]
             per_launch_bytes = (avg["gateup_weight_bytes"] + avg["down_weight_bytes"] + avg["router_bytes"] +
                                 avg["act_bytes"] + 4 * (E + 1))
-            only = set(prof) == {"fused_decode"} and nl == args.steps * n_layers
-            roof = decode_launch_roofline(per_launch_bytes, kms, nl, ms_step / n_layers if only else None, pk,
+            launches = n_layers
+            if block:
+                per_launch_bytes = (per_launch_bytes + avg["dense_bytes"] + 8) / 2
+                launches = 2
+            only = set(prof) == {"fused_decode"} and nl == args.steps * launches
+            roof = decode_launch_roofline(per_launch_bytes, kms, nl, ms_step / launches if only else None, pk,
                                           "k_moe_decode", name)
             dtype = "int16xq4->int32, f32"
         elif T <= 16:

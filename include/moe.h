@@ -110,6 +110,32 @@ int moe_block_forward(const void *x, const float *router_w, const float *router_
                       int f, int f_dense, int E, int k, float *out, void *stream);
 
 /*
+ * Pieces of the layer for an expert-parallel deployment (experts spread over several GPUs:
+ * the routing and the final sum stay with the tokens, the expert rows travel to the GPU that
+ * holds their experts and back).
+ *
+ * moe_route: the layer's selection alone, ids int32 [T, k] and w fp32 [T, k] (as
+ *   moe_debug_get_routing describes them) for T tokens, written to the caller's device
+ *   buffers; the same selection moe_layer_forward makes (the decode routing up to 16 tokens,
+ *   the tiled router product above).
+ * moe_experts_forward: experts on rows the caller has routed, one expert per row:
+ *   out_rows[r] = row_weight[r] * expert_scale[e_r] * Wd_e (gelu_tanh(Wg_e x_r) * (Wu_e x_r)),
+ *   e_r = row_expert[r] in [0, E) (an id outside it gives that row 0 and makes the next
+ *   checking call return MOE_ERR_BAD_ARG); x_rows bf16 [R, d], out_rows fp32 [R, d]; the
+ *   GEMV path up to the AUTO threshold, the grouped GEMM above; R > max_tokens in chunks.
+ * moe_gather_rows: dst[i, :] = src[index[i], :] for i < n, rows of row_bytes (a multiple of
+ *   16), 16-byte aligned bases; index int32 device [n].
+ * moe_combine_slots: out[t, :] = sum_{j < k} y_slots[t k + j, :] in j order; fp32, d % 4 == 0.
+ */
+int moe_route(const void *x, const float *router_w, const float *router_scale, int T, int d, int E, int k,
+              int32_t *ids, float *w, void *stream);
+int moe_experts_forward(const void *x_rows, const int32_t *row_expert, const float *row_weight,
+                        const uint8_t *gate_up_q4, const uint8_t *down_q4, const float *expert_scale,
+                        int R, int d, int f, int E, float *out_rows, void *stream);
+int moe_gather_rows(const void *src, const int32_t *index, int n, size_t row_bytes, void *dst, void *stream);
+int moe_combine_slots(const float *y_slots, int T, int d, int k, float *out, void *stream);
+
+/*
  * moe_rmsnorm_bf16: the fixed normalisation between stacked layers,
  *   x[t, i] = bf16_rne(y[t, i] / sqrt(mean_i y[t, i]^2 + eps))   (unit gain, FP32 math)
  *   y  device fp32 [T, d];  x_out device bf16 [T, d];  1 <= d, T >= 0.

@@ -11,5 +11,6 @@ from ._lib import (  # noqa: F401
     moe_debug_get_hidden, moe_debug_check, moe_workspace_bytes, moe_profile_begin,
     moe_profile_end, PROF_GROUPS, EXPORTED, moe_layer_forward_static, moe_profile_kernel_launches,
     moe_layer_forward_static_check, moe_debug_set_wait_ns, moe_debug_inject, MOE_INJECT_NONE,
-    MOE_INJECT_SKIP_ROUTER_ARRIVAL, moe_block_forward,
+    MOE_INJECT_SKIP_ROUTER_ARRIVAL, moe_block_forward, moe_route, moe_experts_forward, moe_gather_rows,
+    moe_combine_slots,
 )

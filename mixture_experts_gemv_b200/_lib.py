@@ -31,7 +31,8 @@ EXPORTED = (
     "moe_destroy", "moe_last_error", "moe_debug_get_routing", "moe_debug_get_hidden",
     "moe_debug_check", "moe_workspace_bytes", "moe_profile_begin", "moe_profile_end",
     "moe_layer_forward_static", "moe_profile_kernel_launches", "moe_layer_forward_static_check",
-    "moe_debug_set_wait_ns", "moe_debug_inject", "moe_block_forward",
+    "moe_debug_set_wait_ns", "moe_debug_inject", "moe_block_forward", "moe_route", "moe_experts_forward",
+    "moe_gather_rows", "moe_combine_slots",
 )
 MOE_INJECT_NONE = 0
 MOE_INJECT_SKIP_ROUTER_ARRIVAL = 1
@@ -62,6 +63,14 @@ def lib():
         L.moe_init.restype = _i
         L.moe_layer_forward.argtypes = [_p, _p, _p, _p, _p, _p, _i, _i, _i, _i, _i, _p, _p]
         L.moe_layer_forward.restype = _i
+        L.moe_route.argtypes = [_p, _p, _p, _i, _i, _i, _i, _p, _p, _p]
+        L.moe_route.restype = _i
+        L.moe_experts_forward.argtypes = [_p, _p, _p, _p, _p, _p, _i, _i, _i, _i, _p, _p]
+        L.moe_experts_forward.restype = _i
+        L.moe_gather_rows.argtypes = [_p, _p, _i, ctypes.c_size_t, _p, _p]
+        L.moe_gather_rows.restype = _i
+        L.moe_combine_slots.argtypes = [_p, _i, _i, _i, _p, _p]
+        L.moe_combine_slots.restype = _i
         L.moe_block_forward.argtypes = [_p, _p, _p, _p, _p, _p, _p, _p, _i, _i, _i, _i, _i, _i, _p, _p]
         L.moe_block_forward.restype = _i
         L.moe_rmsnorm_bf16.argtypes = [_p, _p, _i, _i, ctypes.c_float, _p]
@@ -140,6 +149,26 @@ def moe_block_forward(x, router_w, router_scale, gate_up_q4, down_q4, expert_sca
     _check(lib().moe_block_forward(_ptr(x), _ptr(router_w), _ptr(router_scale), _ptr(gate_up_q4),
                                    _ptr(down_q4), _ptr(expert_scale), _ptr(gate_up_dense_q4),
                                    _ptr(down_dense_q4), T, d, f, f_dense, E, k, _ptr(out), _stream(stream)))
+
+
+def moe_route(x, router_w, router_scale, T: int, d: int, E: int, k: int, ids, w, stream=None) -> None:
+    _check(lib().moe_route(_ptr(x), _ptr(router_w), _ptr(router_scale), T, d, E, k, _ptr(ids), _ptr(w),
+                           _stream(stream)))
+
+
+def moe_experts_forward(x_rows, row_expert, row_weight, gate_up_q4, down_q4, expert_scale, R: int, d: int,
+                        f: int, E: int, out_rows, stream=None) -> None:
+    _check(lib().moe_experts_forward(_ptr(x_rows), _ptr(row_expert), _ptr(row_weight), _ptr(gate_up_q4),
+                                     _ptr(down_q4), _ptr(expert_scale), R, d, f, E, _ptr(out_rows),
+                                     _stream(stream)))
+
+
+def moe_gather_rows(src, index, n: int, row_bytes: int, dst, stream=None) -> None:
+    _check(lib().moe_gather_rows(_ptr(src), _ptr(index), n, row_bytes, _ptr(dst), _stream(stream)))
+
+
+def moe_combine_slots(y_slots, T: int, d: int, k: int, out, stream=None) -> None:
+    _check(lib().moe_combine_slots(_ptr(y_slots), T, d, k, _ptr(out), _stream(stream)))
 
 
 def moe_rmsnorm_bf16(y, x_out, T: int, d: int, eps: float, stream=None) -> None:

@@ -137,6 +137,9 @@ int check_device_error() {
     *reinterpret_cast<volatile uint32_t *>(g.err_host) = 0;
     // the kernels that gave up left their arrival counters mid-count
     g.reset_pending = true;
+    if ((v & 0xffffu) == MOE_DEV_ERR_BAD_EXPERT)
+      return fail(MOE_ERR_BAD_ARG, "an expert id given to moe_experts_forward was outside [0, E) (its row was "
+                                   "computed with weight 0)");
     return fail(MOE_ERR_DEVICE_TIMEOUT, "device wait timed out (code %u at site %u)", v & 0xffffu, v >> 16);
   }
   return MOE_OK;
@@ -453,6 +456,99 @@ int moe_block_forward(const void *x, const float *router_w, const float *router_
                       gemm, true);
     if (rc) return rc;
   }
+  return MOE_OK;
+}
+
+int moe_route(const void *x, const float *router_w, const float *router_scale, int T, int d, int E, int k,
+              int32_t *ids, float *w, void *stream) {
+  int rc = check_shapes(T, d, 32, E, k);
+  if (rc) return rc;
+  if (!x || !router_w || !router_scale || !ids || !w) return fail(MOE_ERR_BAD_ARG, "null pointer argument");
+  if (!aligned16(router_w) || !aligned16(x)) return fail(MOE_ERR_BAD_ALIGN, "x and router_w must be 16-byte aligned");
+  rc = check_limits(T, d, 32, E, k);
+  if (rc) return rc;
+  rc = check_device_error();
+  if (rc) return rc;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  rc = reset_counters_if_needed(s);
+  if (rc) return rc;
+  MoeLaunch L{s, false};
+  for (int c0 = 0; c0 < T; c0 += g.max_tokens) {
+    const int Tc = T - c0 < g.max_tokens ? T - c0 : g.max_tokens;
+    const void *xc = static_cast<const char *>(x) + (size_t)c0 * d * 2;
+    // the selection the layer itself makes: the decode routing (logits cut as the fused
+    // kernel cuts them) up to 16 tokens, the tiled router product above
+    rc = Tc <= 16 ? moe_launch_route_decode(L, g.W, xc, router_w, router_scale, Tc, d, E, k, g.num_sms)
+                  : moe_launch_route_prefill(L, g.W, xc, router_w, router_scale, Tc, d, E, k, g.num_sms, false, 0);
+    if (rc == -2) return fail(MOE_ERR_BAD_ARG, "shape not supported by the routing kernels");
+    if (rc) return cuda_fail(cudaGetLastError(), "routing launch");
+    cudaError_t e = cudaMemcpyAsync(ids + (size_t)c0 * k, g.W.ids, (size_t)Tc * k * 4, cudaMemcpyDeviceToDevice, s);
+    if (e == cudaSuccess)
+      e = cudaMemcpyAsync(w + (size_t)c0 * k, g.W.w, (size_t)Tc * k * 4, cudaMemcpyDeviceToDevice, s);
+    if (e != cudaSuccess) return cuda_fail(e, "routing copy");
+  }
+  return MOE_OK;
+}
+
+int moe_experts_forward(const void *x_rows, const int32_t *row_expert, const float *row_weight,
+                        const uint8_t *gate_up_q4, const uint8_t *down_q4, const float *expert_scale, int R, int d,
+                        int f, int E, float *out_rows, void *stream) {
+  int rc = check_shapes(R, d, f, E, 1);
+  if (rc) return rc;
+  if (!x_rows || !row_expert || !row_weight || !gate_up_q4 || !down_q4 || !expert_scale || !out_rows)
+    return fail(MOE_ERR_BAD_ARG, "null pointer argument");
+  if (!aligned16(gate_up_q4) || !aligned16(down_q4) || !aligned16(x_rows))
+    return fail(MOE_ERR_BAD_ALIGN, "x_rows, gate_up_q4 and down_q4 must be 16-byte aligned");
+  rc = check_limits(R, d, f, E, 1);
+  if (rc) return rc;
+  rc = check_device_error();
+  if (rc) return rc;
+  if (R == 0) return MOE_OK;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  rc = reset_counters_if_needed(s);
+  if (rc) return rc;
+  MoeLaunch L{s, false};
+  const bool gemm = gemm_path_for(R);
+  for (int c0 = 0; c0 < R; c0 += g.max_tokens) {
+    const int Rc = R - c0 < g.max_tokens ? R - c0 : g.max_tokens;
+    const void *xc = static_cast<const char *>(x_rows) + (size_t)c0 * d * 2;
+    float *oc = out_rows + (size_t)c0 * d;
+    rc = moe_launch_route_given(L, g.W, xc, row_expert + c0, row_weight + c0, Rc, d, E, g.num_sms, !gemm,
+                                gemm ? kTileM : 0);
+    if (rc == -2) return fail(MOE_ERR_BAD_ARG, "E = %d not supported by the permutation kernels", E);
+    if (rc) return cuda_fail(cudaGetLastError(), "routing launch");
+    if (gemm) {
+      const int max_tiles = (int)((size_t)g.max_tokens * g.max_k / kTileM + g.max_E + 1);
+      rc = moe_launch_gemm_experts(L, g.W, xc, gate_up_q4, down_q4, expert_scale, Rc, d, f, E, 1, oc, g.num_sms,
+                                   max_tiles);
+      if (rc == -2) return fail(MOE_ERR_BAD_ARG, "shape not supported by the grouped-GEMM path");
+      if (rc) return cuda_fail(cudaGetLastError(), "grouped-GEMM launch");
+    } else {
+      rc = moe_launch_gemv_experts(L, g.W, gate_up_q4, down_q4, expert_scale, Rc, d, f, E, 1, oc, g.num_sms);
+      if (rc == -2) return fail(MOE_ERR_BAD_ARG, "shape not supported by the GEMV path (d, f too large)");
+      if (rc) return cuda_fail(cudaGetLastError(), "GEMV launch");
+    }
+  }
+  return MOE_OK;
+}
+
+int moe_gather_rows(const void *src, const int32_t *index, int n, size_t row_bytes, void *dst, void *stream) {
+  if (n < 0 || row_bytes == 0 || row_bytes % 16) return fail(MOE_ERR_BAD_ARG, "n >= 0 and row_bytes % 16 == 0 needed");
+  if (!src || !index || !dst) return fail(MOE_ERR_BAD_ARG, "null pointer argument");
+  if (!aligned16(src) || !aligned16(dst)) return fail(MOE_ERR_BAD_ALIGN, "src and dst must be 16-byte aligned");
+  if (n == 0) return MOE_OK;
+  if (moe_launch_gather_rows(static_cast<cudaStream_t>(stream), src, index, n, row_bytes, dst))
+    return cuda_fail(cudaGetLastError(), "gather launch");
+  return MOE_OK;
+}
+
+int moe_combine_slots(const float *y_slots, int T, int d, int k, float *out, void *stream) {
+  if (T < 0 || d <= 0 || d % 4 || k < 1) return fail(MOE_ERR_BAD_ARG, "T >= 0, d % 4 == 0, k >= 1 needed");
+  if (!y_slots || !out) return fail(MOE_ERR_BAD_ARG, "null pointer argument");
+  if (!aligned16(y_slots) || !aligned16(out)) return fail(MOE_ERR_BAD_ALIGN, "y_slots and out must be 16-byte aligned");
+  if (T == 0) return MOE_OK;
+  if (moe_launch_combine_slots(static_cast<cudaStream_t>(stream), y_slots, T, d, k, out))
+    return cuda_fail(cudaGetLastError(), "combine launch");
   return MOE_OK;
 }
 

@@ -17,6 +17,7 @@
 
 // Device error word: code in the low 16 bits, location in the high 16.
 #define MOE_DEV_ERR_TIMEOUT 1u
+#define MOE_DEV_ERR_BAD_EXPERT 2u   // an expert id given to the experts-only path is out of range
 
 // Routing and scratch produced and consumed inside one forward. All device pointers.
 // Decode layout shared by the fused decode kernel and the separate decode kernels, so that
@@ -264,5 +265,16 @@ int moe_launch_fused_decode(const MoeLaunch &L, const MoeWork &W, const void *x,
                             const uint8_t *gate_up_q4, const uint8_t *down_q4, const float *expert_scale, int T,
                             int d, int f, int E, int k, float *out, int num_sms);
 int moe_launch_rmsnorm(cudaStream_t s, const float *y, void *x_out, int T, int d, float eps);
+// Routing given by the caller (one expert and weight per row, k = 1): ids and weights into the
+// workspace, the stable permutation (with the tile lists when tile_m > 0) and, with
+// want_xprep, the GEMV path's activations. Out-of-range ids record MOE_DEV_ERR_BAD_EXPERT and
+// become expert 0 with weight 0.
+int moe_launch_route_given(const MoeLaunch &L, const MoeWork &W, const void *x, const int32_t *row_expert,
+                           const float *row_weight, int R, int d, int E, int num_sms, bool want_xprep, int tile_m);
+// dst row i = src row index[i] (rows of row_bytes, a multiple of 16; 16-byte aligned bases).
+int moe_launch_gather_rows(cudaStream_t s, const void *src, const int32_t *index, int n, size_t row_bytes,
+                           void *dst);
+// out[t, :] = sum_j y[t * k + j, :] in j order (FP32 rows of d).
+int moe_launch_combine_slots(cudaStream_t s, const float *y, int T, int d, int k, float *out);
 int moe_launch_hidden_to_slots(cudaStream_t s, const MoeWork &W, float *h, int T, int f, int k,
                                bool gemm_path);

@@ -443,6 +443,51 @@ k_prep_x(const __nv_bfloat16 *__restrict__ x, int T, int d, MoeWork W) {
   prep_x_range(x, W.xq, W.xblk, T, d, blockIdx.x * blockDim.x + threadIdx.x, gridDim.x * blockDim.x);
 }
 
+// ---------------------------------------------------------------- routing given by the caller
+
+__global__ void __launch_bounds__(256)
+k_route_given(const int32_t *__restrict__ row_expert, const float *__restrict__ row_weight, int R, int E, MoeWork W) {
+  for (int r = blockIdx.x * blockDim.x + threadIdx.x; r < R; r += gridDim.x * blockDim.x) {
+    int e = row_expert[r];
+    float w = row_weight[r];
+    if (e < 0 || e >= E) {
+      report_error(W.err, MOE_DEV_ERR_BAD_EXPERT, 30);
+      e = 0;
+      w = 0.f;
+    }
+    W.ids[r] = e;
+    W.w[r] = w;
+  }
+}
+
+// dst row i = src row index[i], in 16-byte words.
+__global__ void __launch_bounds__(256)
+k_gather_rows(const uint4 *__restrict__ src, const int32_t *__restrict__ index, int n, int words, uint4 *__restrict__ dst) {
+  const long long total = (long long)n * words;
+  for (long long i = blockIdx.x * (long long)blockDim.x + threadIdx.x; i < total; i += (long long)gridDim.x * blockDim.x) {
+    const int row = (int)(i / words), w = (int)(i - (long long)row * words);
+    dst[i] = __ldg(src + (size_t)index[row] * words + w);
+  }
+}
+
+// out[t, c] = sum_{j < k} y[t k + j, c], j ascending (FP32).
+__global__ void __launch_bounds__(256)
+k_combine_slots(const float4 *__restrict__ y, int T, int d4, int k, float4 *__restrict__ out) {
+  const long long total = (long long)T * d4;
+  for (long long i = blockIdx.x * (long long)blockDim.x + threadIdx.x; i < total; i += (long long)gridDim.x * blockDim.x) {
+    const int t = (int)(i / d4), c = (int)(i - (long long)t * d4);
+    float4 s = make_float4(0.f, 0.f, 0.f, 0.f);
+    for (int j = 0; j < k; ++j) {
+      const float4 v = __ldg(y + ((size_t)t * k + j) * d4 + c);
+      s.x += v.x;
+      s.y += v.y;
+      s.z += v.z;
+      s.w += v.w;
+    }
+    out[i] = s;
+  }
+}
+
 }  // namespace
 
 // ---------------------------------------------------------------- launchers
@@ -505,5 +550,58 @@ int moe_launch_route_prefill(const MoeLaunch &L, const MoeWork &W, const void *x
     moe_prof_count(1);
   }
   moe_prof_mark(L.stream, MOE_K_ROUTE, false);
+  return 0;
+}
+
+int moe_launch_route_given(const MoeLaunch &L, const MoeWork &W, const void *x, const int32_t *row_expert,
+                           const float *row_weight, int R, int d, int E, int num_sms, bool want_xprep, int tile_m) {
+  if (E > kRouteThreads) return -2;
+  const int nc = (R + kPermSlots - 1) / kPermSlots;
+  int32_t *ccnt = reinterpret_cast<int32_t *>(W.ybuf);   // per-CTA expert counts (free until the experts run)
+  moe_prof_mark(L.stream, MOE_K_ROUTE, true);
+  int grid = (R + 255) / 256;
+  if (grid > 4 * num_sms) grid = 4 * num_sms;
+  k_route_given<<<grid, 256, 0, L.stream>>>(row_expert, row_weight, R, E, W);
+  if (launch_err()) return -1;
+  k_perm_count<<<nc, kRouteThreads, 0, L.stream>>>(W.ids, R, E, ccnt);
+  if (launch_err()) return -1;
+  k_perm_scan<<<1, kRouteThreads, 0, L.stream>>>(nc, E, tile_m, tile_m > 0, ccnt, W);
+  if (launch_err()) return -1;
+  k_perm_place<<<nc, kRouteThreads, 0, L.stream>>>(R, E, ccnt, W);
+  if (launch_err()) return -1;
+  moe_prof_count(4);
+  if (want_xprep) {
+    const int items = R * (d / MOE_QK);
+    int g2 = (items + 255) / 256;
+    if (g2 > 4 * num_sms) g2 = 4 * num_sms;
+    k_prep_x<<<g2, 256, 0, L.stream>>>(static_cast<const __nv_bfloat16 *>(x), R, d, W);
+    if (launch_err()) return -1;
+    moe_prof_count(1);
+  }
+  moe_prof_mark(L.stream, MOE_K_ROUTE, false);
+  return 0;
+}
+
+int moe_launch_gather_rows(cudaStream_t s, const void *src, const int32_t *index, int n, size_t row_bytes,
+                           void *dst) {
+  const int words = (int)(row_bytes / 16);
+  long long total = (long long)n * words;
+  int grid = (int)((total + 255) / 256);
+  if (grid > 2048) grid = 2048;
+  if (grid < 1) grid = 1;
+  k_gather_rows<<<grid, 256, 0, s>>>(static_cast<const uint4 *>(src), index, n, words, static_cast<uint4 *>(dst));
+  if (launch_err()) return -1;
+  moe_prof_count(1);
+  return 0;
+}
+
+int moe_launch_combine_slots(cudaStream_t s, const float *y, int T, int d, int k, float *out) {
+  const long long total = (long long)T * (d / 4);
+  int grid = (int)((total + 255) / 256);
+  if (grid > 2048) grid = 2048;
+  if (grid < 1) grid = 1;
+  k_combine_slots<<<grid, 256, 0, s>>>(reinterpret_cast<const float4 *>(y), T, d / 4, k, reinterpret_cast<float4 *>(out));
+  if (launch_err()) return -1;
+  moe_prof_count(1);
   return 0;
 }

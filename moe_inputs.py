@@ -172,6 +172,7 @@ WORKLOADS = (
     "skewed_T512",      # 512 tokens, x from seed 4, Zipf-biased router
     "prefill_T10000",   # 10,000-token prefill, x from seed 5 (a long prompt)
     "prefill_T40000",   # 40,000-token prefill, x from seed 6 (the longest prompt)
+    "block_T8",         # decode_T8 through the routed experts plus the block's dense MLP
 )
 
 
@@ -197,7 +198,7 @@ def make_workload(name: str, n_layers: int | None = None, layer_fn=None) -> Work
     get = layer_fn if layer_fn is not None else (lambda i: make_layer(0, i))
     if name == "layer_T1":
         return Workload(name, make_tokens(0, 1), [get(0)])
-    if name == "decode_T8":
+    if name in ("decode_T8", "block_T8"):
         return Workload(name, make_tokens_per_seed(range(1, 9)), [get(0)])
     if name == "stack30_T1":
         L = 30 if n_layers is None else n_layers

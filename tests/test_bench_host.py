@@ -96,7 +96,7 @@ def test_extra_workloads_default_and_none():
     a = bench.parse([])
     assert a.workload == "decode_T8"
     assert bench.extra_workloads(a) == ["layer_T1", "prefill_T4096", "stack30_T1", "prefill_T10000",
-                                        "prefill_T40000"]
+                                        "prefill_T40000", "block_T8"]
     assert bench.extra_workloads(bench.parse(["--extra", "none"])) == []
     assert bench.extra_workloads(bench.parse(["--workload", "prefill_T4096", "--extra", "layer_T1,prefill_T4096"])) \
         == ["layer_T1"]
