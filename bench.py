@@ -589,15 +589,17 @@ class Bench:
         extra = {}
         if T <= 16 and "fused_decode" in prof:
             # the whole layer is one kernel: its algorithmic bytes are the active experts' Q4_0
-            # weights, the router weights, x, out and the scales (with the dense MLP, a step is
-            # two launches: the bytes per launch are the step's over two)
+            # weights, the router weights, x, out and the scales (the dense MLP's weights too,
+            # when it rides in the same launch; when it takes a pass of its own, a step is two
+            # launches and the bytes per launch are the step's over two)
             kms, nl = prof["fused_decode"]
             per_launch_bytes = (avg["gateup_weight_bytes"] + avg["down_weight_bytes"] + avg["router_bytes"] +
                                 avg["act_bytes"] + 4 * (E + 1))
             launches = n_layers
             if block:
-                per_launch_bytes = (per_launch_bytes + avg["dense_bytes"] + 8) / 2
-                launches = 2
+                launches = max(1, round(nl / args.steps))
+                dense_b = (avg["dense_bytes"] - T * d * 6 - d * 4) if launches == 1 else avg["dense_bytes"] + 8
+                per_launch_bytes = (per_launch_bytes + dense_b) / launches
             only = set(prof) == {"fused_decode"} and nl == args.steps * launches
             roof = decode_launch_roofline(per_launch_bytes, kms, nl, ms_step / launches if only else None, pk,
                                           "k_moe_decode", name)

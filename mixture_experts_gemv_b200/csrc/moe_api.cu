@@ -82,7 +82,9 @@ struct Layout {
 size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
 
 Layout make_layout(int maxT, int max_d, int max_f, int max_E, int max_k) {
-  const size_t S = (size_t)maxT * max_k;
+  // per-slot buffers hold k + 1 slots per token: the block's dense MLP takes one more slot per
+  // token when it rides in the fused decode launch
+  const size_t S = (size_t)maxT * (max_k + 1);
   const size_t prow = (S / kTileM + max_E + 1) * kTileM;   // padded tile rows
   const size_t ybuf_bytes = S * max_d * 4 > moe_route_scratch_bytes(maxT, max_E, max_k)
                                 ? S * max_d * 4
@@ -448,6 +450,22 @@ int moe_block_forward(const void *x, const float *router_w, const float *router_
     const int Tc = T - c0 < g.max_tokens ? T - c0 : g.max_tokens;
     const void *xc = static_cast<const char *>(x) + (size_t)c0 * d * 2;
     float *oc = out + (size_t)c0 * d;
+    // Decode with a dense MLP of the experts' width: one fused launch takes it as expert E,
+    // one more slot per token with weight 1, its output added in the combine
+    if (!gemm && g.path != MOE_PATH_GEMV_SPLIT && f_dense == f && moe_fused_decode_supported(Tc, d, f, E, k, true)) {
+      rc = reset_counters_if_needed(s);
+      if (rc) return rc;
+      MoeLaunch L{s, false};
+      rc = moe_launch_fused_decode(L, g.W, xc, nullptr, 0.f, nullptr, router_w, router_scale, gate_up_q4, down_q4,
+                                   expert_scale, Tc, d, f, E, k, oc, g.num_sms, gate_up_dense_q4, down_dense_q4);
+      if (rc) return cuda_fail(cudaGetLastError(), "fused decode launch");
+      g.last_T = Tc;
+      g.last_k = k;
+      g.last_E = E;
+      g.last_f = f;
+      g.last_gemm = false;
+      continue;
+    }
     rc = forward_impl(xc, router_w, router_scale, gate_up_q4, down_q4, expert_scale, Tc, d, f, E, k, oc, s, gemm);
     if (rc) return rc;
     // the dense MLP: one expert every token selects with weight 1 (a zero router row, router
@@ -533,7 +551,7 @@ int moe_experts_forward(const void *x_rows, const int32_t *row_expert, const flo
 }
 
 int moe_gather_rows(const void *src, const int32_t *index, int n, size_t row_bytes, void *dst, void *stream) {
-  if (n < 0 || row_bytes == 0 || row_bytes % 16) return fail(MOE_ERR_BAD_ARG, "n >= 0 and row_bytes % 16 == 0 needed");
+  if (n < 0 || row_bytes == 0 || row_bytes % 16) return fail(MOE_ERR_BAD_ARG, "n >= 0 and row_bytes %% 16 == 0 needed");
   if (!src || !index || !dst) return fail(MOE_ERR_BAD_ARG, "null pointer argument");
   if (!aligned16(src) || !aligned16(dst)) return fail(MOE_ERR_BAD_ALIGN, "src and dst must be 16-byte aligned");
   if (n == 0) return MOE_OK;
@@ -543,7 +561,7 @@ int moe_gather_rows(const void *src, const int32_t *index, int n, size_t row_byt
 }
 
 int moe_combine_slots(const float *y_slots, int T, int d, int k, float *out, void *stream) {
-  if (T < 0 || d <= 0 || d % 4 || k < 1) return fail(MOE_ERR_BAD_ARG, "T >= 0, d % 4 == 0, k >= 1 needed");
+  if (T < 0 || d <= 0 || d % 4 || k < 1) return fail(MOE_ERR_BAD_ARG, "T >= 0, d %% 4 == 0, k >= 1 needed");
   if (!y_slots || !out) return fail(MOE_ERR_BAD_ARG, "null pointer argument");
   if (!aligned16(y_slots) || !aligned16(out)) return fail(MOE_ERR_BAD_ALIGN, "y_slots and out must be 16-byte aligned");
   if (T == 0) return MOE_OK;
@@ -603,7 +621,8 @@ int moe_stack_forward(const void *x_in, int L, const float *const *router_w, con
         // y_prev = g.ylayer is read before the kernel's first grid barrier, yo written after its last
         MoeLaunch Lf{s, false};
         rc = moe_launch_fused_decode(Lf, g.W, nullptr, g.ylayer, eps, trace_i, router_w[i], router_scale[i],
-                                     gate_up_q4[i], down_q4[i], expert_scale[i], Tc, d, f, E, k, yo, g.num_sms);
+                                     gate_up_q4[i], down_q4[i], expert_scale[i], Tc, d, f, E, k, yo, g.num_sms,
+                                     nullptr, nullptr, i + 1 < L ? router_w[i + 1] : nullptr);
         if (rc) return cuda_fail(cudaGetLastError(), "fused decode launch");
         continue;
       }

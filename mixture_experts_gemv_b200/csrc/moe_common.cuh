@@ -200,6 +200,12 @@ __device__ __forceinline__ void bulk_g2s_hint(void *dst, const void *src, uint32
       : "memory");
 }
 
+// Bulk prefetch of [src, src + bytes) into L2 (no shared memory involved, no completion to
+// wait for). src 16-byte aligned, bytes a multiple of 16.
+__device__ __forceinline__ void bulk_prefetch_l2(const void *src, uint32_t bytes) {
+  asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(src), "r"(bytes) : "memory");
+}
+
 __device__ __forceinline__ void fence_proxy_async_smem() {
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
@@ -256,14 +262,16 @@ int moe_launch_gemv_experts(const MoeLaunch &L, const MoeWork &W, const uint8_t 
 int moe_launch_gemm_experts(const MoeLaunch &L, const MoeWork &W, const void *x, const uint8_t *gate_up_q4,
                             const uint8_t *down_q4, const float *expert_scale, int T, int d, int f,
                             int E, int k, float *out, int num_sms, int max_tiles);
-bool moe_fused_decode_supported(int T, int d, int f, int E, int k);
+// dense: the block's dense MLP (same width f) rides along as expert E, one more slot per token.
+bool moe_fused_decode_supported(int T, int d, int f, int E, int k, bool dense = false);
 // The fused decode kernel: x (bf16 [T, d]) as the layer input, or, with y_prev not null, the
 // previous layer's FP32 output normalised in the kernel (x_out, when not null, receives that
 // bf16 x; y_prev may equal out).
 int moe_launch_fused_decode(const MoeLaunch &L, const MoeWork &W, const void *x, const float *y_prev, float eps,
                             void *x_out, const float *router_w, const float *router_scale,
                             const uint8_t *gate_up_q4, const uint8_t *down_q4, const float *expert_scale, int T,
-                            int d, int f, int E, int k, float *out, int num_sms);
+                            int d, int f, int E, int k, float *out, int num_sms, const uint8_t *dense_gu = nullptr,
+                            const uint8_t *dense_dn = nullptr, const float *next_router_w = nullptr);
 int moe_launch_rmsnorm(cudaStream_t s, const float *y, void *x_out, int T, int d, float eps);
 // Routing given by the caller (one expert and weight per row, k = 1): ids and weights into the
 // workspace, the stable permutation (with the tile lists when tile_m > 0) and, with

@@ -79,6 +79,7 @@ struct FusedShared {
   int seq[4];                 // this CTA's unit ranges: gate_up [0, 1), down [2, 3)
   int ok;
   int abort;                  // set by any expired wait: the warps keep their barrier sequence, skip work
+  unsigned long long gbase;   // the grid-barrier counter when this launch started
 };
 
 __device__ __forceinline__ unsigned long long ld_acquire_u64(const unsigned long long *p) {
@@ -90,14 +91,16 @@ __device__ __forceinline__ unsigned long long ld_acquire_u64(const unsigned long
 __device__ __forceinline__ void named_sync(int id, int n) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(n) : "memory");
 }
-// Grid-wide barrier on a monotonically increasing 64-bit counter, split in two: arrival k of
-// a phase returns the end of its window of gridDim.x arrivals; the wait spins (bounded) until
-// the counter reaches it. One thread per CTA, after the CTA's writes are ordered before it.
-__device__ __forceinline__ unsigned long long grid_arrive(unsigned long long *ctr) {
-  __threadfence();
-  const unsigned long long n = gridDim.x;
-  const unsigned long long old = atomicAdd(ctr, 1ull);
-  return (old / n + 1ull) * n;
+// Grid-wide barriers on a monotonically increasing 64-bit counter: every launch adds exactly
+// gridDim.x per barrier, so the counter is a multiple of gridDim.x when a launch starts, and
+// barrier i of the launch (1, 2, 3) completes at that start value + i * gridDim.x. Each CTA
+// reads the start value at its start (CTAs that already arrived at barrier 1 cannot have
+// moved it past the next multiple); an arrival is a release add that returns nothing, and
+// the wait spins (bounded) with acquire loads until the counter reaches the target. One
+// thread per CTA arrives, after the CTA's writes are ordered before it. (After an expired
+// wait the host zeroes the counter before the next launch.)
+__device__ __forceinline__ void grid_arrive(unsigned long long *ctr) {
+  asm volatile("red.release.gpu.global.add.u64 [%0], 1;" ::"l"(ctr) : "memory");
 }
 __device__ bool grid_wait(const unsigned long long *ctr, unsigned long long target, volatile uint32_t *err,
                           uint32_t where, uint64_t limit_ns) {
@@ -120,10 +123,13 @@ __device__ __forceinline__ void named_arrive(int id, int n) {
 }
 // Grid barrier of the compute and epilogue warps (the named barrier kBarTeam inside the CTA).
 // An expired wait sets *abort; the caller keeps going.
-__device__ void grid_barrier_team(unsigned long long *ctr, volatile uint32_t *err, uint32_t where, int nteam,
-                                  volatile int *abort, uint64_t limit_ns) {
+__device__ void grid_barrier_team(unsigned long long *ctr, unsigned long long target, volatile uint32_t *err,
+                                  uint32_t where, int nteam, volatile int *abort, uint64_t limit_ns) {
   named_sync(kBarTeam, nteam);
-  if (threadIdx.x == 0 && !grid_wait(ctr, grid_arrive(ctr), err, where, limit_ns)) *abort = 1;
+  if (threadIdx.x == 0) {
+    grid_arrive(ctr);
+    if (!grid_wait(ctr, target, err, where, limit_ns)) *abort = 1;
+  }
   named_sync(kBarTeam, nteam);
 }
 // Wait for an mbarrier phase, at most limit_ns; gives up at once when *abort is set and sets
@@ -438,10 +444,16 @@ k_moe_decode(const __nv_bfloat16 *__restrict__ x, const float *y_prev, float eps
              const float *__restrict__ router_w, const float *__restrict__ router_scale,
              const uint8_t *__restrict__ gate_up_q4, const uint8_t *__restrict__ down_q4,
              const float *__restrict__ expert_scale, int T, int d, int f, int E, int k, float *out,
-             uint32_t stage_bytes, uint32_t x_bytes, uint32_t red_half, MoeWork W, int accumulate) {
+             uint32_t stage_bytes, uint32_t x_bytes, uint32_t red_half, MoeWork W, int accumulate,
+             const uint8_t *__restrict__ dense_gu, const uint8_t *__restrict__ dense_dn,
+             const float *__restrict__ next_router_w) {
   extern __shared__ __align__(128) uint8_t smem_raw[];
   __shared__ FusedShared sh;
   const int tid = threadIdx.x, lane = tid & 31, wq = tid >> 5, nw = blockDim.x >> 5;
+  // the grid-barrier counter as this launch starts, loaded now by the thread that arrives at
+  // the first barrier (its latency hides behind the router)
+  const int bar_tid = (int)blockDim.x - 32;
+  const unsigned long long gstart = tid == bar_tid ? ld_acquire_u64(W.gbar) : 0ull;
   const int nwc = nw - 2, nct = nwc * 32;   // compute warps 0 .. nwc-1; warp nwc produces, nwc+1 epilogues
   const int nteam = nct + 32;
   const int nb = d / MOE_QK, nbf = f / MOE_QK;
@@ -562,9 +574,12 @@ k_moe_decode(const __nv_bfloat16 *__restrict__ x, const float *y_prev, float eps
   // test-only fault: CTA 0 leaves without arriving, so every other CTA's bounded wait below
   // runs out and reports a timeout
   const bool skip_arrival = W.inject == MOE_INJECT_SKIP_ROUTER_ARRIVAL && blockIdx.x == 0;
-  const int bar_tid = (int)blockDim.x - 32, nconv = (int)blockDim.x - 32;
-  if (tid == bar_tid)
-    sh.ok = (!skip_arrival && grid_wait(W.gbar, grid_arrive(W.gbar), W.err, 20, W.wait_ns)) ? 1 : 0;
+  const int nconv = (int)blockDim.x - 32;
+  if (tid == bar_tid) {
+    sh.gbase = gstart - gstart % gridDim.x;
+    if (!skip_arrival) grid_arrive(W.gbar);
+    sh.ok = (!skip_arrival && grid_wait(W.gbar, sh.gbase + gridDim.x, W.err, 20, W.wait_ns)) ? 1 : 0;
+  }
   if (tid < nconv && wait_phase(&sh.xbar, 0u, &sh.abort, W.err, 26, W.wait_ns)) {
     for (int blk = tid; blk < T * nb; blk += nconv) {
       const int t = blk / nb, b = blk - t * nb;
@@ -594,17 +609,29 @@ k_moe_decode(const __nv_bfloat16 *__restrict__ x, const float *y_prev, float eps
   // ---------------------------------------------------------------- phase 1: selection
   for (int t = wq; t < T; t += nw)
     warp_topk_softmax<kFMaxE>(W.logits + (size_t)t * E, E, k, rs, sh.ids + t * k, sh.w + t * k);
+  // with the block's dense MLP: expert index E, one more slot per token (s = T k + t), weight 1
+  const int Sr = T * k;
+  const bool dense = dense_gu != nullptr;
+  if (dense)
+    for (int t = tid; t < T; t += blockDim.x) {
+      sh.ids[Sr + t] = E;
+      sh.w[Sr + t] = 1.f;
+    }
   __syncthreads();
-  const int S = T * k;
+  const int S = Sr + (dense ? T : 0);
   const int upe_g = f / kUnit, upe_d = d / kUnit;
   // the stable counting sort of the slots by expert, over the whole CTA (its scratch: the
   // reduction buffers, unused until the GEMVs)
-  cta_permutation_small<kFMaxSlots / 32, kFMaxE / 32>(sh.ids, S, E, sh.counts, sh.offsets, sh.perm, sh.inv, sh.act, &sh.n_act,
+  cta_permutation_small<kFMaxSlots / 32, kFMaxE / 32>(sh.ids, S, E + (dense ? 1 : 0), sh.counts, sh.offsets, sh.perm,
+                                                     sh.inv, sh.act, &sh.n_act,
                                          reinterpret_cast<int32_t *>(red));
   const int n_act = sh.n_act;
   // each sorted position's token, and the unit-cost prefix over the active experts in closed
   // form: pc[a] = sum over earlier active experts of (kUnitDecode + kUnitToken * T_e)
-  for (int p = tid; p < S; p += blockDim.x) sh.ptok[p] = sh.perm[p] / k;
+  for (int p = tid; p < S; p += blockDim.x) {
+    const int s = sh.perm[p];
+    sh.ptok[p] = s < Sr ? s / k : s - Sr;
+  }
   for (int a = tid; a < n_act; a += blockDim.x) sh.pc[a] = kUnitDecode * a + kUnitToken * sh.offsets[sh.act[a]];
   const uint32_t ptot = (uint32_t)(kUnitDecode * n_act + kUnitToken * S);
   if (tid < 4) {
@@ -620,7 +647,7 @@ k_moe_decode(const __nv_bfloat16 *__restrict__ x, const float *y_prev, float eps
 #pragma unroll
     for (int j = 0; j < 4; ++j) {
       const uint32_t upe = j < 2 ? upe_g : upe_d;
-      const uint32_t xb = (uint32_t)((unsigned long long)upe * ptot * (blockIdx.x + (j & 1)) / gridDim.x);
+      const uint32_t xb = upe * ptot * (blockIdx.x + (j & 1)) / gridDim.x;   // < 2^32 for d <= 4096
       const uint32_t lo = upe * (uint32_t)sh.pc[a], hi = upe * (uint32_t)sh.pc[a + 1];
       if (xb >= lo && xb < hi) {
         const uint32_t inexp = (xb - lo + (uint32_t)c - 1u) / (uint32_t)c;
@@ -632,6 +659,10 @@ k_moe_decode(const __nv_bfloat16 *__restrict__ x, const float *y_prev, float eps
 
   // ---------------------------------------------------------------- producer warp
   if (wq == nwc) {
+    // in a layer stack, this CTA's row of the next layer's router moves into L2 while this
+    // layer runs (rows are 16-byte aligned: d is a multiple of 32)
+    if (next_router_w != nullptr && lane == 1)
+      for (int e = blockIdx.x; e < E; e += gridDim.x) bulk_prefetch_l2(next_router_w + (size_t)e * d, (uint32_t)d * 4u);
     if (lane == 0) {
       const uint64_t pol = l2_evict_first_policy();   // expert weights are read once per call
       FWalk wk;
@@ -646,7 +677,7 @@ k_moe_decode(const __nv_bfloat16 *__restrict__ x, const float *y_prev, float eps
         const int e = sh.act[c.a];
         uint8_t *dst = smem + (size_t)slot * stage_bytes;
         if (!c.down) {
-          const uint8_t *base = gate_up_q4 + (size_t)e * 2 * f * rb_g;
+          const uint8_t *base = e < E ? gate_up_q4 + (size_t)e * 2 * f * rb_g : dense_gu;
           const uint32_t bytes = (uint32_t)(c.n * kUnit) * rb_g;
           mbar_arrive_expect_tx(&sh.full[slot], 2u * bytes);
           bulk_g2s_hint(dst, base + (size_t)c.r0 * rb_g, bytes, &sh.full[slot], pol);
@@ -654,7 +685,8 @@ k_moe_decode(const __nv_bfloat16 *__restrict__ x, const float *y_prev, float eps
         } else {
           const uint32_t bytes = (uint32_t)(c.n * kUnit) * rb_d;
           mbar_arrive_expect_tx(&sh.full[slot], bytes);
-          bulk_g2s_hint(dst, down_q4 + (size_t)e * d * rb_d + (size_t)c.r0 * rb_d, bytes, &sh.full[slot], pol);
+          const uint8_t *dbase = e < E ? down_q4 + (size_t)e * d * rb_d : dense_dn;
+          bulk_g2s_hint(dst, dbase + (size_t)c.r0 * rb_d, bytes, &sh.full[slot], pol);
         }
         wk.advance(c.n, sh.seq, upe_g, upe_d);
       }
@@ -699,7 +731,7 @@ k_moe_decode(const __nv_bfloat16 *__restrict__ x, const float *y_prev, float eps
       const FChunk c = wk.cur(upe_g, upe_d);
       if (c.down && !down_phase) {
         // all h written (the epilogue warp included) before any CTA reads it
-        grid_barrier_team(W.gbar, W.err, 21, nteam, &sh.abort, W.wait_ns);
+        grid_barrier_team(W.gbar, sh.gbase + 2ull * gridDim.x, W.err, 21, nteam, &sh.abort, W.wait_ns);
         down_phase = true;
       }
       const int slot = it % kFStages;
@@ -789,7 +821,7 @@ k_moe_decode(const __nv_bfloat16 *__restrict__ x, const float *y_prev, float eps
       if (lane == 0) mbar_arrive(&sh.empty[slot]);   // this warp's last read of the stage
       wk.advance(c.n, sh.seq, upe_g, upe_d);
     }
-    if (!down_phase) grid_barrier_team(W.gbar, W.err, 21, nteam, &sh.abort, W.wait_ns);   // no down rows here
+    if (!down_phase) grid_barrier_team(W.gbar, sh.gbase + 2ull * gridDim.x, W.err, 21, nteam, &sh.abort, W.wait_ns);   // no down rows here
     for (int q = pass < 2 ? 0 : pass - 2; q < pass; ++q) named_sync(kBarEmpty0 + (q & 1), nteam);
   } else {
     // the epilogue warp: the same sequence of chunks and passes
@@ -798,7 +830,7 @@ k_moe_decode(const __nv_bfloat16 *__restrict__ x, const float *y_prev, float eps
     while (!wk.done()) {
       const FChunk c = wk.cur(upe_g, upe_d);
       if (c.down && !down_phase) {
-        grid_barrier_team(W.gbar, W.err, 21, nteam, &sh.abort, W.wait_ns);
+        grid_barrier_team(W.gbar, sh.gbase + 2ull * gridDim.x, W.err, 21, nteam, &sh.abort, W.wait_ns);
         down_phase = true;
       }
       const int e = sh.act[c.a];
@@ -838,10 +870,10 @@ k_moe_decode(const __nv_bfloat16 *__restrict__ x, const float *y_prev, float eps
       }
       wk.advance(c.n, sh.seq, upe_g, upe_d);
     }
-    if (!down_phase) grid_barrier_team(W.gbar, W.err, 21, nteam, &sh.abort, W.wait_ns);
+    if (!down_phase) grid_barrier_team(W.gbar, sh.gbase + 2ull * gridDim.x, W.err, 21, nteam, &sh.abort, W.wait_ns);
   }
   // ---------------------------------------------------------------- phase 4: combine
-  grid_barrier_team(W.gbar, W.err, 23, nteam, &sh.abort, W.wait_ns);
+  grid_barrier_team(W.gbar, sh.gbase + 3ull * gridDim.x, W.err, 23, nteam, &sh.abort, W.wait_ns);
   if (sh.abort) return;
   const int ti = wq < nwc ? tid : nct + lane;
   const int r0 = (int)((long long)d * blockIdx.x / gridDim.x), r1 = (int)((long long)d * (blockIdx.x + 1) / gridDim.x);
@@ -853,6 +885,7 @@ k_moe_decode(const __nv_bfloat16 *__restrict__ x, const float *y_prev, float eps
       const int slotid = t * k + j;
       s += sh.w[slotid] * __ldg(expert_scale + sh.ids[slotid]) * __ldcg(W.ybuf + (size_t)slotid * d + r);
     }
+    if (dense) s += __ldcg(W.ybuf + (size_t)(Sr + t) * d + r);   // the dense MLP's output, weight 1
     out[(size_t)t * d + r] = accumulate ? out[(size_t)t * d + r] + s : s;
   }
 }
@@ -880,17 +913,19 @@ static FusedSmem fused_smem(int T, int d, int f) {
   return r;
 }
 
-bool moe_fused_decode_supported(int T, int d, int f, int E, int k) {
+bool moe_fused_decode_supported(int T, int d, int f, int E, int k, bool dense) {
   const int G = (d / MOE_QK + kGran - 1) / kGran;
-  return T >= 1 && T <= kFMaxT && T * k <= kFMaxSlots && E <= kFMaxE && G <= kMaxGran &&
+  const int S = T * k + (dense ? T : 0), Eall = E + (dense ? 1 : 0);
+  return T >= 1 && T <= kFMaxT && S <= kFMaxSlots && Eall <= kFMaxE && G <= kMaxGran &&
          fused_smem(T, d, f).total + sizeof(FusedShared) <= 227 * 1024;
 }
 
 int moe_launch_fused_decode(const MoeLaunch &L, const MoeWork &W, const void *x, const float *y_prev, float eps,
                             void *x_out, const float *router_w, const float *router_scale,
                             const uint8_t *gate_up_q4, const uint8_t *down_q4, const float *expert_scale, int T,
-                            int d, int f, int E, int k, float *out, int num_sms) {
-  if (!moe_fused_decode_supported(T, d, f, E, k)) return -2;
+                            int d, int f, int E, int k, float *out, int num_sms, const uint8_t *dense_gu,
+                            const uint8_t *dense_dn, const float *next_router_w) {
+  if (!moe_fused_decode_supported(T, d, f, E, k, dense_gu != nullptr)) return -2;
   const FusedSmem fs = fused_smem(T, d, f);
   static unsigned long long smem_ok[2] = {0ull, 0ull};   // per device, per kernel
   const bool norm_in = y_prev != nullptr;
@@ -913,7 +948,8 @@ int moe_launch_fused_decode(const MoeLaunch &L, const MoeWork &W, const void *x,
       cudaLaunchKernelEx(&cfg, norm_in ? k_moe_decode<true> : k_moe_decode<false>,
                          static_cast<const __nv_bfloat16 *>(x), y_prev, eps, static_cast<__nv_bfloat16 *>(x_out),
                          router_w, router_scale, gate_up_q4, down_q4, expert_scale, T, d, f, E, k, out,
-                         fs.stage_bytes, fs.x_bytes, fs.red_half, W, L.accumulate ? 1 : 0);
+                         fs.stage_bytes, fs.x_bytes, fs.red_half, W, L.accumulate ? 1 : 0, dense_gu, dense_dn,
+                         next_router_w);
   if (e != cudaSuccess) return -1;
   moe_prof_count(1);
   moe_prof_mark(L.stream, MOE_K_FUSED, false);

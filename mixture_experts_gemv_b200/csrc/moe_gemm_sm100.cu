@@ -320,6 +320,8 @@ k_moe_gemm(const __grid_constant__ CUtensorMap tmap_h, const __nv_bfloat16 *__re
     struct RowSrc {
       const __nv_bfloat16 *arow[kHalves];
       const uint8_t *wrow[kRows];
+      uint32_t wlo[kRows];    // low 4 bits of the row's address
+      bool wtail[kRows];      // the row's last windows can reach past the end of the matrix
       int tile, h1;
     };
     auto item_src = [&](int jj) -> RowSrc {
@@ -348,6 +350,10 @@ k_moe_gemm(const __grid_constant__ CUtensorMap tmap_h, const __nv_bfloat16 *__re
         } else {
           rs.wrow[j] = ebase + (size_t)(nt * kBN + j * 128 + row) * rb;
         }
+        // a K step's 64-byte window starts at most 15 bytes before its blocks and ends at most
+        // 28 bytes past the row's last block
+        rs.wlo[j] = (uint32_t)(reinterpret_cast<uintptr_t>(rs.wrow[j]) & 15u);
+        rs.wtail[j] = rs.wrow[j] != nullptr && rs.wrow[j] + rb + 28 > wq_end;
       }
       return rs;
     };
@@ -376,16 +382,20 @@ k_moe_gemm(const __grid_constant__ CUtensorMap tmap_h, const __nv_bfloat16 *__re
 #pragma unroll
       for (int j = 0; j < kRows; ++j) {
         if (!rs.wrow[j]) continue;   // a zero row: nothing to copy
-        const uintptr_t wa = (reinterpret_cast<uintptr_t>(rs.wrow[j]) + (uintptr_t)ks * 2 * MOE_QBYTES) & ~(uintptr_t)15;
+        const uint32_t kb = (uint32_t)ks * 2u * MOE_QBYTES;
+        const uint8_t *wa = rs.wrow[j] + kb - ((rs.wlo[j] + kb) & 15u);   // 16-byte aligned window start
         const uint32_t rdst = raw_base + (uint32_t)s * kRawStageBytes + (uint32_t)(j * 128 + row) * kRawRowBytes +
                               (uint32_t)hsel * 32u;
 #pragma unroll
         for (int c = 0; c < 2; ++c) {
-          const uintptr_t src = wa + (uintptr_t)(hsel * 32 + c * 16);
-          const uintptr_t end = reinterpret_cast<uintptr_t>(wq_end);
-          const uint32_t nbytes = src >= end ? 0u : (end - src >= 16 ? 16u : (uint32_t)(end - src));
-          cp_async16(rdst + 16u * c, reinterpret_cast<const void *>(nbytes ? src : reinterpret_cast<uintptr_t>(wq)),
-                     nbytes);
+          const uint8_t *src = wa + hsel * 32 + c * 16;
+          if (!rs.wtail[j]) {
+            cp_async16(rdst + 16u * c, src, 16u);
+          } else {   // the matrix's last rows: never read past its end
+            const uintptr_t e = reinterpret_cast<uintptr_t>(wq_end), a = reinterpret_cast<uintptr_t>(src);
+            const uint32_t nbytes = a >= e ? 0u : (e - a >= 16 ? 16u : (uint32_t)(e - a));
+            cp_async16(rdst + 16u * c, nbytes ? static_cast<const void *>(src) : static_cast<const void *>(wq), nbytes);
+          }
         }
       }
     };
@@ -424,9 +434,7 @@ k_moe_gemm(const __grid_constant__ CUtensorMap tmap_h, const __nv_bfloat16 *__re
         if (csrc.wrow[j]) {
           // this thread's block inside the row's window: 20 bytes from its offset rounded down to 4
           RawBlk cur;
-          const uintptr_t babs = reinterpret_cast<uintptr_t>(csrc.wrow[j]) + (uintptr_t)(cks * 2 + hsel) * MOE_QBYTES;
-          const uintptr_t wa = (reinterpret_cast<uintptr_t>(csrc.wrow[j]) + (uintptr_t)cks * 2 * MOE_QBYTES) & ~(uintptr_t)15;
-          const uint32_t off = (uint32_t)(babs - wa);   // < 48
+          const uint32_t off = ((csrc.wlo[j] + (uint32_t)cks * 2u * MOE_QBYTES) & 15u) + (uint32_t)hsel * MOE_QBYTES;   // < 48
           const uint32_t *rp = reinterpret_cast<const uint32_t *>(
               smem_raw + (raw_base - smem_u32(smem_raw)) + (size_t)s * kRawStageBytes + (size_t)n * kRawRowBytes +
               (off & ~3u));
