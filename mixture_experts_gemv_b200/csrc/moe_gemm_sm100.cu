@@ -14,19 +14,24 @@
 // n-tile; a down work item is up to two consecutive tiles of one expert (M = 256 as two
 // 128-row MMA halves sharing the B tile, so the decode work per MMA halves) and one n-tile.
 // The A tile of a K step lands in the 128-byte swizzled K-major layout: gate_up's producers
-// gather the tokens' rows of x with 16-byte asynchronous copies (zero-filled past the
-// expert's rows); down's 128 x 64 tiles of the padded h come by 2-D TMA copies. The raw
-// Q4_0 bytes of the B rows are copied (16-byte asynchronous copies of a 64-byte window per
-// row) into a staging buffer of the stage. The weights never exist in bf16 in global memory:
-// the producers decode (q - 8) * d from the staged bytes and write the swizzled K-major B
-// tile that tcgen05.mma reads.
+// gather the tokens' rows of x with 16-byte asynchronous copies, eight lanes per 128-byte row
+// segment (zero-filled past the expert's rows); down's 128 x 64 tiles of the padded h come by
+// 2-D TMA copies. The raw Q4_0 bytes of the B rows come by TMA too: the weight matrix is seen
+// as lines of 4 consecutive rows (a line's length, 4 x 18 K / 32 bytes, is a multiple of 16
+// for every K that is a multiple of 64), and one box of 48 bytes x 32 lines fetches, for one
+// residue r of the row index mod 4, the K step's two blocks (36 bytes, which start at most 12
+// bytes past a 16-byte boundary) of 32 rows. The weights never exist in bf16 in global
+// memory: the producers decode (q - 8) * d from the staged bytes and write the swizzled
+// K-major B tile that tcgen05.mma reads. B tile row 32 r + i holds weight row 4 i + r of the
+// item (so a warp's lanes read and write shared memory without bank conflicts); the
+// epilogue puts the columns back in weight-row order.
 //
 // One CTA per SM, persistent over work items, warp-specialised:
 //   warps 0-3  epilogue: tcgen05.ld of the 128 x 128 FP32 accumulators (lane = row)
 //   warp  4    TMEM allocation; lane 0 issues tcgen05.mma (M = 128, N = 128, K = 16, one
 //              per 16-wide K slice and item half)
 //   warps 5-20 producers in two groups taking alternate K steps: A copies (gate_up) or the
-//              TMA issue (down), raw-window copies, Q4_0 -> bf16 dequantisation for B
+//              TMA issue (down), the raw-weight TMA issue, Q4_0 -> bf16 dequantisation for B
 // Shared-memory stages are handed over with mbarriers (every wait is time-bounded); the
 // accumulators are double-buffered in TMEM so the epilogue of one item overlaps the next.
 #include <cuda.h>
@@ -39,6 +44,7 @@ namespace {
 constexpr int BM = 128, BK = 64;
 static_assert(BM == MOE_GEMM_TILE_ROWS, "the tile list is built with this tile height");
 constexpr int kMaxStages = 5;
+constexpr int kMaxRawSlots = 3;
 constexpr int kEpiWarps = 4;
 constexpr int kMmaWarp = 4;
 constexpr int kProdGroups = 2;                                // producer groups take alternate K steps
@@ -47,7 +53,9 @@ constexpr int kProdThreads = kProdWarps * 32;
 constexpr int kGroupThreads = kProdThreads / kProdGroups;     // one (row, block) of the B tile each
 constexpr int kThreads = (kEpiWarps + 1 + kProdWarps) * 32;
 constexpr uint32_t kTileBytes = BM * BK * 2;                  // 16 KB: one 128-row A half
-constexpr uint32_t kRawRowBytes = 64;                          // 16-byte-aligned window over a row's 36 bytes
+constexpr int kSubRows = 32;                                   // rows of one raw box (one residue mod 4)
+constexpr uint32_t kWinBytes = 48;                             // a K step's window of one row
+constexpr uint32_t kSubBytes = kSubRows * kWinBytes;           // 1536: one raw box in shared memory
 
 // UMMA instruction descriptor, kind::f16: D FP32 (bits 4-5 = 1), A and B bf16 (bits 7-9,
 // 10-12 = 1), both K-major (bits 15, 16 = 0), N >> 3 in bits 17-22, M >> 4 in bits 24-28.
@@ -73,14 +81,15 @@ struct GemmCfg {
   static constexpr uint32_t kBBytes = (uint32_t)kBN * BK * 2;
   static constexpr uint32_t kBOff = kHalves * kTileBytes;        // B tile after the A halves
   static constexpr uint32_t kStageBytes = kBOff + kBBytes;
-  static constexpr uint32_t kRawStageBytes = (uint32_t)kBN * kRawRowBytes;
+  static constexpr uint32_t kRawSlotBytes = (uint32_t)(kBN / kSubRows) * kSubBytes;   // kBN rows' windows
+  static constexpr int kRawSlots = GATEUP ? 3 : 2;                 // raw ring slots per producer group
   static constexpr uint32_t kTmemCols = 2 * kHalves * kBN;       // two accumulator buffers
-  static constexpr int kSmemBytes = kStages * (kStageBytes + kRawStageBytes) + 1024;
-  static constexpr int kRowsPerThread = kBN / (kGroupThreads / 2);   // B rows a producer thread decodes
+  static constexpr int kSmemBytes = kStages * kStageBytes + kProdGroups * kRawSlots * kRawSlotBytes + 1024;
   static constexpr uint32_t kIdesc = umma_idesc(kBN);
   static_assert(kAhead * kProdGroups <= kStages, "the prologue's stages must be free");
-  static_assert(kStages <= kMaxStages && kTmemCols <= 512, "limits");
-  static_assert(kRowsPerThread * (kGroupThreads / 2) == kBN, "producer threads cover the B rows");
+  static_assert(kStages <= kMaxStages && kRawSlots <= kMaxRawSlots && kTmemCols <= 512, "limits");
+  // the producer group's threads: one B row each (gate_up), or one block of a B row (down)
+  static_assert(kBN * (GATEUP ? 1 : 2) == kGroupThreads, "producer threads cover the B tile");
 };
 
 // Shared-memory matrix descriptor: K-major operand, 128-byte swizzle (layout type 2),
@@ -92,6 +101,7 @@ __device__ __forceinline__ uint64_t sw128_desc(uint32_t saddr) {
 struct GemmBars {
   uint64_t full[kMaxStages];
   uint64_t empty[kMaxStages];
+  uint64_t raw[kProdGroups][kMaxRawSlots];   // a producer group's raw ring slot has landed (TMA bytes)
   uint64_t acc_full[2];
   uint64_t acc_empty[2];
   uint32_t tmem_base;
@@ -149,15 +159,26 @@ __device__ __forceinline__ void umma_commit(uint64_t *bar) {
 __device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
 __device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
 
-__device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t (&r)[16]) {
-  asm volatile(
-      "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, "
-      "%15}, [%16];"
-      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
-        "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
-      : "r"(taddr));
+__device__ __forceinline__ void tmem_ld4(uint32_t taddr, uint32_t (&r)[4]) {
+  asm volatile("tcgen05.ld.sync.aligned.32x32b.x4.b32 {%0, %1, %2, %3}, [%4];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+               : "r"(taddr));
 }
 __device__ __forceinline__ void tmem_ld_wait() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
+
+// Named barrier over n threads that also returns the AND of every thread's v (bar.red).
+__device__ __forceinline__ bool named_bar_and(int id, int n, bool v) {
+  uint32_t r;
+  asm volatile(
+      "{\n\t.reg .pred p, q;\n\t"
+      "setp.ne.u32 q, %1, 0;\n\t"
+      "bar.red.and.pred p, %2, %3, q;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(r)
+      : "r"((uint32_t)v), "r"(id), "r"(n)
+      : "memory");
+  return r != 0;
+}
 
 __device__ __forceinline__ void st_shared_v4(uint32_t addr, uint32_t a, uint32_t b, uint32_t c, uint32_t d) {
   asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(a), "r"(b), "r"(c), "r"(d) : "memory");
@@ -201,37 +222,49 @@ __device__ __forceinline__ void dq_word(uint32_t w, __nv_bfloat162 d2, uint32_t 
   hi23 = cv(h23);
 }
 
-// The 20-byte window holding one 18-byte Q4_0 block (starting at the block's address rounded
-// down to 4 bytes; never past the end of a Q4_0 matrix whose rows are whole blocks, since
-// the last block of a matrix starts at 2 mod 4) and the block's offset in it, in bits.
-struct RawBlk {
-  uint32_t w[5];
-  uint32_t sh;
-};
-
-// Decode one block into its 4 swizzled 16-byte chunks of row `row` (chunks cbase..cbase+3).
-__device__ __forceinline__ void store_blk_bf16(const RawBlk &r, uint32_t tile_saddr, int row, int cbase) {
-  const float d = __half2float(__ushort_as_half((unsigned short)((r.w[0] >> r.sh) & 0xffffu)));
-  const __nv_bfloat162 d2 = __float2bfloat162_rn(d);
-  const uint32_t s2 = r.sh + 16u;
-  uint32_t q[4];
-#pragma unroll
-  for (int i = 0; i < 4; ++i) q[i] = __funnelshift_rc(r.w[i], r.w[i + 1], s2);
+// One block -- fp16 scale bits and its four code words -- into its 4 swizzled 16-byte chunks
+// (cbase .. cbase + 3) of the B tile row at rowbase (x = the row's swizzle phase).
+__device__ __forceinline__ void store_blk_bf16(uint32_t dbits, const uint32_t (&q)[4], uint32_t rowbase, uint32_t x,
+                                               int cbase) {
+  const __nv_bfloat162 d2 = __float2bfloat162_rn(__half2float(__ushort_as_half((unsigned short)(dbits & 0xffffu))));
   uint32_t lo[8], hi[8];   // element pairs (0,1),(2,3),...,(14,15) and (16,17),...,(30,31)
 #pragma unroll
   for (int i = 0; i < 4; ++i) dq_word(q[i], d2, lo[2 * i], lo[2 * i + 1], hi[2 * i], hi[2 * i + 1]);
-  const uint32_t rowbase = tile_saddr + (uint32_t)row * 128u;
-  const uint32_t x = (uint32_t)(row & 7);
   st_shared_v4(rowbase + (((uint32_t)(cbase + 0) ^ x) << 4), lo[0], lo[1], lo[2], lo[3]);   // elements 0-7
   st_shared_v4(rowbase + (((uint32_t)(cbase + 1) ^ x) << 4), lo[4], lo[5], lo[6], lo[7]);   // 8-15
   st_shared_v4(rowbase + (((uint32_t)(cbase + 2) ^ x) << 4), hi[0], hi[1], hi[2], hi[3]);   // 16-23
   st_shared_v4(rowbase + (((uint32_t)(cbase + 3) ^ x) << 4), hi[4], hi[5], hi[6], hi[7]);   // 24-31
 }
 
-// Zeros into the 4 swizzled 16-byte chunks of row `row` (chunks cbase..cbase+3).
-__device__ __forceinline__ void store_blk_zero(uint32_t tile_saddr, int row, int cbase) {
-  const uint32_t rowbase = tile_saddr + (uint32_t)row * 128u;
-  const uint32_t x = (uint32_t)(row & 7);
+// A row's 48-byte window w[12] of a K step whose two blocks start at word WB (byte 4 WB):
+// block 0 = scale in the low half of word WB, codes two bytes further (each code word spans
+// two window words); block 1 = scale in the high half of word WB + 4, codes in words
+// WB + 5 .. WB + 8. BLK selects the blocks decoded: 1, 2 or 3 (both).
+template <int WB, int BLK>
+__device__ __forceinline__ void dec_window(const uint32_t (&w)[12], uint32_t rowbase, uint32_t x) {
+  if (BLK & 1) {
+    uint32_t q[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) q[i] = __byte_perm(w[WB + i], w[WB + i + 1], 0x5432u);
+    store_blk_bf16(w[WB], q, rowbase, x, 0);
+  }
+  if (BLK & 2) {
+    const uint32_t q[4] = {w[WB + 5], w[WB + 6], w[WB + 7], w[WB + 8]};
+    store_blk_bf16(w[WB + 4] >> 16, q, rowbase, x, 4);
+  }
+}
+template <int BLK>
+__device__ __forceinline__ void dec_window_at(int wb, const uint32_t (&w)[12], uint32_t rowbase, uint32_t x) {
+  switch (wb) {   // warp-uniform: the window offset depends on the K step and the row residue only
+    case 0: dec_window<0, BLK>(w, rowbase, x); break;
+    case 1: dec_window<1, BLK>(w, rowbase, x); break;
+    case 2: dec_window<2, BLK>(w, rowbase, x); break;
+    default: dec_window<3, BLK>(w, rowbase, x); break;
+  }
+}
+
+// Zeros into the 4 swizzled 16-byte chunks cbase .. cbase + 3 of the B tile row at rowbase.
+__device__ __forceinline__ void store_blk_zero(uint32_t rowbase, uint32_t x, int cbase) {
 #pragma unroll
   for (int c = 0; c < 4; ++c) st_shared_v4(rowbase + (((uint32_t)(cbase + c) ^ x) << 4), 0u, 0u, 0u, 0u);
 }
@@ -243,11 +276,12 @@ __device__ __forceinline__ void store_blk_zero(uint32_t tile_saddr, int row, int
 //         padded order).
 // DOWN:   A = hb [padded rows, f] (tmap_h: 2-D tiles of 128 rows x 64 columns by TMA), B =
 //         down rows n0..n0+127, K = f; epilogue y * w * s -> yslot (bf16, slot order).
+// tmap_w: the weight matrix (gate_up or down) as lines of 4 rows, boxes of 48 bytes x 32 lines.
 template <bool GATEUP>
 __global__ void __launch_bounds__(kThreads, 1)
-k_moe_gemm(const __grid_constant__ CUtensorMap tmap_h, const __nv_bfloat16 *__restrict__ a_src,
-           const uint8_t *__restrict__ wq, const uint8_t *wq_end,
-           const float *__restrict__ expert_scale, int d, int f, int k, MoeWork W) {
+k_moe_gemm(const __grid_constant__ CUtensorMap tmap_h, const __grid_constant__ CUtensorMap tmap_w,
+           const __nv_bfloat16 *__restrict__ a_src, const float *__restrict__ expert_scale, int d, int f, int k,
+           MoeWork W) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   __shared__ GemmBars bars;
   const uint32_t sbase = (smem_u32(smem_raw) + 1023u) & ~1023u;
@@ -256,15 +290,15 @@ k_moe_gemm(const __grid_constant__ CUtensorMap tmap_h, const __nv_bfloat16 *__re
   const int K = GATEUP ? d : f;
   const int ksteps = K / BK;
   using C = GemmCfg<GATEUP>;
-  constexpr int kBN = C::kBN, kRows = C::kRowsPerThread;
+  constexpr int kBN = C::kBN;
   const int n_ntiles = GATEUP ? (f + kBN / 2 - 1) / (kBN / 2) : d / kBN;
-  const int nb_row = K / MOE_QK;                       // Q4_0 blocks per weight row
-  const size_t rb = (size_t)nb_row * MOE_QBYTES;       // bytes per weight row
-  const size_t expert_bytes = (size_t)(GATEUP ? 2 * f : d) * rb;
+  const int rb = (K / MOE_QK) * MOE_QBYTES;            // bytes per weight row
   constexpr int kHalves = C::kHalves, kStages = C::kStages, kAhead = C::kAhead;
   constexpr uint32_t kBOff = C::kBOff, kStageBytes = C::kStageBytes, kTmemCols = C::kTmemCols;
-  constexpr uint32_t kRawStageBytes = C::kRawStageBytes;
   const int n_items = (GATEUP ? *W.n_tiles : *W.n_pairs) * n_ntiles;
+  // Work order: the n-tiles of one row tile (gate_up) or tile pair (down) follow each other,
+  // so its A rows are read while in L2.
+  auto item_nt = [&](int item) -> int { return item % n_ntiles; };
   // work item -> its first tile, and whether a second tile (rows 128 .. 255 past the first
   // tile's start) belongs to it (down only)
   auto item_tile = [&](int item, int &tile, bool &h1) {
@@ -280,9 +314,11 @@ k_moe_gemm(const __grid_constant__ CUtensorMap tmap_h, const __nv_bfloat16 *__re
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < kStages; ++s) {
-      mbar_init(&bars.full[s], kGroupThreads);   // the step's producer group arrives
+      mbar_init(&bars.full[s], kGroupThreads / 32);   // the step's producer group's warps arrive
       mbar_init(&bars.empty[s], 1);
     }
+    for (int q = 0; q < kProdGroups * kMaxRawSlots; ++q)
+      mbar_init(&bars.raw[q / kMaxRawSlots][q % kMaxRawSlots], kBN / kSubRows);   // one arrival per box
     for (int b = 0; b < 2; ++b) {
       mbar_init(&bars.acc_full[b], 1);
       mbar_init(&bars.acc_empty[b], kEpiWarps * 32);
@@ -301,32 +337,50 @@ k_moe_gemm(const __grid_constant__ CUtensorMap tmap_h, const __nv_bfloat16 *__re
 
   if (warp >= kMmaWarp + 1) {
     // ------------------------------------------------------------ producers
-    // Producer group pg takes the K steps g with g % kProdGroups == pg. Thread pt of a group
-    // owns A row r = pt / 2 (of each half): chunks 4 h .. 4 h + 3 (h = pt & 1) of the row's
-    // 128-byte K-step segment; and B rows r + 128 j (j < kRows): Q4_0 block h of each row's two
-    // blocks per K step.
+    // Producer group pg takes the K steps g with g % kProdGroups == pg (its local steps li:
+    // g = pg + kProdGroups li). Thread pt of a group:
+    //  A (gate_up): 16-byte chunk pt % 8 of A rows pt / 8 + 32 q (q < 4);
+    //  B: warp wg = pt / 32 of the group and lane i decode weight row 4 i + r of the item into
+    //    B tile row j * 128 + 32 r + i, where (gate_up) j = wg / 4 is gate (0) or up (1), both
+    //    blocks of the K step; (down) j = 0 and the thread decodes block h = wg / 4 only;
+    //    r = wg % 4 in both;
+    //  raw: the group has a ring of kRawSlots slots of its own; warp wg < nsub issues box wg of
+    //    a step kRawSlots local steps ahead, once the whole group has read the slot.
+    // Every decision to stop is taken by the whole group at its named barrier (all bounded
+    // waits come before it), so no thread is left waiting there.
     const int pq = threadIdx.x - (kMmaWarp + 1) * 32;
     const int pg = pq / kGroupThreads, pt = pq - pg * kGroupThreads;   // pt 0..255
-    const int row = pt >> 1, hsel = pt & 1;
-    // the raw Q4_0 bytes of B row n for a K step (two blocks, 36 bytes) arrive in a 64-byte
-    // window starting at their address rounded down to 16; hsel copies its half of it
-    const uint32_t raw_base = sbase + (uint32_t)kStages * kStageBytes;
+    const int wg = pt >> 5, res = wg & 3, jh = wg >> 2;
+    const int cb = pt & 7;                                              // A chunk
+    constexpr int nsub = kBN / kSubRows;                                // raw boxes per step
+    constexpr int kRawSlots = C::kRawSlots;
+    constexpr uint32_t kRawSlotBytes = C::kRawSlotBytes;
+    const uint32_t raw_base = sbase + (uint32_t)kStages * kStageBytes + (uint32_t)pg * kRawSlots * kRawSlotBytes;
     const int my_items = blockIdx.x < n_items ? (n_items - 1 - (int)blockIdx.x) / (int)gridDim.x + 1 : 0;
     const int total = my_items * ksteps;
-    // sources of this thread's rows for the CTA's jj-th work item: the A rows of both halves
-    // (null past the expert's rows; gate_up only), the B rows (null past the expert's f gate
-    // or up rows: decoded as zeros), the tile, and whether the second half holds any of the
-    // expert's rows
+    const int n_local = total > pg ? (total - pg + kProdGroups - 1) / kProdGroups : 0;
+    // the first line of the CTA's jj-th item's B rows in the weight map (gate rows for gate_up;
+    // the up rows are f / 4 lines on)
+    auto item_line0 = [&](int jj) -> int {
+      const int item = (int)blockIdx.x + jj * (int)gridDim.x;
+      const int nt = item_nt(item);
+      int tile;
+      bool h1;
+      item_tile(item, tile, h1);
+      const int e = W.tiles[2 * tile];
+      return GATEUP ? (e * 2 * f + nt * (kBN / 2)) >> 2 : (int)(((long long)e * d + (long long)nt * kBN) >> 2);
+    };
+    // sources for the CTA's jj-th work item: this thread's A rows (null past the expert's rows;
+    // gate_up only), whether this thread's B row is one of the expert's (gate_up: gate and up
+    // rows c < f), the tile, and whether the second half holds any of the expert's rows
     struct RowSrc {
-      const __nv_bfloat16 *arow[kHalves];
-      const uint8_t *wrow[kRows];
-      uint32_t wlo[kRows];    // low 4 bits of the row's address
-      bool wtail[kRows];      // the row's last windows can reach past the end of the matrix
+      const __nv_bfloat16 *arow[GATEUP ? 4 : 1];
+      bool wvalid;
       int tile, h1;
     };
     auto item_src = [&](int jj) -> RowSrc {
       const int item = (int)blockIdx.x + jj * (int)gridDim.x;
-      const int nt = item % n_ntiles;
+      const int nt = item_nt(item);
       int tile;
       bool h1;
       item_tile(item, tile, h1);
@@ -335,131 +389,132 @@ k_moe_gemm(const __grid_constant__ CUtensorMap tmap_h, const __nv_bfloat16 *__re
       RowSrc rs;
       rs.tile = tile;
       rs.h1 = h1;
+      if (GATEUP) {
 #pragma unroll
-      for (int h = 0; h < kHalves; ++h) {
-        const int r = m0 + h * BM + row;
-        rs.arow[h] = (GATEUP && r < cnt) ? a_src + (size_t)(W.perm[W.offsets[e] + r] / k) * d : nullptr;
-      }
-      const uint8_t *ebase = wq + (size_t)e * expert_bytes;
-#pragma unroll
-      for (int j = 0; j < kRows; ++j) {
-        if (GATEUP) {
-          // B row j * 128 + row: gate row c0 + row (j = 0) or up row f + c0 + row (j = 1)
-          const int c = nt * (kBN / 2) + row;
-          rs.wrow[j] = c < f ? ebase + (size_t)(j * f + c) * rb : nullptr;
-        } else {
-          rs.wrow[j] = ebase + (size_t)(nt * kBN + j * 128 + row) * rb;
+        for (int q = 0; q < 4; ++q) {
+          const int r = m0 + (pt >> 3) + 32 * q;
+          rs.arow[q] = r < cnt ? a_src + (size_t)(W.perm[W.offsets[e] + r] / k) * d : nullptr;
         }
-        // a K step's 64-byte window starts at most 15 bytes before its blocks and ends at most
-        // 28 bytes past the row's last block
-        rs.wlo[j] = (uint32_t)(reinterpret_cast<uintptr_t>(rs.wrow[j]) & 15u);
-        rs.wtail[j] = rs.wrow[j] != nullptr && rs.wrow[j] + rb + 28 > wq_end;
+        rs.wvalid = nt * (kBN / 2) + 4 * (pt & 31) + res < f;
+      } else {
+        rs.arow[0] = nullptr;
+        rs.wvalid = true;
       }
       return rs;
     };
-    auto issue = [&](const RowSrc &rs, int ks, int s) {
+    // A of step (rs, ks) into stage s: gathered rows (gate_up), or the h tiles by TMA (down)
+    auto issue_a = [&](const RowSrc &rs, int ks, int s) {
       const uint32_t a_saddr = sbase + (uint32_t)s * kStageBytes;
       if (GATEUP) {
 #pragma unroll
-        for (int h = 0; h < kHalves; ++h) {
-          if (h > 0 && !rs.h1) break;   // the MMA skips an empty second half
-          const __nv_bfloat16 *ap = rs.arow[h] ? rs.arow[h] + (size_t)ks * BK + (size_t)hsel * (BK / 2) : a_src;
-          const uint32_t tile_a = a_saddr + (uint32_t)h * kTileBytes;
-#pragma unroll
-          for (int c = 0; c < 4; ++c) {
-            const uint32_t chunk = (uint32_t)(hsel * 4 + c);
-            cp_async16(tile_a + (uint32_t)row * 128u + ((chunk ^ (uint32_t)(row & 7)) << 4),
-                       ap + (rs.arow[h] ? 8 * c : 0), rs.arow[h] ? 16u : 0u);
-          }
+        for (int q = 0; q < 4; ++q) {
+          const int ra = (pt >> 3) + 32 * q;
+          const __nv_bfloat16 *ap = rs.arow[q] ? rs.arow[q] + (size_t)ks * BK + 8 * cb : a_src;
+          cp_async16(a_saddr + (uint32_t)ra * 128u + (((uint32_t)cb ^ (uint32_t)(ra & 7)) << 4), ap,
+                     rs.arow[q] ? 16u : 0u);
         }
       } else if (pt == 0) {
         // the 128 x 64 tiles of h by TMA: their bytes join the stage's full barrier, whose
-        // phase cannot complete before this thread's own arrival for the step (after this call)
+        // phase cannot complete before this thread's warp arrives for the step (after this call)
         mbar_expect_tx(&bars.full[s], kTileBytes * (rs.h1 ? 2u : 1u));
         tma_load_2d(a_saddr, &tmap_h, ks * BK, rs.tile * BM, &bars.full[s]);
         if (rs.h1) tma_load_2d(a_saddr + kTileBytes, &tmap_h, ks * BK, rs.tile * BM + BM, &bars.full[s]);
       }
-#pragma unroll
-      for (int j = 0; j < kRows; ++j) {
-        if (!rs.wrow[j]) continue;   // a zero row: nothing to copy
-        const uint32_t kb = (uint32_t)ks * 2u * MOE_QBYTES;
-        const uint8_t *wa = rs.wrow[j] + kb - ((rs.wlo[j] + kb) & 15u);   // 16-byte aligned window start
-        const uint32_t rdst = raw_base + (uint32_t)s * kRawStageBytes + (uint32_t)(j * 128 + row) * kRawRowBytes +
-                              (uint32_t)hsel * 32u;
-#pragma unroll
-        for (int c = 0; c < 2; ++c) {
-          const uint8_t *src = wa + hsel * 32 + c * 16;
-          if (!rs.wtail[j]) {
-            cp_async16(rdst + 16u * c, src, 16u);
-          } else {   // the matrix's last rows: never read past its end
-            const uintptr_t e = reinterpret_cast<uintptr_t>(wq_end), a = reinterpret_cast<uintptr_t>(src);
-            const uint32_t nbytes = a >= e ? 0u : (e - a >= 16 ? 16u : (uint32_t)(e - a));
-            cp_async16(rdst + 16u * c, nbytes ? static_cast<const void *>(src) : static_cast<const void *>(wq), nbytes);
-          }
-        }
+    };
+    // raw boxes of step (line0, ks) into ring slot q: box wg (residue r = wg % 4 of part wg / 4)
+    // starts at the K step's window rounded down to 16 bytes
+    auto issue_raw = [&](int line0, int ks, int q) {
+      if (lane == 0 && wg < nsub) {
+        const int r = wg & 3, j = wg >> 2;
+        const uint32_t xb = ((uint32_t)r * (uint32_t)rb + (uint32_t)ks * 2u * MOE_QBYTES) & ~15u;
+        mbar_arrive_expect_tx(&bars.raw[pg][q], kSubBytes);
+        tma_load_2d(raw_base + (uint32_t)q * kRawSlotBytes + (uint32_t)wg * kSubBytes, &tmap_w, (int)xb,
+                    line0 + j * (f >> 2), &bars.raw[pg][q]);
       }
     };
     bool ok = true;
-    // issue side and consume side walk this group's steps g = pg, pg + G, ... (G groups);
-    // copies run kAhead group steps ahead of the decode
+    // three walks over this group's steps: the raw issue (kRawSlots steps ahead), the A issue
+    // (kAhead steps ahead) and the decode
+    int rjj = 0, rks = pg, ijj = 0, iks = pg, cjj = 0, cks = pg;
+    while (rks >= ksteps && rjj < my_items) { rks -= ksteps; ++rjj; }
+    ijj = cjj = rjj;
+    iks = cks = rks;
+    int rline = rjj < my_items ? item_line0(rjj) : 0;
     RowSrc isrc{}, csrc{};
-    int ijj = 0, iks = pg, cjj = 0, cks = pg;
-    while (iks >= ksteps && ijj < my_items) { iks -= ksteps; ++ijj; }
-    cjj = ijj;
-    cks = iks;
     if (ijj < my_items) { isrc = item_src(ijj); csrc = isrc; }
-    auto adv = [&](int &jj, int &ks, RowSrc &src) {
+    auto step = [&](int &jj, int &ks) -> bool {   // to the group's next step; true on a new item
       ks += kProdGroups;
       bool moved = false;
       while (ks >= ksteps) { ks -= ksteps; ++jj; moved = true; }
-      if (moved && jj < my_items) src = item_src(jj);
+      return moved && jj < my_items;
     };
-    int gi = pg;
-    for (int a = 0; a < kAhead; ++a, gi += kProdGroups) {   // the first stages are free
-      if (gi < total) {
-        issue(isrc, iks, gi % kStages);
-        adv(ijj, iks, isrc);
-      }
+    int raw_issued = 0;
+    for (int q = 0; q < kRawSlots && q < n_local; ++q, ++raw_issued) {   // the ring's first fill
+      issue_raw(rline, rks, q);
+      if (step(rjj, rks)) rline = item_line0(rjj);
+    }
+    for (int a = 0; a < kAhead && a < n_local; ++a) {   // the first stages are free
+      issue_a(isrc, iks, (pg + kProdGroups * a) % kStages);
+      if (step(ijj, iks)) isrc = item_src(ijj);
       cp_async_commit();
     }
-    for (int g = pg; g < total; g += kProdGroups, gi += kProdGroups) {
-      // step g: its copies have landed (issued kAhead group steps ago); decode B, hand over
+    // this thread's B row in the tile and its raw window in a ring slot
+    const int brow = (GATEUP ? jh * 128 : 0) + res * 32 + lane;
+    const uint32_t win_off = (uint32_t)((GATEUP ? jh * 4 : 0) + res) * kSubBytes + (uint32_t)lane * kWinBytes;
+    int li = 0;
+    for (; li < n_local; ++li) {
+      const int g = pg + kProdGroups * li;
+      const int s = g % kStages, q = li % kRawSlots;
+      // step g: its A copies (this thread's, issued kAhead steps ago) and its raw boxes have landed
       cp_async_wait<kAhead - 1>();
-      __syncwarp();   // a row's window is copied by two lanes
-      const int s = g % kStages;
-      const uint32_t b_saddr = sbase + (uint32_t)s * kStageBytes + kBOff;
-#pragma unroll
-      for (int j = 0; j < kRows; ++j) {
-        const int n = j * 128 + row;   // B row
-        if (csrc.wrow[j]) {
-          // this thread's block inside the row's window: 20 bytes from its offset rounded down to 4
-          RawBlk cur;
-          const uint32_t off = ((csrc.wlo[j] + (uint32_t)cks * 2u * MOE_QBYTES) & 15u) + (uint32_t)hsel * MOE_QBYTES;   // < 48
-          const uint32_t *rp = reinterpret_cast<const uint32_t *>(
-              smem_raw + (raw_base - smem_u32(smem_raw)) + (size_t)s * kRawStageBytes + (size_t)n * kRawRowBytes +
-              (off & ~3u));
-#pragma unroll
-          for (int i = 0; i < 5; ++i) cur.w[i] = rp[i];
-          cur.sh = (off & 3u) * 8u;
-          store_blk_bf16(cur, b_saddr, n, hsel * 4);
-        } else {
-          store_blk_zero(b_saddr, n, hsel * 4);
-        }
+      if (!mbar_wait(&bars.raw[pg][q], (uint32_t)(li / kRawSlots) & 1u, W.err, 14, W.wait_ns)) ok = false;
+      const uint32_t rowbase = sbase + (uint32_t)s * kStageBytes + kBOff + (uint32_t)brow * 128u;
+      const uint32_t x = (uint32_t)(brow & 7);
+      if (ok && csrc.wvalid) {
+        const uint4 *wp = reinterpret_cast<const uint4 *>(smem_raw + (raw_base - smem_u32(smem_raw)) +
+                                                          (size_t)q * kRawSlotBytes + win_off);
+        const uint4 v0 = wp[0], v1 = wp[1], v2 = wp[2];
+        const uint32_t w[12] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w, v2.x, v2.y, v2.z, v2.w};
+        const int wb = (int)((((uint32_t)res * (uint32_t)rb + (uint32_t)cks * 2u * MOE_QBYTES) & 15u) >> 2);
+        if (GATEUP) dec_window_at<3>(wb, w, rowbase, x);
+        else if (jh == 0) dec_window_at<1>(wb, w, rowbase, x);
+        else dec_window_at<2>(wb, w, rowbase, x);
+      } else {
+        store_blk_zero(rowbase, x, 0);
+        store_blk_zero(rowbase, x, 4);
       }
       fence_proxy_async_smem();
-      mbar_arrive(&bars.full[s]);
-      adv(cjj, cks, csrc);
-      // then refill the stage that step gi uses, once the MMA has released it
-      if (gi < total) {
-        const int si = gi % kStages;
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&bars.full[s]);
+      // Slot q is refilled by TMA (the async proxy) only after the group's barrier, and only
+      // once every thread has used the bytes it read from the slot (the decode's stores depend
+      // on them): a shared-memory load still in flight at a barrier is not ordered before a
+      // later TMA write. The barrier is also where the group agrees on going on.
+      if (!named_bar_and(1 + pg, kGroupThreads, ok)) break;
+      if (li + kRawSlots < n_local) {
+        issue_raw(rline, rks, q);
+        ++raw_issued;
+        if (step(rjj, rks)) rline = item_line0(rjj);
+      }
+      if (step(cjj, cks)) csrc = item_src(cjj);
+      // then the A copies of local step li + kAhead, once the MMA has released its stage
+      if (li + kAhead < n_local) {
+        const int gi = g + kProdGroups * kAhead, si = gi % kStages;
         const uint32_t par = ((uint32_t)(gi / kStages) & 1u) ^ 1u;
-        if (!mbar_wait(&bars.empty[si], par, W.err, 10, W.wait_ns)) { ok = false; break; }
-        issue(isrc, iks, si);
-        adv(ijj, iks, isrc);
+        if (mbar_wait(&bars.empty[si], par, W.err, 10, W.wait_ns)) {
+          issue_a(isrc, iks, si);
+          if (step(ijj, iks)) isrc = item_src(ijj);
+        } else {
+          ok = false;   // the group stops at its next barrier
+        }
       }
       cp_async_commit();
     }
     cp_async_wait<0>();   // no copy lands after this thread leaves
+    // after an early stop, the raw boxes still in flight land before the group leaves (each
+    // wait bounded; a completed phase returns at once)
+    for (int lq = li; lq < raw_issued; ++lq)
+      mbar_wait(&bars.raw[pg][lq % kRawSlots], (uint32_t)(lq / kRawSlots) & 1u, W.err, 15, W.wait_ns);
     if (!ok) atomicExch(&bars.abort_flag, 1);
   } else if (warp == kMmaWarp) {
     // ------------------------------------------------------------ MMA issue (one thread)
@@ -508,7 +563,7 @@ k_moe_gemm(const __grid_constant__ CUtensorMap tmap_h, const __nv_bfloat16 *__re
       const bool ok = mbar_wait(&bars.acc_full[b], par, W.err, 13, W.wait_ns);
       if (__any_sync(0xffffffffu, !ok)) { atomicExch(&bars.abort_flag, 1); break; }
       tc_fence_after();
-      const int nt = item % n_ntiles;
+      const int nt = item_nt(item);
       int tile;
       bool h1;
       item_tile(item, tile, h1);
@@ -519,21 +574,29 @@ k_moe_gemm(const __grid_constant__ CUtensorMap tmap_h, const __nv_bfloat16 *__re
         const int mr = m0 + h * BM + r;        // row of the expert
         const bool valid = mr < cnt;
         const uint32_t taddr = tmem + ((uint32_t)(warp * 32) << 16) + (uint32_t)((b * kHalves + h) * kBN);
+        // accumulator column 32 r + i holds weight row 4 i + r of the item (of each part): the
+        // 16 output columns 16 u .. 16 u + 15 are columns 32 r + 4 u + a (r, a < 4), output
+        // column 4 a + r
         if (GATEUP) {
           const int c0 = nt * (kBN / 2);   // first h column of this item
           __nv_bfloat16 *dst = W.hb + (size_t)((tile + h) * BM + r) * f + (size_t)c0;
 #pragma unroll
-          for (int c = 0; c < kBN / 2; c += 16) {
+          for (int u16 = 0; u16 < kBN / 32; ++u16) {
+            const int c = 16 * u16;
             if (c0 + c >= f) break;   // warp-uniform: the item's columns past f are zero rows
-            uint32_t g[16], u[16];
-            tmem_ld16(taddr + (uint32_t)c, g);
-            tmem_ld16(taddr + (uint32_t)(kBN / 2 + c), u);
+            uint32_t g[4][4], u[4][4];
+#pragma unroll
+            for (int rr = 0; rr < 4; ++rr) {
+              tmem_ld4(taddr + (uint32_t)(32 * rr + 4 * u16), g[rr]);
+              tmem_ld4(taddr + (uint32_t)(kBN / 2 + 32 * rr + 4 * u16), u[rr]);
+            }
             tmem_ld_wait();
             uint32_t o[8];
 #pragma unroll
-            for (int i = 0; i < 8; ++i) {
-              const float h0 = gelu_tanh_f(__uint_as_float(g[2 * i])) * __uint_as_float(u[2 * i]);
-              const float hv1 = gelu_tanh_f(__uint_as_float(g[2 * i + 1])) * __uint_as_float(u[2 * i + 1]);
+            for (int i = 0; i < 8; ++i) {   // output columns 2 i, 2 i + 1 = 4 a + r, 4 a + r + 1
+              const int a = i >> 1, r0 = 2 * (i & 1);
+              const float h0 = gelu_tanh_f(__uint_as_float(g[r0][a])) * __uint_as_float(u[r0][a]);
+              const float hv1 = gelu_tanh_f(__uint_as_float(g[r0 + 1][a])) * __uint_as_float(u[r0 + 1][a]);
               o[i] = pack_bf16(h0, hv1);
             }
             if (valid) {
@@ -551,14 +614,18 @@ k_moe_gemm(const __grid_constant__ CUtensorMap tmap_h, const __nv_bfloat16 *__re
           }
           __nv_bfloat16 *dst = reinterpret_cast<__nv_bfloat16 *>(W.yslot) + (size_t)slot * d + (size_t)nt * kBN;
 #pragma unroll
-          for (int c = 0; c < kBN; c += 16) {
-            uint32_t y[16];
-            tmem_ld16(taddr + (uint32_t)c, y);
+          for (int u16 = 0; u16 < kBN / 16; ++u16) {
+            const int c = 16 * u16;
+            uint32_t y[4][4];
+#pragma unroll
+            for (int rr = 0; rr < 4; ++rr) tmem_ld4(taddr + (uint32_t)(32 * rr + 4 * u16), y[rr]);
             tmem_ld_wait();
             uint32_t o[8];
 #pragma unroll
-            for (int i = 0; i < 8; ++i)
-              o[i] = pack_bf16(__uint_as_float(y[2 * i]) * scale, __uint_as_float(y[2 * i + 1]) * scale);
+            for (int i = 0; i < 8; ++i) {
+              const int a = i >> 1, r0 = 2 * (i & 1);
+              o[i] = pack_bf16(__uint_as_float(y[r0][a]) * scale, __uint_as_float(y[r0 + 1][a]) * scale);
+            }
             if (valid) {
               uint4 *dp = reinterpret_cast<uint4 *>(dst + c);
               dp[0] = make_uint4(o[0], o[1], o[2], o[3]);
@@ -649,6 +716,22 @@ static bool make_tmap_h(CUtensorMap *m, const void *base, int cols, long long ro
   return r == CUDA_SUCCESS;
 }
 
+// Tensor map of a Q4_0 weight matrix of `rows` rows of rb bytes (rows a multiple of 4, 4 rb a
+// multiple of 16) seen as rows / 4 lines of 4 rb bytes: boxes of 48 bytes x 32 lines, no
+// swizzle; bytes past a line's end or past the last line read as zeros.
+static bool make_tmap_w(CUtensorMap *m, const void *base, int rb, long long rows) {
+  auto enc = get_encode();
+  if (!enc || rows % 4 || (4 * rb) % 16) return false;
+  cuuint64_t dims[2] = {(cuuint64_t)(4 * rb), (cuuint64_t)(rows / 4)};
+  cuuint64_t strides[1] = {(cuuint64_t)(4 * rb)};
+  cuuint32_t box[2] = {kWinBytes, (cuuint32_t)kSubRows};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void *>(base), dims, strides, box, estr,
+                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
 int moe_launch_gemm_experts(const MoeLaunch &L, const MoeWork &W, const void *x, const uint8_t *gate_up_q4,
                             const uint8_t *down_q4, const float *expert_scale, int T, int d, int f, int E, int k,
                             float *out, int num_sms, int max_tiles) {
@@ -659,18 +742,19 @@ int moe_launch_gemm_experts(const MoeLaunch &L, const MoeWork &W, const void *x,
       !moe_allow_dyn_smem(reinterpret_cast<const void *>(k_moe_gemm<false>), &smem_ok[1]))
     return -1;
   moe_prof_mark(L.stream, MOE_K_GEMM_GATEUP, true);
-  const uint8_t *gu_end = gate_up_q4 + (size_t)E * 2 * f * (d / MOE_QK) * MOE_QBYTES;
-  const uint8_t *dn_end = down_q4 + (size_t)E * d * (f / MOE_QK) * MOE_QBYTES;
-  CUtensorMap th;
+  CUtensorMap th, twg, twd;
   if (!make_tmap_h(&th, W.hb, f, (long long)max_tiles * BM)) return -1;
+  if (!make_tmap_w(&twg, gate_up_q4, (d / MOE_QK) * MOE_QBYTES, (long long)E * 2 * f) ||
+      !make_tmap_w(&twd, down_q4, (f / MOE_QK) * MOE_QBYTES, (long long)E * d))
+    return -1;
   constexpr int kSmemG = GemmCfg<true>::kSmemBytes, kSmemD = GemmCfg<false>::kSmemBytes;
-  k_moe_gemm<true><<<num_sms, kThreads, kSmemG, L.stream>>>(th, static_cast<const __nv_bfloat16 *>(x), gate_up_q4,
-                                                            gu_end, expert_scale, d, f, k, W);
+  k_moe_gemm<true><<<num_sms, kThreads, kSmemG, L.stream>>>(th, twg, static_cast<const __nv_bfloat16 *>(x),
+                                                            expert_scale, d, f, k, W);
   if (launch_err()) return -1;
   moe_prof_count(1);
   moe_prof_mark(L.stream, MOE_K_GEMM_GATEUP, false);
   moe_prof_mark(L.stream, MOE_K_GEMM_DOWN, true);
-  k_moe_gemm<false><<<num_sms, kThreads, kSmemD, L.stream>>>(th, W.hb, down_q4, dn_end, expert_scale, d, f, k, W);
+  k_moe_gemm<false><<<num_sms, kThreads, kSmemD, L.stream>>>(th, twd, W.hb, expert_scale, d, f, k, W);
   if (launch_err()) return -1;
   moe_prof_count(1);
   moe_prof_mark(L.stream, MOE_K_GEMM_DOWN, false);
