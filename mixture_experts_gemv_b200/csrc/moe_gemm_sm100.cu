@@ -53,9 +53,8 @@ constexpr int kProdThreads = kProdWarps * 32;
 constexpr int kGroupThreads = kProdThreads / kProdGroups;     // one (row, block) of the B tile each
 constexpr int kThreads = (kEpiWarps + 1 + kProdWarps) * 32;
 constexpr uint32_t kTileBytes = BM * BK * 2;                  // 16 KB: one 128-row A half
-constexpr int kSubRows = 32;                                   // rows of one raw box (one residue mod 4)
-constexpr uint32_t kWinBytes = 48;                             // a K step's window of one row
-constexpr uint32_t kSubBytes = kSubRows * kWinBytes;           // 1536: one raw box in shared memory
+constexpr int kSubRows = 32;                                   // lines of one raw box (one residue mod 4)
+constexpr int kRawBoxes = 8;                                   // raw boxes per K step: one per producer warp
 
 // UMMA instruction descriptor, kind::f16: D FP32 (bits 4-5 = 1), A and B bf16 (bits 7-9,
 // 10-12 = 1), both K-major (bits 15, 16 = 0), N >> 3 in bits 17-22, M >> 4 in bits 24-28.
@@ -81,7 +80,12 @@ struct GemmCfg {
   static constexpr uint32_t kBBytes = (uint32_t)kBN * BK * 2;
   static constexpr uint32_t kBOff = kHalves * kTileBytes;        // B tile after the A halves
   static constexpr uint32_t kStageBytes = kBOff + kBBytes;
-  static constexpr uint32_t kRawSlotBytes = (uint32_t)(kBN / kSubRows) * kSubBytes;   // kBN rows' windows
+  // raw box width: gate_up, a row's whole 48-byte window (box w = part w / 4, residue w % 4);
+  // down, 32 bytes holding one block (box w = residue w % 4, block w / 4: bytes 0-31 of the
+  // window hold block 0, bytes 16-47 block 1)
+  static constexpr uint32_t kBoxW = GATEUP ? 48 : 32;
+  static constexpr uint32_t kSubBytes = kSubRows * kBoxW;
+  static constexpr uint32_t kRawSlotBytes = kRawBoxes * kSubBytes;
   static constexpr int kRawSlots = GATEUP ? 3 : 2;                 // raw ring slots per producer group
   static constexpr uint32_t kTmemCols = 2 * kHalves * kBN;       // two accumulator buffers
   static constexpr int kSmemBytes = kStages * kStageBytes + kProdGroups * kRawSlots * kRawSlotBytes + 1024;
@@ -165,20 +169,6 @@ __device__ __forceinline__ void tmem_ld4(uint32_t taddr, uint32_t (&r)[4]) {
                : "r"(taddr));
 }
 __device__ __forceinline__ void tmem_ld_wait() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
-
-// Named barrier over n threads that also returns the AND of every thread's v (bar.red).
-__device__ __forceinline__ bool named_bar_and(int id, int n, bool v) {
-  uint32_t r;
-  asm volatile(
-      "{\n\t.reg .pred p, q;\n\t"
-      "setp.ne.u32 q, %1, 0;\n\t"
-      "bar.red.and.pred p, %2, %3, q;\n\t"
-      "selp.u32 %0, 1, 0, p;\n\t}"
-      : "=r"(r)
-      : "r"((uint32_t)v), "r"(id), "r"(n)
-      : "memory");
-  return r != 0;
-}
 
 __device__ __forceinline__ void st_shared_v4(uint32_t addr, uint32_t a, uint32_t b, uint32_t c, uint32_t d) {
   asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(a), "r"(b), "r"(c), "r"(d) : "memory");
@@ -318,7 +308,7 @@ k_moe_gemm(const __grid_constant__ CUtensorMap tmap_h, const __grid_constant__ C
       mbar_init(&bars.empty[s], 1);
     }
     for (int q = 0; q < kProdGroups * kMaxRawSlots; ++q)
-      mbar_init(&bars.raw[q / kMaxRawSlots][q % kMaxRawSlots], kBN / kSubRows);   // one arrival per box
+      mbar_init(&bars.raw[q / kMaxRawSlots][q % kMaxRawSlots], kRawBoxes);   // one arrival per box
     for (int b = 0; b < 2; ++b) {
       mbar_init(&bars.acc_full[b], 1);
       mbar_init(&bars.acc_empty[b], kEpiWarps * 32);
@@ -344,15 +334,14 @@ k_moe_gemm(const __grid_constant__ CUtensorMap tmap_h, const __grid_constant__ C
     //    B tile row j * 128 + 32 r + i, where (gate_up) j = wg / 4 is gate (0) or up (1), both
     //    blocks of the K step; (down) j = 0 and the thread decodes block h = wg / 4 only;
     //    r = wg % 4 in both;
-    //  raw: the group has a ring of kRawSlots slots of its own; warp wg < nsub issues box wg of
-    //    a step kRawSlots local steps ahead, once the whole group has read the slot.
-    // Every decision to stop is taken by the whole group at its named barrier (all bounded
-    // waits come before it), so no thread is left waiting there.
+    //  raw: the group has a ring of kRawSlots slots of its own; warp wg alone reads box wg of a
+    //    slot, and refills it (for the step kRawSlots local steps ahead) once its lanes have
+    //    used the bytes they read. The warps of a group share no other wait.
     const int pq = threadIdx.x - (kMmaWarp + 1) * 32;
     const int pg = pq / kGroupThreads, pt = pq - pg * kGroupThreads;   // pt 0..255
     const int wg = pt >> 5, res = wg & 3, jh = wg >> 2;
     const int cb = pt & 7;                                              // A chunk
-    constexpr int nsub = kBN / kSubRows;                                // raw boxes per step
+    constexpr uint32_t kSubBytes = C::kSubBytes;
     constexpr int kRawSlots = C::kRawSlots;
     constexpr uint32_t kRawSlotBytes = C::kRawSlotBytes;
     const uint32_t raw_base = sbase + (uint32_t)kStages * kStageBytes + (uint32_t)pg * kRawSlots * kRawSlotBytes;
@@ -421,15 +410,16 @@ k_moe_gemm(const __grid_constant__ CUtensorMap tmap_h, const __grid_constant__ C
         if (rs.h1) tma_load_2d(a_saddr + kTileBytes, &tmap_h, ks * BK, rs.tile * BM + BM, &bars.full[s]);
       }
     };
-    // raw boxes of step (line0, ks) into ring slot q: box wg (residue r = wg % 4 of part wg / 4)
-    // starts at the K step's window rounded down to 16 bytes
+    // this warp's raw box of step (line0, ks) into ring slot q (lane 0): residue r = wg % 4;
+    // it starts at the K step's window rounded down to 16 bytes (gate_up: of part wg / 4;
+    // down: plus 16 bytes for block 1)
     auto issue_raw = [&](int line0, int ks, int q) {
-      if (lane == 0 && wg < nsub) {
-        const int r = wg & 3, j = wg >> 2;
-        const uint32_t xb = ((uint32_t)r * (uint32_t)rb + (uint32_t)ks * 2u * MOE_QBYTES) & ~15u;
+      if (lane == 0) {
+        const uint32_t xb = (((uint32_t)res * (uint32_t)rb + (uint32_t)ks * 2u * MOE_QBYTES) & ~15u) +
+                            (GATEUP ? 0u : 16u * (uint32_t)jh);
         mbar_arrive_expect_tx(&bars.raw[pg][q], kSubBytes);
         tma_load_2d(raw_base + (uint32_t)q * kRawSlotBytes + (uint32_t)wg * kSubBytes, &tmap_w, (int)xb,
-                    line0 + j * (f >> 2), &bars.raw[pg][q]);
+                    line0 + (GATEUP ? jh * (f >> 2) : 0), &bars.raw[pg][q]);
       }
     };
     bool ok = true;
@@ -458,27 +448,40 @@ k_moe_gemm(const __grid_constant__ CUtensorMap tmap_h, const __grid_constant__ C
       if (step(ijj, iks)) isrc = item_src(ijj);
       cp_async_commit();
     }
-    // this thread's B row in the tile and its raw window in a ring slot
+    // this thread's B row in the tile and its raw window in a ring slot (box wg, line lane)
     const int brow = (GATEUP ? jh * 128 : 0) + res * 32 + lane;
-    const uint32_t win_off = (uint32_t)((GATEUP ? jh * 4 : 0) + res) * kSubBytes + (uint32_t)lane * kWinBytes;
+    const uint32_t win_off = (uint32_t)wg * kSubBytes + (uint32_t)lane * C::kBoxW;
     int li = 0;
     for (; li < n_local; ++li) {
       const int g = pg + kProdGroups * li;
       const int s = g % kStages, q = li % kRawSlots;
       // step g: its A copies (this thread's, issued kAhead steps ago) and its raw boxes have landed
       cp_async_wait<kAhead - 1>();
-      if (!mbar_wait(&bars.raw[pg][q], (uint32_t)(li / kRawSlots) & 1u, W.err, 14, W.wait_ns)) ok = false;
+      if (!__all_sync(0xffffffffu, mbar_wait(&bars.raw[pg][q], (uint32_t)(li / kRawSlots) & 1u, W.err, 14,
+                                             W.wait_ns)))
+        ok = false;
       const uint32_t rowbase = sbase + (uint32_t)s * kStageBytes + kBOff + (uint32_t)brow * 128u;
       const uint32_t x = (uint32_t)(brow & 7);
       if (ok && csrc.wvalid) {
         const uint4 *wp = reinterpret_cast<const uint4 *>(smem_raw + (raw_base - smem_u32(smem_raw)) +
                                                           (size_t)q * kRawSlotBytes + win_off);
-        const uint4 v0 = wp[0], v1 = wp[1], v2 = wp[2];
-        const uint32_t w[12] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w, v2.x, v2.y, v2.z, v2.w};
         const int wb = (int)((((uint32_t)res * (uint32_t)rb + (uint32_t)cks * 2u * MOE_QBYTES) & 15u) >> 2);
-        if (GATEUP) dec_window_at<3>(wb, w, rowbase, x);
-        else if (jh == 0) dec_window_at<1>(wb, w, rowbase, x);
-        else dec_window_at<2>(wb, w, rowbase, x);
+        if (GATEUP) {
+          const uint4 v0 = wp[0], v1 = wp[1], v2 = wp[2];
+          const uint32_t w[12] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w, v2.x, v2.y, v2.z, v2.w};
+          dec_window_at<3>(wb, w, rowbase, x);
+        } else {
+          // the 32-byte box is window bytes 0-31 (block 0) or 16-47 (block 1): placed at its
+          // words of the 48-byte window
+          const uint4 v0 = wp[0], v1 = wp[1];
+          if (jh == 0) {
+            const uint32_t w[12] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w, 0u, 0u, 0u, 0u};
+            dec_window_at<1>(wb, w, rowbase, x);
+          } else {
+            const uint32_t w[12] = {0u, 0u, 0u, 0u, v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
+            dec_window_at<2>(wb, w, rowbase, x);
+          }
+        }
       } else {
         store_blk_zero(rowbase, x, 0);
         store_blk_zero(rowbase, x, 4);
@@ -486,11 +489,11 @@ k_moe_gemm(const __grid_constant__ CUtensorMap tmap_h, const __grid_constant__ C
       fence_proxy_async_smem();
       __syncwarp();
       if (lane == 0) mbar_arrive(&bars.full[s]);
-      // Slot q is refilled by TMA (the async proxy) only after the group's barrier, and only
-      // once every thread has used the bytes it read from the slot (the decode's stores depend
-      // on them): a shared-memory load still in flight at a barrier is not ordered before a
-      // later TMA write. The barrier is also where the group agrees on going on.
-      if (!named_bar_and(1 + pg, kGroupThreads, ok)) break;
+      if (!ok) break;   // warp-uniform
+      // The warp's box of slot q is refilled by TMA (the async proxy) only once every lane has
+      // used the bytes it read from it (the decode's stores depend on them, and the stores come
+      // before the __syncwarp): a shared-memory load still in flight is not ordered before a
+      // later TMA write by a barrier alone.
       if (li + kRawSlots < n_local) {
         issue_raw(rline, rks, q);
         ++raw_issued;
@@ -501,11 +504,11 @@ k_moe_gemm(const __grid_constant__ CUtensorMap tmap_h, const __grid_constant__ C
       if (li + kAhead < n_local) {
         const int gi = g + kProdGroups * kAhead, si = gi % kStages;
         const uint32_t par = ((uint32_t)(gi / kStages) & 1u) ^ 1u;
-        if (mbar_wait(&bars.empty[si], par, W.err, 10, W.wait_ns)) {
+        if (__all_sync(0xffffffffu, mbar_wait(&bars.empty[si], par, W.err, 10, W.wait_ns))) {
           issue_a(isrc, iks, si);
           if (step(ijj, iks)) isrc = item_src(ijj);
         } else {
-          ok = false;   // the group stops at its next barrier
+          ok = false;   // the warp stops at its next step
         }
       }
       cp_async_commit();
@@ -717,14 +720,14 @@ static bool make_tmap_h(CUtensorMap *m, const void *base, int cols, long long ro
 }
 
 // Tensor map of a Q4_0 weight matrix of `rows` rows of rb bytes (rows a multiple of 4, 4 rb a
-// multiple of 16) seen as rows / 4 lines of 4 rb bytes: boxes of 48 bytes x 32 lines, no
+// multiple of 16) seen as rows / 4 lines of 4 rb bytes: boxes of box_w bytes x 32 lines, no
 // swizzle; bytes past a line's end or past the last line read as zeros.
-static bool make_tmap_w(CUtensorMap *m, const void *base, int rb, long long rows) {
+static bool make_tmap_w(CUtensorMap *m, const void *base, int rb, long long rows, uint32_t box_w) {
   auto enc = get_encode();
   if (!enc || rows % 4 || (4 * rb) % 16) return false;
   cuuint64_t dims[2] = {(cuuint64_t)(4 * rb), (cuuint64_t)(rows / 4)};
   cuuint64_t strides[1] = {(cuuint64_t)(4 * rb)};
-  cuuint32_t box[2] = {kWinBytes, (cuuint32_t)kSubRows};
+  cuuint32_t box[2] = {box_w, (cuuint32_t)kSubRows};
   cuuint32_t estr[2] = {1, 1};
   CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void *>(base), dims, strides, box, estr,
                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
@@ -744,8 +747,8 @@ int moe_launch_gemm_experts(const MoeLaunch &L, const MoeWork &W, const void *x,
   moe_prof_mark(L.stream, MOE_K_GEMM_GATEUP, true);
   CUtensorMap th, twg, twd;
   if (!make_tmap_h(&th, W.hb, f, (long long)max_tiles * BM)) return -1;
-  if (!make_tmap_w(&twg, gate_up_q4, (d / MOE_QK) * MOE_QBYTES, (long long)E * 2 * f) ||
-      !make_tmap_w(&twd, down_q4, (f / MOE_QK) * MOE_QBYTES, (long long)E * d))
+  if (!make_tmap_w(&twg, gate_up_q4, (d / MOE_QK) * MOE_QBYTES, (long long)E * 2 * f, GemmCfg<true>::kBoxW) ||
+      !make_tmap_w(&twd, down_q4, (f / MOE_QK) * MOE_QBYTES, (long long)E * d, GemmCfg<false>::kBoxW))
     return -1;
   constexpr int kSmemG = GemmCfg<true>::kSmemBytes, kSmemD = GemmCfg<false>::kSmemBytes;
   k_moe_gemm<true><<<num_sms, kThreads, kSmemG, L.stream>>>(th, twg, static_cast<const __nv_bfloat16 *>(x),
