@@ -115,8 +115,7 @@ __device__ bool grid_wait(const unsigned long long *ctr, unsigned long long targ
       }
     }
   }
-  __threadfence();
-  return ok;
+  return ok;   // the acquire load that saw the target orders this thread's later reads
 }
 __device__ __forceinline__ void named_arrive(int id, int n) {
   asm volatile("bar.arrive %0, %1;" ::"r"(id), "r"(n) : "memory");
