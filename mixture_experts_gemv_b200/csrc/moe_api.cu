@@ -75,7 +75,7 @@ int cuda_fail(cudaError_t e, const char *what) {
 constexpr int kTileM = MOE_GEMM_TILE_ROWS;   // rows per grouped-GEMM tile
 
 struct Layout {
-  size_t off[24];
+  size_t off[25];
   size_t total;
 };
 
@@ -114,6 +114,7 @@ Layout make_layout(int maxT, int max_d, int max_f, int max_E, int max_k) {
       (size_t)max_E * 4,                 // 21 toff
       64,                                // 22 grid-barrier counter
       (size_t)max_d * 4 + 16,            // 23 dense MLP pass: zero router row, then 1.0f
+      (size_t)3 * 128 * max_d * 2,       // 24 the router weights as three bf16 planes (prefill)
   };
   Layout L{};
   size_t o = 0;
@@ -372,6 +373,7 @@ int moe_init(int device, int max_tokens, int max_d, int max_f, int max_E, int ma
   W.tiles = reinterpret_cast<int32_t *>(b + Lt.off[16]);
   W.toff = reinterpret_cast<int32_t *>(b + Lt.off[21]);
   W.gbar = reinterpret_cast<unsigned long long *>(b + Lt.off[22]);
+  W.wsplit = reinterpret_cast<__nv_bfloat16 *>(b + Lt.off[24]);
   W.err = ed;
   W.wait_ns = MOE_WAIT_NS;
   W.inject = MOE_INJECT_NONE;

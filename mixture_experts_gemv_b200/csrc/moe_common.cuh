@@ -64,6 +64,7 @@ struct MoeWork {
   int32_t *n_tiles;   // [1]
   int32_t *pairs;     // [n_pairs][2]: first tile of up to two consecutive tiles of one expert, second present
   int32_t *n_pairs;   // [1]
+  __nv_bfloat16 *wsplit;   // [3][128][d] the router weights as three bf16 planes (prefill router)
   unsigned long long wait_ns;   // bound on every device-side wait of this launch
   int inject;         // test-only fault (MOE_INJECT_*), 0 in normal operation
 };
@@ -252,6 +253,13 @@ int moe_launch_route_decode(const MoeLaunch &L, const MoeWork &W, const void *x,
                             const float *router_scale, int T, int d, int E, int k, int num_sms);
 // Bytes of the ybuf slot the prefill routing uses as scratch (range partials of the router
 // product, then per-CTA expert counts of the permutation).
+// the prefill router's d splits (partials kept in the route scratch, added in split order)
+#define MOE_ROUTER_MAX_SPLIT 9
+// the prefill router on the tensor cores (W_r as three exact bf16 planes in W.wsplit): E <= 128,
+// d a multiple of 64; writes part[nsplit][T][E] and sets *nsplit; -2 when not supported
+bool moe_router_tc_supported(int d, int E);
+int moe_launch_router_tc(const MoeLaunch &L, const MoeWork &W, const void *x, const float *router_w, int T, int d,
+                         int E, int num_sms, float *part, int *nsplit);
 size_t moe_route_scratch_bytes(int max_tokens, int max_E, int max_k);
 int moe_launch_route_prefill(const MoeLaunch &L, const MoeWork &W, const void *x, const float *router_w,
                              const float *router_scale, int T, int d, int E, int k, int num_sms,

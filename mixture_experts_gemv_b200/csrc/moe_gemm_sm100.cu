@@ -687,6 +687,138 @@ __global__ void __launch_bounds__(256) k_combine(const __nv_bfloat16 *__restrict
   }
 }
 
+// ---------------------------------------------------------------- router on the tensor cores
+//
+// The prefill router product logits[t, e] = sum_i x[t, i] W_r[e, i] (x bf16, W_r FP32) as a
+// bf16 tensor-core GEMM with no loss: W_r = hi + mid + lo, three bf16 planes (each rounds
+// what the planes before it left: 24 significand bits in three of 8), exact for |w| >= 2^-110
+// and within 2^-133 below that (bf16's subnormal step); every product of a bf16 x with a bf16
+// plane is exact, and the three products of a term accumulate in FP32 in the same accumulator. d is split over CTAs (the partials are added in split order by the
+// top-k kernel, as for the FP32 SIMT router).
+
+// wsplit [3][128][d]: planes hi, mid, lo of W_r, rows E..127 zero.
+__global__ void __launch_bounds__(256) k_split_router(const float *__restrict__ w, int E, int d,
+                                                      __nv_bfloat16 *__restrict__ ws) {
+  const long long n = 128LL * d;
+  for (long long i = blockIdx.x * (long long)blockDim.x + threadIdx.x; i < n; i += (long long)gridDim.x * blockDim.x) {
+    const float v = i < (long long)E * d ? __ldg(w + i) : 0.f;
+    const __nv_bfloat16 hi = __float2bfloat16_rn(v);
+    const float r1 = v - __bfloat162float(hi);    // exact: v and hi are within a factor of two
+    const __nv_bfloat16 mid = __float2bfloat16_rn(r1);
+    const float r2 = r1 - __bfloat162float(mid);  // exact, and at most 8 significant bits
+    ws[i] = hi;
+    ws[n + i] = mid;
+    ws[2 * n + i] = __float2bfloat16_rn(r2);
+  }
+}
+
+constexpr int kRtStages = 3;
+constexpr uint32_t kRtA = BM * BK * 2;           // 16 KB: 128 tokens x 64 of d
+constexpr uint32_t kRtB = 128 * BK * 2;          // 16 KB: one plane, 128 experts x 64 of d
+constexpr uint32_t kRtStage = kRtA + 3 * kRtB;   // 64 KB
+constexpr int kRtSmem = kRtStages * (int)kRtStage + 1024;
+constexpr uint32_t kRtIdesc = umma_idesc(128);   // M = 128, N = 128
+constexpr int kRtSplit = 4;                        // d splits (<= MOE_ROUTER_MAX_SPLIT)
+static_assert(kRtSplit <= MOE_ROUTER_MAX_SPLIT, "the route scratch holds that many partials");
+
+struct RtBars {
+  uint64_t full[kRtStages];
+  uint64_t empty[kRtStages];
+  uint64_t acc;
+  uint32_t tmem_base;
+};
+
+// CTA (m, s): tokens 128 m .. 128 m + 127, K steps [s nk / S, (s + 1) nk / S) of the nk = d / 64;
+// 4 warps: warp 0 lane 0 issues the TMA copies (x tile and the three plane tiles of a K step
+// into one stage), warp 1 holds the TMEM accumulator (128 columns) and its lane 0 issues
+// tcgen05.mma (M = 128, N = 128, K = 16; per K step 4 x 3, all into one accumulator); then every
+// warp reads its 32 rows (lane = token) and writes part[s][t][e] for e < E.
+__global__ void __launch_bounds__(128, 1)
+k_router_tc(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ CUtensorMap tmap_w, int T, int d,
+            int E, int nsplit, float *__restrict__ part, MoeWork W) {
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  __shared__ RtBars bars;
+  const uint32_t sbase = (smem_u32(smem_raw) + 1023u) & ~1023u;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int t0 = blockIdx.x * BM, split = blockIdx.y;
+  const int nk = d / BK;
+  const int k0 = (int)((long long)nk * split / nsplit), k1 = (int)((long long)nk * (split + 1) / nsplit);
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kRtStages; ++s) {
+      mbar_init(&bars.full[s], 1);
+      mbar_init(&bars.empty[s], 1);
+    }
+    mbar_init(&bars.acc, 1);
+    fence_mbar_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(&bars.tmem_base, 128);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = bars.tmem_base;
+  if (warp == 0 && lane == 0) {
+    for (int ks = k0, i = 0; ks < k1; ++ks, ++i) {
+      const int s = i % kRtStages;
+      if (i >= kRtStages &&
+          !mbar_wait(&bars.empty[s], (uint32_t)(i / kRtStages - 1) & 1u, W.err, 16, W.wait_ns))
+        break;
+      const uint32_t st = sbase + (uint32_t)s * kRtStage;
+      mbar_arrive_expect_tx(&bars.full[s], kRtStage);
+      tma_load_2d(st, &tmap_x, ks * BK, t0, &bars.full[s]);
+#pragma unroll
+      for (int j = 0; j < 3; ++j) tma_load_2d(st + kRtA + (uint32_t)j * kRtB, &tmap_w, ks * BK, j * 128, &bars.full[s]);
+    }
+  } else if (warp == 1 && lane == 0) {
+    for (int ks = k0, i = 0; ks < k1; ++ks, ++i) {
+      const int s = i % kRtStages;
+      if (!mbar_wait(&bars.full[s], (uint32_t)(i / kRtStages) & 1u, W.err, 17, W.wait_ns)) break;
+      tc_fence_after();
+      const uint32_t st = sbase + (uint32_t)s * kRtStage;
+#pragma unroll
+      for (int kk = 0; kk < BK / 16; ++kk)
+#pragma unroll
+        for (int j = 0; j < 3; ++j)
+          umma_bf16(tmem, sw128_desc(st + (uint32_t)kk * 32u), sw128_desc(st + kRtA + (uint32_t)j * kRtB + (uint32_t)kk * 32u),
+                    kRtIdesc, (i > 0 || kk > 0 || j > 0) ? 1u : 0u);
+      umma_commit(&bars.empty[s]);
+    }
+    umma_commit(&bars.acc);   // arrives once every MMA issued above has completed
+  }
+  __syncwarp();
+  const bool ok = mbar_wait(&bars.acc, 0u, W.err, 18, W.wait_ns);
+  if (__all_sync(0xffffffffu, ok)) {
+    tc_fence_after();
+    const int t = t0 + warp * 32 + lane;
+    float *dst = part + ((size_t)split * T + (size_t)(t < T ? t : 0)) * E;
+    const bool vec = (E & 3) == 0;   // 16-byte stores when every row starts 16-byte aligned
+#pragma unroll
+    for (int c = 0; c < 128; c += 4) {
+      uint32_t v[4];
+      tmem_ld4(tmem + ((uint32_t)(warp * 32) << 16) + (uint32_t)c, v);
+      tmem_ld_wait();
+      if (t < T && c < E) {
+        if (vec) {
+          *reinterpret_cast<float4 *>(dst + c) =
+              make_float4(__uint_as_float(v[0]), __uint_as_float(v[1]), __uint_as_float(v[2]), __uint_as_float(v[3]));
+        } else {
+#pragma unroll
+          for (int q = 0; q < 4; ++q)
+            if (c + q < E) dst[c + q] = __uint_as_float(v[q]);
+        }
+      }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 128);
+  }
+}
+
 }  // namespace
 
 static int launch_err() { return cudaGetLastError() == cudaSuccess ? 0 : -1; }
@@ -733,6 +865,33 @@ static bool make_tmap_w(CUtensorMap *m, const void *base, int rb, long long rows
                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS;
+}
+
+bool moe_router_tc_supported(int d, int E) { return E >= 1 && E <= 128 && d % BK == 0; }
+
+int moe_launch_router_tc(const MoeLaunch &L, const MoeWork &W, const void *x, const float *router_w, int T, int d,
+                         int E, int num_sms, float *part, int *nsplit) {
+  if (!moe_router_tc_supported(d, E) || W.wsplit == nullptr) return -2;
+  static unsigned long long smem_ok = 0ull;   // per device
+  if (!moe_allow_dyn_smem(reinterpret_cast<const void *>(k_router_tc), &smem_ok)) return -1;
+  // a fixed number of d splits, whatever T: a token's logits are then the same bits in a call
+  // of any size (a chunked call gives the bits of one pass); 32 row tiles x 4 splits = 128 CTAs
+  // at 4,096 tokens
+  const int nk = d / BK, mt = (T + BM - 1) / BM;
+  const int ns = kRtSplit < nk ? kRtSplit : nk;
+  (void)num_sms;
+  CUtensorMap tx, tw;
+  if (!make_tmap_h(&tx, x, d, T) || !make_tmap_h(&tw, W.wsplit, d, 3 * 128)) return -1;
+  int grid = (int)((128LL * d + 255) / 256);
+  if (grid > 2 * num_sms) grid = 2 * num_sms;
+  k_split_router<<<grid, 256, 0, L.stream>>>(router_w, E, d, W.wsplit);
+  if (launch_err()) return -1;
+  moe_prof_count(1);
+  k_router_tc<<<dim3(mt, ns), 128, kRtSmem, L.stream>>>(tx, tw, T, d, E, ns, part, W);
+  if (launch_err()) return -1;
+  moe_prof_count(1);
+  *nsplit = ns;
+  return 0;
 }
 
 int moe_launch_gemm_experts(const MoeLaunch &L, const MoeWork &W, const void *x, const uint8_t *gate_up_q4,

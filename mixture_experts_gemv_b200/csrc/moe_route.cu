@@ -226,7 +226,7 @@ k_route_decode(const __nv_bfloat16 *__restrict__ x, const float *__restrict__ ro
 // step's global loads are in flight during this step's FMAs), the d axis split in kRgSplit
 // ranges for parallelism (32 token tiles x 9 ranges = 288 CTAs, two per SM). Each output's
 // terms are summed in K order inside its range; k_topk adds the range partials in range order.
-constexpr int kRgM = 128, kRgN = 128, kRgK = 16, kRgSplit = 9;
+constexpr int kRgM = 128, kRgN = 128, kRgK = 16, kRgSplit = MOE_ROUTER_MAX_SPLIT;
 
 __global__ void __launch_bounds__(256)
 k_router_gemm(const __nv_bfloat16 *__restrict__ x, const float *__restrict__ router_w, int T, int d, int E,
@@ -315,18 +315,18 @@ k_router_gemm(const __nv_bfloat16 *__restrict__ x, const float *__restrict__ rou
   }
 }
 
-// logits = the kRgSplit range partials added in range order; then top-k + softmax per token
+// logits = the nsplit range partials added in range order; then top-k + softmax per token
 // (one warp per token).
 __global__ void __launch_bounds__(256)
 k_topk(const float *__restrict__ part, float *__restrict__ logits, const float *__restrict__ router_scale, int T,
-       int E, int k, int32_t *ids, float *w) {
+       int E, int k, int32_t *ids, float *w, int nsplit) {
   const int wid = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int t = blockIdx.x * 8 + wid;
   if (t >= T) return;
   for (int e = lane; e < E; e += 32) {
     float v = part[(size_t)t * E + e];
 #pragma unroll
-    for (int sp = 1; sp < kRgSplit; ++sp) v += part[((size_t)sp * T + t) * E + e];
+    for (int sp = 1; sp < nsplit; ++sp) v += part[((size_t)sp * T + t) * E + e];
     logits[(size_t)t * E + e] = v;
   }
   __syncwarp();
@@ -527,11 +527,19 @@ int moe_launch_route_prefill(const MoeLaunch &L, const MoeWork &W, const void *x
   const int S = T * k;
   const int nc = (S + kPermSlots - 1) / kPermSlots;
   int32_t *ccnt = reinterpret_cast<int32_t *>(W.ybuf + (size_t)kRgSplit * T * E);
-  dim3 g1((T + kRgM - 1) / kRgM, (E + kRgN - 1) / kRgN, kRgSplit);
   moe_prof_mark(L.stream, MOE_K_ROUTE, true);
-  k_router_gemm<<<g1, 256, 0, L.stream>>>(xb, router_w, T, d, E, part);
-  if (launch_err()) return -1;
-  k_topk<<<(T + 7) / 8, 256, 0, L.stream>>>(part, W.logits, router_scale, T, E, k, W.ids, W.w);
+  // the router product on the tensor cores where the shape allows, else in FP32 on the CUDA cores
+  int nsplit = kRgSplit;
+  const int rc = moe_launch_router_tc(L, W, x, router_w, T, d, E, num_sms, part, &nsplit);
+  if (rc == -2) {
+    dim3 g1((T + kRgM - 1) / kRgM, (E + kRgN - 1) / kRgN, kRgSplit);
+    k_router_gemm<<<g1, 256, 0, L.stream>>>(xb, router_w, T, d, E, part);
+    if (launch_err()) return -1;
+    moe_prof_count(1);
+  } else if (rc) {
+    return -1;
+  }
+  k_topk<<<(T + 7) / 8, 256, 0, L.stream>>>(part, W.logits, router_scale, T, E, k, W.ids, W.w, nsplit);
   if (launch_err()) return -1;
   k_perm_count<<<nc, kRouteThreads, 0, L.stream>>>(W.ids, S, E, ccnt);
   if (launch_err()) return -1;
@@ -539,7 +547,7 @@ int moe_launch_route_prefill(const MoeLaunch &L, const MoeWork &W, const void *x
   if (launch_err()) return -1;
   k_perm_place<<<nc, kRouteThreads, 0, L.stream>>>(S, E, ccnt, W);
   if (launch_err()) return -1;
-  moe_prof_count(5);   // router product, top-k, count, scan, place
+  moe_prof_count(4);   // top-k, count, scan, place
   if (want_xprep) {
     const int nb = d / MOE_QK;
     const int items = T * nb;
