@@ -174,9 +174,15 @@ __device__ __forceinline__ void st_shared_v4(uint32_t addr, uint32_t a, uint32_t
   asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(a), "r"(b), "r"(c), "r"(d) : "memory");
 }
 
+// GELU, tanh form, with the hardware tanh approximation (`tanh.approx.f32`, absolute error
+// about 2^-11): h is rounded to bf16 right after (relative step 2^-8), and this path's outputs
+// are held to 2e-2 of the oracle; it frees the epilogue's issue slots for the producer warps
+// that share the SM's schedulers.
 __device__ __forceinline__ float gelu_tanh_f(float z) {
   const float c = 0.7978845608028654f;   // sqrt(2/pi)
-  return 0.5f * z * (1.0f + tanhf(c * (z + 0.044715f * z * z * z)));
+  float t;
+  asm("tanh.approx.f32 %0, %1;" : "=f"(t) : "f"(c * (z + 0.044715f * z * z * z)));
+  return 0.5f * z * (1.0f + t);
 }
 
 __device__ __forceinline__ uint32_t pack_bf16(float a, float b) {
