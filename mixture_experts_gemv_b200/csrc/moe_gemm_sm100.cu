@@ -702,19 +702,28 @@ __global__ void __launch_bounds__(256) k_combine(const __nv_bfloat16 *__restrict
 // plane is exact, and the three products of a term accumulate in FP32 in the same accumulator. d is split over CTAs (the partials are added in split order by the
 // top-k kernel, as for the FP32 SIMT router).
 
-// wsplit [3][128][d]: planes hi, mid, lo of W_r, rows E..127 zero.
+// wsplit [3][128][d]: planes hi, mid, lo of W_r, rows E..127 zero. Four weights a thread
+// (d is a multiple of 4, so a group never straddles rows; 16-byte loads, 8-byte stores).
 __global__ void __launch_bounds__(256) k_split_router(const float *__restrict__ w, int E, int d,
                                                       __nv_bfloat16 *__restrict__ ws) {
-  const long long n = 128LL * d;
-  for (long long i = blockIdx.x * (long long)blockDim.x + threadIdx.x; i < n; i += (long long)gridDim.x * blockDim.x) {
-    const float v = i < (long long)E * d ? __ldg(w + i) : 0.f;
-    const __nv_bfloat16 hi = __float2bfloat16_rn(v);
-    const float r1 = v - __bfloat162float(hi);    // exact: v and hi are within a factor of two
-    const __nv_bfloat16 mid = __float2bfloat16_rn(r1);
-    const float r2 = r1 - __bfloat162float(mid);  // exact, and at most 8 significant bits
-    ws[i] = hi;
-    ws[n + i] = mid;
-    ws[2 * n + i] = __float2bfloat16_rn(r2);
+  const long long n = 128LL * d, ng = n / 4, nw = (long long)E * d;
+  for (long long g = blockIdx.x * (long long)blockDim.x + threadIdx.x; g < ng; g += (long long)gridDim.x * blockDim.x) {
+    const long long i = 4 * g;
+    const float4 v4 = i < nw ? __ldg(reinterpret_cast<const float4 *>(w + i)) : make_float4(0.f, 0.f, 0.f, 0.f);
+    const float v[4] = {v4.x, v4.y, v4.z, v4.w};
+    __nv_bfloat16 p[3][4];
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      const __nv_bfloat16 hi = __float2bfloat16_rn(v[q]);
+      const float r1 = v[q] - __bfloat162float(hi);    // exact: v and hi are within a factor of two
+      const __nv_bfloat16 mid = __float2bfloat16_rn(r1);
+      const float r2 = r1 - __bfloat162float(mid);     // exact, and at most 8 significant bits
+      p[0][q] = hi;
+      p[1][q] = mid;
+      p[2][q] = __float2bfloat16_rn(r2);
+    }
+#pragma unroll
+    for (int j = 0; j < 3; ++j) *reinterpret_cast<uint2 *>(ws + (size_t)j * n + i) = *reinterpret_cast<const uint2 *>(p[j]);
   }
 }
 
@@ -874,6 +883,7 @@ static bool make_tmap_w(CUtensorMap *m, const void *base, int rb, long long rows
 }
 
 bool moe_router_tc_supported(int d, int E) { return E >= 1 && E <= 128 && d % BK == 0; }
+// (router_w must be 16-byte aligned for the split's 16-byte loads: the layer's entry points check it)
 
 int moe_launch_router_tc(const MoeLaunch &L, const MoeWork &W, const void *x, const float *router_w, int T, int d,
                          int E, int num_sms, float *part, int *nsplit) {
@@ -888,8 +898,8 @@ int moe_launch_router_tc(const MoeLaunch &L, const MoeWork &W, const void *x, co
   (void)num_sms;
   CUtensorMap tx, tw;
   if (!make_tmap_h(&tx, x, d, T) || !make_tmap_h(&tw, W.wsplit, d, 3 * 128)) return -1;
-  int grid = (int)((128LL * d + 255) / 256);
-  if (grid > 2 * num_sms) grid = 2 * num_sms;
+  int grid = (int)((32LL * d + 255) / 256);   // 128 d / 4 groups
+  if (grid > 4 * num_sms) grid = 4 * num_sms;
   k_split_router<<<grid, 256, 0, L.stream>>>(router_w, E, d, W.wsplit);
   if (launch_err()) return -1;
   moe_prof_count(1);

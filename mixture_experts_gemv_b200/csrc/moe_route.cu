@@ -323,6 +323,31 @@ k_topk(const float *__restrict__ part, float *__restrict__ logits, const float *
   const int wid = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int t = blockIdx.x * 8 + wid;
   if (t >= T) return;
+  if (E <= 128 && k <= 8) {
+    // every partial load of the lane's four logits in flight at once; the sums stay in
+    // registers for the selection (the same additions, in split order, as below)
+    float v[4][MOE_ROUTER_MAX_SPLIT];
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+#pragma unroll
+      for (int sp = 0; sp < MOE_ROUTER_MAX_SPLIT; ++sp) {
+        const int e = lane + 32 * i;
+        v[i][sp] = (e < E && sp < nsplit) ? __ldg(part + ((size_t)sp * T + t) * E + e) : 0.f;
+      }
+    uint32_t o[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const int e = lane + 32 * i;
+      float s = v[i][0];
+#pragma unroll
+      for (int sp = 1; sp < MOE_ROUTER_MAX_SPLIT; ++sp)
+        if (sp < nsplit) s += v[i][sp];
+      if (e < E) logits[(size_t)t * E + e] = s;
+      o[i] = e < E ? logit_ord(s) : 0u;
+    }
+    warp_top8_softmax_keys<4>(o, k, *router_scale, ids + (size_t)t * k, w + (size_t)t * k);
+    return;
+  }
   for (int e = lane; e < E; e += 32) {
     float v = part[(size_t)t * E + e];
 #pragma unroll

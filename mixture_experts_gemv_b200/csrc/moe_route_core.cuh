@@ -138,15 +138,11 @@ __device__ __forceinline__ float logit_from_ord(uint32_t o) {
 // largest logit, then, among the lanes holding it, the lowest expert index. A lane keeps its
 // kMaxPer logits (experts lane + 32 i) and clears the one picked. Picks come out in the
 // order (logit descending, index ascending), the same picks as a sort of the 64-bit keys.
+// The selection and softmax of warp_top8_softmax_t from the lane's order keys o[i] of logits
+// lane + 32 i (0 past E).
 template <int kMaxPer>
-__device__ void warp_top8_softmax_t(const float *lg, int E, int k, float rscale, int32_t *ids, float *w) {
+__device__ void warp_top8_softmax_keys(uint32_t (&o)[kMaxPer], int k, float rscale, int32_t *ids, float *w) {
   const int lane = threadIdx.x & 31;
-  uint32_t o[kMaxPer];
-#pragma unroll
-  for (int i = 0; i < kMaxPer; ++i) {
-    const int e = lane + 32 * i;
-    o[i] = (e < E) ? logit_ord(__ldcg(lg + e)) : 0u;
-  }
   uint32_t pick_o[8];
   int pick_e[8];
 #pragma unroll
@@ -187,6 +183,18 @@ __device__ void warp_top8_softmax_t(const float *lg, int E, int k, float rscale,
     w[lane] = mine_v * (rscale / part);
   }
   __syncwarp();
+}
+
+template <int kMaxPer>
+__device__ void warp_top8_softmax_t(const float *lg, int E, int k, float rscale, int32_t *ids, float *w) {
+  const int lane = threadIdx.x & 31;
+  uint32_t o[kMaxPer];
+#pragma unroll
+  for (int i = 0; i < kMaxPer; ++i) {
+    const int e = lane + 32 * i;
+    o[i] = (e < E) ? logit_ord(__ldcg(lg + e)) : 0u;
+  }
+  warp_top8_softmax_keys<kMaxPer>(o, k, rscale, ids, w);
 }
 
 // E <= 32 * kMaxPer logits per lane-strided register file.

@@ -91,6 +91,7 @@ SMALL_GEMM = [  # (E, k, T, d, f): d % 128 == 0, f % 64 == 0
     (8, 2, 33, 256, 64), (4, 4, 130, 128, 128), (128, 8, 300, 512, 128), (16, 4, 257, 2816, 704),
     (128, 2, 17, 256, 64), (3, 3, 40, 384, 192),
     (2, 2, 600, 256, 64),   # 600 rows per expert: five tiles, two tile pairs and a ragged single
+    (256, 8, 200, 256, 64), (200, 4, 150, 512, 128),   # E > 128: the router on the CUDA cores (FP32)
 ]
 
 
