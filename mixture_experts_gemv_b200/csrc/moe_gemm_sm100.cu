@@ -68,13 +68,17 @@ constexpr uint32_t umma_idesc(int n) {
 //    twice the work of an N = 128 one in about the same pipeline time. A rows are gathered by
 //    the producers.
 //  down: an item is up to two consecutive tiles of one expert, M = 256 as two 128-row halves
-//    that share the dequantised N = 128 B tile (A comes by TMA), so the decode work per MMA
-//    halves.
-template <bool GATEUP>
+//    that share the dequantised B tile (A comes by TMA), so the decode work per MMA halves.
+//    WIDE (d a multiple of 256): N = 256 output columns, one accumulator buffer (2 x 256 TMEM
+//    columns), one B row per producer thread as for gate_up; otherwise N = 128, two buffers,
+//    one block of a B row per thread.
+template <bool GATEUP, bool WIDE = false>
 struct GemmCfg {
-  static constexpr int kBN = GATEUP ? 256 : 128;                 // MMA N
+  static constexpr bool kRowDec = GATEUP || WIDE;                 // one B row (both blocks) a thread
+  static constexpr int kBN = kRowDec ? 256 : 128;                 // MMA N
   static constexpr int kHalves = GATEUP ? 1 : 2;
-  static constexpr int kStages = GATEUP ? 3 : 4;
+  static constexpr int kStages = GATEUP ? 3 : (WIDE ? 3 : 4);
+  static constexpr int kAccBufs = WIDE ? 1 : 2;                   // accumulator buffers in TMEM
   // group steps the copies run ahead of the decode
   static constexpr int kAhead = 1;
   static constexpr uint32_t kBBytes = (uint32_t)kBN * BK * 2;
@@ -83,17 +87,17 @@ struct GemmCfg {
   // raw box width: gate_up, a row's whole 48-byte window (box w = part w / 4, residue w % 4);
   // down, 32 bytes holding one block (box w = residue w % 4, block w / 4: bytes 0-31 of the
   // window hold block 0, bytes 16-47 block 1)
-  static constexpr uint32_t kBoxW = GATEUP ? 48 : 32;
+  static constexpr uint32_t kBoxW = kRowDec ? 48 : 32;
   static constexpr uint32_t kSubBytes = kSubRows * kBoxW;
   static constexpr uint32_t kRawSlotBytes = kRawBoxes * kSubBytes;
-  static constexpr int kRawSlots = GATEUP ? 3 : 2;                 // raw ring slots per producer group
-  static constexpr uint32_t kTmemCols = 2 * kHalves * kBN;       // two accumulator buffers
+  static constexpr int kRawSlots = GATEUP ? 3 : (WIDE ? 1 : 2);   // raw ring slots per producer group
+  static constexpr uint32_t kTmemCols = kAccBufs * kHalves * kBN;
   static constexpr int kSmemBytes = kStages * kStageBytes + kProdGroups * kRawSlots * kRawSlotBytes + 1024;
   static constexpr uint32_t kIdesc = umma_idesc(kBN);
   static_assert(kAhead * kProdGroups <= kStages, "the prologue's stages must be free");
   static_assert(kStages <= kMaxStages && kRawSlots <= kMaxRawSlots && kTmemCols <= 512, "limits");
   // the producer group's threads: one B row each (gate_up), or one block of a B row (down)
-  static_assert(kBN * (GATEUP ? 1 : 2) == kGroupThreads, "producer threads cover the B tile");
+  static_assert(kBN * (kRowDec ? 1 : 2) == kGroupThreads, "producer threads cover the B tile");
 };
 
 // Shared-memory matrix descriptor: K-major operand, 128-byte swizzle (layout type 2),
@@ -273,7 +277,7 @@ __device__ __forceinline__ void store_blk_zero(uint32_t rowbase, uint32_t x, int
 // DOWN:   A = hb [padded rows, f] (tmap_h: 2-D tiles of 128 rows x 64 columns by TMA), B =
 //         down rows n0..n0+127, K = f; epilogue y * w * s -> yslot (bf16, slot order).
 // tmap_w: the weight matrix (gate_up or down) as lines of 4 rows, boxes of 48 bytes x 32 lines.
-template <bool GATEUP>
+template <bool GATEUP, bool WIDE = false>
 __global__ void __launch_bounds__(kThreads, 1)
 k_moe_gemm(const __grid_constant__ CUtensorMap tmap_h, const __grid_constant__ CUtensorMap tmap_w,
            const __nv_bfloat16 *__restrict__ a_src, const float *__restrict__ expert_scale, int d, int f, int k,
@@ -285,7 +289,9 @@ k_moe_gemm(const __grid_constant__ CUtensorMap tmap_h, const __grid_constant__ C
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int K = GATEUP ? d : f;
   const int ksteps = K / BK;
-  using C = GemmCfg<GATEUP>;
+  using C = GemmCfg<GATEUP, WIDE>;
+  constexpr bool kRowDec = C::kRowDec;
+  constexpr int kAccBufs = C::kAccBufs;
   constexpr int kBN = C::kBN;
   const int n_ntiles = GATEUP ? (f + kBN / 2 - 1) / (kBN / 2) : d / kBN;
   const int rb = (K / MOE_QK) * MOE_QBYTES;            // bytes per weight row
@@ -422,10 +428,10 @@ k_moe_gemm(const __grid_constant__ CUtensorMap tmap_h, const __grid_constant__ C
     auto issue_raw = [&](int line0, int ks, int q) {
       if (lane == 0) {
         const uint32_t xb = (((uint32_t)res * (uint32_t)rb + (uint32_t)ks * 2u * MOE_QBYTES) & ~15u) +
-                            (GATEUP ? 0u : 16u * (uint32_t)jh);
+                            (kRowDec ? 0u : 16u * (uint32_t)jh);
         mbar_arrive_expect_tx(&bars.raw[pg][q], kSubBytes);
         tma_load_2d(raw_base + (uint32_t)q * kRawSlotBytes + (uint32_t)wg * kSubBytes, &tmap_w, (int)xb,
-                    line0 + (GATEUP ? jh * (f >> 2) : 0), &bars.raw[pg][q]);
+                    line0 + (GATEUP ? jh * (f >> 2) : (WIDE ? jh * 32 : 0)), &bars.raw[pg][q]);
       }
     };
     bool ok = true;
@@ -455,7 +461,7 @@ k_moe_gemm(const __grid_constant__ CUtensorMap tmap_h, const __grid_constant__ C
       cp_async_commit();
     }
     // this thread's B row in the tile and its raw window in a ring slot (box wg, line lane)
-    const int brow = (GATEUP ? jh * 128 : 0) + res * 32 + lane;
+    const int brow = (kRowDec ? jh * 128 : 0) + res * 32 + lane;
     const uint32_t win_off = (uint32_t)wg * kSubBytes + (uint32_t)lane * C::kBoxW;
     int li = 0;
     for (; li < n_local; ++li) {
@@ -472,7 +478,7 @@ k_moe_gemm(const __grid_constant__ CUtensorMap tmap_h, const __grid_constant__ C
         const uint4 *wp = reinterpret_cast<const uint4 *>(smem_raw + (raw_base - smem_u32(smem_raw)) +
                                                           (size_t)q * kRawSlotBytes + win_off);
         const int wb = (int)((((uint32_t)res * (uint32_t)rb + (uint32_t)cks * 2u * MOE_QBYTES) & 15u) >> 2);
-        if (GATEUP) {
+        if (kRowDec) {
           const uint4 v0 = wp[0], v1 = wp[1], v2 = wp[2];
           const uint32_t w[12] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w, v2.x, v2.y, v2.z, v2.w};
           dec_window_at<3>(wb, w, rowbase, x);
@@ -531,8 +537,8 @@ k_moe_gemm(const __grid_constant__ CUtensorMap tmap_h, const __grid_constant__ C
       int it = 0, j = 0;
       bool ok = true;
       for (int item = blockIdx.x; item < n_items && ok; item += gridDim.x, ++j) {
-        const int b = j & 1;
-        const uint32_t upar = ((uint32_t)(j >> 1) & 1u) ^ 1u;
+        const int b = kAccBufs == 2 ? (j & 1) : 0;
+        const uint32_t upar = ((uint32_t)(kAccBufs == 2 ? (j >> 1) : j) & 1u) ^ 1u;
         if (!mbar_wait(&bars.acc_empty[b], upar, W.err, 11, W.wait_ns)) { ok = false; break; }
         tc_fence_after();
         // the second half only where the item holds a second tile
@@ -567,8 +573,8 @@ k_moe_gemm(const __grid_constant__ CUtensorMap tmap_h, const __grid_constant__ C
     const int r = warp * 32 + lane;   // row inside a 128-row half == TMEM lane
     int j = 0;
     for (int item = blockIdx.x; item < n_items; item += gridDim.x, ++j) {
-      const int b = j & 1;
-      const uint32_t par = (uint32_t)(j >> 1) & 1u;
+      const int b = kAccBufs == 2 ? (j & 1) : 0;
+      const uint32_t par = (uint32_t)(kAccBufs == 2 ? (j >> 1) : j) & 1u;
       const bool ok = mbar_wait(&bars.acc_full[b], par, W.err, 13, W.wait_ns);
       if (__any_sync(0xffffffffu, !ok)) { atomicExch(&bars.abort_flag, 1); break; }
       tc_fence_after();
@@ -627,7 +633,8 @@ k_moe_gemm(const __grid_constant__ CUtensorMap tmap_h, const __grid_constant__ C
             const int c = 16 * u16;
             uint32_t y[4][4];
 #pragma unroll
-            for (int rr = 0; rr < 4; ++rr) tmem_ld4(taddr + (uint32_t)(32 * rr + 4 * u16), y[rr]);
+            for (int rr = 0; rr < 4; ++rr)   // part u16 / 8 of 128 columns, as in gate_up's parts
+              tmem_ld4(taddr + (uint32_t)(128 * (u16 >> 3) + 32 * rr + 4 * (u16 & 7)), y[rr]);
             tmem_ld_wait();
             uint32_t o[8];
 #pragma unroll
@@ -915,24 +922,32 @@ int moe_launch_gemm_experts(const MoeLaunch &L, const MoeWork &W, const void *x,
                             float *out, int num_sms, int max_tiles) {
   // K of both GEMMs in whole 64-wide steps; down's output in whole 128-column tiles
   if (d % BK || d % GemmCfg<false>::kBN || f % BK) return -2;
-  static unsigned long long smem_ok[2] = {0ull, 0ull};   // per device, per kernel
+  const bool wide = d % GemmCfg<false, true>::kBN == 0;   // down items of N = 256
+  static unsigned long long smem_ok[3] = {0ull, 0ull, 0ull};   // per device, per kernel
   if (!moe_allow_dyn_smem(reinterpret_cast<const void *>(k_moe_gemm<true>), &smem_ok[0]) ||
-      !moe_allow_dyn_smem(reinterpret_cast<const void *>(k_moe_gemm<false>), &smem_ok[1]))
+      !moe_allow_dyn_smem(wide ? reinterpret_cast<const void *>(k_moe_gemm<false, true>)
+                               : reinterpret_cast<const void *>(k_moe_gemm<false>),
+                          &smem_ok[wide ? 2 : 1]))
     return -1;
   moe_prof_mark(L.stream, MOE_K_GEMM_GATEUP, true);
   CUtensorMap th, twg, twd;
   if (!make_tmap_h(&th, W.hb, f, (long long)max_tiles * BM)) return -1;
   if (!make_tmap_w(&twg, gate_up_q4, (d / MOE_QK) * MOE_QBYTES, (long long)E * 2 * f, GemmCfg<true>::kBoxW) ||
-      !make_tmap_w(&twd, down_q4, (f / MOE_QK) * MOE_QBYTES, (long long)E * d, GemmCfg<false>::kBoxW))
+      !make_tmap_w(&twd, down_q4, (f / MOE_QK) * MOE_QBYTES, (long long)E * d,
+                   wide ? GemmCfg<false, true>::kBoxW : GemmCfg<false>::kBoxW))
     return -1;
-  constexpr int kSmemG = GemmCfg<true>::kSmemBytes, kSmemD = GemmCfg<false>::kSmemBytes;
+  constexpr int kSmemG = GemmCfg<true>::kSmemBytes, kSmemD = GemmCfg<false>::kSmemBytes,
+                kSmemDW = GemmCfg<false, true>::kSmemBytes;
   k_moe_gemm<true><<<num_sms, kThreads, kSmemG, L.stream>>>(th, twg, static_cast<const __nv_bfloat16 *>(x),
                                                             expert_scale, d, f, k, W);
   if (launch_err()) return -1;
   moe_prof_count(1);
   moe_prof_mark(L.stream, MOE_K_GEMM_GATEUP, false);
   moe_prof_mark(L.stream, MOE_K_GEMM_DOWN, true);
-  k_moe_gemm<false><<<num_sms, kThreads, kSmemD, L.stream>>>(th, twd, W.hb, expert_scale, d, f, k, W);
+  if (wide)
+    k_moe_gemm<false, true><<<num_sms, kThreads, kSmemDW, L.stream>>>(th, twd, W.hb, expert_scale, d, f, k, W);
+  else
+    k_moe_gemm<false><<<num_sms, kThreads, kSmemD, L.stream>>>(th, twd, W.hb, expert_scale, d, f, k, W);
   if (launch_err()) return -1;
   moe_prof_count(1);
   moe_prof_mark(L.stream, MOE_K_GEMM_DOWN, false);
