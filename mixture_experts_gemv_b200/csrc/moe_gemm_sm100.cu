@@ -76,7 +76,7 @@ template <bool GATEUP, bool WIDE = false>
 struct GemmCfg {
   static constexpr bool kRowDec = GATEUP || WIDE;                 // one B row (both blocks) a thread
   static constexpr int kBN = kRowDec ? 256 : 128;                 // MMA N
-  static constexpr int kHalves = GATEUP ? 1 : 2;
+  static constexpr int kHalves = (GATEUP && !WIDE) ? 1 : 2;      // M = 128 kHalves
   static constexpr int kStages = GATEUP ? 3 : (WIDE ? 3 : 4);
   static constexpr int kAccBufs = WIDE ? 1 : 2;                   // accumulator buffers in TMEM
   // group steps the copies run ahead of the decode
@@ -90,7 +90,7 @@ struct GemmCfg {
   static constexpr uint32_t kBoxW = kRowDec ? 48 : 32;
   static constexpr uint32_t kSubBytes = kSubRows * kBoxW;
   static constexpr uint32_t kRawSlotBytes = kRawBoxes * kSubBytes;
-  static constexpr int kRawSlots = GATEUP ? 3 : (WIDE ? 1 : 2);   // raw ring slots per producer group
+  static constexpr int kRawSlots = WIDE ? 1 : (GATEUP ? 3 : 2);   // raw ring slots per producer group
   static constexpr uint32_t kTmemCols = kAccBufs * kHalves * kBN;
   static constexpr int kSmemBytes = kStages * kStageBytes + kProdGroups * kRawSlots * kRawSlotBytes + 1024;
   static constexpr uint32_t kIdesc = umma_idesc(kBN);
@@ -297,7 +297,7 @@ k_moe_gemm(const __grid_constant__ CUtensorMap tmap_h, const __grid_constant__ C
   const int rb = (K / MOE_QK) * MOE_QBYTES;            // bytes per weight row
   constexpr int kHalves = C::kHalves, kStages = C::kStages, kAhead = C::kAhead;
   constexpr uint32_t kBOff = C::kBOff, kStageBytes = C::kStageBytes, kTmemCols = C::kTmemCols;
-  const int n_items = (GATEUP ? *W.n_tiles : *W.n_pairs) * n_ntiles;
+  const int n_items = ((GATEUP && !WIDE) ? *W.n_tiles : *W.n_pairs) * n_ntiles;
   // Work order: the n-tiles of one row tile (gate_up) or tile pair (down) follow each other,
   // so its A rows are read while in L2.
   auto item_nt = [&](int item) -> int { return item % n_ntiles; };
@@ -305,7 +305,7 @@ k_moe_gemm(const __grid_constant__ CUtensorMap tmap_h, const __grid_constant__ C
   // tile's start) belongs to it (down only)
   auto item_tile = [&](int item, int &tile, bool &h1) {
     const int q = item / n_ntiles;
-    if (GATEUP) {
+    if (GATEUP && !WIDE) {
       tile = q;
       h1 = false;
     } else {
@@ -375,7 +375,7 @@ k_moe_gemm(const __grid_constant__ CUtensorMap tmap_h, const __grid_constant__ C
     // gate_up only), whether this thread's B row is one of the expert's (gate_up: gate and up
     // rows c < f), the tile, and whether the second half holds any of the expert's rows
     struct RowSrc {
-      const __nv_bfloat16 *arow[GATEUP ? 4 : 1];
+      const __nv_bfloat16 *arow[GATEUP ? 4 * kHalves : 1];
       bool wvalid;
       int tile, h1;
     };
@@ -391,8 +391,10 @@ k_moe_gemm(const __grid_constant__ CUtensorMap tmap_h, const __grid_constant__ C
       rs.tile = tile;
       rs.h1 = h1;
       if (GATEUP) {
+        // A row ra (0 .. 128 kHalves - 1) is row m0 + ra of the expert (a pair's second tile
+        // follows its first)
 #pragma unroll
-        for (int q = 0; q < 4; ++q) {
+        for (int q = 0; q < 4 * kHalves; ++q) {
           const int r = m0 + (pt >> 3) + 32 * q;
           rs.arow[q] = r < cnt ? a_src + (size_t)(W.perm[W.offsets[e] + r] / k) * d : nullptr;
         }
@@ -408,11 +410,13 @@ k_moe_gemm(const __grid_constant__ CUtensorMap tmap_h, const __grid_constant__ C
       const uint32_t a_saddr = sbase + (uint32_t)s * kStageBytes;
       if (GATEUP) {
 #pragma unroll
-        for (int q = 0; q < 4; ++q) {
+        for (int q = 0; q < 4 * kHalves; ++q) {
           const int ra = (pt >> 3) + 32 * q;
+          if (ra >= BM && !rs.h1) break;   // the MMA skips an empty second half
           const __nv_bfloat16 *ap = rs.arow[q] ? rs.arow[q] + (size_t)ks * BK + 8 * cb : a_src;
-          cp_async16(a_saddr + (uint32_t)ra * 128u + (((uint32_t)cb ^ (uint32_t)(ra & 7)) << 4), ap,
-                     rs.arow[q] ? 16u : 0u);
+          cp_async16(a_saddr + (uint32_t)(ra >> 7) * kTileBytes + (uint32_t)(ra & 127) * 128u +
+                         (((uint32_t)cb ^ (uint32_t)(ra & 7)) << 4),
+                     ap, rs.arow[q] ? 16u : 0u);
         }
       } else if (pt == 0) {
         // the 128 x 64 tiles of h by TMA: their bytes join the stage's full barrier, whose
@@ -923,8 +927,14 @@ int moe_launch_gemm_experts(const MoeLaunch &L, const MoeWork &W, const void *x,
   // K of both GEMMs in whole 64-wide steps; down's output in whole 128-column tiles
   if (d % BK || d % GemmCfg<false>::kBN || f % BK) return -2;
   const bool wide = d % GemmCfg<false, true>::kBN == 0;   // down items of N = 256
-  static unsigned long long smem_ok[3] = {0ull, 0ull, 0ull};   // per device, per kernel
-  if (!moe_allow_dyn_smem(reinterpret_cast<const void *>(k_moe_gemm<true>), &smem_ok[0]) ||
+  // gate_up items of a tile pair (M = 256 sharing one decoded B tile, one accumulator buffer)
+  // when the experts hold 1.5 tiles of rows on average, else of one tile (M = 128, two
+  // accumulator buffers, so the epilogue overlaps the next item); both give the same bits
+  const bool gu_pairs = (long long)T * k >= 3LL * BM / 2 * E;
+  static unsigned long long smem_ok[4] = {0ull, 0ull, 0ull, 0ull};   // per device, per kernel
+  if (!moe_allow_dyn_smem(gu_pairs ? reinterpret_cast<const void *>(k_moe_gemm<true, true>)
+                                   : reinterpret_cast<const void *>(k_moe_gemm<true>),
+                          &smem_ok[gu_pairs ? 3 : 0]) ||
       !moe_allow_dyn_smem(wide ? reinterpret_cast<const void *>(k_moe_gemm<false, true>)
                                : reinterpret_cast<const void *>(k_moe_gemm<false>),
                           &smem_ok[wide ? 2 : 1]))
@@ -932,14 +942,20 @@ int moe_launch_gemm_experts(const MoeLaunch &L, const MoeWork &W, const void *x,
   moe_prof_mark(L.stream, MOE_K_GEMM_GATEUP, true);
   CUtensorMap th, twg, twd;
   if (!make_tmap_h(&th, W.hb, f, (long long)max_tiles * BM)) return -1;
+  static_assert(GemmCfg<true, true>::kBoxW == GemmCfg<true>::kBoxW, "one gate_up weight map for both");
   if (!make_tmap_w(&twg, gate_up_q4, (d / MOE_QK) * MOE_QBYTES, (long long)E * 2 * f, GemmCfg<true>::kBoxW) ||
       !make_tmap_w(&twd, down_q4, (f / MOE_QK) * MOE_QBYTES, (long long)E * d,
                    wide ? GemmCfg<false, true>::kBoxW : GemmCfg<false>::kBoxW))
     return -1;
-  constexpr int kSmemG = GemmCfg<true>::kSmemBytes, kSmemD = GemmCfg<false>::kSmemBytes,
+  constexpr int kSmemG = GemmCfg<true>::kSmemBytes, kSmemGP = GemmCfg<true, true>::kSmemBytes,
+                kSmemD = GemmCfg<false>::kSmemBytes,
                 kSmemDW = GemmCfg<false, true>::kSmemBytes;
-  k_moe_gemm<true><<<num_sms, kThreads, kSmemG, L.stream>>>(th, twg, static_cast<const __nv_bfloat16 *>(x),
-                                                            expert_scale, d, f, k, W);
+  if (gu_pairs)
+    k_moe_gemm<true, true><<<num_sms, kThreads, kSmemGP, L.stream>>>(th, twg, static_cast<const __nv_bfloat16 *>(x),
+                                                                     expert_scale, d, f, k, W);
+  else
+    k_moe_gemm<true><<<num_sms, kThreads, kSmemG, L.stream>>>(th, twg, static_cast<const __nv_bfloat16 *>(x),
+                                                              expert_scale, d, f, k, W);
   if (launch_err()) return -1;
   moe_prof_count(1);
   moe_prof_mark(L.stream, MOE_K_GEMM_GATEUP, false);
