@@ -63,22 +63,23 @@ constexpr uint32_t umma_idesc(int n) {
 }
 
 // Per GEMM:
-//  gate_up: an item is one 128-row tile and N = 256 columns, the 128 gate rows c0 .. c0+127 and
-//    the matching 128 up rows (rows past f are zero); measured: one tcgen05.mma of N = 256 does
-//    twice the work of an N = 128 one in about the same pipeline time. A rows are gathered by
-//    the producers.
-//  down: an item is up to two consecutive tiles of one expert, M = 256 as two 128-row halves
-//    that share the dequantised B tile (A comes by TMA), so the decode work per MMA halves.
-//    WIDE (d a multiple of 256): N = 256 output columns, one accumulator buffer (2 x 256 TMEM
-//    columns), one B row per producer thread as for gate_up; otherwise N = 128, two buffers,
-//    one block of a B row per thread.
-template <bool GATEUP, bool WIDE = false>
+//  gate_up: N = 256 columns, the 128 gate rows c0 .. c0+127 and the matching 128 up rows (rows
+//    past f are zero); measured: one tcgen05.mma of N = 256 does twice the work of an N = 128
+//    one in about the same pipeline time. A rows are gathered by the producers.
+//  down: N = 256 (or 128) output columns; A, the padded h, comes by TMA.
+//  Each GEMM comes in shapes BN x HALVES (MMA N, and M = 128 HALVES): an item is one row tile
+//    (HALVES = 1) or a tile pair of one expert (HALVES = 2, the halves sharing the decoded B
+//    tile, so the decode work per flop halves); BN = 256 decodes one B row a producer thread
+//    (down: d a multiple of 256), BN = 128 one block of a B row. TMEM holds two accumulator
+//    buffers where 2 x HALVES x BN <= 512 columns (the epilogue of an item overlaps the next
+//    item's MMAs), else one.
+template <bool GATEUP, int BN, int HALVES>
 struct GemmCfg {
-  static constexpr bool kRowDec = GATEUP || WIDE;                 // one B row (both blocks) a thread
-  static constexpr int kBN = kRowDec ? 256 : 128;                 // MMA N
-  static constexpr int kHalves = (GATEUP && !WIDE) ? 1 : 2;      // M = 128 kHalves
-  static constexpr int kStages = GATEUP ? 3 : (WIDE ? 3 : 4);
-  static constexpr int kAccBufs = WIDE ? 1 : 2;                   // accumulator buffers in TMEM
+  static constexpr bool kRowDec = BN == 256;                      // one B row (both blocks) a thread
+  static constexpr int kBN = BN;                                  // MMA N
+  static constexpr int kHalves = HALVES;                          // M = 128 kHalves
+  static constexpr int kAccBufs = 2 * HALVES * BN <= 512 ? 2 : 1;  // accumulator buffers in TMEM
+  static constexpr int kStages = (HALVES == 2 && BN == 128) ? 4 : 3;
   // group steps the copies run ahead of the decode
   static constexpr int kAhead = 1;
   static constexpr uint32_t kBBytes = (uint32_t)kBN * BK * 2;
@@ -90,12 +91,14 @@ struct GemmCfg {
   static constexpr uint32_t kBoxW = kRowDec ? 48 : 32;
   static constexpr uint32_t kSubBytes = kSubRows * kBoxW;
   static constexpr uint32_t kRawSlotBytes = kRawBoxes * kSubBytes;
-  static constexpr int kRawSlots = WIDE ? 1 : (GATEUP ? 3 : 2);   // raw ring slots per producer group
+  // raw ring slots per producer group (shared memory: 216-225 KB with the stages)
+  static constexpr int kRawSlots = (HALVES == 2 && BN == 256) ? 1 : (BN == 256 ? 3 : 2);
   static constexpr uint32_t kTmemCols = kAccBufs * kHalves * kBN;
   static constexpr int kSmemBytes = kStages * kStageBytes + kProdGroups * kRawSlots * kRawSlotBytes + 1024;
   static constexpr uint32_t kIdesc = umma_idesc(kBN);
   static_assert(kAhead * kProdGroups <= kStages, "the prologue's stages must be free");
   static_assert(kStages <= kMaxStages && kRawSlots <= kMaxRawSlots && kTmemCols <= 512, "limits");
+  static_assert(kSmemBytes <= 231 * 1024, "one CTA per SM, with the static barriers");
   // the producer group's threads: one B row each (gate_up), or one block of a B row (down)
   static_assert(kBN * (kRowDec ? 1 : 2) == kGroupThreads, "producer threads cover the B tile");
 };
@@ -277,7 +280,7 @@ __device__ __forceinline__ void store_blk_zero(uint32_t rowbase, uint32_t x, int
 // DOWN:   A = hb [padded rows, f] (tmap_h: 2-D tiles of 128 rows x 64 columns by TMA), B =
 //         down rows n0..n0+127, K = f; epilogue y * w * s -> yslot (bf16, slot order).
 // tmap_w: the weight matrix (gate_up or down) as lines of 4 rows, boxes of 48 bytes x 32 lines.
-template <bool GATEUP, bool WIDE = false>
+template <bool GATEUP, int BN, int HALVES>
 __global__ void __launch_bounds__(kThreads, 1)
 k_moe_gemm(const __grid_constant__ CUtensorMap tmap_h, const __grid_constant__ CUtensorMap tmap_w,
            const __nv_bfloat16 *__restrict__ a_src, const float *__restrict__ expert_scale, int d, int f, int k,
@@ -289,7 +292,7 @@ k_moe_gemm(const __grid_constant__ CUtensorMap tmap_h, const __grid_constant__ C
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int K = GATEUP ? d : f;
   const int ksteps = K / BK;
-  using C = GemmCfg<GATEUP, WIDE>;
+  using C = GemmCfg<GATEUP, BN, HALVES>;
   constexpr bool kRowDec = C::kRowDec;
   constexpr int kAccBufs = C::kAccBufs;
   constexpr int kBN = C::kBN;
@@ -297,7 +300,7 @@ k_moe_gemm(const __grid_constant__ CUtensorMap tmap_h, const __grid_constant__ C
   const int rb = (K / MOE_QK) * MOE_QBYTES;            // bytes per weight row
   constexpr int kHalves = C::kHalves, kStages = C::kStages, kAhead = C::kAhead;
   constexpr uint32_t kBOff = C::kBOff, kStageBytes = C::kStageBytes, kTmemCols = C::kTmemCols;
-  const int n_items = ((GATEUP && !WIDE) ? *W.n_tiles : *W.n_pairs) * n_ntiles;
+  const int n_items = (HALVES == 1 ? *W.n_tiles : *W.n_pairs) * n_ntiles;
   // Work order: the n-tiles of one row tile (gate_up) or tile pair (down) follow each other,
   // so its A rows are read while in L2.
   auto item_nt = [&](int item) -> int { return item % n_ntiles; };
@@ -305,7 +308,7 @@ k_moe_gemm(const __grid_constant__ CUtensorMap tmap_h, const __grid_constant__ C
   // tile's start) belongs to it (down only)
   auto item_tile = [&](int item, int &tile, bool &h1) {
     const int q = item / n_ntiles;
-    if (GATEUP && !WIDE) {
+    if (HALVES == 1) {
       tile = q;
       h1 = false;
     } else {
@@ -435,7 +438,7 @@ k_moe_gemm(const __grid_constant__ CUtensorMap tmap_h, const __grid_constant__ C
                             (kRowDec ? 0u : 16u * (uint32_t)jh);
         mbar_arrive_expect_tx(&bars.raw[pg][q], kSubBytes);
         tma_load_2d(raw_base + (uint32_t)q * kRawSlotBytes + (uint32_t)wg * kSubBytes, &tmap_w, (int)xb,
-                    line0 + (GATEUP ? jh * (f >> 2) : (WIDE ? jh * 32 : 0)), &bars.raw[pg][q]);
+                    line0 + (GATEUP ? jh * (f >> 2) : (kRowDec ? jh * 32 : 0)), &bars.raw[pg][q]);
       }
     };
     bool ok = true;
@@ -921,49 +924,53 @@ int moe_launch_router_tc(const MoeLaunch &L, const MoeWork &W, const void *x, co
   return 0;
 }
 
+constexpr int kDownWideHalves = 1;   // down with N = 256: single tiles (1) or tile pairs (2)
+
 int moe_launch_gemm_experts(const MoeLaunch &L, const MoeWork &W, const void *x, const uint8_t *gate_up_q4,
                             const uint8_t *down_q4, const float *expert_scale, int T, int d, int f, int E, int k,
                             float *out, int num_sms, int max_tiles) {
   // K of both GEMMs in whole 64-wide steps; down's output in whole 128-column tiles
-  if (d % BK || d % GemmCfg<false>::kBN || f % BK) return -2;
-  const bool wide = d % GemmCfg<false, true>::kBN == 0;   // down items of N = 256
-  // gate_up items of a tile pair (M = 256 sharing one decoded B tile, one accumulator buffer)
-  // when the experts hold 1.5 tiles of rows on average, else of one tile (M = 128, two
-  // accumulator buffers, so the epilogue overlaps the next item); both give the same bits
+  if (d % BK || d % 128 || f % BK) return -2;
+  // gate_up: tile pairs (M = 256 sharing one decoded B tile, one accumulator buffer) when the
+  // experts hold 1.5 tiles of rows on average, else single tiles (two accumulator buffers, the
+  // epilogue overlapping the next item); both give the same bits
   const bool gu_pairs = (long long)T * k >= 3LL * BM / 2 * E;
+  // down: N = 256 over single tiles (two accumulator buffers) where d is a multiple of 256,
+  // else N = 128 over tile pairs
+  const bool wide = d % 256 == 0;
+  using CG1 = GemmCfg<true, 256, 1>;
+  using CG2 = GemmCfg<true, 256, 2>;
+  using CDN = GemmCfg<false, 128, 2>;
+  using CDW = GemmCfg<false, 256, kDownWideHalves>;
   static unsigned long long smem_ok[4] = {0ull, 0ull, 0ull, 0ull};   // per device, per kernel
-  if (!moe_allow_dyn_smem(gu_pairs ? reinterpret_cast<const void *>(k_moe_gemm<true, true>)
-                                   : reinterpret_cast<const void *>(k_moe_gemm<true>),
-                          &smem_ok[gu_pairs ? 3 : 0]) ||
-      !moe_allow_dyn_smem(wide ? reinterpret_cast<const void *>(k_moe_gemm<false, true>)
-                               : reinterpret_cast<const void *>(k_moe_gemm<false>),
-                          &smem_ok[wide ? 2 : 1]))
+  if (!moe_allow_dyn_smem(gu_pairs ? reinterpret_cast<const void *>(k_moe_gemm<true, 256, 2>)
+                                   : reinterpret_cast<const void *>(k_moe_gemm<true, 256, 1>),
+                          &smem_ok[gu_pairs ? 1 : 0]) ||
+      !moe_allow_dyn_smem(wide ? reinterpret_cast<const void *>(k_moe_gemm<false, 256, kDownWideHalves>)
+                               : reinterpret_cast<const void *>(k_moe_gemm<false, 128, 2>),
+                          &smem_ok[wide ? 3 : 2]))
     return -1;
   moe_prof_mark(L.stream, MOE_K_GEMM_GATEUP, true);
   CUtensorMap th, twg, twd;
   if (!make_tmap_h(&th, W.hb, f, (long long)max_tiles * BM)) return -1;
-  static_assert(GemmCfg<true, true>::kBoxW == GemmCfg<true>::kBoxW, "one gate_up weight map for both");
-  if (!make_tmap_w(&twg, gate_up_q4, (d / MOE_QK) * MOE_QBYTES, (long long)E * 2 * f, GemmCfg<true>::kBoxW) ||
-      !make_tmap_w(&twd, down_q4, (f / MOE_QK) * MOE_QBYTES, (long long)E * d,
-                   wide ? GemmCfg<false, true>::kBoxW : GemmCfg<false>::kBoxW))
+  static_assert(CG1::kBoxW == CG2::kBoxW, "one gate_up weight map for both");
+  if (!make_tmap_w(&twg, gate_up_q4, (d / MOE_QK) * MOE_QBYTES, (long long)E * 2 * f, CG1::kBoxW) ||
+      !make_tmap_w(&twd, down_q4, (f / MOE_QK) * MOE_QBYTES, (long long)E * d, wide ? CDW::kBoxW : CDN::kBoxW))
     return -1;
-  constexpr int kSmemG = GemmCfg<true>::kSmemBytes, kSmemGP = GemmCfg<true, true>::kSmemBytes,
-                kSmemD = GemmCfg<false>::kSmemBytes,
-                kSmemDW = GemmCfg<false, true>::kSmemBytes;
+  const __nv_bfloat16 *xb = static_cast<const __nv_bfloat16 *>(x);
   if (gu_pairs)
-    k_moe_gemm<true, true><<<num_sms, kThreads, kSmemGP, L.stream>>>(th, twg, static_cast<const __nv_bfloat16 *>(x),
-                                                                     expert_scale, d, f, k, W);
+    k_moe_gemm<true, 256, 2><<<num_sms, kThreads, CG2::kSmemBytes, L.stream>>>(th, twg, xb, expert_scale, d, f, k, W);
   else
-    k_moe_gemm<true><<<num_sms, kThreads, kSmemG, L.stream>>>(th, twg, static_cast<const __nv_bfloat16 *>(x),
-                                                              expert_scale, d, f, k, W);
+    k_moe_gemm<true, 256, 1><<<num_sms, kThreads, CG1::kSmemBytes, L.stream>>>(th, twg, xb, expert_scale, d, f, k, W);
   if (launch_err()) return -1;
   moe_prof_count(1);
   moe_prof_mark(L.stream, MOE_K_GEMM_GATEUP, false);
   moe_prof_mark(L.stream, MOE_K_GEMM_DOWN, true);
   if (wide)
-    k_moe_gemm<false, true><<<num_sms, kThreads, kSmemDW, L.stream>>>(th, twd, W.hb, expert_scale, d, f, k, W);
+    k_moe_gemm<false, 256, kDownWideHalves><<<num_sms, kThreads, CDW::kSmemBytes, L.stream>>>(th, twd, W.hb, expert_scale,
+                                                                                             d, f, k, W);
   else
-    k_moe_gemm<false><<<num_sms, kThreads, kSmemD, L.stream>>>(th, twd, W.hb, expert_scale, d, f, k, W);
+    k_moe_gemm<false, 128, 2><<<num_sms, kThreads, CDN::kSmemBytes, L.stream>>>(th, twd, W.hb, expert_scale, d, f, k, W);
   if (launch_err()) return -1;
   moe_prof_count(1);
   moe_prof_mark(L.stream, MOE_K_GEMM_DOWN, false);
