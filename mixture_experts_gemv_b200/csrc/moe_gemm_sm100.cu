@@ -10,9 +10,10 @@
 // followed by out[t] = sum_j w_tj * s_e * Y[slot(t, j)] in j order.
 //
 // Layout: the routed rows of each expert are padded to whole 128-row tiles; tile i of the
-// tile list covers padded rows [128 i, 128 i + 128). A gate_up work item is one tile and one
-// n-tile; a down work item is up to two consecutive tiles of one expert (M = 256 as two
-// 128-row MMA halves sharing the B tile, so the decode work per MMA halves) and one n-tile.
+// tile list covers padded rows [128 i, 128 i + 128). A work item is one n-tile of either one
+// row tile (M = 128) or a pair of consecutive tiles of one expert (M = 256 as two 128-row MMA
+// halves sharing the B tile, so the decode work per flop halves); the shapes per call are
+// chosen by the launcher (GemmCfg below).
 // The A tile of a K step lands in the 128-byte swizzled K-major layout: gate_up's producers
 // gather the tokens' rows of x with 16-byte asynchronous copies, eight lanes per 128-byte row
 // segment (zero-filled past the expert's rows); down's 128 x 64 tiles of the padded h come by
@@ -27,13 +28,14 @@
 // epilogue puts the columns back in weight-row order.
 //
 // One CTA per SM, persistent over work items, warp-specialised:
-//   warps 0-3  epilogue: tcgen05.ld of the 128 x 128 FP32 accumulators (lane = row)
-//   warp  4    TMEM allocation; lane 0 issues tcgen05.mma (M = 128, N = 128, K = 16, one
-//              per 16-wide K slice and item half)
+//   warps 0-3  epilogue: tcgen05.ld of the FP32 accumulators (lane = row)
+//   warp  4    TMEM allocation; lane 0 issues tcgen05.mma (M = 128, N = 256 or 128, K = 16,
+//              one per 16-wide K slice and item half)
 //   warps 5-20 producers in two groups taking alternate K steps: A copies (gate_up) or the
 //              TMA issue (down), the raw-weight TMA issue, Q4_0 -> bf16 dequantisation for B
-// Shared-memory stages are handed over with mbarriers (every wait is time-bounded); the
-// accumulators are double-buffered in TMEM so the epilogue of one item overlaps the next.
+// Shared-memory stages are handed over with mbarriers (every wait is time-bounded); where two
+// accumulators fit in TMEM's 512 columns the epilogue of one item overlaps the next item's MMAs.
+// The prefill router product runs in this file too (k_split_router, k_router_tc below).
 #include <cuda.h>
 #include <cudaTypedefs.h>
 
