@@ -205,10 +205,14 @@ __device__ __forceinline__ uint32_t pack_bf16(float a, float b) {
 // (lo01: bytes 0,1; lo23: bytes 2,3) and high nibbles (hi01, hi23). A code q is first made
 // the bf16 value 128 + q by OR-ing it into the mantissa of 128 (exact), then 136 is
 // subtracted (exact) and the result is multiplied by d (one rounding).
-__device__ __forceinline__ void dq_word(uint32_t w, __nv_bfloat162 d2, uint32_t &lo01, uint32_t &lo23,
-                                        uint32_t &hi01, uint32_t &hi23) {
-  const uint32_t v01 = __byte_perm(w, 0u, 0x4140u);   // [b0, 0, b1, 0]
-  const uint32_t v23 = __byte_perm(w, 0u, 0x4342u);   // [b2, 0, b3, 0]
+// The four code bytes may straddle two words: bytes 0, 1 are sel01 of wa and bytes 2, 3 are
+// sel23 of wb (aligned: wa = wb = w, 0x4140 / 0x4342; two bytes past: bytes 2, 3 of w[i] and
+// 0, 1 of w[i + 1], 0x4342 / 0x4140).
+__device__ __forceinline__ void dq_word2(uint32_t wa, uint32_t wb, uint32_t sel01, uint32_t sel23,
+                                         __nv_bfloat162 d2, uint32_t &lo01, uint32_t &lo23, uint32_t &hi01,
+                                         uint32_t &hi23) {
+  const uint32_t v01 = __byte_perm(wa, 0u, sel01);    // [b0, 0, b1, 0]
+  const uint32_t v23 = __byte_perm(wb, 0u, sel23);    // [b2, 0, b3, 0]
   const uint32_t kMag = 0x43004300u;                  // bf16 (128, 128)
   const uint32_t l01 = (v01 & 0x000F000Fu) | kMag;
   const uint32_t l23 = (v23 & 0x000F000Fu) | kMag;
@@ -227,14 +231,24 @@ __device__ __forceinline__ void dq_word(uint32_t w, __nv_bfloat162 d2, uint32_t 
   hi23 = cv(h23);
 }
 
+__device__ __forceinline__ void dq_word(uint32_t w, __nv_bfloat162 d2, uint32_t &lo01, uint32_t &lo23,
+                                        uint32_t &hi01, uint32_t &hi23) {
+  dq_word2(w, w, 0x4140u, 0x4342u, d2, lo01, lo23, hi01, hi23);
+}
+
 // One block -- fp16 scale bits and its four code words -- into its 4 swizzled 16-byte chunks
-// (cbase .. cbase + 3) of the B tile row at rowbase (x = the row's swizzle phase).
-__device__ __forceinline__ void store_blk_bf16(uint32_t dbits, const uint32_t (&q)[4], uint32_t rowbase, uint32_t x,
+// (cbase .. cbase + 3) of the B tile row at rowbase (x = the row's swizzle phase). With SHIFT
+// the block's code word i is bytes 2, 3 of q[i] and 0, 1 of q[i + 1] (q[0 .. 4]).
+template <bool SHIFT>
+__device__ __forceinline__ void store_blk_bf16(uint32_t dbits, const uint32_t *q, uint32_t rowbase, uint32_t x,
                                                int cbase) {
   const __nv_bfloat162 d2 = __float2bfloat162_rn(__half2float(__ushort_as_half((unsigned short)(dbits & 0xffffu))));
   uint32_t lo[8], hi[8];   // element pairs (0,1),(2,3),...,(14,15) and (16,17),...,(30,31)
 #pragma unroll
-  for (int i = 0; i < 4; ++i) dq_word(q[i], d2, lo[2 * i], lo[2 * i + 1], hi[2 * i], hi[2 * i + 1]);
+  for (int i = 0; i < 4; ++i) {
+    if (SHIFT) dq_word2(q[i], q[i + 1], 0x4342u, 0x4140u, d2, lo[2 * i], lo[2 * i + 1], hi[2 * i], hi[2 * i + 1]);
+    else dq_word(q[i], d2, lo[2 * i], lo[2 * i + 1], hi[2 * i], hi[2 * i + 1]);
+  }
   st_shared_v4(rowbase + (((uint32_t)(cbase + 0) ^ x) << 4), lo[0], lo[1], lo[2], lo[3]);   // elements 0-7
   st_shared_v4(rowbase + (((uint32_t)(cbase + 1) ^ x) << 4), lo[4], lo[5], lo[6], lo[7]);   // 8-15
   st_shared_v4(rowbase + (((uint32_t)(cbase + 2) ^ x) << 4), hi[0], hi[1], hi[2], hi[3]);   // 16-23
@@ -247,16 +261,8 @@ __device__ __forceinline__ void store_blk_bf16(uint32_t dbits, const uint32_t (&
 // WB + 5 .. WB + 8. BLK selects the blocks decoded: 1, 2 or 3 (both).
 template <int WB, int BLK>
 __device__ __forceinline__ void dec_window(const uint32_t (&w)[12], uint32_t rowbase, uint32_t x) {
-  if (BLK & 1) {
-    uint32_t q[4];
-#pragma unroll
-    for (int i = 0; i < 4; ++i) q[i] = __byte_perm(w[WB + i], w[WB + i + 1], 0x5432u);
-    store_blk_bf16(w[WB], q, rowbase, x, 0);
-  }
-  if (BLK & 2) {
-    const uint32_t q[4] = {w[WB + 5], w[WB + 6], w[WB + 7], w[WB + 8]};
-    store_blk_bf16(w[WB + 4] >> 16, q, rowbase, x, 4);
-  }
+  if (BLK & 1) store_blk_bf16<true>(w[WB], w + WB, rowbase, x, 0);    // codes from byte 2 of word WB
+  if (BLK & 2) store_blk_bf16<false>(w[WB + 4] >> 16, w + WB + 5, rowbase, x, 4);
 }
 template <int BLK>
 __device__ __forceinline__ void dec_window_at(int wb, const uint32_t (&w)[12], uint32_t rowbase, uint32_t x) {
