@@ -191,15 +191,15 @@ int moe_debug_get_hidden(float *h, void *stream);
 int moe_debug_check(void *stream);
 
 /*
- * Failure detection, for tests. Every device-side wait (mbarrier phases, grid barriers) is
- * bounded; a wait that runs out records MOE_ERR_DEVICE_TIMEOUT in the error word, the
- * kernel ends on its own (it waits, again bounded, for its copies in flight first) and the
- * context stays usable.
+ * Failure detection, for tests. Every device-side wait (mbarrier phases, grid barriers, polls
+ * of launch-tagged words) is bounded; a wait that runs out records MOE_ERR_DEVICE_TIMEOUT in
+ * the error word, the kernel ends on its own (it waits, again bounded, for its copies in
+ * flight first) and the context stays usable.
  *   moe_debug_set_wait_ns: bound of every device-side wait of later forwards, in
  *     nanoseconds (0 restores the default of 2 s).
  *   moe_debug_inject: make the next forward simulate a fault by skipping one step --
- *     MOE_INJECT_SKIP_ROUTER_ARRIVAL: in the fused decode kernel, CTA 0 never arrives at the
- *     first grid barrier, so every other CTA's wait there runs out. Cleared by that forward.
+ *     MOE_INJECT_SKIP_ROUTER_ARRIVAL: in the fused decode kernel, CTA 0 never stores its
+ *     router logits, so every CTA's wait for them runs out. Cleared by that forward.
  */
 #define MOE_INJECT_NONE 0
 #define MOE_INJECT_SKIP_ROUTER_ARRIVAL 1

@@ -75,11 +75,18 @@ int cuda_fail(cudaError_t e, const char *what) {
 constexpr int kTileM = MOE_GEMM_TILE_ROWS;   // rows per grouped-GEMM tile
 
 struct Layout {
-  size_t off[25];
+  size_t off[26];
   size_t total;
 };
 
 size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
+
+// The fused decode kernel's launch-tagged words: logits [MOE_FUSED_MAX_T, E], then per-slot
+// outputs [MOE_FUSED_MAX_SLOTS, d].
+size_t tag_logit_words(int max_E) { return (size_t)MOE_FUSED_MAX_T * max_E; }
+size_t tag_bytes(int max_d, int max_E) {
+  return (align_up(tag_logit_words(max_E), 32) + (size_t)MOE_FUSED_MAX_SLOTS * max_d) * 8;
+}
 
 Layout make_layout(int maxT, int max_d, int max_f, int max_E, int max_k) {
   // per-slot buffers hold k + 1 slots per token: the block's dense MLP takes one more slot per
@@ -115,6 +122,7 @@ Layout make_layout(int maxT, int max_d, int max_f, int max_E, int max_k) {
       64,                                // 22 grid-barrier counter
       (size_t)max_d * 4 + 16,            // 23 dense MLP pass: zero router row, then 1.0f
       (size_t)3 * 128 * max_d * 2,       // 24 the router weights as three bf16 planes (prefill)
+      tag_bytes(max_d, max_E),           // 25 launch-tagged logits and per-slot outputs (fused decode)
   };
   Layout L{};
   size_t o = 0;
@@ -154,6 +162,8 @@ int reset_counters_if_needed(cudaStream_t s) {
   if (!g.reset_pending) return MOE_OK;
   cudaError_t e = cudaMemsetAsync(g.W.gbar, 0, 64, s);
   if (e == cudaSuccess) e = cudaMemsetAsync(g.W.counters, 0, g.counters_bytes, s);
+  // the launch tags restart with the counter: no word may carry a tag a coming launch uses
+  if (e == cudaSuccess) e = cudaMemsetAsync(g.W.ltag, 0, tag_bytes(g.max_d, g.max_E), s);
   if (e != cudaSuccess) return cuda_fail(e, "resetting the arrival counters");
   g.reset_pending = false;
   return MOE_OK;
@@ -374,6 +384,8 @@ int moe_init(int device, int max_tokens, int max_d, int max_f, int max_E, int ma
   W.toff = reinterpret_cast<int32_t *>(b + Lt.off[21]);
   W.gbar = reinterpret_cast<unsigned long long *>(b + Lt.off[22]);
   W.wsplit = reinterpret_cast<__nv_bfloat16 *>(b + Lt.off[24]);
+  W.ltag = reinterpret_cast<unsigned long long *>(b + Lt.off[25]);
+  W.ytag = W.ltag + align_up(tag_logit_words(max_E), 32);
   W.err = ed;
   W.wait_ns = MOE_WAIT_NS;
   W.inject = MOE_INJECT_NONE;

@@ -30,6 +30,8 @@
 //   an even number of blocks), each summed in block order, the parts summed in order.
 constexpr int MOE_DECODE_MIN_COMPUTE = 8, MOE_DECODE_MAX_COMPUTE = 12;
 constexpr int MOE_DN_PARTS = 5;
+// Tokens and slots (T k, with the dense MLP's slots) per launch of the fused decode kernel.
+constexpr int MOE_FUSED_MAX_T = 8, MOE_FUSED_MAX_SLOTS = 128;
 __host__ __device__ inline int moe_decode_router_parts(int d) {
   const int g = (d / 32 + 7) / 8;   // 8-block granules of a gate_up row
   return (g < MOE_DECODE_MIN_COMPUTE ? MOE_DECODE_MIN_COMPUTE : (g > MOE_DECODE_MAX_COMPUTE ? MOE_DECODE_MAX_COMPUTE : g)) + 2;
@@ -61,6 +63,11 @@ struct MoeWork {
   int32_t *tiles;     // [max tiles] (expert, m0) work list
   int32_t *toff;      // [E] index of each expert's first tile
   unsigned long long *gbar;   // grid-barrier counter of the fused decode kernel (monotonic)
+  // Launch-tagged words of the fused decode kernel: high 32 bits a tag unique to the launch,
+  // low 32 bits an FP32 value, stored and polled as one 64-bit word, so that a reader that
+  // sees its launch's tag has the value (zeroed with the barrier counter).
+  unsigned long long *ltag;   // [MOE_FUSED_MAX_T, E] router logits
+  unsigned long long *ytag;   // [MOE_FUSED_MAX_SLOTS, d] per-slot down outputs
   int32_t *n_tiles;   // [1]
   int32_t *pairs;     // [n_pairs][2]: first tile of up to two consecutive tiles of one expert, second present
   int32_t *n_pairs;   // [1]

@@ -3,15 +3,17 @@
 //
 //   phase 0  x into shared memory (a bulk copy of the bf16 input, or, in a layer stack, the
 //            previous layer's FP32 output normalised in place: NORM_IN); router logits (one
-//            expert per CTA, warps split d); arrive at the grid barrier, stage every token's
-//            GEMV activations in shared memory, then wait (bounded)
-//   phase 1  every CTA selects the top-k experts of every token, builds the stable
+//            expert per CTA, warps split d), stored as launch-tagged words
+//   phase 1  every CTA selects the top-k experts of every token as soon as that token's
+//            tagged logits are all in (bounded polls; the other warps stage every token's
+//            GEMV activations in shared memory meanwhile), then builds the stable
 //            permutation and its cost-weighted share of the work in its own shared memory
 //   phase 2  gate_up GEMV + GeGLU over this CTA's share of the active experts' rows
-//   barrier  (h complete)
-//   phase 3  down GEMV over this CTA's share of the active experts' down rows
-//   barrier  (per-slot outputs complete)
-//   phase 4  combine: out[t, r] = sum_j w_tj * s_e * y_tj[r], j in order, rows split over CTAs
+//   barrier  (h complete; the launch's one grid barrier)
+//   phase 3  down GEMV over this CTA's share of the active experts' down rows, stored as
+//            launch-tagged words
+//   phase 4  combine: out[t, r] = sum_j w_tj * s_e * y_tj[r], j in order, rows split over CTAs,
+//            each term polled (bounded) until its tagged word is in
 //
 // One producer warp streams the CTA's weight chunks (gate_up, then down) through a ring of
 // shared-memory stages with 1-D bulk copies from the moment the routing is known, so the
@@ -38,6 +40,8 @@ static_assert(kFMaxE / 32 <= kFMinCompute + 2 && kFMaxSlots / 32 <= kFMinCompute
               "the permutation needs a warp per 32 experts and per 32 slots");
 static_assert(2 * kDnParts * kTX * kDnRows >= (kFMaxSlots / 32) * kFMaxE + 2 * (kFMaxE / 32),
               "the reduction buffers hold the permutation scratch");
+static_assert(kFMaxT == MOE_FUSED_MAX_T && kFMaxSlots == MOE_FUSED_MAX_SLOTS,
+              "the workspace's launch-tagged words are sized for these limits");
 static_assert(kDnParts == MOE_DN_PARTS && kFMinCompute == MOE_DECODE_MIN_COMPUTE &&
                   kFMaxCompute == MOE_DECODE_MAX_COMPUTE && kGran == 8,
               "the separate decode kernels reproduce this kernel's router slices and down parts");
@@ -77,8 +81,9 @@ struct FusedShared {
   };
   int n_act;
   int seq[4];                 // this CTA's unit ranges: gate_up [0, 1), down [2, 3)
-  int ok;
+  int cnext;                  // next activation block to convert (phase 1)
   int abort;                  // set by any expired wait: the warps keep their barrier sequence, skip work
+  uint32_t tag;               // this launch's tag (launch-tagged words)
   unsigned long long gbase;   // the grid-barrier counter when this launch started
 };
 
@@ -88,17 +93,39 @@ __device__ __forceinline__ unsigned long long ld_acquire_u64(const unsigned long
   return v;
 }
 
+__device__ __forceinline__ unsigned long long ld_relaxed_u64(const unsigned long long *p) {
+  unsigned long long v;
+  asm volatile("ld.relaxed.gpu.global.u64 %0, [%1];" : "=l"(v) : "l"(p));
+  return v;
+}
+__device__ __forceinline__ void st_relaxed_u64(unsigned long long *p, unsigned long long v) {
+  asm volatile("st.relaxed.gpu.global.u64 [%0], %1;" ::"l"(p), "l"(v) : "memory");
+}
+__device__ __forceinline__ unsigned long long tag_word(uint32_t tag, float v) {
+  return ((unsigned long long)tag << 32) | __float_as_uint(v);
+}
+__device__ __forceinline__ bool has_tag(unsigned long long v, uint32_t tag) { return (uint32_t)(v >> 32) == tag; }
+__device__ __forceinline__ float tag_value(unsigned long long v) { return __uint_as_float((uint32_t)v); }
+
 __device__ __forceinline__ void named_sync(int id, int n) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(n) : "memory");
 }
-// Grid-wide barriers on a monotonically increasing 64-bit counter: every launch adds exactly
-// gridDim.x per barrier, so the counter is a multiple of gridDim.x when a launch starts, and
-// barrier i of the launch (1, 2, 3) completes at that start value + i * gridDim.x. Each CTA
-// reads the start value at its start (CTAs that already arrived at barrier 1 cannot have
-// moved it past the next multiple); an arrival is a release add that returns nothing, and
-// the wait spins (bounded) with acquire loads until the counter reaches the target. One
-// thread per CTA arrives, after the CTA's writes are ordered before it. (After an expired
-// wait the host zeroes the counter before the next launch.)
+// The grid-wide barrier on a monotonically increasing 64-bit counter: every launch has one
+// (h complete) and adds exactly gridDim.x, so the counter is a multiple of gridDim.x when a
+// launch starts, and the barrier completes at that start value + gridDim.x. Each CTA reads
+// the start value at its start (CTAs that already arrived cannot have moved it past the next
+// multiple); an arrival is a release add that returns nothing, and the wait spins (bounded)
+// with acquire loads until the counter reaches the target. One thread per CTA arrives, after
+// the CTA's writes are ordered before it. (After an expired wait the host zeroes the counter
+// and the tagged words before the next launch.)
+//
+// The start value also names the launch: tag = start / gridDim.x + 1, different for any two
+// consecutive launches (and never 0, the value of zeroed words). The router logits and the
+// per-slot down outputs are stored as launch-tagged 64-bit words, tag << 32 | the FP32 bits,
+// with one relaxed store; a reader polls the word with relaxed loads until it carries its
+// launch's tag, and then holds the value -- no counter, fence or grid barrier in between. A
+// word a reader polls is always written by the reader's own launch, so a stale word carries
+// an older launch's tag.
 __device__ __forceinline__ void grid_arrive(unsigned long long *ctr) {
   asm volatile("red.release.gpu.global.add.u64 [%0], 1;" ::"l"(ctr) : "memory");
 }
@@ -145,6 +172,94 @@ __device__ bool wait_phase(uint64_t *bar, uint32_t parity, volatile int *abort, 
       return false;
     }
   }
+  return true;
+}
+
+// The selection of one token by one warp from its launch-tagged logit words lt[0, E): each
+// lane polls its experts' words (lane + 32 i) until every word of the token carries the
+// launch's tag, then the warp selects as warp_topk_softmax does from the same values. A
+// bound that runs out (decided by the warp as one) reports a timeout, sets *abort and
+// returns false.
+template <int kMaxPer>
+__device__ bool warp_select_tagged(const unsigned long long *lt, uint32_t tag, int E, int k, float rscale,
+                                   int32_t *ids, float *w, volatile int *abort, volatile uint32_t *err,
+                                   uint64_t limit_ns) {
+  const int lane = threadIdx.x & 31;
+  unsigned long long v[kMaxPer];
+#pragma unroll
+  for (int i = 0; i < kMaxPer; ++i) {
+    const int e = lane + 32 * i;
+    v[i] = e < E ? ld_relaxed_u64(lt + e) : tag_word(tag, 0.f);
+  }
+  uint64_t t0 = 0;
+  for (int round = 0;; ++round) {
+    bool mine = true;
+#pragma unroll
+    for (int i = 0; i < kMaxPer; ++i) mine = mine && has_tag(v[i], tag);
+    if (__all_sync(0xffffffffu, mine)) break;
+    if (round == 0) {
+      t0 = globaltimer_ns();
+    } else if (__any_sync(0xffffffffu, globaltimer_ns() - t0 > limit_ns)) {
+      if (lane == 0) {
+        report_error(err, MOE_DEV_ERR_TIMEOUT, 20);
+        *abort = 1;
+      }
+      return false;
+    }
+#pragma unroll
+    for (int i = 0; i < kMaxPer; ++i) {
+      const int e = lane + 32 * i;
+      if (e < E && !has_tag(v[i], tag)) v[i] = ld_relaxed_u64(lt + e);
+    }
+  }
+  if (k <= 8) {
+    uint32_t o[kMaxPer];
+#pragma unroll
+    for (int i = 0; i < kMaxPer; ++i) o[i] = lane + 32 * i < E ? logit_ord(tag_value(v[i])) : 0u;
+    warp_top8_softmax_keys<kMaxPer>(o, k, rscale, ids, w);
+  } else {
+    uint64_t key[kMaxPer];
+#pragma unroll
+    for (int i = 0; i < kMaxPer; ++i) {
+      const int e = lane + 32 * i;
+      key[i] = e < E ? topk_key(tag_value(v[i]), e) : 0ull;
+    }
+    warp_topk_softmax_keys64<kMaxPer>(key, k, rscale, ids, w);
+  }
+  return true;
+}
+
+// Polls the n <= 8 launch-tagged words p[j * stride] (issued together) until each carries
+// the tag; their values go to y[]. False when the bound ran out (reported, *abort set).
+__device__ bool poll_tagged(const unsigned long long *p, size_t stride, int n, uint32_t tag, float (&y)[8],
+                            volatile int *abort, volatile uint32_t *err, uint64_t limit_ns) {
+  unsigned long long v[8];
+#pragma unroll
+  for (int j = 0; j < 8; ++j) v[j] = j < n ? ld_relaxed_u64(p + (size_t)j * stride) : tag_word(tag, 0.f);
+  bool all = true;
+#pragma unroll
+  for (int j = 0; j < 8; ++j) all = all && has_tag(v[j], tag);
+  if (!all) {
+    const uint64_t t0 = globaltimer_ns();
+    for (;;) {
+      all = true;
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        if (!has_tag(v[j], tag)) v[j] = ld_relaxed_u64(p + (size_t)j * stride);
+      }
+#pragma unroll
+      for (int j = 0; j < 8; ++j) all = all && has_tag(v[j], tag);
+      if (all) break;
+      if (*abort) return false;
+      if (globaltimer_ns() - t0 > limit_ns) {
+        report_error(err, MOE_DEV_ERR_TIMEOUT, 23);
+        *abort = 1;
+        return false;
+      }
+    }
+  }
+#pragma unroll
+  for (int j = 0; j < 8; ++j) y[j] = tag_value(v[j]);
   return true;
 }
 
@@ -450,7 +565,7 @@ k_moe_decode(const __nv_bfloat16 *__restrict__ x, const float *y_prev, float eps
   __shared__ FusedShared sh;
   const int tid = threadIdx.x, lane = tid & 31, wq = tid >> 5, nw = blockDim.x >> 5;
   // the grid-barrier counter as this launch starts, loaded now by the thread that arrives at
-  // the first barrier (its latency hides behind the router)
+  // the barrier (its latency hides behind the router); it also gives the launch's tag
   const int bar_tid = (int)blockDim.x - 32;
   const unsigned long long gstart = tid == bar_tid ? ld_acquire_u64(W.gbar) : 0ull;
   const int nwc = nw - 2, nct = nwc * 32;   // compute warps 0 .. nwc-1; warp nwc produces, nwc+1 epilogues
@@ -476,6 +591,7 @@ k_moe_decode(const __nv_bfloat16 *__restrict__ x, const float *y_prev, float eps
     mbar_init(&sh.xbar, 1);
     fence_mbar_init();
     sh.abort = 0;
+    sh.cnext = 0;
     if constexpr (!NORM_IN) {
       // x (bf16) into the activation region now; it is converted in place before the first barrier
       mbar_arrive_expect_tx(&sh.xbar, (uint32_t)(T * d * 2));
@@ -509,6 +625,16 @@ k_moe_decode(const __nv_bfloat16 *__restrict__ x, const float *y_prev, float eps
     if (tid == 0) mbar_arrive(&sh.xbar);   // the activation region holds x (no copy to wait for)
   }
   const float rs = __ldg(router_scale);
+  // test-only fault: CTA 0 never stores its router logits, so every CTA's bounded wait for
+  // them runs out and reports a timeout
+  const bool skip_logits = W.inject == MOE_INJECT_SKIP_ROUTER_ARRIVAL && blockIdx.x == 0;
+  auto publish_base = [&]() {
+    if (tid == bar_tid) {
+      const unsigned long long base = gstart - gstart % gridDim.x;
+      sh.gbase = base;
+      sh.tag = (uint32_t)(base / gridDim.x) + 1u;
+    }
+  };
 
   // ---------------------------------------------------------------- phase 0: router
   // A lane loads its router weights first (up to kRtrW float4 groups at once: their HBM
@@ -527,6 +653,7 @@ k_moe_decode(const __nv_bfloat16 *__restrict__ x, const float *y_prev, float eps
     }
     __syncthreads();   // the x copy's mbarrier is initialised; sh.part is free
     wait_phase(&sh.xbar, 0u, &sh.abort, W.err, 26, W.wait_ns);
+    if (e == (int)blockIdx.x) publish_base();
     float acc[kFMaxT];
 #pragma unroll
     for (int t = 0; t < kFMaxT; ++t) acc[t] = 0.f;
@@ -559,55 +686,62 @@ k_moe_decode(const __nv_bfloat16 *__restrict__ x, const float *y_prev, float eps
       if (lane == 0) sh.part[wq][t] = a;
     }
     __syncthreads();
-    if (tid < T) {
+    if (tid < T && !skip_logits) {
       float s = 0.f;
       for (int q = 0; q < nw; ++q) s += sh.part[q][tid];
-      W.logits[(size_t)tid * E + e] = s;
+      st_relaxed_u64(W.ltag + (size_t)tid * E + e, tag_word(sh.tag, s));
     }
     __syncthreads();
   }
-  // arrive at the grid barrier: lane 0 of the last warp arrives and waits, while the other
-  // warps convert every token's activations in place (x was copied into the activation region
-  // at the start), one (token, block) per thread
-  __syncthreads();
-  // test-only fault: CTA 0 leaves without arriving, so every other CTA's bounded wait below
-  // runs out and reports a timeout
-  const bool skip_arrival = W.inject == MOE_INJECT_SKIP_ROUTER_ARRIVAL && blockIdx.x == 0;
-  const int nconv = (int)blockDim.x - 32;
-  if (tid == bar_tid) {
-    sh.gbase = gstart - gstart % gridDim.x;
-    if (!skip_arrival) grid_arrive(W.gbar);
-    sh.ok = (!skip_arrival && grid_wait(W.gbar, sh.gbase + gridDim.x, W.err, 20, W.wait_ns)) ? 1 : 0;
+  if ((int)blockIdx.x >= E) publish_base();
+  // ---------------------------------------------------------------- phase 1: selection
+  // warp t selects token t as soon as its tagged logits are in; the other warps convert every
+  // token's activations in place meanwhile (x was copied into the activation region at the
+  // start), a thread a (token, block), 32 blocks a warp at a time from a shared counter, and
+  // the selecting warps join them when done
+  __syncthreads();   // the router is done with x; sh.tag is published
+  if (wq < T) {
+    if (E <= 128)
+      warp_select_tagged<4>(W.ltag + (size_t)wq * E, sh.tag, E, k, rs, sh.ids + wq * k, sh.w + wq * k, &sh.abort,
+                            W.err, W.wait_ns);
+    else
+      warp_select_tagged<kFMaxE / 32>(W.ltag + (size_t)wq * E, sh.tag, E, k, rs, sh.ids + wq * k, sh.w + wq * k,
+                                      &sh.abort, W.err, W.wait_ns);
   }
-  if (tid < nconv && wait_phase(&sh.xbar, 0u, &sh.abort, W.err, 26, W.wait_ns)) {
-    for (int blk = tid; blk < T * nb; blk += nconv) {
-      const int t = blk / nb, b = blk - t * nb;
-      const uint4 *src = reinterpret_cast<const uint4 *>(xs + (size_t)t * d + (size_t)b * MOE_QK);
-      uint4 raw[4];
+  if (wait_phase(&sh.xbar, 0u, &sh.abort, W.err, 26, W.wait_ns)) {
+    const int nblk = T * nb;
+    for (;;) {
+      int b0 = 0;
+      if (lane == 0) b0 = atomicAdd(&sh.cnext, 32);
+      b0 = __shfl_sync(0xffffffffu, b0, 0);
+      if (b0 >= nblk) break;
+      const int blk = b0 + lane;
+      if (blk < nblk) {
+        const int t = blk / nb, b = blk - t * nb;
+        const uint4 *src = reinterpret_cast<const uint4 *>(xs + (size_t)t * d + (size_t)b * MOE_QK);
+        uint4 raw[4];
 #pragma unroll
-      for (int i = 0; i < 4; ++i) raw[i] = src[i];
-      float v[MOE_QK];
+        for (int i = 0; i < 4; ++i) raw[i] = src[i];
+        float v[MOE_QK];
 #pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        const uint32_t uu[4] = {raw[i].x, raw[i].y, raw[i].z, raw[i].w};
+        for (int i = 0; i < 4; ++i) {
+          const uint32_t uu[4] = {raw[i].x, raw[i].y, raw[i].z, raw[i].w};
 #pragma unroll
-        for (int h = 0; h < 4; ++h) {
-          v[8 * i + 2 * h] = __uint_as_float(uu[h] << 16);
-          v[8 * i + 2 * h + 1] = __uint_as_float(uu[h] & 0xffff0000u);
+          for (int h = 0; h < 4; ++h) {
+            v[8 * i + 2 * h] = __uint_as_float(uu[h] << 16);
+            v[8 * i + 2 * h + 1] = __uint_as_float(uu[h] & 0xffff0000u);
+          }
         }
+        stage_block_t(v, (b >> 2) & 1, xs + (size_t)t * d + (size_t)b * MOE_QK, ss + (size_t)t * nb + b);
       }
-      stage_block_t(v, (b >> 2) & 1, xs + (size_t)t * d + (size_t)b * MOE_QK, ss + (size_t)t * nb + b);
     }
   }
   __syncthreads();
-  if (!sh.ok) {
+  if (sh.abort) {
     if (tid == 0) mbar_wait(&sh.xbar, 0u, W.err, 27, W.wait_ns);   // no copy may land after the CTA exits
     return;
   }
 
-  // ---------------------------------------------------------------- phase 1: selection
-  for (int t = wq; t < T; t += nw)
-    warp_topk_softmax<kFMaxE>(W.logits + (size_t)t * E, E, k, rs, sh.ids + t * k, sh.w + t * k);
   // with the block's dense MLP: expert index E, one more slot per token (s = T k + t), weight 1
   const int Sr = T * k;
   const bool dense = dense_gu != nullptr;
@@ -730,7 +864,7 @@ k_moe_decode(const __nv_bfloat16 *__restrict__ x, const float *y_prev, float eps
       const FChunk c = wk.cur(upe_g, upe_d);
       if (c.down && !down_phase) {
         // all h written (the epilogue warp included) before any CTA reads it
-        grid_barrier_team(W.gbar, sh.gbase + 2ull * gridDim.x, W.err, 21, nteam, &sh.abort, W.wait_ns);
+        grid_barrier_team(W.gbar, sh.gbase + gridDim.x, W.err, 21, nteam, &sh.abort, W.wait_ns);
         down_phase = true;
       }
       const int slot = it % kFStages;
@@ -820,7 +954,7 @@ k_moe_decode(const __nv_bfloat16 *__restrict__ x, const float *y_prev, float eps
       if (lane == 0) mbar_arrive(&sh.empty[slot]);   // this warp's last read of the stage
       wk.advance(c.n, sh.seq, upe_g, upe_d);
     }
-    if (!down_phase) grid_barrier_team(W.gbar, sh.gbase + 2ull * gridDim.x, W.err, 21, nteam, &sh.abort, W.wait_ns);   // no down rows here
+    if (!down_phase) grid_barrier_team(W.gbar, sh.gbase + gridDim.x, W.err, 21, nteam, &sh.abort, W.wait_ns);   // no down rows here
     for (int q = pass < 2 ? 0 : pass - 2; q < pass; ++q) named_sync(kBarEmpty0 + (q & 1), nteam);
   } else {
     // the epilogue warp: the same sequence of chunks and passes
@@ -829,7 +963,7 @@ k_moe_decode(const __nv_bfloat16 *__restrict__ x, const float *y_prev, float eps
     while (!wk.done()) {
       const FChunk c = wk.cur(upe_g, upe_d);
       if (c.down && !down_phase) {
-        grid_barrier_team(W.gbar, sh.gbase + 2ull * gridDim.x, W.err, 21, nteam, &sh.abort, W.wait_ns);
+        grid_barrier_team(W.gbar, sh.gbase + gridDim.x, W.err, 21, nteam, &sh.abort, W.wait_ns);
         down_phase = true;
       }
       const int e = sh.act[c.a];
@@ -861,7 +995,7 @@ k_moe_decode(const __nv_bfloat16 *__restrict__ x, const float *y_prev, float eps
               const int i = i2 / nr, row = i2 - i * nr;
               float s = 0.f;
               for (int pt = 0; pt < P; ++pt) s += red_b[((size_t)pt * kTX + i) * kDnRows + row];
-              W.ybuf[(size_t)sh.perm[off + g0 + i] * d + c.r0 + row] = s;
+              st_relaxed_u64(W.ytag + (size_t)sh.perm[off + g0 + i] * d + c.r0 + row, tag_word(sh.tag, s));
             }
           }
         }
@@ -869,22 +1003,36 @@ k_moe_decode(const __nv_bfloat16 *__restrict__ x, const float *y_prev, float eps
       }
       wk.advance(c.n, sh.seq, upe_g, upe_d);
     }
-    if (!down_phase) grid_barrier_team(W.gbar, sh.gbase + 2ull * gridDim.x, W.err, 21, nteam, &sh.abort, W.wait_ns);
+    if (!down_phase) grid_barrier_team(W.gbar, sh.gbase + gridDim.x, W.err, 21, nteam, &sh.abort, W.wait_ns);
   }
   // ---------------------------------------------------------------- phase 4: combine
-  grid_barrier_team(W.gbar, sh.gbase + 3ull * gridDim.x, W.err, 23, nteam, &sh.abort, W.wait_ns);
+  // no grid barrier: every term is polled (bounded) from its launch-tagged word, eight slots'
+  // words in flight at once, and summed in j order
   if (sh.abort) return;
   const int ti = wq < nwc ? tid : nct + lane;
   const int r0 = (int)((long long)d * blockIdx.x / gridDim.x), r1 = (int)((long long)d * (blockIdx.x + 1) / gridDim.x);
   const int nr = r1 - r0;
+  const uint32_t tag = sh.tag;
   for (int i2 = ti; i2 < nr * T; i2 += nteam) {
     const int t = i2 / nr, r = r0 + i2 % nr;
     float s = 0.f;
-    for (int j = 0; j < k; ++j) {
-      const int slotid = t * k + j;
-      s += sh.w[slotid] * __ldg(expert_scale + sh.ids[slotid]) * __ldcg(W.ybuf + (size_t)slotid * d + r);
+    float y[8];
+    for (int j0 = 0; j0 < k; j0 += 8) {
+      const int n = min(8, k - j0);
+      if (!poll_tagged(W.ytag + (size_t)(t * k + j0) * d + r, (size_t)d, n, tag, y, &sh.abort, W.err, W.wait_ns))
+        return;
+#pragma unroll
+      for (int q = 0; q < 8; ++q) {
+        if (q < n) {
+          const int slotid = t * k + j0 + q;
+          s += sh.w[slotid] * __ldg(expert_scale + sh.ids[slotid]) * y[q];
+        }
+      }
     }
-    if (dense) s += __ldcg(W.ybuf + (size_t)(Sr + t) * d + r);   // the dense MLP's output, weight 1
+    if (dense) {   // the dense MLP's output, weight 1
+      if (!poll_tagged(W.ytag + (size_t)(Sr + t) * d + r, (size_t)d, 1, tag, y, &sh.abort, W.err, W.wait_ns)) return;
+      s += y[0];
+    }
     out[(size_t)t * d + r] = accumulate ? out[(size_t)t * d + r] + s : s;
   }
 }

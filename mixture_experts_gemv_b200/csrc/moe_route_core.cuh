@@ -81,15 +81,11 @@ __device__ __forceinline__ float topk_key_value(uint64_t key) {
   return __uint_as_float(u);
 }
 
+// The selection and softmax from the lane's keys key[i] = topk_key(logit, e) of experts
+// e = lane + 32 i (0 past E).
 template <int kMaxPer>
-__device__ void warp_topk_softmax_t(const float *lg, int E, int k, float rscale, int32_t *ids, float *w) {
+__device__ void warp_topk_softmax_keys64(uint64_t (&key)[kMaxPer], int k, float rscale, int32_t *ids, float *w) {
   const int lane = threadIdx.x & 31;
-  uint64_t key[kMaxPer];
-#pragma unroll
-  for (int i = 0; i < kMaxPer; ++i) {
-    const int e = lane + 32 * i;
-    key[i] = (e < E) ? topk_key(__ldcg(lg + e), e) : 0ull;
-  }
   for (int j = 0; j < k; ++j) {
     uint64_t best = key[0];
 #pragma unroll
@@ -121,6 +117,18 @@ __device__ void warp_topk_softmax_t(const float *lg, int E, int k, float rscale,
   __syncwarp();
   for (int j = lane; j < k; j += 32) w[j] = expf(w[j] - l1) * inv;
   __syncwarp();
+}
+
+template <int kMaxPer>
+__device__ void warp_topk_softmax_t(const float *lg, int E, int k, float rscale, int32_t *ids, float *w) {
+  const int lane = threadIdx.x & 31;
+  uint64_t key[kMaxPer];
+#pragma unroll
+  for (int i = 0; i < kMaxPer; ++i) {
+    const int e = lane + 32 * i;
+    key[i] = (e < E) ? topk_key(__ldcg(lg + e), e) : 0ull;
+  }
+  warp_topk_softmax_keys64<kMaxPer>(key, k, rscale, ids, w);
 }
 
 // Order-preserving 32-bit image of a logit (larger float -> larger unsigned; NaN ranks as

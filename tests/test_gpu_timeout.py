@@ -1,8 +1,8 @@
 """Failure detection on the GPU without a GPU fault: a forward is told to skip one step (CTA 0
-of the fused decode kernel never arrives at the first grid barrier), every other CTA's
-bounded wait there runs out after the shortened bound, the kernel ends on its own, the call
-reports MOE_ERR_DEVICE_TIMEOUT, and the next forward on the same context is clean and
-matches the oracle.
+of the fused decode kernel never stores its router logits), every CTA's bounded wait for them
+runs out after the shortened bound, the kernel ends on its own, the call reports
+MOE_ERR_DEVICE_TIMEOUT, and the next forward on the same context is clean and matches the
+oracle.
 """
 import numpy as np
 import pytest
