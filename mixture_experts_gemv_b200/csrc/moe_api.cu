@@ -21,15 +21,16 @@ struct Ctx {
   uint32_t *err_host = nullptr;   // mapped pinned word
   MoeWork W{};
   __nv_bfloat16 *xbuf[2] = {nullptr, nullptr};   // stack: inter-layer activations
-  float *ylayer = nullptr;                       // stack: intermediate layer output
+  float *ylayer[2] = {nullptr, nullptr};         // stack: intermediate layer outputs (alternating)
   int path = MOE_PATH_AUTO;
   int gemv_max_tokens = 16;   // AUTO: GEMV for T <= 16, grouped GEMM above
   int last_T = 0, last_k = 0, last_E = 0, last_f = 0;
   bool last_gemm = false;
   size_t counters_bytes = 0;
-  bool reset_pending = false;
+  bool reset_pending = false;      // a device wait expired: zero the launch counter, the arrival
+                                   // counters and the tagged words before the next launch
   float *dense_router = nullptr;   // [max_d] zeros: the router of the dense MLP's one-expert pass
-  float *one = nullptr;            // 1.0f: its router scale and expert scale   // a device wait expired: zero the barrier words before the next launch
+  float *one = nullptr;            // 1.0f: its router scale and expert scale
 };
 
 Ctx g;
@@ -75,17 +76,17 @@ int cuda_fail(cudaError_t e, const char *what) {
 constexpr int kTileM = MOE_GEMM_TILE_ROWS;   // rows per grouped-GEMM tile
 
 struct Layout {
-  size_t off[26];
+  size_t off[27];
   size_t total;
 };
 
 size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
 
 // The fused decode kernel's launch-tagged words: logits [MOE_FUSED_MAX_T, E], then per-slot
-// outputs [MOE_FUSED_MAX_SLOTS, d].
+// outputs [MOE_FUSED_MAX_SLOTS, d], then per-slot hidden vectors [MOE_FUSED_MAX_SLOTS, f].
 size_t tag_logit_words(int max_E) { return (size_t)MOE_FUSED_MAX_T * max_E; }
-size_t tag_bytes(int max_d, int max_E) {
-  return (align_up(tag_logit_words(max_E), 32) + (size_t)MOE_FUSED_MAX_SLOTS * max_d) * 8;
+size_t tag_bytes(int max_d, int max_f, int max_E) {
+  return (align_up(tag_logit_words(max_E), 32) + (size_t)MOE_FUSED_MAX_SLOTS * (max_d + max_f)) * 8;
 }
 
 Layout make_layout(int maxT, int max_d, int max_f, int max_E, int max_k) {
@@ -122,7 +123,8 @@ Layout make_layout(int maxT, int max_d, int max_f, int max_E, int max_k) {
       64,                                // 22 grid-barrier counter
       (size_t)max_d * 4 + 16,            // 23 dense MLP pass: zero router row, then 1.0f
       (size_t)3 * 128 * max_d * 2,       // 24 the router weights as three bf16 planes (prefill)
-      tag_bytes(max_d, max_E),           // 25 launch-tagged logits and per-slot outputs (fused decode)
+      tag_bytes(max_d, max_f, max_E),    // 25 launch-tagged logits, per-slot outputs and hidden vectors
+      (size_t)maxT * max_d * 4,          // 26 ylayer2 (stack: layers alternate between 19 and 26)
   };
   Layout L{};
   size_t o = 0;
@@ -163,7 +165,7 @@ int reset_counters_if_needed(cudaStream_t s) {
   cudaError_t e = cudaMemsetAsync(g.W.gbar, 0, 64, s);
   if (e == cudaSuccess) e = cudaMemsetAsync(g.W.counters, 0, g.counters_bytes, s);
   // the launch tags restart with the counter: no word may carry a tag a coming launch uses
-  if (e == cudaSuccess) e = cudaMemsetAsync(g.W.ltag, 0, tag_bytes(g.max_d, g.max_E), s);
+  if (e == cudaSuccess) e = cudaMemsetAsync(g.W.ltag, 0, tag_bytes(g.max_d, g.max_f, g.max_E), s);
   if (e != cudaSuccess) return cuda_fail(e, "resetting the arrival counters");
   g.reset_pending = false;
   return MOE_OK;
@@ -386,6 +388,7 @@ int moe_init(int device, int max_tokens, int max_d, int max_f, int max_E, int ma
   W.wsplit = reinterpret_cast<__nv_bfloat16 *>(b + Lt.off[24]);
   W.ltag = reinterpret_cast<unsigned long long *>(b + Lt.off[25]);
   W.ytag = W.ltag + align_up(tag_logit_words(max_E), 32);
+  W.htag = W.ytag + (size_t)MOE_FUSED_MAX_SLOTS * max_d;
   W.err = ed;
   W.wait_ns = MOE_WAIT_NS;
   W.inject = MOE_INJECT_NONE;
@@ -407,7 +410,8 @@ int moe_init(int device, int max_tokens, int max_d, int max_f, int max_E, int ma
   g.W = W;
   g.xbuf[0] = reinterpret_cast<__nv_bfloat16 *>(b + Lt.off[17]);
   g.xbuf[1] = reinterpret_cast<__nv_bfloat16 *>(b + Lt.off[18]);
-  g.ylayer = reinterpret_cast<float *>(b + Lt.off[19]);
+  g.ylayer[0] = reinterpret_cast<float *>(b + Lt.off[19]);
+  g.ylayer[1] = reinterpret_cast<float *>(b + Lt.off[26]);
   return MOE_OK;
 }
 
@@ -630,11 +634,12 @@ int moe_stack_forward(const void *x_in, int L, const float *const *router_w, con
     float *out_c = out + (size_t)c0 * d;
     for (int i = 0; i < L; ++i) {
       char *trace_i = x_trace ? static_cast<char *>(x_trace) + ((size_t)i * T + c0) * d * 2 : nullptr;
-      float *yo = (i == L - 1) ? out_c : g.ylayer;
+      // layer i writes ylayer[i & 1] and the fused kernel of layer i + 1 reads it: the kernel has
+      // no grid barrier, so its CTAs may write their output rows while others still read y_prev
+      float *yo = (i == L - 1) ? out_c : g.ylayer[i & 1];
       if (i > 0 && fused) {
-        // y_prev = g.ylayer is read before the kernel's first grid barrier, yo written after its last
         MoeLaunch Lf{s, false};
-        rc = moe_launch_fused_decode(Lf, g.W, nullptr, g.ylayer, eps, trace_i, router_w[i], router_scale[i],
+        rc = moe_launch_fused_decode(Lf, g.W, nullptr, g.ylayer[(i - 1) & 1], eps, trace_i, router_w[i], router_scale[i],
                                      gate_up_q4[i], down_q4[i], expert_scale[i], Tc, d, f, E, k, yo, g.num_sms,
                                      nullptr, nullptr, i + 1 < L ? router_w[i + 1] : nullptr);
         if (rc) return cuda_fail(cudaGetLastError(), "fused decode launch");

@@ -62,12 +62,13 @@ struct MoeWork {
   float *yslot;       // [T*k, d] per-slot weighted down outputs (bf16 in the GEMM path)
   int32_t *tiles;     // [max tiles] (expert, m0) work list
   int32_t *toff;      // [E] index of each expert's first tile
-  unsigned long long *gbar;   // grid-barrier counter of the fused decode kernel (monotonic)
+  unsigned long long *gbar;   // launch counter of the fused decode kernel (monotonic)
   // Launch-tagged words of the fused decode kernel: high 32 bits a tag unique to the launch,
   // low 32 bits an FP32 value, stored and polled as one 64-bit word, so that a reader that
-  // sees its launch's tag has the value (zeroed with the barrier counter).
+  // sees its launch's tag has the value (zeroed with the launch counter).
   unsigned long long *ltag;   // [MOE_FUSED_MAX_T, E] router logits
   unsigned long long *ytag;   // [MOE_FUSED_MAX_SLOTS, d] per-slot down outputs
+  unsigned long long *htag;   // [MOE_FUSED_MAX_SLOTS, f] per-slot hidden vectors
   int32_t *n_tiles;   // [1]
   int32_t *pairs;     // [n_pairs][2]: first tile of up to two consecutive tiles of one expert, second present
   int32_t *n_pairs;   // [1]

@@ -8,10 +8,10 @@
 //            tagged logits are all in (bounded polls; the other warps stage every token's
 //            GEMV activations in shared memory meanwhile), then builds the stable
 //            permutation and its cost-weighted share of the work in its own shared memory
-//   phase 2  gate_up GEMV + GeGLU over this CTA's share of the active experts' rows
-//   barrier  (h complete; the launch's one grid barrier)
-//   phase 3  down GEMV over this CTA's share of the active experts' down rows, stored as
-//            launch-tagged words
+//   phase 2  gate_up GEMV + GeGLU over this CTA's share of the active experts' rows, h stored
+//            as launch-tagged words
+//   phase 3  down GEMV over this CTA's share of the active experts' down rows (the hidden
+//            vectors it needs polled, bounded, until they are in), stored as launch-tagged words
 //   phase 4  combine: out[t, r] = sum_j w_tj * s_e * y_tj[r], j in order, rows split over CTAs,
 //            each term polled (bounded) until its tagged word is in
 //
@@ -46,11 +46,10 @@ static_assert(kDnParts == MOE_DN_PARTS && kFMinCompute == MOE_DECODE_MIN_COMPUTE
                   kFMaxCompute == MOE_DECODE_MAX_COMPUTE && kGran == 8,
               "the separate decode kernels reproduce this kernel's router slices and down parts");
 // Named barriers (0 is __syncthreads): compute warps only; FULL / EMPTY of the two reduction
-// buffers between the compute warps and the epilogue warp; compute + epilogue warps.
+// buffers between the compute warps and the epilogue warp.
 constexpr int kBarCompute = 1;
 constexpr int kBarFull0 = 2;
 constexpr int kBarEmpty0 = 4;
-constexpr int kBarTeam = 6;
 constexpr int kTXg = 3;                   // tokens per gate_up pass (register budget)
 // Cost of a scheduling unit of an expert with T_e tokens: reading the codes is shared by
 // the tokens, the multiply-adds are per token.
@@ -84,19 +83,16 @@ struct FusedShared {
   int cnext;                  // next activation block to convert (phase 1)
   int abort;                  // set by any expired wait: the warps keep their barrier sequence, skip work
   uint32_t tag;               // this launch's tag (launch-tagged words)
-  unsigned long long gbase;   // the grid-barrier counter when this launch started
 };
-
-__device__ __forceinline__ unsigned long long ld_acquire_u64(const unsigned long long *p) {
-  unsigned long long v;
-  asm volatile("ld.acquire.gpu.global.u64 %0, [%1];" : "=l"(v) : "l"(p) : "memory");
-  return v;
-}
 
 __device__ __forceinline__ unsigned long long ld_relaxed_u64(const unsigned long long *p) {
   unsigned long long v;
   asm volatile("ld.relaxed.gpu.global.u64 %0, [%1];" : "=l"(v) : "l"(p));
   return v;
+}
+__device__ __forceinline__ void ld_relaxed_v2_u64(const unsigned long long *p, unsigned long long &a,
+                                                  unsigned long long &b) {
+  asm volatile("ld.relaxed.gpu.global.v2.u64 {%0, %1}, [%2];" : "=l"(a), "=l"(b) : "l"(p));
 }
 __device__ __forceinline__ void st_relaxed_u64(unsigned long long *p, unsigned long long v) {
   asm volatile("st.relaxed.gpu.global.u64 [%0], %1;" ::"l"(p), "l"(v) : "memory");
@@ -110,53 +106,21 @@ __device__ __forceinline__ float tag_value(unsigned long long v) { return __uint
 __device__ __forceinline__ void named_sync(int id, int n) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(n) : "memory");
 }
-// The grid-wide barrier on a monotonically increasing 64-bit counter: every launch has one
-// (h complete) and adds exactly gridDim.x, so the counter is a multiple of gridDim.x when a
-// launch starts, and the barrier completes at that start value + gridDim.x. Each CTA reads
-// the start value at its start (CTAs that already arrived cannot have moved it past the next
-// multiple); an arrival is a release add that returns nothing, and the wait spins (bounded)
-// with acquire loads until the counter reaches the target. One thread per CTA arrives, after
-// the CTA's writes are ordered before it. (After an expired wait the host zeroes the counter
-// and the tagged words before the next launch.)
+// No grid barrier: every value one CTA hands to another -- the router logits, the hidden
+// vectors h and the per-slot down outputs -- is stored as a launch-tagged 64-bit word, tag <<
+// 32 | the FP32 bits, with one relaxed store, and the reader polls the word with relaxed loads
+// (bounded) until it carries its launch's tag; it then holds the value, with no counter or
+// fence in between, and a CTA goes on as soon as the values it needs are in.
 //
-// The start value also names the launch: tag = start / gridDim.x + 1, different for any two
-// consecutive launches (and never 0, the value of zeroed words). The router logits and the
-// per-slot down outputs are stored as launch-tagged 64-bit words, tag << 32 | the FP32 bits,
-// with one relaxed store; a reader polls the word with relaxed loads until it carries its
-// launch's tag, and then holds the value -- no counter, fence or grid barrier in between. A
-// word a reader polls is always written by the reader's own launch, so a stale word carries
-// an older launch's tag.
-__device__ __forceinline__ void grid_arrive(unsigned long long *ctr) {
-  asm volatile("red.release.gpu.global.add.u64 [%0], 1;" ::"l"(ctr) : "memory");
-}
-__device__ bool grid_wait(const unsigned long long *ctr, unsigned long long target, volatile uint32_t *err,
-                          uint32_t where, uint64_t limit_ns) {
-  bool ok = true;
-  if (ld_acquire_u64(ctr) < target) {
-    const uint64_t t0 = globaltimer_ns();
-    while (ld_acquire_u64(ctr) < target) {
-      if (globaltimer_ns() - t0 > limit_ns) {
-        report_error(err, MOE_DEV_ERR_TIMEOUT, where);
-        ok = false;
-        break;
-      }
-    }
-  }
-  return ok;   // the acquire load that saw the target orders this thread's later reads
-}
+// The tag comes from a launch counter: every CTA adds 1 to it once, as it starts, so the
+// counter is a multiple of gridDim.x when a launch starts, and the value a CTA's add returns
+// rounds down to that start value (the adds before it come from CTAs of its own launch). tag =
+// start / gridDim.x + 1 differs for any two consecutive launches and is never 0, the value of
+// zeroed words. A word a reader polls is always written by the reader's own launch, so a stale
+// word carries an older launch's tag. (After an expired wait the host zeroes the counter and
+// the tagged words before the next launch.)
 __device__ __forceinline__ void named_arrive(int id, int n) {
   asm volatile("bar.arrive %0, %1;" ::"r"(id), "r"(n) : "memory");
-}
-// Grid barrier of the compute and epilogue warps (the named barrier kBarTeam inside the CTA).
-// An expired wait sets *abort; the caller keeps going.
-__device__ void grid_barrier_team(unsigned long long *ctr, unsigned long long target, volatile uint32_t *err,
-                                  uint32_t where, int nteam, volatile int *abort, uint64_t limit_ns) {
-  named_sync(kBarTeam, nteam);
-  if (threadIdx.x == 0) {
-    grid_arrive(ctr);
-    if (!grid_wait(ctr, target, err, where, limit_ns)) *abort = 1;
-  }
-  named_sync(kBarTeam, nteam);
 }
 // Wait for an mbarrier phase, at most limit_ns; gives up at once when *abort is set and sets
 // it when the bound expires.
@@ -260,6 +224,40 @@ __device__ bool poll_tagged(const unsigned long long *p, size_t stride, int n, u
   }
 #pragma unroll
   for (int j = 0; j < 8; ++j) y[j] = tag_value(v[j]);
+  return true;
+}
+
+// Polls the 32 launch-tagged words p[0, 32) (16-byte aligned, all loads in flight at once)
+// until each carries the tag; their values go to v[]. False when *abort is set or the bound
+// ran out (reported, *abort set).
+__device__ bool poll_tagged32(const unsigned long long *p, uint32_t tag, float (&v)[MOE_QK], volatile int *abort,
+                              volatile uint32_t *err, uint64_t limit_ns) {
+  unsigned long long w[MOE_QK];
+#pragma unroll
+  for (int i = 0; i < MOE_QK / 2; ++i) ld_relaxed_v2_u64(p + 2 * i, w[2 * i], w[2 * i + 1]);
+  bool all = true;
+#pragma unroll
+  for (int i = 0; i < MOE_QK; ++i) all = all && has_tag(w[i], tag);
+  if (!all) {
+    const uint64_t t0 = globaltimer_ns();
+    for (;;) {
+#pragma unroll
+      for (int i = 0; i < MOE_QK / 2; ++i)
+        if (!has_tag(w[2 * i], tag) || !has_tag(w[2 * i + 1], tag)) ld_relaxed_v2_u64(p + 2 * i, w[2 * i], w[2 * i + 1]);
+      all = true;
+#pragma unroll
+      for (int i = 0; i < MOE_QK; ++i) all = all && has_tag(w[i], tag);
+      if (all) break;
+      if (*abort) return false;
+      if (globaltimer_ns() - t0 > limit_ns) {
+        report_error(err, MOE_DEV_ERR_TIMEOUT, 21);
+        *abort = 1;
+        return false;
+      }
+    }
+  }
+#pragma unroll
+  for (int i = 0; i < MOE_QK; ++i) v[i] = tag_value(w[i]);
   return true;
 }
 
@@ -564,12 +562,12 @@ k_moe_decode(const __nv_bfloat16 *__restrict__ x, const float *y_prev, float eps
   extern __shared__ __align__(128) uint8_t smem_raw[];
   __shared__ FusedShared sh;
   const int tid = threadIdx.x, lane = tid & 31, wq = tid >> 5, nw = blockDim.x >> 5;
-  // the grid-barrier counter as this launch starts, loaded now by the thread that arrives at
-  // the barrier (its latency hides behind the router); it also gives the launch's tag
+  // this CTA's add to the launch counter, which names the launch (its latency hides behind
+  // the router)
   const int bar_tid = (int)blockDim.x - 32;
-  const unsigned long long gstart = tid == bar_tid ? ld_acquire_u64(W.gbar) : 0ull;
+  const unsigned long long gstart = tid == bar_tid ? atomicAdd(W.gbar, 1ull) : 0ull;
   const int nwc = nw - 2, nct = nwc * 32;   // compute warps 0 .. nwc-1; warp nwc produces, nwc+1 epilogues
-  const int nteam = nct + 32;
+  const int nteam = nct + 32;   // compute + epilogue warps
   const int nb = d / MOE_QK, nbf = f / MOE_QK;
   const int G = (nb + kGran - 1) / kGran;
   const uint32_t rb_g = (uint32_t)nb * MOE_QBYTES, rb_d = (uint32_t)nbf * MOE_QBYTES;
@@ -630,9 +628,7 @@ k_moe_decode(const __nv_bfloat16 *__restrict__ x, const float *y_prev, float eps
   const bool skip_logits = W.inject == MOE_INJECT_SKIP_ROUTER_ARRIVAL && blockIdx.x == 0;
   auto publish_base = [&]() {
     if (tid == bar_tid) {
-      const unsigned long long base = gstart - gstart % gridDim.x;
-      sh.gbase = base;
-      sh.tag = (uint32_t)(base / gridDim.x) + 1u;
+      sh.tag = (uint32_t)(gstart / gridDim.x) + 1u;   // gstart rounded down to the launch's start
     }
   };
 
@@ -854,7 +850,6 @@ k_moe_decode(const __nv_bfloat16 *__restrict__ x, const float *y_prev, float eps
   const bool aligned = (nb % kGran) == 0;
   const int n_items = G;
   const int P = kDnParts;
-  bool down_phase = false;
   int pass = 0;
   if (wq < nwc) {
     int hw0 = 0, hw1 = 0;   // sorted positions whose hidden vectors are staged in hs
@@ -862,11 +857,6 @@ k_moe_decode(const __nv_bfloat16 *__restrict__ x, const float *y_prev, float eps
     wk.init(sh.seq, upe_g, upe_d);
     for (int it = 0; !wk.done(); ++it) {
       const FChunk c = wk.cur(upe_g, upe_d);
-      if (c.down && !down_phase) {
-        // all h written (the epilogue warp included) before any CTA reads it
-        grid_barrier_team(W.gbar, sh.gbase + gridDim.x, W.err, 21, nteam, &sh.abort, W.wait_ns);
-        down_phase = true;
-      }
       const int slot = it % kFStages;
       const bool okw = wait_phase(&sh.full[slot], (uint32_t)(it / kFStages) & 1u, &sh.abort, W.err, 22, W.wait_ns);
       const int e = sh.act[c.a];
@@ -912,13 +902,11 @@ k_moe_decode(const __nv_bfloat16 *__restrict__ x, const float *y_prev, float eps
           const int nblk = okw ? (hw1 - hw0) * nbf : 0;
           for (int blk = tid; blk < nblk; blk += nct) {
             const int i = blk / nbf, cb = blk - i * nbf;
-            const float4 *src = reinterpret_cast<const float4 *>(W.h + (size_t)sh.perm[hw0 + i] * f + (size_t)cb * MOE_QK);
             float v[MOE_QK];
-#pragma unroll
-            for (int q = 0; q < 8; ++q) {
-              const float4 a4 = __ldcg(src + q);
-              v[4 * q] = a4.x; v[4 * q + 1] = a4.y; v[4 * q + 2] = a4.z; v[4 * q + 3] = a4.w;
-            }
+            // the block's values as other CTAs' epilogues (or this one's) store them
+            if (!poll_tagged32(W.htag + (size_t)sh.perm[hw0 + i] * f + (size_t)cb * MOE_QK, sh.tag, v, &sh.abort,
+                               W.err, W.wait_ns))
+              break;
             stage_block_t(v, 0, hs + (size_t)i * f + (size_t)cb * MOE_QK, hbk + (size_t)i * nbf + cb);
           }
           named_sync(kBarCompute, nct);
@@ -954,7 +942,6 @@ k_moe_decode(const __nv_bfloat16 *__restrict__ x, const float *y_prev, float eps
       if (lane == 0) mbar_arrive(&sh.empty[slot]);   // this warp's last read of the stage
       wk.advance(c.n, sh.seq, upe_g, upe_d);
     }
-    if (!down_phase) grid_barrier_team(W.gbar, sh.gbase + gridDim.x, W.err, 21, nteam, &sh.abort, W.wait_ns);   // no down rows here
     for (int q = pass < 2 ? 0 : pass - 2; q < pass; ++q) named_sync(kBarEmpty0 + (q & 1), nteam);
   } else {
     // the epilogue warp: the same sequence of chunks and passes
@@ -962,10 +949,6 @@ k_moe_decode(const __nv_bfloat16 *__restrict__ x, const float *y_prev, float eps
     wk.init(sh.seq, upe_g, upe_d);
     while (!wk.done()) {
       const FChunk c = wk.cur(upe_g, upe_d);
-      if (c.down && !down_phase) {
-        grid_barrier_team(W.gbar, sh.gbase + gridDim.x, W.err, 21, nteam, &sh.abort, W.wait_ns);
-        down_phase = true;
-      }
       const int e = sh.act[c.a];
       const int cnt = sh.counts[e];
       const int off = sh.offsets[e];
@@ -987,7 +970,10 @@ k_moe_decode(const __nv_bfloat16 *__restrict__ x, const float *y_prev, float eps
                 g += v.x;
                 uu += v.y;
               }
-              W.h[(size_t)sh.perm[off + g0 + i] * f + c.r0 + pp] = gelu_tanh_f(g) * uu;
+              const float hv = gelu_tanh_f(g) * uu;
+              const size_t hi = (size_t)sh.perm[off + g0 + i] * f + c.r0 + pp;
+              st_relaxed_u64(W.htag + hi, tag_word(sh.tag, hv));
+              W.h[hi] = hv;   // the plain copy for the debug reader
             }
           } else {
             const int nr = c.n * kUnit;
@@ -1003,7 +989,6 @@ k_moe_decode(const __nv_bfloat16 *__restrict__ x, const float *y_prev, float eps
       }
       wk.advance(c.n, sh.seq, upe_g, upe_d);
     }
-    if (!down_phase) grid_barrier_team(W.gbar, sh.gbase + gridDim.x, W.err, 21, nteam, &sh.abort, W.wait_ns);
   }
   // ---------------------------------------------------------------- phase 4: combine
   // no grid barrier: every term is polled (bounded) from its launch-tagged word, eight slots'

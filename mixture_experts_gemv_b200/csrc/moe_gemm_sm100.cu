@@ -185,8 +185,8 @@ __device__ __forceinline__ void st_shared_v4(uint32_t addr, uint32_t a, uint32_t
 
 // GELU, tanh form, with the hardware tanh approximation (`tanh.approx.f32`, absolute error
 // about 2^-11): h is rounded to bf16 right after (relative step 2^-8), and this path's outputs
-// are held to 2e-2 relative to an FP64 evaluation of the layer; it frees the epilogue's issue slots for the producer warps
-// that share the SM's schedulers.
+// are held to 2e-2 relative to an FP64 evaluation of the layer; it frees the epilogue's issue
+// slots for the producer warps that share the SM's schedulers.
 __device__ __forceinline__ float gelu_tanh_f(float z) {
   const float c = 0.7978845608028654f;   // sqrt(2/pi)
   float t;
