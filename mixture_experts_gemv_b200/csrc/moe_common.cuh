@@ -282,7 +282,7 @@ int moe_launch_gemm_experts(const MoeLaunch &L, const MoeWork &W, const void *x,
 bool moe_fused_decode_supported(int T, int d, int f, int E, int k, bool dense = false);
 // The fused decode kernel: x (bf16 [T, d]) as the layer input, or, with y_prev not null, the
 // previous layer's FP32 output normalised in the kernel (x_out, when not null, receives that
-// bf16 x; y_prev may equal out).
+// bf16 x; y_prev must not overlap out).
 int moe_launch_fused_decode(const MoeLaunch &L, const MoeWork &W, const void *x, const float *y_prev, float eps,
                             void *x_out, const float *router_w, const float *router_scale,
                             const uint8_t *gate_up_q4, const uint8_t *down_q4, const float *expert_scale, int T,
