@@ -191,10 +191,10 @@ int moe_debug_get_hidden(float *h, void *stream);
 int moe_debug_check(void *stream);
 
 /*
- * Failure detection, for tests. Every device-side wait (mbarrier phases, grid barriers, polls
- * of launch-tagged words) is bounded; a wait that runs out records MOE_ERR_DEVICE_TIMEOUT in
- * the error word, the kernel ends on its own (it waits, again bounded, for its copies in
- * flight first) and the context stays usable.
+ * Failure detection, for tests. Every device-side wait (mbarrier phases, arrival counters,
+ * polls of launch-tagged words) is bounded; a wait that runs out records
+ * MOE_ERR_DEVICE_TIMEOUT in the error word, the kernel ends on its own (it waits, again
+ * bounded, for its copies in flight first) and the context stays usable.
  *   moe_debug_set_wait_ns: bound of every device-side wait of later forwards, in
  *     nanoseconds (0 restores the default of 2 s).
  *   moe_debug_inject: make the next forward simulate a fault by skipping one step --

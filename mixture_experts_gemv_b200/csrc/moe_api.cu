@@ -120,7 +120,7 @@ Layout make_layout(int maxT, int max_d, int max_f, int max_E, int max_k) {
       (size_t)maxT * max_d * 4,          // 19 ylayer
       (S / kTileM + max_E + 1) * 8,      // 20 tile pairs
       (size_t)max_E * 4,                 // 21 toff
-      64,                                // 22 grid-barrier counter
+      64,                                // 22 launch counter of the fused decode kernel
       (size_t)max_d * 4 + 16,            // 23 dense MLP pass: zero router row, then 1.0f
       (size_t)3 * 128 * max_d * 2,       // 24 the router weights as three bf16 planes (prefill)
       tag_bytes(max_d, max_f, max_E),    // 25 launch-tagged logits, per-slot outputs and hidden vectors
@@ -158,7 +158,7 @@ int check_device_error() {
   return MOE_OK;
 }
 
-// After an expired wait: the grid-barrier counter and the arrival counters start again from
+// After an expired wait: the launch counter and the arrival counters start again from
 // zero (enqueued on the stream of the next launch).
 int reset_counters_if_needed(cudaStream_t s) {
   if (!g.reset_pending) return MOE_OK;

@@ -548,8 +548,8 @@ __device__ __forceinline__ void dn_pass(const uint8_t *st, uint32_t rb, int nbf,
 
 // NORM_IN: the layer input is the previous layer's FP32 output y_prev, normalised here
 // (unit-gain RMSNorm + bf16 cast, as moe_norm.cu) instead of a bf16 x; CTA 0 also writes the
-// bf16 x to x_out when it is not null. y_prev may be the buffer `out` of this call: every CTA
-// reads it before its first grid-barrier arrival, `out` is written after the last barrier.
+// bf16 x to x_out when it is not null. y_prev must not overlap `out`: with no grid barrier, a
+// CTA may write its output rows while another still reads y_prev.
 template <bool NORM_IN>
 __global__ void __launch_bounds__((kFMaxCompute + 2) * 32, 1)
 k_moe_decode(const __nv_bfloat16 *__restrict__ x, const float *y_prev, float eps, __nv_bfloat16 *x_out,
