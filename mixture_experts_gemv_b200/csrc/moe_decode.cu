@@ -117,8 +117,10 @@ __device__ __forceinline__ void named_sync(int id, int n) {
 // rounds down to that start value (the adds before it come from CTAs of its own launch). tag =
 // start / gridDim.x + 1 differs for any two consecutive launches and is never 0, the value of
 // zeroed words. A word a reader polls is always written by the reader's own launch, so a stale
-// word carries an older launch's tag. (After an expired wait the host zeroes the counter and
-// the tagged words before the next launch.)
+// word carries an older launch's tag; the 32-bit tag repeats only every 2^32 launches (about a
+// day of back-to-back single-token layers), so a stale word could pass only if it was last
+// written a multiple of 2^32 launches earlier and is read before its new value lands. (After
+// an expired wait the host zeroes the counter and the tagged words before the next launch.)
 __device__ __forceinline__ void named_arrive(int id, int n) {
   asm volatile("bar.arrive %0, %1;" ::"r"(id), "r"(n) : "memory");
 }
@@ -626,9 +628,10 @@ k_moe_decode(const __nv_bfloat16 *__restrict__ x, const float *y_prev, float eps
   // test-only fault: CTA 0 never stores its router logits, so every CTA's bounded wait for
   // them runs out and reports a timeout
   const bool skip_logits = W.inject == MOE_INJECT_SKIP_ROUTER_ARRIVAL && blockIdx.x == 0;
+  // the launch's tag into shared memory (gstart / gridDim.x rounds down to the launch's start)
   auto publish_base = [&]() {
     if (tid == bar_tid) {
-      sh.tag = (uint32_t)(gstart / gridDim.x) + 1u;   // gstart rounded down to the launch's start
+      sh.tag = (uint32_t)(gstart / gridDim.x) + 1u;
     }
   };
 
