@@ -56,6 +56,8 @@ SMALL = [  # (E, k, T, d, f)
     (4, 1, 1, 64, 32), (4, 4, 7, 64, 32), (8, 2, 33, 256, 64), (8, 8, 2, 96, 64),
     (128, 8, 1, 256, 96), (128, 8, 33, 512, 128), (128, 2, 300, 256, 64), (128, 128, 3, 64, 32),
     (16, 3, 17, 2816, 64), (6, 2, 16, 320, 704),
+    (200, 8, 5, 256, 64),    # E above the CTA count: a CTA computes two router rows
+    (256, 16, 3, 128, 64),   # E = 256 with k > 8: eight logits a lane, 64-bit selection keys
 ]
 
 
